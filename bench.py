@@ -1,0 +1,414 @@
+"""Benchmark of the MSA hot path on B200: route (Q^R projection, K̄^R scan, top-k)
+plus sparse decode attention over the selected documents and the local KV.
+
+One step = one pass of the whole online path for one batch of queries:
+msa_route_topk (projection from H_q, scan + per-document max, top-k) followed by
+msa_sparse_attend (gather of the selected docs' pooled K̄/V̄ + local KV with
+global RoPE, split-KV flash-decode, combine).  Inputs are synthetic (seeded) with
+the shapes of the 1M-token, Qwen3-4B-like workload; see the design doc.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl msa|reference]
+
+Prints one JSON line (rank 0).  Under torchrun each rank runs an independent
+replica of the workload (the path shards by query batch / memory bank with no
+data-path exchange), timing is max over ranks and `value` sums all ranks' work.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "memory tokens routed/s (top-k + sparse attn); scan HBM GB/s vs peak"
+UNIT = "tokens/s"
+N_ROT = 8  # rotating input copies: K̄^R + K̄ + V̄ + local KV x 8 = 1.4 GB > L2 (126 MB)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="msa", choices=["msa", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    return ap.parse_args()
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def workload_config():
+    from long_context_memory_b200 import workloads as W
+
+    c = W.mem1m_config()
+    return c
+
+
+# ----------------------------------------------------------------------------
+# oracle timing (cpu_baseline and --impl reference)
+# ----------------------------------------------------------------------------
+def time_oracle(c, seconds: float):
+    """Oracle route + attend for the workload's query batch, repeated within a time budget."""
+    import oracle as O
+
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(limits=1)
+    except Exception:  # pragma: no cover
+        limiter = None
+    d = c["dims"]
+    co, *_ = O.chunk_layout(c["doc_off"])
+    steps, t0 = 0, time.perf_counter()
+    while True:
+        QR = O.router_query(c["Hq"], c["W_QR"], d.n_r, d.d_r)
+        _, idx, _ = O.route_topk(QR, c["KR"], co, c["k"])
+        O.sparse_attend(c["q"], c["K_bar"], c["V_bar"], co, idx, c["K_loc"], c["V_loc"], c["loc_len"],
+                        c["pos_offset"], d.rope_base)
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or steps >= 50:
+            break
+    if limiter is not None:
+        limiter.unregister() if hasattr(limiter, "unregister") else None
+    per_step = el / steps
+    return dict(value=c["T"] * c["B"] / per_step, unit=UNIT, cores=1, kind="oracle",
+                sample=f"{steps} full steps of the 1M-token workload (B={c['B']}), numpy fp64, 1 thread, "
+                       f"{el:.1f} s", ms_per_step=per_step * 1e3)
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    c = workload_config()
+    steps = max(1, args.steps)
+    budget = min(20.0, max(3.0, 1.0 * steps))
+    r = time_oracle(c, budget)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": args.gpus,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "mem1m: 1M-token memory, Qwen3-4B-like dims, B=1, top-16, 4K local KV"},
+        "cpu_baseline": {"value": r["value"], "unit": UNIT, "cores": r["cores"], "kind": "oracle",
+                         "sample": r["sample"]},
+        "e2e": {"value": r["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.idx), "-lms", "100"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# the GPU arm
+# ----------------------------------------------------------------------------
+def scan_traffic_record(kernel: str):
+    """Per-launch DRAM bytes of `kernel` from a committed ncu summary, or None.
+
+    A summary records the sha256 of the kernel's source file; if the source has
+    changed since the counters were taken the figure is stale and not used."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    kv = {}
+    for line in open(path):
+        if ":" in line and not line.startswith("#"):
+            a, b = line.split(":", 1)
+            kv[a.strip()] = b.strip()
+    src = os.path.join(ROOT, "long_context_memory_b200", "csrc", kv.get("source", ""))
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != kv.get("source_sha256"):
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch_full_size"])
+    except (KeyError, ValueError):
+        return None
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import long_context_memory_b200 as msa
+    from long_context_memory_b200 import workloads as W
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
+
+    c = workload_config()
+    d = c["dims"]
+    B, k, T = c["B"], c["k"], c["T"]
+    co_np, C = msa.chunk_offsets(c["doc_off"])
+    n_docs = len(co_np) - 1
+    chunk_off = torch.from_numpy(co_np).to(dev)
+    t = lambda a: W.to_torch(np.ascontiguousarray(a)).to(dev)
+    base = dict(KR=t(c["KR"]), K_bar=t(c["K_bar"]), V_bar=t(c["V_bar"]), K_loc=t(c["K_loc"]), V_loc=t(c["V_loc"]),
+                Hq=t(c["Hq"]), q=t(c["q"]))
+    W_QR = t(c["W_QR"])
+    loc_len = torch.from_numpy(c["loc_len"]).to(dev)
+    # distinct copies at distinct addresses so that consecutive steps miss L2
+    rot = [base] + [{kk: v.clone() for kk, v in base.items()} for _ in range(N_ROT - 1)]
+    out_idx = [torch.empty((B, k), dtype=torch.int32, device=dev) for _ in range(N_ROT)]
+    out_sc = [torch.empty((B, k), dtype=torch.float32, device=dev) for _ in range(N_ROT)]
+    out_o = [torch.empty((B, d.n_q, d.head_dim), dtype=torch.bfloat16, device=dev) for _ in range(N_ROT)]
+    r_ws = torch.empty(msa.route_workspace_size(d, B, n_docs, C, k) + 256, dtype=torch.uint8, device=dev)
+    a_ws = torch.empty(msa.attend_workspace_size(d, B, k, c["t_loc_max"], c["pos_offset"]) + 256,
+                       dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(i):
+        x = rot[i % N_ROT]
+        j = i % N_ROT
+        msa.route_topk(d, x["Hq"], W_QR, x["KR"], chunk_off, k, out=(out_idx[j], out_sc[j], None), ws=r_ws)
+        msa.sparse_attend(d, x["q"], x["K_bar"], x["V_bar"], chunk_off, out_idx[j], x["K_loc"], x["V_loc"], loc_len,
+                          c["pos_offset"], out=out_o[j], ws=a_ws)
+
+    # ---- capture one graph per rotation copy (untraced) ----
+    graphs = []
+    with torch.cuda.stream(stream):
+        for i in range(N_ROT):  # eager warm-up also sets kernel attributes outside capture
+            step(i)
+    torch.cuda.synchronize()
+    use_graphs = True
+    try:
+        for i in range(N_ROT):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step(i)
+            graphs.append(g)
+    except Exception as e:  # pragma: no cover
+        print(f"graph capture failed ({e}); timing eager launches", file=sys.stderr)
+        use_graphs = False
+    torch.cuda.synchronize()
+
+    def launch(i):
+        if use_graphs:
+            graphs[i % N_ROT].replay()
+        else:
+            with torch.cuda.stream(stream):
+                step(i)
+
+    def timed_region(n, warm):
+        for i in range(warm):
+            launch(i)
+        torch.cuda.synchronize()
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(n):
+            launch(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        if ws > 1:
+            tt = torch.tensor([ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ms = float(tt.item())
+            dist.barrier()
+        torch.cuda.synchronize()
+        return ms
+
+    with ClockSampler(local) as clk:
+        total_ms = timed_region(args.steps, args.warmup)
+    clocks = clk.summary()
+    ms_step = total_ms / args.steps
+    value = T * B * ws / (ms_step * 1e-3)
+
+    # ---- per-kernel device time: the same steps, each kernel bracketed by trace events ----
+    msa.trace_reset()
+    msa.trace_enable(True)
+    tgraphs = []
+    try:
+        for i in range(args.steps):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step(i)
+            tgraphs.append(g)
+    finally:
+        msa.trace_enable(False)
+    for rep in range(2):  # first pass warms up; the events keep the second pass's times
+        for g in tgraphs:
+            g.replay()
+    torch.cuda.synchronize()
+    kt = msa.trace_read()
+    msa.trace_reset()
+    del tgraphs
+
+    # ---- roofline of the dominant kernel ----
+    hbm_peak, peak_kind = peaks()
+    sel = out_idx[0].cpu().numpy()
+    n_sel = int(sum(co_np[i + 1] - co_np[i] for i in sel[0]))
+    per_kernel = {n: (ms, cnt) for n, (ms, cnt) in kt.items() if cnt > 0}
+    scan_bytes = C * d.n_r * d.d_r * 2
+    attn_bytes = B * (n_sel + int(c["loc_len"][0])) * d.n_kv * d.head_dim * 2 * 2
+    cand = {"scan": scan_bytes, "attn_split": attn_bytes}
+    dom = max(cand, key=lambda n: per_kernel.get(n, (0, 1))[0])
+    dms, dcnt = per_kernel[dom]
+    avg_s = dms / dcnt * 1e-3
+    achieved = cand[dom] / avg_s / 1e9
+    traffic = scan_traffic_record(dom)
+    roofline = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": traffic, "peak_kind": peak_kind,
+                "algorithmic_bytes_per_launch": cand[dom], "avg_launch_us": avg_s * 1e6}
+    kernels = {n: {"avg_us": ms / cnt * 1e3 / 1.0, "launches": cnt} for n, (ms, cnt) in per_kernel.items()}
+    for n in kernels:
+        kernels[n]["avg_us"] = per_kernel[n][0] / per_kernel[n][1] * 1e3
+    for n, b in cand.items():
+        if n in per_kernel:
+            kernels[n]["GB/s"] = b / (per_kernel[n][0] / per_kernel[n][1] * 1e-3) / 1e9
+    gpu_launches = sum(cnt for (_, cnt) in per_kernel.values()) // max(1, args.steps) * args.steps
+
+    # ---- end to end through the public API from pinned host buffers ----
+    host = {kk: base[kk].cpu().pin_memory() for kk in ("Hq", "q", "K_loc", "V_loc")}
+    dev_in = {kk: torch.empty_like(base[kk]) for kk in host}
+    h_idx = torch.empty((B, k), dtype=torch.int32).pin_memory()
+    h_sc = torch.empty((B, k), dtype=torch.float32).pin_memory()
+    h_out = torch.empty((B, d.n_q, d.head_dim), dtype=torch.bfloat16).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = h_idx.numel() * 4 + h_sc.numel() * 4 + h_out.numel() * 2
+
+    def e2e_step(i):
+        x = rot[i % N_ROT]
+        for kk in host:
+            dev_in[kk].copy_(host[kk], non_blocking=True)
+        msa.route_topk(d, dev_in["Hq"], W_QR, x["KR"], chunk_off, k, out=(out_idx[0], out_sc[0], None), ws=r_ws)
+        msa.sparse_attend(d, dev_in["q"], x["K_bar"], x["V_bar"], chunk_off, out_idx[0], dev_in["K_loc"],
+                          dev_in["V_loc"], loc_len, c["pos_offset"], out=out_o[0], ws=a_ws)
+        h_idx.copy_(out_idx[0], non_blocking=True)
+        h_sc.copy_(out_sc[0], non_blocking=True)
+        h_out.copy_(out_o[0], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            e2e_step(i)
+        torch.cuda.synchronize()
+        if ws > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            e2e_step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    if ws > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    e2e_val = T * B * ws / (e2e_ms * 1e-3)
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        r = time_oracle(c, args.cpu_seconds)
+        cpu = {kk: r[kk] for kk in ("value", "unit", "cores", "kind", "sample")}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16 pooled memory, lognormal docs)",
+            "config": {"workload": "mem1m: 1M-token memory (C=%d chunks, %d docs), Qwen3-4B-like dims "
+                                   "(hidden 2560, 32q/8kv x 128, 8 router heads x 128), B=%d, top-%d, %d-token local KV"
+                                   % (C, n_docs, B, k, c["t_loc_max"]),
+                       "l2": "8 rotating input copies (%.2f GB) > L2" % (N_ROT * sum(v.numel() * 2 for v in base.values()) / 1e9),
+                       "graphs": use_graphs, "parallelism": f"replicas x{ws}"},
+            "roofline": roofline, "kernels": kernels, "gpu_launches": gpu_launches,
+            "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms},
+            "cpu_baseline": cpu, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,193 @@
+/*
+ * msa.h - C ABI of the Memory Sparse Attention (MSA) hot path on NVIDIA B200.
+ *
+ * The method ("MSA: Memory Sparse Attention for Efficient End-to-End Memory
+ * Model Scaling to 100M Tokens") serves a memory of N documents in three
+ * stages (IRMaD reading, "M. Materials & Methods", three-stage inference item;
+ * project overview, "three-stage inference pipeline" figure):
+ *   1. offline encoding: K = H W_K with document-wise RoPE, V = H W_V,
+ *      K^R = H W^KR, each mean-pooled over 64-token chunks that never cross a
+ *      document boundary -> K̄, V̄, K̄^R;
+ *   2. online routing: Q^R = H_q W^QR, chunk score = head-mean cosine against
+ *      every K̄^R, document score = max over its chunks, top-k documents;
+ *   3. sparse generation: GQA decode attention over [selected docs' K̄; local K]
+ *      with global RoPE offset by k on the active context.
+ *
+ * Conventions for every call
+ *   - Return an msa_status; no exception or abort crosses the ABI.  The message
+ *     of the last failure on the calling thread is msa_last_error().
+ *   - Tensor arguments are DEVICE pointers owned by the caller, unless the
+ *     comment says host.  bf16 tensors are passed as void* and hold IEEE
+ *     bfloat16 bit patterns.  Layouts are dense row-major; the memory tensors
+ *     are chunk-major [C, heads, dim].
+ *   - The library allocates no device memory.  Scratch comes from the caller's
+ *     workspace `ws` of at least msa_*_workspace_size(...) bytes (256-byte
+ *     aligned).  `ws` may be NULL only if that size is 0.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream).  Arguments are validated on the host before any
+ *     launch; a call that returns an error has launched nothing.  Errors raised
+ *     by the device surface at the caller's next synchronisation, or through
+ *     msa_check_device_errors().
+ *   - Every tensor pointer must be 16-byte aligned (MSA_ERR_INVALID_ARG).
+ *   - Device-resident index arrays (doc_off, chunk_off, topk_idx, loc_len) must
+ *     hold what their comments say (monotone offsets, ids in range); they are
+ *     read on the device and cannot be checked on the host.
+ */
+#ifndef MSA_H_
+#define MSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MSA_OK = 0,
+  MSA_ERR_INVALID_ARG = 1, /* bad size, pointer, alignment or value */
+  MSA_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. head_dim not 64/128) */
+  MSA_ERR_WORKSPACE = 3,   /* ws_bytes smaller than the matching *_workspace_size */
+  MSA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed; see msa_last_error() */
+  MSA_ERR_TIMEOUT = 5,     /* a bounded wait gave up (device error word set) */
+} msa_status;
+
+/* Model dimensions of one routed layer.  hidden = width of H; n_q / n_kv =
+ * query / key-value heads (GQA, n_q a multiple of n_kv, n_q / n_kv <= 16);
+ * head_dim in {64, 128}; n_r router heads of dim d_r in {64, 128}, n_r <= 8;
+ * chunk = tokens per pooled chunk (P, 64 on the pages); rope_base = RoPE base. */
+typedef struct {
+  int32_t hidden;
+  int32_t n_q;
+  int32_t n_kv;
+  int32_t head_dim;
+  int32_t n_r;
+  int32_t d_r;
+  int32_t chunk;
+  float rope_base;
+} msa_dims;
+
+/* Document score from its chunk scores: max over chunks (the pages' s_i =
+ * max_j S_ij) or the mean (an alternative reading; see routing notes). */
+typedef enum { MSA_AGG_MAX = 0, MSA_AGG_MEAN = 1 } msa_doc_agg;
+
+/* Thread-local message of the last failing call on this thread ("" if none). */
+const char* msa_last_error(void);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int32_t msa_version(void);
+
+/* Reads and clears the device error word of the current device (bit 0: a
+ * bounded wait gave up; bit 1: a device-side index was out of range).
+ * Synchronises the device.  *bits_out may be NULL. */
+msa_status msa_check_device_errors(uint32_t* bits_out);
+
+/* ---------------------------------------------------------------------------
+ * Stage 1 - chunk layout (host helper).
+ * Pages: digest "Method step details", Stage 1 (chunk mean pooling, P = 64);
+ * chunks never cross a document boundary, the last chunk of a document holds
+ * the remaining L mod P tokens.
+ *   doc_off_host   [n_docs + 1] host, int64 token offsets, doc_off[0] = 0,
+ *                  strictly increasing (every document has >= 1 token).
+ *   chunk_off_host [n_docs + 1] host, out: chunk_off[i+1] = chunk_off[i] +
+ *                  ceil((doc_off[i+1] - doc_off[i]) / chunk).
+ *   n_chunks_out   host, out: C = chunk_off[n_docs] (< 2^31).
+ * ------------------------------------------------------------------------- */
+msa_status msa_chunk_offsets(const int64_t* doc_off_host, int32_t n_docs, int32_t chunk,
+                             int32_t* chunk_off_host, int32_t* n_chunks_out);
+
+/* ---------------------------------------------------------------------------
+ * Stage 1 - offline memory encoding.
+ * Pages: IRMaD "M. Materials & Methods", routing item (K = H W_K, V = H W_V,
+ * K^R = H W^KR, K̄ = φ(K), V̄ = φ(V), K̄^R = φ(K^R)) and position item
+ * (document-wise RoPE: positions restart at 0 in every document).
+ *   H        [T, hidden] bf16, the layer's hidden states of the whole corpus.
+ *   doc_off  [n_docs + 1] device int64 token offsets (as msa_chunk_offsets).
+ *   chunk_off[n_docs + 1] device int32 chunk offsets from msa_chunk_offsets.
+ *   W_K, W_V [hidden, n_kv * head_dim] bf16; W_KR [hidden, n_r * d_r] bf16.
+ *   K_bar, V_bar [C, n_kv, head_dim] bf16 out: chunk means of RoPE(H W_K) at
+ *            document-relative positions and of H W_V.
+ *   KR_bar   [C, n_r, d_r] bf16 out: chunk means of H W^KR.
+ * Requirements: hidden % 64 == 0; n_kv * head_dim and n_r * d_r multiples of
+ * 256; chunk == 64.  Rounding: fp32 accumulation, outputs rounded to bf16.
+ * ------------------------------------------------------------------------- */
+size_t msa_encode_workspace_size(const msa_dims* dims, int64_t T, int32_t n_docs, int32_t n_chunks);
+msa_status msa_encode_memory(const msa_dims* dims, const void* H, int64_t T, const int64_t* doc_off,
+                             int32_t n_docs, const int32_t* chunk_off, int32_t n_chunks, const void* W_K,
+                             const void* W_V, const void* W_KR, void* K_bar, void* V_bar, void* KR_bar,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Stage 2 - online routing and top-k.
+ * Pages: IRMaD "M. Materials & Methods", routing item:
+ *   Q^R = H_q W^QR;  S_ij = max_t mean_h cos(Q^R_h, K̄^R_ij,h);
+ *   s_i = max_j S_ij;  I = Top-k({s_i});  k = 16 on the pages.
+ *   Hq       [B, hidden] bf16 query hidden states, or, when W_QR == NULL,
+ *            [B, n_r * d_r] bf16 router queries Q^R given directly.
+ *   W_QR     [hidden, n_r * d_r] bf16 or NULL.
+ *   KR_bar   [n_chunks, n_r, d_r] bf16 pooled router keys.
+ *   chunk_off[n_docs + 1] device int32 chunk offsets of the documents.
+ *   doc_scores [B, n_docs] fp32 out, optional (NULL = not written).
+ *   topk_idx [B, k] int32 out: document ids, descending score, ties to the
+ *            lower id.  topk_score [B, k] fp32 out: their scores.
+ * Cosines use norms clamped below at 1e-12 (a zero vector scores 0).  One
+ * query token per row of Hq (the max over t is over that single token).
+ * Limits: 1 <= k <= min(n_docs, 256); 1 <= B; n_r <= 8; d_r in {64, 128}.
+ * Rounding: Q^R in fp32; the cosine dot products run on the tensor cores with
+ * the normalised query split into two bf16 terms (hi + lo) and fp32
+ * accumulation, so scores carry ~1e-6 relative error.
+ * ------------------------------------------------------------------------- */
+size_t msa_route_workspace_size(const msa_dims* dims, int32_t B, int32_t n_docs, int32_t n_chunks,
+                                int32_t k, msa_doc_agg agg);
+msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR, int32_t B,
+                          const void* KR_bar, const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks,
+                          int32_t k, msa_doc_agg agg, float* doc_scores, int32_t* topk_idx,
+                          float* topk_score, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Stage 3 - sparse generation attention (one decode step).
+ * Pages: IRMaD "M. Materials & Methods", routing item (K_ctx = [{K̄_i}_{i in I};
+ * K_q], V_ctx likewise, Output = Attention(Q_q, K_ctx, V_ctx)) and position item
+ * (global RoPE on the active context, offset by k); project overview "key
+ * technical details" 1.
+ *   q        [B, n_q, head_dim] bf16, before RoPE; rotated to position
+ *            pos_offset + loc_len[b] - 1 (the decode token is the last local token).
+ *   K_bar, V_bar [n_chunks, n_kv, head_dim] bf16 pooled memory (device).
+ *   chunk_off[n_docs + 1] device int32; topk_idx [B, k] device int32 doc ids.
+ *   K_loc, V_loc [B, t_loc_max, n_kv, head_dim] bf16 local KV, K before RoPE;
+ *            local token j is rotated to position pos_offset + j.
+ *   loc_len  [B] device int32, 0 <= loc_len[b] <= t_loc_max.
+ *   softmax_scale  0 -> 1/sqrt(head_dim).
+ *   out      [B, n_q, head_dim] bf16.
+ * Query head g attends with KV head g / (n_q / n_kv).  No mask: the decode
+ * token sees every gathered chunk and every local token.  Pooled keys keep
+ * their document-wise rotation only.  Rounding: q is rotated and scaled in
+ * fp32 then rounded to bf16; local keys are rotated in fp32 and rounded to
+ * bf16; products and softmax in fp32.
+ * ------------------------------------------------------------------------- */
+size_t msa_attend_workspace_size(const msa_dims* dims, int32_t B, int32_t k, int32_t t_loc_max,
+                                 int32_t pos_offset);
+msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, const void* K_bar,
+                             const void* V_bar, const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks,
+                             const int32_t* topk_idx, int32_t k, const void* K_loc, const void* V_loc,
+                             const int32_t* loc_len, int32_t t_loc_max, int32_t pos_offset,
+                             float softmax_scale, void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Tracing: per-kernel device time.
+ * While enabled, every kernel launch is bracketed by CUDA events recorded on
+ * the stream it is launched on.  msa_trace_read synchronises on those events
+ * and returns, for kernel `kernel_id`, the summed device milliseconds and the
+ * launch count since the last reset.  Kernel ids run 0 .. msa_trace_num_kernels()-1.
+ * ------------------------------------------------------------------------- */
+msa_status msa_trace_enable(int32_t on);
+msa_status msa_trace_reset(void);
+int32_t msa_trace_num_kernels(void);
+const char* msa_trace_kernel_name(int32_t kernel_id);
+msa_status msa_trace_read(int32_t kernel_id, double* total_ms, int64_t* launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H_ */

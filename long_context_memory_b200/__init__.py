@@ -1,0 +1,265 @@
+"""Memory Sparse Attention (MSA) hot path for NVIDIA B200: Python binding.
+
+A thin ctypes layer over ``libmsa.so`` (C ABI declared in ``include/msa.h``).
+It only marshals arguments: every step of the path runs in the library's CUDA
+kernels.  PyTorch supplies device memory (outputs and workspaces) and the
+current stream.  Importing this package fails loudly when the library is
+missing; there is no CPU fallback.
+
+Entry points (same names as the C ABI, minus the ``msa_`` prefix):
+  chunk_offsets, encode_memory, route_topk, sparse_attend,
+  *_workspace_size, check_device_errors, trace_*.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+__all__ = [
+    "Dims", "MSAError", "lib", "chunk_offsets", "encode_memory", "route_topk", "sparse_attend",
+    "route_workspace_size", "attend_workspace_size", "encode_workspace_size", "check_device_errors",
+    "trace_enable", "trace_reset", "trace_read", "trace_kernel_names", "AGG_MAX", "AGG_MEAN",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmsa.so")
+
+AGG_MAX = 0
+AGG_MEAN = 1
+
+STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED", 3: "MSA_ERR_WORKSPACE",
+          4: "MSA_ERR_CUDA", 5: "MSA_ERR_TIMEOUT"}
+
+
+class MSAError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{STATUS.get(code, code)}: {msg}")
+        self.code = code
+
+
+class Dims(ctypes.Structure):
+    """msa_dims: hidden, n_q, n_kv, head_dim, n_r, d_r, chunk, rope_base."""
+    _fields_ = [("hidden", ctypes.c_int32), ("n_q", ctypes.c_int32), ("n_kv", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("n_r", ctypes.c_int32), ("d_r", ctypes.c_int32),
+                ("chunk", ctypes.c_int32), ("rope_base", ctypes.c_float)]
+
+    @classmethod
+    def of(cls, d) -> "Dims":
+        return cls(d.hidden, d.n_q, d.n_kv, d.head_dim, d.n_r, d.d_r, d.chunk, float(d.rope_base))
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libmsa.so not found at {LIB_PATH}; build it with `python -m long_context_memory_b200.build` "
+            "(nvcc, sm_100a). There is no CPU fallback.")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, SZ, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+    DP = ctypes.POINTER(Dims)
+    sig = {
+        "msa_last_error": (ctypes.c_char_p, []),
+        "msa_version": (I32, []),
+        "msa_check_device_errors": (I32, [ctypes.POINTER(ctypes.c_uint32)]),
+        "msa_chunk_offsets": (I32, [P, I32, I32, P, ctypes.POINTER(I32)]),
+        "msa_encode_workspace_size": (SZ, [DP, I64, I32, I32]),
+        "msa_encode_memory": (I32, [DP, P, I64, P, I32, P, I32, P, P, P, P, P, P, P, SZ, P]),
+        "msa_route_workspace_size": (SZ, [DP, I32, I32, I32, I32, I32]),
+        "msa_route_topk": (I32, [DP, P, P, I32, P, P, I32, I32, I32, I32, P, P, P, P, SZ, P]),
+        "msa_attend_workspace_size": (SZ, [DP, I32, I32, I32, I32]),
+        "msa_sparse_attend": (I32, [DP, P, I32, P, P, P, I32, I32, P, I32, P, P, P, I32, I32, F, P, P, SZ, P]),
+        "msa_trace_enable": (I32, [I32]),
+        "msa_trace_reset": (I32, []),
+        "msa_trace_num_kernels": (I32, []),
+        "msa_trace_kernel_name": (ctypes.c_char_p, [I32]),
+        "msa_trace_read": (I32, [I32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(I64)]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    return L
+
+
+class _LazyLib:
+    """Loads libmsa.so on first use, so that the seeded generators in
+    ``workloads`` import without the compiled library."""
+
+    _cdll = None
+
+    def __getattr__(self, name):
+        if _LazyLib._cdll is None:
+            _LazyLib._cdll = _load()
+        return getattr(_LazyLib._cdll, name)
+
+
+lib = _LazyLib()
+
+
+def _check(code: int):
+    if code != 0:
+        raise MSAError(code, lib.msa_last_error().decode())
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _workspace(nbytes: int, device, ws=None):
+    import torch
+
+    if nbytes == 0:
+        return None
+    if ws is not None:
+        if ws.numel() * ws.element_size() < nbytes:
+            raise MSAError(3, f"workspace of {ws.numel() * ws.element_size()} bytes < {nbytes}")
+        return ws
+    return torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+
+
+def _aligned_ptr(ws) -> Optional[int]:
+    if ws is None:
+        return None
+    p = ws.data_ptr()
+    return (p + 255) & ~255
+
+
+# ----------------------------------------------------------------------------
+# host helper
+# ----------------------------------------------------------------------------
+def chunk_offsets(doc_off, chunk: int = 64):
+    """chunk_off [n_docs+1] int32 (numpy) and n_chunks from doc_off [n_docs+1] int64 (host)."""
+    import numpy as np
+
+    doc_off = np.ascontiguousarray(doc_off, dtype=np.int64)
+    n_docs = len(doc_off) - 1
+    out = np.zeros(n_docs + 1, dtype=np.int32)
+    n = ctypes.c_int32(0)
+    _check(lib.msa_chunk_offsets(doc_off.ctypes.data, n_docs, chunk, out.ctypes.data, ctypes.byref(n)))
+    return out, int(n.value)
+
+
+# ----------------------------------------------------------------------------
+# stage 1
+# ----------------------------------------------------------------------------
+def encode_workspace_size(dims, T: int, n_docs: int, n_chunks: int) -> int:
+    return int(lib.msa_encode_workspace_size(ctypes.byref(Dims.of(dims)), T, n_docs, n_chunks))
+
+
+def encode_memory(dims, H, doc_off, chunk_off, n_chunks: int, W_K, W_V, W_KR, out=None, ws=None, stream=None):
+    """Pooled (K̄, V̄, K̄^R) of a corpus; all tensors on the same CUDA device."""
+    import torch
+
+    dd = Dims.of(dims)
+    T, n_docs = H.shape[0], doc_off.numel() - 1
+    dev = H.device
+    if out is None:
+        out = (torch.empty((n_chunks, dims.n_kv, dims.head_dim), dtype=torch.bfloat16, device=dev),
+               torch.empty((n_chunks, dims.n_kv, dims.head_dim), dtype=torch.bfloat16, device=dev),
+               torch.empty((n_chunks, dims.n_r, dims.d_r), dtype=torch.bfloat16, device=dev))
+    nbytes = encode_workspace_size(dims, T, n_docs, n_chunks)
+    ws = _workspace(nbytes, dev, ws)
+    _check(lib.msa_encode_memory(ctypes.byref(dd), _ptr(H), T, _ptr(doc_off), n_docs, _ptr(chunk_off), n_chunks,
+                                 _ptr(W_K), _ptr(W_V), _ptr(W_KR), _ptr(out[0]), _ptr(out[1]), _ptr(out[2]),
+                                 _aligned_ptr(ws), nbytes, _stream(stream)))
+    return out
+
+
+# ----------------------------------------------------------------------------
+# stage 2
+# ----------------------------------------------------------------------------
+def route_workspace_size(dims, B: int, n_docs: int, n_chunks: int, k: int, agg: int = AGG_MAX) -> int:
+    return int(lib.msa_route_workspace_size(ctypes.byref(Dims.of(dims)), B, n_docs, n_chunks, k, agg))
+
+
+def route_topk(dims, Hq, W_QR, KR_bar, chunk_off, k: int, agg: int = AGG_MAX, want_doc_scores: bool = False,
+               out=None, ws=None, stream=None):
+    """Top-k documents per query.  Returns (topk_idx [B,k] int32, topk_score [B,k] fp32, doc_scores|None).
+
+    ``W_QR=None`` means ``Hq`` already holds the router queries Q^R [B, n_r*d_r].
+    """
+    import torch
+
+    dd = Dims.of(dims)
+    B = Hq.shape[0]
+    n_docs = chunk_off.numel() - 1
+    n_chunks = KR_bar.shape[0]
+    dev = KR_bar.device
+    if out is None:
+        out = (torch.empty((B, k), dtype=torch.int32, device=dev), torch.empty((B, k), dtype=torch.float32, device=dev),
+               torch.empty((B, n_docs), dtype=torch.float32, device=dev) if want_doc_scores else None)
+    nbytes = route_workspace_size(dims, B, n_docs, n_chunks, k, agg)
+    ws = _workspace(nbytes, dev, ws)
+    _check(lib.msa_route_topk(ctypes.byref(dd), _ptr(Hq), _ptr(W_QR), B, _ptr(KR_bar), _ptr(chunk_off), n_docs,
+                              n_chunks, k, agg, _ptr(out[2]), _ptr(out[0]), _ptr(out[1]), _aligned_ptr(ws), nbytes,
+                              _stream(stream)))
+    return out
+
+
+# ----------------------------------------------------------------------------
+# stage 3
+# ----------------------------------------------------------------------------
+def attend_workspace_size(dims, B: int, k: int, t_loc_max: int, pos_offset: int) -> int:
+    return int(lib.msa_attend_workspace_size(ctypes.byref(Dims.of(dims)), B, k, t_loc_max, pos_offset))
+
+
+def sparse_attend(dims, q, K_bar, V_bar, chunk_off, topk_idx, K_loc, V_loc, loc_len, pos_offset: int,
+                  softmax_scale: float = 0.0, out=None, ws=None, stream=None):
+    """One GQA decode step over [selected docs' K̄; local K].  Returns out [B, n_q, head_dim] bf16."""
+    import torch
+
+    dd = Dims.of(dims)
+    B, k = topk_idx.shape
+    t_loc_max = K_loc.shape[1] if K_loc is not None else 0
+    n_docs = chunk_off.numel() - 1
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, dims.n_q, dims.head_dim), dtype=torch.bfloat16, device=dev)
+    nbytes = attend_workspace_size(dims, B, k, t_loc_max, pos_offset)
+    ws = _workspace(nbytes, dev, ws)
+    _check(lib.msa_sparse_attend(ctypes.byref(dd), _ptr(q), B, _ptr(K_bar), _ptr(V_bar), _ptr(chunk_off), n_docs,
+                                 K_bar.shape[0], _ptr(topk_idx), k, _ptr(K_loc), _ptr(V_loc), _ptr(loc_len),
+                                 t_loc_max, pos_offset, float(softmax_scale), _ptr(out), _aligned_ptr(ws), nbytes,
+                                 _stream(stream)))
+    return out
+
+
+# ----------------------------------------------------------------------------
+# diagnostics
+# ----------------------------------------------------------------------------
+def check_device_errors() -> int:
+    bits = ctypes.c_uint32(0)
+    _check(lib.msa_check_device_errors(ctypes.byref(bits)))
+    return int(bits.value)
+
+
+def trace_enable(on: bool = True):
+    _check(lib.msa_trace_enable(1 if on else 0))
+
+
+def trace_reset():
+    _check(lib.msa_trace_reset())
+
+
+def trace_kernel_names():
+    return [lib.msa_trace_kernel_name(i).decode() for i in range(lib.msa_trace_num_kernels())]
+
+
+def trace_read() -> dict:
+    """{kernel name: (total ms, launches)} since the last reset (synchronises on the trace events)."""
+    out = {}
+    for i, name in enumerate(trace_kernel_names()):
+        ms, n = ctypes.c_double(0), ctypes.c_int64(0)
+        _check(lib.msa_trace_read(i, ctypes.byref(ms), ctypes.byref(n)))
+        out[name] = (ms.value, n.value)
+    return out

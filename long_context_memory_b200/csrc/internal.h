@@ -1,0 +1,114 @@
+// Host-side internals shared by the MSA C-ABI implementation files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/msa.h"
+
+namespace msa {
+
+// ---------------------------------------------------------------------------
+// errors
+// ---------------------------------------------------------------------------
+void set_error(const char* fmt, ...);
+msa_status fail(msa_status code, const char* fmt, ...);
+msa_status cuda_fail(cudaError_t e, const char* what);
+
+#define MSA_CUDA_CHECK(expr)                             \
+  do {                                                   \
+    cudaError_t e_ = (expr);                             \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #expr);  \
+  } while (0)
+
+// Host-side fault injection for the error-path tests: when the environment
+// variable MSA_FAULT is "launch", every entry point fails with MSA_ERR_CUDA
+// after validation and before its first launch.
+bool fault_injected();
+
+// ---------------------------------------------------------------------------
+// kernel ids for tracing
+// ---------------------------------------------------------------------------
+enum KernelId : int {
+  kKQrProj = 0,
+  kKQPrep,
+  kKScan,
+  kKTopkSlice,
+  kKTopkMerge,
+  kKRopeTable,
+  kKAttnSplit,
+  kKAttnCombine,
+  kKEncChunkMap,
+  kKEncTransposeW,
+  kKEncGemmK,
+  kKEncPoolH,
+  kKEncGemmPooled,
+  kKernelCount
+};
+
+// Brackets one kernel launch with trace events when tracing is enabled.
+struct TraceScope {
+  TraceScope(int kernel_id, cudaStream_t s);
+  ~TraceScope();
+  int id;
+  cudaStream_t stream;
+  int slot;
+  unsigned flags;
+};
+
+// ---------------------------------------------------------------------------
+// workspace carving: 256-byte aligned bump allocation inside the caller's ws
+// ---------------------------------------------------------------------------
+struct Carver {
+  char* base;  // may be null when only measuring
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+  template <class T>
+  T* take(size_t count) {
+    off = (off + 255) & ~size_t(255);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += count * sizeof(T);
+    return p;
+  }
+  size_t size() const { return (off + 255) & ~size_t(255); }
+};
+
+// ---------------------------------------------------------------------------
+// device properties and the driver's tensor-map encoder
+// ---------------------------------------------------------------------------
+int sm_count();
+int max_smem_optin();
+msa_status encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, void* gaddr,
+                             const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                             CUtensorMapSwizzle swizzle);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------------------
+// stage implementations (route.cu, attend.cu, encode.cu)
+// ---------------------------------------------------------------------------
+size_t route_workspace(const msa_dims& d, int B, int n_docs, int n_chunks, int k, msa_doc_agg agg,
+                       void* ws, struct RouteWs* out);
+msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int B, const void* KR_bar,
+                        const int32_t* chunk_off, int n_docs, int n_chunks, int k, msa_doc_agg agg,
+                        float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws,
+                        cudaStream_t s);
+
+size_t attend_workspace(const msa_dims& d, int B, int k, int t_loc_max, int pos_offset, void* ws,
+                        struct AttendWs* out);
+msa_status attend_launch(const msa_dims& d, const void* q, int B, const void* K_bar, const void* V_bar,
+                         const int32_t* chunk_off, int n_docs, const int32_t* topk_idx, int k,
+                         const void* K_loc, const void* V_loc, const int32_t* loc_len, int t_loc_max,
+                         int pos_offset, float scale, void* out, void* ws, cudaStream_t s);
+
+size_t encode_workspace(const msa_dims& d, int64_t T, int n_docs, int n_chunks, void* ws,
+                        struct EncodeWs* out);
+msa_status encode_launch(const msa_dims& d, const void* H, int64_t T, const int64_t* doc_off, int n_docs,
+                         const int32_t* chunk_off, int n_chunks, const void* W_K, const void* W_V,
+                         const void* W_KR, void* K_bar, void* V_bar, void* KR_bar, void* ws,
+                         cudaStream_t s);
+
+}  // namespace msa

@@ -1,0 +1,401 @@
+// C ABI of the MSA hot path: argument validation, workspace sizing, tracing,
+// error reporting.  Every entry point validates on the host before it launches
+// anything and never allocates device memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace msa {
+
+__device__ uint32_t g_dev_error = 0;
+
+// ---------------------------------------------------------------------------
+// errors
+// ---------------------------------------------------------------------------
+static thread_local char t_err[512] = "";
+
+void set_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_err, sizeof(t_err), fmt, ap);
+  va_end(ap);
+}
+
+msa_status fail(msa_status code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_err, sizeof(t_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+msa_status cuda_fail(cudaError_t e, const char* what) {
+  set_error("%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+  return MSA_ERR_CUDA;
+}
+
+bool fault_injected() {
+  const char* f = std::getenv("MSA_FAULT");
+  return f && std::strcmp(f, "launch") == 0;
+}
+
+// ---------------------------------------------------------------------------
+// device properties
+// ---------------------------------------------------------------------------
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+int max_smem_optin() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  return n;
+}
+
+// ---------------------------------------------------------------------------
+// tensor maps through the driver entry point (no link-time libcuda dependency)
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+msa_status encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, void* gaddr,
+                             const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                             CUtensorMapSwizzle swizzle) {
+  auto fn = get_encoder();
+  if (!fn) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  uint32_t elem_strides[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, dtype, rank, gaddr, dims, strides_bytes, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+  return MSA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// tracing
+// ---------------------------------------------------------------------------
+namespace {
+const char* kKernelNames[kKernelCount] = {
+    "qr_proj", "q_prep", "scan", "topk_slice", "topk_merge", "rope_table", "attn_split", "attn_combine",
+    "enc_chunk_map", "enc_transpose_w", "enc_gemm_k", "enc_pool_h", "enc_gemm_pooled"};
+
+struct TraceState {
+  std::mutex mu;
+  bool on = false;
+  std::vector<cudaEvent_t> pool;  // reusable events
+  size_t next = 0;
+  struct Rec {
+    int id;
+    cudaEvent_t a, b;
+  };
+  std::vector<Rec> recs;
+  double total_ms[kKernelCount] = {};
+  int64_t launches[kKernelCount] = {};
+};
+TraceState& trace() {
+  static TraceState t;
+  return t;
+}
+
+cudaEvent_t take_event(TraceState& t) {
+  if (t.next == t.pool.size()) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    t.pool.push_back(e);
+  }
+  return t.pool[t.next++];
+}
+
+void flush_trace(TraceState& t) {
+  for (auto& r : t.recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) == cudaSuccess && cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess) {
+      t.total_ms[r.id] += ms;
+      t.launches[r.id] += 1;
+    }
+  }
+  t.recs.clear();
+  t.next = 0;
+}
+}  // namespace
+
+TraceScope::TraceScope(int kernel_id, cudaStream_t s) : id(kernel_id), stream(s), slot(-1), flags(0) {
+  TraceState& t = trace();
+  std::lock_guard<std::mutex> g(t.mu);
+  if (!t.on) return;
+  if (t.pool.size() > 4096 && t.next + 2 > t.pool.size()) flush_trace(t);
+  cudaEvent_t a = take_event(t), b = take_event(t);
+  if (!a || !b) return;
+  // inside stream capture an event becomes a timing node only when recorded as external
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(s, &cs);
+  flags = (cs == cudaStreamCaptureStatusActive) ? cudaEventRecordExternal : cudaEventRecordDefault;
+  cudaEventRecordWithFlags(a, s, flags);
+  t.recs.push_back({kernel_id, a, b});
+  slot = (int)t.recs.size() - 1;
+}
+
+TraceScope::~TraceScope() {
+  if (slot < 0) return;
+  TraceState& t = trace();
+  std::lock_guard<std::mutex> g(t.mu);
+  if (slot < (int)t.recs.size()) cudaEventRecordWithFlags(t.recs[slot].b, stream, flags);
+}
+
+}  // namespace msa
+
+using namespace msa;
+
+// ===========================================================================
+// validation helpers
+// ===========================================================================
+static msa_status check_dims(const msa_dims* d, bool need_kv, bool need_router) {
+  if (!d) return fail(MSA_ERR_INVALID_ARG, "dims is NULL");
+  if (d->chunk != 64) return fail(MSA_ERR_UNSUPPORTED, "chunk must be 64 (got %d)", d->chunk);
+  if (need_router) {
+    if (d->n_r < 1 || d->n_r > 8) return fail(MSA_ERR_UNSUPPORTED, "n_r must be in [1, 8] (got %d)", d->n_r);
+    if (d->d_r != 64 && d->d_r != 128) return fail(MSA_ERR_UNSUPPORTED, "d_r must be 64 or 128 (got %d)", d->d_r);
+  }
+  if (need_kv) {
+    if (d->head_dim != 64 && d->head_dim != 128)
+      return fail(MSA_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", d->head_dim);
+    if (d->n_kv < 1 || d->n_q < 1 || d->n_q % d->n_kv != 0)
+      return fail(MSA_ERR_INVALID_ARG, "n_q (%d) must be a positive multiple of n_kv (%d)", d->n_q, d->n_kv);
+    if (d->n_q / d->n_kv > 16) return fail(MSA_ERR_UNSUPPORTED, "n_q / n_kv must be <= 16");
+    if (!(d->rope_base > 1.0f) || !std::isfinite(d->rope_base))
+      return fail(MSA_ERR_INVALID_ARG, "rope_base must be finite and > 1");
+  }
+  return MSA_OK;
+}
+
+#define CHECK_PTR(p)                                                                           \
+  do {                                                                                         \
+    if (!(p)) return fail(MSA_ERR_INVALID_ARG, "%s is NULL", #p);                              \
+    if (!aligned16(p)) return fail(MSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p);      \
+  } while (0)
+
+#define CHECK_OPT_PTR(p)                                                                       \
+  do {                                                                                         \
+    if ((p) && !aligned16(p)) return fail(MSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p); \
+  } while (0)
+
+// ===========================================================================
+// entry points
+// ===========================================================================
+extern "C" {
+
+const char* msa_last_error(void) { return t_err; }
+
+int32_t msa_version(void) { return 100; }
+
+msa_status msa_check_device_errors(uint32_t* bits_out) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  uint32_t bits = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&bits, g_dev_error, sizeof(bits));
+  if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+  e = cudaMemcpyToSymbol(g_dev_error, &zero, sizeof(zero));
+  if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
+  if (bits_out) *bits_out = bits;
+  if (bits & kDevErrWaitTimeout) return fail(MSA_ERR_TIMEOUT, "a bounded device wait gave up (bits 0x%x)", bits);
+  if (bits) return fail(MSA_ERR_INVALID_ARG, "device reported an out-of-range index (bits 0x%x)", bits);
+  return MSA_OK;
+}
+
+msa_status msa_chunk_offsets(const int64_t* doc_off_host, int32_t n_docs, int32_t chunk, int32_t* chunk_off_host,
+                             int32_t* n_chunks_out) {
+  if (!doc_off_host || !chunk_off_host) return fail(MSA_ERR_INVALID_ARG, "NULL offset array");
+  if (n_docs < 1) return fail(MSA_ERR_INVALID_ARG, "n_docs must be >= 1 (got %d)", n_docs);
+  if (chunk < 1) return fail(MSA_ERR_INVALID_ARG, "chunk must be >= 1 (got %d)", chunk);
+  if (doc_off_host[0] != 0) return fail(MSA_ERR_INVALID_ARG, "doc_off[0] must be 0");
+  int64_t c = 0;
+  chunk_off_host[0] = 0;
+  for (int32_t i = 0; i < n_docs; ++i) {
+    const int64_t len = doc_off_host[i + 1] - doc_off_host[i];
+    if (len < 1) return fail(MSA_ERR_INVALID_ARG, "document %d has %lld tokens (must be >= 1)", i, (long long)len);
+    c += (len + chunk - 1) / chunk;
+    if (c > INT32_MAX) return fail(MSA_ERR_INVALID_ARG, "more than 2^31-1 chunks");
+    chunk_off_host[i + 1] = (int32_t)c;
+  }
+  if (n_chunks_out) *n_chunks_out = (int32_t)c;
+  return MSA_OK;
+}
+
+// ------------------------------ routing ------------------------------
+size_t msa_route_workspace_size(const msa_dims* dims, int32_t B, int32_t n_docs, int32_t n_chunks, int32_t k,
+                                msa_doc_agg agg) {
+  if (!dims || B < 1 || n_docs < 1 || n_chunks < 1 || k < 1) return 0;
+  return route_workspace(*dims, B, n_docs, n_chunks, k, agg, nullptr, nullptr);
+}
+
+msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR, int32_t B, const void* KR_bar,
+                          const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks, int32_t k, msa_doc_agg agg,
+                          float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws, size_t ws_bytes,
+                          void* stream) {
+  msa_status st = check_dims(dims, false, true);
+  if (st != MSA_OK) return st;
+  if (W_QR && (dims->hidden < 64 || dims->hidden % 64 != 0))
+    return fail(MSA_ERR_UNSUPPORTED, "hidden must be a positive multiple of 64 (got %d)", dims->hidden);
+  if (B < 1) return fail(MSA_ERR_INVALID_ARG, "B must be >= 1 (got %d)", B);
+  if (n_docs < 1 || n_chunks < n_docs)
+    return fail(MSA_ERR_INVALID_ARG, "need 1 <= n_docs <= n_chunks (got %d, %d)", n_docs, n_chunks);
+  if (k < 1 || k > n_docs || k > 256)
+    return fail(MSA_ERR_INVALID_ARG, "k must be in [1, min(n_docs, 256)] (got %d, n_docs %d)", k, n_docs);
+  if (agg != MSA_AGG_MAX && agg != MSA_AGG_MEAN) return fail(MSA_ERR_INVALID_ARG, "unknown aggregation %d", (int)agg);
+  const int n_slices = (n_docs + 4095) / 4096;
+  if ((size_t)n_slices * k > 24576) return fail(MSA_ERR_UNSUPPORTED, "n_docs * k too large for the top-k merge");
+  CHECK_PTR(Hq);
+  CHECK_OPT_PTR(W_QR);
+  CHECK_PTR(KR_bar);
+  CHECK_PTR(chunk_off);
+  CHECK_OPT_PTR(doc_scores);
+  CHECK_PTR(topk_idx);
+  CHECK_PTR(topk_score);
+  const size_t need = route_workspace(*dims, B, n_docs, n_chunks, k, agg, nullptr, nullptr);
+  if (ws_bytes < need) return fail(MSA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
+  if (need && (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)))
+    return fail(MSA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
+  if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
+  return route_launch(*dims, Hq, W_QR, B, KR_bar, chunk_off, n_docs, n_chunks, k, agg, doc_scores, topk_idx,
+                      topk_score, ws, static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------ attention ------------------------------
+size_t msa_attend_workspace_size(const msa_dims* dims, int32_t B, int32_t k, int32_t t_loc_max, int32_t pos_offset) {
+  if (!dims || B < 1 || k < 1 || t_loc_max < 0) return 0;
+  return attend_workspace(*dims, B, k, t_loc_max, pos_offset, nullptr, nullptr);
+}
+
+msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, const void* K_bar, const void* V_bar,
+                             const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks, const int32_t* topk_idx,
+                             int32_t k, const void* K_loc, const void* V_loc, const int32_t* loc_len,
+                             int32_t t_loc_max, int32_t pos_offset, float softmax_scale, void* out, void* ws,
+                             size_t ws_bytes, void* stream) {
+  msa_status st = check_dims(dims, true, false);
+  if (st != MSA_OK) return st;
+  if (B < 1) return fail(MSA_ERR_INVALID_ARG, "B must be >= 1 (got %d)", B);
+  if (n_docs < 1 || n_chunks < n_docs)
+    return fail(MSA_ERR_INVALID_ARG, "need 1 <= n_docs <= n_chunks (got %d, %d)", n_docs, n_chunks);
+  if (k < 1 || k > n_docs || k > 256)
+    return fail(MSA_ERR_INVALID_ARG, "k must be in [1, min(n_docs, 256)] (got %d)", k);
+  if (t_loc_max < 0) return fail(MSA_ERR_INVALID_ARG, "t_loc_max must be >= 0");
+  if (pos_offset < 0 || (int64_t)pos_offset + t_loc_max > (1 << 24))
+    return fail(MSA_ERR_INVALID_ARG, "positions must lie in [0, 2^24)");
+  if (!(softmax_scale >= 0.f) || !std::isfinite(softmax_scale))
+    return fail(MSA_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+  CHECK_PTR(q);
+  CHECK_PTR(K_bar);
+  CHECK_PTR(V_bar);
+  CHECK_PTR(chunk_off);
+  CHECK_PTR(topk_idx);
+  if (t_loc_max > 0) {
+    CHECK_PTR(K_loc);
+    CHECK_PTR(V_loc);
+  }
+  CHECK_PTR(loc_len);
+  CHECK_PTR(out);
+  const size_t need = attend_workspace(*dims, B, k, t_loc_max, pos_offset, nullptr, nullptr);
+  if (ws_bytes < need) return fail(MSA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
+  if (need && (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)))
+    return fail(MSA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
+  if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
+  return attend_launch(*dims, q, B, K_bar, V_bar, chunk_off, n_docs, topk_idx, k, K_loc, V_loc, loc_len, t_loc_max,
+                       pos_offset, softmax_scale, out, ws, static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------ encode ------------------------------
+size_t msa_encode_workspace_size(const msa_dims* dims, int64_t T, int32_t n_docs, int32_t n_chunks) {
+  if (!dims || T < 1 || n_docs < 1 || n_chunks < 1) return 0;
+  return encode_workspace(*dims, T, n_docs, n_chunks, nullptr, nullptr);
+}
+
+msa_status msa_encode_memory(const msa_dims* dims, const void* H, int64_t T, const int64_t* doc_off, int32_t n_docs,
+                             const int32_t* chunk_off, int32_t n_chunks, const void* W_K, const void* W_V,
+                             const void* W_KR, void* K_bar, void* V_bar, void* KR_bar, void* ws, size_t ws_bytes,
+                             void* stream) {
+  msa_status st = check_dims(dims, true, true);
+  if (st != MSA_OK) return st;
+  if (dims->hidden < 64 || dims->hidden % 64 != 0)
+    return fail(MSA_ERR_UNSUPPORTED, "hidden must be a positive multiple of 64 (got %d)", dims->hidden);
+  if ((dims->n_kv * dims->head_dim) % 256 != 0 || (dims->n_r * dims->d_r) % 256 != 0)
+    return fail(MSA_ERR_UNSUPPORTED, "n_kv*head_dim and n_r*d_r must be multiples of 256");
+  if (T < 1 || n_docs < 1 || n_chunks < n_docs || (int64_t)n_chunks > (T + 63) / 64 + n_docs)
+    return fail(MSA_ERR_INVALID_ARG, "inconsistent T / n_docs / n_chunks (%lld, %d, %d)", (long long)T, n_docs,
+                n_chunks);
+  CHECK_PTR(H);
+  CHECK_PTR(doc_off);
+  CHECK_PTR(chunk_off);
+  CHECK_PTR(W_K);
+  CHECK_PTR(W_V);
+  CHECK_PTR(W_KR);
+  CHECK_PTR(K_bar);
+  CHECK_PTR(V_bar);
+  CHECK_PTR(KR_bar);
+  const size_t need = encode_workspace(*dims, T, n_docs, n_chunks, nullptr, nullptr);
+  if (ws_bytes < need) return fail(MSA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
+  if (need && (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)))
+    return fail(MSA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
+  if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
+  return encode_launch(*dims, H, T, doc_off, n_docs, chunk_off, n_chunks, W_K, W_V, W_KR, K_bar, V_bar, KR_bar, ws,
+                       static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------ tracing ------------------------------
+msa_status msa_trace_enable(int32_t on) {
+  TraceState& t = trace();
+  std::lock_guard<std::mutex> g(t.mu);
+  t.on = on != 0;
+  return MSA_OK;
+}
+
+msa_status msa_trace_reset(void) {
+  TraceState& t = trace();
+  std::lock_guard<std::mutex> g(t.mu);
+  flush_trace(t);
+  for (int i = 0; i < kKernelCount; ++i) {
+    t.total_ms[i] = 0.0;
+    t.launches[i] = 0;
+  }
+  return MSA_OK;
+}
+
+int32_t msa_trace_num_kernels(void) { return kKernelCount; }
+
+const char* msa_trace_kernel_name(int32_t kernel_id) {
+  if (kernel_id < 0 || kernel_id >= kKernelCount) return "";
+  return kKernelNames[kernel_id];
+}
+
+msa_status msa_trace_read(int32_t kernel_id, double* total_ms, int64_t* launches) {
+  if (kernel_id < 0 || kernel_id >= kKernelCount) return fail(MSA_ERR_INVALID_ARG, "bad kernel id %d", kernel_id);
+  TraceState& t = trace();
+  std::lock_guard<std::mutex> g(t.mu);
+  flush_trace(t);
+  if (total_ms) *total_ms = t.total_ms[kernel_id];
+  if (launches) *launches = t.launches[kernel_id];
+  return MSA_OK;
+}
+
+}  // extern "C"

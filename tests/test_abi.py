@@ -1,0 +1,140 @@
+"""Host-side tests of the C ABI: the library loads, exports every declared
+symbol, computes the chunk layout, sizes workspaces and rejects bad arguments
+with the documented status before launching anything (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as O
+from long_context_memory_b200 import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def msa():
+    from long_context_memory_b200 import build
+
+    if build.needs_build():
+        build.build()
+    import long_context_memory_b200 as m
+
+    return m
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "msa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(msa_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(msa):
+    names = declared_symbols()
+    assert len(names) >= 14
+    cdll = ctypes.CDLL(msa.LIB_PATH)
+    for n in names:
+        assert hasattr(cdll, n), f"missing export {n}"
+    assert msa.lib.msa_version() >= 100
+
+
+def test_library_targets_sm100a_only(msa):
+    # the build passes exactly one gencode: compute_100a -> sm_100a
+    from long_context_memory_b200 import build
+
+    src = open(build.__file__).read()
+    assert "arch=compute_100a,code=sm_100a" in src
+
+
+@pytest.mark.parametrize("lens", [[1], [64, 65, 1, 128], [3000, 7, 64 * 9 + 1]])
+def test_chunk_offsets_match_oracle(msa, lens):
+    doc_off = W.offsets_from_lengths(np.asarray(lens))
+    co, n = msa.chunk_offsets(doc_off)
+    o_co, tok0, *_ = O.chunk_layout(doc_off)
+    assert np.array_equal(co, o_co) and n == len(tok0)
+
+
+def test_chunk_offsets_rejects_empty_doc(msa):
+    with pytest.raises(msa.MSAError) as e:
+        msa.chunk_offsets(np.array([0, 5, 5, 9]))
+    assert e.value.code == 1 and "document 1" in str(e.value)
+
+
+def _dims(**kw):
+    d = dict(hidden=256, n_q=8, n_kv=2, head_dim=64, n_r=4, d_r=64, chunk=64, rope_base=1e6)
+    d.update(kw)
+    return W.Dims(**d)
+
+
+FAKE = 0x10000  # 16-byte aligned non-null "device" address; never dereferenced
+
+
+def _route(msa, dims, B=1, n_docs=10, n_chunks=20, k=4, agg=0, ws_bytes=None, Hq=FAKE, kr=FAKE, idx=FAKE):
+    dd = msa.Dims.of(dims)
+    need = msa.lib.msa_route_workspace_size(ctypes.byref(dd), B, n_docs, n_chunks, k, agg)
+    if ws_bytes is None:
+        ws_bytes = need
+    return msa.lib.msa_route_topk(ctypes.byref(dd), Hq, None, B, kr, FAKE, n_docs, n_chunks, k, agg, None, idx, FAKE,
+                                  0x100000 if ws_bytes else None, ws_bytes, None)
+
+
+def test_route_validation(msa):
+    ok = _dims()
+    assert _route(msa, ok, k=0) == 1
+    assert _route(msa, ok, k=11) == 1                       # k > n_docs
+    assert _route(msa, ok, B=0) == 1
+    assert _route(msa, ok, n_chunks=5) == 1                 # fewer chunks than docs
+    assert _route(msa, _dims(d_r=96)) == 2                  # unsupported router dim
+    assert _route(msa, _dims(n_r=9)) == 2
+    assert _route(msa, _dims(chunk=32)) == 2
+    assert _route(msa, ok, Hq=FAKE + 4) == 1                # misaligned
+    assert _route(msa, ok, kr=None) == 1                    # NULL
+    assert _route(msa, ok, agg=7) == 1
+    assert _route(msa, ok, ws_bytes=16) == 3                # workspace too small
+    assert "workspace too small" in msa.lib.msa_last_error().decode()
+
+
+def test_route_fault_injection_before_launch(msa, monkeypatch):
+    monkeypatch.setenv("MSA_FAULT", "launch")
+    assert _route(msa, _dims()) == 4
+    assert "injected" in msa.lib.msa_last_error().decode()
+
+
+def _attend(msa, dims, B=1, k=2, n_docs=4, n_chunks=8, t_loc=16, pos=2, scale=0.0, ws_bytes=None, q=FAKE):
+    dd = msa.Dims.of(dims)
+    need = msa.lib.msa_attend_workspace_size(ctypes.byref(dd), B, k, t_loc, pos)
+    if ws_bytes is None:
+        ws_bytes = need
+    return msa.lib.msa_sparse_attend(ctypes.byref(dd), q, B, FAKE, FAKE, FAKE, n_docs, n_chunks, FAKE, k, FAKE, FAKE,
+                                     FAKE, t_loc, pos, scale, FAKE, 0x100000, ws_bytes, None)
+
+
+def test_attend_validation(msa):
+    ok = _dims()
+    assert _attend(msa, _dims(head_dim=96)) == 2
+    assert _attend(msa, _dims(n_q=6, n_kv=4)) == 1          # n_q not a multiple of n_kv
+    assert _attend(msa, _dims(n_q=64, n_kv=2)) == 2         # GQA group > 16
+    assert _attend(msa, ok, k=5) == 1                       # k > n_docs
+    assert _attend(msa, ok, pos=-1) == 1
+    assert _attend(msa, ok, scale=float("nan")) == 1
+    assert _attend(msa, ok, q=FAKE + 2) == 1
+    assert _attend(msa, ok, ws_bytes=8) == 3
+
+
+def test_encode_validation(msa):
+    dd = msa.Dims.of(_dims(hidden=100))
+    r = msa.lib.msa_encode_memory(ctypes.byref(dd), FAKE, 1000, FAKE, 3, FAKE, 20, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                  None, 0, None)
+    assert r == 2
+
+
+def test_workspace_sizes_grow_with_problem(msa):
+    d = msa.Dims.of(W.QWEN3_4B_DIMS)
+    a = msa.lib.msa_route_workspace_size(ctypes.byref(d), 1, 500, 16000, 16, 0)
+    b = msa.lib.msa_route_workspace_size(ctypes.byref(d), 32, 500, 16000, 16, 0)
+    assert 0 < a < b
+    assert msa.lib.msa_route_workspace_size(ctypes.byref(d), 0, 500, 16000, 16, 0) == 0
+    x = msa.lib.msa_attend_workspace_size(ctypes.byref(d), 1, 16, 4096, 16)
+    assert x >= 4096 * 64 * 8   # the local RoPE table alone

@@ -1,0 +1,137 @@
+"""GPU parity of stage 3 (sparse generation attention) against the CPU oracle, through the C ABI."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle as O
+from long_context_memory_b200 import workloads as W
+from helpers import bf16_of, check_attention
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def msa(cuda_device):
+    import long_context_memory_b200 as m
+
+    return m
+
+
+def _dev(a, device):
+    return W.to_torch(np.ascontiguousarray(a)).to(device)
+
+
+def _attend(msa, dims, c, device, pos_offset, scale=0.0):
+    import torch
+
+    co, C = msa.chunk_offsets(c["doc_off"])
+    out = msa.sparse_attend(dims, _dev(c["q"], device), _dev(c["K_bar"], device), _dev(c["V_bar"], device),
+                            torch.from_numpy(co).to(device), torch.from_numpy(c["topk"].astype(np.int32)).to(device),
+                            _dev(c["K_loc"], device), _dev(c["V_loc"], device),
+                            torch.from_numpy(c["loc_len"].astype(np.int32)).to(device), pos_offset, scale)
+    torch.cuda.synchronize()
+    assert msa.check_device_errors() == 0
+    return out.float().cpu().numpy()
+
+
+def _case(seed, B, n_q, n_kv, D, n_docs, k, t_loc, loc_len=None, lo=1, hi=900):
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(lo, hi + 1, size=n_docs)
+    doc_off = W.offsets_from_lengths(lens)
+    co, *_ = O.chunk_layout(doc_off)
+    C = int(co[-1])
+    topk = np.stack([rng.permutation(n_docs)[:k] for _ in range(B)])
+    if loc_len is None:
+        loc_len = rng.integers(1, t_loc + 1, size=B)
+    return dict(doc_off=doc_off, chunk_off=co, q=W.normal_bf16(rng, (B, n_q, D)),
+                K_bar=W.normal_bf16(rng, (C, n_kv, D)), V_bar=W.normal_bf16(rng, (C, n_kv, D)),
+                K_loc=W.normal_bf16(rng, (B, t_loc, n_kv, D)), V_loc=W.normal_bf16(rng, (B, t_loc, n_kv, D)),
+                loc_len=np.asarray(loc_len), topk=topk)
+
+
+def _oracle(c, pos_offset, base, scale=0.0):
+    return O.sparse_attend(c["q"], c["K_bar"], c["V_bar"], c["chunk_off"], c["topk"], c["K_loc"], c["V_loc"],
+                           c["loc_len"], pos_offset, base, scale)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("n_q,n_kv", [(8, 2), (32, 8), (16, 16), (16, 1)])
+def test_attend_parity_shapes(msa, cuda_device, D, n_q, n_kv):
+    B = 3
+    c = _case(D + n_q + n_kv, B, n_q, n_kv, D, n_docs=40, k=6, t_loc=200)
+    dims = W.Dims(hidden=256, n_q=n_q, n_kv=n_kv, head_dim=D, n_r=4, d_r=64, rope_base=1e6)
+    out = _attend(msa, dims, c, cuda_device, pos_offset=6)
+    check_attention(out, _oracle(c, 6, 1e6), where=f"D={D} G={n_q // n_kv}")
+
+
+@pytest.mark.parametrize("pos_offset,base", [(0, 1e4), (16, 1e6), (5000, 1e6), (123457, 5e5)])
+def test_attend_positions(msa, cuda_device, pos_offset, base):
+    c = _case(3, 2, 8, 2, 128, n_docs=20, k=4, t_loc=300, loc_len=[300, 1])
+    dims = W.Dims(hidden=256, n_q=8, n_kv=2, head_dim=128, n_r=4, d_r=64, rope_base=base)
+    out = _attend(msa, dims, c, cuda_device, pos_offset=pos_offset)
+    check_attention(out, _oracle(c, pos_offset, base), where=f"o={pos_offset}")
+
+
+def test_attend_no_local_tokens_and_scale(msa, cuda_device):
+    c = _case(4, 2, 8, 2, 64, n_docs=10, k=3, t_loc=8, loc_len=[0, 8])
+    dims = W.Dims(hidden=256, n_q=8, n_kv=2, head_dim=64, n_r=4, d_r=64)
+    out = _attend(msa, dims, c, cuda_device, pos_offset=3, scale=0.05)
+    check_attention(out, _oracle(c, 3, 1e6, 0.05))
+
+
+def test_attend_long_docs_many_splits(msa, cuda_device):
+    c = _case(5, 1, 32, 8, 128, n_docs=30, k=16, t_loc=2000, loc_len=[1999], lo=2000, hi=20000)
+    dims = W.Dims(hidden=2560, n_q=32, n_kv=8, head_dim=128, n_r=8, d_r=128)
+    out = _attend(msa, dims, c, cuda_device, pos_offset=16)
+    check_attention(out, _oracle(c, 16, 1e6))
+
+
+def test_attend_single_key_closed_form(msa, cuda_device):
+    # one one-chunk doc and no local tokens: the output is that chunk's value row
+    rng = np.random.default_rng(6)
+    c = dict(doc_off=np.array([0, 10]), chunk_off=np.array([0, 1]), q=W.normal_bf16(rng, (1, 4, 64)),
+             K_bar=W.normal_bf16(rng, (1, 2, 64)), V_bar=W.normal_bf16(rng, (1, 2, 64)),
+             K_loc=W.normal_bf16(rng, (1, 4, 2, 64)), V_loc=W.normal_bf16(rng, (1, 4, 2, 64)),
+             loc_len=np.array([0]), topk=np.array([[0]]))
+    dims = W.Dims(hidden=256, n_q=4, n_kv=2, head_dim=64, n_r=4, d_r=64)
+    out = _attend(msa, dims, c, cuda_device, pos_offset=1)
+    V = O.bf16_to_f64(c["V_bar"])[0]
+    for g in range(4):
+        assert np.allclose(out[0, g], V[g // 2], atol=1e-2)
+
+
+def test_attend_tiny_config_full_pipeline(msa, cuda_device):
+    c = W.tiny_config()
+    d = c["dims"]
+    Kb, Vb, KRb = O.encode_memory(c["H"], c["doc_off"], c["W_K"], c["W_V"], c["W_KR"], d.n_kv, d.head_dim, d.n_r,
+                                  d.d_r)
+    co, *_ = O.chunk_layout(c["doc_off"])
+    KR = bf16_of(KRb)
+    _, idx, _ = O.route_topk(O.router_query(c["Hq"], c["W_QR"], d.n_r, d.d_r), KR, co, c["k"])
+    case = dict(doc_off=c["doc_off"], chunk_off=co, q=c["q"], K_bar=bf16_of(Kb), V_bar=bf16_of(Vb), K_loc=c["K_loc"],
+                V_loc=c["V_loc"], loc_len=c["loc_len"], topk=idx)
+    out = _attend(msa, d, case, cuda_device, pos_offset=c["pos_offset"])
+    check_attention(out, _oracle(case, c["pos_offset"], d.rope_base))
+
+
+def test_attend_mem1m_full_size(msa, cuda_device):
+    m = W.mem1m_config()
+    d = m["dims"]
+    co, *_ = O.chunk_layout(m["doc_off"])
+    case = dict(doc_off=m["doc_off"], chunk_off=co, q=m["q"], K_bar=m["K_bar"], V_bar=m["V_bar"], K_loc=m["K_loc"],
+                V_loc=m["V_loc"], loc_len=m["loc_len"], topk=m["planted_docs"])
+    out = _attend(msa, d, case, cuda_device, pos_offset=m["pos_offset"])
+    check_attention(out, _oracle(case, m["pos_offset"], d.rope_base))
+
+
+def test_attend_mem16m_batch32_sampled(msa, cuda_device):
+    m = W.mem16m_config()
+    d = m["dims"]
+    co, *_ = O.chunk_layout(m["doc_off"])
+    case = dict(doc_off=m["doc_off"], chunk_off=co, q=m["q"], K_bar=m["K_bar"], V_bar=m["V_bar"], K_loc=m["K_loc"],
+                V_loc=m["V_loc"], loc_len=m["loc_len"], topk=m["planted_docs"])
+    out = _attend(msa, d, case, cuda_device, pos_offset=m["pos_offset"])
+    for b in [0, 7, 31]:
+        sub = {kk: (v[b:b + 1] if kk in ("q", "K_loc", "V_loc", "loc_len", "topk") else v) for kk, v in case.items()}
+        check_attention(out[b:b + 1], _oracle(sub, m["pos_offset"], d.rope_base), where=f"b={b}")

@@ -1,0 +1,174 @@
+"""GPU parity of stage 2 (routing + top-k) against the CPU oracle, through the C ABI."""
+import numpy as np
+import pytest
+
+import oracle as O
+from long_context_memory_b200 import workloads as W
+from helpers import SCORE_ATOL, bf16_of, check_topk
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def msa(cuda_device):
+    import long_context_memory_b200 as m
+
+    return m
+
+
+def _dev(a, device):
+    import torch
+
+    return W.to_torch(np.ascontiguousarray(a)).to(device)
+
+
+def _route_case(seed, n_docs, B, n_r, d_r, lo=1, hi=700, hidden=256):
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(lo, hi + 1, size=n_docs)
+    doc_off = W.offsets_from_lengths(lens)
+    chunk_off, C = None, None
+    dims = W.Dims(hidden=hidden, n_q=8, n_kv=2, head_dim=64, n_r=n_r, d_r=d_r)
+    co, *_ = O.chunk_layout(doc_off)
+    C = int(co[-1])
+    KR = W.normal_bf16(rng, (C, n_r, d_r))
+    QR = W.normal_bf16(rng, (B, n_r * d_r))
+    Hq = W.normal_bf16(rng, (B, hidden))
+    Wqr = W.normal_bf16(rng, (hidden, n_r * d_r), 1 / np.sqrt(hidden))
+    return dims, doc_off, KR, QR, Hq, Wqr, rng
+
+
+def _run(msa, dims, Hq, Wqr, KR, doc_off, k, agg, device):
+    import torch
+
+    co, C = msa.chunk_offsets(doc_off)
+    idx, sc, ds = msa.route_topk(dims, _dev(Hq, device), None if Wqr is None else _dev(Wqr, device),
+                                 _dev(KR, device), torch.from_numpy(co).to(device), k, agg=agg, want_doc_scores=True)
+    torch.cuda.synchronize()
+    assert msa.check_device_errors() == 0
+    return idx.cpu().numpy(), sc.cpu().numpy(), ds.cpu().numpy()
+
+
+@pytest.mark.parametrize("B", [1, 3, 8, 13, 32, 40])
+@pytest.mark.parametrize("n_r,d_r", [(8, 128), (4, 64), (3, 128)])
+def test_route_direct_query_parity(msa, cuda_device, B, n_r, d_r):
+    dims, doc_off, KR, QR, Hq, Wqr, _ = _route_case(100 + B + n_r, 300, B, n_r, d_r)
+    k = 16
+    idx, sc, ds = _run(msa, dims, QR, None, KR, doc_off, k, msa.AGG_MAX, cuda_device)
+    co, *_ = O.chunk_layout(doc_off)
+    s, _, _ = O.route_topk(O.bf16_to_f64(QR).reshape(B, n_r, d_r), KR, co, k)
+    assert np.max(np.abs(ds - s)) < SCORE_ATOL, np.max(np.abs(ds - s))
+    for b in range(B):
+        check_topk(idx[b], sc[b], s[b], k, where=f"b={b}")
+
+
+@pytest.mark.parametrize("agg", [0, 1])
+def test_route_projection_and_aggregation(msa, cuda_device, agg):
+    B = 5
+    dims, doc_off, KR, QR, Hq, Wqr, _ = _route_case(7, 257, B, 8, 128, hidden=512)
+    k = 9
+    idx, sc, ds = _run(msa, dims, Hq, Wqr, KR, doc_off, k, agg, cuda_device)
+    co, *_ = O.chunk_layout(doc_off)
+    QRo = O.router_query(Hq, Wqr, 8, 128)
+    S = O.chunk_scores(QRo, KR)
+    s = O.doc_scores(S, co, "max" if agg == 0 else "mean")
+    assert np.max(np.abs(ds - s)) < SCORE_ATOL
+    for b in range(B):
+        check_topk(idx[b], sc[b], s[b], k, where=f"agg={agg} b={b}")
+
+
+def test_route_edge_shapes(msa, cuda_device):
+    # one-chunk docs, k = n_docs, chunk count not a multiple of the tile, single doc
+    for seed, n_docs, lo, hi, k in [(1, 17, 1, 64, 17), (2, 1, 5, 5, 1), (3, 40, 1, 1, 40), (4, 33, 60, 70, 1)]:
+        dims, doc_off, KR, QR, *_ = _route_case(seed, n_docs, 2, 8, 128, lo=lo, hi=hi)
+        idx, sc, ds = _run(msa, dims, QR, None, KR, doc_off, k, 0, cuda_device)
+        co, *_ = O.chunk_layout(doc_off)
+        s, _, _ = O.route_topk(O.bf16_to_f64(QR).reshape(2, 8, 128), KR, co, k)
+        for b in range(2):
+            check_topk(idx[b], sc[b], s[b], k, where=f"case {seed} b={b}")
+
+
+def test_route_many_docs_two_pass_merge(msa, cuda_device):
+    # > 4096 docs forces slice top-k + merge
+    dims, doc_off, KR, QR, *_ = _route_case(11, 9000, 3, 4, 64, lo=1, hi=130)
+    idx, sc, ds = _run(msa, dims, QR, None, KR, doc_off, 32, 0, cuda_device)
+    co, *_ = O.chunk_layout(doc_off)
+    s, _, _ = O.route_topk(O.bf16_to_f64(QR).reshape(3, 4, 64), KR, co, 32)
+    assert np.max(np.abs(ds - s)) < SCORE_ATOL
+    for b in range(3):
+        check_topk(idx[b], sc[b], s[b], 32, where=f"b={b}")
+
+
+def test_route_ties_prefer_lower_id(msa, cuda_device):
+    # identical documents -> identical scores -> ids ascending
+    rng = np.random.default_rng(5)
+    dims = W.Dims(hidden=256, n_q=8, n_kv=2, head_dim=64, n_r=8, d_r=128)
+    one = W.normal_bf16(rng, (3, 8, 128))
+    KR = np.concatenate([one] * 50)
+    doc_off = W.offsets_from_lengths(np.full(50, 150))        # 3 chunks each
+    QR = W.normal_bf16(rng, (1, 1024))
+    idx, sc, ds = _run(msa, dims, QR, None, KR, doc_off, 10, 0, cuda_device)
+    assert list(idx[0]) == list(range(10))
+    assert np.all(sc[0] == sc[0][0])
+
+
+def test_route_planted_equal_key_scores_one(msa, cuda_device):
+    dims, doc_off, KR, QR, *_ = _route_case(21, 100, 2, 8, 128)
+    co, *_ = O.chunk_layout(doc_off)
+    KR[co[37] + 0] = QR[0].reshape(8, 128)
+    KR[co[81] + 0] = QR[1].reshape(8, 128)
+    idx, sc, ds = _run(msa, dims, QR, None, KR, doc_off, 4, 0, cuda_device)
+    assert idx[0, 0] == 37 and idx[1, 0] == 81
+    assert abs(sc[0, 0] - 1.0) < 1e-5 and abs(sc[1, 0] - 1.0) < 1e-5
+    assert np.all(np.abs(ds) <= 1.0 + 1e-5)
+
+
+def test_route_tiny_config_full_pipeline(msa, cuda_device):
+    c = W.tiny_config()
+    d = c["dims"]
+    _, _, KRb = O.encode_memory(c["H"], c["doc_off"], c["W_K"], c["W_V"], c["W_KR"], d.n_kv, d.head_dim, d.n_r, d.d_r)
+    KR = bf16_of(KRb)
+    idx, sc, ds = _run(msa, d, c["Hq"], c["W_QR"], KR, c["doc_off"], c["k"], 0, cuda_device)
+    co, *_ = O.chunk_layout(c["doc_off"])
+    s, _, _ = O.route_topk(O.router_query(c["Hq"], c["W_QR"], d.n_r, d.d_r), KR, co, c["k"])
+    check_topk(idx[0], sc[0], s[0], c["k"])
+    assert set(idx[0, :2].tolist()) == set(c["planted"])
+
+
+def test_route_mem1m_full_size(msa, cuda_device):
+    c = W.mem1m_config(with_kv=False)
+    d = c["dims"]
+    idx, sc, ds = _run(msa, d, c["QR"], None, c["KR"], c["doc_off"], 16, 0, cuda_device)
+    co, *_ = O.chunk_layout(c["doc_off"])
+    s, _, _ = O.route_topk(O.bf16_to_f64(c["QR"]).reshape(1, d.n_r, d.d_r), c["KR"], co, 16)
+    assert np.max(np.abs(ds - s)) < SCORE_ATOL
+    check_topk(idx[0], sc[0], s[0], 16)
+    assert set(idx[0].tolist()) == set(c["planted_docs"][0].tolist())
+    # the projection path at full size
+    idx2, sc2, ds2 = _run(msa, d, c["Hq"], c["W_QR"], c["KR"], c["doc_off"], 16, 0, cuda_device)
+    s2, _, _ = O.route_topk(O.router_query(c["Hq"], c["W_QR"], d.n_r, d.d_r), c["KR"], co, 16)
+    assert np.max(np.abs(ds2 - s2)) < SCORE_ATOL
+    check_topk(idx2[0], sc2[0], s2[0], 16)
+
+
+def test_route_mem16m_batch32_sampled(msa, cuda_device):
+    c = W.mem16m_config(with_kv=False)
+    d = c["dims"]
+    B = c["B"]
+    idx, sc, ds = _run(msa, d, c["QR"], None, c["KR"], c["doc_off"], 16, 0, cuda_device)
+    co, *_ = O.chunk_layout(c["doc_off"])
+    rng = np.random.default_rng(0)
+    sample = np.unique(np.concatenate([c["planted_docs"].ravel(), rng.choice(len(co) - 1, 600, replace=False)]))
+    rows = np.concatenate([np.arange(co[i], co[i + 1]) for i in sample])
+    S = O.chunk_scores(O.bf16_to_f64(c["QR"]).reshape(B, d.n_r, d.d_r), c["KR"], rows=rows)
+    pos = 0
+    for i in sample:
+        n = co[i + 1] - co[i]
+        s_i = S[:, pos:pos + n].max(axis=1)
+        pos += n
+        assert np.max(np.abs(ds[:, i] - s_i)) < SCORE_ATOL
+    for b in range(B):
+        # planted cosines 0.21 + 0.01 p: the top-16 are the planted docs, strongest first
+        want = c["planted_docs"][b][::-1]
+        assert list(idx[b]) == list(want), (b, idx[b], want)
+        others = np.setdiff1d(np.arange(len(co) - 1), c["planted_docs"][b])
+        assert ds[b, others].max() < sc[b, -1] - 2e-3
