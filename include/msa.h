@@ -109,7 +109,7 @@ msa_status msa_chunk_offsets(const int64_t* doc_off_host, int32_t n_docs, int32_
  *            document-relative positions and of H W_V.
  *   KR_bar   [C, n_r, d_r] bf16 out: chunk means of H W^KR.
  * Requirements: hidden % 64 == 0; n_kv * head_dim and n_r * d_r multiples of
- * 256; chunk == 64.  Rounding: fp32 accumulation, outputs rounded to bf16.
+ * 128; chunk == 64; T < 2^31 - 64.  Rounding: fp32 accumulation, outputs rounded to bf16.
  * ------------------------------------------------------------------------- */
 size_t msa_encode_workspace_size(const msa_dims* dims, int64_t T, int32_t n_docs, int32_t n_chunks);
 msa_status msa_encode_memory(const msa_dims* dims, const void* H, int64_t T, const int64_t* doc_off,

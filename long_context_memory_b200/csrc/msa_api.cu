@@ -339,8 +339,8 @@ msa_status msa_encode_memory(const msa_dims* dims, const void* H, int64_t T, con
   if (st != MSA_OK) return st;
   if (dims->hidden < 64 || dims->hidden % 64 != 0)
     return fail(MSA_ERR_UNSUPPORTED, "hidden must be a positive multiple of 64 (got %d)", dims->hidden);
-  if ((dims->n_kv * dims->head_dim) % 256 != 0 || (dims->n_r * dims->d_r) % 256 != 0)
-    return fail(MSA_ERR_UNSUPPORTED, "n_kv*head_dim and n_r*d_r must be multiples of 256");
+  if ((dims->n_kv * dims->head_dim) % 128 != 0 || (dims->n_r * dims->d_r) % 128 != 0)
+    return fail(MSA_ERR_UNSUPPORTED, "n_kv*head_dim and n_r*d_r must be multiples of 128");
   if (T < 1 || n_docs < 1 || n_chunks < n_docs || (int64_t)n_chunks > (T + 63) / 64 + n_docs)
     return fail(MSA_ERR_INVALID_ARG, "inconsistent T / n_docs / n_chunks (%lld, %d, %d)", (long long)T, n_docs,
                 n_chunks);

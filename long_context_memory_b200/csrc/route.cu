@@ -364,9 +364,11 @@ __global__ void __launch_bounds__(288, 1) scan_kernel(const __grid_constant__ CU
 // --------------------------------------------------------------------------
 // exact block-wide top-k of distinct 64-bit keys in shared memory
 // key = (ordered score << 32) | (0xFFFFFFFF - doc id): larger key = better,
-// equal scores prefer the lower id.  Writes the k best keys, descending, to out.
+// equal scores prefer the lower id.  Radix select from the most significant
+// byte; it stops as soon as the k-th key's bucket is taken whole.  Writes the
+// k best keys, descending, to out[0..k); tmp holds k unsorted winners.
 // --------------------------------------------------------------------------
-__device__ void block_topk(const uint64_t* keys, int n, int k, uint64_t* out, uint32_t* hist,
+__device__ void block_topk(const uint64_t* keys, int n, int k, uint64_t* out, uint64_t* tmp, uint32_t* hist,
                            uint64_t* sh_state) {
   const int tid = threadIdx.x, nt = blockDim.x;
   uint64_t prefix = 0, mask = 0;
@@ -398,13 +400,12 @@ __device__ void block_topk(const uint64_t* keys, int n, int k, uint64_t* out, ui
       const uint32_t excl = incl - tot;  // keys in higher digits than this lane's range
       if (excl < (uint32_t)kk && (uint32_t)kk <= incl) {
         uint32_t above = excl;
-        int digit = 0;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           if (above < (uint32_t)kk && (uint32_t)kk <= above + cnt[j]) {
-            digit = 255 - 8 * tid - j;
             sh_state[0] = above;
-            sh_state[1] = (uint64_t)digit;
+            sh_state[1] = (uint64_t)(255 - 8 * tid - j);
+            sh_state[3] = (above + cnt[j] == (uint32_t)kk) ? 1ull : 0ull;  // bucket taken whole
             break;
           }
           above += cnt[j];
@@ -415,40 +416,29 @@ __device__ void block_topk(const uint64_t* keys, int n, int k, uint64_t* out, ui
     kk -= (int)sh_state[0];
     prefix |= (sh_state[1] & 255ull) << shift;
     mask |= 255ull << shift;
+    const bool done = sh_state[3] != 0;
     __syncthreads();
+    if (done) break;
   }
-  // keys are distinct: the selected set is every key >= prefix
+  // the winners are the keys whose decided high bits are >= prefix (exactly k of them)
   if (tid == 0) sh_state[2] = 0;
   __syncthreads();
   for (int i = tid; i < n; i += nt) {
     const uint64_t key = keys[i];
-    if (key >= prefix) {
+    if ((key & mask) >= prefix) {
       const int pos = (int)atomicAdd(reinterpret_cast<unsigned long long*>(&sh_state[2]), 1ull);
-      if (pos < k) out[pos] = key;
+      if (pos < k) tmp[pos] = key;
     }
   }
   __syncthreads();
-  // bitonic sort (descending) of the k winners, padded to a power of two
-  int m = 1;
-  while (m < k) m <<= 1;
-  for (int i = k + tid; i < m; i += nt) out[i] = 0;
-  __syncthreads();
-  for (int size = 2; size <= m; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = tid; i < m; i += nt) {
-        const int j = i ^ stride;
-        if (j > i) {
-          const bool desc = (i & size) == 0;
-          const uint64_t a = out[i], b = out[j];
-          if (desc ? (a < b) : (a > b)) {
-            out[i] = b;
-            out[j] = a;
-          }
-        }
-      }
-      __syncthreads();
-    }
+  // rank sort: keys are distinct, so each winner's rank is the number of larger winners
+  for (int i = tid; i < k; i += nt) {
+    const uint64_t key = tmp[i];
+    int rank = 0;
+    for (int j = 0; j < k; ++j) rank += tmp[j] > key;
+    out[rank] = key;
   }
+  __syncthreads();
 }
 
 __device__ __forceinline__ uint64_t make_key(uint32_t ordered, int id) {
@@ -462,7 +452,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_slice_kernel(
   extern __shared__ uint64_t sm64[];
   uint64_t* keys = sm64;              // [kSliceDocs]
   uint64_t* out = keys + kSliceDocs;  // [256]
-  uint64_t* state = out + 256;        // [4]
+  uint64_t* tmp = out + 256;          // [256]
+  uint64_t* state = tmp + 256;        // [4]
   uint32_t* hist = reinterpret_cast<uint32_t*>(state + 4);
   const int slice = blockIdx.x, b = blockIdx.y;
   const int d0 = slice * kSliceDocs;
@@ -484,7 +475,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_slice_kernel(
   }
   __syncthreads();
   const int kk = min(k, n);
-  block_topk(keys, n, kk, out, hist, state);
+  block_topk(keys, n, kk, out, tmp, hist, state);
   if (n_slices == 1) {
     for (int i = threadIdx.x; i < kk; i += blockDim.x) {
       topk_idx[(size_t)b * k + i] = (int32_t)(0xFFFFFFFFu - (uint32_t)(out[i] & 0xFFFFFFFFu));
@@ -504,12 +495,13 @@ __global__ void __launch_bounds__(kTopkThreads) topk_merge_kernel(const uint64_t
   const int n = n_slices * k;
   uint64_t* keys = sm64;
   uint64_t* out = keys + n;
-  uint64_t* state = out + 256;
+  uint64_t* tmp = out + 256;
+  uint64_t* state = tmp + 256;
   uint32_t* hist = reinterpret_cast<uint32_t*>(state + 4);
   const int b = blockIdx.x;
   for (int i = threadIdx.x; i < n; i += blockDim.x) keys[i] = cand[(size_t)b * n + i];
   __syncthreads();
-  block_topk(keys, n, k, out, hist, state);
+  block_topk(keys, n, k, out, tmp, hist, state);
   for (int i = threadIdx.x; i < k; i += blockDim.x) {
     topk_idx[(size_t)b * k + i] = (int32_t)(0xFFFFFFFFu - (uint32_t)(out[i] & 0xFFFFFFFFu));
     topk_score[(size_t)b * k + i] = ordered_to_float((uint32_t)(out[i] >> 32));
@@ -542,8 +534,8 @@ size_t scan_smem_bytes(int n_r, int d_r, int nb) {
          2 * kStages * sizeof(uint64_t);
 }
 
-size_t topk_slice_smem() { return (kSliceDocs + 256 + 4) * sizeof(uint64_t) + 256 * sizeof(uint32_t); }
-size_t topk_merge_smem(int n) { return ((size_t)n + 256 + 4) * sizeof(uint64_t) + 256 * sizeof(uint32_t); }
+size_t topk_slice_smem() { return (kSliceDocs + 512 + 4) * sizeof(uint64_t) + 256 * sizeof(uint32_t); }
+size_t topk_merge_smem(int n) { return ((size_t)n + 512 + 4) * sizeof(uint64_t) + 256 * sizeof(uint32_t); }
 
 }  // namespace
 

@@ -271,16 +271,36 @@ def mem16m_config(seed: int = BASE_SEED + 2, T: int = 16_000_000, B: int = 32, *
 # encode workload
 # ----------------------------------------------------------------------------
 def encode_config(T: int = 1_000_000, seed: int = BASE_SEED + 5, median: int = 2048,
-                  dims: Dims = QWEN3_4B_DIMS) -> dict:
-    """Offline encoding: H [T, hidden] ~ N(0,1) bf16, W_K/W_V/W^KR ~ N(0, 1/hidden)."""
+                  dims: Dims = QWEN3_4B_DIMS, with_hidden: bool = True) -> dict:
+    """Offline encoding: H [T, hidden] ~ N(0,1) bf16, W_K/W_V/W^KR ~ N(0, 1/hidden).
+
+    ``with_hidden=False`` leaves H out; draw it on a device with ``encode_hidden``
+    (a [1M x 2560] corpus is 5 GB, too slow to draw and convert in numpy).
+    """
     rng = np.random.default_rng(seed)
     lens = doc_lengths_lognormal(rng, T, median)
     doc_off = offsets_from_lengths(lens)
     hs = 1.0 / math.sqrt(dims.hidden)
-    return dict(
-        name="encode", dims=dims, T=T, doc_off=doc_off, lens=lens,
-        H=normal_bf16(rng, (T, dims.hidden)),
+    out = dict(
+        name="encode", dims=dims, T=T, doc_off=doc_off, lens=lens, seed=seed,
         W_K=normal_bf16(rng, (dims.hidden, dims.n_kv * dims.head_dim), hs),
         W_V=normal_bf16(rng, (dims.hidden, dims.n_kv * dims.head_dim), hs),
         W_KR=normal_bf16(rng, (dims.hidden, dims.n_r * dims.d_r), hs),
     )
+    if with_hidden:
+        out["H"] = normal_bf16(rng, (T, dims.hidden))
+    return out
+
+
+def encode_hidden(T: int, hidden: int, seed: int, device):
+    """H [T, hidden] ~ N(0,1) rounded to bf16, drawn by torch's seeded generator on ``device``."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    H = torch.empty((T, hidden), dtype=torch.bfloat16, device=device)
+    step = 1 << 16
+    for r in range(0, T, step):
+        e = min(T, r + step)
+        H[r:e] = torch.randn((e - r, hidden), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+    return H
