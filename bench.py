@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--impl", default="msa", choices=["msa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the 16M/100M-token routing and the encode measurements")
     return ap.parse_args()
 
 
@@ -199,6 +201,103 @@ def scan_traffic_record(kernel: str):
         return None
 
 
+def kernel_times(msa, stream, step, n):
+    """Per-kernel device time of n eager steps, each kernel bracketed by trace events.
+
+    The launches are queued behind a bounded sleep kernel so that the host is far
+    ahead of the device and every bracket holds only its kernel."""
+    import torch
+
+    msa.trace_reset()
+    msa.trace_enable(True)
+    try:
+        with torch.cuda.stream(stream):
+            torch.cuda._sleep(40_000_000)  # ~20 ms of device time, bounded by the clock
+            for i in range(n):
+                step(i)
+        torch.cuda.synchronize()
+    finally:
+        msa.trace_enable(False)
+    kt = msa.trace_read()
+    msa.trace_reset()
+    return kt
+
+
+def run_extras(msa, dev, hbm_peak):
+    """Routing at 16M (B=32) and 100M tokens (36 layer instances, B=1 and 16), and encoding 1M tokens."""
+    import torch
+
+    from long_context_memory_b200 import profile_cases as PC
+    from long_context_memory_b200 import workloads as W
+
+    out = {}
+    stream = torch.cuda.Stream(device=dev)
+
+    def timed(fn, n, warm=2):
+        with torch.cuda.stream(stream):
+            for _ in range(warm):
+                fn(0)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for i in range(n):
+                fn(i)
+            e1.record(stream)
+            torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    def route_entry(name, case, layers):
+        n = 6 * layers
+        ms = timed(lambda i: case.run(i % layers), n)
+        kt = kernel_times(msa, stream, lambda i: case.run(i % layers), n)
+        sms, scnt = kt["scan"]
+        scan_us = sms / scnt * 1e3
+        gbs = case.scan_bytes / (scan_us * 1e-6) / 1e9
+        out[name] = {"workload": f"{case.T / 1e6:.0f}M-token memory, C={case.C} chunks, B={case.B}, top-{case.k}",
+                     "layers": layers, "ms_per_layer": ms, "memory_tokens_routed_per_s": case.T * case.B / (ms * 1e-3),
+                     "scan": {"avg_us": scan_us, "GB/s": gbs, "frac": gbs / hbm_peak, "bound": "hbm",
+                              "algorithmic_bytes_per_launch": case.scan_bytes},
+                     "kernels_us": {k: v[0] / v[1] * 1e3 for k, v in kt.items() if v[1]}}
+
+    try:
+        c16 = PC.RouteCase(16_000_000, 32, 2048, W.BASE_SEED + 2, dev)
+        route_entry("mem16m_b32_route", c16, 1)
+        del c16
+        free = torch.cuda.mem_get_info(dev)[0]
+        layers = int(max(1, min(36, (free - (8 << 30)) // 3_300_000_000)))
+        c100 = PC.RouteCase(100_000_000, 1, 4096, W.BASE_SEED + 4, dev, layers=layers)
+        route_entry("mem100m_b1_route", c100, layers)
+        c100.set_batch(16, seed=W.BASE_SEED + 40)
+        route_entry("mem100m_b16_route", c100, layers)
+        del c100
+        torch.cuda.empty_cache()
+        enc = PC.EncodeCase(1_000_000, W.BASE_SEED + 5, dev)
+        ms = timed(lambda i: enc.run(), 3, warm=1)
+        kt = kernel_times(msa, stream, lambda i: enc.run(), 3)
+        gms, gcnt = kt["enc_gemm_k"]
+        g_us = gms / gcnt * 1e3
+        tflops = enc.flops_k / (g_us * 1e-6) / 1e12
+        out["encode_1m"] = {"workload": f"encode 1M tokens, hidden 2560, C={enc.C} chunks", "ms": ms,
+                            "tokens_per_s": enc.T / (ms * 1e-3),
+                            "gemm_k": {"avg_us": g_us, "TFLOP/s": tflops, "bound": "tensor",
+                                       "frac_of_bf16_sustained": tflops / bf16_peak()[0],
+                                       "algorithmic_flops": enc.flops_k},
+                            "kernels_us": {k: v[0] / v[1] * 1e3 for k, v in kt.items() if v[1]}}
+        del enc
+        torch.cuda.empty_cache()
+    except Exception as e:  # report, do not hide, a failed extra measurement
+        out["error"] = f"{type(e).__name__}: {e}"
+    return out
+
+
+def bf16_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    return 1400.0, "fallback"
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -232,13 +331,15 @@ def run_gpu(args):
     a_ws = torch.empty(msa.attend_workspace_size(d, B, k, c["t_loc_max"], c["pos_offset"]) + 256,
                        dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(device=dev)
+    # rotation table of the local positions: a constant of the decode session (like the KV cache)
+    rope = msa.rope_cache_build(d, c["t_loc_max"], c["pos_offset"], device=dev)
 
     def step(i):
         x = rot[i % N_ROT]
         j = i % N_ROT
         msa.route_topk(d, x["Hq"], W_QR, x["KR"], chunk_off, k, out=(out_idx[j], out_sc[j], None), ws=r_ws)
         msa.sparse_attend(d, x["q"], x["K_bar"], x["V_bar"], chunk_off, out_idx[j], x["K_loc"], x["V_loc"], loc_len,
-                          c["pos_offset"], out=out_o[j], ws=a_ws)
+                          c["pos_offset"], out=out_o[j], ws=a_ws, rope_cache=rope)
 
     # ---- capture one graph per rotation copy (untraced) ----
     graphs = []
@@ -294,25 +395,7 @@ def run_gpu(args):
     value = T * B * ws / (ms_step * 1e-3)
 
     # ---- per-kernel device time: the same steps, each kernel bracketed by trace events ----
-    msa.trace_reset()
-    msa.trace_enable(True)
-    tgraphs = []
-    try:
-        for i in range(args.steps):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                step(i)
-            tgraphs.append(g)
-    finally:
-        msa.trace_enable(False)
-    with torch.cuda.stream(stream):
-        for rep in range(2):  # first pass warms up; the events keep the second pass's times
-            for g in tgraphs:
-                g.replay()
-    torch.cuda.synchronize()
-    kt = msa.trace_read()
-    msa.trace_reset()
-    del tgraphs
+    kt = kernel_times(msa, stream, step, args.steps)
 
     # ---- roofline of the dominant kernel ----
     hbm_peak, peak_kind = peaks()
@@ -361,7 +444,7 @@ def run_gpu(args):
         x["V_loc"][:, Lm1].copy_(host["v_new"], non_blocking=True)
         msa.route_topk(d, dev_hq, W_QR, x["KR"], chunk_off, k, out=(out_idx[0], out_sc[0], None), ws=r_ws)
         msa.sparse_attend(d, dev_q, x["K_bar"], x["V_bar"], chunk_off, out_idx[0], x["K_loc"], x["V_loc"], loc_len,
-                          c["pos_offset"], out=out_o[0], ws=a_ws)
+                          c["pos_offset"], out=out_o[0], ws=a_ws, rope_cache=rope)
         h_idx.copy_(out_idx[0], non_blocking=True)
         h_sc.copy_(out_sc[0], non_blocking=True)
         h_out.copy_(out_o[0], non_blocking=True)
@@ -385,6 +468,10 @@ def run_gpu(args):
         e2e_ms = float(tt.item())
     e2e_val = T * B * ws / (e2e_ms * 1e-3)
 
+    extras = None
+    if ws == 1 and not args.no_extras:
+        extras = run_extras(msa, dev, hbm_peak)
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         r = time_oracle(c, args.cpu_seconds)
@@ -403,7 +490,10 @@ def run_gpu(args):
             "roofline": roofline, "kernels": kernels, "gpu_launches": gpu_launches,
             "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms},
-            "cpu_baseline": cpu, "clocks": clocks,
+            "cpu_baseline": cpu, "clocks": clocks, "extras": extras,
+            "notes": "value: device time of CUDA-graph replays of the full step; kernels: trace-event brackets "
+                     "of eager launches queued behind a bounded sleep kernel; the local-position RoPE table is "
+                     "built once per decode session (msa_rope_cache_build), outside the step",
         }
         print(json.dumps(line), flush=True)
     if ws > 1:

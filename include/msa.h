@@ -157,6 +157,7 @@ msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR
  *   K_loc, V_loc [B, t_loc_max, n_kv, head_dim] bf16 local KV, K before RoPE;
  *            local token j is rotated to position pos_offset + j.
  *   loc_len  [B] device int32, 0 <= loc_len[b] <= t_loc_max.
+ *   rope_cache  optional table from msa_rope_cache_build (NULL = built in ws).
  *   softmax_scale  0 -> 1/sqrt(head_dim).
  *   out      [B, n_q, head_dim] bf16.
  * Query head g attends with KV head g / (n_q / n_kv).  No mask: the decode
@@ -171,7 +172,26 @@ msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, con
                              const void* V_bar, const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks,
                              const int32_t* topk_idx, int32_t k, const void* K_loc, const void* V_loc,
                              const int32_t* loc_len, int32_t t_loc_max, int32_t pos_offset,
-                             float softmax_scale, void* out, void* ws, size_t ws_bytes, void* stream);
+                             const void* rope_cache, float softmax_scale, void* out, void* ws, size_t ws_bytes,
+                             void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Global-RoPE cache for the active context (optional input of msa_sparse_attend).
+ * Pages: IRMaD "M. Materials & Methods", position item (global RoPE on the
+ * active context, positions offset by k).  The rotation angles of the local
+ * positions pos_offset + j (j < t_loc_max) depend only on positions, not on
+ * data, so a decode session can build them once:
+ *   cache  [t_loc_max, head_dim/2] (cos, sin) fp32 pairs, device, caller-owned,
+ *          msa_rope_cache_size(...) bytes; entry (j, i) is the rotation of pair
+ *          (i, i + head_dim/2) at position pos_offset + j, theta_i =
+ *          rope_base^(-2i/head_dim), angle reduced in fp64.
+ * msa_sparse_attend uses a cache built for its own (pos_offset, t_loc_max,
+ * head_dim, rope_base); passing rope_cache = NULL makes the call build the
+ * table in its workspace first.
+ * ------------------------------------------------------------------------- */
+size_t msa_rope_cache_size(const msa_dims* dims, int32_t t_loc_max);
+msa_status msa_rope_cache_build(const msa_dims* dims, int32_t t_loc_max, int32_t pos_offset, void* cache,
+                                size_t cache_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Tracing: per-kernel device time.

@@ -18,7 +18,7 @@ from typing import Optional
 
 __all__ = [
     "Dims", "MSAError", "lib", "chunk_offsets", "encode_memory", "route_topk", "sparse_attend",
-    "route_workspace_size", "attend_workspace_size", "encode_workspace_size", "check_device_errors",
+    "route_workspace_size", "attend_workspace_size", "rope_cache_build", "encode_workspace_size", "check_device_errors",
     "trace_enable", "trace_reset", "trace_read", "trace_kernel_names", "AGG_MAX", "AGG_MEAN",
 ]
 
@@ -67,7 +67,9 @@ def _load():
         "msa_route_workspace_size": (SZ, [DP, I32, I32, I32, I32, I32]),
         "msa_route_topk": (I32, [DP, P, P, I32, P, P, I32, I32, I32, I32, P, P, P, P, SZ, P]),
         "msa_attend_workspace_size": (SZ, [DP, I32, I32, I32, I32]),
-        "msa_sparse_attend": (I32, [DP, P, I32, P, P, P, I32, I32, P, I32, P, P, P, I32, I32, F, P, P, SZ, P]),
+        "msa_sparse_attend": (I32, [DP, P, I32, P, P, P, I32, I32, P, I32, P, P, P, I32, I32, P, F, P, P, SZ, P]),
+        "msa_rope_cache_size": (SZ, [DP, I32]),
+        "msa_rope_cache_build": (I32, [DP, I32, I32, P, SZ, P]),
         "msa_trace_enable": (I32, [I32]),
         "msa_trace_reset": (I32, []),
         "msa_trace_num_kernels": (I32, []),
@@ -213,9 +215,24 @@ def attend_workspace_size(dims, B: int, k: int, t_loc_max: int, pos_offset: int)
     return int(lib.msa_attend_workspace_size(ctypes.byref(Dims.of(dims)), B, k, t_loc_max, pos_offset))
 
 
+def rope_cache_build(dims, t_loc_max: int, pos_offset: int, device=None, out=None, stream=None):
+    """(cos, sin) table of the local positions pos_offset + j, j < t_loc_max (fp32 pairs)."""
+    import torch
+
+    nbytes = int(lib.msa_rope_cache_size(ctypes.byref(Dims.of(dims)), t_loc_max))
+    if out is None:
+        out = torch.empty(nbytes // 4, dtype=torch.float32, device=device)
+    _check(lib.msa_rope_cache_build(ctypes.byref(Dims.of(dims)), t_loc_max, pos_offset, _ptr(out),
+                                    out.numel() * out.element_size(), _stream(stream)))
+    return out
+
+
 def sparse_attend(dims, q, K_bar, V_bar, chunk_off, topk_idx, K_loc, V_loc, loc_len, pos_offset: int,
-                  softmax_scale: float = 0.0, out=None, ws=None, stream=None):
-    """One GQA decode step over [selected docs' K̄; local K].  Returns out [B, n_q, head_dim] bf16."""
+                  softmax_scale: float = 0.0, out=None, ws=None, stream=None, rope_cache=None):
+    """One GQA decode step over [selected docs' K̄; local K].  Returns out [B, n_q, head_dim] bf16.
+
+    ``rope_cache`` (from ``rope_cache_build`` with the same pos_offset and t_loc_max) skips
+    rebuilding the local-position rotation table."""
     import torch
 
     dd = Dims.of(dims)
@@ -229,8 +246,8 @@ def sparse_attend(dims, q, K_bar, V_bar, chunk_off, topk_idx, K_loc, V_loc, loc_
     ws = _workspace(nbytes, dev, ws)
     _check(lib.msa_sparse_attend(ctypes.byref(dd), _ptr(q), B, _ptr(K_bar), _ptr(V_bar), _ptr(chunk_off), n_docs,
                                  K_bar.shape[0], _ptr(topk_idx), k, _ptr(K_loc), _ptr(V_loc), _ptr(loc_len),
-                                 t_loc_max, pos_offset, float(softmax_scale), _ptr(out), _aligned_ptr(ws), nbytes,
-                                 _stream(stream)))
+                                 t_loc_max, pos_offset, _ptr(rope_cache), float(softmax_scale), _ptr(out),
+                                 _aligned_ptr(ws), nbytes, _stream(stream)))
     return out
 
 

@@ -39,7 +39,7 @@ struct AttendWs {
 namespace {
 
 constexpr int kTK = 64;          // keys per tile
-constexpr int kAttnStages = 2;
+constexpr int kAttnStages = 3;
 constexpr int kAttnThreads = 128;
 constexpr int kMaxK = 256;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -53,6 +53,8 @@ __global__ void __launch_bounds__(256) rope_table_kernel(float2* __restrict__ ta
                                                          int pos_offset, double log_base, int head_dim) {
   __shared__ float2 coarse[128];
   __shared__ float theta_f[128];
+  pdl_launch_dependents();
+  pdl_wait();
   const int jh = blockIdx.x;
   for (int i = threadIdx.x; i < half; i += blockDim.x) {
     const double theta = exp(-2.0 * (double)i / (double)head_dim * log_base);
@@ -110,6 +112,17 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnPara
   const int G = p.n_q / p.n_kv;
   const int k = p.k;
 
+  // zero the stage buffers once (rows past a range end are never copied) and set up barriers:
+  // nothing here touches global memory, so it overlaps the previous kernel's tail
+  for (int i = tid; i < kAttnStages * 2 * TILEB / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(stage_mem)[i] = make_uint4(0, 0, 0, 0);
+  if (tid == 0) {
+    for (int s = 0; s < kAttnStages; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+  }
+  pdl_launch_dependents();
+  pdl_wait();
+
   // ---- segment table of this query: selected docs in top-k order, then local ----
   for (int r = tid; r < k; r += blockDim.x) {
     int doc = p.topk_idx[(size_t)b * k + r];
@@ -123,13 +136,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnPara
     seg_c[r] = c0;
     seg_v[r + 1] = n;
   }
-  // zero the stage buffers once (rows past a range end are never copied)
-  for (int i = tid; i < kAttnStages * 2 * TILEB / 16; i += blockDim.x)
-    reinterpret_cast<uint4*>(stage_mem)[i] = make_uint4(0, 0, 0, 0);
-  if (tid == 0) {
-    for (int s = 0; s < kAttnStages; ++s) mbar_init(&bars[s], 1);
-    fence_mbar_init();
-  }
+  int L = p.loc_len[b];
+  L = max(0, min(L, p.t_loc_max));
   __syncthreads();
   if (warp == 0) {
     // inclusive scan of chunk counts -> virtual starts (lane owns a run of entries)
@@ -159,8 +167,6 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnPara
   __syncthreads();
 
   const int n_sel = seg_v[k];
-  int L = p.loc_len[b];
-  L = max(0, min(L, p.t_loc_max));
   const int n_keys = n_sel + L;
   int per_split = (n_keys + p.n_splits - 1) / p.n_splits;
   per_split = (per_split + 15) & ~15;
@@ -168,15 +174,54 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnPara
   const int v1 = min(n_keys, v0 + per_split);
   const int n_tiles = (v1 - v0 + kTK - 1) / kTK;
 
+  // ---- issue one tile's row copies (warp 0); every other warp just waits ----
+  const size_t kv_stride_c = (size_t)p.n_kv * D;  // elements between chunks / local tokens
+  auto issue = [&](int t, int st) {
+    if (warp != 0) return;
+    const int tv0 = v0 + t * kTK;
+    const int rows = min(kTK, v1 - tv0);
+    if (lane == 0) mbar_arrive_expect_tx(&bars[st], (uint32_t)(2 * rows * D * 2));
+    __syncwarp();
+    uint8_t* kdst = stage_mem + (size_t)st * 2 * TILEB;
+    uint8_t* vdst = kdst + TILEB;
+    for (int r = lane; r < rows; r += 32) {
+      const int v = tv0 + r;
+      const __nv_bfloat16 *ks, *vs;
+      if (v < n_sel) {
+        int lo = 0, hi = k - 1;  // segment with seg_v[lo] <= v < seg_v[lo + 1]
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (seg_v[mid] <= v) lo = mid; else hi = mid - 1;
+        }
+        const size_t ch = (size_t)(seg_c[lo] + (v - seg_v[lo]));
+        ks = p.K_bar + ch * kv_stride_c + (size_t)h * D;
+        vs = p.V_bar + ch * kv_stride_c + (size_t)h * D;
+      } else {
+        const size_t j = (size_t)(v - n_sel);
+        const size_t off = ((size_t)b * p.t_loc_max + j) * kv_stride_c + (size_t)h * D;
+        ks = p.K_loc + off;
+        vs = p.V_loc + off;
+      }
+      bulk_load(kdst + r * ROWB, ks, D * 2, &bars[st]);
+      bulk_load(vdst + r * ROWB, vs, D * 2, &bars[st]);
+    }
+  };
+  // start streaming before the query fragments are built
+  for (int t = 0; t < kAttnStages - 1 && t < n_tiles; ++t) issue(t, t % kAttnStages);
+
   // ---- query fragments: rotate to pos_offset + L - 1, scale, bf16 (A operand, rows = GQA heads) ----
   float2* qcs = reinterpret_cast<float2*>(seg_c + kMaxK);  // [D/2] cos/sin at the query position
   for (int i = tid; i < D / 2; i += blockDim.x) {
-    double a = (double)(p.pos_offset + L - 1) * exp(-2.0 * (double)i / (double)D * p.log_base);
-    const double two_pi = 6.283185307179586476925286766559;
-    a -= two_pi * rint(a / two_pi);
-    double sv, cv;
-    sincos(a, &sv, &cv);
-    qcs[i] = make_float2((float)cv, (float)sv);
+    if (L >= 1) {
+      qcs[i] = p.rope_tab[(size_t)(L - 1) * (D / 2) + i];  // the decode token is local token L - 1
+    } else {
+      double a = (double)(p.pos_offset - 1) * exp(-2.0 * (double)i / (double)D * p.log_base);
+      const double two_pi = 6.283185307179586476925286766559;
+      a -= two_pi * rint(a / two_pi);
+      double sv, cv;
+      sincos(a, &sv, &cv);
+      qcs[i] = make_float2((float)cv, (float)sv);
+    }
   }
   __syncthreads();
   const int g = lane >> 2, c = lane & 3;
@@ -213,46 +258,11 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnPara
     }
   }
 
-  // ---- issue one tile's row copies (warp 0); every other warp just waits ----
-  const size_t kv_stride_c = (size_t)p.n_kv * D;  // elements between chunks / local tokens
-  auto issue = [&](int t, int st) {
-    if (warp != 0) return;
-    const int tv0 = v0 + t * kTK;
-    const int rows = min(kTK, v1 - tv0);
-    if (lane == 0) mbar_arrive_expect_tx(&bars[st], (uint32_t)(2 * rows * D * 2));
-    __syncwarp();
-    uint8_t* kdst = stage_mem + (size_t)st * 2 * TILEB;
-    uint8_t* vdst = kdst + TILEB;
-    for (int r = lane; r < rows; r += 32) {
-      const int v = tv0 + r;
-      const __nv_bfloat16 *ks, *vs;
-      if (v < n_sel) {
-        int lo = 0, hi = k - 1;  // segment with seg_v[lo] <= v < seg_v[lo + 1]
-        while (lo < hi) {
-          const int mid = (lo + hi + 1) >> 1;
-          if (seg_v[mid] <= v) lo = mid; else hi = mid - 1;
-        }
-        const size_t ch = (size_t)(seg_c[lo] + (v - seg_v[lo]));
-        ks = p.K_bar + ch * kv_stride_c + (size_t)h * D;
-        vs = p.V_bar + ch * kv_stride_c + (size_t)h * D;
-      } else {
-        const size_t j = (size_t)(v - n_sel);
-        const size_t off = ((size_t)b * p.t_loc_max + j) * kv_stride_c + (size_t)h * D;
-        ks = p.K_loc + off;
-        vs = p.V_loc + off;
-      }
-      bulk_load(kdst + r * ROWB, ks, D * 2, &bars[st]);
-      bulk_load(vdst + r * ROWB, vs, D * 2, &bars[st]);
-    }
-  };
-
   float acc[NBLK][4];
 #pragma unroll
   for (int n = 0; n < NBLK; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
   float m_run[2] = {-INFINITY, -INFINITY};
   float l_run[2] = {0.f, 0.f};
-
-  for (int t = 0; t < kAttnStages - 1 && t < n_tiles; ++t) issue(t, t % kAttnStages);
 
   for (int t = 0; t < n_tiles; ++t) {
     const int st = t % kAttnStages;
@@ -413,6 +423,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnPara
 template <int D>
 __global__ void attn_combine_kernel(const float* __restrict__ part_ml, const float* __restrict__ part_o,
                                     int n_splits, __nv_bfloat16* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait();
   const size_t qh = (size_t)blockIdx.y * gridDim.x + blockIdx.x;  // b * n_q + head
   const float* ml = part_ml + qh * n_splits * 2;
   float M = -INFINITY;
@@ -456,19 +468,28 @@ size_t attend_workspace(const msa_dims& d, int B, int k, int t_loc_max, int pos_
   return cv.size();
 }
 
+msa_status rope_cache_build(const msa_dims& d, int t_loc_max, int pos_offset, float2* tab, cudaStream_t s) {
+  if (t_loc_max <= 0) return MSA_OK;
+  const int D = d.head_dim;
+  TraceScope ts(kKRopeTable, s);
+  MSA_CUDA_CHECK(launch_pdl(rope_table_kernel, dim3((t_loc_max + 63) / 64), dim3(256), 0, s, tab, t_loc_max, D / 2,
+                            pos_offset, std::log((double)d.rope_base), D));
+  return MSA_OK;
+}
+
 msa_status attend_launch(const msa_dims& d, const void* q, int B, const void* K_bar, const void* V_bar,
                          const int32_t* chunk_off, int n_docs, const int32_t* topk_idx, int k, const void* K_loc,
-                         const void* V_loc, const int32_t* loc_len, int t_loc_max, int pos_offset, float scale,
-                         void* out, void* ws, cudaStream_t s) {
+                         const void* V_loc, const int32_t* loc_len, int t_loc_max, int pos_offset,
+                         const void* rope_cache, float scale, void* out, void* ws, cudaStream_t s) {
   AttendWs w;
   attend_workspace(d, B, k, t_loc_max, pos_offset, ws, &w);
   const int D = d.head_dim;
   const double log_base = std::log((double)d.rope_base);
-  if (t_loc_max > 0) {
-    TraceScope ts(kKRopeTable, s);
-    const int blocks = (t_loc_max + 63) / 64;
-    rope_table_kernel<<<blocks, 256, 0, s>>>(w.rope_tab, t_loc_max, D / 2, pos_offset, log_base, D);
-    MSA_CUDA_CHECK(cudaGetLastError());
+  const float2* tab = static_cast<const float2*>(rope_cache);
+  if (!tab) {
+    msa_status st = rope_cache_build(d, t_loc_max, pos_offset, w.rope_tab, s);
+    if (st != MSA_OK) return st;
+    tab = w.rope_tab;
   }
   AttnParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -479,7 +500,7 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, const void* K_
   p.K_loc = static_cast<const __nv_bfloat16*>(K_loc);
   p.V_loc = static_cast<const __nv_bfloat16*>(V_loc);
   p.loc_len = loc_len;
-  p.rope_tab = w.rope_tab;
+  p.rope_tab = tab;
   p.part_ml = w.part_ml;
   p.part_o = w.part_o;
   p.n_q = d.n_q;
@@ -497,22 +518,23 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, const void* K_
     if (D == 128) {
       const size_t sm = attn_smem<128>();
       MSA_CUDA_CHECK(cudaFuncSetAttribute(attn_split_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-      attn_split_kernel<128><<<grid, kAttnThreads, sm, s>>>(p);
+      MSA_CUDA_CHECK(launch_pdl(attn_split_kernel<128>, grid, dim3(kAttnThreads), sm, s, p));
     } else {
       const size_t sm = attn_smem<64>();
       MSA_CUDA_CHECK(cudaFuncSetAttribute(attn_split_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-      attn_split_kernel<64><<<grid, kAttnThreads, sm, s>>>(p);
+      MSA_CUDA_CHECK(launch_pdl(attn_split_kernel<64>, grid, dim3(kAttnThreads), sm, s, p));
     }
-    MSA_CUDA_CHECK(cudaGetLastError());
   }
   {
     TraceScope ts(kKAttnCombine, s);
     dim3 grid(d.n_q, B);
+    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
     if (D == 128)
-      attn_combine_kernel<128><<<grid, 128, 0, s>>>(w.part_ml, w.part_o, w.n_splits, static_cast<__nv_bfloat16*>(out));
+      MSA_CUDA_CHECK(launch_pdl(attn_combine_kernel<128>, grid, dim3(128), 0, s, (const float*)w.part_ml,
+                                (const float*)w.part_o, w.n_splits, o));
     else
-      attn_combine_kernel<64><<<grid, 64, 0, s>>>(w.part_ml, w.part_o, w.n_splits, static_cast<__nv_bfloat16*>(out));
-    MSA_CUDA_CHECK(cudaGetLastError());
+      MSA_CUDA_CHECK(launch_pdl(attn_combine_kernel<64>, grid, dim3(64), 0, s, (const float*)w.part_ml,
+                                (const float*)w.part_o, w.n_splits, o));
   }
   return MSA_OK;
 }

@@ -122,7 +122,9 @@ size_t attend_workspace(const msa_dims& d, int B, int k, int t_loc_max, int pos_
 msa_status attend_launch(const msa_dims& d, const void* q, int B, const void* K_bar, const void* V_bar,
                          const int32_t* chunk_off, int n_docs, const int32_t* topk_idx, int k,
                          const void* K_loc, const void* V_loc, const int32_t* loc_len, int t_loc_max,
-                         int pos_offset, float scale, void* out, void* ws, cudaStream_t s);
+                         int pos_offset, const void* rope_cache, float scale, void* out, void* ws,
+                         cudaStream_t s);
+msa_status rope_cache_build(const msa_dims& d, int t_loc_max, int pos_offset, float2* tab, cudaStream_t s);
 
 size_t encode_workspace(const msa_dims& d, int64_t T, int n_docs, int n_chunks, void* ws,
                         struct EncodeWs* out);

@@ -291,7 +291,8 @@ size_t msa_attend_workspace_size(const msa_dims* dims, int32_t B, int32_t k, int
 msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, const void* K_bar, const void* V_bar,
                              const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks, const int32_t* topk_idx,
                              int32_t k, const void* K_loc, const void* V_loc, const int32_t* loc_len,
-                             int32_t t_loc_max, int32_t pos_offset, float softmax_scale, void* out, void* ws,
+                             int32_t t_loc_max, int32_t pos_offset, const void* rope_cache, float softmax_scale,
+                             void* out, void* ws,
                              size_t ws_bytes, void* stream) {
   msa_status st = check_dims(dims, true, false);
   if (st != MSA_OK) return st;
@@ -315,6 +316,7 @@ msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, con
     CHECK_PTR(V_loc);
   }
   CHECK_PTR(loc_len);
+  CHECK_OPT_PTR(rope_cache);
   CHECK_PTR(out);
   const size_t need = attend_workspace(*dims, B, k, t_loc_max, pos_offset, nullptr, nullptr);
   if (ws_bytes < need) return fail(MSA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
@@ -322,7 +324,27 @@ msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, con
     return fail(MSA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
   if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
   return attend_launch(*dims, q, B, K_bar, V_bar, chunk_off, n_docs, topk_idx, k, K_loc, V_loc, loc_len, t_loc_max,
-                       pos_offset, softmax_scale, out, ws, static_cast<cudaStream_t>(stream));
+                       pos_offset, rope_cache, softmax_scale, out, ws, static_cast<cudaStream_t>(stream));
+}
+
+size_t msa_rope_cache_size(const msa_dims* dims, int32_t t_loc_max) {
+  if (!dims || t_loc_max < 1 || (dims->head_dim != 64 && dims->head_dim != 128)) return 0;
+  return (size_t)t_loc_max * (dims->head_dim / 2) * sizeof(float2);
+}
+
+msa_status msa_rope_cache_build(const msa_dims* dims, int32_t t_loc_max, int32_t pos_offset, void* cache,
+                                size_t cache_bytes, void* stream) {
+  msa_status st = check_dims(dims, true, false);
+  if (st != MSA_OK) return st;
+  if (t_loc_max < 1) return fail(MSA_ERR_INVALID_ARG, "t_loc_max must be >= 1");
+  if (pos_offset < 0 || (int64_t)pos_offset + t_loc_max > (1 << 24))
+    return fail(MSA_ERR_INVALID_ARG, "positions must lie in [0, 2^24)");
+  CHECK_PTR(cache);
+  if (cache_bytes < msa_rope_cache_size(dims, t_loc_max))
+    return fail(MSA_ERR_WORKSPACE, "rope cache too small: %zu < %zu bytes", cache_bytes,
+                msa_rope_cache_size(dims, t_loc_max));
+  if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
+  return rope_cache_build(*dims, t_loc_max, pos_offset, static_cast<float2*>(cache), static_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------ encode ------------------------------

@@ -58,6 +58,8 @@ __global__ void __launch_bounds__(256) qr_proj_kernel(const __nv_bfloat16* __res
                                                       const __nv_bfloat16* __restrict__ W, int B, int hidden,
                                                       int NR, int rows_per_split, float* __restrict__ part) {
   __shared__ float red[8][kQpQB][kQpCols];
+  pdl_launch_dependents();
+  pdl_wait();
   const int col0 = blockIdx.x * kQpCols;
   const int split = blockIdx.y;
   const int k_begin = split * rows_per_split;
@@ -124,6 +126,8 @@ __global__ void __launch_bounds__(256) q_prep_kernel(const float* __restrict__ p
                                                      int n_r, int d_r, int nb_total, uint4* __restrict__ qfrag,
                                                      uint32_t* __restrict__ doc_key, int n_docs) {
   extern __shared__ float qs[];  // [n_r * d_r] then inv norms [n_r]
+  pdl_launch_dependents();
+  pdl_wait();
   const int b = blockIdx.x;      // padded query index (< 8 * nb_total)
   const int NR = n_r * d_r;
   float* invn = qs + NR;
@@ -212,13 +216,15 @@ __global__ void __launch_bounds__(288, 1) scan_kernel(const __grid_constant__ CU
       mbar_init(&empty[s], n_r);
     }
     fence_mbar_init();
+    prefetch_tensormap(&kr_map);
   }
+  pdl_launch_dependents();
+  pdl_wait();
   __syncthreads();
 
   if (warp == n_r) {
     // ---------------- producer: one thread streams tiles with TMA ----------------
     if (lane == 0) {
-      prefetch_tensormap(&kr_map);
       for (int it = 0; it < n_it; ++it) {
         const int st = it % kStages;
         if (it >= kStages) mbar_wait(&empty[st], ((it / kStages) - 1) & 1);
@@ -455,6 +461,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_slice_kernel(
   uint64_t* tmp = out + 256;          // [256]
   uint64_t* state = tmp + 256;        // [4]
   uint32_t* hist = reinterpret_cast<uint32_t*>(state + 4);
+  pdl_launch_dependents();
+  pdl_wait();
   const int slice = blockIdx.x, b = blockIdx.y;
   const int d0 = slice * kSliceDocs;
   const int n = min(kSliceDocs, n_docs - d0);
@@ -498,6 +506,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_merge_kernel(const uint64_t
   uint64_t* tmp = out + 256;
   uint64_t* state = tmp + 256;
   uint32_t* hist = reinterpret_cast<uint32_t*>(state + 4);
+  pdl_launch_dependents();
+  pdl_wait();
   const int b = blockIdx.x;
   for (int i = threadIdx.x; i < n; i += blockDim.x) keys[i] = cand[(size_t)b * n + i];
   __syncthreads();
@@ -513,8 +523,7 @@ cudaError_t launch_scan_t(const CUtensorMap& map, const ScanParams& p, int grid,
   auto kern = scan_kernel<NB, DR, MEAN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, (p.n_r + 1) * 32, smem, s>>>(map, p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3((p.n_r + 1) * 32), smem, s, map, p);
 }
 
 template <int DR, bool MEAN>
@@ -568,19 +577,17 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
   if (W_QR) {
     TraceScope ts(kKQrProj, s);
     const int rows = (d.hidden + w.ksplit - 1) / w.ksplit;
-    qr_proj_kernel<<<dim3(NR / kQpCols, w.ksplit), 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(Hq), static_cast<const __nv_bfloat16*>(W_QR), B, d.hidden, NR, rows,
-        w.qr_part);
-    MSA_CUDA_CHECK(cudaGetLastError());
+    MSA_CUDA_CHECK(launch_pdl(qr_proj_kernel, dim3(NR / kQpCols, w.ksplit), dim3(256), 0, s,
+                              static_cast<const __nv_bfloat16*>(Hq), static_cast<const __nv_bfloat16*>(W_QR), B,
+                              d.hidden, NR, rows, w.qr_part));
   }
   // K2: normalise + fragments + clear document keys
   {
     TraceScope ts(kKQPrep, s);
     const size_t sm = (size_t)(NR + d.n_r) * sizeof(float);
-    q_prep_kernel<<<w.nb_total * 8, 256, sm, s>>>(
-        w.qr_part, w.ksplit, W_QR ? nullptr : static_cast<const __nv_bfloat16*>(Hq), B, d.n_r, d.d_r,
-        w.nb_total, w.qfrag, w.doc_key, n_docs);
-    MSA_CUDA_CHECK(cudaGetLastError());
+    MSA_CUDA_CHECK(launch_pdl(q_prep_kernel, dim3(w.nb_total * 8), dim3(256), sm, s, (const float*)w.qr_part,
+                              w.ksplit, W_QR ? nullptr : static_cast<const __nv_bfloat16*>(Hq), B, d.n_r, d.d_r,
+                              w.nb_total, w.qfrag, w.doc_key, n_docs));
   }
   // K3: scan, 32 queries per pass
   {
@@ -623,22 +630,17 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
   {
     TraceScope ts(kKTopkSlice, s);
     const size_t sm = topk_slice_smem();
-    static bool attr_set = false;
-    if (!attr_set) {
-      MSA_CUDA_CHECK(cudaFuncSetAttribute(topk_slice_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-      attr_set = true;
-    }
-    topk_slice_kernel<<<dim3(w.n_slices, B), kTopkThreads, sm, s>>>(
-        w.doc_key, w.chunk_s, chunk_off, n_docs, n_chunks, k, w.n_slices, doc_scores, w.cand, topk_idx,
-        topk_score);
-    MSA_CUDA_CHECK(cudaGetLastError());
+    MSA_CUDA_CHECK(cudaFuncSetAttribute(topk_slice_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+    MSA_CUDA_CHECK(launch_pdl(topk_slice_kernel, dim3(w.n_slices, B), dim3(kTopkThreads), sm, s,
+                              (const uint32_t*)w.doc_key, (const float*)w.chunk_s, chunk_off, n_docs, n_chunks, k,
+                              w.n_slices, doc_scores, w.cand, topk_idx, topk_score));
   }
   if (w.n_slices > 1) {
     TraceScope ts(kKTopkMerge, s);
     const size_t sm = topk_merge_smem(w.n_slices * k);
     MSA_CUDA_CHECK(cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-    topk_merge_kernel<<<B, kTopkThreads, sm, s>>>(w.cand, w.n_slices, k, topk_idx, topk_score);
-    MSA_CUDA_CHECK(cudaGetLastError());
+    MSA_CUDA_CHECK(launch_pdl(topk_merge_kernel, dim3(B), dim3(kTopkThreads), sm, s, (const uint64_t*)w.cand,
+                              w.n_slices, k, topk_idx, topk_score));
   }
   return MSA_OK;
 }

@@ -1,0 +1,198 @@
+"""Run one stage of the MSA path on one synthetic workload, for timing and profiling.
+
+    python -m long_context_memory_b200.profile_cases --case route16m --launches 3
+
+Inputs are drawn on the device by torch's seeded generator (timing only: no
+parity check here; the tests do that).  Each launch is timed with CUDA events
+on the launching stream and printed; under a profiler, the printed times are
+not benchmark values.
+
+Cases
+  route1m    1M-token memory, B = 1   (K̄^R 33 MB)
+  route16m   16M-token memory, B = 32 (K̄^R 520 MB)
+  route100m  100M-token memory, B = 1 (K̄^R 3.2 GB); --batch to change B
+  attend1m   sparse attention, 1M-token memory, B = 1, 4K local tokens
+  attend16m  sparse attention, 16M-token memory, B = 32, 8K local tokens
+  encode     offline encoding of --tokens tokens (default 1M), hidden 2560
+"""
+from __future__ import annotations
+
+import argparse
+import math
+
+import numpy as np
+
+from . import workloads as W
+
+
+def chunk_layout_host(T: int, median: int, seed: int):
+    import long_context_memory_b200 as msa
+
+    rng = np.random.default_rng(seed)
+    lens = W.doc_lengths_lognormal(rng, T, median)
+    doc_off = W.offsets_from_lengths(lens)
+    co, C = msa.chunk_offsets(doc_off)
+    return doc_off, co, C
+
+
+def randn_bf16(shape, g, device):
+    import torch
+
+    out = torch.empty(shape, dtype=torch.bfloat16, device=device)
+    flat = out.view(-1)
+    step = 1 << 26
+    for i in range(0, flat.numel(), step):
+        e = min(flat.numel(), i + step)
+        flat[i:e] = torch.randn(e - i, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+    return out
+
+
+class RouteCase:
+    def __init__(self, T, B, median, seed, device, k=16, dims=W.QWEN3_4B_DIMS, layers=1):
+        import torch
+
+        import long_context_memory_b200 as msa
+
+        self.msa, self.d, self.B, self.k, self.T = msa, dims, B, k, T
+        doc_off, co, C = chunk_layout_host(T, median, seed)
+        self.C, self.n_docs = C, len(co) - 1
+        g = torch.Generator(device=device)
+        g.manual_seed(seed)
+        self.chunk_off = torch.from_numpy(co).to(device)
+        self.KR = [randn_bf16((C, dims.n_r, dims.d_r), g, device) for _ in range(layers)]
+        self.Hq = randn_bf16((B, dims.hidden), g, device)
+        self.W_QR = (torch.randn((dims.hidden, dims.n_r * dims.d_r), generator=g, device=device) /
+                     math.sqrt(dims.hidden)).to(torch.bfloat16)
+        self.idx = torch.empty((B, k), dtype=torch.int32, device=device)
+        self.sc = torch.empty((B, k), dtype=torch.float32, device=device)
+        self.ws = torch.empty(msa.route_workspace_size(dims, B, self.n_docs, C, k) + 256, dtype=torch.uint8,
+                              device=device)
+
+    def set_batch(self, B, seed=0):
+        """Same memory, a new batch of B queries."""
+        import torch
+
+        dev = self.KR[0].device
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed)
+        self.B = B
+        self.Hq = randn_bf16((B, self.d.hidden), g, dev)
+        self.idx = torch.empty((B, self.k), dtype=torch.int32, device=dev)
+        self.sc = torch.empty((B, self.k), dtype=torch.float32, device=dev)
+        self.ws = torch.empty(self.msa.route_workspace_size(self.d, B, self.n_docs, self.C, self.k) + 256,
+                              dtype=torch.uint8, device=dev)
+
+    def run(self, layer=0):
+        self.msa.route_topk(self.d, self.Hq, self.W_QR, self.KR[layer], self.chunk_off, self.k,
+                            out=(self.idx, self.sc, None), ws=self.ws)
+
+    @property
+    def scan_bytes(self):
+        return self.C * self.d.n_r * self.d.d_r * 2
+
+
+class AttendCase:
+    def __init__(self, T, B, median, t_loc, seed, device, k=16, dims=W.QWEN3_4B_DIMS):
+        import torch
+
+        import long_context_memory_b200 as msa
+
+        self.msa, self.d, self.B, self.k = msa, dims, B, k
+        doc_off, co, C = chunk_layout_host(T, median, seed)
+        n_docs = len(co) - 1
+        g = torch.Generator(device=device)
+        g.manual_seed(seed + 1)
+        self.chunk_off = torch.from_numpy(co).to(device)
+        self.K_bar = randn_bf16((C, dims.n_kv, dims.head_dim), g, device)
+        self.V_bar = randn_bf16((C, dims.n_kv, dims.head_dim), g, device)
+        self.q = randn_bf16((B, dims.n_q, dims.head_dim), g, device)
+        self.K_loc = randn_bf16((B, t_loc, dims.n_kv, dims.head_dim), g, device)
+        self.V_loc = randn_bf16((B, t_loc, dims.n_kv, dims.head_dim), g, device)
+        self.loc_len = torch.full((B,), t_loc, dtype=torch.int32, device=device)
+        rng = np.random.default_rng(seed)
+        sel = np.stack([rng.permutation(n_docs)[:k] for _ in range(B)]).astype(np.int32)
+        self.topk = torch.from_numpy(sel).to(device)
+        self.pos = k
+        self.rope = msa.rope_cache_build(dims, t_loc, self.pos, device=device)
+        self.out = torch.empty((B, dims.n_q, dims.head_dim), dtype=torch.bfloat16, device=device)
+        self.ws = torch.empty(msa.attend_workspace_size(dims, B, k, t_loc, self.pos) + 256, dtype=torch.uint8,
+                              device=device)
+        n_sel = sum(int(co[i + 1] - co[i]) for row in sel for i in row)
+        self.kv_bytes = (n_sel + B * t_loc) * dims.n_kv * dims.head_dim * 2 * 2
+
+    def run(self):
+        self.msa.sparse_attend(self.d, self.q, self.K_bar, self.V_bar, self.chunk_off, self.topk, self.K_loc,
+                               self.V_loc, self.loc_len, self.pos, out=self.out, ws=self.ws, rope_cache=self.rope)
+
+
+class EncodeCase:
+    def __init__(self, T, seed, device, dims=W.QWEN3_4B_DIMS):
+        import torch
+
+        import long_context_memory_b200 as msa
+
+        self.msa, self.d, self.T = msa, dims, T
+        c = W.encode_config(T=T, seed=seed, with_hidden=False)
+        co, C = msa.chunk_offsets(c["doc_off"])
+        self.C = C
+        self.H = W.encode_hidden(T, dims.hidden, seed, device)
+        t = lambda a: W.to_torch(np.ascontiguousarray(a)).to(device)
+        self.doc_off = torch.from_numpy(c["doc_off"]).to(device)
+        self.chunk_off = torch.from_numpy(co).to(device)
+        self.W = (t(c["W_K"]), t(c["W_V"]), t(c["W_KR"]))
+        self.out = (torch.empty((C, dims.n_kv, dims.head_dim), dtype=torch.bfloat16, device=device),
+                    torch.empty((C, dims.n_kv, dims.head_dim), dtype=torch.bfloat16, device=device),
+                    torch.empty((C, dims.n_r, dims.d_r), dtype=torch.bfloat16, device=device))
+        self.ws = torch.empty(msa.encode_workspace_size(dims, T, len(co) - 1, C) + 256, dtype=torch.uint8,
+                              device=device)
+        NK = dims.n_kv * dims.head_dim
+        NVR = NK + dims.n_r * dims.d_r
+        self.flops_k = 2.0 * T * dims.hidden * NK
+        self.flops_pooled = 2.0 * C * (2 * dims.hidden) * NVR
+
+    def run(self):
+        self.msa.encode_memory(self.d, self.H, self.doc_off, self.chunk_off, self.C, *self.W, out=self.out,
+                               ws=self.ws)
+
+
+def main():
+    import torch
+
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--case", required=True,
+                    choices=["route1m", "route16m", "route100m", "attend1m", "attend16m", "encode"])
+    ap.add_argument("--launches", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=2)
+    ap.add_argument("--batch", type=int, default=None)
+    ap.add_argument("--tokens", type=int, default=1_000_000)
+    a = ap.parse_args()
+    dev = torch.device("cuda:0")
+    seed = W.BASE_SEED + 7
+    if a.case == "route1m":
+        case = RouteCase(1_000_000, a.batch or 1, 2048, seed, dev)
+    elif a.case == "route16m":
+        case = RouteCase(16_000_000, a.batch or 32, 2048, seed, dev)
+    elif a.case == "route100m":
+        case = RouteCase(100_000_000, a.batch or 1, 4096, seed, dev)
+    elif a.case == "attend1m":
+        case = AttendCase(1_000_000, a.batch or 1, 2048, 4096, seed, dev)
+    elif a.case == "attend16m":
+        case = AttendCase(16_000_000, a.batch or 32, 2048, 8192, seed, dev)
+    else:
+        case = EncodeCase(a.tokens, seed, dev)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        for _ in range(a.warmup):
+            case.run()
+        torch.cuda.synchronize()
+        for i in range(a.launches):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            case.run()
+            e1.record(s)
+            torch.cuda.synchronize()
+            print(f"{a.case} launch {i}: {e0.elapsed_time(e1) * 1e3:.1f} us", flush=True)
+
+
+if __name__ == "__main__":
+    main()

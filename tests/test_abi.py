@@ -108,7 +108,7 @@ def _attend(msa, dims, B=1, k=2, n_docs=4, n_chunks=8, t_loc=16, pos=2, scale=0.
     if ws_bytes is None:
         ws_bytes = need
     return msa.lib.msa_sparse_attend(ctypes.byref(dd), q, B, FAKE, FAKE, FAKE, n_docs, n_chunks, FAKE, k, FAKE, FAKE,
-                                     FAKE, t_loc, pos, scale, FAKE, 0x100000, ws_bytes, None)
+                                     FAKE, t_loc, pos, None, scale, FAKE, 0x100000, ws_bytes, None)
 
 
 def test_attend_validation(msa):
