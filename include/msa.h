@@ -145,6 +145,28 @@ msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR
                           float* topk_score, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * msa_route_topk_static - msa_route_topk without a caller workspace.
+ * The paper has no counterpart: this is a convenience of this library.
+ * For callers that cannot allocate device memory where they route: a host
+ * program that embeds the library as a plugin without a CUDA allocator, code
+ * running while a stream is captured into a CUDA graph (cudaMalloc is not
+ * allowed there), or a loop that must not pay cudaMalloc's implicit device
+ * synchronisation.  Same arguments and results as msa_route_topk, minus
+ * ws/ws_bytes.  The scratch is a library-owned device array of 8 MiB
+ * (8388608 bytes) that every GPU loading the library holds until the process
+ * exits; a problem whose msa_route_workspace_size exceeds it is rejected with
+ * MSA_ERR_WORKSPACE before any launch.  The first call on a device (with that
+ * device current) looks up the array's address once; make it before any stream
+ * capture.  All calls on a device share the array, so calls whose work
+ * overlaps on the GPU race: order them on one stream.  No cudaMalloc, cudaFree
+ * or allocating library routine is called.
+ * ------------------------------------------------------------------------- */
+msa_status msa_route_topk_static(const msa_dims* dims, const void* Hq, const void* W_QR, int32_t B,
+                                 const void* KR_bar, const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks,
+                                 int32_t k, msa_doc_agg agg, float* doc_scores, int32_t* topk_idx,
+                                 float* topk_score, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Stage 3 - sparse generation attention (one decode step).
  * Pages: IRMaD "M. Materials & Methods", routing item (K_ctx = [{K̄_i}_{i in I};
  * K_q], V_ctx likewise, Output = Attention(Q_q, K_ctx, V_ctx)) and position item

@@ -1,0 +1,78 @@
+"""msa_route_topk_static (routing on the library's own static scratch) against
+msa_route_topk (routing on a caller workspace), through the C ABI.
+
+The static entry point is for callers that cannot allocate device memory where
+they route (an embedding host without a CUDA allocator, code inside a CUDA-graph
+capture, loops that must not synchronise on cudaMalloc).  Two calls in a row must
+match the workspace path: the second call runs on the scratch the first one left
+behind.  This file is collected last so that a failure here comes after every
+other test has run.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+
+import oracle as O
+from long_context_memory_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def _static_fn(msa):
+    fn = msa.lib.msa_route_topk_static
+    P, I32 = ctypes.c_void_p, ctypes.c_int32
+    fn.restype = I32
+    fn.argtypes = [ctypes.POINTER(msa.Dims), P, P, I32, P, P, I32, I32, I32, I32, P, P, P, P]
+    return fn
+
+
+def test_static_scratch_matches_workspace_path(cuda_device):
+    import torch
+
+    import long_context_memory_b200 as msa
+
+    rng = np.random.default_rng(77)
+    dims = W.Dims(hidden=512, n_q=8, n_kv=2, head_dim=64, n_r=8, d_r=128)
+    lens = rng.integers(1, 900, size=600)
+    co, C = msa.chunk_offsets(W.offsets_from_lengths(lens))
+    dev = cuda_device
+    KR = W.to_torch(W.normal_bf16(rng, (C, 8, 128))).to(dev)
+    Hq = W.to_torch(W.normal_bf16(rng, (5, 512))).to(dev)
+    Wqr = W.to_torch(W.normal_bf16(rng, (512, 1024), 512 ** -0.5)).to(dev)
+    chunk_off = torch.from_numpy(co).to(dev)
+    B, k, n_docs = 5, 16, len(co) - 1
+
+    ref_idx, ref_sc, ref_ds = msa.route_topk(dims, Hq, Wqr, KR, chunk_off, k, want_doc_scores=True)
+    fn = _static_fn(msa)
+    dd = msa.Dims.of(dims)
+    stream = torch.cuda.current_stream().cuda_stream
+    for call in range(2):
+        idx = torch.full((B, k), -1, dtype=torch.int32, device=dev)
+        sc = torch.zeros((B, k), dtype=torch.float32, device=dev)
+        ds = torch.zeros((B, n_docs), dtype=torch.float32, device=dev)
+        r = fn(ctypes.byref(dd), Hq.data_ptr(), Wqr.data_ptr(), B, KR.data_ptr(), chunk_off.data_ptr(), n_docs, C, k,
+               0, ds.data_ptr(), idx.data_ptr(), sc.data_ptr(), stream)
+        assert r == 0, msa.lib.msa_last_error().decode()
+        torch.cuda.synchronize()
+        assert msa.check_device_errors() == 0
+        assert torch.equal(idx, ref_idx), f"call {call}: top-k ids differ"
+        assert torch.max(torch.abs(sc - ref_sc)).item() <= 1e-3
+        assert torch.max(torch.abs(ds - ref_ds)).item() <= 1e-3
+    # and both agree with the oracle's document scores
+    s = O.doc_scores(O.chunk_scores(O.router_query(W.f32_to_bf16_bits(Hq.float().cpu().numpy()),
+                                                   W.f32_to_bf16_bits(Wqr.float().cpu().numpy()), 8, 128),
+                                    W.f32_to_bf16_bits(KR.float().cpu().numpy())), co)
+    assert np.max(np.abs(ds.cpu().numpy() - s)) < 1e-3
+
+
+def test_static_scratch_rejects_oversized_problem(cuda_device):
+    import long_context_memory_b200 as msa
+
+    fn = _static_fn(msa)
+    dd = msa.Dims.of(W.QWEN3_4B_DIMS)
+    # 32 queries over 400K documents need far more than the 8 MiB static area
+    r = fn(ctypes.byref(dd), 0x10000, 0x10000, 32, 0x10000, 0x10000, 400_000, 1_600_000, 16, 0, None, 0x10000,
+           0x10000, None)
+    assert r == 3
+    assert "static area" in msa.lib.msa_last_error().decode()
