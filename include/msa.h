@@ -53,7 +53,7 @@ typedef enum {
 } msa_status;
 
 /* Model dimensions of one routed layer.  hidden = width of H; n_q / n_kv =
- * query / key-value heads (GQA, n_q a multiple of n_kv, n_q / n_kv <= 16);
+ * query / key-value heads (GQA, n_q a multiple of n_kv, n_kv <= 8, n_q / n_kv <= 16);
  * head_dim in {64, 128}; n_r router heads of dim d_r in {64, 128}, n_r <= 8;
  * chunk = tokens per pooled chunk (P, 64 on the pages); rope_base = RoPE base. */
 typedef struct {
@@ -143,6 +143,21 @@ msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR
                           const void* KR_bar, const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks,
                           int32_t k, msa_doc_agg agg, float* doc_scores, int32_t* topk_idx,
                           float* topk_score, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Merge of top-k candidates (memory-parallel routing).
+ * Pages: IRMaD "M. Materials & Methods", Memory Parallel item; EverMind article
+ * 2.3: the router keys are sharded over GPUs, the query is broadcast, every GPU
+ * scores its shard and a global reduction picks the top-k documents.  After
+ * each rank's msa_route_topk on its shard and an exchange of the B x k_local
+ * (score, global document id) pairs, this call selects the global top-k.
+ *   cand_score [B, n_cand] fp32, cand_idx [B, n_cand] int32 global ids (device).
+ *   topk_idx [B, k], topk_score [B, k] out: descending score, ties to the lower id
+ *   (the same order as msa_route_topk on the unsharded memory).
+ * Limits: 1 <= k <= min(n_cand, 256), n_cand <= 24576.
+ * ------------------------------------------------------------------------- */
+msa_status msa_topk_merge(const float* cand_score, const int32_t* cand_idx, int32_t B, int32_t n_cand, int32_t k,
+                          int32_t* topk_idx, float* topk_score, void* stream);
 
 /* ---------------------------------------------------------------------------
  * msa_route_topk_static - msa_route_topk without a caller workspace.

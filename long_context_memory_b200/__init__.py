@@ -18,7 +18,7 @@ from typing import Optional
 
 __all__ = [
     "Dims", "MSAError", "lib", "chunk_offsets", "encode_memory", "route_topk", "sparse_attend",
-    "route_workspace_size", "attend_workspace_size", "rope_cache_build", "encode_workspace_size", "check_device_errors",
+    "route_workspace_size", "attend_workspace_size", "rope_cache_build", "topk_merge", "encode_workspace_size", "check_device_errors",
     "trace_enable", "trace_reset", "trace_read", "trace_kernel_names", "AGG_MAX", "AGG_MEAN",
 ]
 
@@ -70,6 +70,7 @@ def _load():
         "msa_sparse_attend": (I32, [DP, P, I32, P, P, P, I32, I32, P, I32, P, P, P, I32, I32, P, F, P, P, SZ, P]),
         "msa_rope_cache_size": (SZ, [DP, I32]),
         "msa_rope_cache_build": (I32, [DP, I32, I32, P, SZ, P]),
+        "msa_topk_merge": (I32, [P, P, I32, I32, I32, P, P, P]),
         "msa_trace_enable": (I32, [I32]),
         "msa_trace_reset": (I32, []),
         "msa_trace_num_kernels": (I32, []),
@@ -205,6 +206,18 @@ def route_topk(dims, Hq, W_QR, KR_bar, chunk_off, k: int, agg: int = AGG_MAX, wa
     _check(lib.msa_route_topk(ctypes.byref(dd), _ptr(Hq), _ptr(W_QR), B, _ptr(KR_bar), _ptr(chunk_off), n_docs,
                               n_chunks, k, agg, _ptr(out[2]), _ptr(out[0]), _ptr(out[1]), _aligned_ptr(ws), nbytes,
                               _stream(stream)))
+    return out
+
+
+def topk_merge(cand_score, cand_idx, k: int, out=None, stream=None):
+    """Global top-k of [B, n_cand] (score, global id) candidates (memory-parallel routing)."""
+    import torch
+
+    B, n = cand_score.shape
+    dev = cand_score.device
+    if out is None:
+        out = (torch.empty((B, k), dtype=torch.int32, device=dev), torch.empty((B, k), dtype=torch.float32, device=dev))
+    _check(lib.msa_topk_merge(_ptr(cand_score), _ptr(cand_idx), B, n, k, _ptr(out[0]), _ptr(out[1]), _stream(stream)))
     return out
 
 

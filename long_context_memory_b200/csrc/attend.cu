@@ -38,10 +38,10 @@ struct AttendWs {
 
 namespace {
 
-constexpr int kTK = 64;          // keys per tile
-constexpr int kAttnStages = 3;
-constexpr int kAttnThreads = 128;
+constexpr int kTK = 16;          // keys per tile (one mma K-step of P V)
+constexpr int kMaxStages = 4;
 constexpr int kMaxK = 256;
+constexpr int kMaxSplits = 1024;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // cos/sin of (pos_offset + j) * theta_i, theta_i = base^(-2i/D), for local
@@ -90,40 +90,63 @@ struct AttnParams {
   const float2* rope_tab;
   float* part_ml;
   float* part_o;
-  int n_q, n_kv, k, n_docs, t_loc_max, pos_offset, n_splits;
+  int n_q, n_kv, k, n_docs, t_loc_max, pos_offset, n_splits, n_stages;
   float scale_log2;  // softmax scale * log2(e)
   double log_base;
 };
 
-template <int D>
-__global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnParams p) {
-  constexpr int KS = D / 16;
-  constexpr int ROWB = D * 2 + 16;          // padded smem row (bytes): conflict-free ldmatrix
-  constexpr int TILEB = kTK * ROWB;         // one tensor (K or V) of one stage
-  constexpr int NBLK = D / 8;               // output column blocks
-  extern __shared__ __align__(128) uint8_t sm[];
-  uint8_t* stage_mem = sm;                                         // [stages][K tile | V tile]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kAttnStages * 2 * TILEB);
-  int* seg_v = reinterpret_cast<int*>(bars + kAttnStages);         // [k + 1] virtual starts
-  int* seg_c = seg_v + kMaxK + 2;                                  // [k] chunk starts (8-byte aligned end)
+// Shared memory of one CTA (dynamic size, n_stages stages):
+//   stage s: K rows [kTK][krow] | V rows [kTK][krow] | RoPE rows [kTK][D/2] (cos, sin)
+//   krow = n_kv * D * 2 + 16 bytes: one key's rows of every KV head, padded so
+//   that consecutive rows start one 16-byte unit apart (conflict-free ldmatrix)
+//   then barriers, the segment table, the query's cos/sin and the raw query.
+struct AttnSmem {
+  int krow, kbytes, tbytes, stage_bytes, n_stages;
+  __host__ __device__ AttnSmem(int n_kv, int D, int stages) {
+    krow = n_kv * D * 2 + 16;
+    kbytes = kTK * krow;
+    tbytes = kTK * (D / 2) * 8;
+    stage_bytes = 2 * kbytes + tbytes;
+    n_stages = stages;
+  }
+  __host__ __device__ size_t fixed_bytes(int n_q, int D) const {
+    return kMaxStages * 8 + (2 * kMaxK + 2) * 4 + (size_t)(D / 2) * 8 + (size_t)n_q * D * 2;
+  }
+  __host__ __device__ size_t total(int n_q, int D) const { return (size_t)n_stages * stage_bytes + fixed_bytes(n_q, D); }
+};
 
-  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+template <int D>
+__global__ void __launch_bounds__(256, 1) attn_split_kernel(const AttnParams p) {
+  constexpr int KS = D / 16;
+  constexpr int NBLK = D / 8;
+  const int n_kv = p.n_kv, G = p.n_q / n_kv;
+  const AttnSmem L_(n_kv, D, p.n_stages);
+  extern __shared__ __align__(128) uint8_t sm[];
+  // offsets: every region below starts on a 16-byte boundary (stage rows, query rows and
+  // the RoPE rows are bulk-copy or 16-byte vector destinations)
+  uint8_t* stage_mem = sm;
+  uint16_t* qsm = reinterpret_cast<uint16_t*>(sm + (size_t)L_.n_stages * L_.stage_bytes);  // [n_q][D] raw query
+  uint64_t* bars = reinterpret_cast<uint64_t*>(qsm + (size_t)p.n_q * D);
+  int* seg_v = reinterpret_cast<int*>(bars + kMaxStages);  // [k + 1] virtual starts
+  int* seg_c = seg_v + kMaxK + 2;                          // [k] chunk starts
+  float2* qcs = reinterpret_cast<float2*>(seg_c + kMaxK);  // [D/2] cos/sin at the query position
+
+  const int split = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int G = p.n_q / p.n_kv;
+  const int h = warp;  // the KV head this warp serves
   const int k = p.k;
 
-  // zero the stage buffers once (rows past a range end are never copied) and set up barriers:
-  // nothing here touches global memory, so it overlaps the previous kernel's tail
-  for (int i = tid; i < kAttnStages * 2 * TILEB / 16; i += blockDim.x)
+  // ---- no global memory yet: overlaps the previous kernel's tail ----
+  for (int i = tid; i < L_.n_stages * L_.stage_bytes / 16; i += blockDim.x)
     reinterpret_cast<uint4*>(stage_mem)[i] = make_uint4(0, 0, 0, 0);
   if (tid == 0) {
-    for (int s = 0; s < kAttnStages; ++s) mbar_init(&bars[s], 1);
+    for (int s = 0; s < L_.n_stages; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
   }
   pdl_launch_dependents();
   pdl_wait();
 
-  // ---- segment table of this query: selected docs in top-k order, then local ----
+  // ---- segment table (selected docs in top-k order, then local) and the raw query ----
   for (int r = tid; r < k; r += blockDim.x) {
     int doc = p.topk_idx[(size_t)b * k + r];
     int c0 = 0, n = 0;
@@ -135,6 +158,10 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnPara
     }
     seg_c[r] = c0;
     seg_v[r + 1] = n;
+  }
+  {
+    const uint4* qg = reinterpret_cast<const uint4*>(p.q + (size_t)b * p.n_q * D);
+    for (int i = tid; i < p.n_q * D / 8; i += blockDim.x) reinterpret_cast<uint4*>(qsm)[i] = __ldg(qg + i);
   }
   int L = p.loc_len[b];
   L = max(0, min(L, p.t_loc_max));
@@ -169,23 +196,27 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnPara
   const int n_sel = seg_v[k];
   const int n_keys = n_sel + L;
   int per_split = (n_keys + p.n_splits - 1) / p.n_splits;
-  per_split = (per_split + 15) & ~15;
+  per_split = (per_split + kTK - 1) / kTK * kTK;
   const int v0 = min(n_keys, split * per_split);
   const int v1 = min(n_keys, v0 + per_split);
   const int n_tiles = (v1 - v0 + kTK - 1) / kTK;
+  const int row_bytes = n_kv * D * 2;  // one key, every KV head
+  const bool table = p.rope_tab != nullptr;
 
-  // ---- issue one tile's row copies (warp 0); every other warp just waits ----
-  const size_t kv_stride_c = (size_t)p.n_kv * D;  // elements between chunks / local tokens
+  // ---- one tile = kTK keys: a 2-row bulk copy pair per key plus one copy of the RoPE rows ----
   auto issue = [&](int t, int st) {
     if (warp != 0) return;
     const int tv0 = v0 + t * kTK;
     const int rows = min(kTK, v1 - tv0);
-    if (lane == 0) mbar_arrive_expect_tx(&bars[st], (uint32_t)(2 * rows * D * 2));
+    const int n_chunk_rows = max(0, min(rows, n_sel - tv0));
+    const int n_loc_rows = rows - n_chunk_rows;
+    const uint32_t tb = (table && n_loc_rows > 0) ? (uint32_t)(n_loc_rows * (D / 2) * 8) : 0u;
+    if (lane == 0) mbar_arrive_expect_tx(&bars[st], (uint32_t)(2 * rows * row_bytes) + tb);
     __syncwarp();
-    uint8_t* kdst = stage_mem + (size_t)st * 2 * TILEB;
-    uint8_t* vdst = kdst + TILEB;
-    for (int r = lane; r < rows; r += 32) {
-      const int v = tv0 + r;
+    uint8_t* kdst = stage_mem + (size_t)st * L_.stage_bytes;
+    uint8_t* vdst = kdst + L_.kbytes;
+    if (lane < rows) {
+      const int v = tv0 + lane;
       const __nv_bfloat16 *ks, *vs;
       if (v < n_sel) {
         int lo = 0, hi = k - 1;  // segment with seg_v[lo] <= v < seg_v[lo + 1]
@@ -194,40 +225,37 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnPara
           if (seg_v[mid] <= v) lo = mid; else hi = mid - 1;
         }
         const size_t ch = (size_t)(seg_c[lo] + (v - seg_v[lo]));
-        ks = p.K_bar + ch * kv_stride_c + (size_t)h * D;
-        vs = p.V_bar + ch * kv_stride_c + (size_t)h * D;
+        ks = p.K_bar + ch * n_kv * D;
+        vs = p.V_bar + ch * n_kv * D;
       } else {
-        const size_t j = (size_t)(v - n_sel);
-        const size_t off = ((size_t)b * p.t_loc_max + j) * kv_stride_c + (size_t)h * D;
+        const size_t off = ((size_t)b * p.t_loc_max + (size_t)(v - n_sel)) * n_kv * D;
         ks = p.K_loc + off;
         vs = p.V_loc + off;
       }
-      bulk_load(kdst + r * ROWB, ks, D * 2, &bars[st]);
-      bulk_load(vdst + r * ROWB, vs, D * 2, &bars[st]);
+      bulk_load(kdst + lane * L_.krow, ks, row_bytes, &bars[st]);
+      bulk_load(vdst + lane * L_.krow, vs, row_bytes, &bars[st]);
+    }
+    if (tb && lane == 31) {
+      const int j0 = tv0 + n_chunk_rows - n_sel;
+      bulk_load(vdst + L_.kbytes + n_chunk_rows * (D / 2) * 8, p.rope_tab + (size_t)j0 * (D / 2), tb, &bars[st]);
     }
   };
-  // start streaming before the query fragments are built
-  for (int t = 0; t < kAttnStages - 1 && t < n_tiles; ++t) issue(t, t % kAttnStages);
+  for (int t = 0; t < L_.n_stages - 1 && t < n_tiles; ++t) issue(t, t % L_.n_stages);
 
-  // ---- query fragments: rotate to pos_offset + L - 1, scale, bf16 (A operand, rows = GQA heads) ----
-  float2* qcs = reinterpret_cast<float2*>(seg_c + kMaxK);  // [D/2] cos/sin at the query position
+  // ---- query fragments of this warp's GQA group: rotate to pos_offset + L - 1, scale, bf16 ----
   for (int i = tid; i < D / 2; i += blockDim.x) {
-    if (L >= 1) {
-      qcs[i] = p.rope_tab[(size_t)(L - 1) * (D / 2) + i];  // the decode token is local token L - 1
-    } else {
-      double a = (double)(p.pos_offset - 1) * exp(-2.0 * (double)i / (double)D * p.log_base);
-      const double two_pi = 6.283185307179586476925286766559;
-      a -= two_pi * rint(a / two_pi);
-      double sv, cv;
-      sincos(a, &sv, &cv);
-      qcs[i] = make_float2((float)cv, (float)sv);
-    }
+    double a = (double)(p.pos_offset + L - 1) * exp(-2.0 * (double)i / (double)D * p.log_base);
+    const double two_pi = 6.283185307179586476925286766559;
+    a -= two_pi * rint(a / two_pi);
+    double sv, cv;
+    sincos(a, &sv, &cv);
+    qcs[i] = make_float2((float)cv, (float)sv);
   }
   __syncthreads();
   const int g = lane >> 2, c = lane & 3;
   uint32_t qa[KS][4];
   {
-    const uint16_t* qb = reinterpret_cast<const uint16_t*>(p.q) + ((size_t)b * p.n_q + (size_t)h * G) * D;
+    const uint16_t* qb = qsm + (size_t)h * G * D;
 #pragma unroll
     for (int s = 0; s < KS; ++s) {
 #pragma unroll
@@ -244,8 +272,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnPara
               const bool first = dd < D / 2;
               const int i = first ? dd : dd - D / 2;
               const int partner = first ? dd + D / 2 : dd - D / 2;
-              const float x = bf16_bits_to_float(qb[(size_t)row * D + dd]);
-              const float y = bf16_bits_to_float(qb[(size_t)row * D + partner]);
+              const float x = bf16_bits_to_float(qb[row * D + dd]);
+              const float y = bf16_bits_to_float(qb[row * D + partner]);
               const float2 cs = qcs[i];
               // first half: x cos - y sin; second half: x cos + y sin (y = first-half partner)
               const float rot = first ? (x * cs.x - y * cs.y) : (x * cs.x + y * cs.y);
@@ -263,39 +291,42 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnPara
   for (int n = 0; n < NBLK; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
   float m_run[2] = {-INFINITY, -INFINITY};
   float l_run[2] = {0.f, 0.f};
+  const int hoff = h * D * 2;  // this head's bytes within a key row
 
   for (int t = 0; t < n_tiles; ++t) {
-    const int st = t % kAttnStages;
-    if (t + kAttnStages - 1 < n_tiles) issue(t + kAttnStages - 1, (t + kAttnStages - 1) % kAttnStages);
-    mbar_wait(&bars[st], (t / kAttnStages) & 1);
+    const int st = t % L_.n_stages;
+    if (t + L_.n_stages - 1 < n_tiles) issue(t + L_.n_stages - 1, (t + L_.n_stages - 1) % L_.n_stages);
+    mbar_wait(&bars[st], (t / L_.n_stages) & 1);
 
     const int tv0 = v0 + t * kTK;
-    const uint32_t kbase = smem_u32(stage_mem + (size_t)st * 2 * TILEB);
-    const uint32_t vbase = kbase + TILEB;
-    const int wkey0 = 16 * warp;  // this warp's 16 keys within the tile
+    const uint8_t* kst = stage_mem + (size_t)st * L_.stage_bytes;
+    const uint32_t kbase = smem_u32(kst) + hoff;
+    const uint32_t vbase = kbase + L_.kbytes;
+    const float2* tab = reinterpret_cast<const float2*>(kst + 2 * L_.kbytes);
 
-    if (tv0 + wkey0 < v1) {
-      // ---- K fragments (B operand, keys = n) ----
-      uint32_t kb[KS][2][2];
-      {
-        const int key = wkey0 + (lane & 7) + 8 * (lane >> 4);
-        const int dsel = 8 * ((lane >> 3) & 1);
+    // ---- K fragments (B operand, keys = n) ----
+    uint32_t kb[KS][2][2];
+    {
+      const int key = (lane & 7) + 8 * (lane >> 4);
+      const int dsel = 8 * ((lane >> 3) & 1);
 #pragma unroll
-        for (int s = 0; s < KS; ++s)
-          ldmatrix_x4(kb[s][0][0], kb[s][0][1], kb[s][1][0], kb[s][1][1], kbase + key * ROWB + (16 * s + dsel) * 2);
-      }
-      // ---- rotate local keys in registers (pairs i, i + D/2 sit in ksteps s, s + KS/2) ----
+      for (int s = 0; s < KS; ++s)
+        ldmatrix_x4(kb[s][0][0], kb[s][0][1], kb[s][1][0], kb[s][1][1], kbase + key * L_.krow + (16 * s + dsel) * 2);
+    }
+    // ---- rotate local keys in registers (pairs i, i + D/2 sit in ksteps s, s + KS/2) ----
+    if (table) {
 #pragma unroll
       for (int nb = 0; nb < 2; ++nb) {
-        const int v = tv0 + wkey0 + 8 * nb + g;
+        const int r = 8 * nb + g;
+        const int v = tv0 + r;
         if (v >= n_sel && v < v1) {
-          const float2* tab = p.rope_tab + (size_t)(v - n_sel) * (D / 2);
+          const float2* trow = tab + r * (D / 2);
 #pragma unroll
           for (int s = 0; s < KS / 2; ++s) {
 #pragma unroll
             for (int hk = 0; hk < 2; ++hk) {
               const int i = 16 * s + 8 * hk + 2 * c;
-              const float4 cs = *reinterpret_cast<const float4*>(tab + i);  // (cos_i, sin_i, cos_i+1, sin_i+1)
+              const float4 cs = *reinterpret_cast<const float4*>(trow + i);  // (cos_i, sin_i, cos_i+1, sin_i+1)
               const float2 x = unpack_bf16x2(kb[s][nb][hk]);
               const float2 y = unpack_bf16x2(kb[s + KS / 2][nb][hk]);
               const float x0 = x.x * cs.x - y.x * cs.y, y0 = y.x * cs.x + x.x * cs.y;
@@ -306,152 +337,158 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnPara
           }
         }
       }
-      // ---- S = q K^T (rows = heads, cols = 16 keys) ----
-      float sc[2][4];
+    }
+    // ---- S = q K^T (rows = heads, cols = 16 keys) ----
+    float sc[2][4];
 #pragma unroll
-      for (int nb = 0; nb < 2; ++nb) {
-        sc[nb][0] = sc[nb][1] = sc[nb][2] = sc[nb][3] = 0.f;
+    for (int nb = 0; nb < 2; ++nb) {
+      sc[nb][0] = sc[nb][1] = sc[nb][2] = sc[nb][3] = 0.f;
 #pragma unroll
-        for (int s = 0; s < KS; ++s)
-          mma_bf16_16816(sc[nb], qa[s][0], qa[s][1], qa[s][2], qa[s][3], kb[s][nb][0], kb[s][nb][1]);
+      for (int s = 0; s < KS; ++s)
+        mma_bf16_16816(sc[nb], qa[s][0], qa[s][1], qa[s][2], qa[s][3], kb[s][nb][0], kb[s][nb][1]);
+    }
+#pragma unroll
+    for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int v = tv0 + 8 * nb + 2 * c + e;
+        if (v >= v1) {
+          sc[nb][e] = -INFINITY;
+          sc[nb][2 + e] = -INFINITY;
+        }
       }
-      // mask keys past the range end
+    // ---- online softmax (rows g and g + 8) ----
+    float alpha[2];
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      float mx = fmaxf(fmaxf(sc[0][2 * rr], sc[0][2 * rr + 1]), fmaxf(sc[1][2 * rr], sc[1][2 * rr + 1]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float m_new = fmaxf(m_run[rr], mx);
+      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+      alpha[rr] = exp2f(m_run[rr] - m_use);
+      m_run[rr] = m_new;
+      float ls = 0.f;
 #pragma unroll
       for (int nb = 0; nb < 2; ++nb)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int v = tv0 + wkey0 + 8 * nb + 2 * c + e;
-          if (v >= v1) {
-            sc[nb][e] = -INFINITY;
-            sc[nb][2 + e] = -INFINITY;
-          }
+          const float pv = exp2f(sc[nb][2 * rr + e] - m_use);
+          sc[nb][2 * rr + e] = pv;
+          ls += pv;
         }
-      // ---- online softmax (rows g and g + 8) ----
-      float alpha[2];
+      l_run[rr] = l_run[rr] * alpha[rr] + ls;
+    }
 #pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        float mx = fmaxf(fmaxf(sc[0][2 * rr], sc[0][2 * rr + 1]), fmaxf(sc[1][2 * rr], sc[1][2 * rr + 1]));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const float m_new = fmaxf(m_run[rr], mx);
-        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-        alpha[rr] = exp2f(m_run[rr] - m_use);
-        m_run[rr] = m_new;
-        float ls = 0.f;
+    for (int n = 0; n < NBLK; ++n) {
+      acc[n][0] *= alpha[0];
+      acc[n][1] *= alpha[0];
+      acc[n][2] *= alpha[1];
+      acc[n][3] *= alpha[1];
+    }
+    // ---- O += P V ----
+    const uint32_t pa0 = pack_bf16x2(sc[0][0], sc[0][1]);
+    const uint32_t pa1 = pack_bf16x2(sc[0][2], sc[0][3]);
+    const uint32_t pa2 = pack_bf16x2(sc[1][0], sc[1][1]);
+    const uint32_t pa3 = pack_bf16x2(sc[1][2], sc[1][3]);
+    {
+      const int key = (lane & 7) + 8 * ((lane >> 3) & 1);
+      const int dsel = 8 * (lane >> 4);
 #pragma unroll
-        for (int nb = 0; nb < 2; ++nb)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float pv = exp2f(sc[nb][2 * rr + e] - m_use);
-            sc[nb][2 * rr + e] = pv;
-            ls += pv;
-          }
-        l_run[rr] = l_run[rr] * alpha[rr] + ls;
-      }
-#pragma unroll
-      for (int n = 0; n < NBLK; ++n) {
-        acc[n][0] *= alpha[0];
-        acc[n][1] *= alpha[0];
-        acc[n][2] *= alpha[1];
-        acc[n][3] *= alpha[1];
-      }
-      // ---- O += P V ----
-      const uint32_t pa0 = pack_bf16x2(sc[0][0], sc[0][1]);
-      const uint32_t pa1 = pack_bf16x2(sc[0][2], sc[0][3]);
-      const uint32_t pa2 = pack_bf16x2(sc[1][0], sc[1][1]);
-      const uint32_t pa3 = pack_bf16x2(sc[1][2], sc[1][3]);
-      {
-        const int key = wkey0 + (lane & 7) + 8 * ((lane >> 3) & 1);
-        const int dsel = 8 * (lane >> 4);
-#pragma unroll
-        for (int n = 0; n < NBLK; n += 2) {
-          uint32_t b0, b1, b2, b3;
-          ldmatrix_x4_trans(b0, b1, b2, b3, vbase + key * ROWB + (8 * n + dsel) * 2);
-          mma_bf16_16816(acc[n], pa0, pa1, pa2, pa3, b0, b1);
-          mma_bf16_16816(acc[n + 1], pa0, pa1, pa2, pa3, b2, b3);
-        }
+      for (int n = 0; n < NBLK; n += 2) {
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4_trans(b0, b1, b2, b3, vbase + key * L_.krow + (8 * n + dsel) * 2);
+        mma_bf16_16816(acc[n], pa0, pa1, pa2, pa3, b0, b1);
+        mma_bf16_16816(acc[n + 1], pa0, pa1, pa2, pa3, b2, b3);
       }
     }
     __syncthreads();  // every warp is done with stage st before it is refilled
   }
 
-  // ---- merge the 4 warps' partial softmax states and write this split's partial ----
+  // ---- this warp's split partial: unnormalised output, running max and sum per q head ----
 #pragma unroll
   for (int rr = 0; rr < 2; ++rr) {
     l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 1);
     l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 2);
   }
-  float* wm = reinterpret_cast<float*>(stage_mem);   // [4][16]
-  float* wl = wm + 4 * 16;                           // [4][16]
-  float* wo = wl + 4 * 16;                           // [4][16][D]
-  if (c == 0) {
-    wm[warp * 16 + g] = m_run[0];
-    wm[warp * 16 + g + 8] = m_run[1];
-    wl[warp * 16 + g] = l_run[0];
-    wl[warp * 16 + g + 8] = l_run[1];
-  }
 #pragma unroll
-  for (int n = 0; n < NBLK; ++n) {
-    wo[(warp * 16 + g) * D + 8 * n + 2 * c] = acc[n][0];
-    wo[(warp * 16 + g) * D + 8 * n + 2 * c + 1] = acc[n][1];
-    wo[(warp * 16 + g + 8) * D + 8 * n + 2 * c] = acc[n][2];
-    wo[(warp * 16 + g + 8) * D + 8 * n + 2 * c + 1] = acc[n][3];
-  }
-  __syncthreads();
-  for (int idx = tid; idx < G * D; idx += blockDim.x) {
-    const int row = idx / D, dim = idx % D;
-    float M = -INFINITY;
+  for (int rr = 0; rr < 2; ++rr) {
+    const int row = g + 8 * rr;
+    if (row < G) {
+      const size_t qh = (size_t)b * p.n_q + (size_t)h * G + row;
+      float* po = p.part_o + (qh * p.n_splits + split) * D;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, wm[w * 16 + row]);
-    const float Mu = (M == -INFINITY) ? 0.f : M;
-    float o = 0.f, l = 0.f;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const float sw = exp2f(wm[w * 16 + row] - Mu);
-      o += sw * wo[(w * 16 + row) * D + dim];
-      l += sw * wl[w * 16 + row];
-    }
-    const size_t qh = (size_t)b * p.n_q + (size_t)h * G + row;
-    p.part_o[(qh * p.n_splits + split) * D + dim] = o;
-    if (dim == 0) {
-      p.part_ml[(qh * p.n_splits + split) * 2 + 0] = M;
-      p.part_ml[(qh * p.n_splits + split) * 2 + 1] = l;
+      for (int n = 0; n < NBLK; ++n)
+        *reinterpret_cast<float2*>(po + 8 * n + 2 * c) = make_float2(acc[n][2 * rr], acc[n][2 * rr + 1]);
+      if (c == 0) {
+        p.part_ml[(qh * p.n_splits + split) * 2 + 0] = m_run[rr];
+        p.part_ml[(qh * p.n_splits + split) * 2 + 1] = l_run[rr];
+      }
     }
   }
 }
 
+// log-sum-exp merge of the split partials of one (query, q head); splits are read in parallel
 template <int D>
-__global__ void attn_combine_kernel(const float* __restrict__ part_ml, const float* __restrict__ part_o,
-                                    int n_splits, __nv_bfloat16* __restrict__ out) {
+__global__ void __launch_bounds__(128) attn_combine_kernel(const float* __restrict__ part_ml,
+                                                           const float* __restrict__ part_o, int n_splits,
+                                                           __nv_bfloat16* __restrict__ out) {
+  __shared__ float w_s[kMaxSplits];
+  __shared__ float red[2][4];
   pdl_launch_dependents();
   pdl_wait();
   const size_t qh = (size_t)blockIdx.y * gridDim.x + blockIdx.x;  // b * n_q + head
   const float* ml = part_ml + qh * n_splits * 2;
-  float M = -INFINITY;
-  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, ml[2 * s]);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float m = -INFINITY;
+  for (int s = tid; s < n_splits; s += blockDim.x) m = fmaxf(m, ml[2 * s]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) red[0][warp] = m;
+  __syncthreads();
+  float M = fmaxf(fmaxf(red[0][0], red[0][1]), fmaxf(red[0][2], red[0][3]));
   const float Mu = (M == -INFINITY) ? 0.f : M;
-  for (int dim = threadIdx.x; dim < D; dim += blockDim.x) {
-    float o = 0.f, l = 0.f;
-    for (int s = 0; s < n_splits; ++s) {
-      const float w = exp2f(ml[2 * s] - Mu);
-      o += w * part_o[(qh * n_splits + s) * D + dim];
-      l += w * ml[2 * s + 1];
+  float l = 0.f;
+  for (int s = tid; s < n_splits; s += blockDim.x) {
+    const float w = exp2f(ml[2 * s] - Mu);
+    w_s[s] = w;
+    l += w * ml[2 * s + 1];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+  if (lane == 0) red[1][warp] = l;
+  __syncthreads();
+  const float Ls = (red[1][0] + red[1][1]) + (red[1][2] + red[1][3]);
+  const float* po = part_o + qh * n_splits * D;
+  for (int dim = tid; dim < D; dim += blockDim.x) {
+    float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+    int s = 0;
+    for (; s + 4 <= n_splits; s += 4) {
+      o0 += w_s[s] * po[(size_t)s * D + dim];
+      o1 += w_s[s + 1] * po[(size_t)(s + 1) * D + dim];
+      o2 += w_s[s + 2] * po[(size_t)(s + 2) * D + dim];
+      o3 += w_s[s + 3] * po[(size_t)(s + 3) * D + dim];
     }
-    out[qh * D + dim] = __float2bfloat16_rn(l > 0.f ? o / l : 0.f);
+    for (; s < n_splits; ++s) o0 += w_s[s] * po[(size_t)s * D + dim];
+    const float o = (o0 + o1) + (o2 + o3);
+    out[qh * D + dim] = __float2bfloat16_rn(Ls > 0.f ? o / Ls : 0.f);
   }
 }
 
-template <int D>
-size_t attn_smem() {
-  return (size_t)kAttnStages * 2 * kTK * (D * 2 + 16) + kAttnStages * sizeof(uint64_t) +
-         (2 * kMaxK + 2) * sizeof(int) + (D / 2) * sizeof(float2);
+int stages_that_fit(int n_kv, int n_q, int D) {
+  const int budget = 200 * 1024;
+  for (int st = kMaxStages; st >= 2; --st) {
+    AttnSmem L(n_kv, D, st);
+    if (L.total(n_q, D) <= (size_t)budget) return st;
+  }
+  return 2;
 }
 
-int choose_splits(int B, int n_kv, int t_loc_max, int k) {
-  const int target = 2 * sm_count();
-  int s = (target + B * n_kv - 1) / (B * n_kv);
-  const int max_useful = std::max(1, (t_loc_max + 64 * k) / 64);
-  return std::max(1, std::min({s, max_useful, 128}));
+int choose_splits(int B, int t_loc_max, int k) {
+  const int target = 4 * sm_count();
+  int s = (target + B - 1) / B;
+  const int max_useful = std::max(1, (t_loc_max + 16 * k) / 32);
+  return std::max(1, std::min({s, max_useful, kMaxSplits}));
 }
 
 }  // namespace
@@ -460,7 +497,7 @@ size_t attend_workspace(const msa_dims& d, int B, int k, int t_loc_max, int pos_
   (void)pos_offset;
   Carver cv(ws);
   AttendWs w{};
-  w.n_splits = choose_splits(B, d.n_kv, t_loc_max, k);
+  w.n_splits = choose_splits(B, t_loc_max, k);
   w.rope_tab = cv.take<float2>((size_t)std::max(1, t_loc_max) * (d.head_dim / 2));
   w.part_ml = cv.take<float>((size_t)B * d.n_q * w.n_splits * 2);
   w.part_o = cv.take<float>((size_t)B * d.n_q * w.n_splits * d.head_dim);
@@ -512,17 +549,17 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, const void* K_
   p.n_splits = w.n_splits;
   p.scale_log2 = (scale > 0.f ? scale : 1.0f / std::sqrt((float)D)) * kLog2e;
   p.log_base = log_base;
+  p.n_stages = stages_that_fit(d.n_kv, d.n_q, D);
   {
     TraceScope ts(kKAttnSplit, s);
-    dim3 grid(w.n_splits, d.n_kv, B);
+    dim3 grid(w.n_splits, B);
+    const size_t sm = AttnSmem(d.n_kv, D, p.n_stages).total(d.n_q, D);
     if (D == 128) {
-      const size_t sm = attn_smem<128>();
       MSA_CUDA_CHECK(cudaFuncSetAttribute(attn_split_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-      MSA_CUDA_CHECK(launch_pdl(attn_split_kernel<128>, grid, dim3(kAttnThreads), sm, s, p));
+      MSA_CUDA_CHECK(launch_pdl(attn_split_kernel<128>, grid, dim3(32 * d.n_kv), sm, s, p));
     } else {
-      const size_t sm = attn_smem<64>();
       MSA_CUDA_CHECK(cudaFuncSetAttribute(attn_split_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-      MSA_CUDA_CHECK(launch_pdl(attn_split_kernel<64>, grid, dim3(kAttnThreads), sm, s, p));
+      MSA_CUDA_CHECK(launch_pdl(attn_split_kernel<64>, grid, dim3(32 * d.n_kv), sm, s, p));
     }
   }
   {
@@ -533,7 +570,7 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, const void* K_
       MSA_CUDA_CHECK(launch_pdl(attn_combine_kernel<128>, grid, dim3(128), 0, s, (const float*)w.part_ml,
                                 (const float*)w.part_o, w.n_splits, o));
     else
-      MSA_CUDA_CHECK(launch_pdl(attn_combine_kernel<64>, grid, dim3(64), 0, s, (const float*)w.part_ml,
+      MSA_CUDA_CHECK(launch_pdl(attn_combine_kernel<64>, grid, dim3(128), 0, s, (const float*)w.part_ml,
                                 (const float*)w.part_o, w.n_splits, o));
   }
   return MSA_OK;

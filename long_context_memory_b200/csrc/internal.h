@@ -117,6 +117,9 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
                         float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws,
                         cudaStream_t s);
 
+msa_status topk_merge_launch(const float* cand_score, const int32_t* cand_idx, int B, int n_cand, int k,
+                             int32_t* topk_idx, float* topk_score, cudaStream_t s);
+
 size_t attend_workspace(const msa_dims& d, int B, int k, int t_loc_max, int pos_offset, void* ws,
                         struct AttendWs* out);
 msa_status attend_launch(const msa_dims& d, const void* q, int B, const void* K_bar, const void* V_bar,

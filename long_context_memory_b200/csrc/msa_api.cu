@@ -184,6 +184,7 @@ static msa_status check_dims(const msa_dims* d, bool need_kv, bool need_router) 
     if (d->n_kv < 1 || d->n_q < 1 || d->n_q % d->n_kv != 0)
       return fail(MSA_ERR_INVALID_ARG, "n_q (%d) must be a positive multiple of n_kv (%d)", d->n_q, d->n_kv);
     if (d->n_q / d->n_kv > 16) return fail(MSA_ERR_UNSUPPORTED, "n_q / n_kv must be <= 16");
+    if (d->n_kv > 8) return fail(MSA_ERR_UNSUPPORTED, "n_kv must be <= 8 (got %d)", d->n_kv);
     if (!(d->rope_base > 1.0f) || !std::isfinite(d->rope_base))
       return fail(MSA_ERR_INVALID_ARG, "rope_base must be finite and > 1");
   }
@@ -280,6 +281,20 @@ msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR
   if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
   return route_launch(*dims, Hq, W_QR, B, KR_bar, chunk_off, n_docs, n_chunks, k, agg, doc_scores, topk_idx,
                       topk_score, ws, static_cast<cudaStream_t>(stream));
+}
+
+msa_status msa_topk_merge(const float* cand_score, const int32_t* cand_idx, int32_t B, int32_t n_cand, int32_t k,
+                          int32_t* topk_idx, float* topk_score, void* stream) {
+  if (B < 1) return fail(MSA_ERR_INVALID_ARG, "B must be >= 1 (got %d)", B);
+  if (n_cand < 1 || n_cand > 24576) return fail(MSA_ERR_INVALID_ARG, "n_cand must be in [1, 24576] (got %d)", n_cand);
+  if (k < 1 || k > n_cand || k > 256)
+    return fail(MSA_ERR_INVALID_ARG, "k must be in [1, min(n_cand, 256)] (got %d)", k);
+  CHECK_PTR(cand_score);
+  CHECK_PTR(cand_idx);
+  CHECK_PTR(topk_idx);
+  CHECK_PTR(topk_score);
+  if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
+  return topk_merge_launch(cand_score, cand_idx, B, n_cand, k, topk_idx, topk_score, static_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------ attention ------------------------------

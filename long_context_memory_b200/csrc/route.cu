@@ -32,19 +32,15 @@ namespace msa {
 
 struct RouteWs {
   float* qr_part;     // [ksplit][B][NR] fp32 partial sums of Q^R (W_QR given)
-  uint4* qfrag;       // [n_r][KS][NBtot][32] bf16 hi/lo query fragments
+  __nv_bfloat16* q_hl; // [passes][n_r][2][NQ][d_r] normalised query, bf16 hi and lo terms
   uint32_t* doc_key;  // [B][n_docs] ordered-uint32 doc max (MAX)
   float* chunk_s;     // [B][n_chunks] chunk scores (MEAN)
   uint64_t* cand;     // [B][n_slices][k] slice winners
-  int ksplit, nb_total, n_slices;
+  int ksplit, nq, passes, n_slices;
 };
 
 namespace {
 
-constexpr int kTileC = 16;         // chunks per pipeline stage (one mma m-tile)
-constexpr int kStages = 4;         // TMA ring depth
-constexpr int kBoxBytes = kTileC * 128;  // one 64-dim x 16-row box, 128B-swizzled
-constexpr int kPartStride = 20;    // padded row stride of the per-head partial tile
 constexpr int kSliceDocs = 4096;   // documents per top-k slice CTA
 constexpr int kTopkThreads = 1024;
 constexpr int kQpCols = 64;
@@ -118,17 +114,18 @@ __global__ void __launch_bounds__(256) qr_proj_kernel(const __nv_bfloat16* __res
 }
 
 // --------------------------------------------------------------------------
-// normalise Q^R per head and lay it out as mma.m16n8k16 B fragments
-// (hi and lo bf16 terms); clear the document keys of this query
+// normalise Q^R per head and write it as two bf16 terms (hi + lo) in the
+// layout the scan's TMA reads: q_hl[pass][head][hi|lo][NQ query rows][d_r];
+// rows of padding queries are zero.  Also clears this query's document keys.
 // --------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) q_prep_kernel(const float* __restrict__ part, int ksplit,
                                                      const __nv_bfloat16* __restrict__ qr_direct, int B,
-                                                     int n_r, int d_r, int nb_total, uint4* __restrict__ qfrag,
+                                                     int n_r, int d_r, int nq, __nv_bfloat16* __restrict__ q_hl,
                                                      uint32_t* __restrict__ doc_key, int n_docs) {
   extern __shared__ float qs[];  // [n_r * d_r] then inv norms [n_r]
   pdl_launch_dependents();
   pdl_wait();
-  const int b = blockIdx.x;      // padded query index (< 8 * nb_total)
+  const int b = blockIdx.x;      // padded query index (< passes * nq)
   const int NR = n_r * d_r;
   float* invn = qs + NR;
   const bool real = b < B;
@@ -138,7 +135,14 @@ __global__ void __launch_bounds__(256) q_prep_kernel(const float* __restrict__ p
       if (qr_direct) {
         v = bf16_bits_to_float(reinterpret_cast<const uint16_t*>(qr_direct)[(size_t)b * NR + n]);
       } else {
-        for (int s = 0; s < ksplit; ++s) v += part[((size_t)s * B + b) * NR + n];
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        int s = 0;
+        for (; s + 4 <= ksplit; s += 4) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) acc[u] += part[((size_t)(s + u) * B + b) * NR + n];
+        }
+        for (; s < ksplit; ++s) acc[0] += part[((size_t)s * B + b) * NR + n];
+        v = (acc[0] + acc[1]) + (acc[2] + acc[3]);
       }
     }
     qs[n] = v;
@@ -153,23 +157,15 @@ __global__ void __launch_bounds__(256) q_prep_kernel(const float* __restrict__ p
     if (lane == 0) invn[h] = 1.0f / fmaxf(sqrtf(ss), kEps);
   }
   __syncthreads();
-  const int KS = d_r / 16;
-  const int nb = b >> 3, g = b & 7;
-  for (int idx = threadIdx.x; idx < n_r * KS * 4; idx += blockDim.x) {
-    const int h = idx / (KS * 4), s = (idx >> 2) % KS, c = idx & 3;
-    const float* qh = qs + h * d_r + 16 * s + 2 * c;
-    const float sc = invn[h];
-    const float x0 = qh[0] * sc, x1 = qh[1] * sc, x2 = qh[8] * sc, x3 = qh[9] * sc;
-    const float h0 = __bfloat162float(__float2bfloat16_rn(x0));
-    const float h1 = __bfloat162float(__float2bfloat16_rn(x1));
-    const float h2 = __bfloat162float(__float2bfloat16_rn(x2));
-    const float h3 = __bfloat162float(__float2bfloat16_rn(x3));
-    uint4 f;
-    f.x = pack_bf16x2(h0, h1);
-    f.y = pack_bf16x2(h2, h3);
-    f.z = pack_bf16x2(x0 - h0, x1 - h1);
-    f.w = pack_bf16x2(x2 - h2, x3 - h3);
-    qfrag[((size_t)(h * KS + s) * nb_total + nb) * 32 + 4 * g + c] = f;
+  const int pass = b / nq, row = b % nq;
+  for (int idx = threadIdx.x; idx < NR; idx += blockDim.x) {
+    const int h = idx / d_r, dd = idx % d_r;
+    const float x = qs[idx] * invn[h];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+    const size_t base = (((size_t)pass * n_r + h) * 2) * nq;
+    q_hl[(base + row) * d_r + dd] = hi;
+    q_hl[(base + nq + row) * d_r + dd] = lo;
   }
   if (real && doc_key) {
     for (int i = threadIdx.x; i < n_docs; i += blockDim.x) doc_key[(size_t)b * n_docs + i] = 0u;
@@ -177,194 +173,242 @@ __global__ void __launch_bounds__(256) q_prep_kernel(const float* __restrict__ p
 }
 
 // --------------------------------------------------------------------------
-// the K̄^R scan
+// the K̄^R scan on tcgen05 tensor cores
+//
+// Tile = 128 consecutive chunks; the tile is streamed one router head at a
+// time.  A pipeline stage holds that head's 128 x d_r slice of K̄^R (the MMA's
+// A operand, 128B-swizzled TMA boxes) and the head's normalised query terms
+// (B operand: hi and lo bf16 rows, NQ queries).  One thread issues
+//   D[128 chunks, h*NQ .. h*NQ+NQ) += K̄^R_h (128 x d_r) . (q_hi + q_lo)^T
+// into a double-buffered TMEM accumulator; four warps read the same stage from
+// shared memory for the per-chunk squared norms, and after the tile's last
+// head they read D, apply 1/||K̄^R_h||, average the heads and fold each
+// document's maximum into doc_key with one atomicMax per document segment.
 // --------------------------------------------------------------------------
+constexpr int kScanM = 128;         // chunks per tile (MMA M)
+constexpr int kScanStages = 4;
+constexpr int kScanThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 norms + epilogue
+
 struct ScanParams {
-  const uint4* qfrag;
   const int32_t* chunk_off;
   uint32_t* doc_key;
   float* chunk_s;
   int n_r, n_docs, n_chunks, n_tiles;
-  int q_base, q_count, nb_total, nb_base;
+  int q_base, q_count, pass;
+  uint32_t tmem_cols;
   float inv_nr;
 };
 
-template <int NB, int DR, bool MEAN>
-__global__ void __launch_bounds__(288, 1) scan_kernel(const __grid_constant__ CUtensorMap kr_map,
-                                                      const ScanParams p) {
+template <int DR, int NQ>
+struct ScanGeom {
+  static constexpr int kHalves = DR / 64;
+  static constexpr int kKBox = kScanM * 128;            // one 64-dim x 128-row box
+  static constexpr int kQBox = NQ * 128;                // one 64-dim x NQ-row box
+  static constexpr int kKBytes = kHalves * kKBox;
+  static constexpr int kQBytes = 2 * kHalves * kQBox;   // hi and lo
+  static constexpr int kStageBytes = kKBytes + kQBytes;
+};
+
+template <int DR, int NQ, bool MEAN>
+__global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_constant__ CUtensorMap kr_map,
+                                                               const __grid_constant__ CUtensorMap q_map,
+                                                               const ScanParams p) {
+  using Gm = ScanGeom<DR, NQ>;
   constexpr int KS = DR / 16;
-  constexpr int HALVES = DR / 64;
-  constexpr int QP = 8 * NB;  // padded queries in this pass
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int n_r = p.n_r;
-  const int stage_bytes = n_r * HALVES * kBoxBytes;
   uint8_t* stages = smem;
-  float* partial = reinterpret_cast<float*>(smem + kStages * stage_bytes);  // [2][n_r][QP][kPartStride]
-  int* docids = reinterpret_cast<int*>(partial + 2 * n_r * QP * kPartStride);  // [2][16]
-  uint64_t* full = reinterpret_cast<uint64_t*>(docids + 32);
-  uint64_t* empty = full + kStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kScanStages * Gm::kStageBytes);
+  uint64_t* empty = full + kScanStages;
+  uint64_t* tfull = empty + kScanStages;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_r = p.n_r;
   const int t_begin = (int)(((long long)blockIdx.x * p.n_tiles) / gridDim.x);
   const int t_end = (int)(((long long)(blockIdx.x + 1) * p.n_tiles) / gridDim.x);
-  const int n_it = t_end - t_begin;
+  const int n_it = (t_end - t_begin) * n_r;  // (tile, head) stages of this CTA
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kScanStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], n_r);
+      mbar_init(&empty[s], 1 + 4);  // MMA commit + the four norm warps
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
     }
     fence_mbar_init();
     prefetch_tensormap(&kr_map);
+    prefetch_tensormap(&q_map);
   }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t buf_cols = (uint32_t)n_r * NQ;
   pdl_launch_dependents();
   pdl_wait();
-  __syncthreads();
 
-  if (warp == n_r) {
-    // ---------------- producer: one thread streams tiles with TMA ----------------
+  if (warp == 0) {
+    // ------------------------- TMA producer -------------------------
     if (lane == 0) {
       for (int it = 0; it < n_it; ++it) {
-        const int st = it % kStages;
-        if (it >= kStages) mbar_wait(&empty[st], ((it / kStages) - 1) & 1);
-        mbar_arrive_expect_tx(&full[st], stage_bytes);
-        uint8_t* dst = stages + st * stage_bytes;
-        const int y = (t_begin + it) * kTileC;
-        for (int h = 0; h < n_r; ++h)
-          for (int j = 0; j < HALVES; ++j)
-            tma_load_2d(dst + (h * HALVES + j) * kBoxBytes, &kr_map, &full[st], h * DR + j * 64, y);
-      }
-    }
-    return;
-  }
-
-  // ---------------- consumers: warp h owns router head h ----------------
-  const int h = warp;
-  uint4 qreg[KS][NB];
+        const int tile = t_begin + it / n_r, h = it % n_r;
+        const int st = it % kScanStages;
+        if (it >= kScanStages) mbar_wait(&empty[st], ((it / kScanStages) - 1) & 1);
+        uint8_t* k_s = stages + st * Gm::kStageBytes;
+        uint8_t* q_s = k_s + Gm::kKBytes;
+        mbar_arrive_expect_tx(&full[st], Gm::kStageBytes);
 #pragma unroll
-  for (int s = 0; s < KS; ++s)
+        for (int j = 0; j < Gm::kHalves; ++j) {
+          tma_load_2d(k_s + j * Gm::kKBox, &kr_map, &full[st], h * DR + j * 64, tile * kScanM);
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb)
-      qreg[s][nb] = p.qfrag[((size_t)(h * KS + s) * p.nb_total + p.nb_base + nb) * 32 + lane];
-
-  const int g = lane >> 2, c = lane & 3;
-  const int lrow = (lane & 7) + ((lane >> 3) & 1) * 8;  // ldmatrix source row
-  const int khalf = lane >> 4;
-  const int diag_src = 4 * g + (g >> 1);
-  const int n_consumers = n_r * 32;
-
-  // document cursor (warp 0): index of the document holding this CTA's first chunk
-  int cur = 0;
-  if (warp == 0 && n_it > 0) {
-    const int j0 = t_begin * kTileC;
-    int lo = 0, hi = p.n_docs;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (__ldg(&p.chunk_off[mid]) <= j0) lo = mid; else hi = mid - 1;
-    }
-    cur = lo;
-  }
-
-  for (int it = 0; it < n_it; ++it) {
-    const int tile = t_begin + it;
-    const int st = it % kStages;
-    const int buf = it & 1;
-    mbar_wait(&full[st], (it / kStages) & 1);
-
-    float dot[NB][4];
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) dot[nb][0] = dot[nb][1] = dot[nb][2] = dot[nb][3] = 0.f;
-    float g0[4] = {0.f, 0.f, 0.f, 0.f}, g1[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint32_t stage_base = smem_u32(stages + st * stage_bytes) + h * HALVES * kBoxBytes;
-#pragma unroll
-    for (int s = 0; s < KS; ++s) {
-      const int unit = ((2 * (s & 3) + khalf) ^ (lrow & 7));
-      const uint32_t addr = stage_base + (s >> 2) * kBoxBytes + lrow * 128 + unit * 16;
-      uint32_t a0, a1, a2, a3;
-      ldmatrix_x4(a0, a1, a2, a3, addr);
-#pragma unroll
-      for (int nb = 0; nb < NB; ++nb) {
-        mma_bf16_16816(dot[nb], a0, a1, a2, a3, qreg[s][nb].x, qreg[s][nb].y);
-        mma_bf16_16816(dot[nb], a0, a1, a2, a3, qreg[s][nb].z, qreg[s][nb].w);
-      }
-      mma_bf16_16816(g0, a0, a1, a2, a3, a0, a2);  // Gram, rows x chunks 0..7
-      mma_bf16_16816(g1, a0, a1, a2, a3, a1, a3);  // Gram, rows x chunks 8..15
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[st]);
-
-    // squared norms of rows g and g+8 sit on the Gram diagonals
-    const float d0 = (g & 1) ? g0[1] : g0[0];
-    const float d1 = (g & 1) ? g1[3] : g1[2];
-    const float n2a = __shfl_sync(0xffffffffu, d0, diag_src);
-    const float n2b = __shfl_sync(0xffffffffu, d1, diag_src);
-    const float inva = 1.0f / fmaxf(sqrtf(n2a), kEps);
-    const float invb = 1.0f / fmaxf(sqrtf(n2b), kEps);
-    float* P = partial + ((size_t)buf * n_r + h) * QP * kPartStride;
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-      const int q0 = 8 * nb + 2 * c;
-      P[q0 * kPartStride + g] = dot[nb][0] * inva;
-      P[(q0 + 1) * kPartStride + g] = dot[nb][1] * inva;
-      P[q0 * kPartStride + g + 8] = dot[nb][2] * invb;
-      P[(q0 + 1) * kPartStride + g + 8] = dot[nb][3] * invb;
-    }
-
-    if (warp == 0) {
-      // document id of every row of this tile (at most 16 boundaries ahead of cur)
-      const int j0 = tile * kTileC;
-      const int li = lane & 15;
-      const int bi = cur + 1 + li;
-      const int bnd = (lane < 16 && bi <= p.n_docs) ? __ldg(&p.chunk_off[bi]) : 0x7fffffff;
-      int mydoc = cur;
-#pragma unroll
-      for (int r = 0; r < kTileC; ++r) {
-        const unsigned m = __ballot_sync(0xffffffffu, lane < 16 && bnd <= j0 + r);
-        if (lane == r) mydoc = cur + __popc(m);
-      }
-      if (lane < 16) {
-        int dv = (j0 + lane < p.n_chunks) ? mydoc : -1;
-        if (dv >= p.n_docs) {  // inconsistent chunk_off: drop the row
-          raise_dev_error(kDevErrBadIndex);
-          dv = -1;
+          for (int hl = 0; hl < 2; ++hl)
+            tma_load_2d(q_s + (hl * Gm::kHalves + j) * Gm::kQBox, &q_map, &full[st], j * 64,
+                        ((p.pass * n_r + h) * 2 + hl) * NQ);
         }
-        docids[buf * 16 + lane] = dv;
       }
-      cur = __shfl_sync(0xffffffffu, mydoc, 15);
     }
-    named_bar_sync(1, n_consumers);
-
-    // head mean + per-document segmented max over the 16 rows
-    const float* PB = partial + (size_t)buf * n_r * QP * kPartStride;
-    const int r = lane & 15;
-    const int doc = docids[buf * 16 + r];
-    const int rounds = (p.q_count + 2 * n_r - 1) / (2 * n_r);
-    for (int m = 0; m < rounds; ++m) {
-      const int qq = m * 2 * n_r + 2 * h + (lane >> 4);
-      const bool qok = qq < p.q_count;
-      float v = 0.f;
-      if (qok) {
-        for (int hh = 0; hh < n_r; ++hh) v += PB[(hh * QP + qq) * kPartStride + r];
-        v *= p.inv_nr;
-      }
-      if (MEAN) {
-        if (qok && doc >= 0) p.chunk_s[(size_t)(p.q_base + qq) * p.n_chunks + tile * kTileC + r] = v;
-      } else {
-        float x = (qok && doc >= 0) ? v : -__int_as_float(0x7f800000);
+  } else if (warp == 1) {
+    // ------------------------- MMA issuer -------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(kScanM, NQ);
+      for (int it = 0; it < n_it; ++it) {
+        const int lt = it / n_r, h = it % n_r;
+        const int buf = lt & 1;
+        const int st = it % kScanStages;
+        if (h == 0 && lt >= 2) mbar_wait(&tempty[buf], ((lt >> 1) - 1) & 1);
+        mbar_wait(&full[st], (it / kScanStages) & 1);
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * buf_cols + h * NQ;
+        const uint32_t k_addr = smem_u32(stages + st * Gm::kStageBytes);
+        const uint32_t q_addr = k_addr + Gm::kKBytes;
 #pragma unroll
-        for (int off = 1; off < 16; off <<= 1) {
-          const float ox = __shfl_down_sync(0xffffffffu, x, off, 16);
-          const int od = __shfl_down_sync(0xffffffffu, doc, off, 16);
-          if (r + off < 16 && od == doc) x = fmaxf(x, ox);
+        for (int ks = 0; ks < KS; ++ks) {
+          const int j = ks >> 2, off = (ks & 3) * 32;
+          const uint64_t a_desc = umma_desc_k_sw128(k_addr + j * Gm::kKBox + off);
+          umma_bf16(d_tmem, a_desc, umma_desc_k_sw128(q_addr + j * Gm::kQBox + off), idesc, ks > 0);
+          umma_bf16(d_tmem, a_desc, umma_desc_k_sw128(q_addr + (Gm::kHalves + j) * Gm::kQBox + off), idesc, 1);
         }
-        const int prev = __shfl_up_sync(0xffffffffu, doc, 1, 16);
-        const bool head = (r == 0) || (prev != doc);
-        if (qok && head && doc >= 0)
-          atomicMax(&p.doc_key[(size_t)(p.q_base + qq) * p.n_docs + doc], float_to_ordered(x));
+        umma_commit(&empty[st]);
+        if (h == n_r - 1) umma_commit(&tfull[buf]);
+      }
+    }
+  } else {
+    // --------------- norm + epilogue warps (TMEM lane quarter = warp % 4) ---------------
+    const int q4 = warp & 3;
+    const int row = 32 * q4 + lane;            // chunk within the tile
+    float inv[8];
+    int cur = 0;                               // lower bound for this warp's document search
+    for (int it = 0; it < n_it; ++it) {
+      const int lt = it / n_r, h = it % n_r;
+      const int st = it % kScanStages;
+      mbar_wait(&full[st], (it / kScanStages) & 1);
+      // squared norm of this row's head-h slice, read from the swizzled boxes
+      const uint8_t* k_s = stages + st * Gm::kStageBytes;
+      float n2p[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent partial sums
+#pragma unroll
+      for (int j = 0; j < Gm::kHalves; ++j) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 w = *reinterpret_cast<const uint4*>(k_s + j * Gm::kKBox + row * 128 + ((u ^ (row & 7)) << 4));
+          float2 f;
+          f = unpack_bf16x2(w.x); n2p[0] = fmaf(f.x, f.x, n2p[0]); n2p[1] = fmaf(f.y, f.y, n2p[1]);
+          f = unpack_bf16x2(w.y); n2p[2] = fmaf(f.x, f.x, n2p[2]); n2p[3] = fmaf(f.y, f.y, n2p[3]);
+          f = unpack_bf16x2(w.z); n2p[4] = fmaf(f.x, f.x, n2p[4]); n2p[5] = fmaf(f.y, f.y, n2p[5]);
+          f = unpack_bf16x2(w.w); n2p[6] = fmaf(f.x, f.x, n2p[6]); n2p[7] = fmaf(f.y, f.y, n2p[7]);
+        }
+      }
+      const float n2 = ((n2p[0] + n2p[1]) + (n2p[2] + n2p[3])) + ((n2p[4] + n2p[5]) + (n2p[6] + n2p[7]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+#pragma unroll
+      for (int hh = 0; hh < 8; ++hh)
+        if (hh == h) inv[hh] = 1.0f / fmaxf(sqrtf(n2), kEps);
+      if (h != n_r - 1) continue;
+
+      // ---- epilogue of tile lt: head mean of cosines, per-document max ----
+      const int tile = t_begin + lt;
+      const int buf = lt & 1;
+      mbar_wait(&tfull[buf], (lt >> 1) & 1);
+      tc_fence_after();
+      float acc[NQ];
+#pragma unroll
+      for (int b = 0; b < NQ; ++b) acc[b] = 0.f;
+      const uint32_t t_row = tmem_base + ((uint32_t)(32 * q4) << 16) + buf * buf_cols;
+#pragma unroll
+      for (int hh = 0; hh < 8; ++hh) {
+        if (hh < n_r) {
+          if constexpr (NQ == 32) {
+            float v[32];
+            tmem_ld32(t_row + hh * NQ, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int b = 0; b < 32; ++b) acc[b] = fmaf(v[b], inv[hh], acc[b]);
+          } else {
+            float v[16];
+            tmem_ld16(t_row + hh * NQ, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int b = 0; b < 16; ++b) acc[b] = fmaf(v[b], inv[hh], acc[b]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+
+      // document of this row: search chunk_off from the warp's cursor
+      const int j = tile * kScanM + row;
+      int doc = -1;
+      if (j < p.n_chunks) {
+        int lo = cur, hi = p.n_docs - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (__ldg(&p.chunk_off[mid]) <= j) lo = mid; else hi = mid - 1;
+        }
+        doc = lo;
+      }
+      const int last = __shfl_sync(0xffffffffu, doc, 31);
+      if (last >= 0) cur = last;
+      const int prev = __shfl_up_sync(0xffffffffu, doc, 1);
+      const bool head = (lane == 0) || (prev != doc);
+      // the document pattern is the same for every query: which shuffle partners share my document
+      uint32_t same = 0;
+#pragma unroll
+      for (int e = 0; e < 5; ++e) {
+        const int od = __shfl_down_sync(0xffffffffu, doc, 1 << e);
+        if (lane + (1 << e) < 32 && od == doc) same |= 1u << e;
+      }
+#pragma unroll
+      for (int b = 0; b < NQ; ++b) {
+        if (b >= p.q_count) continue;  // warp-uniform
+        const float sc = acc[b] * p.inv_nr;
+        if (MEAN) {
+          if (doc >= 0) p.chunk_s[(size_t)(p.q_base + b) * p.n_chunks + j] = sc;
+        } else {
+          float x = doc >= 0 ? sc : -__int_as_float(0x7f800000);
+#pragma unroll
+          for (int e = 0; e < 5; ++e) {
+            const float ox = __shfl_down_sync(0xffffffffu, x, 1 << e);
+            if (same & (1u << e)) x = fmaxf(x, ox);
+          }
+          if (head && doc >= 0)
+            atomicMax(&p.doc_key[(size_t)(p.q_base + b) * p.n_docs + doc], float_to_ordered(x));
+        }
       }
     }
   }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, p.tmem_cols);
 }
 
 // --------------------------------------------------------------------------
@@ -518,29 +562,53 @@ __global__ void __launch_bounds__(kTopkThreads) topk_merge_kernel(const uint64_t
   }
 }
 
-template <int NB, int DR, bool MEAN>
-cudaError_t launch_scan_t(const CUtensorMap& map, const ScanParams& p, int grid, size_t smem, cudaStream_t s) {
-  auto kern = scan_kernel<NB, DR, MEAN>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3(grid), dim3((p.n_r + 1) * 32), smem, s, map, p);
-}
-
-template <int DR, bool MEAN>
-cudaError_t launch_scan_nb(int nb, const CUtensorMap& map, const ScanParams& p, int grid, size_t smem,
-                           cudaStream_t s) {
-  switch (nb) {
-    case 1: return launch_scan_t<1, DR, MEAN>(map, p, grid, smem, s);
-    case 2: return launch_scan_t<2, DR, MEAN>(map, p, grid, smem, s);
-    case 3: return launch_scan_t<3, DR, MEAN>(map, p, grid, smem, s);
-    default: return launch_scan_t<4, DR, MEAN>(map, p, grid, smem, s);
+// exact top-k of (score, global document id) candidate pairs, one block per query
+__global__ void __launch_bounds__(kTopkThreads) topk_merge_pairs_kernel(const float* __restrict__ cand_score,
+                                                                        const int32_t* __restrict__ cand_idx,
+                                                                        int n_cand, int k,
+                                                                        int32_t* __restrict__ topk_idx,
+                                                                        float* __restrict__ topk_score) {
+  extern __shared__ uint64_t sm64[];
+  uint64_t* keys = sm64;
+  uint64_t* out = keys + n_cand;
+  uint64_t* tmp = out + 256;
+  uint64_t* state = tmp + 256;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(state + 4);
+  pdl_launch_dependents();
+  pdl_wait();
+  const int b = blockIdx.x;
+  for (int i = threadIdx.x; i < n_cand; i += blockDim.x)
+    keys[i] = make_key(float_to_ordered(cand_score[(size_t)b * n_cand + i]), cand_idx[(size_t)b * n_cand + i]);
+  __syncthreads();
+  block_topk(keys, n_cand, k, out, tmp, hist, state);
+  for (int i = threadIdx.x; i < k; i += blockDim.x) {
+    topk_idx[(size_t)b * k + i] = (int32_t)(0xFFFFFFFFu - (uint32_t)(out[i] & 0xFFFFFFFFu));
+    topk_score[(size_t)b * k + i] = ordered_to_float((uint32_t)(out[i] >> 32));
   }
 }
 
-size_t scan_smem_bytes(int n_r, int d_r, int nb) {
-  const size_t stage = (size_t)n_r * (d_r / 64) * kBoxBytes;
-  return 1024 + kStages * stage + 2ull * n_r * 8 * nb * kPartStride * sizeof(float) + 32 * sizeof(int) +
-         2 * kStages * sizeof(uint64_t);
+template <int DR, int NQ, bool MEAN>
+cudaError_t launch_scan_t(const CUtensorMap& kmap, const CUtensorMap& qmap, const ScanParams& p, int grid,
+                          cudaStream_t s) {
+  auto kern = scan_kernel<DR, NQ, MEAN>;
+  const size_t smem = 1024 + (size_t)kScanStages * ScanGeom<DR, NQ>::kStageBytes + (2 * kScanStages + 4) * 8 + 16;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3(grid), dim3(kScanThreads), smem, s, kmap, qmap, p);
+}
+
+cudaError_t launch_scan(int d_r, int nq, bool mean, const CUtensorMap& kmap, const CUtensorMap& qmap,
+                        const ScanParams& p, int grid, cudaStream_t s) {
+  if (d_r == 128) {
+    if (nq == 16) return mean ? launch_scan_t<128, 16, true>(kmap, qmap, p, grid, s)
+                              : launch_scan_t<128, 16, false>(kmap, qmap, p, grid, s);
+    return mean ? launch_scan_t<128, 32, true>(kmap, qmap, p, grid, s)
+                : launch_scan_t<128, 32, false>(kmap, qmap, p, grid, s);
+  }
+  if (nq == 16) return mean ? launch_scan_t<64, 16, true>(kmap, qmap, p, grid, s)
+                            : launch_scan_t<64, 16, false>(kmap, qmap, p, grid, s);
+  return mean ? launch_scan_t<64, 32, true>(kmap, qmap, p, grid, s)
+              : launch_scan_t<64, 32, false>(kmap, qmap, p, grid, s);
 }
 
 size_t topk_slice_smem() { return (kSliceDocs + 512 + 4) * sizeof(uint64_t) + 256 * sizeof(uint32_t); }
@@ -548,16 +616,27 @@ size_t topk_merge_smem(int n) { return ((size_t)n + 512 + 4) * sizeof(uint64_t) 
 
 }  // namespace
 
+msa_status topk_merge_launch(const float* cand_score, const int32_t* cand_idx, int B, int n_cand, int k,
+                             int32_t* topk_idx, float* topk_score, cudaStream_t s) {
+  TraceScope ts(kKTopkMerge, s);
+  const size_t sm = topk_merge_smem(n_cand);
+  MSA_CUDA_CHECK(cudaFuncSetAttribute(topk_merge_pairs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+  MSA_CUDA_CHECK(launch_pdl(topk_merge_pairs_kernel, dim3(B), dim3(kTopkThreads), sm, s, cand_score, cand_idx, n_cand,
+                            k, topk_idx, topk_score));
+  return MSA_OK;
+}
+
 size_t route_workspace(const msa_dims& d, int B, int n_docs, int n_chunks, int k, msa_doc_agg agg, void* ws,
                        RouteWs* out) {
   Carver cv(ws);
   RouteWs w{};
   const int NR = d.n_r * d.d_r;
   w.ksplit = std::max(1, std::min(32, d.hidden / 160));
-  w.nb_total = (B + 7) / 8;
+  w.nq = B <= 16 ? 16 : 32;
+  w.passes = (B + w.nq - 1) / w.nq;
   w.n_slices = (n_docs + kSliceDocs - 1) / kSliceDocs;
   w.qr_part = cv.take<float>((size_t)w.ksplit * B * NR);
-  w.qfrag = cv.take<uint4>((size_t)d.n_r * (d.d_r / 16) * w.nb_total * 32);
+  w.q_hl = cv.take<__nv_bfloat16>((size_t)w.passes * d.n_r * 2 * w.nq * d.d_r);
   w.doc_key = agg == MSA_AGG_MAX ? cv.take<uint32_t>((size_t)B * n_docs) : nullptr;
   w.chunk_s = agg == MSA_AGG_MEAN ? cv.take<float>((size_t)B * n_chunks) : nullptr;
   w.cand = w.n_slices > 1 ? cv.take<uint64_t>((size_t)B * w.n_slices * k) : nullptr;
@@ -585,25 +664,31 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
   {
     TraceScope ts(kKQPrep, s);
     const size_t sm = (size_t)(NR + d.n_r) * sizeof(float);
-    MSA_CUDA_CHECK(launch_pdl(q_prep_kernel, dim3(w.nb_total * 8), dim3(256), sm, s, (const float*)w.qr_part,
+    MSA_CUDA_CHECK(launch_pdl(q_prep_kernel, dim3(w.passes * w.nq), dim3(256), sm, s, (const float*)w.qr_part,
                               w.ksplit, W_QR ? nullptr : static_cast<const __nv_bfloat16*>(Hq), B, d.n_r, d.d_r,
-                              w.nb_total, w.qfrag, w.doc_key, n_docs));
+                              w.nq, w.q_hl, w.doc_key, n_docs));
   }
-  // K3: scan, 32 queries per pass
+  // K3: scan, NQ (16 or 32) queries per pass
   {
-    CUtensorMap map;
+    CUtensorMap kmap, qmap;
     const uint64_t dims[2] = {(uint64_t)NR, (uint64_t)n_chunks};
     const uint64_t strides[1] = {(uint64_t)NR * 2};
-    const uint32_t box[2] = {64, (uint32_t)kTileC};
-    msa_status st = encode_tensor_map(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(KR_bar), dims,
+    const uint32_t box[2] = {64, (uint32_t)kScanM};
+    msa_status st = encode_tensor_map(&kmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(KR_bar), dims,
                                       strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != MSA_OK) return st;
-    const int n_tiles = (n_chunks + kTileC - 1) / kTileC;
+    const uint64_t qdims[2] = {(uint64_t)d.d_r, (uint64_t)w.passes * d.n_r * 2 * w.nq};
+    const uint64_t qstrides[1] = {(uint64_t)d.d_r * 2};
+    const uint32_t qbox[2] = {64, (uint32_t)w.nq};
+    st = encode_tensor_map(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w.q_hl, qdims, qstrides, qbox,
+                           CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != MSA_OK) return st;
+    const int n_tiles = (n_chunks + kScanM - 1) / kScanM;
     const int grid = std::max(1, std::min(sm_count(), n_tiles));
-    for (int nb_base = 0; nb_base < w.nb_total; nb_base += 4) {
-      const int nb = std::min(4, w.nb_total - nb_base);
+    uint32_t cols = 32;
+    while (cols < 2u * d.n_r * w.nq) cols <<= 1;
+    for (int pass = 0; pass < w.passes; ++pass) {
       ScanParams p;
-      p.qfrag = w.qfrag;
       p.chunk_off = chunk_off;
       p.doc_key = w.doc_key;
       p.chunk_s = w.chunk_s;
@@ -611,18 +696,13 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
       p.n_docs = n_docs;
       p.n_chunks = n_chunks;
       p.n_tiles = n_tiles;
-      p.q_base = nb_base * 8;
-      p.q_count = std::min(B - p.q_base, nb * 8);
-      p.nb_total = w.nb_total;
-      p.nb_base = nb_base;
+      p.q_base = pass * w.nq;
+      p.q_count = std::min(B - p.q_base, w.nq);
+      p.pass = pass;
+      p.tmem_cols = cols;
       p.inv_nr = 1.0f / (float)d.n_r;
-      const size_t smem = scan_smem_bytes(d.n_r, d.d_r, nb);
       TraceScope ts(kKScan, s);
-      cudaError_t e;
-      if (d.d_r == 128)
-        e = mean ? launch_scan_nb<128, true>(nb, map, p, grid, smem, s) : launch_scan_nb<128, false>(nb, map, p, grid, smem, s);
-      else
-        e = mean ? launch_scan_nb<64, true>(nb, map, p, grid, smem, s) : launch_scan_nb<64, false>(nb, map, p, grid, smem, s);
+      cudaError_t e = launch_scan(d.d_r, w.nq, mean, kmap, qmap, p, grid, s);
       if (e != cudaSuccess) return cuda_fail(e, "scan_kernel launch");
     }
   }
