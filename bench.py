@@ -263,6 +263,19 @@ def run_extras(msa, dev, hbm_peak):
         c16 = PC.RouteCase(16_000_000, 32, 2048, W.BASE_SEED + 2, dev)
         route_entry("mem16m_b32_route", c16, 1)
         del c16
+        a16 = PC.AttendCase(16_000_000, 32, 2048, 8192, W.BASE_SEED + 2, dev, rotated=True)
+        ms = timed(lambda i: a16.run(), 10)
+        kt = kernel_times(msa, stream, lambda i: a16.run(), 10)
+        ams, acnt = kt["attn_split"]
+        a_us = ams / acnt * 1e3
+        agbs = a16.kv_bytes / (a_us * 1e-6) / 1e9
+        out["mem16m_b32_attend"] = {"workload": "sparse attention, 16M-token memory, B=32, top-16, 8K local KV "
+                                                "(rotated cache)", "ms": ms,
+                                    "attn_split": {"avg_us": a_us, "GB/s": agbs, "frac": agbs / hbm_peak,
+                                                   "bound": "hbm", "algorithmic_bytes_per_launch": a16.kv_bytes},
+                                    "kernels_us": {k: v[0] / v[1] * 1e3 for k, v in kt.items() if v[1]}}
+        del a16
+        torch.cuda.empty_cache()
         free = torch.cuda.mem_get_info(dev)[0]
         layers = int(max(1, min(36, (free - (8 << 30)) // 3_300_000_000)))
         c100 = PC.RouteCase(100_000_000, 1, 4096, W.BASE_SEED + 4, dev, layers=layers)
@@ -331,15 +344,28 @@ def run_gpu(args):
     a_ws = torch.empty(msa.attend_workspace_size(d, B, k, c["t_loc_max"], c["pos_offset"]) + 256,
                        dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(device=dev)
-    # rotation table of the local positions: a constant of the decode session (like the KV cache)
-    rope = msa.rope_cache_build(d, c["t_loc_max"], c["pos_offset"], device=dev)
+    # The local key cache holds keys already rotated at their global positions (rotated once,
+    # when appended).  Each decode step rotates and appends only the new token's key, then
+    # attends over the rotated cache.
+    Lm1 = int(c["loc_len"][0]) - 1
+    T_loc = c["t_loc_max"]
+    for x in rot:
+        msa.rope_rows(d, x["K_loc"].view(B * T_loc, d.n_kv, d.head_dim),
+                      (c["pos_offset"] + torch.arange(T_loc, dtype=torch.int32, device=dev)).repeat(B))
+    k_new = base["K_loc"][:, Lm1].clone()          # the new token's key before RoPE (synthetic)
+    kn_buf = torch.empty_like(k_new)
+    new_pos = torch.full((B,), c["pos_offset"] + Lm1, dtype=torch.int32, device=dev)
+    torch.cuda.synchronize()
 
     def step(i):
         x = rot[i % N_ROT]
         j = i % N_ROT
         msa.route_topk(d, x["Hq"], W_QR, x["KR"], chunk_off, k, out=(out_idx[j], out_sc[j], None), ws=r_ws)
+        kn_buf.copy_(k_new)
+        msa.rope_rows(d, kn_buf, new_pos)
+        x["K_loc"][:, Lm1].copy_(kn_buf)
         msa.sparse_attend(d, x["q"], x["K_bar"], x["V_bar"], chunk_off, out_idx[j], x["K_loc"], x["V_loc"], loc_len,
-                          c["pos_offset"], out=out_o[j], ws=a_ws, rope_cache=rope)
+                          c["pos_offset"], out=out_o[j], ws=a_ws, k_loc_rotated=True)
 
     # ---- capture one graph per rotation copy (untraced) ----
     graphs = []
@@ -423,11 +449,11 @@ def run_gpu(args):
 
     # ---- end to end through the public API from pinned host buffers ----
     # Per decode step the host supplies the query hidden state H_q, the query q and
-    # the new token's K/V row, which is appended to the device-resident local KV
-    # cache at position loc_len - 1; the step returns top-k ids/scores and the output.
-    Lm1 = int(c["loc_len"][0]) - 1
+    # the new token's K/V row, which is rotated and appended to the device-resident
+    # local KV cache at position loc_len - 1; the step returns top-k ids/scores and
+    # the attention output.
     host = {"Hq": base["Hq"].cpu().pin_memory(), "q": base["q"].cpu().pin_memory(),
-            "k_new": base["K_loc"][:, Lm1].cpu().contiguous().pin_memory(),
+            "k_new": k_new.cpu().contiguous().pin_memory(),
             "v_new": base["V_loc"][:, Lm1].cpu().contiguous().pin_memory()}
     dev_hq, dev_q = torch.empty_like(base["Hq"]), torch.empty_like(base["q"])
     h_idx = torch.empty((B, k), dtype=torch.int32).pin_memory()
@@ -440,11 +466,13 @@ def run_gpu(args):
         x = rot[i % N_ROT]
         dev_hq.copy_(host["Hq"], non_blocking=True)
         dev_q.copy_(host["q"], non_blocking=True)
-        x["K_loc"][:, Lm1].copy_(host["k_new"], non_blocking=True)
+        kn_buf.copy_(host["k_new"], non_blocking=True)
+        msa.rope_rows(d, kn_buf, new_pos)
+        x["K_loc"][:, Lm1].copy_(kn_buf)
         x["V_loc"][:, Lm1].copy_(host["v_new"], non_blocking=True)
         msa.route_topk(d, dev_hq, W_QR, x["KR"], chunk_off, k, out=(out_idx[0], out_sc[0], None), ws=r_ws)
         msa.sparse_attend(d, dev_q, x["K_bar"], x["V_bar"], chunk_off, out_idx[0], x["K_loc"], x["V_loc"], loc_len,
-                          c["pos_offset"], out=out_o[0], ws=a_ws, rope_cache=rope)
+                          c["pos_offset"], out=out_o[0], ws=a_ws, k_loc_rotated=True)
         h_idx.copy_(out_idx[0], non_blocking=True)
         h_sc.copy_(out_sc[0], non_blocking=True)
         h_out.copy_(out_o[0], non_blocking=True)
@@ -491,9 +519,9 @@ def run_gpu(args):
             "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms},
             "cpu_baseline": cpu, "clocks": clocks, "extras": extras,
-            "notes": "value: device time of CUDA-graph replays of the full step; kernels: trace-event brackets "
-                     "of eager launches queued behind a bounded sleep kernel; the local-position RoPE table is "
-                     "built once per decode session (msa_rope_cache_build), outside the step",
+            "notes": "value: device time of CUDA-graph replays of the full decode step (route, rotate+append "
+                     "the new token's key, sparse attention over the rotated local cache); kernels: trace-event "
+                     "brackets of eager launches queued behind a bounded sleep kernel",
         }
         print(json.dumps(line), flush=True)
     if ws > 1:

@@ -195,6 +195,9 @@ msa_status msa_route_topk_static(const msa_dims* dims, const void* Hq, const voi
  *            local token j is rotated to position pos_offset + j.
  *   loc_len  [B] device int32, 0 <= loc_len[b] <= t_loc_max.
  *   rope_cache  optional table from msa_rope_cache_build (NULL = built in ws).
+ *   k_loc_rotated  0: K_loc holds keys before RoPE (rotated here, as above);
+ *              1: K_loc already holds every local key rotated at pos_offset + j
+ *              (see msa_rope_rows); rope_cache is then unused.
  *   softmax_scale  0 -> 1/sqrt(head_dim).
  *   out      [B, n_q, head_dim] bf16.
  * Query head g attends with KV head g / (n_q / n_kv).  No mask: the decode
@@ -209,8 +212,47 @@ msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, con
                              const void* V_bar, const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks,
                              const int32_t* topk_idx, int32_t k, const void* K_loc, const void* V_loc,
                              const int32_t* loc_len, int32_t t_loc_max, int32_t pos_offset,
-                             const void* rope_cache, float softmax_scale, void* out, void* ws, size_t ws_bytes,
-                             void* stream);
+                             const void* rope_cache, int32_t k_loc_rotated, float softmax_scale, void* out,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Host tier: gather the selected documents' pooled K̄/V̄ from pinned host memory.
+ * Pages: IRMaD "M. Materials & Methods", Memory Parallel and tiered storage
+ * item; EverMind article 2.3: the content K̄/V̄ live in host DRAM and only the
+ * top-k documents are loaded, asynchronously, after routing.
+ *   K_bar_host, V_bar_host [n_chunks, n_kv, head_dim] bf16 in pinned (page-locked,
+ *            device-mapped) host memory; read by the GPU over the bus.
+ *   chunk_off [n_docs + 1], topk_idx [B, k] device int32 (msa_route_topk's output).
+ *   K_stage, V_stage  device out, room for capacity_chunks rows each: the chunks of
+ *            query b's r-th document land as staged document b * k + r.
+ *   stage_chunk_off [B * k + 1] device out: chunk offsets of the staged documents.
+ *   stage_topk_idx  [B, k] device out: b * k + r.
+ *   ws       device workspace, >= B * k * 4 bytes, 256-byte aligned.
+ * msa_sparse_attend(K_stage, V_stage, stage_chunk_off, B * k docs, stage_topk_idx, ...)
+ * then attends exactly as over the device-resident memory.  The call needs no
+ * host synchronisation (the indices stay on the device); enqueue it on a side
+ * stream to overlap the host-to-device traffic with other work.  If the
+ * selection needs more than capacity_chunks rows, only what fits is staged and
+ * the device error word reports it.
+ * ------------------------------------------------------------------------- */
+msa_status msa_gather_kv(const msa_dims* dims, const void* K_bar_host, const void* V_bar_host, int32_t n_chunks,
+                         const int32_t* chunk_off, int32_t n_docs, const int32_t* topk_idx, int32_t B, int32_t k,
+                         void* K_stage, void* V_stage, int32_t capacity_chunks, int32_t* stage_chunk_off,
+                         int32_t* stage_topk_idx, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * In-place RoPE of key rows (global positions of the active context).
+ * Pages: IRMaD "M. Materials & Methods", position item.  A decode loop that
+ * keeps its local key cache rotated calls this once per appended token (row
+ * at pos_offset + j) and then runs msa_sparse_attend with k_loc_rotated = 1,
+ * instead of re-rotating every local key at every step.
+ *   x          [rows, heads, head_dim] bf16, rotated in place (rotate-half pairs
+ *              (i, i + head_dim/2), theta_i = rope_base^(-2i/head_dim), angle
+ *              reduced in fp64, result rounded to bf16).
+ *   positions  [rows] device int32, absolute positions.
+ * ------------------------------------------------------------------------- */
+msa_status msa_rope_rows(const msa_dims* dims, void* x, int32_t rows, int32_t heads, const int32_t* positions,
+                         void* stream);
 
 /* ---------------------------------------------------------------------------
  * Global-RoPE cache for the active context (optional input of msa_sparse_attend).

@@ -18,7 +18,7 @@ from typing import Optional
 
 __all__ = [
     "Dims", "MSAError", "lib", "chunk_offsets", "encode_memory", "route_topk", "sparse_attend",
-    "route_workspace_size", "attend_workspace_size", "rope_cache_build", "topk_merge", "encode_workspace_size", "check_device_errors",
+    "route_workspace_size", "attend_workspace_size", "rope_cache_build", "topk_merge", "rope_rows", "gather_kv", "encode_workspace_size", "check_device_errors",
     "trace_enable", "trace_reset", "trace_read", "trace_kernel_names", "AGG_MAX", "AGG_MEAN",
 ]
 
@@ -67,7 +67,9 @@ def _load():
         "msa_route_workspace_size": (SZ, [DP, I32, I32, I32, I32, I32]),
         "msa_route_topk": (I32, [DP, P, P, I32, P, P, I32, I32, I32, I32, P, P, P, P, SZ, P]),
         "msa_attend_workspace_size": (SZ, [DP, I32, I32, I32, I32]),
-        "msa_sparse_attend": (I32, [DP, P, I32, P, P, P, I32, I32, P, I32, P, P, P, I32, I32, P, F, P, P, SZ, P]),
+        "msa_sparse_attend": (I32, [DP, P, I32, P, P, P, I32, I32, P, I32, P, P, P, I32, I32, P, I32, F, P, P, SZ, P]),
+        "msa_rope_rows": (I32, [DP, P, I32, I32, P, P]),
+        "msa_gather_kv": (I32, [DP, P, P, I32, P, I32, P, I32, I32, P, P, I32, P, P, P, SZ, P]),
         "msa_rope_cache_size": (SZ, [DP, I32]),
         "msa_rope_cache_build": (I32, [DP, I32, I32, P, SZ, P]),
         "msa_topk_merge": (I32, [P, P, I32, I32, I32, P, P, P]),
@@ -240,8 +242,38 @@ def rope_cache_build(dims, t_loc_max: int, pos_offset: int, device=None, out=Non
     return out
 
 
+def gather_kv(dims, K_bar_host, V_bar_host, chunk_off, topk_idx, capacity_chunks: int, out=None, stream=None):
+    """Stage the selected documents' pooled K̄/V̄ from pinned host memory onto the device.
+
+    Returns (K_stage, V_stage, stage_chunk_off [B*k+1], stage_topk_idx [B, k]) for sparse_attend.
+    """
+    import torch
+
+    B, k = topk_idx.shape
+    dev = topk_idx.device
+    n_docs = chunk_off.numel() - 1
+    if out is None:
+        shape = (capacity_chunks, dims.n_kv, dims.head_dim)
+        out = (torch.empty(shape, dtype=torch.bfloat16, device=dev), torch.empty(shape, dtype=torch.bfloat16, device=dev),
+               torch.empty(B * k + 1, dtype=torch.int32, device=dev), torch.empty((B, k), dtype=torch.int32, device=dev))
+    ws = torch.empty(B * k * 4 + 256, dtype=torch.uint8, device=dev)
+    _check(lib.msa_gather_kv(ctypes.byref(Dims.of(dims)), _ptr(K_bar_host), _ptr(V_bar_host), K_bar_host.shape[0],
+                             _ptr(chunk_off), n_docs, _ptr(topk_idx), B, k, _ptr(out[0]), _ptr(out[1]),
+                             capacity_chunks, _ptr(out[2]), _ptr(out[3]), _aligned_ptr(ws), B * k * 4,
+                             _stream(stream)))
+    return out
+
+
+def rope_rows(dims, x, positions, stream=None):
+    """Rotate x [rows, heads, head_dim] (bf16, in place) at positions [rows] (int32, device)."""
+    rows, heads = x.shape[0], x.shape[1]
+    _check(lib.msa_rope_rows(ctypes.byref(Dims.of(dims)), _ptr(x), rows, heads, _ptr(positions), _stream(stream)))
+    return x
+
+
 def sparse_attend(dims, q, K_bar, V_bar, chunk_off, topk_idx, K_loc, V_loc, loc_len, pos_offset: int,
-                  softmax_scale: float = 0.0, out=None, ws=None, stream=None, rope_cache=None):
+                  softmax_scale: float = 0.0, out=None, ws=None, stream=None, rope_cache=None,
+                  k_loc_rotated: bool = False):
     """One GQA decode step over [selected docs' K̄; local K].  Returns out [B, n_q, head_dim] bf16.
 
     ``rope_cache`` (from ``rope_cache_build`` with the same pos_offset and t_loc_max) skips
@@ -259,7 +291,8 @@ def sparse_attend(dims, q, K_bar, V_bar, chunk_off, topk_idx, K_loc, V_loc, loc_
     ws = _workspace(nbytes, dev, ws)
     _check(lib.msa_sparse_attend(ctypes.byref(dd), _ptr(q), B, _ptr(K_bar), _ptr(V_bar), _ptr(chunk_off), n_docs,
                                  K_bar.shape[0], _ptr(topk_idx), k, _ptr(K_loc), _ptr(V_loc), _ptr(loc_len),
-                                 t_loc_max, pos_offset, _ptr(rope_cache), float(softmax_scale), _ptr(out),
+                                 t_loc_max, pos_offset, _ptr(rope_cache), int(bool(k_loc_rotated)),
+                                 float(softmax_scale), _ptr(out),
                                  _aligned_ptr(ws), nbytes, _stream(stream)))
     return out
 

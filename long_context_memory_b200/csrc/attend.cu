@@ -102,45 +102,51 @@ struct AttnParams {
 //   then barriers, the segment table, the query's cos/sin and the raw query.
 struct AttnSmem {
   int krow, kbytes, tbytes, stage_bytes, n_stages;
-  __host__ __device__ AttnSmem(int n_kv, int D, int stages) {
+  __host__ __device__ AttnSmem(int n_kv, int D, int stages, bool table) {
     krow = n_kv * D * 2 + 16;
     kbytes = kTK * krow;
-    tbytes = kTK * (D / 2) * 8;
+    tbytes = table ? kTK * (D / 2) * 8 : 0;
     stage_bytes = 2 * kbytes + tbytes;
     n_stages = stages;
   }
   __host__ __device__ size_t fixed_bytes(int n_q, int D) const {
-    return kMaxStages * 8 + (2 * kMaxK + 2) * 4 + (size_t)(D / 2) * 8 + (size_t)n_q * D * 2;
+    return 2 * kMaxStages * 8 + (2 * kMaxK + 2) * 4 + (size_t)(D / 2) * 8 + (size_t)n_q * D * 2;
   }
   __host__ __device__ size_t total(int n_q, int D) const { return (size_t)n_stages * stage_bytes + fixed_bytes(n_q, D); }
 };
 
 template <int D>
-__global__ void __launch_bounds__(256, 1) attn_split_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) {
   constexpr int KS = D / 16;
   constexpr int NBLK = D / 8;
   const int n_kv = p.n_kv, G = p.n_q / n_kv;
-  const AttnSmem L_(n_kv, D, p.n_stages);
+  const bool table = p.rope_tab != nullptr;  // local keys still need their global rotation
+  const AttnSmem L_(n_kv, D, p.n_stages, table);
   extern __shared__ __align__(128) uint8_t sm[];
   // offsets: every region below starts on a 16-byte boundary (stage rows, query rows and
   // the RoPE rows are bulk-copy or 16-byte vector destinations)
   uint8_t* stage_mem = sm;
   uint16_t* qsm = reinterpret_cast<uint16_t*>(sm + (size_t)L_.n_stages * L_.stage_bytes);  // [n_q][D] raw query
-  uint64_t* bars = reinterpret_cast<uint64_t*>(qsm + (size_t)p.n_q * D);
-  int* seg_v = reinterpret_cast<int*>(bars + kMaxStages);  // [k + 1] virtual starts
+  uint64_t* bars = reinterpret_cast<uint64_t*>(qsm + (size_t)p.n_q * D);  // [stage] tile landed
+  uint64_t* ebars = bars + kMaxStages;                                      // [stage] every warp done with it
+  int* seg_v = reinterpret_cast<int*>(ebars + kMaxStages);  // [k + 1] virtual starts
   int* seg_c = seg_v + kMaxK + 2;                          // [k] chunk starts
   float2* qcs = reinterpret_cast<float2*>(seg_c + kMaxK);  // [D/2] cos/sin at the query position
 
   const int split = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int h = warp;  // the KV head this warp serves
+  const int h = warp;               // the KV head this warp serves (warps 0 .. n_kv-1)
+  const bool producer = warp == n_kv;  // the last warp only streams tiles in
   const int k = p.k;
 
   // ---- no global memory yet: overlaps the previous kernel's tail ----
   for (int i = tid; i < L_.n_stages * L_.stage_bytes / 16; i += blockDim.x)
     reinterpret_cast<uint4*>(stage_mem)[i] = make_uint4(0, 0, 0, 0);
   if (tid == 0) {
-    for (int s = 0; s < L_.n_stages; ++s) mbar_init(&bars[s], 1);
+    for (int s = 0; s < L_.n_stages; ++s) {
+      mbar_init(&bars[s], 1);
+      mbar_init(&ebars[s], n_kv);
+    }
     fence_mbar_init();
   }
   pdl_launch_dependents();
@@ -201,11 +207,10 @@ __global__ void __launch_bounds__(256, 1) attn_split_kernel(const AttnParams p) 
   const int v1 = min(n_keys, v0 + per_split);
   const int n_tiles = (v1 - v0 + kTK - 1) / kTK;
   const int row_bytes = n_kv * D * 2;  // one key, every KV head
-  const bool table = p.rope_tab != nullptr;
 
   // ---- one tile = kTK keys: a 2-row bulk copy pair per key plus one copy of the RoPE rows ----
   auto issue = [&](int t, int st) {
-    if (warp != 0) return;
+    if (t >= L_.n_stages) mbar_wait(&ebars[st], ((t / L_.n_stages) - 1) & 1);
     const int tv0 = v0 + t * kTK;
     const int rows = min(kTK, v1 - tv0);
     const int n_chunk_rows = max(0, min(rows, n_sel - tv0));
@@ -240,10 +245,14 @@ __global__ void __launch_bounds__(256, 1) attn_split_kernel(const AttnParams p) 
       bulk_load(vdst + L_.kbytes + n_chunk_rows * (D / 2) * 8, p.rope_tab + (size_t)j0 * (D / 2), tb, &bars[st]);
     }
   };
-  for (int t = 0; t < L_.n_stages - 1 && t < n_tiles; ++t) issue(t, t % L_.n_stages);
+  if (producer) {
+    for (int t = 0; t < n_tiles; ++t) issue(t, t % L_.n_stages);
+    return;  // the compute warps no longer synchronise with the whole block
+  }
 
   // ---- query fragments of this warp's GQA group: rotate to pos_offset + L - 1, scale, bf16 ----
-  for (int i = tid; i < D / 2; i += blockDim.x) {
+  const int n_compute = 32 * n_kv;
+  for (int i = tid; i < D / 2; i += n_compute) {
     double a = (double)(p.pos_offset + L - 1) * exp(-2.0 * (double)i / (double)D * p.log_base);
     const double two_pi = 6.283185307179586476925286766559;
     a -= two_pi * rint(a / two_pi);
@@ -251,7 +260,7 @@ __global__ void __launch_bounds__(256, 1) attn_split_kernel(const AttnParams p) 
     sincos(a, &sv, &cv);
     qcs[i] = make_float2((float)cv, (float)sv);
   }
-  __syncthreads();
+  named_bar_sync(1, n_compute);
   const int g = lane >> 2, c = lane & 3;
   uint32_t qa[KS][4];
   {
@@ -295,7 +304,6 @@ __global__ void __launch_bounds__(256, 1) attn_split_kernel(const AttnParams p) 
 
   for (int t = 0; t < n_tiles; ++t) {
     const int st = t % L_.n_stages;
-    if (t + L_.n_stages - 1 < n_tiles) issue(t + L_.n_stages - 1, (t + L_.n_stages - 1) % L_.n_stages);
     mbar_wait(&bars[st], (t / L_.n_stages) & 1);
 
     const int tv0 = v0 + t * kTK;
@@ -402,7 +410,8 @@ __global__ void __launch_bounds__(256, 1) attn_split_kernel(const AttnParams p) 
         mma_bf16_16816(acc[n + 1], pa0, pa1, pa2, pa3, b2, b3);
       }
     }
-    __syncthreads();  // every warp is done with stage st before it is refilled
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ebars[st]);  // this warp is done with stage st
   }
 
   // ---- this warp's split partial: unnormalised output, running max and sum per q head ----
@@ -475,20 +484,154 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float* __restri
   }
 }
 
-int stages_that_fit(int n_kv, int n_q, int D) {
-  const int budget = 200 * 1024;
+int stages_that_fit(int n_kv, int n_q, int D, bool table) {
+  const int budget = 210 * 1024;
   for (int st = kMaxStages; st >= 2; --st) {
-    AttnSmem L(n_kv, D, st);
+    AttnSmem L(n_kv, D, st, table);
     if (L.total(n_q, D) <= (size_t)budget) return st;
   }
   return 2;
 }
 
+// rotate rows of x [rows, heads, D] in place: pair (i, i + D/2) of row r by pos[r] * theta_i
+template <int D>
+__global__ void __launch_bounds__(256) rope_rows_kernel(__nv_bfloat16* __restrict__ x, int rows, int heads,
+                                                        const int32_t* __restrict__ pos, double log_base) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int64_t n = (int64_t)rows * heads * (D / 2);
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const int i = (int)(e % (D / 2));
+    const int64_t rh = e / (D / 2);
+    const int r = (int)(rh / heads);
+    double a = (double)pos[r] * exp(-2.0 * (double)i / (double)D * log_base);
+    const double two_pi = 6.283185307179586476925286766559;
+    a -= two_pi * rint(a / two_pi);
+    double sv, cv;
+    sincos(a, &sv, &cv);
+    const float cs = (float)cv, sn = (float)sv;
+    __nv_bfloat16* v = x + rh * D;
+    const float x1 = __bfloat162float(v[i]), x2 = __bfloat162float(v[i + D / 2]);
+    v[i] = __float2bfloat16_rn(x1 * cs - x2 * sn);
+    v[i + D / 2] = __float2bfloat16_rn(x2 * cs + x1 * sn);
+  }
+}
+
+// splits per query: enough CTAs for about four waves, rounded so that B * splits is a
+// whole number of waves on this GPU (one CTA per SM), and at least ~32 keys per split
 int choose_splits(int B, int t_loc_max, int k) {
-  const int target = 4 * sm_count();
-  int s = (target + B - 1) / B;
-  const int max_useful = std::max(1, (t_loc_max + 16 * k) / 32);
-  return std::max(1, std::min({s, max_useful, kMaxSplits}));
+  const int sms = sm_count();
+  const int max_useful = std::max(1, std::min((t_loc_max + 16 * k) / 32, kMaxSplits));
+  const int want = std::max(1, (4 * sms + B - 1) / B);
+  int g = sms, b = B;
+  while (b) {
+    const int t = g % b;
+    g = b;
+    b = t;
+  }
+  const int wave = sms / g;  // B * (multiple of wave) is a multiple of sms
+  int s = (want + wave - 1) / wave * wave;
+  if (s > max_useful) s = std::min(want, max_useful);
+  return std::max(1, s);
+}
+
+// ---------------------------------------------------------------------------
+// host tier: gather the selected documents' pooled K̄/V̄ rows from pinned host
+// memory into a device staging area (zero-copy 16-byte loads over the bus)
+// ---------------------------------------------------------------------------
+// one block: staged chunk offsets of the B*k selected documents, their new ids
+__global__ void __launch_bounds__(1024) gather_plan_kernel(const int32_t* __restrict__ chunk_off, int n_docs,
+                                                           const int32_t* __restrict__ topk_idx, int n_sel,
+                                                           int capacity, int32_t* __restrict__ stage_off,
+                                                           int32_t* __restrict__ stage_src,
+                                                           int32_t* __restrict__ stage_idx) {
+  __shared__ int cnt[1024];
+  __shared__ int carry;
+  pdl_launch_dependents();
+  pdl_wait();
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < n_sel; base += blockDim.x) {
+    const int i = base + threadIdx.x;
+    int n = 0, src = 0;
+    if (i < n_sel) {
+      const int doc = topk_idx[i];
+      if (doc >= 0 && doc < n_docs) {
+        src = chunk_off[doc];
+        n = chunk_off[doc + 1] - src;
+      } else {
+        raise_dev_error(kDevErrBadIndex);
+      }
+      stage_src[i] = src;
+      stage_idx[i] = i;  // query b's r-th document is staged document b * k + r
+    }
+    cnt[threadIdx.x] = n;
+    __syncthreads();
+    // inclusive scan (Hillis-Steele) over this batch of up to 1024 documents
+    for (int o = 1; o < (int)blockDim.x; o <<= 1) {
+      const int v = threadIdx.x >= (unsigned)o ? cnt[threadIdx.x - o] : 0;
+      __syncthreads();
+      cnt[threadIdx.x] += v;
+      __syncthreads();
+    }
+    if (i < n_sel) {
+      int end = carry + cnt[threadIdx.x];
+      if (end > capacity) {  // staging too small: keep what fits, report
+        raise_dev_error(kDevErrBadIndex);
+        end = capacity;
+      }
+      stage_off[i + 1] = end;
+    }
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) carry = carry + cnt[threadIdx.x];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) stage_off[0] = 0;
+}
+
+// copy the planned chunk rows (row = n_kv*D bf16 of K and of V) from host to the staging
+__global__ void __launch_bounds__(256) gather_copy_kernel(const uint4* __restrict__ K_host,
+                                                          const uint4* __restrict__ V_host,
+                                                          const int32_t* __restrict__ stage_off,
+                                                          const int32_t* __restrict__ stage_src, int n_sel,
+                                                          int row_vec, uint4* __restrict__ K_stage,
+                                                          uint4* __restrict__ V_stage) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int total_rows = stage_off[n_sel];
+  const int64_t n = (int64_t)total_rows * row_vec;  // 16-byte vectors
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += 4 * stride) {
+    uint4 kv[4], vv[4];
+    int64_t dst[4], src[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t ee = e + u * stride;
+      dst[u] = -1;
+      if (ee < n) {
+        const int row = (int)(ee / row_vec), col = (int)(ee % row_vec);
+        int lo = 0, hi = n_sel - 1;  // staged document holding this row
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (stage_off[mid] <= row) lo = mid; else hi = mid - 1;
+        }
+        dst[u] = ee;
+        src[u] = (int64_t)(stage_src[lo] + (row - stage_off[lo])) * row_vec + col;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (dst[u] >= 0) {
+        kv[u] = K_host[src[u]];
+        vv[u] = V_host[src[u]];
+      }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (dst[u] >= 0) {
+        K_stage[dst[u]] = kv[u];
+        V_stage[dst[u]] = vv[u];
+      }
+  }
 }
 
 }  // namespace
@@ -505,6 +648,27 @@ size_t attend_workspace(const msa_dims& d, int B, int k, int t_loc_max, int pos_
   return cv.size();
 }
 
+msa_status gather_kv_launch(const msa_dims& d, const void* K_host, const void* V_host, const int32_t* chunk_off,
+                            int n_docs, const int32_t* topk_idx, int B, int k, void* K_stage, void* V_stage,
+                            int capacity_chunks, int32_t* stage_off, int32_t* stage_idx, int32_t* stage_src,
+                            cudaStream_t s) {
+  const int n_sel = B * k;
+  {
+    TraceScope ts(kKGatherPlan, s);
+    MSA_CUDA_CHECK(launch_pdl(gather_plan_kernel, dim3(1), dim3(1024), 0, s, chunk_off, n_docs, topk_idx, n_sel,
+                              capacity_chunks, stage_off, stage_src, stage_idx));
+  }
+  {
+    TraceScope ts(kKGatherCopy, s);
+    const int row_vec = d.n_kv * d.head_dim * 2 / 16;
+    MSA_CUDA_CHECK(launch_pdl(gather_copy_kernel, dim3(4 * sm_count()), dim3(256), 0, s,
+                              static_cast<const uint4*>(K_host), static_cast<const uint4*>(V_host),
+                              (const int32_t*)stage_off, (const int32_t*)stage_src, n_sel, row_vec,
+                              static_cast<uint4*>(K_stage), static_cast<uint4*>(V_stage)));
+  }
+  return MSA_OK;
+}
+
 msa_status rope_cache_build(const msa_dims& d, int t_loc_max, int pos_offset, float2* tab, cudaStream_t s) {
   if (t_loc_max <= 0) return MSA_OK;
   const int D = d.head_dim;
@@ -514,16 +678,31 @@ msa_status rope_cache_build(const msa_dims& d, int t_loc_max, int pos_offset, fl
   return MSA_OK;
 }
 
+msa_status rope_rows_launch(const msa_dims& d, void* x, int rows, int heads, const int32_t* pos, cudaStream_t s) {
+  TraceScope ts(kKRopeRows, s);
+  const int64_t n = (int64_t)rows * heads * (d.head_dim / 2);
+  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 8 * sm_count()));
+  const double lb = std::log((double)d.rope_base);
+  if (d.head_dim == 128)
+    MSA_CUDA_CHECK(launch_pdl(rope_rows_kernel<128>, dim3(blocks), dim3(256), 0, s, static_cast<__nv_bfloat16*>(x),
+                              rows, heads, pos, lb));
+  else
+    MSA_CUDA_CHECK(launch_pdl(rope_rows_kernel<64>, dim3(blocks), dim3(256), 0, s, static_cast<__nv_bfloat16*>(x),
+                              rows, heads, pos, lb));
+  return MSA_OK;
+}
+
 msa_status attend_launch(const msa_dims& d, const void* q, int B, const void* K_bar, const void* V_bar,
                          const int32_t* chunk_off, int n_docs, const int32_t* topk_idx, int k, const void* K_loc,
                          const void* V_loc, const int32_t* loc_len, int t_loc_max, int pos_offset,
-                         const void* rope_cache, float scale, void* out, void* ws, cudaStream_t s) {
+                         const void* rope_cache, int k_loc_rotated, float scale, void* out, void* ws,
+                         cudaStream_t s) {
   AttendWs w;
   attend_workspace(d, B, k, t_loc_max, pos_offset, ws, &w);
   const int D = d.head_dim;
   const double log_base = std::log((double)d.rope_base);
-  const float2* tab = static_cast<const float2*>(rope_cache);
-  if (!tab) {
+  const float2* tab = k_loc_rotated ? nullptr : static_cast<const float2*>(rope_cache);
+  if (!tab && !k_loc_rotated && t_loc_max > 0) {
     msa_status st = rope_cache_build(d, t_loc_max, pos_offset, w.rope_tab, s);
     if (st != MSA_OK) return st;
     tab = w.rope_tab;
@@ -549,17 +728,17 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, const void* K_
   p.n_splits = w.n_splits;
   p.scale_log2 = (scale > 0.f ? scale : 1.0f / std::sqrt((float)D)) * kLog2e;
   p.log_base = log_base;
-  p.n_stages = stages_that_fit(d.n_kv, d.n_q, D);
+  p.n_stages = stages_that_fit(d.n_kv, d.n_q, D, tab != nullptr);
   {
     TraceScope ts(kKAttnSplit, s);
     dim3 grid(w.n_splits, B);
-    const size_t sm = AttnSmem(d.n_kv, D, p.n_stages).total(d.n_q, D);
+    const size_t sm = AttnSmem(d.n_kv, D, p.n_stages, tab != nullptr).total(d.n_q, D);
     if (D == 128) {
       MSA_CUDA_CHECK(cudaFuncSetAttribute(attn_split_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-      MSA_CUDA_CHECK(launch_pdl(attn_split_kernel<128>, grid, dim3(32 * d.n_kv), sm, s, p));
+      MSA_CUDA_CHECK(launch_pdl(attn_split_kernel<128>, grid, dim3(32 * (d.n_kv + 1)), sm, s, p));
     } else {
       MSA_CUDA_CHECK(cudaFuncSetAttribute(attn_split_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-      MSA_CUDA_CHECK(launch_pdl(attn_split_kernel<64>, grid, dim3(32 * d.n_kv), sm, s, p));
+      MSA_CUDA_CHECK(launch_pdl(attn_split_kernel<64>, grid, dim3(32 * (d.n_kv + 1)), sm, s, p));
     }
   }
   {

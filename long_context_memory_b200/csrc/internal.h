@@ -47,6 +47,9 @@ enum KernelId : int {
   kKEncGemmK,
   kKEncPoolH,
   kKEncGemmPooled,
+  kKRopeRows,
+  kKGatherPlan,
+  kKGatherCopy,
   kKernelCount
 };
 
@@ -125,8 +128,13 @@ size_t attend_workspace(const msa_dims& d, int B, int k, int t_loc_max, int pos_
 msa_status attend_launch(const msa_dims& d, const void* q, int B, const void* K_bar, const void* V_bar,
                          const int32_t* chunk_off, int n_docs, const int32_t* topk_idx, int k,
                          const void* K_loc, const void* V_loc, const int32_t* loc_len, int t_loc_max,
-                         int pos_offset, const void* rope_cache, float scale, void* out, void* ws,
-                         cudaStream_t s);
+                         int pos_offset, const void* rope_cache, int k_loc_rotated, float scale, void* out,
+                         void* ws, cudaStream_t s);
+msa_status gather_kv_launch(const msa_dims& d, const void* K_host, const void* V_host, const int32_t* chunk_off,
+                            int n_docs, const int32_t* topk_idx, int B, int k, void* K_stage, void* V_stage,
+                            int capacity_chunks, int32_t* stage_off, int32_t* stage_idx, int32_t* stage_src,
+                            cudaStream_t s);
+msa_status rope_rows_launch(const msa_dims& d, void* x, int rows, int heads, const int32_t* pos, cudaStream_t s);
 msa_status rope_cache_build(const msa_dims& d, int t_loc_max, int pos_offset, float2* tab, cudaStream_t s);
 
 size_t encode_workspace(const msa_dims& d, int64_t T, int n_docs, int n_chunks, void* ws,

@@ -99,7 +99,7 @@ msa_status encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int ra
 namespace {
 const char* kKernelNames[kKernelCount] = {
     "qr_proj", "q_prep", "scan", "topk_slice", "topk_merge", "rope_table", "attn_split", "attn_combine",
-    "enc_chunk_map", "enc_transpose_w", "enc_gemm_k", "enc_pool_h", "enc_gemm_pooled"};
+    "enc_chunk_map", "enc_transpose_w", "enc_gemm_k", "enc_pool_h", "enc_gemm_pooled", "rope_rows", "gather_plan", "gather_copy"};
 
 struct TraceState {
   std::mutex mu;
@@ -306,8 +306,8 @@ size_t msa_attend_workspace_size(const msa_dims* dims, int32_t B, int32_t k, int
 msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, const void* K_bar, const void* V_bar,
                              const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks, const int32_t* topk_idx,
                              int32_t k, const void* K_loc, const void* V_loc, const int32_t* loc_len,
-                             int32_t t_loc_max, int32_t pos_offset, const void* rope_cache, float softmax_scale,
-                             void* out, void* ws,
+                             int32_t t_loc_max, int32_t pos_offset, const void* rope_cache,
+                             int32_t k_loc_rotated, float softmax_scale, void* out, void* ws,
                              size_t ws_bytes, void* stream) {
   msa_status st = check_dims(dims, true, false);
   if (st != MSA_OK) return st;
@@ -339,7 +339,58 @@ msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, con
     return fail(MSA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
   if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
   return attend_launch(*dims, q, B, K_bar, V_bar, chunk_off, n_docs, topk_idx, k, K_loc, V_loc, loc_len, t_loc_max,
-                       pos_offset, rope_cache, softmax_scale, out, ws, static_cast<cudaStream_t>(stream));
+                       pos_offset, rope_cache, k_loc_rotated, softmax_scale, out, ws,
+                       static_cast<cudaStream_t>(stream));
+}
+
+msa_status msa_gather_kv(const msa_dims* dims, const void* K_bar_host, const void* V_bar_host, int32_t n_chunks,
+                         const int32_t* chunk_off, int32_t n_docs, const int32_t* topk_idx, int32_t B, int32_t k,
+                         void* K_stage, void* V_stage, int32_t capacity_chunks, int32_t* stage_chunk_off,
+                         int32_t* stage_topk_idx, void* ws, size_t ws_bytes, void* stream) {
+  msa_status st = check_dims(dims, true, false);
+  if (st != MSA_OK) return st;
+  if (B < 1 || k < 1 || k > n_docs || n_docs < 1 || n_chunks < n_docs)
+    return fail(MSA_ERR_INVALID_ARG, "bad sizes (B %d, k %d, n_docs %d, n_chunks %d)", B, k, n_docs, n_chunks);
+  if (capacity_chunks < 1) return fail(MSA_ERR_INVALID_ARG, "capacity_chunks must be >= 1");
+  CHECK_PTR(K_bar_host);
+  CHECK_PTR(V_bar_host);
+  CHECK_PTR(chunk_off);
+  CHECK_PTR(topk_idx);
+  CHECK_PTR(K_stage);
+  CHECK_PTR(V_stage);
+  CHECK_PTR(stage_chunk_off);
+  CHECK_PTR(stage_topk_idx);
+  const size_t need = (size_t)B * k * sizeof(int32_t);
+  if (ws_bytes < need) return fail(MSA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(MSA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
+  // the pooled memory must be pinned host memory that the device can address
+  const void* dev_ptr[2] = {nullptr, nullptr};
+  const void* host_ptr[2] = {K_bar_host, V_bar_host};
+  for (int i = 0; i < 2; ++i) {
+    cudaPointerAttributes a;
+    cudaError_t e = cudaPointerGetAttributes(&a, host_ptr[i]);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaPointerGetAttributes");
+    if (a.type != cudaMemoryTypeHost || !a.devicePointer)
+      return fail(MSA_ERR_INVALID_ARG, "%s must be pinned (page-locked, device-mapped) host memory",
+                  i ? "V_bar_host" : "K_bar_host");
+    dev_ptr[i] = a.devicePointer;
+  }
+  if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
+  return gather_kv_launch(*dims, dev_ptr[0], dev_ptr[1], chunk_off, n_docs, topk_idx, B, k, K_stage, V_stage,
+                          capacity_chunks, stage_chunk_off, stage_topk_idx, static_cast<int32_t*>(ws),
+                          static_cast<cudaStream_t>(stream));
+}
+
+msa_status msa_rope_rows(const msa_dims* dims, void* x, int32_t rows, int32_t heads, const int32_t* positions,
+                         void* stream) {
+  msa_status st = check_dims(dims, true, false);
+  if (st != MSA_OK) return st;
+  if (rows < 1 || heads < 1) return fail(MSA_ERR_INVALID_ARG, "rows and heads must be >= 1 (got %d, %d)", rows, heads);
+  CHECK_PTR(x);
+  if (!positions) return fail(MSA_ERR_INVALID_ARG, "positions is NULL");
+  if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
+  return rope_rows_launch(*dims, x, rows, heads, positions, static_cast<cudaStream_t>(stream));
 }
 
 size_t msa_rope_cache_size(const msa_dims* dims, int32_t t_loc_max) {

@@ -187,7 +187,8 @@ __global__ void __launch_bounds__(256) q_prep_kernel(const float* __restrict__ p
 // --------------------------------------------------------------------------
 constexpr int kScanM = 128;         // chunks per tile (MMA M)
 constexpr int kScanStages = 4;
-constexpr int kScanThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 norms + epilogue
+constexpr int kScanThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2..9 norms + epilogue
+constexpr int kScanEpiWarps = 8;    // two per TMEM lane quarter
 
 struct ScanParams {
   const int32_t* chunk_off;
@@ -218,7 +219,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kScanStages * Gm::kStageBytes);
+  float* n2s = reinterpret_cast<float*>(smem + kScanStages * Gm::kStageBytes);  // [2 tiles][8 heads][2 halves][128]
+  uint64_t* full = reinterpret_cast<uint64_t*>(n2s + 2 * 8 * 2 * kScanM);
   uint64_t* empty = full + kScanStages;
   uint64_t* tfull = empty + kScanStages;
   uint64_t* tempty = tfull + 2;
@@ -233,11 +235,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   if (threadIdx.x == 0) {
     for (int s = 0; s < kScanStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + 4);  // MMA commit + the four norm warps
+      mbar_init(&empty[s], 1 + kScanEpiWarps);  // MMA commit + the norm warps
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&tempty[b], kScanEpiWarps);
     }
     fence_mbar_init();
     prefetch_tensormap(&kr_map);
@@ -301,82 +303,101 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       }
     }
   } else {
-    // --------------- norm + epilogue warps (TMEM lane quarter = warp % 4) ---------------
+    // ------- norm + epilogue warps: TMEM lane quarter = warp % 4, half = which pair member -------
+    constexpr int QH = NQ / 2;                 // queries per half
     const int q4 = warp & 3;
+    const int hf = (warp - 2) >> 2;            // 0 or 1
     const int row = 32 * q4 + lane;            // chunk within the tile
-    float inv[8];
     int cur = 0;                               // lower bound for this warp's document search
     for (int it = 0; it < n_it; ++it) {
       const int lt = it / n_r, h = it % n_r;
       const int st = it % kScanStages;
       mbar_wait(&full[st], (it / kScanStages) & 1);
-      // squared norm of this row's head-h slice, read from the swizzled boxes
+      // partial squared norm of this row's head-h slice (this warp's half of the dims)
       const uint8_t* k_s = stages + st * Gm::kStageBytes;
-      float n2p[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent partial sums
+      float n2p[4] = {0.f, 0.f, 0.f, 0.f};
+      constexpr int UN = (Gm::kHalves == 2) ? 8 : 4;   // 16-byte units per half
 #pragma unroll
-      for (int j = 0; j < Gm::kHalves; ++j) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint4 w = *reinterpret_cast<const uint4*>(k_s + j * Gm::kKBox + row * 128 + ((u ^ (row & 7)) << 4));
-          float2 f;
-          f = unpack_bf16x2(w.x); n2p[0] = fmaf(f.x, f.x, n2p[0]); n2p[1] = fmaf(f.y, f.y, n2p[1]);
-          f = unpack_bf16x2(w.y); n2p[2] = fmaf(f.x, f.x, n2p[2]); n2p[3] = fmaf(f.y, f.y, n2p[3]);
-          f = unpack_bf16x2(w.z); n2p[4] = fmaf(f.x, f.x, n2p[4]); n2p[5] = fmaf(f.y, f.y, n2p[5]);
-          f = unpack_bf16x2(w.w); n2p[6] = fmaf(f.x, f.x, n2p[6]); n2p[7] = fmaf(f.y, f.y, n2p[7]);
-        }
+      for (int uu = 0; uu < UN; ++uu) {
+        const int j = (Gm::kHalves == 2) ? hf : 0;
+        const int u = (Gm::kHalves == 2) ? uu : 4 * hf + uu;
+        const uint4 w = *reinterpret_cast<const uint4*>(k_s + j * Gm::kKBox + row * 128 + ((u ^ (row & 7)) << 4));
+        float2 f;
+        f = unpack_bf16x2(w.x); n2p[0] = fmaf(f.x, f.x, n2p[0]); n2p[1] = fmaf(f.y, f.y, n2p[1]);
+        f = unpack_bf16x2(w.y); n2p[2] = fmaf(f.x, f.x, n2p[2]); n2p[3] = fmaf(f.y, f.y, n2p[3]);
+        f = unpack_bf16x2(w.z); n2p[0] = fmaf(f.x, f.x, n2p[0]); n2p[1] = fmaf(f.y, f.y, n2p[1]);
+        f = unpack_bf16x2(w.w); n2p[2] = fmaf(f.x, f.x, n2p[2]); n2p[3] = fmaf(f.y, f.y, n2p[3]);
       }
-      const float n2 = ((n2p[0] + n2p[1]) + (n2p[2] + n2p[3])) + ((n2p[4] + n2p[5]) + (n2p[6] + n2p[7]));
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
-#pragma unroll
-      for (int hh = 0; hh < 8; ++hh)
-        if (hh == h) inv[hh] = 1.0f / fmaxf(sqrtf(n2), kEps);
+      n2s[(((lt & 1) * 8 + h) * 2 + hf) * kScanM + row] = (n2p[0] + n2p[1]) + (n2p[2] + n2p[3]);
       if (h != n_r - 1) continue;
 
       // ---- epilogue of tile lt: head mean of cosines, per-document max ----
       const int tile = t_begin + lt;
       const int buf = lt & 1;
+      named_bar_sync(1 + q4, 64);  // both halves of this lane quarter have written their norms
+      const float* nb2 = n2s + (size_t)(lt & 1) * 8 * 2 * kScanM;
       mbar_wait(&tfull[buf], (lt >> 1) & 1);
       tc_fence_after();
-      float acc[NQ];
+      float acc[QH];
 #pragma unroll
-      for (int b = 0; b < NQ; ++b) acc[b] = 0.f;
-      const uint32_t t_row = tmem_base + ((uint32_t)(32 * q4) << 16) + buf * buf_cols;
+      for (int b = 0; b < QH; ++b) acc[b] = 0.f;
+      const bool any_q = hf * QH < p.q_count;
+      const uint32_t t_row = tmem_base + ((uint32_t)(32 * q4) << 16) + buf * buf_cols + hf * QH;
 #pragma unroll
       for (int hh = 0; hh < 8; ++hh) {
-        if (hh < n_r) {
-          if constexpr (NQ == 32) {
-            float v[32];
-            tmem_ld32(t_row + hh * NQ, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int b = 0; b < 32; ++b) acc[b] = fmaf(v[b], inv[hh], acc[b]);
-          } else {
+        if (hh < n_r && any_q) {
+          const float n2 = nb2[(hh * 2 + 0) * kScanM + row] + nb2[(hh * 2 + 1) * kScanM + row];
+          const float inv = 1.0f / fmaxf(sqrtf(n2), kEps);
+          if constexpr (QH == 16) {
             float v[16];
             tmem_ld16(t_row + hh * NQ, v);
             tmem_ld_wait();
 #pragma unroll
-            for (int b = 0; b < 16; ++b) acc[b] = fmaf(v[b], inv[hh], acc[b]);
+            for (int b = 0; b < 16; ++b) acc[b] = fmaf(v[b], inv, acc[b]);
+          } else {
+            float v[8];
+            tmem_ld8(t_row + hh * NQ, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int b = 0; b < 8; ++b) acc[b] = fmaf(v[b], inv, acc[b]);
           }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
+      if (!any_q) continue;
 
-      // document of this row: search chunk_off from the warp's cursor
+      // documents of this warp's 32 rows: a warp-wide 32-ary search for the first row's
+      // document, then one lookahead of 32 document boundaries (32 consecutive rows cross at
+      // most 31 of them)
       const int j = tile * kScanM + row;
+      const int j0 = tile * kScanM + 32 * q4;
       int doc = -1;
-      if (j < p.n_chunks) {
-        int lo = cur, hi = p.n_docs - 1;
-        while (lo < hi) {
-          const int mid = (lo + hi + 1) >> 1;
-          if (__ldg(&p.chunk_off[mid]) <= j) lo = mid; else hi = mid - 1;
+      if (j0 < p.n_chunks) {
+        int lo = cur, hi = p.n_docs;  // answer in [lo, hi): largest d with chunk_off[d] <= j0
+        while (hi - lo > 1) {
+          const int step = (hi - lo + 31) >> 5;
+          const int probe = lo + lane * step;
+          const bool ok = probe < hi && __ldg(&p.chunk_off[probe]) <= j0;
+          const unsigned m = __ballot_sync(0xffffffffu, ok);
+          const int L = 31 - __clz(m);  // lane 0 always qualifies (chunk_off[lo] <= j0)
+          lo = lo + L * step;
+          hi = min(hi, lo + step);
         }
-        doc = lo;
+        const int d0 = lo;
+        const int bi = d0 + 1 + lane;
+        const int bnd = bi <= p.n_docs ? __ldg(&p.chunk_off[bi]) : 0x7fffffff;
+#pragma unroll 4
+        for (int r = 0; r < 32; ++r) {
+          const unsigned m = __ballot_sync(0xffffffffu, bnd <= j0 + r);
+          if (lane == r) doc = d0 + __popc(m);
+        }
+        if (j >= p.n_chunks) doc = -1;
+        cur = d0;
       }
-      const int last = __shfl_sync(0xffffffffu, doc, 31);
-      if (last >= 0) cur = last;
       const int prev = __shfl_up_sync(0xffffffffu, doc, 1);
       const bool head = (lane == 0) || (prev != doc);
       // the document pattern is the same for every query: which shuffle partners share my document
@@ -387,9 +408,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         if (lane + (1 << e) < 32 && od == doc) same |= 1u << e;
       }
 #pragma unroll
-      for (int b = 0; b < NQ; ++b) {
+      for (int bb = 0; bb < QH; ++bb) {
+        const int b = hf * QH + bb;
         if (b >= p.q_count) continue;  // warp-uniform
-        const float sc = acc[b] * p.inv_nr;
+        const float sc = acc[bb] * p.inv_nr;
         if (MEAN) {
           if (doc >= 0) p.chunk_s[(size_t)(p.q_base + b) * p.n_chunks + j] = sc;
         } else {
@@ -591,7 +613,8 @@ template <int DR, int NQ, bool MEAN>
 cudaError_t launch_scan_t(const CUtensorMap& kmap, const CUtensorMap& qmap, const ScanParams& p, int grid,
                           cudaStream_t s) {
   auto kern = scan_kernel<DR, NQ, MEAN>;
-  const size_t smem = 1024 + (size_t)kScanStages * ScanGeom<DR, NQ>::kStageBytes + (2 * kScanStages + 4) * 8 + 16;
+  const size_t smem = 1024 + (size_t)kScanStages * ScanGeom<DR, NQ>::kStageBytes + 2 * 8 * 2 * kScanM * sizeof(float) +
+                      (2 * kScanStages + 4) * 8 + 16;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(grid), dim3(kScanThreads), smem, s, kmap, qmap, p);

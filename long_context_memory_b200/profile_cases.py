@@ -11,8 +11,8 @@ Cases
   route1m    1M-token memory, B = 1   (K̄^R 33 MB)
   route16m   16M-token memory, B = 32 (K̄^R 520 MB)
   route100m  100M-token memory, B = 1 (K̄^R 3.2 GB); --batch to change B
-  attend1m   sparse attention, 1M-token memory, B = 1, 4K local tokens
-  attend16m  sparse attention, 16M-token memory, B = 32, 8K local tokens
+  attend1m   sparse attention, 1M-token memory, B = 1, 4K local tokens (rotated key cache)
+  attend16m  sparse attention, 16M-token memory, B = 32, 8K local tokens (rotated key cache)
   encode     offline encoding of --tokens tokens (default 1M), hidden 2560
 """
 from __future__ import annotations
@@ -92,7 +92,7 @@ class RouteCase:
 
 
 class AttendCase:
-    def __init__(self, T, B, median, t_loc, seed, device, k=16, dims=W.QWEN3_4B_DIMS):
+    def __init__(self, T, B, median, t_loc, seed, device, k=16, dims=W.QWEN3_4B_DIMS, rotated=True):
         import torch
 
         import long_context_memory_b200 as msa
@@ -113,7 +113,13 @@ class AttendCase:
         sel = np.stack([rng.permutation(n_docs)[:k] for _ in range(B)]).astype(np.int32)
         self.topk = torch.from_numpy(sel).to(device)
         self.pos = k
-        self.rope = msa.rope_cache_build(dims, t_loc, self.pos, device=device)
+        self.rotated = rotated
+        if rotated:  # the local key cache holds keys rotated at their global positions
+            msa.rope_rows(dims, self.K_loc.view(B * t_loc, dims.n_kv, dims.head_dim),
+                          (self.pos + torch.arange(t_loc, dtype=torch.int32, device=device)).repeat(B))
+            self.rope = None
+        else:
+            self.rope = msa.rope_cache_build(dims, t_loc, self.pos, device=device)
         self.out = torch.empty((B, dims.n_q, dims.head_dim), dtype=torch.bfloat16, device=device)
         self.ws = torch.empty(msa.attend_workspace_size(dims, B, k, t_loc, self.pos) + 256, dtype=torch.uint8,
                               device=device)
@@ -122,7 +128,8 @@ class AttendCase:
 
     def run(self):
         self.msa.sparse_attend(self.d, self.q, self.K_bar, self.V_bar, self.chunk_off, self.topk, self.K_loc,
-                               self.V_loc, self.loc_len, self.pos, out=self.out, ws=self.ws, rope_cache=self.rope)
+                               self.V_loc, self.loc_len, self.pos, out=self.out, ws=self.ws, rope_cache=self.rope,
+                               k_loc_rotated=self.rotated)
 
 
 class EncodeCase:

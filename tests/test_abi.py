@@ -108,7 +108,7 @@ def _attend(msa, dims, B=1, k=2, n_docs=4, n_chunks=8, t_loc=16, pos=2, scale=0.
     if ws_bytes is None:
         ws_bytes = need
     return msa.lib.msa_sparse_attend(ctypes.byref(dd), q, B, FAKE, FAKE, FAKE, n_docs, n_chunks, FAKE, k, FAKE, FAKE,
-                                     FAKE, t_loc, pos, None, scale, FAKE, 0x100000, ws_bytes, None)
+                                     FAKE, t_loc, pos, None, 0, scale, FAKE, 0x100000, ws_bytes, None)
 
 
 def test_attend_validation(msa):
@@ -116,6 +116,7 @@ def test_attend_validation(msa):
     assert _attend(msa, _dims(head_dim=96)) == 2
     assert _attend(msa, _dims(n_q=6, n_kv=4)) == 1          # n_q not a multiple of n_kv
     assert _attend(msa, _dims(n_q=64, n_kv=2)) == 2         # GQA group > 16
+    assert _attend(msa, _dims(n_q=16, n_kv=16)) == 2        # more than 8 KV heads
     assert _attend(msa, ok, k=5) == 1                       # k > n_docs
     assert _attend(msa, ok, pos=-1) == 1
     assert _attend(msa, ok, scale=float("nan")) == 1
@@ -128,6 +129,14 @@ def test_encode_validation(msa):
     r = msa.lib.msa_encode_memory(ctypes.byref(dd), FAKE, 1000, FAKE, 3, FAKE, 20, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
                                   None, 0, None)
     assert r == 2
+
+
+def test_topk_merge_validation(msa):
+    lib = msa.lib
+    assert lib.msa_topk_merge(FAKE, FAKE, 1, 8, 9, FAKE, FAKE, None) == 1      # k > n_cand
+    assert lib.msa_topk_merge(FAKE, FAKE, 0, 8, 4, FAKE, FAKE, None) == 1      # B < 1
+    assert lib.msa_topk_merge(FAKE, FAKE + 4, 1, 8, 4, FAKE, FAKE, None) == 1  # misaligned
+    assert lib.msa_topk_merge(FAKE, FAKE, 1, 30000, 4, FAKE, FAKE, None) == 1  # too many candidates
 
 
 def test_workspace_sizes_grow_with_problem(msa):

@@ -135,3 +135,118 @@ def test_attend_mem16m_batch32_sampled(msa, cuda_device):
     for b in [0, 7, 31]:
         sub = {kk: (v[b:b + 1] if kk in ("q", "K_loc", "V_loc", "loc_len", "topk") else v) for kk, v in case.items()}
         check_attention(out[b:b + 1], _oracle(sub, m["pos_offset"], d.rope_base), where=f"b={b}")
+
+
+def _rotated_cache(msa, dims, c, device, pos_offset):
+    """The local keys rotated in place on the GPU at pos_offset + j (every row of the cache)."""
+    import torch
+
+    B, T, n_kv, D = c["K_loc"].shape
+    K = _dev(c["K_loc"], device).reshape(B * T, n_kv, D).clone()
+    pos = (pos_offset + torch.arange(T, dtype=torch.int32, device=device)).repeat(B)
+    msa.rope_rows(dims, K, pos)
+    return K.reshape(B, T, n_kv, D)
+
+
+def test_rope_rows_matches_oracle_rotation(msa, cuda_device):
+    import torch
+
+    from helpers import torch_bits
+
+    rng = np.random.default_rng(12)
+    for D, base in [(128, 1e6), (64, 1e4)]:
+        x = W.normal_bf16(rng, (300, 3, D))
+        pos = rng.integers(0, 200000, size=300).astype(np.int32)
+        dims = W.Dims(hidden=256, n_q=3, n_kv=3, head_dim=D, n_r=4, d_r=64, rope_base=base)
+        xd = _dev(x, cuda_device)
+        msa.rope_rows(dims, xd, torch.from_numpy(pos).to(cuda_device))
+        torch.cuda.synchronize()
+        got = O.bf16_to_f64(torch_bits(xd))
+        want = O.rope(O.bf16_to_f64(x), pos[:, None], base)
+        # one bf16 rounding of the rotated value
+        assert np.all(np.abs(got - want) <= 2.0 ** -8 * np.abs(want) + 1e-6)
+
+
+@pytest.mark.parametrize("D,n_q,n_kv", [(128, 32, 8), (64, 8, 2), (128, 16, 1)])
+def test_attend_rotated_cache_mode(msa, cuda_device, D, n_q, n_kv):
+    import torch
+
+    c = _case(40 + D + n_kv, 3, n_q, n_kv, D, n_docs=30, k=5, t_loc=300)
+    dims = W.Dims(hidden=256, n_q=n_q, n_kv=n_kv, head_dim=D, n_r=4, d_r=64, rope_base=1e6)
+    Krot = _rotated_cache(msa, dims, c, cuda_device, 5)
+    co, C = msa.chunk_offsets(c["doc_off"])
+    out = msa.sparse_attend(dims, _dev(c["q"], cuda_device), _dev(c["K_bar"], cuda_device),
+                            _dev(c["V_bar"], cuda_device), torch.from_numpy(co).to(cuda_device),
+                            torch.from_numpy(c["topk"].astype(np.int32)).to(cuda_device), Krot,
+                            _dev(c["V_loc"], cuda_device), torch.from_numpy(c["loc_len"].astype(np.int32)).to(cuda_device),
+                            5, k_loc_rotated=True)
+    torch.cuda.synchronize()
+    assert msa.check_device_errors() == 0
+    check_attention(out.float().cpu().numpy(), _oracle(c, 5, 1e6), where=f"rotated D={D}")
+
+
+def test_attend_rotated_cache_mem16m_sampled(msa, cuda_device):
+    import torch
+
+    m = W.mem16m_config()
+    d = m["dims"]
+    co, *_ = O.chunk_layout(m["doc_off"])
+    case = dict(doc_off=m["doc_off"], chunk_off=co, q=m["q"], K_bar=m["K_bar"], V_bar=m["V_bar"], K_loc=m["K_loc"],
+                V_loc=m["V_loc"], loc_len=m["loc_len"], topk=m["planted_docs"])
+    Krot = _rotated_cache(msa, d, case, cuda_device, m["pos_offset"])
+    out = msa.sparse_attend(d, _dev(m["q"], cuda_device), _dev(m["K_bar"], cuda_device), _dev(m["V_bar"], cuda_device),
+                            torch.from_numpy(co.astype(np.int32)).to(cuda_device),
+                            torch.from_numpy(m["planted_docs"].astype(np.int32)).to(cuda_device), Krot,
+                            _dev(m["V_loc"], cuda_device), torch.from_numpy(m["loc_len"]).to(cuda_device),
+                            m["pos_offset"], k_loc_rotated=True).float().cpu().numpy()
+    for b in [0, 13, 31]:
+        sub = {kk: (v[b:b + 1] if kk in ("q", "K_loc", "V_loc", "loc_len", "topk") else v) for kk, v in case.items()}
+        check_attention(out[b:b + 1], _oracle(sub, m["pos_offset"], d.rope_base), where=f"b={b}")
+
+
+@pytest.mark.parametrize("B,D,n_kv", [(1, 128, 8), (4, 64, 2)])
+def test_host_tier_gather_then_attend(msa, cuda_device, B, D, n_kv):
+    import torch
+
+    from helpers import torch_bits
+
+    n_q = 4 * n_kv
+    c = _case(70 + B, B, n_q, n_kv, D, n_docs=50, k=6, t_loc=100)
+    dims = W.Dims(hidden=256, n_q=n_q, n_kv=n_kv, head_dim=D, n_r=4, d_r=64, rope_base=1e6)
+    co, C = msa.chunk_offsets(c["doc_off"])
+    dev = cuda_device
+    Kh = W.to_torch(c["K_bar"]).pin_memory()
+    Vh = W.to_torch(c["V_bar"]).pin_memory()
+    topk = torch.from_numpy(c["topk"].astype(np.int32)).to(dev)
+    chunk_off = torch.from_numpy(co).to(dev)
+    Ks, Vs, soff, sidx = msa.gather_kv(dims, Kh, Vh, chunk_off, topk, capacity_chunks=C)
+    torch.cuda.synchronize()
+    assert msa.check_device_errors() == 0
+    # the staging holds exactly the selected documents' rows, query by query in top-k order
+    so = soff.cpu().numpy()
+    assert so[0] == 0
+    assert sidx.cpu().tolist() == [[b * 6 + r for r in range(6)] for b in range(B)]
+    Ksb = torch_bits(Ks)
+    for b in range(B):
+        for r in range(6):
+            doc = c["topk"][b, r]
+            i = b * 6 + r
+            assert so[i + 1] - so[i] == co[doc + 1] - co[doc]
+            assert np.array_equal(Ksb[so[i]:so[i + 1]], c["K_bar"][co[doc]:co[doc + 1]])
+    out = msa.sparse_attend(dims, _dev(c["q"], dev), Ks, Vs, soff, sidx, _dev(c["K_loc"], dev), _dev(c["V_loc"], dev),
+                            torch.from_numpy(c["loc_len"].astype(np.int32)).to(dev), 6)
+    torch.cuda.synchronize()
+    check_attention(out.float().cpu().numpy(), _oracle(c, 6, 1e6), where="host tier")
+
+
+def test_host_tier_rejects_pageable_memory(msa, cuda_device):
+    import torch
+
+    dims = W.Dims(hidden=256, n_q=8, n_kv=2, head_dim=64, n_r=4, d_r=64)
+    K = torch.zeros((10, 2, 64), dtype=torch.bfloat16)          # pageable, not pinned
+    V = torch.zeros((10, 2, 64), dtype=torch.bfloat16)
+    co = torch.tensor([0, 5, 10], dtype=torch.int32, device=cuda_device)
+    tk = torch.tensor([[0]], dtype=torch.int32, device=cuda_device)
+    with pytest.raises(msa.MSAError) as e:
+        msa.gather_kv(dims, K, V, co, tk, capacity_chunks=10)
+    assert e.value.code == 1 and "pinned" in str(e.value)
