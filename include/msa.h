@@ -107,7 +107,8 @@ msa_status msa_chunk_offsets(const int64_t* doc_off_host, int32_t n_docs, int32_
  *   W_K, W_V [hidden, n_kv * head_dim] bf16; W_KR [hidden, n_r * d_r] bf16.
  *   K_bar, V_bar [C, n_kv, head_dim] bf16 out: chunk means of RoPE(H W_K) at
  *            document-relative positions and of H W_V.
- *   KR_bar   [C, n_r, d_r] bf16 out: chunk means of H W^KR.
+ *   KR_bar   bf16 out: chunk means of H W^KR, [C, n_r, d_r] (kr_layout 0) or
+ *            head-major [n_r, C, d_r] (kr_layout 1, the layout the scan reads best).
  * Requirements: hidden % 64 == 0; n_kv * head_dim and n_r * d_r multiples of
  * 128; chunk == 64; T < 2^31 - 64.  Rounding: fp32 accumulation, outputs rounded to bf16.
  * ------------------------------------------------------------------------- */
@@ -115,7 +116,7 @@ size_t msa_encode_workspace_size(const msa_dims* dims, int64_t T, int32_t n_docs
 msa_status msa_encode_memory(const msa_dims* dims, const void* H, int64_t T, const int64_t* doc_off,
                              int32_t n_docs, const int32_t* chunk_off, int32_t n_chunks, const void* W_K,
                              const void* W_V, const void* W_KR, void* K_bar, void* V_bar, void* KR_bar,
-                             void* ws, size_t ws_bytes, void* stream);
+                             int32_t kr_layout, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Stage 2 - online routing and top-k.
@@ -125,7 +126,9 @@ msa_status msa_encode_memory(const msa_dims* dims, const void* H, int64_t T, con
  *   Hq       [B, hidden] bf16 query hidden states, or, when W_QR == NULL,
  *            [B, n_r * d_r] bf16 router queries Q^R given directly.
  *   W_QR     [hidden, n_r * d_r] bf16 or NULL.
- *   KR_bar   [n_chunks, n_r, d_r] bf16 pooled router keys.
+ *   KR_bar   pooled router keys, bf16: [n_chunks, n_r, d_r] for kr_layout 0, or
+ *            head-major [n_r, n_chunks, d_r] for kr_layout 1 (each head's keys contiguous:
+ *            the scan then streams whole 32 KB slices instead of 256-byte pieces).
  *   chunk_off[n_docs + 1] device int32 chunk offsets of the documents.
  *   doc_scores [B, n_docs] fp32 out, optional (NULL = not written).
  *   topk_idx [B, k] int32 out: document ids, descending score, ties to the
@@ -141,7 +144,7 @@ size_t msa_route_workspace_size(const msa_dims* dims, int32_t B, int32_t n_docs,
                                 int32_t k, msa_doc_agg agg);
 msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR, int32_t B,
                           const void* KR_bar, const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks,
-                          int32_t k, msa_doc_agg agg, float* doc_scores, int32_t* topk_idx,
+                          int32_t k, msa_doc_agg agg, int32_t kr_layout, float* doc_scores, int32_t* topk_idx,
                           float* topk_score, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------

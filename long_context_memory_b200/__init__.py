@@ -63,9 +63,9 @@ def _load():
         "msa_check_device_errors": (I32, [ctypes.POINTER(ctypes.c_uint32)]),
         "msa_chunk_offsets": (I32, [P, I32, I32, P, ctypes.POINTER(I32)]),
         "msa_encode_workspace_size": (SZ, [DP, I64, I32, I32]),
-        "msa_encode_memory": (I32, [DP, P, I64, P, I32, P, I32, P, P, P, P, P, P, P, SZ, P]),
+        "msa_encode_memory": (I32, [DP, P, I64, P, I32, P, I32, P, P, P, P, P, P, I32, P, SZ, P]),
         "msa_route_workspace_size": (SZ, [DP, I32, I32, I32, I32, I32]),
-        "msa_route_topk": (I32, [DP, P, P, I32, P, P, I32, I32, I32, I32, P, P, P, P, SZ, P]),
+        "msa_route_topk": (I32, [DP, P, P, I32, P, P, I32, I32, I32, I32, I32, P, P, P, P, SZ, P]),
         "msa_attend_workspace_size": (SZ, [DP, I32, I32, I32, I32]),
         "msa_sparse_attend": (I32, [DP, P, I32, P, P, P, I32, I32, P, I32, P, P, P, I32, I32, P, I32, F, P, P, SZ, P]),
         "msa_rope_rows": (I32, [DP, P, I32, I32, P, P]),
@@ -161,22 +161,26 @@ def encode_workspace_size(dims, T: int, n_docs: int, n_chunks: int) -> int:
     return int(lib.msa_encode_workspace_size(ctypes.byref(Dims.of(dims)), T, n_docs, n_chunks))
 
 
-def encode_memory(dims, H, doc_off, chunk_off, n_chunks: int, W_K, W_V, W_KR, out=None, ws=None, stream=None):
-    """Pooled (K̄, V̄, K̄^R) of a corpus; all tensors on the same CUDA device."""
+def encode_memory(dims, H, doc_off, chunk_off, n_chunks: int, W_K, W_V, W_KR, out=None, ws=None, stream=None,
+                  kr_head_major: bool = False):
+    """Pooled (K̄, V̄, K̄^R) of a corpus; all tensors on the same CUDA device.
+
+    ``kr_head_major`` stores K̄^R as [n_r, C, d_r] (the layout the scan reads best)."""
     import torch
 
     dd = Dims.of(dims)
     T, n_docs = H.shape[0], doc_off.numel() - 1
     dev = H.device
     if out is None:
+        kr_shape = (dims.n_r, n_chunks, dims.d_r) if kr_head_major else (n_chunks, dims.n_r, dims.d_r)
         out = (torch.empty((n_chunks, dims.n_kv, dims.head_dim), dtype=torch.bfloat16, device=dev),
                torch.empty((n_chunks, dims.n_kv, dims.head_dim), dtype=torch.bfloat16, device=dev),
-               torch.empty((n_chunks, dims.n_r, dims.d_r), dtype=torch.bfloat16, device=dev))
+               torch.empty(kr_shape, dtype=torch.bfloat16, device=dev))
     nbytes = encode_workspace_size(dims, T, n_docs, n_chunks)
     ws = _workspace(nbytes, dev, ws)
     _check(lib.msa_encode_memory(ctypes.byref(dd), _ptr(H), T, _ptr(doc_off), n_docs, _ptr(chunk_off), n_chunks,
                                  _ptr(W_K), _ptr(W_V), _ptr(W_KR), _ptr(out[0]), _ptr(out[1]), _ptr(out[2]),
-                                 _aligned_ptr(ws), nbytes, _stream(stream)))
+                                 int(bool(kr_head_major)), _aligned_ptr(ws), nbytes, _stream(stream)))
     return out
 
 
@@ -188,17 +192,18 @@ def route_workspace_size(dims, B: int, n_docs: int, n_chunks: int, k: int, agg: 
 
 
 def route_topk(dims, Hq, W_QR, KR_bar, chunk_off, k: int, agg: int = AGG_MAX, want_doc_scores: bool = False,
-               out=None, ws=None, stream=None):
+               out=None, ws=None, stream=None, kr_head_major: bool = False):
     """Top-k documents per query.  Returns (topk_idx [B,k] int32, topk_score [B,k] fp32, doc_scores|None).
 
     ``W_QR=None`` means ``Hq`` already holds the router queries Q^R [B, n_r*d_r].
+    ``kr_head_major``: KR_bar is [n_r, C, d_r] instead of [C, n_r, d_r].
     """
     import torch
 
     dd = Dims.of(dims)
     B = Hq.shape[0]
     n_docs = chunk_off.numel() - 1
-    n_chunks = KR_bar.shape[0]
+    n_chunks = KR_bar.shape[1] if kr_head_major else KR_bar.shape[0]
     dev = KR_bar.device
     if out is None:
         out = (torch.empty((B, k), dtype=torch.int32, device=dev), torch.empty((B, k), dtype=torch.float32, device=dev),
@@ -206,7 +211,7 @@ def route_topk(dims, Hq, W_QR, KR_bar, chunk_off, k: int, agg: int = AGG_MAX, wa
     nbytes = route_workspace_size(dims, B, n_docs, n_chunks, k, agg)
     ws = _workspace(nbytes, dev, ws)
     _check(lib.msa_route_topk(ctypes.byref(dd), _ptr(Hq), _ptr(W_QR), B, _ptr(KR_bar), _ptr(chunk_off), n_docs,
-                              n_chunks, k, agg, _ptr(out[2]), _ptr(out[0]), _ptr(out[1]), _aligned_ptr(ws), nbytes,
+                              n_chunks, k, agg, int(bool(kr_head_major)), _ptr(out[2]), _ptr(out[0]), _ptr(out[1]), _aligned_ptr(ws), nbytes,
                               _stream(stream)))
     return out
 

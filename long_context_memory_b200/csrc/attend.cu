@@ -44,37 +44,15 @@ constexpr int kMaxK = 256;
 constexpr int kMaxSplits = 1024;
 constexpr float kLog2e = 1.4426950408889634f;
 
-// cos/sin of (pos_offset + j) * theta_i, theta_i = base^(-2i/D), for local
-// positions j.  One block per 64 positions: the block's base angle
-// (pos_offset + 64 jh) theta_i is reduced and evaluated in fp64, the in-block
-// offset jl * theta_i (< 64 rad) in fp32, and the two are combined by the
-// angle-addition identities.
+// cos/sin of (pos_offset + j) * theta_i, theta_i = base^(-2i/D), for local positions j
 __global__ void __launch_bounds__(256) rope_table_kernel(float2* __restrict__ tab, int t_loc_max, int half,
-                                                         int pos_offset, double log_base, int head_dim) {
-  __shared__ float2 coarse[128];
-  __shared__ float theta_f[128];
+                                                         int pos_offset, const RopeTurns turns) {
   pdl_launch_dependents();
   pdl_wait();
-  const int jh = blockIdx.x;
-  for (int i = threadIdx.x; i < half; i += blockDim.x) {
-    const double theta = exp(-2.0 * (double)i / (double)head_dim * log_base);
-    double a = (double)(pos_offset + 64 * jh) * theta;
-    const double two_pi = 6.283185307179586476925286766559;
-    a -= two_pi * rint(a / two_pi);
-    double sv, cv;
-    sincos(a, &sv, &cv);
-    coarse[i] = make_float2((float)cv, (float)sv);
-    theta_f[i] = (float)theta;
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < 64 * half; e += blockDim.x) {
-    const int jl = e / half, i = e % half;
-    const int j = 64 * jh + jl;
-    if (j >= t_loc_max) break;
-    float sf, cf;
-    sincosf((float)jl * theta_f[i], &sf, &cf);
-    const float2 cb = coarse[i];
-    tab[(size_t)j * half + i] = make_float2(cb.x * cf - cb.y * sf, cb.y * cf + cb.x * sf);
+  const int64_t n = (int64_t)t_loc_max * half;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const int j = (int)(e / half), i = (int)(e % half);
+    tab[e] = rope_cos_sin(turns, i, (int64_t)pos_offset + j);
   }
 }
 
@@ -92,7 +70,7 @@ struct AttnParams {
   float* part_o;
   int n_q, n_kv, k, n_docs, t_loc_max, pos_offset, n_splits, n_stages;
   float scale_log2;  // softmax scale * log2(e)
-  double log_base;
+  RopeTurns turns;   // RoPE frequencies as 64-bit fractions of a turn
 };
 
 // Shared memory of one CTA (dynamic size, n_stages stages):
@@ -252,14 +230,7 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
 
   // ---- query fragments of this warp's GQA group: rotate to pos_offset + L - 1, scale, bf16 ----
   const int n_compute = 32 * n_kv;
-  for (int i = tid; i < D / 2; i += n_compute) {
-    double a = (double)(p.pos_offset + L - 1) * exp(-2.0 * (double)i / (double)D * p.log_base);
-    const double two_pi = 6.283185307179586476925286766559;
-    a -= two_pi * rint(a / two_pi);
-    double sv, cv;
-    sincos(a, &sv, &cv);
-    qcs[i] = make_float2((float)cv, (float)sv);
-  }
+  for (int i = tid; i < D / 2; i += n_compute) qcs[i] = rope_cos_sin(p.turns, i, (int64_t)p.pos_offset + L - 1);
   named_bar_sync(1, n_compute);
   const int g = lane >> 2, c = lane & 3;
   uint32_t qa[KS][4];
@@ -437,13 +408,16 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
   }
 }
 
-// log-sum-exp merge of the split partials of one (query, q head); splits are read in parallel
+// log-sum-exp merge of the split partials of one (query, q head).  Warp w sums the splits
+// s = w (mod 8); lane l holds D/32 consecutive dims; the warps' sums meet in shared memory.
 template <int D>
-__global__ void __launch_bounds__(128) attn_combine_kernel(const float* __restrict__ part_ml,
+__global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restrict__ part_ml,
                                                            const float* __restrict__ part_o, int n_splits,
                                                            __nv_bfloat16* __restrict__ out) {
+  constexpr int PER = D / 32;
   __shared__ float w_s[kMaxSplits];
-  __shared__ float red[2][4];
+  __shared__ float red[2][8];
+  __shared__ float osum[8][D];
   pdl_launch_dependents();
   pdl_wait();
   const size_t qh = (size_t)blockIdx.y * gridDim.x + blockIdx.x;  // b * n_q + head
@@ -455,7 +429,9 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float* __restri
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if (lane == 0) red[0][warp] = m;
   __syncthreads();
-  float M = fmaxf(fmaxf(red[0][0], red[0][1]), fmaxf(red[0][2], red[0][3]));
+  float M = red[0][0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) M = fmaxf(M, red[0][w]);
   const float Mu = (M == -INFINITY) ? 0.f : M;
   float l = 0.f;
   for (int s = tid; s < n_splits; s += blockDim.x) {
@@ -467,19 +443,31 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float* __restri
   for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
   if (lane == 0) red[1][warp] = l;
   __syncthreads();
-  const float Ls = (red[1][0] + red[1][1]) + (red[1][2] + red[1][3]);
-  const float* po = part_o + qh * n_splits * D;
-  for (int dim = tid; dim < D; dim += blockDim.x) {
-    float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
-    int s = 0;
-    for (; s + 4 <= n_splits; s += 4) {
-      o0 += w_s[s] * po[(size_t)s * D + dim];
-      o1 += w_s[s + 1] * po[(size_t)(s + 1) * D + dim];
-      o2 += w_s[s + 2] * po[(size_t)(s + 2) * D + dim];
-      o3 += w_s[s + 3] * po[(size_t)(s + 3) * D + dim];
+  float Ls = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) Ls += red[1][w];
+  const float* po = part_o + qh * n_splits * D + lane * PER;
+  float acc[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+#pragma unroll 4
+  for (int s = warp; s < n_splits; s += 8) {
+    const float w = w_s[s];
+    if constexpr (PER == 4) {
+      const float4 v = *reinterpret_cast<const float4*>(po + (size_t)s * D);
+      acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
+    } else {
+      const float2 v = *reinterpret_cast<const float2*>(po + (size_t)s * D);
+      acc[0] += w * v.x; acc[1] += w * v.y;
     }
-    for (; s < n_splits; ++s) o0 += w_s[s] * po[(size_t)s * D + dim];
-    const float o = (o0 + o1) + (o2 + o3);
+  }
+#pragma unroll
+  for (int e = 0; e < PER; ++e) osum[warp][lane * PER + e] = acc[e];
+  __syncthreads();
+  for (int dim = tid; dim < D; dim += blockDim.x) {
+    float o = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) o += osum[w][dim];
     out[qh * D + dim] = __float2bfloat16_rn(Ls > 0.f ? o / Ls : 0.f);
   }
 }
@@ -496,7 +484,7 @@ int stages_that_fit(int n_kv, int n_q, int D, bool table) {
 // rotate rows of x [rows, heads, D] in place: pair (i, i + D/2) of row r by pos[r] * theta_i
 template <int D>
 __global__ void __launch_bounds__(256) rope_rows_kernel(__nv_bfloat16* __restrict__ x, int rows, int heads,
-                                                        const int32_t* __restrict__ pos, double log_base) {
+                                                        const int32_t* __restrict__ pos, const RopeTurns turns) {
   pdl_launch_dependents();
   pdl_wait();
   const int64_t n = (int64_t)rows * heads * (D / 2);
@@ -504,16 +492,11 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(__nv_bfloat16* __restric
     const int i = (int)(e % (D / 2));
     const int64_t rh = e / (D / 2);
     const int r = (int)(rh / heads);
-    double a = (double)pos[r] * exp(-2.0 * (double)i / (double)D * log_base);
-    const double two_pi = 6.283185307179586476925286766559;
-    a -= two_pi * rint(a / two_pi);
-    double sv, cv;
-    sincos(a, &sv, &cv);
-    const float cs = (float)cv, sn = (float)sv;
+    const float2 cs = rope_cos_sin(turns, i, (int64_t)pos[r]);
     __nv_bfloat16* v = x + rh * D;
     const float x1 = __bfloat162float(v[i]), x2 = __bfloat162float(v[i + D / 2]);
-    v[i] = __float2bfloat16_rn(x1 * cs - x2 * sn);
-    v[i + D / 2] = __float2bfloat16_rn(x2 * cs + x1 * sn);
+    v[i] = __float2bfloat16_rn(x1 * cs.x - x2 * cs.y);
+    v[i + D / 2] = __float2bfloat16_rn(x2 * cs.x + x1 * cs.y);
   }
 }
 
@@ -673,8 +656,10 @@ msa_status rope_cache_build(const msa_dims& d, int t_loc_max, int pos_offset, fl
   if (t_loc_max <= 0) return MSA_OK;
   const int D = d.head_dim;
   TraceScope ts(kKRopeTable, s);
-  MSA_CUDA_CHECK(launch_pdl(rope_table_kernel, dim3((t_loc_max + 63) / 64), dim3(256), 0, s, tab, t_loc_max, D / 2,
-                            pos_offset, std::log((double)d.rope_base), D));
+  RopeTurns turns;
+  rope_turns(d, turns.f);
+  const int blocks = (int)std::min<int64_t>(((int64_t)t_loc_max * (D / 2) + 255) / 256, 8 * sm_count());
+  MSA_CUDA_CHECK(launch_pdl(rope_table_kernel, dim3(blocks), dim3(256), 0, s, tab, t_loc_max, D / 2, pos_offset, turns));
   return MSA_OK;
 }
 
@@ -682,13 +667,14 @@ msa_status rope_rows_launch(const msa_dims& d, void* x, int rows, int heads, con
   TraceScope ts(kKRopeRows, s);
   const int64_t n = (int64_t)rows * heads * (d.head_dim / 2);
   const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 8 * sm_count()));
-  const double lb = std::log((double)d.rope_base);
+  RopeTurns turns;
+  rope_turns(d, turns.f);
   if (d.head_dim == 128)
     MSA_CUDA_CHECK(launch_pdl(rope_rows_kernel<128>, dim3(blocks), dim3(256), 0, s, static_cast<__nv_bfloat16*>(x),
-                              rows, heads, pos, lb));
+                              rows, heads, pos, turns));
   else
     MSA_CUDA_CHECK(launch_pdl(rope_rows_kernel<64>, dim3(blocks), dim3(256), 0, s, static_cast<__nv_bfloat16*>(x),
-                              rows, heads, pos, lb));
+                              rows, heads, pos, turns));
   return MSA_OK;
 }
 
@@ -700,7 +686,6 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, const void* K_
   AttendWs w;
   attend_workspace(d, B, k, t_loc_max, pos_offset, ws, &w);
   const int D = d.head_dim;
-  const double log_base = std::log((double)d.rope_base);
   const float2* tab = k_loc_rotated ? nullptr : static_cast<const float2*>(rope_cache);
   if (!tab && !k_loc_rotated && t_loc_max > 0) {
     msa_status st = rope_cache_build(d, t_loc_max, pos_offset, w.rope_tab, s);
@@ -727,7 +712,7 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, const void* K_
   p.pos_offset = pos_offset;
   p.n_splits = w.n_splits;
   p.scale_log2 = (scale > 0.f ? scale : 1.0f / std::sqrt((float)D)) * kLog2e;
-  p.log_base = log_base;
+  rope_turns(d, p.turns.f);
   p.n_stages = stages_that_fit(d.n_kv, d.n_q, D, tab != nullptr);
   {
     TraceScope ts(kKAttnSplit, s);
@@ -746,10 +731,10 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, const void* K_
     dim3 grid(d.n_q, B);
     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
     if (D == 128)
-      MSA_CUDA_CHECK(launch_pdl(attn_combine_kernel<128>, grid, dim3(128), 0, s, (const float*)w.part_ml,
+      MSA_CUDA_CHECK(launch_pdl(attn_combine_kernel<128>, grid, dim3(256), 0, s, (const float*)w.part_ml,
                                 (const float*)w.part_o, w.n_splits, o));
     else
-      MSA_CUDA_CHECK(launch_pdl(attn_combine_kernel<64>, grid, dim3(128), 0, s, (const float*)w.part_ml,
+      MSA_CUDA_CHECK(launch_pdl(attn_combine_kernel<64>, grid, dim3(256), 0, s, (const float*)w.part_ml,
                                 (const float*)w.part_o, w.n_splits, o));
   }
   return MSA_OK;

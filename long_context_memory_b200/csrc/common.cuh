@@ -309,3 +309,24 @@ namespace msa {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 }  // namespace msa
+
+namespace msa {
+// ---------------------------------------------------------------------------
+// RoPE angles without floating-point range reduction.  f[i] = theta_i / (2 pi)
+// as a 64-bit binary fraction (theta_i = base^(-2i/d) < 1, so f[i] < 1); the
+// fractional turns of pos * theta_i are then exactly (pos * f[i]) mod 2^64 in
+// wrapping integer arithmetic, whatever the size of pos.  The top 24 bits of
+// that fraction give the angle to within 2^-24 turns for sincospif.
+// ---------------------------------------------------------------------------
+struct RopeTurns {
+  uint64_t f[64];  // head_dim / 2 <= 64 entries
+};
+
+__device__ __forceinline__ float2 rope_cos_sin(const RopeTurns& t, int i, int64_t pos) {
+  const uint64_t u = (uint64_t)pos * t.f[i];
+  const float x = (float)(uint32_t)(u >> 40) * 1.1920928955078125e-7f;  // 2 * turns in [0, 2): x * pi = angle
+  float sn, cs;
+  sincospif(x, &sn, &cs);
+  return make_float2(cs, sn);
+}
+}  // namespace msa

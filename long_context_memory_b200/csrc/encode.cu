@@ -43,7 +43,7 @@ struct EncodeWs {
 namespace {
 
 constexpr int kBM = 128, kBK = 64;
-constexpr int kEncStages = 4;
+constexpr int kEncStagesMax = 4;
 constexpr int kABytes = kBM * kBK * 2;  // 16 KB
 constexpr int kEncThreads = 192;        // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 
@@ -146,7 +146,7 @@ struct GemmParams {
   int m_tiles;
   int n_chunks;
   int head_dim;
-  double log_base;
+  RopeTurns turns;
   const int64_t* tok0;
   const int32_t* clen;
   const int32_t* pos0;
@@ -154,6 +154,8 @@ struct GemmParams {
   __nv_bfloat16* out1;   // K̄^R (pooled)
   int n_out0;            // columns of out0 (n_kv*D); pooled: columns >= n_out0 go to out1
   int n_out1;
+  int out1_head_major;   // out1 (K̄^R) stored [n_r][C][d_r]
+  int d_r;
 };
 
 template <int MODE, int kBN>
@@ -162,13 +164,18 @@ __global__ void __launch_bounds__(kEncThreads, 1) gemm_kernel(const __grid_const
                                                               const GemmParams p) {
   constexpr int kBBytes = kBN * kBK * 2;
   constexpr int kStageBytes = kABytes + kBBytes;
+  constexpr int kEncStages = MODE == kModeK ? 3 : 4;  // mode K gives one stage to the RoPE tables
   constexpr uint32_t kTmemCols = 2 * kBN;  // two 128 x kBN fp32 accumulators
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  float* red = reinterpret_cast<float*>(smem + kEncStages * kStageBytes);  // [2][4][256]
-  double* theta = reinterpret_cast<double*>(red + 2 * 4 * kBN);            // [64]
-  uint64_t* full = reinterpret_cast<uint64_t*>(theta + 64);
+  float* red = reinterpret_cast<float*>(smem + kEncStages * kStageBytes);  // [2][4][kBN]
+  // RoPE tables (mode K): fine[i][r] = (cos, sin)(r * theta_i) for the 64 offsets r inside a
+  // chunk (pair-major, so the 32 rows of a warp read consecutive words), and per tile
+  // coarse[c][i] = (cos, sin)(pos0(c) * theta_i) for its two chunks, reduced in fp64.
+  float2* fine = reinterpret_cast<float2*>(red + 2 * 4 * kBN);             // [64 pairs][64 rows]
+  float2* coarse = fine + (MODE == kModeK ? 64 * 64 : 0);                  // [2 chunks][64 pairs]
+  uint64_t* full = reinterpret_cast<uint64_t*>(coarse + (MODE == kModeK ? 2 * 64 : 0));
   uint64_t* empty = full + kEncStages;
   uint64_t* tfull = empty + kEncStages;
   uint64_t* tempty = tfull + 2;
@@ -189,8 +196,8 @@ __global__ void __launch_bounds__(kEncThreads, 1) gemm_kernel(const __grid_const
     fence_mbar_init();
   }
   if (MODE == kModeK) {
-    for (int i = threadIdx.x; i < p.head_dim / 2; i += blockDim.x)
-      theta[i] = exp(-2.0 * (double)i / (double)p.head_dim * p.log_base);
+    const int half = p.head_dim / 2;
+    for (int e = threadIdx.x; e < half * 64; e += blockDim.x) fine[e] = rope_cos_sin(p.turns, e / 64, e % 64);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -276,10 +283,18 @@ __global__ void __launch_bounds__(kEncThreads, 1) gemm_kernel(const __grid_const
         const bool chunk_ok = chunk < p.n_chunks;
         const int len = chunk_ok ? p.clen[chunk] : 0;
         const bool valid = rr < len;
-        const double pos = chunk_ok ? (double)(p.pos0[chunk] + rr) : 0.0;
         const int D = p.head_dim, half = D / 2;
+        // this tile's per-chunk base angles: 128 epilogue threads = 2 chunks x 64 pairs
+        {
+          const int et = threadIdx.x - 64;
+          const int c2 = et >> 6, i = et & 63;
+          const int ch = 2 * m + c2;
+          if (i < half) coarse[c2 * 64 + i] = rope_cos_sin(p.turns, i, ch < p.n_chunks ? p.pos0[ch] : 0);
+          named_bar_sync(2, 128);
+        }
+        const float2* cb = coarse + (row >> 6) * 64;
         float* rbuf = red + (size_t)(buf * 4 + ew) * kBN;
-        // 256 columns = 256/D heads; pairs (i, i + D/2) inside each head, 32 pairs per pass
+        // kBN columns = kBN/D heads; pairs (i, i + D/2) inside each head, 32 pairs per pass
         for (int c0 = 0; c0 < kBN; c0 += D) {
           for (int i0 = 0; i0 < half; i0 += 32) {
             float x[32], y[32];
@@ -288,10 +303,10 @@ __global__ void __launch_bounds__(kEncThreads, 1) gemm_kernel(const __grid_const
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-              double a = pos * theta[i0 + j];
-              a -= 6.283185307179586476925286766559 * rint(a * 0.15915494309189533576888376337251);
-              float sn, cs;
-              sincosf((float)a, &sn, &cs);
+              const float2 f = fine[(i0 + j) * 64 + rr];
+              const float2 c = cb[i0 + j];
+              const float cs = c.x * f.x - c.y * f.y;   // cos((pos0 + rr) theta)
+              const float sn = c.y * f.x + c.x * f.y;   // sin((pos0 + rr) theta)
               const float xr = x[j] * cs - y[j] * sn;
               const float yr = y[j] * cs + x[j] * sn;
               x[j] = valid ? xr : 0.f;
@@ -322,17 +337,24 @@ __global__ void __launch_bounds__(kEncThreads, 1) gemm_kernel(const __grid_const
         const int chunk = m * kBM + row;
         const int gc0 = n * kBN;
         const bool to0 = gc0 < p.n_out0;
-        __nv_bfloat16* dst = to0 ? p.out0 + (size_t)chunk * p.n_out0 + gc0
-                                 : p.out1 + (size_t)chunk * p.n_out1 + (gc0 - p.n_out0);
         for (int c0 = 0; c0 < kBN; c0 += 32) {
           float x[32];
           tmem_ld32(t_row + c0, x);
           tmem_ld_wait();
           if (chunk < p.n_chunks) {
+            __nv_bfloat16* dst;
+            if (to0) {
+              dst = p.out0 + (size_t)chunk * p.n_out0 + gc0 + c0;
+            } else {
+              const int col = gc0 - p.n_out0 + c0;  // 32 columns inside one router head
+              dst = p.out1_head_major
+                        ? p.out1 + ((size_t)(col / p.d_r) * p.n_chunks + chunk) * p.d_r + col % p.d_r
+                        : p.out1 + (size_t)chunk * p.n_out1 + col;
+            }
             uint32_t w[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(x[2 * j], x[2 * j + 1]);
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
             for (int j = 0; j < 4; ++j) d4[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
           }
@@ -349,9 +371,11 @@ __global__ void __launch_bounds__(kEncThreads, 1) gemm_kernel(const __grid_const
   if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
 }
 
-size_t gemm_smem_bytes(int bn) {
-  return 1024 + (size_t)kEncStages * (kABytes + bn * kBK * 2) + 2 * 4 * bn * sizeof(float) + 64 * sizeof(double) +
-         (2 * kEncStages + 4) * sizeof(uint64_t) + 16;
+size_t gemm_smem_bytes(int mode, int bn) {
+  const int stages = mode == kModeK ? 3 : 4;
+  const size_t tables = mode == kModeK ? (64 * 64 + 2 * 64) * sizeof(float2) : 0;
+  return 1024 + (size_t)stages * (kABytes + bn * kBK * 2) + 2 * 4 * bn * sizeof(float) + tables +
+         (2 * kEncStagesMax + 4) * sizeof(uint64_t) + 16;
 }
 
 template <int MODE>
@@ -391,7 +415,7 @@ size_t encode_workspace(const msa_dims& d, int64_t T, int n_docs, int n_chunks, 
 
 msa_status encode_launch(const msa_dims& d, const void* H, int64_t T, const int64_t* doc_off, int n_docs,
                          const int32_t* chunk_off, int n_chunks, const void* W_K, const void* W_V, const void* W_KR,
-                         void* K_bar, void* V_bar, void* KR_bar, void* ws, cudaStream_t s) {
+                         void* K_bar, void* V_bar, void* KR_bar, int kr_layout, void* ws, cudaStream_t s) {
   if (T > INT32_MAX - 64) return fail(MSA_ERR_UNSUPPORTED, "T must be < 2^31 - 64 tokens");
   EncodeWs w;
   encode_workspace(d, T, n_docs, n_chunks, ws, &w);
@@ -436,7 +460,7 @@ msa_status encode_launch(const msa_dims& d, const void* H, int64_t T, const int6
     p.m_tiles = (n_chunks + 1) / 2;
     p.n_chunks = n_chunks;
     p.head_dim = d.head_dim;
-    p.log_base = std::log((double)d.rope_base);
+    rope_turns(d, p.turns.f);
     p.tok0 = w.tok0;
     p.clen = w.clen;
     p.pos0 = w.pos0;
@@ -444,7 +468,7 @@ msa_status encode_launch(const msa_dims& d, const void* H, int64_t T, const int6
     p.n_out0 = NK;
     const int grid = std::max(1, std::min(sm_count(), p.m_tiles * p.n_tiles));
     TraceScope ts(kKEncGemmK, s);
-    MSA_CUDA_CHECK(launch_gemm<kModeK>(bn, grid, gemm_smem_bytes(bn), s, ma, mb, p));
+    MSA_CUDA_CHECK(launch_gemm<kModeK>(bn, grid, gemm_smem_bytes(kModeK, bn), s, ma, mb, p));
   }
   // ---- H̄ (hi | lo) ----
   {
@@ -480,9 +504,11 @@ msa_status encode_launch(const msa_dims& d, const void* H, int64_t T, const int6
     p.out1 = static_cast<__nv_bfloat16*>(KR_bar);
     p.n_out0 = NV;
     p.n_out1 = NR;
+    p.out1_head_major = kr_layout == 1;
+    p.d_r = d.d_r;
     const int grid = std::max(1, std::min(sm_count(), p.m_tiles * p.n_tiles));
     TraceScope ts(kKEncGemmPooled, s);
-    MSA_CUDA_CHECK(launch_gemm<kModePooled>(bn, grid, gemm_smem_bytes(bn), s, ma, mb, p));
+    MSA_CUDA_CHECK(launch_gemm<kModePooled>(bn, grid, gemm_smem_bytes(kModePooled, bn), s, ma, mb, p));
   }
   return MSA_OK;
 }

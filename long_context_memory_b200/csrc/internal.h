@@ -34,8 +34,7 @@ bool fault_injected();
 // kernel ids for tracing
 // ---------------------------------------------------------------------------
 enum KernelId : int {
-  kKQrProj = 0,
-  kKQPrep,
+  kKRouterQuery = 0,
   kKScan,
   kKTopkSlice,
   kKTopkMerge,
@@ -91,6 +90,9 @@ msa_status encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int ra
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// theta_i / (2 pi) as 64-bit binary fractions, theta_i = base^(-2i/head_dim) (computed in long double)
+void rope_turns(const msa_dims& d, uint64_t* f /* [head_dim / 2] */);
+
 // Launch with programmatic stream serialization: the kernel may be scheduled
 // while the previous kernel on the stream finishes; every kernel launched this
 // way calls pdl_wait() before its first global-memory access.
@@ -116,7 +118,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 size_t route_workspace(const msa_dims& d, int B, int n_docs, int n_chunks, int k, msa_doc_agg agg,
                        void* ws, struct RouteWs* out);
 msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int B, const void* KR_bar,
-                        const int32_t* chunk_off, int n_docs, int n_chunks, int k, msa_doc_agg agg,
+                        const int32_t* chunk_off, int n_docs, int n_chunks, int k, msa_doc_agg agg, int kr_layout,
                         float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws,
                         cudaStream_t s);
 
@@ -141,7 +143,7 @@ size_t encode_workspace(const msa_dims& d, int64_t T, int n_docs, int n_chunks, 
                         struct EncodeWs* out);
 msa_status encode_launch(const msa_dims& d, const void* H, int64_t T, const int64_t* doc_off, int n_docs,
                          const int32_t* chunk_off, int n_chunks, const void* W_K, const void* W_V,
-                         const void* W_KR, void* K_bar, void* V_bar, void* KR_bar, void* ws,
+                         const void* W_KR, void* K_bar, void* V_bar, void* KR_bar, int kr_layout, void* ws,
                          cudaStream_t s);
 
 }  // namespace msa

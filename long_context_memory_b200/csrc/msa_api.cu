@@ -50,6 +50,16 @@ bool fault_injected() {
   return f && std::strcmp(f, "launch") == 0;
 }
 
+void rope_turns(const msa_dims& d, uint64_t* f) {
+  const long double two_pi = 6.283185307179586476925286766559005768L;
+  const long double lb = logl((long double)d.rope_base);
+  for (int i = 0; i < d.head_dim / 2; ++i) {
+    const long double theta = expl(-2.0L * (long double)i / (long double)d.head_dim * lb);
+    const long double turns = theta / two_pi;  // in (0, 1)
+    f[i] = (uint64_t)ldexpl(turns, 64);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // device properties
 // ---------------------------------------------------------------------------
@@ -98,7 +108,7 @@ msa_status encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int ra
 // ---------------------------------------------------------------------------
 namespace {
 const char* kKernelNames[kKernelCount] = {
-    "qr_proj", "q_prep", "scan", "topk_slice", "topk_merge", "rope_table", "attn_split", "attn_combine",
+    "router_query", "scan", "topk_slice", "topk_merge", "rope_table", "attn_split", "attn_combine",
     "enc_chunk_map", "enc_transpose_w", "enc_gemm_k", "enc_pool_h", "enc_gemm_pooled", "rope_rows", "gather_plan", "gather_copy"};
 
 struct TraceState {
@@ -253,18 +263,19 @@ size_t msa_route_workspace_size(const msa_dims* dims, int32_t B, int32_t n_docs,
 
 msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR, int32_t B, const void* KR_bar,
                           const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks, int32_t k, msa_doc_agg agg,
-                          float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws, size_t ws_bytes,
+                          int32_t kr_layout, float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws, size_t ws_bytes,
                           void* stream) {
   msa_status st = check_dims(dims, false, true);
   if (st != MSA_OK) return st;
-  if (W_QR && (dims->hidden < 64 || dims->hidden % 64 != 0))
-    return fail(MSA_ERR_UNSUPPORTED, "hidden must be a positive multiple of 64 (got %d)", dims->hidden);
+  if (W_QR && (dims->hidden < 64 || dims->hidden % 64 != 0 || dims->hidden > 8192))
+    return fail(MSA_ERR_UNSUPPORTED, "hidden must be a multiple of 64 in [64, 8192] (got %d)", dims->hidden);
   if (B < 1) return fail(MSA_ERR_INVALID_ARG, "B must be >= 1 (got %d)", B);
   if (n_docs < 1 || n_chunks < n_docs)
     return fail(MSA_ERR_INVALID_ARG, "need 1 <= n_docs <= n_chunks (got %d, %d)", n_docs, n_chunks);
   if (k < 1 || k > n_docs || k > 256)
     return fail(MSA_ERR_INVALID_ARG, "k must be in [1, min(n_docs, 256)] (got %d, n_docs %d)", k, n_docs);
   if (agg != MSA_AGG_MAX && agg != MSA_AGG_MEAN) return fail(MSA_ERR_INVALID_ARG, "unknown aggregation %d", (int)agg);
+  if (kr_layout != 0 && kr_layout != 1) return fail(MSA_ERR_INVALID_ARG, "kr_layout must be 0 or 1 (got %d)", kr_layout);
   const int n_slices = (n_docs + 4095) / 4096;
   if ((size_t)n_slices * k > 24576) return fail(MSA_ERR_UNSUPPORTED, "n_docs * k too large for the top-k merge");
   CHECK_PTR(Hq);
@@ -279,7 +290,7 @@ msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR
   if (need && (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)))
     return fail(MSA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
   if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
-  return route_launch(*dims, Hq, W_QR, B, KR_bar, chunk_off, n_docs, n_chunks, k, agg, doc_scores, topk_idx,
+  return route_launch(*dims, Hq, W_QR, B, KR_bar, chunk_off, n_docs, n_chunks, k, agg, kr_layout, doc_scores, topk_idx,
                       topk_score, ws, static_cast<cudaStream_t>(stream));
 }
 
@@ -421,8 +432,8 @@ size_t msa_encode_workspace_size(const msa_dims* dims, int64_t T, int32_t n_docs
 
 msa_status msa_encode_memory(const msa_dims* dims, const void* H, int64_t T, const int64_t* doc_off, int32_t n_docs,
                              const int32_t* chunk_off, int32_t n_chunks, const void* W_K, const void* W_V,
-                             const void* W_KR, void* K_bar, void* V_bar, void* KR_bar, void* ws, size_t ws_bytes,
-                             void* stream) {
+                             const void* W_KR, void* K_bar, void* V_bar, void* KR_bar, int32_t kr_layout, void* ws,
+                             size_t ws_bytes, void* stream) {
   msa_status st = check_dims(dims, true, true);
   if (st != MSA_OK) return st;
   if (dims->hidden < 64 || dims->hidden % 64 != 0)
@@ -445,9 +456,10 @@ msa_status msa_encode_memory(const msa_dims* dims, const void* H, int64_t T, con
   if (ws_bytes < need) return fail(MSA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
   if (need && (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)))
     return fail(MSA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
+  if (kr_layout != 0 && kr_layout != 1) return fail(MSA_ERR_INVALID_ARG, "kr_layout must be 0 or 1 (got %d)", kr_layout);
   if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
-  return encode_launch(*dims, H, T, doc_off, n_docs, chunk_off, n_chunks, W_K, W_V, W_KR, K_bar, V_bar, KR_bar, ws,
-                       static_cast<cudaStream_t>(stream));
+  return encode_launch(*dims, H, T, doc_off, n_docs, chunk_off, n_chunks, W_K, W_V, W_KR, K_bar, V_bar, KR_bar,
+                       kr_layout, ws, static_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------ tracing ------------------------------

@@ -8,9 +8,9 @@
 // with the memory size (complexity item of the same section: O(ML/P)).
 //
 // Kernels, in launch order:
-//   qr_proj_kernel   Q^R partial sums (HBM-bound read of W^QR, split over K)
-//   q_prep_kernel    sums the partials, normalises each head, writes the query
-//                    as bf16 hi + lo mma B-fragments; clears the doc keys
+//   router_query_kernel  Q^R = H_q W^QR (each CTA 8 columns over the whole hidden
+//                    dimension), per-head normalisation by the head's last CTA,
+//                    bf16 hi + lo rows for the scan's TMA; clears the doc keys
 //   scan_kernel      TMA-staged streaming scan of K̄^R: tensor-core dots and
 //                    Gram diagonal (norm), cosine, head mean, per-document
 //                    segmented max folded in with atomicMax on ordered keys
@@ -31,144 +31,152 @@
 namespace msa {
 
 struct RouteWs {
-  float* qr_part;     // [ksplit][B][NR] fp32 partial sums of Q^R (W_QR given)
+  float* qr;          // [B][NR] fp32 router queries (W_QR given)
+  uint32_t* head_done;  // [n_r] CTAs finished per router head (back to 0 after each call)
   __nv_bfloat16* q_hl; // [passes][n_r][2][NQ][d_r] normalised query, bf16 hi and lo terms
   uint32_t* doc_key;  // [B][n_docs] ordered-uint32 doc max (MAX)
   float* chunk_s;     // [B][n_chunks] chunk scores (MEAN)
   uint64_t* cand;     // [B][n_slices][k] slice winners
-  int ksplit, nq, passes, n_slices;
+  int nq, passes, n_slices;
 };
 
 namespace {
 
 constexpr int kSliceDocs = 4096;   // documents per top-k slice CTA
 constexpr int kTopkThreads = 1024;
-constexpr int kQpCols = 64;
-constexpr int kQpQB = 8;
 constexpr float kEps = 1e-12f;
 
 // --------------------------------------------------------------------------
-// Q^R = H_q W^QR, partial sums over a slice of the hidden dimension
+// Router query, one kernel: Q^R = H_q W^QR, per-head normalisation, bf16 hi + lo
+// terms in the layout the scan's TMA reads (q_hl[pass][head][hi|lo][NQ rows][d_r];
+// rows of padding queries are zero), and the clearing of the document keys.
+// CTA = 8 columns of Q^R over the whole hidden dimension: thread t reads rows
+// t, t+256, ... of W as 16-byte vectors, all in flight at once.  The last CTA
+// to finish a router head (a per-head counter) normalises that head.
+// With W_QR == NULL the rows of Hq already hold Q^R and only the head step runs.
 // --------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) qr_proj_kernel(const __nv_bfloat16* __restrict__ Hq,
-                                                      const __nv_bfloat16* __restrict__ W, int B, int hidden,
-                                                      int NR, int rows_per_split, float* __restrict__ part) {
-  __shared__ float red[8][kQpQB][kQpCols];
-  pdl_launch_dependents();
-  pdl_wait();
-  const int col0 = blockIdx.x * kQpCols;
-  const int split = blockIdx.y;
-  const int k_begin = split * rows_per_split;
-  const int k_end = min(hidden, k_begin + rows_per_split);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int cg = lane & 7, rl = lane >> 3;
-  const uint16_t* hq = reinterpret_cast<const uint16_t*>(Hq);
-  for (int b0 = 0; b0 < B; b0 += kQpQB) {
-    float acc[kQpQB][8];
-#pragma unroll
-    for (int j = 0; j < kQpQB; ++j)
-#pragma unroll
-      for (int c = 0; c < 8; ++c) acc[j][c] = 0.f;
-    for (int k = k_begin + warp * 4 + rl; k < k_end; k += 32) {
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(W + (size_t)k * NR + col0 + cg * 8));
-      float wf[8];
-      float2 t;
-      t = unpack_bf16x2(w.x); wf[0] = t.x; wf[1] = t.y;
-      t = unpack_bf16x2(w.y); wf[2] = t.x; wf[3] = t.y;
-      t = unpack_bf16x2(w.z); wf[4] = t.x; wf[5] = t.y;
-      t = unpack_bf16x2(w.w); wf[6] = t.x; wf[7] = t.y;
-#pragma unroll
-      for (int j = 0; j < kQpQB; ++j) {
-        if (b0 + j < B) {
-          const float h = bf16_bits_to_float(hq[(size_t)(b0 + j) * hidden + k]);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) acc[j][c] = fmaf(h, wf[c], acc[j][c]);
-        }
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < kQpQB; ++j)
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        acc[j][c] += __shfl_xor_sync(0xffffffffu, acc[j][c], 8);
-        acc[j][c] += __shfl_xor_sync(0xffffffffu, acc[j][c], 16);
-      }
-    if (rl == 0) {
-#pragma unroll
-      for (int j = 0; j < kQpQB; ++j)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) red[warp][j][cg * 8 + c] = acc[j][c];
-    }
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < kQpQB * kQpCols; idx += 256) {
-      const int j = idx / kQpCols, c = idx % kQpCols;
-      if (b0 + j < B) {
-        float s = 0.f;
-#pragma unroll
-        for (int w8 = 0; w8 < 8; ++w8) s += red[w8][j][c];
-        part[((size_t)split * B + b0 + j) * NR + col0 + c] = s;
-      }
-    }
-    __syncthreads();
-  }
-}
+constexpr int kQrCols = 8;
+constexpr int kQrThreads = 256;
+constexpr int kQrMaxRows = 32;  // rows of W per thread: hidden <= 8192
+constexpr int kQrRowChunk = 8;  // rows loaded together
+constexpr int kQrQB = 8;        // queries per register group
 
-// --------------------------------------------------------------------------
-// normalise Q^R per head and write it as two bf16 terms (hi + lo) in the
-// layout the scan's TMA reads: q_hl[pass][head][hi|lo][NQ query rows][d_r];
-// rows of padding queries are zero.  Also clears this query's document keys.
-// --------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) q_prep_kernel(const float* __restrict__ part, int ksplit,
-                                                     const __nv_bfloat16* __restrict__ qr_direct, int B,
-                                                     int n_r, int d_r, int nq, __nv_bfloat16* __restrict__ q_hl,
-                                                     uint32_t* __restrict__ doc_key, int n_docs) {
-  extern __shared__ float qs[];  // [n_r * d_r] then inv norms [n_r]
+__global__ void __launch_bounds__(kQrThreads) router_query_kernel(
+    const __nv_bfloat16* __restrict__ Hq, const __nv_bfloat16* __restrict__ W, int B, int b_pad, int hidden,
+    int n_r, int d_r, int nq, float* __restrict__ qr, uint32_t* __restrict__ head_done,
+    __nv_bfloat16* __restrict__ q_hl, uint32_t* __restrict__ doc_key, int n_docs) {
+  __shared__ float red[kQrThreads / 32][kQrQB][kQrCols];
+  __shared__ float invn[32];
+  __shared__ bool last;
   pdl_launch_dependents();
   pdl_wait();
-  const int b = blockIdx.x;      // padded query index (< passes * nq)
   const int NR = n_r * d_r;
-  float* invn = qs + NR;
-  const bool real = b < B;
-  for (int n = threadIdx.x; n < NR; n += blockDim.x) {
-    float v = 0.f;
-    if (real) {
-      if (qr_direct) {
-        v = bf16_bits_to_float(reinterpret_cast<const uint16_t*>(qr_direct)[(size_t)b * NR + n]);
-      } else {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        int s = 0;
-        for (; s + 4 <= ksplit; s += 4) {
+  const int col0 = blockIdx.x * kQrCols;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint16_t* hq = reinterpret_cast<const uint16_t*>(Hq);
+
+  // clear the document keys (grid-stride); the scan only runs after this kernel completes
+  if (doc_key)
+    for (size_t i = blockIdx.x * (size_t)kQrThreads + tid; i < (size_t)B * n_docs; i += (size_t)gridDim.x * kQrThreads)
+      doc_key[i] = 0u;
+
+  if (W) {
+    for (int b0 = 0; b0 < B; b0 += kQrQB) {
+      float acc[kQrQB][kQrCols];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) acc[u] += part[((size_t)(s + u) * B + b) * NR + n];
+      for (int j = 0; j < kQrQB; ++j)
+#pragma unroll
+        for (int c = 0; c < kQrCols; ++c) acc[j][c] = 0.f;
+      for (int u0 = 0; u0 < kQrMaxRows; u0 += kQrRowChunk) {
+        if (tid + kQrThreads * u0 >= hidden) break;
+        uint4 wv[kQrRowChunk];  // this chunk's rows of W, all in flight at once
+#pragma unroll
+        for (int u = 0; u < kQrRowChunk; ++u) {
+          const int k = tid + kQrThreads * (u0 + u);
+          wv[u] = k < hidden ? __ldg(reinterpret_cast<const uint4*>(W + (size_t)k * NR + col0)) : make_uint4(0, 0, 0, 0);
         }
-        for (; s < ksplit; ++s) acc[0] += part[((size_t)s * B + b) * NR + n];
-        v = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+#pragma unroll
+        for (int u = 0; u < kQrRowChunk; ++u) {
+          const int k = tid + kQrThreads * (u0 + u);
+          if (k < hidden) {
+            float wf[8];
+            float2 t;
+            t = unpack_bf16x2(wv[u].x); wf[0] = t.x; wf[1] = t.y;
+            t = unpack_bf16x2(wv[u].y); wf[2] = t.x; wf[3] = t.y;
+            t = unpack_bf16x2(wv[u].z); wf[4] = t.x; wf[5] = t.y;
+            t = unpack_bf16x2(wv[u].w); wf[6] = t.x; wf[7] = t.y;
+#pragma unroll
+            for (int j = 0; j < kQrQB; ++j) {
+              const float h = b0 + j < B ? bf16_bits_to_float(hq[(size_t)(b0 + j) * hidden + k]) : 0.f;
+#pragma unroll
+              for (int c = 0; c < kQrCols; ++c) acc[j][c] = fmaf(h, wf[c], acc[j][c]);
+            }
+          }
+        }
       }
+#pragma unroll
+      for (int j = 0; j < kQrQB; ++j)
+#pragma unroll
+        for (int c = 0; c < kQrCols; ++c) {
+          float v = acc[j][c];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          if (lane == 0) red[warp][j][c] = v;
+        }
+      __syncthreads();
+      if (tid < kQrQB * kQrCols) {
+        const int j = tid / kQrCols, c = tid % kQrCols;
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < kQrThreads / 32; ++w) v += red[w][j][c];
+        if (b0 + j < B) qr[(size_t)(b0 + j) * NR + col0 + c] = v;
+      }
+      __syncthreads();
     }
-    qs[n] = v;
+    // this head's columns are written: count the CTA in and let the head's last CTA go on
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+      const int h = col0 / d_r;
+      const uint32_t prev = atomicAdd(&head_done[h], 1u);
+      last = prev == (uint32_t)(d_r / kQrCols - 1);
+      if (last) head_done[h] = 0u;  // ready for the next call
+    }
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+  } else if (col0 % d_r != 0) {
+    return;  // Q^R given: one CTA per head does the head step
   }
-  __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int h = warp; h < n_r; h += blockDim.x / 32) {
+
+  // ---- head step: normalise head h of every query and write the bf16 hi/lo rows ----
+  const int h = col0 / d_r;
+  const float* src = W ? qr : nullptr;
+  for (int b = warp; b < b_pad; b += kQrThreads / 32) {
     float ss = 0.f;
-    for (int i = lane; i < d_r; i += 32) ss = fmaf(qs[h * d_r + i], qs[h * d_r + i], ss);
+    for (int i = lane; i < d_r; i += 32) {
+      float v = 0.f;
+      if (b < B) v = src ? __ldcg(&src[(size_t)b * NR + h * d_r + i])
+                         : bf16_bits_to_float(hq[(size_t)b * NR + h * d_r + i]);
+      ss = fmaf(v, v, ss);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (lane == 0) invn[h] = 1.0f / fmaxf(sqrtf(ss), kEps);
-  }
-  __syncthreads();
-  const int pass = b / nq, row = b % nq;
-  for (int idx = threadIdx.x; idx < NR; idx += blockDim.x) {
-    const int h = idx / d_r, dd = idx % d_r;
-    const float x = qs[idx] * invn[h];
-    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+    if (lane == 0) invn[b % 32] = 1.0f / fmaxf(sqrtf(ss), kEps);
+    __syncwarp();
+    const float sc = invn[b % 32];
+    const int pass = b / nq, row = b % nq;
     const size_t base = (((size_t)pass * n_r + h) * 2) * nq;
-    q_hl[(base + row) * d_r + dd] = hi;
-    q_hl[(base + nq + row) * d_r + dd] = lo;
-  }
-  if (real && doc_key) {
-    for (int i = threadIdx.x; i < n_docs; i += blockDim.x) doc_key[(size_t)b * n_docs + i] = 0u;
+    for (int i = lane; i < d_r; i += 32) {
+      float v = 0.f;
+      if (b < B) v = src ? __ldcg(&src[(size_t)b * NR + h * d_r + i])
+                         : bf16_bits_to_float(hq[(size_t)b * NR + h * d_r + i]);
+      const float x = v * sc;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+      q_hl[(base + row) * d_r + i] = hi;
+      q_hl[(base + nq + row) * d_r + i] = lo;
+    }
   }
 }
 
@@ -196,6 +204,7 @@ struct ScanParams {
   float* chunk_s;
   int n_r, n_docs, n_chunks, n_tiles;
   int q_base, q_count, pass;
+  int head_major;  // K̄^R stored [n_r][C][d_r] instead of [C][n_r][d_r]
   uint32_t tmem_cols;
   float inv_nr;
 };
@@ -269,7 +278,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         mbar_arrive_expect_tx(&full[st], Gm::kStageBytes);
 #pragma unroll
         for (int j = 0; j < Gm::kHalves; ++j) {
-          tma_load_2d(k_s + j * Gm::kKBox, &kr_map, &full[st], h * DR + j * 64, tile * kScanM);
+          if (p.head_major)
+            tma_load_3d(k_s + j * Gm::kKBox, &kr_map, &full[st], j * 64, tile * kScanM, h);
+          else
+            tma_load_2d(k_s + j * Gm::kKBox, &kr_map, &full[st], h * DR + j * 64, tile * kScanM);
 #pragma unroll
           for (int hl = 0; hl < 2; ++hl)
             tma_load_2d(q_s + (hl * Gm::kHalves + j) * Gm::kQBox, &q_map, &full[st], j * 64,
@@ -654,11 +666,11 @@ size_t route_workspace(const msa_dims& d, int B, int n_docs, int n_chunks, int k
   Carver cv(ws);
   RouteWs w{};
   const int NR = d.n_r * d.d_r;
-  w.ksplit = std::max(1, std::min(32, d.hidden / 160));
   w.nq = B <= 16 ? 16 : 32;
   w.passes = (B + w.nq - 1) / w.nq;
   w.n_slices = (n_docs + kSliceDocs - 1) / kSliceDocs;
-  w.qr_part = cv.take<float>((size_t)w.ksplit * B * NR);
+  w.qr = cv.take<float>((size_t)B * NR);
+  w.head_done = cv.take<uint32_t>(8);
   w.q_hl = cv.take<__nv_bfloat16>((size_t)w.passes * d.n_r * 2 * w.nq * d.d_r);
   w.doc_key = agg == MSA_AGG_MAX ? cv.take<uint32_t>((size_t)B * n_docs) : nullptr;
   w.chunk_s = agg == MSA_AGG_MEAN ? cv.take<float>((size_t)B * n_chunks) : nullptr;
@@ -668,37 +680,39 @@ size_t route_workspace(const msa_dims& d, int B, int n_docs, int n_chunks, int k
 }
 
 msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int B, const void* KR_bar,
-                        const int32_t* chunk_off, int n_docs, int n_chunks, int k, msa_doc_agg agg,
+                        const int32_t* chunk_off, int n_docs, int n_chunks, int k, msa_doc_agg agg, int kr_layout,
                         float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws, cudaStream_t s) {
   RouteWs w;
   route_workspace(d, B, n_docs, n_chunks, k, agg, ws, &w);
   const int NR = d.n_r * d.d_r;
   const bool mean = agg == MSA_AGG_MEAN;
 
-  // K1: Q^R partial sums
-  if (W_QR) {
-    TraceScope ts(kKQrProj, s);
-    const int rows = (d.hidden + w.ksplit - 1) / w.ksplit;
-    MSA_CUDA_CHECK(launch_pdl(qr_proj_kernel, dim3(NR / kQpCols, w.ksplit), dim3(256), 0, s,
-                              static_cast<const __nv_bfloat16*>(Hq), static_cast<const __nv_bfloat16*>(W_QR), B,
-                              d.hidden, NR, rows, w.qr_part));
-  }
-  // K2: normalise + fragments + clear document keys
+  // K1: router query (projection, normalisation, hi/lo layout) and document keys cleared
   {
-    TraceScope ts(kKQPrep, s);
-    const size_t sm = (size_t)(NR + d.n_r) * sizeof(float);
-    MSA_CUDA_CHECK(launch_pdl(q_prep_kernel, dim3(w.passes * w.nq), dim3(256), sm, s, (const float*)w.qr_part,
-                              w.ksplit, W_QR ? nullptr : static_cast<const __nv_bfloat16*>(Hq), B, d.n_r, d.d_r,
-                              w.nq, w.q_hl, w.doc_key, n_docs));
+    MSA_CUDA_CHECK(cudaMemsetAsync(w.head_done, 0, 8 * sizeof(uint32_t), s));
+    TraceScope ts(kKRouterQuery, s);
+    MSA_CUDA_CHECK(launch_pdl(router_query_kernel, dim3(NR / kQrCols), dim3(kQrThreads), 0, s,
+                              static_cast<const __nv_bfloat16*>(Hq), static_cast<const __nv_bfloat16*>(W_QR), B,
+                              w.passes * w.nq, d.hidden, d.n_r, d.d_r, w.nq, w.qr, w.head_done, w.q_hl, w.doc_key,
+                              n_docs));
   }
   // K3: scan, NQ (16 or 32) queries per pass
   {
     CUtensorMap kmap, qmap;
-    const uint64_t dims[2] = {(uint64_t)NR, (uint64_t)n_chunks};
-    const uint64_t strides[1] = {(uint64_t)NR * 2};
-    const uint32_t box[2] = {64, (uint32_t)kScanM};
-    msa_status st = encode_tensor_map(&kmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(KR_bar), dims,
-                                      strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    msa_status st;
+    if (kr_layout == 1) {  // head-major [n_r][C][d_r]: one head's rows are contiguous
+      const uint64_t dims[3] = {(uint64_t)d.d_r, (uint64_t)n_chunks, (uint64_t)d.n_r};
+      const uint64_t strides[2] = {(uint64_t)d.d_r * 2, (uint64_t)n_chunks * d.d_r * 2};
+      const uint32_t box[3] = {64, (uint32_t)kScanM, 1};
+      st = encode_tensor_map(&kmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(KR_bar), dims, strides, box,
+                             CU_TENSOR_MAP_SWIZZLE_128B);
+    } else {
+      const uint64_t dims[2] = {(uint64_t)NR, (uint64_t)n_chunks};
+      const uint64_t strides[1] = {(uint64_t)NR * 2};
+      const uint32_t box[2] = {64, (uint32_t)kScanM};
+      st = encode_tensor_map(&kmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(KR_bar), dims, strides, box,
+                             CU_TENSOR_MAP_SWIZZLE_128B);
+    }
     if (st != MSA_OK) return st;
     const uint64_t qdims[2] = {(uint64_t)d.d_r, (uint64_t)w.passes * d.n_r * 2 * w.nq};
     const uint64_t qstrides[1] = {(uint64_t)d.d_r * 2};
@@ -722,6 +736,7 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
       p.q_base = pass * w.nq;
       p.q_count = std::min(B - p.q_base, w.nq);
       p.pass = pass;
+      p.head_major = kr_layout == 1;
       p.tmem_cols = cols;
       p.inv_nr = 1.0f / (float)d.n_r;
       TraceScope ts(kKScan, s);

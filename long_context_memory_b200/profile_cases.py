@@ -11,6 +11,7 @@ Cases
   route1m    1M-token memory, B = 1   (K̄^R 33 MB)
   route16m   16M-token memory, B = 32 (K̄^R 520 MB)
   route100m  100M-token memory, B = 1 (K̄^R 3.2 GB); --batch to change B
+             (route cases: --kr-layout head stores K̄^R head-major [n_r, C, d_r])
   attend1m   sparse attention, 1M-token memory, B = 1, 4K local tokens (rotated key cache)
   attend16m  sparse attention, 16M-token memory, B = 32, 8K local tokens (rotated key cache)
   encode     offline encoding of --tokens tokens (default 1M), hidden 2560
@@ -48,7 +49,7 @@ def randn_bf16(shape, g, device):
 
 
 class RouteCase:
-    def __init__(self, T, B, median, seed, device, k=16, dims=W.QWEN3_4B_DIMS, layers=1):
+    def __init__(self, T, B, median, seed, device, k=16, dims=W.QWEN3_4B_DIMS, layers=1, head_major=False):
         import torch
 
         import long_context_memory_b200 as msa
@@ -59,7 +60,9 @@ class RouteCase:
         g = torch.Generator(device=device)
         g.manual_seed(seed)
         self.chunk_off = torch.from_numpy(co).to(device)
-        self.KR = [randn_bf16((C, dims.n_r, dims.d_r), g, device) for _ in range(layers)]
+        self.head_major = head_major
+        kr_shape = (dims.n_r, C, dims.d_r) if head_major else (C, dims.n_r, dims.d_r)
+        self.KR = [randn_bf16(kr_shape, g, device) for _ in range(layers)]
         self.Hq = randn_bf16((B, dims.hidden), g, device)
         self.W_QR = (torch.randn((dims.hidden, dims.n_r * dims.d_r), generator=g, device=device) /
                      math.sqrt(dims.hidden)).to(torch.bfloat16)
@@ -84,7 +87,7 @@ class RouteCase:
 
     def run(self, layer=0):
         self.msa.route_topk(self.d, self.Hq, self.W_QR, self.KR[layer], self.chunk_off, self.k,
-                            out=(self.idx, self.sc, None), ws=self.ws)
+                            out=(self.idx, self.sc, None), ws=self.ws, kr_head_major=self.head_major)
 
     @property
     def scan_bytes(self):
@@ -172,15 +175,17 @@ def main():
     ap.add_argument("--warmup", type=int, default=2)
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--tokens", type=int, default=1_000_000)
+    ap.add_argument("--kr-layout", choices=["chunk", "head"], default="chunk")
     a = ap.parse_args()
     dev = torch.device("cuda:0")
     seed = W.BASE_SEED + 7
+    hm = a.kr_layout == "head"
     if a.case == "route1m":
-        case = RouteCase(1_000_000, a.batch or 1, 2048, seed, dev)
+        case = RouteCase(1_000_000, a.batch or 1, 2048, seed, dev, head_major=hm)
     elif a.case == "route16m":
-        case = RouteCase(16_000_000, a.batch or 32, 2048, seed, dev)
+        case = RouteCase(16_000_000, a.batch or 32, 2048, seed, dev, head_major=hm)
     elif a.case == "route100m":
-        case = RouteCase(100_000_000, a.batch or 1, 4096, seed, dev)
+        case = RouteCase(100_000_000, a.batch or 1, 4096, seed, dev, head_major=hm)
     elif a.case == "attend1m":
         case = AttendCase(1_000_000, a.batch or 1, 2048, 4096, seed, dev)
     elif a.case == "attend16m":
@@ -198,7 +203,8 @@ def main():
             case.run()
             e1.record(s)
             torch.cuda.synchronize()
-            print(f"{a.case} launch {i}: {e0.elapsed_time(e1) * 1e3:.1f} us", flush=True)
+            tag = f"{a.case}[{a.kr_layout}]" if a.case.startswith("route") else a.case
+            print(f"{tag} launch {i}: {e0.elapsed_time(e1) * 1e3:.1f} us", flush=True)
 
 
 if __name__ == "__main__":

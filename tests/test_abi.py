@@ -71,12 +71,13 @@ def _dims(**kw):
 FAKE = 0x10000  # 16-byte aligned non-null "device" address; never dereferenced
 
 
-def _route(msa, dims, B=1, n_docs=10, n_chunks=20, k=4, agg=0, ws_bytes=None, Hq=FAKE, kr=FAKE, idx=FAKE):
+def _route(msa, dims, B=1, n_docs=10, n_chunks=20, k=4, agg=0, ws_bytes=None, Hq=FAKE, kr=FAKE, idx=FAKE, layout=0):
     dd = msa.Dims.of(dims)
     need = msa.lib.msa_route_workspace_size(ctypes.byref(dd), B, n_docs, n_chunks, k, agg)
     if ws_bytes is None:
         ws_bytes = need
-    return msa.lib.msa_route_topk(ctypes.byref(dd), Hq, None, B, kr, FAKE, n_docs, n_chunks, k, agg, None, idx, FAKE,
+    return msa.lib.msa_route_topk(ctypes.byref(dd), Hq, None, B, kr, FAKE, n_docs, n_chunks, k, agg, layout, None, idx,
+                                  FAKE,
                                   0x100000 if ws_bytes else None, ws_bytes, None)
 
 
@@ -92,6 +93,7 @@ def test_route_validation(msa):
     assert _route(msa, ok, Hq=FAKE + 4) == 1                # misaligned
     assert _route(msa, ok, kr=None) == 1                    # NULL
     assert _route(msa, ok, agg=7) == 1
+    assert _route(msa, ok, layout=2) == 1                   # K̄^R layout is 0 (chunk-major) or 1 (head-major)
     assert _route(msa, ok, ws_bytes=16) == 3                # workspace too small
     assert "workspace too small" in msa.lib.msa_last_error().decode()
 
@@ -127,8 +129,14 @@ def test_attend_validation(msa):
 def test_encode_validation(msa):
     dd = msa.Dims.of(_dims(hidden=100))
     r = msa.lib.msa_encode_memory(ctypes.byref(dd), FAKE, 1000, FAKE, 3, FAKE, 20, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
-                                  None, 0, None)
+                                  0, None, 0, None)
     assert r == 2
+    dd = msa.Dims.of(_dims())
+    need = msa.lib.msa_encode_workspace_size(ctypes.byref(dd), 1000, 3, 20)
+    for layout, want in ((2, 1), (-1, 1)):
+        r = msa.lib.msa_encode_memory(ctypes.byref(dd), FAKE, 1000, FAKE, 3, FAKE, 20, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                      FAKE, layout, 0x100000, need, None)
+        assert r == want, (layout, r, msa.lib.msa_last_error())
 
 
 def test_topk_merge_validation(msa):

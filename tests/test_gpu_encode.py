@@ -29,13 +29,13 @@ def _dev(a, device):
     return W.to_torch(np.ascontiguousarray(a)).to(device)
 
 
-def _encode(msa, dims, H, doc_off, WK, WV, WKR, device):
+def _encode(msa, dims, H, doc_off, WK, WV, WKR, device, head_major=False):
     import torch
 
     co, C = msa.chunk_offsets(doc_off)
     out = msa.encode_memory(dims, _dev(H, device), torch.from_numpy(np.asarray(doc_off, dtype=np.int64)).to(device),
                             torch.from_numpy(co).to(device), C, _dev(WK, device), _dev(WV, device),
-                            _dev(WKR, device))
+                            _dev(WKR, device), kr_head_major=head_major)
     torch.cuda.synchronize()
     assert msa.check_device_errors() == 0
     return [O.bf16_to_f64(torch_bits(t)) for t in out], co
@@ -77,6 +77,27 @@ def test_encode_edge_lengths(msa, cuda_device, head_dim, n_kv, n_r, d_r):
     _close(Kg, Kb, "K_bar")
     _close(Vg, Vb, "V_bar")
     _close(KRg, KRb, "KR_bar")
+
+
+@pytest.mark.parametrize("n_r,d_r", [(8, 128), (2, 64), (6, 64)])
+def test_encode_head_major_router_keys(msa, cuda_device, n_r, d_r):
+    # K̄^R written [n_r, C, d_r]: the same values as the chunk-major output, moved
+    rng = np.random.default_rng(40 + n_r)
+    lens = np.array([5, 64, 129, 300, 1, 77, 640, 65])
+    doc_off = W.offsets_from_lengths(lens)
+    T, hid = int(doc_off[-1]), 256
+    d = W.Dims(hidden=hid, n_q=4, n_kv=2, head_dim=64, n_r=n_r, d_r=d_r)
+    H = W.normal_bf16(rng, (T, hid))
+    WK = W.normal_bf16(rng, (hid, 2 * 64), hid ** -0.5)
+    WV = W.normal_bf16(rng, (hid, 2 * 64), hid ** -0.5)
+    WKR = W.normal_bf16(rng, (hid, n_r * d_r), hid ** -0.5)
+    (Kg, Vg, KRg), co = _encode(msa, d, H, doc_off, WK, WV, WKR, cuda_device, head_major=True)
+    assert KRg.shape == (n_r, co[-1], d_r)
+    Kb, Vb, KRb = O.encode_memory(H, doc_off, WK, WV, WKR, 2, 64, n_r, d_r)
+    _close(KRg, KRb.transpose(1, 0, 2), "KR_bar head-major")
+    _close(Kg, Kb, "K_bar")
+    (_, _, KR0), _ = _encode(msa, d, H, doc_off, WK, WV, WKR, cuda_device)
+    assert np.array_equal(KRg, KR0.transpose(1, 0, 2))
 
 
 def test_encode_long_documents_positions(msa, cuda_device):

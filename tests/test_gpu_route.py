@@ -37,12 +37,14 @@ def _route_case(seed, n_docs, B, n_r, d_r, lo=1, hi=700, hidden=256):
     return dims, doc_off, KR, QR, Hq, Wqr, rng
 
 
-def _run(msa, dims, Hq, Wqr, KR, doc_off, k, agg, device):
+def _run(msa, dims, Hq, Wqr, KR, doc_off, k, agg, device, head_major=False):
     import torch
 
     co, C = msa.chunk_offsets(doc_off)
+    kr = np.ascontiguousarray(KR.transpose(1, 0, 2)) if head_major else KR
     idx, sc, ds = msa.route_topk(dims, _dev(Hq, device), None if Wqr is None else _dev(Wqr, device),
-                                 _dev(KR, device), torch.from_numpy(co).to(device), k, agg=agg, want_doc_scores=True)
+                                 _dev(kr, device), torch.from_numpy(co).to(device), k, agg=agg, want_doc_scores=True,
+                                 kr_head_major=head_major)
     torch.cuda.synchronize()
     assert msa.check_device_errors() == 0
     return idx.cpu().numpy(), sc.cpu().numpy(), ds.cpu().numpy()
@@ -74,6 +76,22 @@ def test_route_projection_and_aggregation(msa, cuda_device, agg):
     assert np.max(np.abs(ds - s)) < SCORE_ATOL
     for b in range(B):
         check_topk(idx[b], sc[b], s[b], k, where=f"agg={agg} b={b}")
+
+
+@pytest.mark.parametrize("B", [1, 13, 40])
+@pytest.mark.parametrize("n_r,d_r", [(8, 128), (3, 128), (4, 64)])
+def test_route_head_major_keys(msa, cuda_device, B, n_r, d_r):
+    # K̄^R stored [n_r, C, d_r]: same products in the same order, so the scores are the chunk-major ones, bit for bit
+    dims, doc_off, KR, QR, Hq, Wqr, _ = _route_case(300 + B + n_r, 211, B, n_r, d_r)
+    k = 12
+    idx, sc, ds = _run(msa, dims, QR, None, KR, doc_off, k, msa.AGG_MAX, cuda_device, head_major=True)
+    co, *_ = O.chunk_layout(doc_off)
+    s, _, _ = O.route_topk(O.bf16_to_f64(QR).reshape(B, n_r, d_r), KR, co, k)
+    assert np.max(np.abs(ds - s)) < SCORE_ATOL, np.max(np.abs(ds - s))
+    for b in range(B):
+        check_topk(idx[b], sc[b], s[b], k, where=f"b={b}")
+    idx0, sc0, ds0 = _run(msa, dims, QR, None, KR, doc_off, k, msa.AGG_MAX, cuda_device)
+    assert np.array_equal(ds, ds0) and np.array_equal(idx, idx0) and np.array_equal(sc, sc0)
 
 
 def test_route_edge_shapes(msa, cuda_device):
