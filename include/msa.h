@@ -123,8 +123,11 @@ msa_status msa_encode_memory(const msa_dims* dims, const void* H, int64_t T, con
  * Pages: IRMaD "M. Materials & Methods", routing item:
  *   Q^R = H_q W^QR;  S_ij = max_t mean_h cos(Q^R_h, K̄^R_ij,h);
  *   s_i = max_j S_ij;  I = Top-k({s_i});  k = 16 on the pages.
- *   Hq       [B, hidden] bf16 query hidden states, or, when W_QR == NULL,
- *            [B, n_r * d_r] bf16 router queries Q^R given directly.
+ *   q_tokens M >= 1 tokens per query (the t of max_t): row b * M + t of Hq is
+ *            token t of query b.  A query's chunk score is the largest over its
+ *            tokens of the head-mean cosine.
+ *   Hq       [B * M, hidden] bf16 query hidden states, or, when W_QR == NULL,
+ *            [B * M, n_r * d_r] bf16 router queries Q^R given directly.
  *   W_QR     [hidden, n_r * d_r] bf16 or NULL.
  *   KR_bar   pooled router keys, bf16: [n_chunks, n_r, d_r] for kr_layout 0, or
  *            head-major [n_r, n_chunks, d_r] for kr_layout 1 (each head's keys contiguous:
@@ -133,16 +136,16 @@ msa_status msa_encode_memory(const msa_dims* dims, const void* H, int64_t T, con
  *   doc_scores [B, n_docs] fp32 out, optional (NULL = not written).
  *   topk_idx [B, k] int32 out: document ids, descending score, ties to the
  *            lower id.  topk_score [B, k] fp32 out: their scores.
- * Cosines use norms clamped below at 1e-12 (a zero vector scores 0).  One
- * query token per row of Hq (the max over t is over that single token).
- * Limits: 1 <= k <= min(n_docs, 256); 1 <= B; n_r <= 8; d_r in {64, 128}.
+ * Cosines use norms clamped below at 1e-12 (a zero vector scores 0).
+ * Limits: 1 <= k <= min(n_docs, 256); 1 <= B; 1 <= M; B * M <= 65535; n_r <= 8;
+ * d_r in {64, 128}.
  * Rounding: Q^R in fp32; the cosine dot products run on the tensor cores with
  * the normalised query split into two bf16 terms (hi + lo) and fp32
  * accumulation, so scores carry ~1e-6 relative error.
  * ------------------------------------------------------------------------- */
-size_t msa_route_workspace_size(const msa_dims* dims, int32_t B, int32_t n_docs, int32_t n_chunks,
-                                int32_t k, msa_doc_agg agg);
-msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR, int32_t B,
+size_t msa_route_workspace_size(const msa_dims* dims, int32_t B, int32_t q_tokens, int32_t n_docs,
+                                int32_t n_chunks, int32_t k, msa_doc_agg agg);
+msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR, int32_t B, int32_t q_tokens,
                           const void* KR_bar, const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks,
                           int32_t k, msa_doc_agg agg, int32_t kr_layout, float* doc_scores, int32_t* topk_idx,
                           float* topk_score, void* ws, size_t ws_bytes, void* stream);
@@ -180,7 +183,7 @@ msa_status msa_topk_merge(const float* cand_score, const int32_t* cand_idx, int3
  * or allocating library routine is called.
  * ------------------------------------------------------------------------- */
 msa_status msa_route_topk_static(const msa_dims* dims, const void* Hq, const void* W_QR, int32_t B,
-                                 const void* KR_bar, const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks,
+                                 int32_t q_tokens, const void* KR_bar, const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks,
                                  int32_t k, msa_doc_agg agg, float* doc_scores, int32_t* topk_idx,
                                  float* topk_score, void* stream);
 
@@ -190,8 +193,11 @@ msa_status msa_route_topk_static(const msa_dims* dims, const void* Hq, const voi
  * K_q], V_ctx likewise, Output = Attention(Q_q, K_ctx, V_ctx)) and position item
  * (global RoPE on the active context, offset by k); project overview "key
  * technical details" 1.
- *   q        [B, n_q, head_dim] bf16, before RoPE; rotated to position
- *            pos_offset + loc_len[b] - 1 (the decode token is the last local token).
+ *   q_tokens M >= 1 query tokens per query: the last M local tokens (M = 1 is
+ *            the decode step; M > 1 the query-prefill step of the same call).
+ *   q        [B, M, n_q, head_dim] bf16, before RoPE; token t is rotated to
+ *            position pos_offset + loc_len[b] - M + t (the query tokens are the
+ *            last M local tokens).
  *   K_bar, V_bar [n_chunks, n_kv, head_dim] bf16 pooled memory (device).
  *   chunk_off[n_docs + 1] device int32; topk_idx [B, k] device int32 doc ids.
  *   K_loc, V_loc [B, t_loc_max, n_kv, head_dim] bf16 local KV, K before RoPE;
@@ -202,16 +208,18 @@ msa_status msa_route_topk_static(const msa_dims* dims, const void* Hq, const voi
  *              1: K_loc already holds every local key rotated at pos_offset + j
  *              (see msa_rope_rows); rope_cache is then unused.
  *   softmax_scale  0 -> 1/sqrt(head_dim).
- *   out      [B, n_q, head_dim] bf16.
- * Query head g attends with KV head g / (n_q / n_kv).  No mask: the decode
- * token sees every gathered chunk and every local token.  Pooled keys keep
- * their document-wise rotation only.  Rounding: q is rotated and scaled in
+ *   out      [B, M, n_q, head_dim] bf16.
+ * Limits: 1 <= M, B * M <= 65535.
+ * Query head g attends with KV head g / (n_q / n_kv).  Every query token sees
+ * every gathered chunk; token t sees the local tokens j <= loc_len[b] - M + t
+ * (causal; for M = 1 that is every local token).  Pooled keys keep their
+ * document-wise rotation only.  Rounding: q is rotated and scaled in
  * fp32 then rounded to bf16; local keys are rotated in fp32 and rounded to
  * bf16; products and softmax in fp32.
  * ------------------------------------------------------------------------- */
-size_t msa_attend_workspace_size(const msa_dims* dims, int32_t B, int32_t k, int32_t t_loc_max,
-                                 int32_t pos_offset);
-msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, const void* K_bar,
+size_t msa_attend_workspace_size(const msa_dims* dims, int32_t B, int32_t q_tokens, int32_t k,
+                                 int32_t t_loc_max, int32_t pos_offset);
+msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, int32_t q_tokens, const void* K_bar,
                              const void* V_bar, const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks,
                              const int32_t* topk_idx, int32_t k, const void* K_loc, const void* V_loc,
                              const int32_t* loc_len, int32_t t_loc_max, int32_t pos_offset,

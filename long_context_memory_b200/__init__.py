@@ -64,10 +64,11 @@ def _load():
         "msa_chunk_offsets": (I32, [P, I32, I32, P, ctypes.POINTER(I32)]),
         "msa_encode_workspace_size": (SZ, [DP, I64, I32, I32]),
         "msa_encode_memory": (I32, [DP, P, I64, P, I32, P, I32, P, P, P, P, P, P, I32, P, SZ, P]),
-        "msa_route_workspace_size": (SZ, [DP, I32, I32, I32, I32, I32]),
-        "msa_route_topk": (I32, [DP, P, P, I32, P, P, I32, I32, I32, I32, I32, P, P, P, P, SZ, P]),
-        "msa_attend_workspace_size": (SZ, [DP, I32, I32, I32, I32]),
-        "msa_sparse_attend": (I32, [DP, P, I32, P, P, P, I32, I32, P, I32, P, P, P, I32, I32, P, I32, F, P, P, SZ, P]),
+        "msa_route_workspace_size": (SZ, [DP, I32, I32, I32, I32, I32, I32]),
+        "msa_route_topk": (I32, [DP, P, P, I32, I32, P, P, I32, I32, I32, I32, I32, P, P, P, P, SZ, P]),
+        "msa_attend_workspace_size": (SZ, [DP, I32, I32, I32, I32, I32]),
+        "msa_sparse_attend": (I32, [DP, P, I32, I32, P, P, P, I32, I32, P, I32, P, P, P, I32, I32, P, I32, F, P, P, SZ,
+                                    P]),
         "msa_rope_rows": (I32, [DP, P, I32, I32, P, P]),
         "msa_gather_kv": (I32, [DP, P, P, I32, P, I32, P, I32, I32, P, P, I32, P, P, P, SZ, P]),
         "msa_rope_cache_size": (SZ, [DP, I32]),
@@ -187,30 +188,35 @@ def encode_memory(dims, H, doc_off, chunk_off, n_chunks: int, W_K, W_V, W_KR, ou
 # ----------------------------------------------------------------------------
 # stage 2
 # ----------------------------------------------------------------------------
-def route_workspace_size(dims, B: int, n_docs: int, n_chunks: int, k: int, agg: int = AGG_MAX) -> int:
-    return int(lib.msa_route_workspace_size(ctypes.byref(Dims.of(dims)), B, n_docs, n_chunks, k, agg))
+def route_workspace_size(dims, B: int, n_docs: int, n_chunks: int, k: int, agg: int = AGG_MAX,
+                         q_tokens: int = 1) -> int:
+    return int(lib.msa_route_workspace_size(ctypes.byref(Dims.of(dims)), B, q_tokens, n_docs, n_chunks, k, agg))
 
 
 def route_topk(dims, Hq, W_QR, KR_bar, chunk_off, k: int, agg: int = AGG_MAX, want_doc_scores: bool = False,
-               out=None, ws=None, stream=None, kr_head_major: bool = False):
+               out=None, ws=None, stream=None, kr_head_major: bool = False, q_tokens: int = 1):
     """Top-k documents per query.  Returns (topk_idx [B,k] int32, topk_score [B,k] fp32, doc_scores|None).
 
-    ``W_QR=None`` means ``Hq`` already holds the router queries Q^R [B, n_r*d_r].
+    ``Hq`` holds B * q_tokens rows (token t of query b at row b * q_tokens + t); a chunk's
+    score for a query is the largest over its tokens.
+    ``W_QR=None`` means ``Hq`` already holds the router queries Q^R [B * q_tokens, n_r*d_r].
     ``kr_head_major``: KR_bar is [n_r, C, d_r] instead of [C, n_r, d_r].
     """
     import torch
 
     dd = Dims.of(dims)
-    B = Hq.shape[0]
+    if Hq.shape[0] % q_tokens:
+        raise ValueError(f"Hq has {Hq.shape[0]} rows, not a multiple of q_tokens={q_tokens}")
+    B = Hq.shape[0] // q_tokens
     n_docs = chunk_off.numel() - 1
     n_chunks = KR_bar.shape[1] if kr_head_major else KR_bar.shape[0]
     dev = KR_bar.device
     if out is None:
         out = (torch.empty((B, k), dtype=torch.int32, device=dev), torch.empty((B, k), dtype=torch.float32, device=dev),
                torch.empty((B, n_docs), dtype=torch.float32, device=dev) if want_doc_scores else None)
-    nbytes = route_workspace_size(dims, B, n_docs, n_chunks, k, agg)
+    nbytes = route_workspace_size(dims, B, n_docs, n_chunks, k, agg, q_tokens)
     ws = _workspace(nbytes, dev, ws)
-    _check(lib.msa_route_topk(ctypes.byref(dd), _ptr(Hq), _ptr(W_QR), B, _ptr(KR_bar), _ptr(chunk_off), n_docs,
+    _check(lib.msa_route_topk(ctypes.byref(dd), _ptr(Hq), _ptr(W_QR), B, q_tokens, _ptr(KR_bar), _ptr(chunk_off), n_docs,
                               n_chunks, k, agg, int(bool(kr_head_major)), _ptr(out[2]), _ptr(out[0]), _ptr(out[1]), _aligned_ptr(ws), nbytes,
                               _stream(stream)))
     return out
@@ -231,8 +237,8 @@ def topk_merge(cand_score, cand_idx, k: int, out=None, stream=None):
 # ----------------------------------------------------------------------------
 # stage 3
 # ----------------------------------------------------------------------------
-def attend_workspace_size(dims, B: int, k: int, t_loc_max: int, pos_offset: int) -> int:
-    return int(lib.msa_attend_workspace_size(ctypes.byref(Dims.of(dims)), B, k, t_loc_max, pos_offset))
+def attend_workspace_size(dims, B: int, k: int, t_loc_max: int, pos_offset: int, q_tokens: int = 1) -> int:
+    return int(lib.msa_attend_workspace_size(ctypes.byref(Dims.of(dims)), B, q_tokens, k, t_loc_max, pos_offset))
 
 
 def rope_cache_build(dims, t_loc_max: int, pos_offset: int, device=None, out=None, stream=None):
@@ -279,22 +285,25 @@ def rope_rows(dims, x, positions, stream=None):
 def sparse_attend(dims, q, K_bar, V_bar, chunk_off, topk_idx, K_loc, V_loc, loc_len, pos_offset: int,
                   softmax_scale: float = 0.0, out=None, ws=None, stream=None, rope_cache=None,
                   k_loc_rotated: bool = False):
-    """One GQA decode step over [selected docs' K̄; local K].  Returns out [B, n_q, head_dim] bf16.
+    """GQA attention of the query tokens over [selected docs' K̄; local K].
 
+    ``q`` is [B, n_q, head_dim] (one decode token) or [B, M, n_q, head_dim] (the last M local
+    tokens, causal among the local keys); ``out`` has the shape of ``q``.
     ``rope_cache`` (from ``rope_cache_build`` with the same pos_offset and t_loc_max) skips
     rebuilding the local-position rotation table."""
     import torch
 
     dd = Dims.of(dims)
     B, k = topk_idx.shape
+    M = q.shape[1] if q.dim() == 4 else 1
     t_loc_max = K_loc.shape[1] if K_loc is not None else 0
     n_docs = chunk_off.numel() - 1
     dev = q.device
     if out is None:
-        out = torch.empty((B, dims.n_q, dims.head_dim), dtype=torch.bfloat16, device=dev)
-    nbytes = attend_workspace_size(dims, B, k, t_loc_max, pos_offset)
+        out = torch.empty(tuple(q.shape), dtype=torch.bfloat16, device=dev)
+    nbytes = attend_workspace_size(dims, B, k, t_loc_max, pos_offset, M)
     ws = _workspace(nbytes, dev, ws)
-    _check(lib.msa_sparse_attend(ctypes.byref(dd), _ptr(q), B, _ptr(K_bar), _ptr(V_bar), _ptr(chunk_off), n_docs,
+    _check(lib.msa_sparse_attend(ctypes.byref(dd), _ptr(q), B, M, _ptr(K_bar), _ptr(V_bar), _ptr(chunk_off), n_docs,
                                  K_bar.shape[0], _ptr(topk_idx), k, _ptr(K_loc), _ptr(V_loc), _ptr(loc_len),
                                  t_loc_max, pos_offset, _ptr(rope_cache), int(bool(k_loc_rotated)),
                                  float(softmax_scale), _ptr(out),

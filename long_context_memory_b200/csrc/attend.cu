@@ -69,6 +69,9 @@ struct AttnParams {
   float* part_ml;
   float* part_o;
   int n_q, n_kv, k, n_docs, t_loc_max, pos_offset, n_splits, n_stages;
+  int q_tokens;      // M: query tokens per query (the last M local tokens)
+  int tok_per_cta;   // MT: tokens per CTA, MT * G <= 16 mma rows
+  int n_tgroups;     // ceil(M / MT)
   float scale_log2;  // softmax scale * log2(e)
   RopeTurns turns;   // RoPE frequencies as 64-bit fractions of a turn
 };
@@ -77,7 +80,7 @@ struct AttnParams {
 //   stage s: K rows [kTK][krow] | V rows [kTK][krow] | RoPE rows [kTK][D/2] (cos, sin)
 //   krow = n_kv * D * 2 + 16 bytes: one key's rows of every KV head, padded so
 //   that consecutive rows start one 16-byte unit apart (conflict-free ldmatrix)
-//   then barriers, the segment table, the query's cos/sin and the raw query.
+//   then barriers, the segment table, the query tokens' cos/sin and raw rows.
 struct AttnSmem {
   int krow, kbytes, tbytes, stage_bytes, n_stages;
   __host__ __device__ AttnSmem(int n_kv, int D, int stages, bool table) {
@@ -87,10 +90,12 @@ struct AttnSmem {
     stage_bytes = 2 * kbytes + tbytes;
     n_stages = stages;
   }
-  __host__ __device__ size_t fixed_bytes(int n_q, int D) const {
-    return 2 * kMaxStages * 8 + (2 * kMaxK + 2) * 4 + (size_t)(D / 2) * 8 + (size_t)n_q * D * 2;
+  __host__ __device__ size_t fixed_bytes(int n_q, int D, int mt) const {
+    return 2 * kMaxStages * 8 + (2 * kMaxK + 2) * 4 + (size_t)mt * (D / 2) * 8 + (size_t)mt * n_q * D * 2;
   }
-  __host__ __device__ size_t total(int n_q, int D) const { return (size_t)n_stages * stage_bytes + fixed_bytes(n_q, D); }
+  __host__ __device__ size_t total(int n_q, int D, int mt) const {
+    return (size_t)n_stages * stage_bytes + fixed_bytes(n_q, D, mt);
+  }
 };
 
 template <int D>
@@ -104,14 +109,18 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
   // offsets: every region below starts on a 16-byte boundary (stage rows, query rows and
   // the RoPE rows are bulk-copy or 16-byte vector destinations)
   uint8_t* stage_mem = sm;
-  uint16_t* qsm = reinterpret_cast<uint16_t*>(sm + (size_t)L_.n_stages * L_.stage_bytes);  // [n_q][D] raw query
-  uint64_t* bars = reinterpret_cast<uint64_t*>(qsm + (size_t)p.n_q * D);  // [stage] tile landed
+  const int MT = p.tok_per_cta;
+  uint16_t* qsm = reinterpret_cast<uint16_t*>(sm + (size_t)L_.n_stages * L_.stage_bytes);  // [MT][n_q][D] raw query
+  uint64_t* bars = reinterpret_cast<uint64_t*>(qsm + (size_t)MT * p.n_q * D);  // [stage] tile landed
   uint64_t* ebars = bars + kMaxStages;                                      // [stage] every warp done with it
   int* seg_v = reinterpret_cast<int*>(ebars + kMaxStages);  // [k + 1] virtual starts
   int* seg_c = seg_v + kMaxK + 2;                          // [k] chunk starts
-  float2* qcs = reinterpret_cast<float2*>(seg_c + kMaxK);  // [D/2] cos/sin at the query position
+  float2* qcs = reinterpret_cast<float2*>(seg_c + kMaxK);  // [MT][D/2] cos/sin at the tokens' positions
 
-  const int split = blockIdx.x, b = blockIdx.y;
+  const int split = blockIdx.x;
+  const int b = blockIdx.y / p.n_tgroups;                       // query
+  const int t0 = (blockIdx.y % p.n_tgroups) * MT;               // first token of this CTA
+  const int nt = min(MT, p.q_tokens - t0);                      // tokens of this CTA
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = warp;               // the KV head this warp serves (warps 0 .. n_kv-1)
   const bool producer = warp == n_kv;  // the last warp only streams tiles in
@@ -144,8 +153,8 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
     seg_v[r + 1] = n;
   }
   {
-    const uint4* qg = reinterpret_cast<const uint4*>(p.q + (size_t)b * p.n_q * D);
-    for (int i = tid; i < p.n_q * D / 8; i += blockDim.x) reinterpret_cast<uint4*>(qsm)[i] = __ldg(qg + i);
+    const uint4* qg = reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.q_tokens + t0) * p.n_q * D);
+    for (int i = tid; i < nt * p.n_q * D / 8; i += blockDim.x) reinterpret_cast<uint4*>(qsm)[i] = __ldg(qg + i);
   }
   int L = p.loc_len[b];
   L = max(0, min(L, p.t_loc_max));
@@ -228,33 +237,37 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
     return;  // the compute warps no longer synchronise with the whole block
   }
 
-  // ---- query fragments of this warp's GQA group: rotate to pos_offset + L - 1, scale, bf16 ----
+  // ---- query fragments of this warp's GQA group: mma row = tt * G + gg (token t0 + tt,
+  //      q head h * G + gg); token t sits at pos_offset + L - M + t; scale, bf16 ----
   const int n_compute = 32 * n_kv;
-  for (int i = tid; i < D / 2; i += n_compute) qcs[i] = rope_cos_sin(p.turns, i, (int64_t)p.pos_offset + L - 1);
+  const int64_t pos_q0 = (int64_t)p.pos_offset + L - p.q_tokens + t0;
+  for (int i = tid; i < nt * (D / 2); i += n_compute)
+    qcs[i] = rope_cos_sin(p.turns, i % (D / 2), pos_q0 + i / (D / 2));
   named_bar_sync(1, n_compute);
   const int g = lane >> 2, c = lane & 3;
   uint32_t qa[KS][4];
   {
-    const uint16_t* qb = qsm + (size_t)h * G * D;
 #pragma unroll
     for (int s = 0; s < KS; ++s) {
 #pragma unroll
       for (int rr = 0; rr < 2; ++rr) {        // rows g and g + 8
         const int row = g + 8 * rr;
+        const int tt = row / G, gg = row - tt * G;
+        const uint16_t* qb = qsm + ((size_t)tt * p.n_q + h * G + gg) * D;
 #pragma unroll
         for (int hk = 0; hk < 2; ++hk) {      // k cols 2c.. and 2c+8..
           const int dim = 16 * s + 8 * hk + 2 * c;
           float v[2] = {0.f, 0.f};
-          if (row < G) {
+          if (tt < nt) {
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
               const int dd = dim + e;
               const bool first = dd < D / 2;
               const int i = first ? dd : dd - D / 2;
               const int partner = first ? dd + D / 2 : dd - D / 2;
-              const float x = bf16_bits_to_float(qb[row * D + dd]);
-              const float y = bf16_bits_to_float(qb[row * D + partner]);
-              const float2 cs = qcs[i];
+              const float x = bf16_bits_to_float(qb[dd]);
+              const float y = bf16_bits_to_float(qb[partner]);
+              const float2 cs = qcs[tt * (D / 2) + i];
               // first half: x cos - y sin; second half: x cos + y sin (y = first-half partner)
               const float rot = first ? (x * cs.x - y * cs.y) : (x * cs.x + y * cs.y);
               v[e] = rot * p.scale_log2;
@@ -272,6 +285,13 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
   float m_run[2] = {-INFINITY, -INFINITY};
   float l_run[2] = {0.f, 0.f};
   const int hoff = h * D * 2;  // this head's bytes within a key row
+  // causal limit of rows g and g + 8: token t sees the chunks and local tokens j <= L - M + t
+  int lim[2];
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr) {
+    const int tt = (g + 8 * rr) / G;
+    lim[rr] = tt < nt ? n_sel + max(0, min(L, L - p.q_tokens + t0 + tt + 1)) : v1;
+  }
 
   for (int t = 0; t < n_tiles; ++t) {
     const int st = t % L_.n_stages;
@@ -331,10 +351,8 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int v = tv0 + 8 * nb + 2 * c + e;
-        if (v >= v1) {
-          sc[nb][e] = -INFINITY;
-          sc[nb][2 + e] = -INFINITY;
-        }
+        if (v >= v1 || v >= lim[0]) sc[nb][e] = -INFINITY;
+        if (v >= v1 || v >= lim[1]) sc[nb][2 + e] = -INFINITY;
       }
     // ---- online softmax (rows g and g + 8) ----
     float alpha[2];
@@ -394,8 +412,9 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
 #pragma unroll
   for (int rr = 0; rr < 2; ++rr) {
     const int row = g + 8 * rr;
-    if (row < G) {
-      const size_t qh = (size_t)b * p.n_q + (size_t)h * G + row;
+    const int tt = row / G;
+    if (tt < nt) {
+      const size_t qh = ((size_t)b * p.q_tokens + t0 + tt) * p.n_q + (size_t)h * G + (row - tt * G);
       float* po = p.part_o + (qh * p.n_splits + split) * D;
 #pragma unroll
       for (int n = 0; n < NBLK; ++n)
@@ -472,14 +491,17 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
   }
 }
 
-int stages_that_fit(int n_kv, int n_q, int D, bool table) {
+int stages_that_fit(int n_kv, int n_q, int D, bool table, int mt) {
   const int budget = 210 * 1024;
   for (int st = kMaxStages; st >= 2; --st) {
     AttnSmem L(n_kv, D, st, table);
-    if (L.total(n_q, D) <= (size_t)budget) return st;
+    if (L.total(n_q, D, mt) <= (size_t)budget) return st;
   }
   return 2;
 }
+
+// query tokens per CTA: as many as fill the 16 mma rows of a warp (GQA group G each)
+int tokens_per_cta(const msa_dims& d, int M) { return std::max(1, std::min(M, 16 / (d.n_q / d.n_kv))); }
 
 // rotate rows of x [rows, heads, D] in place: pair (i, i + D/2) of row r by pos[r] * theta_i
 template <int D>
@@ -619,14 +641,17 @@ __global__ void __launch_bounds__(256) gather_copy_kernel(const uint4* __restric
 
 }  // namespace
 
-size_t attend_workspace(const msa_dims& d, int B, int k, int t_loc_max, int pos_offset, void* ws, AttendWs* out) {
+size_t attend_workspace(const msa_dims& d, int B, int M, int k, int t_loc_max, int pos_offset, void* ws,
+                        AttendWs* out) {
   (void)pos_offset;
   Carver cv(ws);
   AttendWs w{};
-  w.n_splits = choose_splits(B, t_loc_max, k);
+  const int mt = tokens_per_cta(d, M);
+  const int n_tg = (M + mt - 1) / mt;
+  w.n_splits = choose_splits(B * n_tg, t_loc_max, k);
   w.rope_tab = cv.take<float2>((size_t)std::max(1, t_loc_max) * (d.head_dim / 2));
-  w.part_ml = cv.take<float>((size_t)B * d.n_q * w.n_splits * 2);
-  w.part_o = cv.take<float>((size_t)B * d.n_q * w.n_splits * d.head_dim);
+  w.part_ml = cv.take<float>((size_t)B * M * d.n_q * w.n_splits * 2);
+  w.part_o = cv.take<float>((size_t)B * M * d.n_q * w.n_splits * d.head_dim);
   if (out) *out = w;
   return cv.size();
 }
@@ -678,13 +703,13 @@ msa_status rope_rows_launch(const msa_dims& d, void* x, int rows, int heads, con
   return MSA_OK;
 }
 
-msa_status attend_launch(const msa_dims& d, const void* q, int B, const void* K_bar, const void* V_bar,
+msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const void* K_bar, const void* V_bar,
                          const int32_t* chunk_off, int n_docs, const int32_t* topk_idx, int k, const void* K_loc,
                          const void* V_loc, const int32_t* loc_len, int t_loc_max, int pos_offset,
                          const void* rope_cache, int k_loc_rotated, float scale, void* out, void* ws,
                          cudaStream_t s) {
   AttendWs w;
-  attend_workspace(d, B, k, t_loc_max, pos_offset, ws, &w);
+  attend_workspace(d, B, M, k, t_loc_max, pos_offset, ws, &w);
   const int D = d.head_dim;
   const float2* tab = k_loc_rotated ? nullptr : static_cast<const float2*>(rope_cache);
   if (!tab && !k_loc_rotated && t_loc_max > 0) {
@@ -711,13 +736,16 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, const void* K_
   p.t_loc_max = t_loc_max;
   p.pos_offset = pos_offset;
   p.n_splits = w.n_splits;
+  p.q_tokens = M;
+  p.tok_per_cta = tokens_per_cta(d, M);
+  p.n_tgroups = (M + p.tok_per_cta - 1) / p.tok_per_cta;
   p.scale_log2 = (scale > 0.f ? scale : 1.0f / std::sqrt((float)D)) * kLog2e;
   rope_turns(d, p.turns.f);
-  p.n_stages = stages_that_fit(d.n_kv, d.n_q, D, tab != nullptr);
+  p.n_stages = stages_that_fit(d.n_kv, d.n_q, D, tab != nullptr, p.tok_per_cta);
   {
     TraceScope ts(kKAttnSplit, s);
-    dim3 grid(w.n_splits, B);
-    const size_t sm = AttnSmem(d.n_kv, D, p.n_stages, tab != nullptr).total(d.n_q, D);
+    dim3 grid(w.n_splits, B * p.n_tgroups);
+    const size_t sm = AttnSmem(d.n_kv, D, p.n_stages, tab != nullptr).total(d.n_q, D, p.tok_per_cta);
     if (D == 128) {
       MSA_CUDA_CHECK(cudaFuncSetAttribute(attn_split_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
       MSA_CUDA_CHECK(launch_pdl(attn_split_kernel<128>, grid, dim3(32 * (d.n_kv + 1)), sm, s, p));
@@ -728,7 +756,7 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, const void* K_
   }
   {
     TraceScope ts(kKAttnCombine, s);
-    dim3 grid(d.n_q, B);
+    dim3 grid(d.n_q, B * M);
     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
     if (D == 128)
       MSA_CUDA_CHECK(launch_pdl(attn_combine_kernel<128>, grid, dim3(256), 0, s, (const float*)w.part_ml,

@@ -115,9 +115,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // ---------------------------------------------------------------------------
 // stage implementations (route.cu, attend.cu, encode.cu)
 // ---------------------------------------------------------------------------
-size_t route_workspace(const msa_dims& d, int B, int n_docs, int n_chunks, int k, msa_doc_agg agg,
+size_t route_workspace(const msa_dims& d, int B, int M, int n_docs, int n_chunks, int k, msa_doc_agg agg,
                        void* ws, struct RouteWs* out);
-msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int B, const void* KR_bar,
+msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int B, int M, const void* KR_bar,
                         const int32_t* chunk_off, int n_docs, int n_chunks, int k, msa_doc_agg agg, int kr_layout,
                         float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws,
                         cudaStream_t s);
@@ -125,9 +125,9 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
 msa_status topk_merge_launch(const float* cand_score, const int32_t* cand_idx, int B, int n_cand, int k,
                              int32_t* topk_idx, float* topk_score, cudaStream_t s);
 
-size_t attend_workspace(const msa_dims& d, int B, int k, int t_loc_max, int pos_offset, void* ws,
+size_t attend_workspace(const msa_dims& d, int B, int M, int k, int t_loc_max, int pos_offset, void* ws,
                         struct AttendWs* out);
-msa_status attend_launch(const msa_dims& d, const void* q, int B, const void* K_bar, const void* V_bar,
+msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const void* K_bar, const void* V_bar,
                          const int32_t* chunk_off, int n_docs, const int32_t* topk_idx, int k,
                          const void* K_loc, const void* V_loc, const int32_t* loc_len, int t_loc_max,
                          int pos_offset, const void* rope_cache, int k_loc_rotated, float scale, void* out,

@@ -255,13 +255,14 @@ msa_status msa_chunk_offsets(const int64_t* doc_off_host, int32_t n_docs, int32_
 }
 
 // ------------------------------ routing ------------------------------
-size_t msa_route_workspace_size(const msa_dims* dims, int32_t B, int32_t n_docs, int32_t n_chunks, int32_t k,
-                                msa_doc_agg agg) {
-  if (!dims || B < 1 || n_docs < 1 || n_chunks < 1 || k < 1) return 0;
-  return route_workspace(*dims, B, n_docs, n_chunks, k, agg, nullptr, nullptr);
+size_t msa_route_workspace_size(const msa_dims* dims, int32_t B, int32_t q_tokens, int32_t n_docs, int32_t n_chunks,
+                                int32_t k, msa_doc_agg agg) {
+  if (!dims || B < 1 || q_tokens < 1 || (int64_t)B * q_tokens > 65535 || n_docs < 1 || n_chunks < 1 || k < 1) return 0;
+  return route_workspace(*dims, B, q_tokens, n_docs, n_chunks, k, agg, nullptr, nullptr);
 }
 
-msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR, int32_t B, const void* KR_bar,
+msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR, int32_t B, int32_t q_tokens,
+                          const void* KR_bar,
                           const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks, int32_t k, msa_doc_agg agg,
                           int32_t kr_layout, float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws, size_t ws_bytes,
                           void* stream) {
@@ -270,6 +271,8 @@ msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR
   if (W_QR && (dims->hidden < 64 || dims->hidden % 64 != 0 || dims->hidden > 8192))
     return fail(MSA_ERR_UNSUPPORTED, "hidden must be a multiple of 64 in [64, 8192] (got %d)", dims->hidden);
   if (B < 1) return fail(MSA_ERR_INVALID_ARG, "B must be >= 1 (got %d)", B);
+  if (q_tokens < 1 || (int64_t)B * q_tokens > 65535)
+    return fail(MSA_ERR_INVALID_ARG, "q_tokens must be >= 1 with B * q_tokens <= 65535 (got %d, B %d)", q_tokens, B);
   if (n_docs < 1 || n_chunks < n_docs)
     return fail(MSA_ERR_INVALID_ARG, "need 1 <= n_docs <= n_chunks (got %d, %d)", n_docs, n_chunks);
   if (k < 1 || k > n_docs || k > 256)
@@ -285,12 +288,12 @@ msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR
   CHECK_OPT_PTR(doc_scores);
   CHECK_PTR(topk_idx);
   CHECK_PTR(topk_score);
-  const size_t need = route_workspace(*dims, B, n_docs, n_chunks, k, agg, nullptr, nullptr);
+  const size_t need = route_workspace(*dims, B, q_tokens, n_docs, n_chunks, k, agg, nullptr, nullptr);
   if (ws_bytes < need) return fail(MSA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
   if (need && (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)))
     return fail(MSA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
   if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
-  return route_launch(*dims, Hq, W_QR, B, KR_bar, chunk_off, n_docs, n_chunks, k, agg, kr_layout, doc_scores, topk_idx,
+  return route_launch(*dims, Hq, W_QR, B, q_tokens, KR_bar, chunk_off, n_docs, n_chunks, k, agg, kr_layout, doc_scores, topk_idx,
                       topk_score, ws, static_cast<cudaStream_t>(stream));
 }
 
@@ -309,12 +312,15 @@ msa_status msa_topk_merge(const float* cand_score, const int32_t* cand_idx, int3
 }
 
 // ------------------------------ attention ------------------------------
-size_t msa_attend_workspace_size(const msa_dims* dims, int32_t B, int32_t k, int32_t t_loc_max, int32_t pos_offset) {
-  if (!dims || B < 1 || k < 1 || t_loc_max < 0) return 0;
-  return attend_workspace(*dims, B, k, t_loc_max, pos_offset, nullptr, nullptr);
+size_t msa_attend_workspace_size(const msa_dims* dims, int32_t B, int32_t q_tokens, int32_t k, int32_t t_loc_max,
+                                 int32_t pos_offset) {
+  if (!dims || B < 1 || q_tokens < 1 || (int64_t)B * q_tokens > 65535 || k < 1 || t_loc_max < 0) return 0;
+  if (dims->n_kv < 1 || dims->n_q < dims->n_kv) return 0;
+  return attend_workspace(*dims, B, q_tokens, k, t_loc_max, pos_offset, nullptr, nullptr);
 }
 
-msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, const void* K_bar, const void* V_bar,
+msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, int32_t q_tokens, const void* K_bar,
+                             const void* V_bar,
                              const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks, const int32_t* topk_idx,
                              int32_t k, const void* K_loc, const void* V_loc, const int32_t* loc_len,
                              int32_t t_loc_max, int32_t pos_offset, const void* rope_cache,
@@ -323,6 +329,8 @@ msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, con
   msa_status st = check_dims(dims, true, false);
   if (st != MSA_OK) return st;
   if (B < 1) return fail(MSA_ERR_INVALID_ARG, "B must be >= 1 (got %d)", B);
+  if (q_tokens < 1 || (int64_t)B * q_tokens > 65535)
+    return fail(MSA_ERR_INVALID_ARG, "q_tokens must be >= 1 with B * q_tokens <= 65535 (got %d, B %d)", q_tokens, B);
   if (n_docs < 1 || n_chunks < n_docs)
     return fail(MSA_ERR_INVALID_ARG, "need 1 <= n_docs <= n_chunks (got %d, %d)", n_docs, n_chunks);
   if (k < 1 || k > n_docs || k > 256)
@@ -344,12 +352,12 @@ msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, con
   CHECK_PTR(loc_len);
   CHECK_OPT_PTR(rope_cache);
   CHECK_PTR(out);
-  const size_t need = attend_workspace(*dims, B, k, t_loc_max, pos_offset, nullptr, nullptr);
+  const size_t need = attend_workspace(*dims, B, q_tokens, k, t_loc_max, pos_offset, nullptr, nullptr);
   if (ws_bytes < need) return fail(MSA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
   if (need && (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)))
     return fail(MSA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
   if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
-  return attend_launch(*dims, q, B, K_bar, V_bar, chunk_off, n_docs, topk_idx, k, K_loc, V_loc, loc_len, t_loc_max,
+  return attend_launch(*dims, q, B, q_tokens, K_bar, V_bar, chunk_off, n_docs, topk_idx, k, K_loc, V_loc, loc_len, t_loc_max,
                        pos_offset, rope_cache, k_loc_rotated, softmax_scale, out, ws,
                        static_cast<cudaStream_t>(stream));
 }

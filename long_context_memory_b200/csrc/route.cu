@@ -8,9 +8,10 @@
 // with the memory size (complexity item of the same section: O(ML/P)).
 //
 // Kernels, in launch order:
-//   router_query_kernel  Q^R = H_q W^QR (each CTA 8 columns over the whole hidden
-//                    dimension), per-head normalisation by the head's last CTA,
-//                    bf16 hi + lo rows for the scan's TMA; clears the doc keys
+//   router_query_kernel  Q^R = H_q W^QR (CTA = a row slab of one head's columns,
+//                    split-K partials summed in a fixed order by the head's
+//                    last CTA), per-head normalisation, bf16 hi + lo rows for
+//                    the scan's TMA; clears the doc keys
 //   scan_kernel      TMA-staged streaming scan of K̄^R: tensor-core dots and
 //                    Gram diagonal (norm), cosine, head mean, per-document
 //                    segmented max folded in with atomicMax on ordered keys
@@ -31,13 +32,13 @@
 namespace msa {
 
 struct RouteWs {
-  float* qr;          // [B][NR] fp32 router queries (W_QR given)
+  float* qr;          // [rq_splits][B][NR] fp32 partial router queries (W_QR given)
   uint32_t* head_done;  // [n_r] CTAs finished per router head (back to 0 after each call)
   __nv_bfloat16* q_hl; // [passes][n_r][2][NQ][d_r] normalised query, bf16 hi and lo terms
   uint32_t* doc_key;  // [B][n_docs] ordered-uint32 doc max (MAX)
-  float* chunk_s;     // [B][n_chunks] chunk scores (MEAN)
+  uint32_t* chunk_k;  // [B][n_chunks] ordered chunk scores (MEAN)
   uint64_t* cand;     // [B][n_slices][k] slice winners
-  int nq, passes, n_slices;
+  int nq, passes, n_slices, rq_splits;
 };
 
 namespace {
@@ -49,133 +50,197 @@ constexpr float kEps = 1e-12f;
 // --------------------------------------------------------------------------
 // Router query, one kernel: Q^R = H_q W^QR, per-head normalisation, bf16 hi + lo
 // terms in the layout the scan's TMA reads (q_hl[pass][head][hi|lo][NQ rows][d_r];
-// rows of padding queries are zero), and the clearing of the document keys.
-// CTA = 8 columns of Q^R over the whole hidden dimension: thread t reads rows
-// t, t+256, ... of W as 16-byte vectors, all in flight at once.  The last CTA
-// to finish a router head (a per-head counter) normalises that head.
-// With W_QR == NULL the rows of Hq already hold Q^R and only the head step runs.
+// rows of padding queries are zero), and the clearing of the scan's max keys.
+// A row is one query token (B queries x M tokens).
+//
+// Grid (n_splits, n_r): CTA (s, h) multiplies rows [s*RS, (s+1)*RS) of W^QR's
+// head-h column block (a contiguous RS x d_r slab, read once, coalesced: each
+// warp reads whole 256-byte row pieces) by the matching slice of every query,
+// staged in shared memory, and writes fp32 partial sums qpart[s][b][h*d_r + c].
+// The last CTA of a head (per-head ticket) sums the n_splits partials in split
+// order (so the result does not depend on scheduling), normalises the head and
+// writes the hi/lo rows.  With W_QR == NULL the rows of Hq already hold Q^R and
+// only the head step runs (grid (1, n_r)).
 // --------------------------------------------------------------------------
-constexpr int kQrCols = 8;
-constexpr int kQrThreads = 256;
-constexpr int kQrMaxRows = 32;  // rows of W per thread: hidden <= 8192
-constexpr int kQrRowChunk = 8;  // rows loaded together
-constexpr int kQrQB = 8;        // queries per register group
+constexpr int kRqThreads = 256;
+constexpr int kRqRows = 12;      // rows of W held in registers per thread (resident case)
+constexpr int kRqQB = 8;         // queries per register group
+constexpr int kRqMaxSplitRows = 1024;
+constexpr int kRqTargetCtas = 144;
 
-__global__ void __launch_bounds__(kQrThreads) router_query_kernel(
+struct RqGeom {
+  int n_splits, rows;  // CTAs per head, rows of W per CTA (multiple of 16)
+};
+
+RqGeom rq_geom(int hidden, int n_r) {
+  int splits = std::max(1, kRqTargetCtas / n_r);
+  splits = std::max(splits, (hidden + kRqMaxSplitRows - 1) / kRqMaxSplitRows);
+  int rows = (hidden + splits - 1) / splits;
+  rows = (rows + 15) / 16 * 16;
+  return RqGeom{(hidden + rows - 1) / rows, rows};
+}
+
+size_t rq_smem_bytes(int d_r, int rows) {
+  return (size_t)(kRqThreads / 32) * kRqQB * d_r * sizeof(float) + (size_t)kRqQB * rows * sizeof(uint16_t);
+}
+
+__global__ void __launch_bounds__(kRqThreads) router_query_kernel(
     const __nv_bfloat16* __restrict__ Hq, const __nv_bfloat16* __restrict__ W, int B, int b_pad, int hidden,
-    int n_r, int d_r, int nq, float* __restrict__ qr, uint32_t* __restrict__ head_done,
-    __nv_bfloat16* __restrict__ q_hl, uint32_t* __restrict__ doc_key, int n_docs) {
-  __shared__ float red[kQrThreads / 32][kQrQB][kQrCols];
-  __shared__ float invn[32];
+    int n_r, int d_r, int nq, int split_rows, float* __restrict__ qpart, uint32_t* __restrict__ head_done,
+    __nv_bfloat16* __restrict__ q_hl, uint32_t* __restrict__ clear, size_t n_clear) {
+  extern __shared__ __align__(16) uint8_t rq_smem[];
+  float* red = reinterpret_cast<float*>(rq_smem);                                 // [8 warps][kRqQB][d_r]
+  uint16_t* hs = reinterpret_cast<uint16_t*>(red + (kRqThreads / 32) * kRqQB * d_r);  // [kRqQB][split_rows]
+  __shared__ float invn[kRqThreads / 32];
   __shared__ bool last;
   pdl_launch_dependents();
   pdl_wait();
   const int NR = n_r * d_r;
-  const int col0 = blockIdx.x * kQrCols;
+  const int h = blockIdx.y, split = blockIdx.x, n_splits = gridDim.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint16_t* hq = reinterpret_cast<const uint16_t*>(Hq);
 
-  // clear the document keys (grid-stride); the scan only runs after this kernel completes
-  if (doc_key)
-    for (size_t i = blockIdx.x * (size_t)kQrThreads + tid; i < (size_t)B * n_docs; i += (size_t)gridDim.x * kQrThreads)
-      doc_key[i] = 0u;
+  // clear the scan's max keys (grid-stride); the scan only runs after this kernel completes
+  if (clear) {
+    const size_t cta = (size_t)blockIdx.y * gridDim.x + blockIdx.x, n_cta = (size_t)gridDim.x * gridDim.y;
+    for (size_t i = cta * kRqThreads + tid; i < n_clear; i += n_cta * kRqThreads) clear[i] = 0u;
+  }
 
   if (W) {
-    for (int b0 = 0; b0 < B; b0 += kQrQB) {
-      float acc[kQrQB][kQrCols];
+    const int CG = d_r / 8;               // 8-column groups of the head (16 or 8)
+    const int RT = kRqThreads / CG;       // row threads (16 or 32)
+    const int cg = tid % CG, rt = tid / CG;
+    const int k0 = split * split_rows;
+    const int nrows = min(split_rows, hidden - k0);
+    const bool resident = (nrows + RT - 1) / RT <= kRqRows;  // block-uniform
+    const __nv_bfloat16* wcol = W + (size_t)k0 * NR + h * d_r + cg * 8;
+    uint4 wv[kRqRows];
+    if (resident) {
 #pragma unroll
-      for (int j = 0; j < kQrQB; ++j)
+      for (int u = 0; u < kRqRows; ++u) {
+        const int r = rt + RT * u;
+        wv[u] = r < nrows ? __ldg(reinterpret_cast<const uint4*>(wcol + (size_t)r * NR)) : make_uint4(0, 0, 0, 0);
+      }
+    }
+    for (int b0 = 0; b0 < B; b0 += kRqQB) {
+      // stage this query group's slice of H_q (zero rows past B)
+      __syncthreads();
+      const int vec = nrows / 8;  // 16-byte vectors per query row
+      for (int i = tid; i < kRqQB * vec; i += kRqThreads) {
+        const int j = i / vec, v = i % vec;
+        uint4 x = make_uint4(0, 0, 0, 0);
+        if (b0 + j < B) x = __ldg(reinterpret_cast<const uint4*>(hq + (size_t)(b0 + j) * hidden + k0) + v);
+        reinterpret_cast<uint4*>(hs + (size_t)j * split_rows)[v] = x;
+      }
+      __syncthreads();
+      float acc[kRqQB][8];
 #pragma unroll
-        for (int c = 0; c < kQrCols; ++c) acc[j][c] = 0.f;
-      for (int u0 = 0; u0 < kQrMaxRows; u0 += kQrRowChunk) {
-        if (tid + kQrThreads * u0 >= hidden) break;
-        uint4 wv[kQrRowChunk];  // this chunk's rows of W, all in flight at once
+      for (int j = 0; j < kRqQB; ++j)
 #pragma unroll
-        for (int u = 0; u < kQrRowChunk; ++u) {
-          const int k = tid + kQrThreads * (u0 + u);
-          wv[u] = k < hidden ? __ldg(reinterpret_cast<const uint4*>(W + (size_t)k * NR + col0)) : make_uint4(0, 0, 0, 0);
+        for (int c = 0; c < 8; ++c) acc[j][c] = 0.f;
+      auto fma_row = [&](const uint4 w4, int r) {
+        float wf[8];
+        float2 t;
+        t = unpack_bf16x2(w4.x); wf[0] = t.x; wf[1] = t.y;
+        t = unpack_bf16x2(w4.y); wf[2] = t.x; wf[3] = t.y;
+        t = unpack_bf16x2(w4.z); wf[4] = t.x; wf[5] = t.y;
+        t = unpack_bf16x2(w4.w); wf[6] = t.x; wf[7] = t.y;
+#pragma unroll
+        for (int j = 0; j < kRqQB; ++j) {
+          const float hv = bf16_bits_to_float(hs[(size_t)j * split_rows + r]);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) acc[j][c] = fmaf(hv, wf[c], acc[j][c]);
         }
+      };
+      if (resident) {
 #pragma unroll
-        for (int u = 0; u < kQrRowChunk; ++u) {
-          const int k = tid + kQrThreads * (u0 + u);
-          if (k < hidden) {
-            float wf[8];
-            float2 t;
-            t = unpack_bf16x2(wv[u].x); wf[0] = t.x; wf[1] = t.y;
-            t = unpack_bf16x2(wv[u].y); wf[2] = t.x; wf[3] = t.y;
-            t = unpack_bf16x2(wv[u].z); wf[4] = t.x; wf[5] = t.y;
-            t = unpack_bf16x2(wv[u].w); wf[6] = t.x; wf[7] = t.y;
+        for (int u = 0; u < kRqRows; ++u) {
+          const int r = rt + RT * u;
+          if (r < nrows) fma_row(wv[u], r);
+        }
+      } else {
+        for (int r0 = rt; r0 < nrows; r0 += RT * kRqRows) {
 #pragma unroll
-            for (int j = 0; j < kQrQB; ++j) {
-              const float h = b0 + j < B ? bf16_bits_to_float(hq[(size_t)(b0 + j) * hidden + k]) : 0.f;
+          for (int u = 0; u < kRqRows; ++u) {
+            const int r = r0 + RT * u;
+            wv[u] = r < nrows ? __ldg(reinterpret_cast<const uint4*>(wcol + (size_t)r * NR)) : make_uint4(0, 0, 0, 0);
+          }
 #pragma unroll
-              for (int c = 0; c < kQrCols; ++c) acc[j][c] = fmaf(h, wf[c], acc[j][c]);
-            }
+          for (int u = 0; u < kRqRows; ++u) {
+            const int r = r0 + RT * u;
+            if (r < nrows) fma_row(wv[u], r);
           }
         }
       }
+      // reduce over the row threads: lanes cg, cg + CG, ... of a warp, then the 8 warps
 #pragma unroll
-      for (int j = 0; j < kQrQB; ++j)
+      for (int j = 0; j < kRqQB; ++j)
 #pragma unroll
-        for (int c = 0; c < kQrCols; ++c) {
+        for (int c = 0; c < 8; ++c) {
           float v = acc[j][c];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-          if (lane == 0) red[warp][j][c] = v;
+          for (int o = CG; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          if (lane < CG) red[((size_t)warp * kRqQB + j) * d_r + cg * 8 + c] = v;
         }
       __syncthreads();
-      if (tid < kQrQB * kQrCols) {
-        const int j = tid / kQrCols, c = tid % kQrCols;
+      for (int i = tid; i < kRqQB * d_r; i += kRqThreads) {
+        const int j = i / d_r, col = i % d_r;
         float v = 0.f;
 #pragma unroll
-        for (int w = 0; w < kQrThreads / 32; ++w) v += red[w][j][c];
-        if (b0 + j < B) qr[(size_t)(b0 + j) * NR + col0 + c] = v;
+        for (int w = 0; w < kRqThreads / 32; ++w) v += red[((size_t)w * kRqQB + j) * d_r + col];
+        if (b0 + j < B) qpart[((size_t)split * B + b0 + j) * NR + h * d_r + col] = v;
       }
-      __syncthreads();
     }
-    // this head's columns are written: count the CTA in and let the head's last CTA go on
+    // this CTA's partials are written: take a ticket; the head's last CTA goes on
     __threadfence();
     __syncthreads();
     if (tid == 0) {
-      const int h = col0 / d_r;
       const uint32_t prev = atomicAdd(&head_done[h], 1u);
-      last = prev == (uint32_t)(d_r / kQrCols - 1);
+      last = prev == (uint32_t)(n_splits - 1);
       if (last) head_done[h] = 0u;  // ready for the next call
     }
     __syncthreads();
     if (!last) return;
     __threadfence();
-  } else if (col0 % d_r != 0) {
-    return;  // Q^R given: one CTA per head does the head step
   }
 
-  // ---- head step: normalise head h of every query and write the bf16 hi/lo rows ----
-  const int h = col0 / d_r;
-  const float* src = W ? qr : nullptr;
-  for (int b = warp; b < b_pad; b += kQrThreads / 32) {
+  // ---- head step: Q^R of head h for every query (partials summed in split order),
+  //      normalised, written as bf16 hi/lo rows ----
+  const int n_parts = W ? n_splits : 0;
+  for (int b = warp; b < b_pad; b += kRqThreads / 32) {
+    float v[4] = {0.f, 0.f, 0.f, 0.f};  // dims lane, lane + 32, ... (d_r <= 128)
     float ss = 0.f;
-    for (int i = lane; i < d_r; i += 32) {
-      float v = 0.f;
-      if (b < B) v = src ? __ldcg(&src[(size_t)b * NR + h * d_r + i])
-                         : bf16_bits_to_float(hq[(size_t)b * NR + h * d_r + i]);
-      ss = fmaf(v, v, ss);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = lane + 32 * e;
+      if (i < d_r && b < B) {
+        if (W) {
+          float x = 0.f;
+          for (int sp = 0; sp < n_parts; ++sp) x += __ldcg(&qpart[((size_t)sp * B + b) * NR + h * d_r + i]);
+          v[e] = x;
+        } else {
+          v[e] = bf16_bits_to_float(hq[(size_t)b * NR + h * d_r + i]);
+        }
+        ss = fmaf(v[e], v[e], ss);
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (lane == 0) invn[b % 32] = 1.0f / fmaxf(sqrtf(ss), kEps);
+    if (lane == 0) invn[warp] = 1.0f / fmaxf(sqrtf(ss), kEps);
     __syncwarp();
-    const float sc = invn[b % 32];
+    const float sc = invn[warp];
+    __syncwarp();
     const int pass = b / nq, row = b % nq;
     const size_t base = (((size_t)pass * n_r + h) * 2) * nq;
-    for (int i = lane; i < d_r; i += 32) {
-      float v = 0.f;
-      if (b < B) v = src ? __ldcg(&src[(size_t)b * NR + h * d_r + i])
-                         : bf16_bits_to_float(hq[(size_t)b * NR + h * d_r + i]);
-      const float x = v * sc;
-      const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-      const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
-      q_hl[(base + row) * d_r + i] = hi;
-      q_hl[(base + nq + row) * d_r + i] = lo;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = lane + 32 * e;
+      if (i < d_r) {
+        const float x = v[e] * sc;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+        q_hl[(base + row) * d_r + i] = hi;
+        q_hl[(base + nq + row) * d_r + i] = lo;
+      }
     }
   }
 }
@@ -201,8 +266,9 @@ constexpr int kScanEpiWarps = 8;    // two per TMEM lane quarter
 struct ScanParams {
   const int32_t* chunk_off;
   uint32_t* doc_key;
-  float* chunk_s;
+  uint32_t* chunk_k;
   int n_r, n_docs, n_chunks, n_tiles;
+  int q_tokens;    // query tokens per query: scan row r belongs to query r / q_tokens
   int q_base, q_count, pass;
   int head_major;  // K̄^R stored [n_r][C][d_r] instead of [C][n_r][d_r]
   uint32_t tmem_cols;
@@ -424,8 +490,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         const int b = hf * QH + bb;
         if (b >= p.q_count) continue;  // warp-uniform
         const float sc = acc[bb] * p.inv_nr;
+        const size_t qi = (size_t)((p.q_base + b) / p.q_tokens);  // max over a query's tokens: atomicMax
         if (MEAN) {
-          if (doc >= 0) p.chunk_s[(size_t)(p.q_base + b) * p.n_chunks + j] = sc;
+          if (doc >= 0) {
+            uint32_t* dst = &p.chunk_k[qi * p.n_chunks + j];
+            if (p.q_tokens == 1) *dst = float_to_ordered(sc);
+            else atomicMax(dst, float_to_ordered(sc));
+          }
         } else {
           float x = doc >= 0 ? sc : -__int_as_float(0x7f800000);
 #pragma unroll
@@ -433,8 +504,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
             const float ox = __shfl_down_sync(0xffffffffu, x, 1 << e);
             if (same & (1u << e)) x = fmaxf(x, ox);
           }
-          if (head && doc >= 0)
-            atomicMax(&p.doc_key[(size_t)(p.q_base + b) * p.n_docs + doc], float_to_ordered(x));
+          if (head && doc >= 0) atomicMax(&p.doc_key[qi * p.n_docs + doc], float_to_ordered(x));
         }
       }
     }
@@ -530,7 +600,7 @@ __device__ __forceinline__ uint64_t make_key(uint32_t ordered, int id) {
 }
 
 __global__ void __launch_bounds__(kTopkThreads) topk_slice_kernel(
-    const uint32_t* __restrict__ doc_key, const float* __restrict__ chunk_s, const int32_t* __restrict__ chunk_off,
+    const uint32_t* __restrict__ doc_key, const uint32_t* __restrict__ chunk_k, const int32_t* __restrict__ chunk_off,
     int n_docs, int n_chunks, int k, int n_slices, float* __restrict__ doc_scores, uint64_t* __restrict__ cand,
     int32_t* __restrict__ topk_idx, float* __restrict__ topk_score) {
   extern __shared__ uint64_t sm64[];
@@ -547,10 +617,10 @@ __global__ void __launch_bounds__(kTopkThreads) topk_slice_kernel(
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
     const int doc = d0 + i;
     uint32_t ok;
-    if (chunk_s) {
+    if (chunk_k) {
       const int c0 = __ldg(&chunk_off[doc]), c1 = __ldg(&chunk_off[doc + 1]);
       float s = 0.f;
-      for (int j = c0; j < c1; ++j) s += chunk_s[(size_t)b * n_chunks + j];
+      for (int j = c0; j < c1; ++j) s += ordered_to_float(chunk_k[(size_t)b * n_chunks + j]);
       const float mean = s / (float)max(1, c1 - c0);
       ok = float_to_ordered(mean);
     } else {
@@ -661,40 +731,50 @@ msa_status topk_merge_launch(const float* cand_score, const int32_t* cand_idx, i
   return MSA_OK;
 }
 
-size_t route_workspace(const msa_dims& d, int B, int n_docs, int n_chunks, int k, msa_doc_agg agg, void* ws,
+size_t route_workspace(const msa_dims& d, int B, int M, int n_docs, int n_chunks, int k, msa_doc_agg agg, void* ws,
                        RouteWs* out) {
   Carver cv(ws);
   RouteWs w{};
   const int NR = d.n_r * d.d_r;
-  w.nq = B <= 16 ? 16 : 32;
-  w.passes = (B + w.nq - 1) / w.nq;
+  const int R = B * M;  // query-token rows
+  w.nq = R <= 16 ? 16 : 32;
+  w.passes = (R + w.nq - 1) / w.nq;
   w.n_slices = (n_docs + kSliceDocs - 1) / kSliceDocs;
-  w.qr = cv.take<float>((size_t)B * NR);
+  w.rq_splits = rq_geom(d.hidden, d.n_r).n_splits;
+  w.qr = cv.take<float>((size_t)w.rq_splits * R * NR);
   w.head_done = cv.take<uint32_t>(8);
   w.q_hl = cv.take<__nv_bfloat16>((size_t)w.passes * d.n_r * 2 * w.nq * d.d_r);
   w.doc_key = agg == MSA_AGG_MAX ? cv.take<uint32_t>((size_t)B * n_docs) : nullptr;
-  w.chunk_s = agg == MSA_AGG_MEAN ? cv.take<float>((size_t)B * n_chunks) : nullptr;
+  w.chunk_k = agg == MSA_AGG_MEAN ? cv.take<uint32_t>((size_t)B * n_chunks) : nullptr;
   w.cand = w.n_slices > 1 ? cv.take<uint64_t>((size_t)B * w.n_slices * k) : nullptr;
   if (out) *out = w;
   return cv.size();
 }
 
-msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int B, const void* KR_bar,
+msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int B, int M, const void* KR_bar,
                         const int32_t* chunk_off, int n_docs, int n_chunks, int k, msa_doc_agg agg, int kr_layout,
                         float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws, cudaStream_t s) {
   RouteWs w;
-  route_workspace(d, B, n_docs, n_chunks, k, agg, ws, &w);
+  route_workspace(d, B, M, n_docs, n_chunks, k, agg, ws, &w);
   const int NR = d.n_r * d.d_r;
+  const int R = B * M;
   const bool mean = agg == MSA_AGG_MEAN;
+  // keys folded in with atomicMax start at 0 (below every ordered score): the document keys,
+  // and the chunk keys when several tokens of a query meet in one chunk
+  uint32_t* clear = mean ? (M > 1 ? w.chunk_k : nullptr) : w.doc_key;
+  const size_t n_clear = clear ? (size_t)B * (mean ? n_chunks : n_docs) : 0;
 
   // K1: router query (projection, normalisation, hi/lo layout) and document keys cleared
   {
     MSA_CUDA_CHECK(cudaMemsetAsync(w.head_done, 0, 8 * sizeof(uint32_t), s));
     TraceScope ts(kKRouterQuery, s);
-    MSA_CUDA_CHECK(launch_pdl(router_query_kernel, dim3(NR / kQrCols), dim3(kQrThreads), 0, s,
-                              static_cast<const __nv_bfloat16*>(Hq), static_cast<const __nv_bfloat16*>(W_QR), B,
-                              w.passes * w.nq, d.hidden, d.n_r, d.d_r, w.nq, w.qr, w.head_done, w.q_hl, w.doc_key,
-                              n_docs));
+    const RqGeom g = rq_geom(d.hidden, d.n_r);
+    const size_t sm = W_QR ? rq_smem_bytes(d.d_r, g.rows) : 0;
+    MSA_CUDA_CHECK(cudaFuncSetAttribute(router_query_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+    MSA_CUDA_CHECK(launch_pdl(router_query_kernel, dim3(W_QR ? g.n_splits : 1, d.n_r), dim3(kRqThreads), sm, s,
+                              static_cast<const __nv_bfloat16*>(Hq), static_cast<const __nv_bfloat16*>(W_QR), R,
+                              w.passes * w.nq, d.hidden, d.n_r, d.d_r, w.nq, g.rows, w.qr, w.head_done, w.q_hl,
+                              clear, n_clear));
   }
   // K3: scan, NQ (16 or 32) queries per pass
   {
@@ -728,13 +808,14 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
       ScanParams p;
       p.chunk_off = chunk_off;
       p.doc_key = w.doc_key;
-      p.chunk_s = w.chunk_s;
+      p.chunk_k = w.chunk_k;
+      p.q_tokens = M;
       p.n_r = d.n_r;
       p.n_docs = n_docs;
       p.n_chunks = n_chunks;
       p.n_tiles = n_tiles;
       p.q_base = pass * w.nq;
-      p.q_count = std::min(B - p.q_base, w.nq);
+      p.q_count = std::min(R - p.q_base, w.nq);
       p.pass = pass;
       p.head_major = kr_layout == 1;
       p.tmem_cols = cols;
@@ -750,7 +831,7 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
     const size_t sm = topk_slice_smem();
     MSA_CUDA_CHECK(cudaFuncSetAttribute(topk_slice_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
     MSA_CUDA_CHECK(launch_pdl(topk_slice_kernel, dim3(w.n_slices, B), dim3(kTopkThreads), sm, s,
-                              (const uint32_t*)w.doc_key, (const float*)w.chunk_s, chunk_off, n_docs, n_chunks, k,
+                              (const uint32_t*)w.doc_key, (const uint32_t*)w.chunk_k, chunk_off, n_docs, n_chunks, k,
                               w.n_slices, doc_scores, w.cand, topk_idx, topk_score));
   }
   if (w.n_slices > 1) {

@@ -10,7 +10,7 @@ not benchmark values.
 Cases
   route1m    1M-token memory, B = 1   (K̄^R 33 MB)
   route16m   16M-token memory, B = 32 (K̄^R 520 MB)
-  route100m  100M-token memory, B = 1 (K̄^R 3.2 GB); --batch to change B
+  route100m  100M-token memory, B = 1 (K̄^R 3.2 GB); --batch to change B, --tokens the size
              (route cases: --kr-layout head stores K̄^R head-major [n_r, C, d_r])
   attend1m   sparse attention, 1M-token memory, B = 1, 4K local tokens (rotated key cache)
   attend16m  sparse attention, 16M-token memory, B = 32, 8K local tokens (rotated key cache)
@@ -174,24 +174,25 @@ def main():
     ap.add_argument("--launches", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=2)
     ap.add_argument("--batch", type=int, default=None)
-    ap.add_argument("--tokens", type=int, default=1_000_000)
+    ap.add_argument("--tokens", type=int, default=None, help="memory tokens (encode default 1M; route cases: "
+                    "their own size unless given)")
     ap.add_argument("--kr-layout", choices=["chunk", "head"], default="chunk")
     a = ap.parse_args()
     dev = torch.device("cuda:0")
     seed = W.BASE_SEED + 7
     hm = a.kr_layout == "head"
     if a.case == "route1m":
-        case = RouteCase(1_000_000, a.batch or 1, 2048, seed, dev, head_major=hm)
+        case = RouteCase(a.tokens or 1_000_000, a.batch or 1, 2048, seed, dev, head_major=hm)
     elif a.case == "route16m":
-        case = RouteCase(16_000_000, a.batch or 32, 2048, seed, dev, head_major=hm)
+        case = RouteCase(a.tokens or 16_000_000, a.batch or 32, 2048, seed, dev, head_major=hm)
     elif a.case == "route100m":
-        case = RouteCase(100_000_000, a.batch or 1, 4096, seed, dev, head_major=hm)
+        case = RouteCase(a.tokens or 100_000_000, a.batch or 1, 4096, seed, dev, head_major=hm)
     elif a.case == "attend1m":
         case = AttendCase(1_000_000, a.batch or 1, 2048, 4096, seed, dev)
     elif a.case == "attend16m":
         case = AttendCase(16_000_000, a.batch or 32, 2048, 8192, seed, dev)
     else:
-        case = EncodeCase(a.tokens, seed, dev)
+        case = EncodeCase(a.tokens or 1_000_000, seed, dev)
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
         for _ in range(a.warmup):

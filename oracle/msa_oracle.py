@@ -35,7 +35,10 @@ with its reason in the design notes):
     last local token, at pos_offset + loc_len - 1; gathered chunk keys keep
     only their document-wise rotation;
   * attention has no causal mask over the gathered context and uses the
-    scale 1/sqrt(head_dim) unless another is given.
+    scale 1/sqrt(head_dim) unless another is given;
+  * a query of M > 1 tokens (the query-prefill step) is the last M local
+    tokens: token t sits at pos_offset + loc_len - M + t and sees every
+    gathered chunk and the local tokens j <= loc_len - M + t (causal).
 
 Every function here is pinned by tests in ``tests/test_oracle.py`` against
 closed forms, invariants, brute force and hand-derived values.
@@ -279,4 +282,41 @@ def sparse_attend(q, K_bar, V_bar, chunk_off, topk_idx, K_loc, V_loc, loc_len, p
         for g in range(n_q):
             h = g // G
             out[b, g] = attention(qr[g], K_ctx[:, h], V_ctx[:, h], scale)
+    return out
+
+
+def sparse_attend_tokens(q, K_bar, V_bar, chunk_off, topk_idx, K_loc, V_loc, loc_len, pos_offset: int,
+                         rope_base: float = 1.0e6, scale: float = 0.0) -> np.ndarray:
+    """Attention of M query tokens per query; q [B, M, n_q, d] -> out [B, M, n_q, d] float64.
+
+    The query tokens are the last M local tokens.  Each token's logits run over the
+    whole explicit context [selected docs' pooled keys; every local key] and a mask
+    removes the local keys after the token's own position (chunk keys are always
+    visible), so the softmax is taken over exactly the keys the token may see.
+    """
+    qf = bf16_to_f64(q)
+    B, M, n_q, d = qf.shape
+    n_kv = np.asarray(K_bar).shape[1]
+    G = n_q // n_kv
+    if scale == 0.0:
+        scale = 1.0 / math.sqrt(d)
+    out = np.empty((B, M, n_q, d))
+    for b in range(B):
+        L = int(loc_len[b])
+        K_ctx, V_ctx = sparse_context(K_bar, V_bar, chunk_off, topk_idx[b], K_loc[b], V_loc[b],
+                                      L, pos_offset, rope_base)
+        n_sel = K_ctx.shape[0] - L
+        is_chunk = np.arange(K_ctx.shape[0]) < n_sel
+        local_j = np.arange(K_ctx.shape[0]) - n_sel
+        for t in range(M):
+            own = L - M + t                                   # this token's local index
+            visible = is_chunk | (local_j <= own)
+            qr = rope(qf[b, t], pos_offset + own, rope_base)
+            for g in range(n_q):
+                h = g // G
+                logits = (K_ctx[:, h] @ qr[g]) * scale
+                logits = np.where(visible, logits, -np.inf)
+                m = logits.max()
+                p = np.exp(logits - m)
+                out[b, t, g] = (p[:, None] * V_ctx[:, h]).sum(axis=0) / p.sum()
     return out

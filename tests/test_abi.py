@@ -71,12 +71,14 @@ def _dims(**kw):
 FAKE = 0x10000  # 16-byte aligned non-null "device" address; never dereferenced
 
 
-def _route(msa, dims, B=1, n_docs=10, n_chunks=20, k=4, agg=0, ws_bytes=None, Hq=FAKE, kr=FAKE, idx=FAKE, layout=0):
+def _route(msa, dims, B=1, n_docs=10, n_chunks=20, k=4, agg=0, ws_bytes=None, Hq=FAKE, kr=FAKE, idx=FAKE, layout=0,
+           M=1):
     dd = msa.Dims.of(dims)
-    need = msa.lib.msa_route_workspace_size(ctypes.byref(dd), B, n_docs, n_chunks, k, agg)
+    need = msa.lib.msa_route_workspace_size(ctypes.byref(dd), B, max(M, 1), n_docs, n_chunks, k, agg)
     if ws_bytes is None:
         ws_bytes = need
-    return msa.lib.msa_route_topk(ctypes.byref(dd), Hq, None, B, kr, FAKE, n_docs, n_chunks, k, agg, layout, None, idx,
+    return msa.lib.msa_route_topk(ctypes.byref(dd), Hq, None, B, M, kr, FAKE, n_docs, n_chunks, k, agg, layout, None,
+                                  idx,
                                   FAKE,
                                   0x100000 if ws_bytes else None, ws_bytes, None)
 
@@ -94,6 +96,8 @@ def test_route_validation(msa):
     assert _route(msa, ok, kr=None) == 1                    # NULL
     assert _route(msa, ok, agg=7) == 1
     assert _route(msa, ok, layout=2) == 1                   # K̄^R layout is 0 (chunk-major) or 1 (head-major)
+    assert _route(msa, ok, M=0) == 1                        # at least one query token
+    assert _route(msa, ok, B=4096, M=17) == 1               # B * M above 65535
     assert _route(msa, ok, ws_bytes=16) == 3                # workspace too small
     assert "workspace too small" in msa.lib.msa_last_error().decode()
 
@@ -104,12 +108,12 @@ def test_route_fault_injection_before_launch(msa, monkeypatch):
     assert "injected" in msa.lib.msa_last_error().decode()
 
 
-def _attend(msa, dims, B=1, k=2, n_docs=4, n_chunks=8, t_loc=16, pos=2, scale=0.0, ws_bytes=None, q=FAKE):
+def _attend(msa, dims, B=1, k=2, n_docs=4, n_chunks=8, t_loc=16, pos=2, scale=0.0, ws_bytes=None, q=FAKE, M=1):
     dd = msa.Dims.of(dims)
-    need = msa.lib.msa_attend_workspace_size(ctypes.byref(dd), B, k, t_loc, pos)
+    need = msa.lib.msa_attend_workspace_size(ctypes.byref(dd), B, max(M, 1), k, t_loc, pos)
     if ws_bytes is None:
         ws_bytes = need
-    return msa.lib.msa_sparse_attend(ctypes.byref(dd), q, B, FAKE, FAKE, FAKE, n_docs, n_chunks, FAKE, k, FAKE, FAKE,
+    return msa.lib.msa_sparse_attend(ctypes.byref(dd), q, B, M, FAKE, FAKE, FAKE, n_docs, n_chunks, FAKE, k, FAKE, FAKE,
                                      FAKE, t_loc, pos, None, 0, scale, FAKE, 0x100000, ws_bytes, None)
 
 
@@ -124,6 +128,7 @@ def test_attend_validation(msa):
     assert _attend(msa, ok, scale=float("nan")) == 1
     assert _attend(msa, ok, q=FAKE + 2) == 1
     assert _attend(msa, ok, ws_bytes=8) == 3
+    assert _attend(msa, ok, M=0) == 1
 
 
 def test_encode_validation(msa):
@@ -149,9 +154,11 @@ def test_topk_merge_validation(msa):
 
 def test_workspace_sizes_grow_with_problem(msa):
     d = msa.Dims.of(W.QWEN3_4B_DIMS)
-    a = msa.lib.msa_route_workspace_size(ctypes.byref(d), 1, 500, 16000, 16, 0)
-    b = msa.lib.msa_route_workspace_size(ctypes.byref(d), 32, 500, 16000, 16, 0)
-    assert 0 < a < b
-    assert msa.lib.msa_route_workspace_size(ctypes.byref(d), 0, 500, 16000, 16, 0) == 0
-    x = msa.lib.msa_attend_workspace_size(ctypes.byref(d), 1, 16, 4096, 16)
+    a = msa.lib.msa_route_workspace_size(ctypes.byref(d), 1, 1, 500, 16000, 16, 0)
+    b = msa.lib.msa_route_workspace_size(ctypes.byref(d), 32, 1, 500, 16000, 16, 0)
+    c = msa.lib.msa_route_workspace_size(ctypes.byref(d), 32, 8, 500, 16000, 16, 0)
+    assert 0 < a < b < c
+    assert msa.lib.msa_route_workspace_size(ctypes.byref(d), 0, 1, 500, 16000, 16, 0) == 0
+    x = msa.lib.msa_attend_workspace_size(ctypes.byref(d), 1, 1, 16, 4096, 16)
     assert x >= 4096 * 64 * 8   # the local RoPE table alone
+    assert msa.lib.msa_attend_workspace_size(ctypes.byref(d), 1, 8, 16, 4096, 16) > x

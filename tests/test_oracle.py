@@ -371,6 +371,72 @@ def test_attend_topk_order_irrelevant_and_matches_explicit_concat():
     assert len(K_ctx) == (co[3] - co[2]) + (co[1] - co[0]) + 6
 
 
+def test_attend_tokens_prefill_equals_sequence_of_decodes():
+    # the M-token call masks a shared context; token t must equal a decode step that
+    # simply has loc_len - M + t + 1 local tokens (a truncated context, no mask)
+    c = _attend_case(L=7)
+    rng = np.random.default_rng(12)
+    M = 4
+    q = W.normal_bf16(rng, (1, M, 8, 16))
+    args = {k: v for k, v in c.items() if k != "q"}
+    out = O.sparse_attend_tokens(q, pos_offset=3, rope_base=1e4, **args)
+    for t in range(M):
+        a2 = dict(args)
+        a2["loc_len"] = np.array([7 - M + t + 1])
+        dec = O.sparse_attend(q[:, t], pos_offset=3, rope_base=1e4, **a2)
+        assert np.allclose(out[:, t], dec, atol=1e-13), t
+    # M = 1 is the decode step itself
+    one = O.sparse_attend_tokens(c["q"][:, None], pos_offset=3, rope_base=1e4, **args)
+    assert np.allclose(one[:, 0], O.sparse_attend(pos_offset=3, rope_base=1e4, **c), atol=1e-13)
+
+
+def test_attend_tokens_first_token_sees_chunk_and_first_local_key():
+    # context: one pooled chunk key + 3 local keys; with M = 3 = loc_len, token 0 sees the chunk and
+    # local key 0 only: its chunk weight is the two-key logistic of the rotated logits
+    d, base, o = 16, 1e4, 2
+    rng = np.random.default_rng(13)
+    q = _bits(rng.standard_normal((1, 3, 1, d)))
+    kb = _bits(rng.standard_normal((1, 1, d)))
+    kl = _bits(rng.standard_normal((1, 3, 1, d)))
+    vb = _bits(np.eye(d)[0][None, None])
+    vl = np.zeros((1, 3, 1, d), dtype=np.uint16)
+    out = O.sparse_attend_tokens(q, kb, vb, np.array([0, 1]), np.array([[0]]), kl, vl, np.array([3]),
+                                 pos_offset=o, rope_base=base, scale=0.5)
+    theta = base ** (-np.arange(0, d, 2) / d)
+
+    def rot(v, p):
+        z = (v[: d // 2] + 1j * v[d // 2:]) * np.exp(1j * p * theta)
+        return np.concatenate([z.real, z.imag])
+
+    qf = O.bf16_to_f64(q)[0, 0, 0]
+    l_chunk = 0.5 * rot(qf, o) @ O.bf16_to_f64(kb)[0, 0]
+    l_loc = 0.5 * rot(qf, o) @ rot(O.bf16_to_f64(kl)[0, 0, 0], o)
+    want = 1.0 / (1.0 + math.exp(l_loc - l_chunk))
+    assert math.isclose(out[0, 0, 0, 0], want, rel_tol=1e-12)
+    # the last token sees all four keys: its chunk weight is strictly below token 0's unless
+    # the extra local logits are -inf, which they are not
+    assert 0.0 < out[0, 2, 0, 0] < 1.0
+
+
+def test_attend_tokens_before_local_context_see_only_chunks():
+    # loc_len < M: the first tokens come before every local key; they attend over the gathered
+    # chunks alone (every chunk, none dropped), i.e. plain attention over the pooled rows
+    c = _attend_case(L=2)
+    rng = np.random.default_rng(14)
+    M = 5
+    q = W.normal_bf16(rng, (1, M, 8, 16))
+    args = {k: v for k, v in c.items() if k != "q"}
+    out = O.sparse_attend_tokens(q, pos_offset=3, rope_base=1e4, **args)
+    co = c["chunk_off"]
+    Kc = np.concatenate([O.bf16_to_f64(c["K_bar"])[co[i]:co[i + 1]] for i in (2, 0)])
+    Vc = np.concatenate([O.bf16_to_f64(c["V_bar"])[co[i]:co[i + 1]] for i in (2, 0)])
+    for t in range(M - 2):                       # own local index 2 - 5 + t < 0
+        qr = O.rope(O.bf16_to_f64(q)[0, t], 3 + 2 - M + t, 1e4)
+        for g in range(8):
+            want = O.attention(qr[g], Kc[:, g // 4], Vc[:, g // 4], 1 / math.sqrt(16))
+            assert np.allclose(out[0, t, g], want, atol=1e-13), (t, g)
+
+
 # ----------------------------------------------------------------------------
 # pages' footprint arithmetic
 # ----------------------------------------------------------------------------

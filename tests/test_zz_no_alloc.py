@@ -23,7 +23,7 @@ def _static_fn(msa):
     fn = msa.lib.msa_route_topk_static
     P, I32 = ctypes.c_void_p, ctypes.c_int32
     fn.restype = I32
-    fn.argtypes = [ctypes.POINTER(msa.Dims), P, P, I32, P, P, I32, I32, I32, I32, P, P, P, P]
+    fn.argtypes = [ctypes.POINTER(msa.Dims), P, P, I32, I32, P, P, I32, I32, I32, I32, P, P, P, P]
     return fn
 
 
@@ -51,7 +51,7 @@ def test_static_scratch_matches_workspace_path(cuda_device):
         idx = torch.full((B, k), -1, dtype=torch.int32, device=dev)
         sc = torch.zeros((B, k), dtype=torch.float32, device=dev)
         ds = torch.zeros((B, n_docs), dtype=torch.float32, device=dev)
-        r = fn(ctypes.byref(dd), Hq.data_ptr(), Wqr.data_ptr(), B, KR.data_ptr(), chunk_off.data_ptr(), n_docs, C, k,
+        r = fn(ctypes.byref(dd), Hq.data_ptr(), Wqr.data_ptr(), B, 1, KR.data_ptr(), chunk_off.data_ptr(), n_docs, C, k,
                0, ds.data_ptr(), idx.data_ptr(), sc.data_ptr(), stream)
         assert r == 0, msa.lib.msa_last_error().decode()
         torch.cuda.synchronize()
@@ -72,7 +72,7 @@ def test_static_scratch_rejects_oversized_problem(cuda_device):
     fn = _static_fn(msa)
     dd = msa.Dims.of(W.QWEN3_4B_DIMS)
     # 32 queries over 400K documents need far more than the 8 MiB static area
-    r = fn(ctypes.byref(dd), 0x10000, 0x10000, 32, 0x10000, 0x10000, 400_000, 1_600_000, 16, 0, None, 0x10000,
+    r = fn(ctypes.byref(dd), 0x10000, 0x10000, 32, 1, 0x10000, 0x10000, 400_000, 1_600_000, 16, 0, None, 0x10000,
            0x10000, None)
     assert r == 3
     assert "static area" in msa.lib.msa_last_error().decode()
