@@ -119,6 +119,34 @@ msa_status msa_encode_memory(const msa_dims* dims, const void* H, int64_t T, con
                              int32_t kr_layout, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Incremental memory append: encode new documents behind an existing memory.
+ * Pages: IRMaD "M. Materials & Methods", three-stage inference item (1) (the
+ * memory is encoded offline, document by document, and cached); paper digest,
+ * "limitations and improvements" section, future directions (streaming memory
+ * updates by incremental encoding instead of re-encoding the corpus).  Because
+ * positions restart at 0 in every document and chunks never cross documents,
+ * the new documents' pooled rows do not depend on the existing ones: appending
+ * gives bit for bit the rows a full msa_encode_memory of all documents gives.
+ *   H_new [T_new, hidden], doc_off_new [n_docs_new + 1] (device int64, relative
+ *            to H_new), chunk_off_new [n_docs_new + 1] (device int32, relative),
+ *            n_chunks_new: the new documents alone, as for msa_encode_memory.
+ *   K_bar, V_bar [chunk_capacity, n_kv, head_dim], KR_bar [chunk_capacity, n_r, d_r]
+ *            chunk-major bf16: rows n_chunks_old .. n_chunks_old + n_chunks_new - 1
+ *            are written, earlier rows are left alone.
+ *   chunk_off  device int32 [n_docs_old + n_docs_new + 1], the whole memory's
+ *            chunk offsets: entries n_docs_old .. n_docs_old + n_docs_new are
+ *            written (n_chunks_old + chunk_off_new[i]).
+ *   ws, ws_bytes  as msa_encode_workspace_size(dims, T_new, n_docs_new, n_chunks_new).
+ * Errors: MSA_ERR_INVALID_ARG when n_chunks_old + n_chunks_new > chunk_capacity;
+ * otherwise those of msa_encode_memory.  Stream-ordered; no host synchronisation.
+ * ------------------------------------------------------------------------- */
+msa_status msa_append_memory(const msa_dims* dims, const void* H_new, int64_t T_new, const int64_t* doc_off_new,
+                             int32_t n_docs_new, const int32_t* chunk_off_new, int32_t n_chunks_new,
+                             const void* W_K, const void* W_V, const void* W_KR, void* K_bar, void* V_bar,
+                             void* KR_bar, int32_t chunk_capacity, int32_t* chunk_off, int32_t n_docs_old,
+                             int32_t n_chunks_old, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Stage 2 - online routing and top-k.
  * Pages: IRMaD "M. Materials & Methods", routing item:
  *   Q^R = H_q W^QR;  S_ij = max_t mean_h cos(Q^R_h, K̄^R_ij,h);

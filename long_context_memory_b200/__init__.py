@@ -7,7 +7,7 @@ current stream.  Importing this package fails loudly when the library is
 missing; there is no CPU fallback.
 
 Entry points (same names as the C ABI, minus the ``msa_`` prefix):
-  chunk_offsets, encode_memory, route_topk, sparse_attend,
+  chunk_offsets, encode_memory, append_memory, route_topk, sparse_attend,
   *_workspace_size, check_device_errors, trace_*.
 """
 from __future__ import annotations
@@ -17,7 +17,7 @@ import os
 from typing import Optional
 
 __all__ = [
-    "Dims", "MSAError", "lib", "chunk_offsets", "encode_memory", "route_topk", "sparse_attend",
+    "Dims", "MSAError", "lib", "chunk_offsets", "encode_memory", "append_memory", "route_topk", "sparse_attend",
     "route_workspace_size", "attend_workspace_size", "rope_cache_build", "topk_merge", "rope_rows", "gather_kv", "encode_workspace_size", "check_device_errors",
     "trace_enable", "trace_reset", "trace_read", "trace_kernel_names", "AGG_MAX", "AGG_MEAN",
 ]
@@ -64,6 +64,7 @@ def _load():
         "msa_chunk_offsets": (I32, [P, I32, I32, P, ctypes.POINTER(I32)]),
         "msa_encode_workspace_size": (SZ, [DP, I64, I32, I32]),
         "msa_encode_memory": (I32, [DP, P, I64, P, I32, P, I32, P, P, P, P, P, P, I32, P, SZ, P]),
+        "msa_append_memory": (I32, [DP, P, I64, P, I32, P, I32, P, P, P, P, P, P, I32, P, I32, I32, P, SZ, P]),
         "msa_route_workspace_size": (SZ, [DP, I32, I32, I32, I32, I32, I32]),
         "msa_route_topk": (I32, [DP, P, P, I32, I32, P, P, I32, I32, I32, I32, I32, P, P, P, P, SZ, P]),
         "msa_attend_workspace_size": (SZ, [DP, I32, I32, I32, I32, I32]),
@@ -183,6 +184,26 @@ def encode_memory(dims, H, doc_off, chunk_off, n_chunks: int, W_K, W_V, W_KR, ou
                                  _ptr(W_K), _ptr(W_V), _ptr(W_KR), _ptr(out[0]), _ptr(out[1]), _ptr(out[2]),
                                  int(bool(kr_head_major)), _aligned_ptr(ws), nbytes, _stream(stream)))
     return out
+
+
+def append_memory(dims, H_new, doc_off_new, chunk_off_new, n_chunks_new: int, W_K, W_V, W_KR, memory, chunk_off,
+                  n_docs_old: int, n_chunks_old: int, ws=None, stream=None):
+    """Encode new documents behind an existing chunk-major memory, in place.
+
+    ``memory`` = (K_bar, V_bar, KR_bar) with room for the new chunks (first dimension = the
+    capacity in chunks); ``chunk_off`` (device int32, room for every document + 1) gets the new
+    documents' offsets.  Returns (n_docs_old + n_docs_new, n_chunks_old + n_chunks_new).
+    """
+    K_bar, V_bar, KR_bar = memory
+    T = H_new.shape[0]
+    n_new = doc_off_new.numel() - 1
+    nbytes = encode_workspace_size(dims, T, n_new, n_chunks_new)
+    ws = _workspace(nbytes, H_new.device, ws)
+    _check(lib.msa_append_memory(ctypes.byref(Dims.of(dims)), _ptr(H_new), T, _ptr(doc_off_new), n_new,
+                                 _ptr(chunk_off_new), n_chunks_new, _ptr(W_K), _ptr(W_V), _ptr(W_KR), _ptr(K_bar),
+                                 _ptr(V_bar), _ptr(KR_bar), K_bar.shape[0], _ptr(chunk_off), n_docs_old,
+                                 n_chunks_old, _aligned_ptr(ws), nbytes, _stream(stream)))
+    return n_docs_old + n_new, n_chunks_old + n_chunks_new
 
 
 # ----------------------------------------------------------------------------

@@ -395,6 +395,28 @@ cudaError_t launch_gemm(int bn, int grid, size_t smem, cudaStream_t s, const CUt
 
 }  // namespace
 
+namespace {
+// chunk_off[n_docs_old + i] = n_chunks_old + chunk_off_new[i], i = 0 .. n_docs_new
+__global__ void __launch_bounds__(256) chunk_off_extend_kernel(int32_t* __restrict__ chunk_off, int n_docs_old,
+                                                               int n_chunks_old,
+                                                               const int32_t* __restrict__ chunk_off_new,
+                                                               int n_docs_new) {
+  pdl_launch_dependents();
+  pdl_wait();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i <= n_docs_new; i += gridDim.x * blockDim.x)
+    chunk_off[n_docs_old + i] = n_chunks_old + chunk_off_new[i];
+}
+}  // namespace
+
+msa_status chunk_off_extend_launch(int32_t* chunk_off, int n_docs_old, int n_chunks_old, const int32_t* chunk_off_new,
+                                   int n_docs_new, cudaStream_t s) {
+  TraceScope ts(kKChunkOffExtend, s);
+  const int blocks = std::max(1, std::min(148, (n_docs_new + 1 + 255) / 256));
+  MSA_CUDA_CHECK(launch_pdl(chunk_off_extend_kernel, dim3(blocks), dim3(256), 0, s, chunk_off, n_docs_old,
+                            n_chunks_old, chunk_off_new, n_docs_new));
+  return MSA_OK;
+}
+
 size_t encode_workspace(const msa_dims& d, int64_t T, int n_docs, int n_chunks, void* ws, EncodeWs* out) {
   (void)T;
   (void)n_docs;

@@ -49,6 +49,7 @@ enum KernelId : int {
   kKRopeRows,
   kKGatherPlan,
   kKGatherCopy,
+  kKChunkOffExtend,
   kKernelCount
 };
 
@@ -139,6 +140,8 @@ msa_status gather_kv_launch(const msa_dims& d, const void* K_host, const void* V
 msa_status rope_rows_launch(const msa_dims& d, void* x, int rows, int heads, const int32_t* pos, cudaStream_t s);
 msa_status rope_cache_build(const msa_dims& d, int t_loc_max, int pos_offset, float2* tab, cudaStream_t s);
 
+msa_status chunk_off_extend_launch(int32_t* chunk_off, int n_docs_old, int n_chunks_old, const int32_t* chunk_off_new,
+                                   int n_docs_new, cudaStream_t s);
 size_t encode_workspace(const msa_dims& d, int64_t T, int n_docs, int n_chunks, void* ws,
                         struct EncodeWs* out);
 msa_status encode_launch(const msa_dims& d, const void* H, int64_t T, const int64_t* doc_off, int n_docs,

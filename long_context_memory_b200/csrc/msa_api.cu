@@ -109,7 +109,8 @@ msa_status encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int ra
 namespace {
 const char* kKernelNames[kKernelCount] = {
     "router_query", "scan", "topk_slice", "topk_merge", "rope_table", "attn_split", "attn_combine",
-    "enc_chunk_map", "enc_transpose_w", "enc_gemm_k", "enc_pool_h", "enc_gemm_pooled", "rope_rows", "gather_plan", "gather_copy"};
+    "enc_chunk_map", "enc_transpose_w", "enc_gemm_k", "enc_pool_h", "enc_gemm_pooled", "rope_rows", "gather_plan", "gather_copy",
+    "chunk_off_extend"};
 
 struct TraceState {
   std::mutex mu;
@@ -468,6 +469,32 @@ msa_status msa_encode_memory(const msa_dims* dims, const void* H, int64_t T, con
   if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
   return encode_launch(*dims, H, T, doc_off, n_docs, chunk_off, n_chunks, W_K, W_V, W_KR, K_bar, V_bar, KR_bar,
                        kr_layout, ws, static_cast<cudaStream_t>(stream));
+}
+
+msa_status msa_append_memory(const msa_dims* dims, const void* H_new, int64_t T_new, const int64_t* doc_off_new,
+                             int32_t n_docs_new, const int32_t* chunk_off_new, int32_t n_chunks_new,
+                             const void* W_K, const void* W_V, const void* W_KR, void* K_bar, void* V_bar,
+                             void* KR_bar, int32_t chunk_capacity, int32_t* chunk_off, int32_t n_docs_old,
+                             int32_t n_chunks_old, void* ws, size_t ws_bytes, void* stream) {
+  if (n_docs_old < 0 || n_chunks_old < n_docs_old || n_chunks_new < 1 ||
+      (int64_t)n_chunks_old + n_chunks_new > chunk_capacity)
+    return fail(MSA_ERR_INVALID_ARG, "append of %d chunks after %d (%d docs) exceeds the capacity of %d chunks",
+                n_chunks_new, n_chunks_old, n_docs_old, chunk_capacity);
+  CHECK_PTR(chunk_off);
+  CHECK_PTR(K_bar);
+  CHECK_PTR(V_bar);
+  CHECK_PTR(KR_bar);
+  if (!dims) return fail(MSA_ERR_INVALID_ARG, "dims is NULL");
+  // the new documents' chunks land after the existing ones (chunk-major rows: a pointer offset)
+  const size_t row_kv = (size_t)dims->n_kv * dims->head_dim, row_r = (size_t)dims->n_r * dims->d_r;
+  uint16_t* Kb = static_cast<uint16_t*>(K_bar) + (size_t)n_chunks_old * row_kv;
+  uint16_t* Vb = static_cast<uint16_t*>(V_bar) + (size_t)n_chunks_old * row_kv;
+  uint16_t* KRb = static_cast<uint16_t*>(KR_bar) + (size_t)n_chunks_old * row_r;
+  msa_status st = msa_encode_memory(dims, H_new, T_new, doc_off_new, n_docs_new, chunk_off_new, n_chunks_new, W_K,
+                                    W_V, W_KR, Kb, Vb, KRb, 0, ws, ws_bytes, stream);
+  if (st != MSA_OK) return st;
+  return chunk_off_extend_launch(chunk_off, n_docs_old, n_chunks_old, chunk_off_new, n_docs_new,
+                                 static_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------ tracing ------------------------------

@@ -320,3 +320,67 @@ def sparse_attend_tokens(q, K_bar, V_bar, chunk_off, topk_idx, K_loc, V_loc, loc
                 p = np.exp(logits - m)
                 out[b, t, g] = (p[:, None] * V_ctx[:, h]).sum(axis=0) / p.sum()
     return out
+
+
+# ----------------------------------------------------------------------------
+# Router training signal: the contrastive auxiliary loss
+#   L_aux = -(1/|P|) sum_i log( exp(s_i^+/tau) / (exp(s_i^+/tau) + sum_j exp(s_ij^-/tau)) )
+#   [IRMaD M&M, training item: per-layer routing supervision that separates
+#   positive from negative document chunks; digest "Core method"]
+# Reading: a score s is the routing score of the chunk, the head mean of the
+# cosines between the router query and the pooled router key (the S_ij of the
+# routing formula with one query token).
+# ----------------------------------------------------------------------------
+def _norm_clamped(a):
+    n = np.sqrt((a * a).sum(-1))
+    return np.maximum(n, EPS), n > EPS
+
+
+def aux_loss(QR, K_pos, K_neg, tau: float):
+    """Loss and gradients of L_aux for P positives, each with N negatives.
+
+    QR [P, n_r, d_r], K_pos [P, n_r, d_r], K_neg [P, N, n_r, d_r] (bf16 bits or float).
+    Returns (loss, dQR, dK_pos, dK_neg) in float64.  A norm below EPS is clamped
+    (its gradient through the clamp is zero).
+    """
+    def f64(x):
+        x = np.asarray(x)
+        return bf16_to_f64(x) if x.dtype == np.uint16 else x.astype(np.float64)
+
+    Q, Kp, Kn = f64(QR), f64(K_pos), f64(K_neg)
+    P, n_r, d_r = Q.shape
+    N = Kn.shape[1]
+    loss = 0.0
+    dQ = np.zeros_like(Q)
+    dKp = np.zeros_like(Kp)
+    dKn = np.zeros_like(Kn)
+    for i in range(P):
+        keys = np.concatenate([Kp[i][None], Kn[i]], axis=0)      # [1 + N, n_r, d_r], positive first
+        nq, q_live = _norm_clamped(Q[i])                            # [n_r]
+        nk, k_live = _norm_clamped(keys)                            # [1 + N, n_r]
+        dots = (keys * Q[i][None]).sum(-1)                          # [1 + N, n_r]
+        cos = dots / (nq[None] * nk)
+        s = cos.mean(axis=1)                                        # [1 + N] routing scores
+        z = s / tau
+        zmax = z.max()
+        w = np.exp(z - zmax)
+        p = w / w.sum()                                             # softmax over positive + negatives
+        loss += -(z[0] - zmax - math.log(w.sum())) / P
+        g = p / (tau * P)                                           # dL/ds_j for the negatives
+        g[0] = -(1.0 - p[0]) / (tau * P)                            # dL/ds for the positive
+        for j in range(1 + N):
+            for h in range(n_r):
+                gc = g[j] / n_r                                     # through the head mean
+                # d cos / d q = k / (|q||k|) - cos * q / |q|^2   (the second term only off the clamp)
+                dq = keys[j, h] / (nq[h] * nk[j, h])
+                if q_live[h]:
+                    dq = dq - cos[j, h] * Q[i, h] / (nq[h] ** 2)
+                dk = Q[i, h] / (nq[h] * nk[j, h])
+                if k_live[j, h]:
+                    dk = dk - cos[j, h] * keys[j, h] / (nk[j, h] ** 2)
+                dQ[i, h] += gc * dq
+                if j == 0:
+                    dKp[i, h] += gc * dk
+                else:
+                    dKn[i, j - 1, h] += gc * dk
+    return loss, dQ, dKp, dKn

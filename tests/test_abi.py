@@ -144,6 +144,18 @@ def test_encode_validation(msa):
         assert r == want, (layout, r, msa.lib.msa_last_error())
 
 
+def test_append_validation(msa):
+    dd = msa.Dims.of(_dims())
+    need = msa.lib.msa_encode_workspace_size(ctypes.byref(dd), 1000, 3, 20)
+    # 20 new chunks after 90 do not fit a capacity of 100
+    r = msa.lib.msa_append_memory(ctypes.byref(dd), FAKE, 1000, FAKE, 3, FAKE, 20, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                  100, FAKE, 30, 90, 0x100000, need, None)
+    assert r == 1 and "capacity" in msa.lib.msa_last_error().decode()
+    r = msa.lib.msa_append_memory(ctypes.byref(dd), FAKE, 1000, FAKE, 3, FAKE, 20, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                  200, None, 30, 90, 0x100000, need, None)
+    assert r == 1                                                              # NULL chunk_off
+
+
 def test_topk_merge_validation(msa):
     lib = msa.lib
     assert lib.msa_topk_merge(FAKE, FAKE, 1, 8, 9, FAKE, FAKE, None) == 1      # k > n_cand

@@ -147,3 +147,52 @@ def test_encode_1m_tokens_sampled(msa, cuda_device):
     _close(Kg[rows], Kb, "K_bar")
     _close(Vg[rows], Vb, "V_bar")
     _close(KRg[rows], KRb, "KR_bar")
+
+
+def test_append_memory_equals_full_encode(msa, cuda_device):
+    # encode docs A, then append docs B (in two steps) into a memory with spare rows: the rows and the
+    # chunk offsets must equal a single encode of A + B bit for bit (positions restart per document,
+    # chunks never cross documents), and routing over the grown memory must agree with the oracle
+    import torch
+
+    rng = np.random.default_rng(2024)
+    d = W.Dims(hidden=256, n_q=8, n_kv=2, head_dim=64, n_r=4, d_r=64, rope_base=1e6)
+    lens = rng.integers(1, 500, size=23)
+    parts = [lens[:10], lens[10:17], lens[17:]]
+    doc_off = W.offsets_from_lengths(lens)
+    T = int(doc_off[-1])
+    H = W.normal_bf16(rng, (T, 256))
+    WK, WV = W.normal_bf16(rng, (256, 128), 1 / 16), W.normal_bf16(rng, (256, 128), 1 / 16)
+    WKR = W.normal_bf16(rng, (256, 256), 1 / 16)
+    dev = cuda_device
+    Wd = (_dev(WK, dev), _dev(WV, dev), _dev(WKR, dev))
+    co_all, C = msa.chunk_offsets(doc_off)
+    full = msa.encode_memory(d, _dev(H, dev), torch.from_numpy(doc_off).to(dev), torch.from_numpy(co_all).to(dev), C,
+                             *Wd)
+    cap = C + 9
+    mem = (torch.full((cap, 2, 64), 7, dtype=torch.bfloat16, device=dev),
+           torch.full((cap, 2, 64), 7, dtype=torch.bfloat16, device=dev),
+           torch.full((cap, 4, 64), 7, dtype=torch.bfloat16, device=dev))
+    chunk_off = torch.full((len(lens) + 1 + 5,), -1, dtype=torch.int32, device=dev)
+    n_docs, n_chunks, t0 = 0, 0, 0
+    for part in parts:
+        off = W.offsets_from_lengths(part)
+        co, Cn = msa.chunk_offsets(off)
+        Hp = H[t0:t0 + int(off[-1])]
+        n_docs, n_chunks = msa.append_memory(d, _dev(Hp, dev), torch.from_numpy(off).to(dev),
+                                             torch.from_numpy(co).to(dev), Cn, *Wd, mem, chunk_off, n_docs, n_chunks)
+        t0 += int(off[-1])
+    torch.cuda.synchronize()
+    assert msa.check_device_errors() == 0
+    assert (n_docs, n_chunks) == (len(lens), C)
+    assert np.array_equal(chunk_off[:n_docs + 1].cpu().numpy(), co_all)
+    for a, b in zip(mem, full):
+        assert torch.equal(a[:C], b)
+        assert bool((a[C:].float() == 7).all())          # rows past the memory are untouched
+    # routing over the appended memory
+    QR = W.normal_bf16(rng, (2, 256))
+    idx, sc, ds = msa.route_topk(d, _dev(QR, dev), None, mem[2][:C], chunk_off[:n_docs + 1], 5, want_doc_scores=True)
+    _, _, KRb = O.encode_memory(H, doc_off, WK, WV, WKR, 2, 64, 4, 64, rope_base=1e6)
+    s = O.doc_scores(O.chunk_scores(O.bf16_to_f64(QR).reshape(2, 4, 64), W.f32_to_bf16_bits(KRb.astype(np.float32))),
+                     co_all)
+    assert np.max(np.abs(ds.cpu().numpy() - s)) < 2e-3   # stored K̄^R is bf16-rounded; scores from it

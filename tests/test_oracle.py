@@ -438,6 +438,58 @@ def test_attend_tokens_before_local_context_see_only_chunks():
 
 
 # ----------------------------------------------------------------------------
+# router training: L_aux forward and backward
+# ----------------------------------------------------------------------------
+def test_aux_loss_hand_derived_golden():
+    g = json.load(open(os.path.join(GOLD, "aux_loss_hand.json")))
+    Q = np.array(g["q"])[None, None]
+    Kp = np.array(g["k_pos"])[None, None]
+    Kn = np.array(g["k_neg"])[None, None, None]
+    loss, dQ, dKp, dKn = O.aux_loss(Q, Kp, Kn, g["tau"])
+    assert math.isclose(loss, g["loss"], rel_tol=1e-14)
+    assert np.allclose(dQ[0, 0], g["dq"], atol=1e-15)
+    assert np.allclose(dKp[0, 0], g["dk_pos"], atol=1e-15)
+    assert np.allclose(dKn[0, 0, 0], g["dk_neg"], atol=1e-15)
+
+
+def test_aux_loss_gradients_match_finite_differences():
+    rng = np.random.default_rng(21)
+    P, N, n_r, d_r, tau = 3, 4, 2, 5, 0.07
+    Q = rng.standard_normal((P, n_r, d_r))
+    Kp = Q + 0.5 * rng.standard_normal((P, n_r, d_r))
+    Kn = rng.standard_normal((P, N, n_r, d_r))
+    loss, dQ, dKp, dKn = O.aux_loss(Q, Kp, Kn, tau)
+    eps = 1e-6
+    for arr, grad in ((Q, dQ), (Kp, dKp), (Kn, dKn)):
+        for _ in range(12):
+            idx = tuple(rng.integers(0, n) for n in arr.shape)
+            orig = arr[idx]
+            arr[idx] = orig + eps
+            lp = O.aux_loss(Q, Kp, Kn, tau)[0]
+            arr[idx] = orig - eps
+            lm = O.aux_loss(Q, Kp, Kn, tau)[0]
+            arr[idx] = orig
+            fd = (lp - lm) / (2 * eps)
+            assert abs(fd - grad[idx]) <= 1e-7 * max(1.0, abs(fd)), (idx, fd, grad[idx])
+
+
+def test_aux_loss_indistinguishable_negatives_and_batch_mean():
+    rng = np.random.default_rng(22)
+    P, N, n_r, d_r = 2, 6, 3, 8
+    Q = rng.standard_normal((P, n_r, d_r))
+    Kp = rng.standard_normal((P, n_r, d_r))
+    Kn = np.repeat(Kp[:, None], N, axis=1) * 2.5      # same directions: every score equal
+    loss, dQ, dKp, dKn = O.aux_loss(Q, Kp, Kn, 0.1)
+    assert math.isclose(loss, math.log(N + 1), rel_tol=1e-13)
+    assert np.allclose(dQ, 0.0, atol=1e-13)           # the positive's pull cancels the negatives' push
+    # the loss over P positives is the mean of the single-positive losses
+    Kn2 = rng.standard_normal((P, N, n_r, d_r))
+    whole = O.aux_loss(Q, Kp, Kn2, 0.2)[0]
+    parts = [O.aux_loss(Q[i:i + 1], Kp[i:i + 1], Kn2[i:i + 1], 0.2)[0] for i in range(P)]
+    assert math.isclose(whole, sum(parts) / P, rel_tol=1e-13)
+
+
+# ----------------------------------------------------------------------------
 # pages' footprint arithmetic
 # ----------------------------------------------------------------------------
 def test_footprint_matches_pages():
