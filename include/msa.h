@@ -216,6 +216,32 @@ msa_status msa_route_topk_static(const msa_dims* dims, const void* Hq, const voi
                                  float* topk_score, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Router training: the contrastive auxiliary loss and its gradients.
+ * Pages: IRMaD "M. Materials & Methods", training item:
+ *   L_aux = -(1/|P|) sum_i log( exp(s_i^+/tau) / (exp(s_i^+/tau) + sum_j exp(s_ij^-/tau)) ),
+ * applied to every layer's router (the digest's "Core method": it supervises the
+ * routing decision that top-k alone cannot pass a gradient through).  Reading: a
+ * score s is the routing score of a chunk, the head mean of the cosines between
+ * the router query and the chunk's pooled router key (one query token).
+ *   QR       [P, n_r, d_r] bf16 router queries, one per positive.
+ *   K_pos    [P, n_r, d_r] bf16 pooled router key of each positive chunk.
+ *   K_neg    [P, N, n_r, d_r] bf16 pooled router keys of its N negatives (NULL if N = 0).
+ *   tau      temperature, > 0.
+ *   loss     [1] fp32 device out.
+ *   grad_QR, grad_K_pos [P, n_r, d_r], grad_K_neg [P, N, n_r, d_r] fp32 device out;
+ *            each optional (NULL = not computed).
+ *   ws       >= msa_aux_loss_workspace_size bytes, 256-byte aligned.
+ * A norm below 1e-12 is clamped (cosine 0 for a zero vector) and contributes no
+ * gradient through the clamp.  fp32 arithmetic throughout; the loss is summed
+ * in positive order, independent of scheduling.
+ * Limits: 1 <= P <= 2^20; 0 <= N <= 1023; n_r <= 8; d_r in {64, 128}.
+ * ------------------------------------------------------------------------- */
+size_t msa_aux_loss_workspace_size(const msa_dims* dims, int32_t P, int32_t N);
+msa_status msa_aux_loss(const msa_dims* dims, const void* QR, const void* K_pos, const void* K_neg, int32_t P,
+                        int32_t N, float tau, float* loss, float* grad_QR, float* grad_K_pos, float* grad_K_neg,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Stage 3 - sparse generation attention (one decode step).
  * Pages: IRMaD "M. Materials & Methods", routing item (K_ctx = [{K̄_i}_{i in I};
  * K_q], V_ctx likewise, Output = Attention(Q_q, K_ctx, V_ctx)) and position item

@@ -7,7 +7,7 @@ current stream.  Importing this package fails loudly when the library is
 missing; there is no CPU fallback.
 
 Entry points (same names as the C ABI, minus the ``msa_`` prefix):
-  chunk_offsets, encode_memory, append_memory, route_topk, sparse_attend,
+  chunk_offsets, encode_memory, append_memory, route_topk, sparse_attend, aux_loss,
   *_workspace_size, check_device_errors, trace_*.
 """
 from __future__ import annotations
@@ -18,6 +18,7 @@ from typing import Optional
 
 __all__ = [
     "Dims", "MSAError", "lib", "chunk_offsets", "encode_memory", "append_memory", "route_topk", "sparse_attend",
+    "aux_loss",
     "route_workspace_size", "attend_workspace_size", "rope_cache_build", "topk_merge", "rope_rows", "gather_kv", "encode_workspace_size", "check_device_errors",
     "trace_enable", "trace_reset", "trace_read", "trace_kernel_names", "AGG_MAX", "AGG_MEAN",
 ]
@@ -65,6 +66,8 @@ def _load():
         "msa_encode_workspace_size": (SZ, [DP, I64, I32, I32]),
         "msa_encode_memory": (I32, [DP, P, I64, P, I32, P, I32, P, P, P, P, P, P, I32, P, SZ, P]),
         "msa_append_memory": (I32, [DP, P, I64, P, I32, P, I32, P, P, P, P, P, P, I32, P, I32, I32, P, SZ, P]),
+        "msa_aux_loss_workspace_size": (SZ, [DP, I32, I32]),
+        "msa_aux_loss": (I32, [DP, P, P, P, I32, I32, F, P, P, P, P, P, SZ, P]),
         "msa_route_workspace_size": (SZ, [DP, I32, I32, I32, I32, I32, I32]),
         "msa_route_topk": (I32, [DP, P, P, I32, I32, P, P, I32, I32, I32, I32, I32, P, P, P, P, SZ, P]),
         "msa_attend_workspace_size": (SZ, [DP, I32, I32, I32, I32, I32]),
@@ -329,6 +332,33 @@ def sparse_attend(dims, q, K_bar, V_bar, chunk_off, topk_idx, K_loc, V_loc, loc_
                                  t_loc_max, pos_offset, _ptr(rope_cache), int(bool(k_loc_rotated)),
                                  float(softmax_scale), _ptr(out),
                                  _aligned_ptr(ws), nbytes, _stream(stream)))
+    return out
+
+
+# ----------------------------------------------------------------------------
+# router training
+# ----------------------------------------------------------------------------
+def aux_loss(dims, QR, K_pos, K_neg, tau: float, grads: bool = True, out=None, ws=None, stream=None):
+    """Contrastive routing loss L_aux and (optionally) its gradients.
+
+    QR, K_pos [P, n_r, d_r] bf16; K_neg [P, N, n_r, d_r] bf16 (N may be 0).  Returns
+    (loss [1] fp32, dQR, dK_pos, dK_neg) with fp32 gradients, or None for each when grads=False.
+    """
+    import torch
+
+    P = QR.shape[0]
+    N = K_neg.shape[1] if K_neg is not None else 0
+    dev = QR.device
+    if out is None:
+        out = (torch.empty(1, dtype=torch.float32, device=dev),
+               torch.empty(tuple(QR.shape), dtype=torch.float32, device=dev) if grads else None,
+               torch.empty(tuple(K_pos.shape), dtype=torch.float32, device=dev) if grads else None,
+               torch.empty(tuple(K_neg.shape), dtype=torch.float32, device=dev) if grads and N > 0 else None)
+    nbytes = int(lib.msa_aux_loss_workspace_size(ctypes.byref(Dims.of(dims)), P, N))
+    ws = _workspace(nbytes, dev, ws)
+    _check(lib.msa_aux_loss(ctypes.byref(Dims.of(dims)), _ptr(QR), _ptr(K_pos), _ptr(K_neg) if N > 0 else None, P, N,
+                            float(tau), _ptr(out[0]), _ptr(out[1]), _ptr(out[2]), _ptr(out[3]), _aligned_ptr(ws),
+                            nbytes, _stream(stream)))
     return out
 
 

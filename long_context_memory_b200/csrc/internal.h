@@ -50,6 +50,7 @@ enum KernelId : int {
   kKGatherPlan,
   kKGatherCopy,
   kKChunkOffExtend,
+  kKAuxLoss,
   kKernelCount
 };
 
@@ -140,6 +141,14 @@ msa_status gather_kv_launch(const msa_dims& d, const void* K_host, const void* V
 msa_status rope_rows_launch(const msa_dims& d, void* x, int rows, int heads, const int32_t* pos, cudaStream_t s);
 msa_status rope_cache_build(const msa_dims& d, int t_loc_max, int pos_offset, float2* tab, cudaStream_t s);
 
+struct AuxWs {
+  float* term;        // [P] per-positive loss terms
+  uint32_t* ticket;   // CTAs finished
+};
+size_t aux_workspace(const msa_dims& d, int P, int N, void* ws, AuxWs* out);
+msa_status aux_loss_launch(const msa_dims& d, const void* QR, const void* K_pos, const void* K_neg, int P, int N,
+                           float tau, float* loss, float* dQ, float* dK_pos, float* dK_neg, void* ws,
+                           cudaStream_t s);
 msa_status chunk_off_extend_launch(int32_t* chunk_off, int n_docs_old, int n_chunks_old, const int32_t* chunk_off_new,
                                    int n_docs_new, cudaStream_t s);
 size_t encode_workspace(const msa_dims& d, int64_t T, int n_docs, int n_chunks, void* ws,

@@ -110,7 +110,7 @@ namespace {
 const char* kKernelNames[kKernelCount] = {
     "router_query", "scan", "topk_slice", "topk_merge", "rope_table", "attn_split", "attn_combine",
     "enc_chunk_map", "enc_transpose_w", "enc_gemm_k", "enc_pool_h", "enc_gemm_pooled", "rope_rows", "gather_plan", "gather_copy",
-    "chunk_off_extend"};
+    "chunk_off_extend", "aux_loss"};
 
 struct TraceState {
   std::mutex mu;
@@ -431,6 +431,36 @@ msa_status msa_rope_cache_build(const msa_dims* dims, int32_t t_loc_max, int32_t
                 msa_rope_cache_size(dims, t_loc_max));
   if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
   return rope_cache_build(*dims, t_loc_max, pos_offset, static_cast<float2*>(cache), static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------ router training ------------------------------
+size_t msa_aux_loss_workspace_size(const msa_dims* dims, int32_t P, int32_t N) {
+  if (!dims || P < 1 || N < 0) return 0;
+  return aux_workspace(*dims, P, N, nullptr, nullptr);
+}
+
+msa_status msa_aux_loss(const msa_dims* dims, const void* QR, const void* K_pos, const void* K_neg, int32_t P,
+                        int32_t N, float tau, float* loss, float* grad_QR, float* grad_K_pos, float* grad_K_neg,
+                        void* ws, size_t ws_bytes, void* stream) {
+  msa_status st = check_dims(dims, false, true);
+  if (st != MSA_OK) return st;
+  if (P < 1 || P > (1 << 20)) return fail(MSA_ERR_INVALID_ARG, "P must be in [1, 2^20] (got %d)", P);
+  if (N < 0 || N > 1023) return fail(MSA_ERR_INVALID_ARG, "N must be in [0, 1023] (got %d)", N);
+  if (!(tau > 0.f) || !std::isfinite(tau)) return fail(MSA_ERR_INVALID_ARG, "tau must be finite and > 0");
+  CHECK_PTR(QR);
+  CHECK_PTR(K_pos);
+  if (N > 0) CHECK_PTR(K_neg);
+  CHECK_PTR(loss);
+  CHECK_OPT_PTR(grad_QR);
+  CHECK_OPT_PTR(grad_K_pos);
+  CHECK_OPT_PTR(grad_K_neg);
+  const size_t need = aux_workspace(*dims, P, N, nullptr, nullptr);
+  if (ws_bytes < need) return fail(MSA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(MSA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
+  if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
+  return aux_loss_launch(*dims, QR, K_pos, K_neg, P, N, tau, loss, grad_QR, grad_K_pos, grad_K_neg, ws,
+                         static_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------ encode ------------------------------

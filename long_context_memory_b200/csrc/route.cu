@@ -84,6 +84,81 @@ size_t rq_smem_bytes(int d_r, int rows) {
   return (size_t)(kRqThreads / 32) * kRqQB * d_r * sizeof(float) + (size_t)kRqQB * rows * sizeof(uint16_t);
 }
 
+// one group of QB queries: stage their slice of H_q, multiply by the W slab, reduce over the
+// row threads and write the split's partial sums
+template <int QB>
+__device__ __forceinline__ void rq_group(const uint16_t* hq, const __nv_bfloat16* wcol, uint4 (&wv)[kRqRows],
+                                         bool resident, int B, int b0, int hidden, int NR, int h, int d_r, int k0,
+                                         int nrows, int split, int split_rows, int cg, int rt, int RT, int CG, int lane,
+                                         int warp, int tid, uint16_t* hs, float* red, float* qpart) {
+  __syncthreads();
+  const int vec = nrows / 8;  // 16-byte vectors per query row
+  for (int i = tid; i < QB * vec; i += kRqThreads) {
+    const int j = i / vec, v = i % vec;
+    uint4 x = make_uint4(0, 0, 0, 0);
+    if (b0 + j < B) x = __ldg(reinterpret_cast<const uint4*>(hq + (size_t)(b0 + j) * hidden + k0) + v);
+    reinterpret_cast<uint4*>(hs + (size_t)j * split_rows)[v] = x;
+  }
+  __syncthreads();
+  float acc[QB][8];
+#pragma unroll
+  for (int j = 0; j < QB; ++j)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[j][c] = 0.f;
+  auto fma_row = [&](const uint4 w4, int r) {
+    float wf[8];
+    float2 t;
+    t = unpack_bf16x2(w4.x); wf[0] = t.x; wf[1] = t.y;
+    t = unpack_bf16x2(w4.y); wf[2] = t.x; wf[3] = t.y;
+    t = unpack_bf16x2(w4.z); wf[4] = t.x; wf[5] = t.y;
+    t = unpack_bf16x2(w4.w); wf[6] = t.x; wf[7] = t.y;
+#pragma unroll
+    for (int j = 0; j < QB; ++j) {
+      const float hv = bf16_bits_to_float(hs[(size_t)j * split_rows + r]);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[j][c] = fmaf(hv, wf[c], acc[j][c]);
+    }
+  };
+  if (resident) {
+#pragma unroll
+    for (int u = 0; u < kRqRows; ++u) {
+      const int r = rt + RT * u;
+      if (r < nrows) fma_row(wv[u], r);
+    }
+  } else {
+    for (int r0 = rt; r0 < nrows; r0 += RT * kRqRows) {
+      uint4 w2[kRqRows];
+#pragma unroll
+      for (int u = 0; u < kRqRows; ++u) {
+        const int r = r0 + RT * u;
+        w2[u] = r < nrows ? __ldg(reinterpret_cast<const uint4*>(wcol + (size_t)r * NR)) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < kRqRows; ++u) {
+        const int r = r0 + RT * u;
+        if (r < nrows) fma_row(w2[u], r);
+      }
+    }
+  }
+  // reduce over the row threads: lanes cg, cg + CG, ... of a warp, then the 8 warps
+#pragma unroll
+  for (int j = 0; j < QB; ++j)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      float v = acc[j][c];
+      for (int o = CG; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane < CG) red[((size_t)warp * kRqQB + j) * d_r + cg * 8 + c] = v;
+    }
+  __syncthreads();
+  for (int i = tid; i < QB * d_r; i += kRqThreads) {
+    const int j = i / d_r, col = i % d_r;
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kRqThreads / 32; ++w) v += red[((size_t)w * kRqQB + j) * d_r + col];
+    if (b0 + j < B) qpart[((size_t)split * B + b0 + j) * NR + h * d_r + col] = v;
+  }
+}
+
 __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
     const __nv_bfloat16* __restrict__ Hq, const __nv_bfloat16* __restrict__ W, int B, int b_pad, int hidden,
     int n_r, int d_r, int nq, int split_rows, float* __restrict__ qpart, uint32_t* __restrict__ head_done,
@@ -123,72 +198,15 @@ __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
       }
     }
     for (int b0 = 0; b0 < B; b0 += kRqQB) {
-      // stage this query group's slice of H_q (zero rows past B)
-      __syncthreads();
-      const int vec = nrows / 8;  // 16-byte vectors per query row
-      for (int i = tid; i < kRqQB * vec; i += kRqThreads) {
-        const int j = i / vec, v = i % vec;
-        uint4 x = make_uint4(0, 0, 0, 0);
-        if (b0 + j < B) x = __ldg(reinterpret_cast<const uint4*>(hq + (size_t)(b0 + j) * hidden + k0) + v);
-        reinterpret_cast<uint4*>(hs + (size_t)j * split_rows)[v] = x;
-      }
-      __syncthreads();
-      float acc[kRqQB][8];
-#pragma unroll
-      for (int j = 0; j < kRqQB; ++j)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[j][c] = 0.f;
-      auto fma_row = [&](const uint4 w4, int r) {
-        float wf[8];
-        float2 t;
-        t = unpack_bf16x2(w4.x); wf[0] = t.x; wf[1] = t.y;
-        t = unpack_bf16x2(w4.y); wf[2] = t.x; wf[3] = t.y;
-        t = unpack_bf16x2(w4.z); wf[4] = t.x; wf[5] = t.y;
-        t = unpack_bf16x2(w4.w); wf[6] = t.x; wf[7] = t.y;
-#pragma unroll
-        for (int j = 0; j < kRqQB; ++j) {
-          const float hv = bf16_bits_to_float(hs[(size_t)j * split_rows + r]);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) acc[j][c] = fmaf(hv, wf[c], acc[j][c]);
-        }
-      };
-      if (resident) {
-#pragma unroll
-        for (int u = 0; u < kRqRows; ++u) {
-          const int r = rt + RT * u;
-          if (r < nrows) fma_row(wv[u], r);
-        }
-      } else {
-        for (int r0 = rt; r0 < nrows; r0 += RT * kRqRows) {
-#pragma unroll
-          for (int u = 0; u < kRqRows; ++u) {
-            const int r = r0 + RT * u;
-            wv[u] = r < nrows ? __ldg(reinterpret_cast<const uint4*>(wcol + (size_t)r * NR)) : make_uint4(0, 0, 0, 0);
-          }
-#pragma unroll
-          for (int u = 0; u < kRqRows; ++u) {
-            const int r = r0 + RT * u;
-            if (r < nrows) fma_row(wv[u], r);
-          }
-        }
-      }
-      // reduce over the row threads: lanes cg, cg + CG, ... of a warp, then the 8 warps
-#pragma unroll
-      for (int j = 0; j < kRqQB; ++j)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          float v = acc[j][c];
-          for (int o = CG; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-          if (lane < CG) red[((size_t)warp * kRqQB + j) * d_r + cg * 8 + c] = v;
-        }
-      __syncthreads();
-      for (int i = tid; i < kRqQB * d_r; i += kRqThreads) {
-        const int j = i / d_r, col = i % d_r;
-        float v = 0.f;
-#pragma unroll
-        for (int w = 0; w < kRqThreads / 32; ++w) v += red[((size_t)w * kRqQB + j) * d_r + col];
-        if (b0 + j < B) qpart[((size_t)split * B + b0 + j) * NR + h * d_r + col] = v;
-      }
+      const int nb = min(kRqQB, B - b0);  // queries in this group (block-uniform)
+      if (nb == 1) rq_group<1>(hq, wcol, wv, resident, B, b0, hidden, NR, h, d_r, k0, nrows, split, split_rows, cg, rt,
+                               RT, CG, lane, warp, tid, hs, red, qpart);
+      else if (nb == 2) rq_group<2>(hq, wcol, wv, resident, B, b0, hidden, NR, h, d_r, k0, nrows, split, split_rows, cg,
+                                    rt, RT, CG, lane, warp, tid, hs, red, qpart);
+      else if (nb <= 4) rq_group<4>(hq, wcol, wv, resident, B, b0, hidden, NR, h, d_r, k0, nrows, split, split_rows, cg,
+                                    rt, RT, CG, lane, warp, tid, hs, red, qpart);
+      else rq_group<8>(hq, wcol, wv, resident, B, b0, hidden, NR, h, d_r, k0, nrows, split, split_rows, cg, rt, RT, CG,
+                       lane, warp, tid, hs, red, qpart);
     }
     // this CTA's partials are written: take a ticket; the head's last CTA goes on
     __threadfence();
@@ -209,19 +227,30 @@ __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
   for (int b = warp; b < b_pad; b += kRqThreads / 32) {
     float v[4] = {0.f, 0.f, 0.f, 0.f};  // dims lane, lane + 32, ... (d_r <= 128)
     float ss = 0.f;
+    if (b < B) {
+      if (W) {
+        // eight splits' loads in flight at a time; the sum still runs in split order
+        const float* src = qpart + (size_t)b * NR + h * d_r + lane;
+        const size_t sstride = (size_t)B * NR;
+        for (int sp0 = 0; sp0 < n_parts; sp0 += 8) {
+          float x[8][4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int i = lane + 32 * e;
-      if (i < d_r && b < B) {
-        if (W) {
-          float x = 0.f;
-          for (int sp = 0; sp < n_parts; ++sp) x += __ldcg(&qpart[((size_t)sp * B + b) * NR + h * d_r + i]);
-          v[e] = x;
-        } else {
-          v[e] = bf16_bits_to_float(hq[(size_t)b * NR + h * d_r + i]);
+          for (int u = 0; u < 8; ++u)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              x[u][e] = (sp0 + u < n_parts && lane + 32 * e < d_r) ? __ldcg(src + (sp0 + u) * sstride + 32 * e) : 0.f;
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[e] += x[u][e];
         }
-        ss = fmaf(v[e], v[e], ss);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (lane + 32 * e < d_r) v[e] = bf16_bits_to_float(hq[(size_t)b * NR + h * d_r + lane + 32 * e]);
       }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) ss = fmaf(v[e], v[e], ss);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -253,15 +282,17 @@ __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
 // A operand, 128B-swizzled TMA boxes) and the head's normalised query terms
 // (B operand: hi and lo bf16 rows, NQ queries).  One thread issues
 //   D[128 chunks, h*NQ .. h*NQ+NQ) += K̄^R_h (128 x d_r) . (q_hi + q_lo)^T
-// into a double-buffered TMEM accumulator; four warps read the same stage from
-// shared memory for the per-chunk squared norms, and after the tile's last
-// head they read D, apply 1/||K̄^R_h||, average the heads and fold each
-// document's maximum into doc_key with one atomicMax per document segment.
+// into a double-buffered TMEM accumulator.  Four norm warps read each stage
+// from shared memory for the per-chunk squared norms and release it at once;
+// four epilogue warps, separate from them, take a finished tile (its TMEM
+// buffer and its norms), apply 1/||K̄^R_h||, average the heads and fold each
+// document's maximum into doc_key with one atomicMax per document segment,
+// while the next tile streams in.
 // --------------------------------------------------------------------------
 constexpr int kScanM = 128;         // chunks per tile (MMA M)
-constexpr int kScanStages = 4;
-constexpr int kScanThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2..9 norms + epilogue
-constexpr int kScanEpiWarps = 8;    // two per TMEM lane quarter
+constexpr int kScanThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2..5 norms, warps 6..9 epilogue
+constexpr int kScanNormWarps = 4;   // one per TMEM lane quarter (32 rows each)
+constexpr int kScanEpiWarps = 4;
 
 struct ScanParams {
   const int32_t* chunk_off;
@@ -283,6 +314,10 @@ struct ScanGeom {
   static constexpr int kKBytes = kHalves * kKBox;
   static constexpr int kQBytes = 2 * kHalves * kQBox;   // hi and lo
   static constexpr int kStageBytes = kKBytes + kQBytes;
+  static constexpr int kStages = (NQ == 16 || DR == 64) ? 5 : 4;
+  static constexpr int kNormBytes = 2 * 8 * kScanM * 4;  // [2 tiles][8 heads][128 rows] fp32
+  static constexpr int kBars = 2 * kStages + 6;
+  static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + kNormBytes + kBars * 8 + 16;
 };
 
 template <int DR, int NQ, bool MEAN>
@@ -291,30 +326,34 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
                                                                const ScanParams p) {
   using Gm = ScanGeom<DR, NQ>;
   constexpr int KS = DR / 16;
+  constexpr int S = Gm::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  float* n2s = reinterpret_cast<float*>(smem + kScanStages * Gm::kStageBytes);  // [2 tiles][8 heads][2 halves][128]
-  uint64_t* full = reinterpret_cast<uint64_t*>(n2s + 2 * 8 * 2 * kScanM);
-  uint64_t* empty = full + kScanStages;
-  uint64_t* tfull = empty + kScanStages;
-  uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  float* n2s = reinterpret_cast<float*>(smem + S * Gm::kStageBytes);  // [2 tiles][8 heads][128]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * Gm::kStageBytes + Gm::kNormBytes);
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;   // [2] MMA of a tile committed
+  uint64_t* tempty = tfull + 2;  // [2] epilogue done with a tile's TMEM buffer and norms
+  uint64_t* nfull = tempty + 2;  // [2] norms of a tile written
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(nfull + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_r = p.n_r;
   const int t_begin = (int)(((long long)blockIdx.x * p.n_tiles) / gridDim.x);
   const int t_end = (int)(((long long)(blockIdx.x + 1) * p.n_tiles) / gridDim.x);
-  const int n_it = (t_end - t_begin) * n_r;  // (tile, head) stages of this CTA
+  const int n_lt = t_end - t_begin;
+  const int n_it = n_lt * n_r;  // (tile, head) stages of this CTA
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kScanStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + kScanEpiWarps);  // MMA commit + the norm warps
+      mbar_init(&empty[s], 1 + kScanNormWarps);  // MMA commit + the norm warps
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], kScanEpiWarps);
+      mbar_init(&nfull[b], kScanNormWarps);
     }
     fence_mbar_init();
     prefetch_tensormap(&kr_map);
@@ -337,8 +376,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     if (lane == 0) {
       for (int it = 0; it < n_it; ++it) {
         const int tile = t_begin + it / n_r, h = it % n_r;
-        const int st = it % kScanStages;
-        if (it >= kScanStages) mbar_wait(&empty[st], ((it / kScanStages) - 1) & 1);
+        const int st = it % S;
+        if (it >= S) mbar_wait(&empty[st], ((it / S) - 1) & 1);
         uint8_t* k_s = stages + st * Gm::kStageBytes;
         uint8_t* q_s = k_s + Gm::kKBytes;
         mbar_arrive_expect_tx(&full[st], Gm::kStageBytes);
@@ -362,9 +401,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       for (int it = 0; it < n_it; ++it) {
         const int lt = it / n_r, h = it % n_r;
         const int buf = lt & 1;
-        const int st = it % kScanStages;
+        const int st = it % S;
         if (h == 0 && lt >= 2) mbar_wait(&tempty[buf], ((lt >> 1) - 1) & 1);
-        mbar_wait(&full[st], (it / kScanStages) & 1);
+        mbar_wait(&full[st], (it / S) & 1);
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * buf_cols + h * NQ;
         const uint32_t k_addr = smem_u32(stages + st * Gm::kStageBytes);
@@ -380,73 +419,68 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         if (h == n_r - 1) umma_commit(&tfull[buf]);
       }
     }
-  } else {
-    // ------- norm + epilogue warps: TMEM lane quarter = warp % 4, half = which pair member -------
-    constexpr int QH = NQ / 2;                 // queries per half
-    const int q4 = warp & 3;
-    const int hf = (warp - 2) >> 2;            // 0 or 1
-    const int row = 32 * q4 + lane;            // chunk within the tile
-    int cur = 0;                               // lower bound for this warp's document search
+  } else if (warp < 2 + kScanNormWarps) {
+    // ------- norm warps: squared norm of every row's head-h slice, stage released at once -------
+    const int row = 32 * (warp & 3) + lane;  // chunk within the tile
     for (int it = 0; it < n_it; ++it) {
       const int lt = it / n_r, h = it % n_r;
-      const int st = it % kScanStages;
-      mbar_wait(&full[st], (it / kScanStages) & 1);
-      // partial squared norm of this row's head-h slice (this warp's half of the dims)
+      const int buf = lt & 1;
+      const int st = it % S;
+      if (h == 0 && lt >= 2) mbar_wait(&tempty[buf], ((lt >> 1) - 1) & 1);  // n2s[buf] is free again
+      mbar_wait(&full[st], (it / S) & 1);
       const uint8_t* k_s = stages + st * Gm::kStageBytes;
       float n2p[4] = {0.f, 0.f, 0.f, 0.f};
-      constexpr int UN = (Gm::kHalves == 2) ? 8 : 4;   // 16-byte units per half
 #pragma unroll
-      for (int uu = 0; uu < UN; ++uu) {
-        const int j = (Gm::kHalves == 2) ? hf : 0;
-        const int u = (Gm::kHalves == 2) ? uu : 4 * hf + uu;
-        const uint4 w = *reinterpret_cast<const uint4*>(k_s + j * Gm::kKBox + row * 128 + ((u ^ (row & 7)) << 4));
-        float2 f;
-        f = unpack_bf16x2(w.x); n2p[0] = fmaf(f.x, f.x, n2p[0]); n2p[1] = fmaf(f.y, f.y, n2p[1]);
-        f = unpack_bf16x2(w.y); n2p[2] = fmaf(f.x, f.x, n2p[2]); n2p[3] = fmaf(f.y, f.y, n2p[3]);
-        f = unpack_bf16x2(w.z); n2p[0] = fmaf(f.x, f.x, n2p[0]); n2p[1] = fmaf(f.y, f.y, n2p[1]);
-        f = unpack_bf16x2(w.w); n2p[2] = fmaf(f.x, f.x, n2p[2]); n2p[3] = fmaf(f.y, f.y, n2p[3]);
+      for (int j = 0; j < Gm::kHalves; ++j) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 w = *reinterpret_cast<const uint4*>(k_s + j * Gm::kKBox + row * 128 + ((u ^ (row & 7)) << 4));
+          float2 f;
+          f = unpack_bf16x2(w.x); n2p[0] = fmaf(f.x, f.x, n2p[0]); n2p[1] = fmaf(f.y, f.y, n2p[1]);
+          f = unpack_bf16x2(w.y); n2p[2] = fmaf(f.x, f.x, n2p[2]); n2p[3] = fmaf(f.y, f.y, n2p[3]);
+          f = unpack_bf16x2(w.z); n2p[0] = fmaf(f.x, f.x, n2p[0]); n2p[1] = fmaf(f.y, f.y, n2p[1]);
+          f = unpack_bf16x2(w.w); n2p[2] = fmaf(f.x, f.x, n2p[2]); n2p[3] = fmaf(f.y, f.y, n2p[3]);
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
-      n2s[(((lt & 1) * 8 + h) * 2 + hf) * kScanM + row] = (n2p[0] + n2p[1]) + (n2p[2] + n2p[3]);
-      if (h != n_r - 1) continue;
-
-      // ---- epilogue of tile lt: head mean of cosines, per-document max ----
+      n2s[(buf * 8 + h) * kScanM + row] = (n2p[0] + n2p[1]) + (n2p[2] + n2p[3]);
+      if (h == n_r - 1) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&nfull[buf]);
+      }
+    }
+  } else {
+    // ------- epilogue warps: head mean of cosines, per-document max (TMEM lane quarter = warp % 4) -------
+    const int q4 = warp & 3;
+    const int row = 32 * q4 + lane;  // chunk within the tile
+    int cur = 0;                     // lower bound for this warp's document search
+    for (int lt = 0; lt < n_lt; ++lt) {
       const int tile = t_begin + lt;
       const int buf = lt & 1;
-      named_bar_sync(1 + q4, 64);  // both halves of this lane quarter have written their norms
-      const float* nb2 = n2s + (size_t)(lt & 1) * 8 * 2 * kScanM;
+      mbar_wait(&nfull[buf], (lt >> 1) & 1);
       mbar_wait(&tfull[buf], (lt >> 1) & 1);
       tc_fence_after();
-      float acc[QH];
+      const float* nb2 = n2s + (size_t)buf * 8 * kScanM;
+      float acc[NQ];
 #pragma unroll
-      for (int b = 0; b < QH; ++b) acc[b] = 0.f;
-      const bool any_q = hf * QH < p.q_count;
-      const uint32_t t_row = tmem_base + ((uint32_t)(32 * q4) << 16) + buf * buf_cols + hf * QH;
+      for (int b = 0; b < NQ; ++b) acc[b] = 0.f;
+      const uint32_t t_row = tmem_base + ((uint32_t)(32 * q4) << 16) + buf * buf_cols;
 #pragma unroll
       for (int hh = 0; hh < 8; ++hh) {
-        if (hh < n_r && any_q) {
-          const float n2 = nb2[(hh * 2 + 0) * kScanM + row] + nb2[(hh * 2 + 1) * kScanM + row];
-          const float inv = 1.0f / fmaxf(sqrtf(n2), kEps);
-          if constexpr (QH == 16) {
-            float v[16];
-            tmem_ld16(t_row + hh * NQ, v);
-            tmem_ld_wait();
+        if (hh < n_r) {
+          const float inv = 1.0f / fmaxf(sqrtf(nb2[hh * kScanM + row]), kEps);
+          float v[NQ];
+          if constexpr (NQ == 16) tmem_ld16(t_row + hh * NQ, v);
+          else tmem_ld32(t_row + hh * NQ, v);
+          tmem_ld_wait();
 #pragma unroll
-            for (int b = 0; b < 16; ++b) acc[b] = fmaf(v[b], inv, acc[b]);
-          } else {
-            float v[8];
-            tmem_ld8(t_row + hh * NQ, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int b = 0; b < 8; ++b) acc[b] = fmaf(v[b], inv, acc[b]);
-          }
+          for (int b = 0; b < NQ; ++b) acc[b] = fmaf(v[b], inv, acc[b]);
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
-      if (!any_q) continue;
 
       // documents of this warp's 32 rows: a warp-wide 32-ary search for the first row's
       // document, then one lookahead of 32 document boundaries (32 consecutive rows cross at
@@ -486,10 +520,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         if (lane + (1 << e) < 32 && od == doc) same |= 1u << e;
       }
 #pragma unroll
-      for (int bb = 0; bb < QH; ++bb) {
-        const int b = hf * QH + bb;
-        if (b >= p.q_count) continue;  // warp-uniform
-        const float sc = acc[bb] * p.inv_nr;
+      for (int b = 0; b < NQ; ++b) {
+        if (b >= p.q_count) break;  // warp-uniform
+        const float sc = acc[b] * p.inv_nr;
         const size_t qi = (size_t)((p.q_base + b) / p.q_tokens);  // max over a query's tokens: atomicMax
         if (MEAN) {
           if (doc >= 0) {
@@ -695,8 +728,7 @@ template <int DR, int NQ, bool MEAN>
 cudaError_t launch_scan_t(const CUtensorMap& kmap, const CUtensorMap& qmap, const ScanParams& p, int grid,
                           cudaStream_t s) {
   auto kern = scan_kernel<DR, NQ, MEAN>;
-  const size_t smem = 1024 + (size_t)kScanStages * ScanGeom<DR, NQ>::kStageBytes + 2 * 8 * 2 * kScanM * sizeof(float) +
-                      (2 * kScanStages + 4) * 8 + 16;
+  const size_t smem = ScanGeom<DR, NQ>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(grid), dim3(kScanThreads), smem, s, kmap, qmap, p);

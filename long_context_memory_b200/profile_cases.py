@@ -15,6 +15,8 @@ Cases
   attend1m   sparse attention, 1M-token memory, B = 1, 4K local tokens (rotated key cache)
   attend16m  sparse attention, 16M-token memory, B = 32, 8K local tokens (rotated key cache)
   encode     offline encoding of --tokens tokens (default 1M), hidden 2560
+  aux        router training loss L_aux + gradients: P = 4096 positives x (1 + 63 negatives),
+             8 router heads x 128 (--batch to change P)
 """
 from __future__ import annotations
 
@@ -135,6 +137,28 @@ class AttendCase:
                                k_loc_rotated=self.rotated)
 
 
+class AuxCase:
+    def __init__(self, P, N, seed, device, dims=W.QWEN3_4B_DIMS, tau=0.05):
+        import torch
+
+        import long_context_memory_b200 as msa
+
+        self.msa, self.d, self.tau = msa, dims, tau
+        g = torch.Generator(device=device)
+        g.manual_seed(seed)
+        self.Q = randn_bf16((P, dims.n_r, dims.d_r), g, device)
+        self.Kp = randn_bf16((P, dims.n_r, dims.d_r), g, device)
+        self.Kn = randn_bf16((P, N, dims.n_r, dims.d_r), g, device)
+        self.out = None
+        self.ws = None
+        row = dims.n_r * dims.d_r
+        # HBM bytes: queries and keys read once (bf16), gradients written (fp32)
+        self.bytes = P * (N + 2) * row * 2 + P * (N + 2) * row * 4
+
+    def run(self):
+        self.out = self.msa.aux_loss(self.d, self.Q, self.Kp, self.Kn, self.tau, out=self.out, ws=self.ws)
+
+
 class EncodeCase:
     def __init__(self, T, seed, device, dims=W.QWEN3_4B_DIMS):
         import torch
@@ -170,7 +194,7 @@ def main():
 
     ap = argparse.ArgumentParser()
     ap.add_argument("--case", required=True,
-                    choices=["route1m", "route16m", "route100m", "attend1m", "attend16m", "encode"])
+                    choices=["route1m", "route16m", "route100m", "attend1m", "attend16m", "encode", "aux"])
     ap.add_argument("--launches", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=2)
     ap.add_argument("--batch", type=int, default=None)
@@ -191,6 +215,8 @@ def main():
         case = AttendCase(1_000_000, a.batch or 1, 2048, 4096, seed, dev)
     elif a.case == "attend16m":
         case = AttendCase(16_000_000, a.batch or 32, 2048, 8192, seed, dev)
+    elif a.case == "aux":
+        case = AuxCase(a.batch or 4096, 63, seed, dev)
     else:
         case = EncodeCase(a.tokens or 1_000_000, seed, dev)
     s = torch.cuda.Stream()

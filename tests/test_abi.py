@@ -156,6 +156,23 @@ def test_append_validation(msa):
     assert r == 1                                                              # NULL chunk_off
 
 
+def test_aux_loss_validation(msa):
+    dd = msa.Dims.of(_dims())
+    lib = msa.lib
+    need = lib.msa_aux_loss_workspace_size(ctypes.byref(dd), 4, 8)
+    assert need > 0
+    call = lambda P=4, N=8, tau=0.1, ws=need, kn=FAKE: lib.msa_aux_loss(
+        ctypes.byref(dd), FAKE, FAKE, kn, P, N, tau, FAKE, FAKE, None, None, 0x100000, ws, None)
+    assert call(P=0) == 1
+    assert call(N=1024) == 1
+    assert call(tau=0.0) == 1
+    assert call(tau=float("inf")) == 1
+    assert call(kn=None) == 1            # N > 0 needs negatives
+    assert call(ws=4) == 3
+    assert lib.msa_aux_loss(ctypes.byref(msa.Dims.of(_dims(d_r=96))), FAKE, FAKE, FAKE, 4, 8, 0.1, FAKE, None, None,
+                            None, 0x100000, need, None) == 2
+
+
 def test_topk_merge_validation(msa):
     lib = msa.lib
     assert lib.msa_topk_merge(FAKE, FAKE, 1, 8, 9, FAKE, FAKE, None) == 1      # k > n_cand
