@@ -353,17 +353,15 @@ def run_gpu(args):
         msa.rope_rows(d, x["K_loc"].view(B * T_loc, d.n_kv, d.head_dim),
                       (c["pos_offset"] + torch.arange(T_loc, dtype=torch.int32, device=dev)).repeat(B))
     k_new = base["K_loc"][:, Lm1].clone()          # the new token's key before RoPE (synthetic)
-    kn_buf = torch.empty_like(k_new)
-    new_pos = torch.full((B,), c["pos_offset"] + Lm1, dtype=torch.int32, device=dev)
+    v_new = base["V_loc"][:, Lm1].clone()
+    slots = torch.full((B,), Lm1, dtype=torch.int32, device=dev)
     torch.cuda.synchronize()
 
     def step(i):
         x = rot[i % N_ROT]
         j = i % N_ROT
         msa.route_topk(d, x["Hq"], W_QR, x["KR"], chunk_off, k, out=(out_idx[j], out_sc[j], None), ws=r_ws)
-        kn_buf.copy_(k_new)
-        msa.rope_rows(d, kn_buf, new_pos)
-        x["K_loc"][:, Lm1].copy_(kn_buf)
+        msa.kv_append(d, k_new, v_new, x["K_loc"], x["V_loc"], slots, c["pos_offset"])
         msa.sparse_attend(d, x["q"], x["K_bar"], x["V_bar"], chunk_off, out_idx[j], x["K_loc"], x["V_loc"], loc_len,
                           c["pos_offset"], out=out_o[j], ws=a_ws, k_loc_rotated=True)
 
@@ -456,6 +454,7 @@ def run_gpu(args):
             "k_new": k_new.cpu().contiguous().pin_memory(),
             "v_new": base["V_loc"][:, Lm1].cpu().contiguous().pin_memory()}
     dev_hq, dev_q = torch.empty_like(base["Hq"]), torch.empty_like(base["q"])
+    dev_kn, dev_vn = torch.empty_like(k_new), torch.empty_like(v_new)
     h_idx = torch.empty((B, k), dtype=torch.int32).pin_memory()
     h_sc = torch.empty((B, k), dtype=torch.float32).pin_memory()
     h_out = torch.empty((B, d.n_q, d.head_dim), dtype=torch.bfloat16).pin_memory()
@@ -466,10 +465,9 @@ def run_gpu(args):
         x = rot[i % N_ROT]
         dev_hq.copy_(host["Hq"], non_blocking=True)
         dev_q.copy_(host["q"], non_blocking=True)
-        kn_buf.copy_(host["k_new"], non_blocking=True)
-        msa.rope_rows(d, kn_buf, new_pos)
-        x["K_loc"][:, Lm1].copy_(kn_buf)
-        x["V_loc"][:, Lm1].copy_(host["v_new"], non_blocking=True)
+        dev_kn.copy_(host["k_new"], non_blocking=True)
+        dev_vn.copy_(host["v_new"], non_blocking=True)
+        msa.kv_append(d, dev_kn, dev_vn, x["K_loc"], x["V_loc"], slots, c["pos_offset"])
         msa.route_topk(d, dev_hq, W_QR, x["KR"], chunk_off, k, out=(out_idx[0], out_sc[0], None), ws=r_ws)
         msa.sparse_attend(d, dev_q, x["K_bar"], x["V_bar"], chunk_off, out_idx[0], x["K_loc"], x["V_loc"], loc_len,
                           c["pos_offset"], out=out_o[0], ws=a_ws, k_loc_rotated=True)
@@ -519,8 +517,9 @@ def run_gpu(args):
             "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms},
             "cpu_baseline": cpu, "clocks": clocks, "extras": extras,
-            "notes": "value: device time of CUDA-graph replays of the full decode step (route, rotate+append "
-                     "the new token's key, sparse attention over the rotated local cache); kernels: trace-event "
+            "notes": "value: device time of CUDA-graph replays of the full decode step (route, append the new "
+                     "token's rotated key and value to the local cache, sparse attention over the rotated cache); "
+                     "kernels: trace-event "
                      "brackets of eager launches queued behind a bounded sleep kernel",
         }
         print(json.dumps(line), flush=True)

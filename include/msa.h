@@ -312,12 +312,29 @@ msa_status msa_gather_kv(const msa_dims* dims, const void* K_bar_host, const voi
  * at pos_offset + j) and then runs msa_sparse_attend with k_loc_rotated = 1,
  * instead of re-rotating every local key at every step.
  *   x          [rows, heads, head_dim] bf16, rotated in place (rotate-half pairs
- *              (i, i + head_dim/2), theta_i = rope_base^(-2i/head_dim), angle
- *              reduced in fp64, result rounded to bf16).
+ *              (i, i + head_dim/2), theta_i = rope_base^(-2i/head_dim); the angle
+ *              p * theta_i is reduced exactly, as a 64-bit fraction of a turn;
+ *              result rounded to bf16).
  *   positions  [rows] device int32, absolute positions.
  * ------------------------------------------------------------------------- */
 msa_status msa_rope_rows(const msa_dims* dims, void* x, int32_t rows, int32_t heads, const int32_t* positions,
                          void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Append one token per query to a rotated local KV cache.
+ * Pages: IRMaD "M. Materials & Methods", position item (global RoPE on the
+ * active context: local token j at pos_offset + j).  The decode step's new
+ * token joins the local context: its key is rotated at its global position and
+ * written, with its value, into the cache slot, in one launch.
+ *   k_new, v_new  [B, n_kv, head_dim] bf16, the new token's key (before RoPE) and value.
+ *   K_loc, V_loc  [B, t_loc_max, n_kv, head_dim] bf16 cache; row slots[b] of query b is
+ *            written: K_loc = RoPE(k_new[b], pos_offset + slots[b]), V_loc = v_new[b].
+ *   slots    [B] device int32, 0 <= slots[b] < t_loc_max (a slot outside is skipped and
+ *            the device error word records it).
+ * The result equals msa_rope_rows on a copy of k_new followed by the two row copies.
+ * ------------------------------------------------------------------------- */
+msa_status msa_kv_append(const msa_dims* dims, const void* k_new, const void* v_new, void* K_loc, void* V_loc,
+                         int32_t B, int32_t t_loc_max, const int32_t* slots, int32_t pos_offset, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Global-RoPE cache for the active context (optional input of msa_sparse_attend).

@@ -7,7 +7,7 @@ current stream.  Importing this package fails loudly when the library is
 missing; there is no CPU fallback.
 
 Entry points (same names as the C ABI, minus the ``msa_`` prefix):
-  chunk_offsets, encode_memory, append_memory, route_topk, sparse_attend, aux_loss,
+  chunk_offsets, encode_memory, append_memory, route_topk, sparse_attend, kv_append, aux_loss,
   *_workspace_size, check_device_errors, trace_*.
 """
 from __future__ import annotations
@@ -18,7 +18,7 @@ from typing import Optional
 
 __all__ = [
     "Dims", "MSAError", "lib", "chunk_offsets", "encode_memory", "append_memory", "route_topk", "sparse_attend",
-    "aux_loss",
+    "aux_loss", "kv_append",
     "route_workspace_size", "attend_workspace_size", "rope_cache_build", "topk_merge", "rope_rows", "gather_kv", "encode_workspace_size", "check_device_errors",
     "trace_enable", "trace_reset", "trace_read", "trace_kernel_names", "AGG_MAX", "AGG_MEAN",
 ]
@@ -74,6 +74,7 @@ def _load():
         "msa_sparse_attend": (I32, [DP, P, I32, I32, P, P, P, I32, I32, P, I32, P, P, P, I32, I32, P, I32, F, P, P, SZ,
                                     P]),
         "msa_rope_rows": (I32, [DP, P, I32, I32, P, P]),
+        "msa_kv_append": (I32, [DP, P, P, P, P, I32, I32, P, I32, P]),
         "msa_gather_kv": (I32, [DP, P, P, I32, P, I32, P, I32, I32, P, P, I32, P, P, P, SZ, P]),
         "msa_rope_cache_size": (SZ, [DP, I32]),
         "msa_rope_cache_build": (I32, [DP, I32, I32, P, SZ, P]),
@@ -304,6 +305,17 @@ def rope_rows(dims, x, positions, stream=None):
     rows, heads = x.shape[0], x.shape[1]
     _check(lib.msa_rope_rows(ctypes.byref(Dims.of(dims)), _ptr(x), rows, heads, _ptr(positions), _stream(stream)))
     return x
+
+
+def kv_append(dims, k_new, v_new, K_loc, V_loc, slots, pos_offset: int, stream=None):
+    """Write the new token of every query into the rotated local cache, in place.
+
+    k_new, v_new [B, n_kv, head_dim]; K_loc, V_loc [B, t_loc_max, n_kv, head_dim]; slots [B] int32
+    (device): K_loc[b, slots[b]] = RoPE(k_new[b], pos_offset + slots[b]), V_loc[b, slots[b]] = v_new[b].
+    """
+    B, t_loc_max = K_loc.shape[0], K_loc.shape[1]
+    _check(lib.msa_kv_append(ctypes.byref(Dims.of(dims)), _ptr(k_new), _ptr(v_new), _ptr(K_loc), _ptr(V_loc), B,
+                             t_loc_max, _ptr(slots), pos_offset, _stream(stream)))
 
 
 def sparse_attend(dims, q, K_bar, V_bar, chunk_off, topk_idx, K_loc, V_loc, loc_len, pos_offset: int,

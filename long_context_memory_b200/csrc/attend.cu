@@ -522,6 +522,38 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(__nv_bfloat16* __restric
   }
 }
 
+// the decode step's new token into the rotated cache: CTA = one query; key rotated at
+// pos_offset + slot, value copied (D/2 pairs x n_kv heads per thread block)
+template <int D>
+__global__ void __launch_bounds__(256) kv_append_kernel(const __nv_bfloat16* __restrict__ k_new,
+                                                        const __nv_bfloat16* __restrict__ v_new,
+                                                        __nv_bfloat16* __restrict__ K_loc,
+                                                        __nv_bfloat16* __restrict__ V_loc, int n_kv, int t_loc_max,
+                                                        const int32_t* __restrict__ slots, int pos_offset,
+                                                        const RopeTurns turns) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int b = blockIdx.x;
+  const int slot = slots[b];
+  if (slot < 0 || slot >= t_loc_max) {
+    if (threadIdx.x == 0) raise_dev_error(kDevErrBadIndex);
+    return;
+  }
+  const size_t src = (size_t)b * n_kv * D;
+  const size_t dst = ((size_t)b * t_loc_max + slot) * n_kv * D;
+  for (int e = threadIdx.x; e < n_kv * (D / 2); e += blockDim.x) {
+    const int h = e / (D / 2), i = e % (D / 2);
+    const float2 cs = rope_cos_sin(turns, i, (int64_t)pos_offset + slot);
+    const __nv_bfloat16* kr = k_new + src + (size_t)h * D;
+    const float x1 = __bfloat162float(kr[i]), x2 = __bfloat162float(kr[i + D / 2]);
+    __nv_bfloat16* kd = K_loc + dst + (size_t)h * D;
+    kd[i] = __float2bfloat16_rn(x1 * cs.x - x2 * cs.y);
+    kd[i + D / 2] = __float2bfloat16_rn(x2 * cs.x + x1 * cs.y);
+  }
+  for (int e = threadIdx.x; e < n_kv * D / 8; e += blockDim.x)
+    reinterpret_cast<uint4*>(V_loc + dst)[e] = __ldg(reinterpret_cast<const uint4*>(v_new + src) + e);
+}
+
 // splits per query: enough CTAs for about four waves, rounded so that B * splits is a
 // whole number of waves on this GPU (one CTA per SM), and at least ~32 keys per split
 int choose_splits(int B, int t_loc_max, int k) {
@@ -700,6 +732,24 @@ msa_status rope_rows_launch(const msa_dims& d, void* x, int rows, int heads, con
   else
     MSA_CUDA_CHECK(launch_pdl(rope_rows_kernel<64>, dim3(blocks), dim3(256), 0, s, static_cast<__nv_bfloat16*>(x),
                               rows, heads, pos, turns));
+  return MSA_OK;
+}
+
+msa_status kv_append_launch(const msa_dims& d, const void* k_new, const void* v_new, void* K_loc, void* V_loc, int B,
+                            int t_loc_max, const int32_t* slots, int pos_offset, cudaStream_t s) {
+  TraceScope ts(kKKvAppend, s);
+  RopeTurns turns;
+  rope_turns(d, turns.f);
+  auto kb = static_cast<const __nv_bfloat16*>(k_new);
+  auto vb = static_cast<const __nv_bfloat16*>(v_new);
+  auto Kl = static_cast<__nv_bfloat16*>(K_loc);
+  auto Vl = static_cast<__nv_bfloat16*>(V_loc);
+  if (d.head_dim == 128)
+    MSA_CUDA_CHECK(launch_pdl(kv_append_kernel<128>, dim3(B), dim3(256), 0, s, kb, vb, Kl, Vl, d.n_kv, t_loc_max, slots,
+                              pos_offset, turns));
+  else
+    MSA_CUDA_CHECK(launch_pdl(kv_append_kernel<64>, dim3(B), dim3(256), 0, s, kb, vb, Kl, Vl, d.n_kv, t_loc_max, slots,
+                              pos_offset, turns));
   return MSA_OK;
 }
 

@@ -6,17 +6,20 @@
 // with s the routing score of a chunk: the head mean of the cosines between
 // the router query and the chunk's pooled router key.
 //
-// Kernel aux_loss_kernel: CTA = one positive i (its query, its positive key
-// and its N negative keys).  Pass 1 reads every key once (lane = 8 or 16
-// consecutive 16-byte pieces of one head) for the per-head dot products and
-// norms, giving the cosines and scores; a block softmax over the 1 + N scores
-// gives the loss term and dL/ds.  Pass 2 re-reads the keys (L2-resident: this
-// CTA just streamed them) and forms
+// Kernel aux_loss_kernel: a persistent grid; CTA c takes positives c, c + grid, ...
+// One producer warp streams every positive's 1 + N key rows (positive first)
+// through a shared-memory ring with bulk async copies, 8 rows per stage, twice:
+// pass 1 (from HBM) for the per-head dot products and norms -> cosines ->
+// scores -> a block softmax -> the loss term and dL/ds; pass 2 (the same rows,
+// now in L2) for
 //   dL/dq_h = (1/n_r) sum_j g_j (k_jh / (|q_h||k_jh|) - cos_jh q_h / |q_h|^2)
 //   dL/dk_jh = (g_j/n_r)      (q_h / (|q_h||k_jh|) - cos_jh k_jh / |k_jh|^2)
-// (a norm below eps is clamped and its own term dropped).  The per-CTA loss
-// terms are summed in positive order by the last CTA (a ticket), so the loss
-// does not depend on scheduling.
+// (a norm below eps is clamped and its own term dropped).  The producer runs
+// ahead into the next positive while the compute warps finish the current one,
+// so the copy engine never waits on the softmax.  Eight compute warps, one key
+// row each per stage; lane = (head, quarter of the head), its query values in
+// registers.  The per-positive loss terms are summed in positive order by the
+// last CTA (a ticket), so the loss does not depend on scheduling.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -30,8 +33,10 @@
 namespace msa {
 namespace {
 
-constexpr int kAuxThreads = 256;
-constexpr int kAuxWarps = kAuxThreads / 32;
+constexpr int kAuxCompute = 8;                      // compute warps
+constexpr int kAuxThreads = 32 * (kAuxCompute + 1);  // + the producer warp
+constexpr int kAuxRows = 8;                         // key rows per stage (one per compute warp)
+constexpr int kAuxStages = 6;
 constexpr float kAuxEps = 1e-12f;
 
 struct AuxParams {
@@ -43,193 +48,265 @@ struct AuxParams {
   float* dK_pos;               // [P][n_r][d_r] or null
   float* dK_neg;               // [P][N][n_r][d_r] or null
   float* term;                 // [P] per-positive loss terms (workspace)
-  uint32_t* ticket;            // [1] CTAs done (workspace, back to 0 after each call)
+  uint32_t* ticket;            // [1] CTAs done (workspace)
   int P, N, n_r;
   float inv_tau;
 };
 
-// lane -> (head, 16-byte pieces): 4 lanes per head, DR/32 bf16 values per lane
+// shared memory: ring [kAuxStages][kAuxRows][n_r * DR] bf16 | cos, |k| [NK][8] fp32 | g [NK] |
+// dq partials [kAuxCompute][n_r * DR] fp32 | barriers
 template <int DR>
-struct AuxLane {
-  static constexpr int kVals = DR / 4;   // values per lane (32 or 16)
-  static constexpr int kVecs = kVals / 8;  // uint4 per lane (4 or 2)
+struct AuxSmem {
+  static constexpr int kRowBytes = 8 * DR * 2;  // room for 8 router heads
+  static constexpr int kStageBytes = kAuxRows * kRowBytes;
+  static __host__ __device__ size_t bytes(int nk) {
+    return (size_t)kAuxStages * kStageBytes + (size_t)nk * 8 * 4 * 2 + (size_t)nk * 4 +
+           (size_t)kAuxCompute * 8 * DR * 4 + 2 * kAuxStages * 8 + 16;
+  }
 };
 
+// lane l of a compute warp owns head l / 4, quarter l % 4: U 16-byte units of the row.
+// Slot e of a lane holds unit (e + rot) % U of its quarter (rot = l / (8 / U)), so that a
+// warp's 16-byte loads from shared memory fall in 8 distinct bank groups (4 wavefronts, no
+// conflict).  Every per-lane array (key values, query values, gradient partials) is kept
+// in slot order; only addresses are rotated.
 template <int DR>
-__device__ __forceinline__ void load_key(const __nv_bfloat16* row, int h, int part, float* v) {
-  using Ln = AuxLane<DR>;
-  const uint4* src = reinterpret_cast<const uint4*>(row + (size_t)h * DR + part * Ln::kVals);
-  uint4 u[Ln::kVecs];
-#pragma unroll
-  for (int e = 0; e < Ln::kVecs; ++e) u[e] = __ldg(src + e);
-#pragma unroll
-  for (int e = 0; e < Ln::kVecs; ++e) {
-    float2 f;
-    f = unpack_bf16x2(u[e].x); v[8 * e + 0] = f.x; v[8 * e + 1] = f.y;
-    f = unpack_bf16x2(u[e].y); v[8 * e + 2] = f.x; v[8 * e + 3] = f.y;
-    f = unpack_bf16x2(u[e].z); v[8 * e + 4] = f.x; v[8 * e + 5] = f.y;
-    f = unpack_bf16x2(u[e].w); v[8 * e + 6] = f.x; v[8 * e + 7] = f.y;
-  }
+__device__ __forceinline__ int unit_of_slot(int e, int lane) {
+  constexpr int U = DR / 32;
+  return (e + lane / (8 / U)) % U;
 }
 
 template <int DR>
-__global__ void __launch_bounds__(kAuxThreads) aux_loss_kernel(const AuxParams p) {
-  using Ln = AuxLane<DR>;
-  extern __shared__ __align__(16) float aux_sm[];
+__device__ __forceinline__ void load_row_quarter(const uint8_t* row, int lane, float* v) {
+  constexpr int U = DR / 32;  // 16-byte units per lane (4 or 2)
+  const uint8_t* base = row + lane * U * 16;
+#pragma unroll
+  for (int e = 0; e < U; ++e) {
+    const uint4 w = *reinterpret_cast<const uint4*>(base + unit_of_slot<DR>(e, lane) * 16);
+    float2 f;
+    f = unpack_bf16x2(w.x); v[8 * e + 0] = f.x; v[8 * e + 1] = f.y;
+    f = unpack_bf16x2(w.y); v[8 * e + 2] = f.x; v[8 * e + 3] = f.y;
+    f = unpack_bf16x2(w.z); v[8 * e + 4] = f.x; v[8 * e + 5] = f.y;
+    f = unpack_bf16x2(w.w); v[8 * e + 6] = f.x; v[8 * e + 7] = f.y;
+  }
+}
+
+__device__ __forceinline__ void aux_bar_sync() { named_bar_sync(1, 32 * kAuxCompute); }
+
+template <int DR>
+__global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParams p) {
+  using Sm = AuxSmem<DR>;
+  constexpr int V = DR / 4;  // values per lane
+  extern __shared__ __align__(128) uint8_t aux_sm[];
   const int n_r = p.n_r, NK = p.N + 1, NR = n_r * DR;
-  float* qs = aux_sm;                         // [n_r][DR] query (fp32)
-  float* cosv = qs + 8 * DR;                  // [NK][8] cosines
-  float* nkv = cosv + (size_t)NK * 8;         // [NK][8] clamped key norms (negative: below eps)
-  float* gs = nkv + (size_t)NK * 8;           // [NK] dL/ds_j
-  float* red = gs + NK;                       // [kAuxWarps][NR] partial dL/dq
-  __shared__ float qn[8];                     // clamped query norms (negative: below eps)
-  __shared__ float chead[8];                  // sum_j g_j cos_jh
-  __shared__ float wred[kAuxWarps];
+  uint8_t* ring = aux_sm;
+  float* cosv = reinterpret_cast<float*>(aux_sm + kAuxStages * Sm::kStageBytes);  // [NK][8]
+  float* nkv = cosv + (size_t)NK * 8;                                            // [NK][8]
+  float* gs = nkv + (size_t)NK * 8;                                              // [NK]
+  float* red = gs + NK;                                                          // [kAuxCompute][8 * DR]
+  uint64_t* full = reinterpret_cast<uint64_t*>(
+      (reinterpret_cast<uintptr_t>(red + (size_t)kAuxCompute * 8 * DR) + 7) & ~uintptr_t(7));
+  uint64_t* empty = full + kAuxStages;
+  __shared__ float qn[8];      // clamped query norms (negative: below eps)
+  __shared__ float chead[8];   // sum_j g_j cos_jh
+  __shared__ float wred[kAuxCompute];
   __shared__ bool last;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool grads = p.dQ != nullptr || p.dK_pos != nullptr || p.dK_neg != nullptr;
+  const int n_ch = (NK + kAuxRows - 1) / kAuxRows;  // stages per pass
+  const int passes = grads ? 2 : 1;
+  const size_t row_bytes = (size_t)NR * 2;
+  if (tid == 0) {
+    for (int s = 0; s < kAuxStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kAuxCompute);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
   pdl_launch_dependents();
   pdl_wait();
 
-  const int i = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int h = lane >> 2, part = lane & 3;   // this lane's head and quarter of it
-  const bool hl = h < n_r;
-  const __nv_bfloat16* qrow = p.Q + (size_t)i * NR;
-  for (int e = tid; e < NR; e += kAuxThreads) qs[e] = __bfloat162float(qrow[e]);
-  __syncthreads();
-  if (warp < n_r) {
-    float ss = 0.f;
-    for (int e = lane; e < DR; e += 32) ss = fmaf(qs[warp * DR + e], qs[warp * DR + e], ss);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (warp == kAuxCompute) {
+    // ------------------------- producer -------------------------
     if (lane == 0) {
-      const float n = sqrtf(ss);
-      qn[warp] = n > kAuxEps ? n : -kAuxEps;  // sign marks a clamped norm
-    }
-  }
-  __syncthreads();
-
-  auto key_row = [&](int j) -> const __nv_bfloat16* {
-    return j == 0 ? p.K_pos + (size_t)i * NR : p.K_neg + ((size_t)i * p.N + (j - 1)) * NR;
-  };
-
-  // ---- pass 1: cosines and scores ----
-  for (int j = warp; j < NK; j += kAuxWarps) {
-    float kv[Ln::kVals];
-    float dot = 0.f, kk = 0.f;
-    if (hl) {
-      load_key<DR>(key_row(j), h, part, kv);
-      const float* qv = qs + h * DR + part * Ln::kVals;
-#pragma unroll
-      for (int e = 0; e < Ln::kVals; ++e) {
-        dot = fmaf(kv[e], qv[e], dot);
-        kk = fmaf(kv[e], kv[e], kk);
+      int it = 0;
+      for (int i = blockIdx.x; i < p.P; i += gridDim.x) {
+        for (int pass = 0; pass < passes; ++pass) {
+          for (int c = 0; c < n_ch; ++c, ++it) {
+            const int st = it % kAuxStages;
+            if (it >= kAuxStages) mbar_wait(&empty[st], ((it / kAuxStages) - 1) & 1);
+            const int j0 = c * kAuxRows, j1 = min(NK, j0 + kAuxRows);
+            uint8_t* dst = ring + (size_t)st * Sm::kStageBytes;
+            mbar_arrive_expect_tx(&full[st], (uint32_t)((j1 - j0) * row_bytes));
+            int j = j0;
+            if (j == 0) {  // the positive's key, then its negatives (contiguous rows)
+              bulk_load(dst, p.K_pos + (size_t)i * NR, (uint32_t)row_bytes, &full[st]);
+              ++j;
+            }
+            if (j < j1)
+              bulk_load(dst + (size_t)(j - j0) * row_bytes, p.K_neg + ((size_t)i * p.N + (j - 1)) * NR,
+                        (uint32_t)((j1 - j) * row_bytes), &full[st]);
+          }
+        }
       }
     }
-#pragma unroll
-    for (int o = 1; o < 4; o <<= 1) {
-      dot += __shfl_xor_sync(0xffffffffu, dot, o);
-      kk += __shfl_xor_sync(0xffffffffu, kk, o);
-    }
-    if (hl && part == 0) {
-      const float nk = sqrtf(kk);
-      const float nkc = fmaxf(nk, kAuxEps), nqc = fabsf(qn[h]);
-      cosv[(size_t)j * 8 + h] = dot / (nqc * nkc);
-      nkv[(size_t)j * 8 + h] = nk > kAuxEps ? nk : -kAuxEps;
-    }
+    return;
   }
-  __syncthreads();
 
-  // ---- softmax over the 1 + N scores (z = s / tau) ----
-  float zmax = -INFINITY;
-  for (int j = tid; j < NK; j += kAuxThreads) {
-    float s = 0.f;
-    for (int hh = 0; hh < n_r; ++hh) s += cosv[(size_t)j * 8 + hh];
-    s /= (float)n_r;
-    gs[j] = s * p.inv_tau;  // z_j for now
-    zmax = fmaxf(zmax, gs[j]);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) zmax = fmaxf(zmax, __shfl_xor_sync(0xffffffffu, zmax, o));
-  if (lane == 0) wred[warp] = zmax;
-  __syncthreads();
-  zmax = wred[0];
-#pragma unroll
-  for (int w = 1; w < kAuxWarps; ++w) zmax = fmaxf(zmax, wred[w]);
-  __syncthreads();
-  // the negatives' share, kept apart from the positive's so that neither the loss term
-  // log(1 + sum_j e^(z_j - z_0)) nor 1 - p_0 suffers cancellation when p_0 is near 1
-  float se = 0.f;
-  for (int j = tid; j < NK; j += kAuxThreads)
-    if (j > 0) se += expf(gs[j] - zmax);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) se += __shfl_xor_sync(0xffffffffu, se, o);
-  if (lane == 0) wred[warp] = se;
-  __syncthreads();
-  float se_neg = 0.f;
-#pragma unroll
-  for (int w = 0; w < kAuxWarps; ++w) se_neg += wred[w];
-  const float z0 = gs[0];
-  const float e0 = expf(z0 - zmax);
-  const float den = e0 + se_neg;  // sum_j e^(z_j - zmax), positive included
-  __syncthreads();                // every thread has read gs[0] and wred
-  const float inv_p = 1.0f / (float)p.P;
-  const float scale = p.inv_tau * inv_p / den;
-  // dL/ds_j = p_j / (tau P) for a negative, -(1 - p_0) / (tau P) = -(sum of negatives' p_j) / (tau P)
-  for (int j = tid; j < NK; j += kAuxThreads)
-    gs[j] = j == 0 ? -se_neg * scale : expf(gs[j] - zmax) * scale;
-  if (tid == 0) p.term[i] = (zmax - z0) + log1pf((e0 - 1.0f) + se_neg);  // -log p_0
-  __syncthreads();
-  if (warp < n_r) {  // c_h = sum_j g_j cos_jh
-    float c = 0.f;
-    for (int j = lane; j < NK; j += 32) c = fmaf(gs[j], cosv[(size_t)j * 8 + warp], c);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-    if (lane == 0) chead[warp] = c;
-  }
-  __syncthreads();
-
-  // ---- pass 2: gradients ----
+  // ------------------------- compute warps -------------------------
+  const int h = lane >> 2;  // this lane's head (lanes of heads >= n_r idle in the row work)
+  const bool hl = h < n_r;
   const float inv_nr = 1.0f / (float)n_r;
-  float acc[Ln::kVals];
+  const float inv_p = 1.0f / (float)p.P;
+  int it = 0;
+  for (int i = blockIdx.x; i < p.P; i += gridDim.x) {
+    // this lane's query values (rotated unit order as in load_row_quarter) and the head norms
+    float q[V];
+    {
+      const uint16_t* qrow = reinterpret_cast<const uint16_t*>(p.Q + (size_t)i * NR);
 #pragma unroll
-  for (int e = 0; e < Ln::kVals; ++e) acc[e] = 0.f;
-  const bool want_dk = p.dK_pos != nullptr || p.dK_neg != nullptr;
-  if (p.dQ != nullptr || want_dk) {
-    for (int j = warp; j < NK; j += kAuxWarps) {
-      if (!hl) continue;
-      float kv[Ln::kVals];
-      load_key<DR>(key_row(j), h, part, kv);
-      const float nks = nkv[(size_t)j * 8 + h], nqs = qn[h];
-      const float nk = fabsf(nks), nq = fabsf(nqs);
-      const float g = gs[j] * inv_nr;
-      const float a = g / (nq * nk);  // coefficient of k in dL/dq (summed) and of q in dL/dk
+      for (int e = 0; e < V; ++e)
+        q[e] = hl ? bf16_bits_to_float(__ldg(qrow + lane * V + unit_of_slot<DR>(e / 8, lane) * 8 + e % 8)) : 0.f;
+      float ss = 0.f;
 #pragma unroll
-      for (int e = 0; e < Ln::kVals; ++e) acc[e] = fmaf(a, kv[e], acc[e]);
-      float* dk = j == 0 ? (p.dK_pos ? p.dK_pos + (size_t)i * NR : nullptr)
-                         : (p.dK_neg ? p.dK_neg + ((size_t)i * p.N + (j - 1)) * NR : nullptr);
-      if (dk) {
-        const float b = nks > 0.f ? g * cosv[(size_t)j * 8 + h] / (nk * nk) : 0.f;
-        const float* qv = qs + h * DR + part * Ln::kVals;
-        float4* d4 = reinterpret_cast<float4*>(dk + h * DR + part * Ln::kVals);
-#pragma unroll
-        for (int e = 0; e < Ln::kVals / 4; ++e)
-          d4[e] = make_float4(a * qv[4 * e + 0] - b * kv[4 * e + 0], a * qv[4 * e + 1] - b * kv[4 * e + 1],
-                              a * qv[4 * e + 2] - b * kv[4 * e + 2], a * qv[4 * e + 3] - b * kv[4 * e + 3]);
+      for (int e = 0; e < V; ++e) ss = fmaf(q[e], q[e], ss);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+      aux_bar_sync();  // the previous positive's readers of qn, cos, g and the dq partials are done
+      if (warp == 0 && hl && (lane & 3) == 0) {
+        const float n = sqrtf(ss);
+        qn[h] = n > kAuxEps ? n : -kAuxEps;  // sign marks a clamped norm
       }
+    }
+    aux_bar_sync();  // qn written
+
+    // ---- pass 1: cosines ----
+    for (int c = 0; c < n_ch; ++c, ++it) {
+      const int st = it % kAuxStages;
+      mbar_wait(&full[st], (it / kAuxStages) & 1);
+      const int j = c * kAuxRows + warp;
+      if (j < NK) {
+        float kv[V];
+        float dot = 0.f, kk = 0.f;
+        if (hl) {
+          load_row_quarter<DR>(ring + (size_t)st * Sm::kStageBytes + (size_t)warp * row_bytes, lane, kv);
+#pragma unroll
+          for (int e = 0; e < V; ++e) {
+            dot = fmaf(kv[e], q[e], dot);
+            kk = fmaf(kv[e], kv[e], kk);
+          }
+        }
+        dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+        kk += __shfl_xor_sync(0xffffffffu, kk, 1);
+        dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+        kk += __shfl_xor_sync(0xffffffffu, kk, 2);
+        if (hl && (lane & 3) == 0) {
+          const float nk = sqrtf(kk);
+          cosv[(size_t)j * 8 + h] = dot / (fabsf(qn[h]) * fmaxf(nk, kAuxEps));
+          nkv[(size_t)j * 8 + h] = nk > kAuxEps ? nk : -kAuxEps;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+    }
+    aux_bar_sync();
+
+    // ---- softmax over the 1 + N scores (z = s / tau), the negatives kept apart so that
+    //      neither log(1 + sum_j e^(z_j - z_0)) nor 1 - p_0 cancels when p_0 is near 1 ----
+    const int ct = tid;  // 0 .. 255
+    float zmax = -INFINITY;
+    for (int j = ct; j < NK; j += 32 * kAuxCompute) {
+      float sc = 0.f;
+      for (int hh = 0; hh < n_r; ++hh) sc += cosv[(size_t)j * 8 + hh];
+      gs[j] = sc * inv_nr * p.inv_tau;  // z_j for now
+      zmax = fmaxf(zmax, gs[j]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) zmax = fmaxf(zmax, __shfl_xor_sync(0xffffffffu, zmax, o));
+    if (lane == 0) wred[warp] = zmax;
+    aux_bar_sync();
+    zmax = wred[0];
+#pragma unroll
+    for (int w = 1; w < kAuxCompute; ++w) zmax = fmaxf(zmax, wred[w]);
+    aux_bar_sync();
+    float se = 0.f;
+    for (int j = ct; j < NK; j += 32 * kAuxCompute)
+      if (j > 0) se += expf(gs[j] - zmax);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) se += __shfl_xor_sync(0xffffffffu, se, o);
+    if (lane == 0) wred[warp] = se;
+    aux_bar_sync();
+    float se_neg = 0.f;
+#pragma unroll
+    for (int w = 0; w < kAuxCompute; ++w) se_neg += wred[w];
+    const float z0 = gs[0];
+    const float e0 = expf(z0 - zmax);
+    aux_bar_sync();  // every thread has read gs[0] and wred
+    const float scale = p.inv_tau * inv_p / (e0 + se_neg);
+    for (int j = ct; j < NK; j += 32 * kAuxCompute)
+      gs[j] = j == 0 ? -se_neg * scale : expf(gs[j] - zmax) * scale;  // dL/ds_j
+    if (ct == 0) p.term[i] = (zmax - z0) + log1pf((e0 - 1.0f) + se_neg);  // -log p_0
+    aux_bar_sync();
+    if (!grads) continue;
+    if (warp < n_r) {  // c_h = sum_j g_j cos_jh
+      float cc = 0.f;
+      for (int j = lane; j < NK; j += 32) cc = fmaf(gs[j], cosv[(size_t)j * 8 + warp], cc);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) cc += __shfl_xor_sync(0xffffffffu, cc, o);
+      if (lane == 0) chead[warp] = cc;
+    }
+
+    // ---- pass 2: gradients (the rows again, from L2) ----
+    float acc[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) acc[e] = 0.f;
+    const float nq = hl ? fabsf(qn[h]) : 1.f;
+    for (int c = 0; c < n_ch; ++c, ++it) {
+      const int st = it % kAuxStages;
+      mbar_wait(&full[st], (it / kAuxStages) & 1);
+      const int j = c * kAuxRows + warp;
+      if (j < NK && hl) {
+        float kv[V];
+        load_row_quarter<DR>(ring + (size_t)st * Sm::kStageBytes + (size_t)warp * row_bytes, lane, kv);
+        const float nks = nkv[(size_t)j * 8 + h], nk = fabsf(nks);
+        const float g = gs[j] * inv_nr;
+        const float a = g / (nq * nk);  // coefficient of k in dL/dq and of q in dL/dk
+#pragma unroll
+        for (int e = 0; e < V; ++e) acc[e] = fmaf(a, kv[e], acc[e]);
+        float* dk = j == 0 ? (p.dK_pos ? p.dK_pos + (size_t)i * NR : nullptr)
+                           : (p.dK_neg ? p.dK_neg + ((size_t)i * p.N + (j - 1)) * NR : nullptr);
+        if (dk) {
+          const float b = nks > 0.f ? g * cosv[(size_t)j * 8 + h] / (nk * nk) : 0.f;
+#pragma unroll
+          for (int e = 0; e < V / 4; ++e) {
+            float4* d4 = reinterpret_cast<float4*>(dk + lane * V + unit_of_slot<DR>(e / 2, lane) * 8 + (e % 2) * 4);
+            *d4 = make_float4(a * q[4 * e + 0] - b * kv[4 * e + 0], a * q[4 * e + 1] - b * kv[4 * e + 1],
+                              a * q[4 * e + 2] - b * kv[4 * e + 2], a * q[4 * e + 3] - b * kv[4 * e + 3]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
     }
     if (p.dQ != nullptr) {
       if (hl) {
 #pragma unroll
-        for (int e = 0; e < Ln::kVals; ++e) red[(size_t)warp * NR + h * DR + part * Ln::kVals + e] = acc[e];
+        for (int e = 0; e < V; ++e)
+          red[(size_t)warp * 8 * DR + lane * V + unit_of_slot<DR>(e / 8, lane) * 8 + e % 8] = acc[e];
       }
-      __syncthreads();
-      for (int e = tid; e < NR; e += kAuxThreads) {
+      aux_bar_sync();
+      for (int e = ct; e < NR; e += 32 * kAuxCompute) {
         const int hh = e / DR;
         float v = 0.f;
 #pragma unroll
-        for (int w = 0; w < kAuxWarps; ++w) v += red[(size_t)w * NR + e];
-        const float nqs = qn[hh], nq = fabsf(nqs);
-        if (nqs > 0.f) v -= chead[hh] * inv_nr * qs[e] / (nq * nq);
+        for (int w = 0; w < kAuxCompute; ++w) v += red[(size_t)w * 8 * DR + e];
+        const float nqs = qn[hh], nqa = fabsf(nqs);
+        if (nqs > 0.f) {
+          const float qe = bf16_bits_to_float(__ldg(reinterpret_cast<const uint16_t*>(p.Q) + (size_t)i * NR + e));
+          v -= chead[hh] * inv_nr * qe / (nqa * nqa);
+        }
         p.dQ[(size_t)i * NR + e] = v;
       }
     }
@@ -237,27 +314,23 @@ __global__ void __launch_bounds__(kAuxThreads) aux_loss_kernel(const AuxParams p
 
   // ---- loss: the last CTA sums the terms in positive order ----
   __threadfence();
-  __syncthreads();
+  aux_bar_sync();
   if (tid == 0) {
     const uint32_t prev = atomicAdd(p.ticket, 1u);
-    last = prev == (uint32_t)(p.P - 1);
+    last = prev == gridDim.x - 1;
     if (last) *p.ticket = 0u;
   }
-  __syncthreads();
+  aux_bar_sync();
   if (!last) return;
   __threadfence();
   if (warp == 0) {
     // lane l sums terms l, l + 32, ... in order; the 32 partial sums are added in lane order
-    float s = 0.f;
-    for (int e = lane; e < p.P; e += 32) s += __ldcg(&p.term[e]);
+    float sum = 0.f;
+    for (int e = lane; e < p.P; e += 32) sum += __ldcg(&p.term[e]);
     float tot = 0.f;
-    for (int l = 0; l < 32; ++l) tot += __shfl_sync(0xffffffffu, s, l);
+    for (int l = 0; l < 32; ++l) tot += __shfl_sync(0xffffffffu, sum, l);
     if (lane == 0) *p.loss = tot / (float)p.P;
   }
-}
-
-size_t aux_smem_bytes(int d_r, int n_keys) {
-  return ((size_t)8 * d_r + (size_t)n_keys * 8 * 2 + n_keys + (size_t)kAuxWarps * 8 * d_r) * sizeof(float);
 }
 
 }  // namespace
@@ -293,14 +366,16 @@ msa_status aux_loss_launch(const msa_dims& d, const void* QR, const void* K_pos,
   p.N = N;
   p.n_r = d.n_r;
   p.inv_tau = 1.0f / tau;
-  const size_t sm = aux_smem_bytes(d.d_r, N + 1);
+  const int grid = std::max(1, std::min(P, sm_count()));
   TraceScope ts(kKAuxLoss, s);
   if (d.d_r == 128) {
+    const size_t sm = AuxSmem<128>::bytes(N + 1);
     MSA_CUDA_CHECK(cudaFuncSetAttribute(aux_loss_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-    MSA_CUDA_CHECK(launch_pdl(aux_loss_kernel<128>, dim3(P), dim3(kAuxThreads), sm, s, p));
+    MSA_CUDA_CHECK(launch_pdl(aux_loss_kernel<128>, dim3(grid), dim3(kAuxThreads), sm, s, p));
   } else {
+    const size_t sm = AuxSmem<64>::bytes(N + 1);
     MSA_CUDA_CHECK(cudaFuncSetAttribute(aux_loss_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-    MSA_CUDA_CHECK(launch_pdl(aux_loss_kernel<64>, dim3(P), dim3(kAuxThreads), sm, s, p));
+    MSA_CUDA_CHECK(launch_pdl(aux_loss_kernel<64>, dim3(grid), dim3(kAuxThreads), sm, s, p));
   }
   return MSA_OK;
 }

@@ -51,6 +51,7 @@ enum KernelId : int {
   kKGatherCopy,
   kKChunkOffExtend,
   kKAuxLoss,
+  kKKvAppend,
   kKernelCount
 };
 
@@ -141,6 +142,8 @@ msa_status gather_kv_launch(const msa_dims& d, const void* K_host, const void* V
 msa_status rope_rows_launch(const msa_dims& d, void* x, int rows, int heads, const int32_t* pos, cudaStream_t s);
 msa_status rope_cache_build(const msa_dims& d, int t_loc_max, int pos_offset, float2* tab, cudaStream_t s);
 
+msa_status kv_append_launch(const msa_dims& d, const void* k_new, const void* v_new, void* K_loc, void* V_loc, int B,
+                            int t_loc_max, const int32_t* slots, int pos_offset, cudaStream_t s);
 struct AuxWs {
   float* term;        // [P] per-positive loss terms
   uint32_t* ticket;   // CTAs finished

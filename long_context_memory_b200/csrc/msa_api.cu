@@ -110,7 +110,7 @@ namespace {
 const char* kKernelNames[kKernelCount] = {
     "router_query", "scan", "topk_slice", "topk_merge", "rope_table", "attn_split", "attn_combine",
     "enc_chunk_map", "enc_transpose_w", "enc_gemm_k", "enc_pool_h", "enc_gemm_pooled", "rope_rows", "gather_plan", "gather_copy",
-    "chunk_off_extend", "aux_loss"};
+    "chunk_off_extend", "aux_loss", "kv_append"};
 
 struct TraceState {
   std::mutex mu;
@@ -411,6 +411,23 @@ msa_status msa_rope_rows(const msa_dims* dims, void* x, int32_t rows, int32_t he
   if (!positions) return fail(MSA_ERR_INVALID_ARG, "positions is NULL");
   if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
   return rope_rows_launch(*dims, x, rows, heads, positions, static_cast<cudaStream_t>(stream));
+}
+
+msa_status msa_kv_append(const msa_dims* dims, const void* k_new, const void* v_new, void* K_loc, void* V_loc,
+                         int32_t B, int32_t t_loc_max, const int32_t* slots, int32_t pos_offset, void* stream) {
+  msa_status st = check_dims(dims, true, false);
+  if (st != MSA_OK) return st;
+  if (B < 1 || t_loc_max < 1) return fail(MSA_ERR_INVALID_ARG, "B and t_loc_max must be >= 1 (got %d, %d)", B, t_loc_max);
+  if (pos_offset < 0 || (int64_t)pos_offset + t_loc_max > (1 << 24))
+    return fail(MSA_ERR_INVALID_ARG, "positions must lie in [0, 2^24)");
+  CHECK_PTR(k_new);
+  CHECK_PTR(v_new);
+  CHECK_PTR(K_loc);
+  CHECK_PTR(V_loc);
+  if (!slots) return fail(MSA_ERR_INVALID_ARG, "slots is NULL");
+  if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
+  return kv_append_launch(*dims, k_new, v_new, K_loc, V_loc, B, t_loc_max, slots, pos_offset,
+                          static_cast<cudaStream_t>(stream));
 }
 
 size_t msa_rope_cache_size(const msa_dims* dims, int32_t t_loc_max) {

@@ -34,6 +34,7 @@ namespace msa {
 struct RouteWs {
   float* qr;          // [rq_splits][B][NR] fp32 partial router queries (W_QR given)
   uint32_t* head_done;  // [n_r] CTAs finished per router head (back to 0 after each call)
+  uint32_t* scan_ticket;  // scan CTAs finished (fused top-k); zeroed by the router query kernel
   __nv_bfloat16* q_hl; // [passes][n_r][2][NQ][d_r] normalised query, bf16 hi and lo terms
   uint32_t* doc_key;  // [B][n_docs] ordered-uint32 doc max (MAX)
   uint32_t* chunk_k;  // [B][n_chunks] ordered chunk scores (MEAN)
@@ -44,6 +45,7 @@ struct RouteWs {
 namespace {
 
 constexpr int kSliceDocs = 4096;   // documents per top-k slice CTA
+constexpr int kFuseTopkMaxQueries = 4;  // top-k in the scan's last CTA up to this many queries
 constexpr int kTopkThreads = 1024;
 constexpr float kEps = 1e-12f;
 
@@ -162,7 +164,8 @@ __device__ __forceinline__ void rq_group(const uint16_t* hq, const __nv_bfloat16
 __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
     const __nv_bfloat16* __restrict__ Hq, const __nv_bfloat16* __restrict__ W, int B, int b_pad, int hidden,
     int n_r, int d_r, int nq, int split_rows, float* __restrict__ qpart, uint32_t* __restrict__ head_done,
-    __nv_bfloat16* __restrict__ q_hl, uint32_t* __restrict__ clear, size_t n_clear) {
+    __nv_bfloat16* __restrict__ q_hl, uint32_t* __restrict__ clear, size_t n_clear,
+    uint32_t* __restrict__ scan_ticket) {
   extern __shared__ __align__(16) uint8_t rq_smem[];
   float* red = reinterpret_cast<float*>(rq_smem);                                 // [8 warps][kRqQB][d_r]
   uint16_t* hs = reinterpret_cast<uint16_t*>(red + (kRqThreads / 32) * kRqQB * d_r);  // [kRqQB][split_rows]
@@ -175,7 +178,9 @@ __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint16_t* hq = reinterpret_cast<const uint16_t*>(Hq);
 
-  // clear the scan's max keys (grid-stride); the scan only runs after this kernel completes
+  // clear the scan's max keys (grid-stride) and its ticket; the scan only runs after this
+  // kernel completes
+  if (scan_ticket && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *scan_ticket = 0u;
   if (clear) {
     const size_t cta = (size_t)blockIdx.y * gridDim.x + blockIdx.x, n_cta = (size_t)gridDim.x * gridDim.y;
     for (size_t i = cta * kRqThreads + tid; i < n_clear; i += n_cta * kRqThreads) clear[i] = 0u;
@@ -294,10 +299,21 @@ constexpr int kScanThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2..5 norms,
 constexpr int kScanNormWarps = 4;   // one per TMEM lane quarter (32 rows each)
 constexpr int kScanEpiWarps = 4;
 
+__device__ void slice_topk(const uint32_t* doc_key, const uint32_t* chunk_k, const int32_t* chunk_off, int n_docs,
+                           int n_chunks, int k, int n_slices, float* doc_scores, uint64_t* cand, int32_t* topk_idx,
+                           float* topk_score, int slice, int b, uint64_t* sm64);
+
 struct ScanParams {
   const int32_t* chunk_off;
   uint32_t* doc_key;
   uint32_t* chunk_k;
+  // top-k fused into the scan (one slice of documents, few queries): the last CTA to finish
+  // (ticket) selects the top-k of every query
+  uint32_t* ticket;  // null: top-k runs as its own kernel
+  int n_queries, k;
+  float* doc_scores;
+  int32_t* topk_idx;
+  float* topk_score;
   int n_r, n_docs, n_chunks, n_tiles;
   int q_tokens;    // query tokens per query: scan row r belongs to query r / q_tokens
   int q_base, q_count, pass;
@@ -546,6 +562,25 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, p.tmem_cols);
+
+  if (p.ticket) {
+    // every CTA's document maxima are in L2: the last one selects the top-k (the pipeline's
+    // shared memory is free again and holds the keys)
+    __shared__ bool last_cta;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const uint32_t prev = atomicAdd(p.ticket, 1u);
+      last_cta = prev == gridDim.x - 1;
+      if (last_cta) *p.ticket = 0u;
+    }
+    __syncthreads();
+    if (!last_cta) return;
+    __threadfence();
+    for (int b = 0; b < p.n_queries; ++b)
+      slice_topk(p.doc_key, p.chunk_k, p.chunk_off, p.n_docs, p.n_chunks, p.k, 1, p.doc_scores, nullptr,
+                 p.topk_idx, p.topk_score, 0, b, reinterpret_cast<uint64_t*>(smem));
+  }
 }
 
 // --------------------------------------------------------------------------
@@ -632,19 +667,18 @@ __device__ __forceinline__ uint64_t make_key(uint32_t ordered, int id) {
   return ((uint64_t)ordered << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)id);
 }
 
-__global__ void __launch_bounds__(kTopkThreads) topk_slice_kernel(
-    const uint32_t* __restrict__ doc_key, const uint32_t* __restrict__ chunk_k, const int32_t* __restrict__ chunk_off,
-    int n_docs, int n_chunks, int k, int n_slices, float* __restrict__ doc_scores, uint64_t* __restrict__ cand,
-    int32_t* __restrict__ topk_idx, float* __restrict__ topk_score) {
-  extern __shared__ uint64_t sm64[];
+// top-k of one slice of documents for query b (whole block): document scores from the
+// scan's max keys (or the mean of its chunk keys), written out when asked, then the block
+// top-k; with one slice the result is final, otherwise the slice's winners become
+// candidates for the merge.  sm64 holds (kSliceDocs + 516) 64-bit words + 256 words of 32 bits.
+__device__ void slice_topk(const uint32_t* doc_key, const uint32_t* chunk_k, const int32_t* chunk_off, int n_docs,
+                           int n_chunks, int k, int n_slices, float* doc_scores, uint64_t* cand, int32_t* topk_idx,
+                           float* topk_score, int slice, int b, uint64_t* sm64) {
   uint64_t* keys = sm64;              // [kSliceDocs]
   uint64_t* out = keys + kSliceDocs;  // [256]
   uint64_t* tmp = out + 256;          // [256]
   uint64_t* state = tmp + 256;        // [4]
   uint32_t* hist = reinterpret_cast<uint32_t*>(state + 4);
-  pdl_launch_dependents();
-  pdl_wait();
-  const int slice = blockIdx.x, b = blockIdx.y;
   const int d0 = slice * kSliceDocs;
   const int n = min(kSliceDocs, n_docs - d0);
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
@@ -653,11 +687,11 @@ __global__ void __launch_bounds__(kTopkThreads) topk_slice_kernel(
     if (chunk_k) {
       const int c0 = __ldg(&chunk_off[doc]), c1 = __ldg(&chunk_off[doc + 1]);
       float s = 0.f;
-      for (int j = c0; j < c1; ++j) s += ordered_to_float(chunk_k[(size_t)b * n_chunks + j]);
+      for (int j = c0; j < c1; ++j) s += ordered_to_float(__ldcg(&chunk_k[(size_t)b * n_chunks + j]));
       const float mean = s / (float)max(1, c1 - c0);
       ok = float_to_ordered(mean);
     } else {
-      ok = doc_key[(size_t)b * n_docs + doc];
+      ok = __ldcg(&doc_key[(size_t)b * n_docs + doc]);
     }
     if (doc_scores) doc_scores[(size_t)b * n_docs + doc] = ordered_to_float(ok);
     keys[i] = make_key(ok, doc);
@@ -674,6 +708,18 @@ __global__ void __launch_bounds__(kTopkThreads) topk_slice_kernel(
     for (int i = threadIdx.x; i < k; i += blockDim.x)
       cand[((size_t)b * n_slices + slice) * k + i] = (i < kk) ? out[i] : 0ull;
   }
+  __syncthreads();  // shared memory free for the next call
+}
+
+__global__ void __launch_bounds__(kTopkThreads) topk_slice_kernel(
+    const uint32_t* __restrict__ doc_key, const uint32_t* __restrict__ chunk_k, const int32_t* __restrict__ chunk_off,
+    int n_docs, int n_chunks, int k, int n_slices, float* __restrict__ doc_scores, uint64_t* __restrict__ cand,
+    int32_t* __restrict__ topk_idx, float* __restrict__ topk_score) {
+  extern __shared__ uint64_t sm64[];
+  pdl_launch_dependents();
+  pdl_wait();
+  slice_topk(doc_key, chunk_k, chunk_off, n_docs, n_chunks, k, n_slices, doc_scores, cand, topk_idx, topk_score,
+             blockIdx.x, blockIdx.y, sm64);
 }
 
 __global__ void __launch_bounds__(kTopkThreads) topk_merge_kernel(const uint64_t* __restrict__ cand,
@@ -775,6 +821,7 @@ size_t route_workspace(const msa_dims& d, int B, int M, int n_docs, int n_chunks
   w.rq_splits = rq_geom(d.hidden, d.n_r).n_splits;
   w.qr = cv.take<float>((size_t)w.rq_splits * R * NR);
   w.head_done = cv.take<uint32_t>(8);
+  w.scan_ticket = cv.take<uint32_t>(1);
   w.q_hl = cv.take<__nv_bfloat16>((size_t)w.passes * d.n_r * 2 * w.nq * d.d_r);
   w.doc_key = agg == MSA_AGG_MAX ? cv.take<uint32_t>((size_t)B * n_docs) : nullptr;
   w.chunk_k = agg == MSA_AGG_MEAN ? cv.take<uint32_t>((size_t)B * n_chunks) : nullptr;
@@ -794,6 +841,8 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
   // keys folded in with atomicMax start at 0 (below every ordered score): the document keys,
   // and the chunk keys when several tokens of a query meet in one chunk
   uint32_t* clear = mean ? (M > 1 ? w.chunk_k : nullptr) : w.doc_key;
+  // few queries over one slice of documents: the scan's last CTA runs the top-k itself
+  const bool fuse_topk = w.n_slices == 1 && w.passes == 1 && B <= kFuseTopkMaxQueries;
   const size_t n_clear = clear ? (size_t)B * (mean ? n_chunks : n_docs) : 0;
 
   // K1: router query (projection, normalisation, hi/lo layout) and document keys cleared
@@ -806,7 +855,7 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
     MSA_CUDA_CHECK(launch_pdl(router_query_kernel, dim3(W_QR ? g.n_splits : 1, d.n_r), dim3(kRqThreads), sm, s,
                               static_cast<const __nv_bfloat16*>(Hq), static_cast<const __nv_bfloat16*>(W_QR), R,
                               w.passes * w.nq, d.hidden, d.n_r, d.d_r, w.nq, g.rows, w.qr, w.head_done, w.q_hl,
-                              clear, n_clear));
+                              clear, n_clear, w.scan_ticket));
   }
   // K3: scan, NQ (16 or 32) queries per pass
   {
@@ -841,6 +890,12 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
       p.chunk_off = chunk_off;
       p.doc_key = w.doc_key;
       p.chunk_k = w.chunk_k;
+      p.ticket = fuse_topk ? w.scan_ticket : nullptr;
+      p.n_queries = B;
+      p.k = k;
+      p.doc_scores = doc_scores;
+      p.topk_idx = topk_idx;
+      p.topk_score = topk_score;
       p.q_tokens = M;
       p.n_r = d.n_r;
       p.n_docs = n_docs;
@@ -858,7 +913,7 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
     }
   }
   // K4: top-k
-  {
+  if (!fuse_topk) {
     TraceScope ts(kKTopkSlice, s);
     const size_t sm = topk_slice_smem();
     MSA_CUDA_CHECK(cudaFuncSetAttribute(topk_slice_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));

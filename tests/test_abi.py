@@ -173,6 +173,17 @@ def test_aux_loss_validation(msa):
                             None, 0x100000, need, None) == 2
 
 
+def test_kv_append_validation(msa):
+    dd = msa.Dims.of(_dims())
+    lib = msa.lib
+    assert lib.msa_kv_append(ctypes.byref(dd), FAKE, FAKE, FAKE, FAKE, 0, 16, FAKE, 2, None) == 1   # B < 1
+    assert lib.msa_kv_append(ctypes.byref(dd), FAKE, FAKE, FAKE, FAKE, 1, 16, None, 2, None) == 1   # no slots
+    assert lib.msa_kv_append(ctypes.byref(dd), FAKE + 2, FAKE, FAKE, FAKE, 1, 16, FAKE, 2, None) == 1
+    assert lib.msa_kv_append(ctypes.byref(dd), FAKE, FAKE, FAKE, FAKE, 1, 16, FAKE, -1, None) == 1
+    assert lib.msa_kv_append(ctypes.byref(msa.Dims.of(_dims(head_dim=96))), FAKE, FAKE, FAKE, FAKE, 1, 16, FAKE, 2,
+                             None) == 2
+
+
 def test_topk_merge_validation(msa):
     lib = msa.lib
     assert lib.msa_topk_merge(FAKE, FAKE, 1, 8, 9, FAKE, FAKE, None) == 1      # k > n_cand

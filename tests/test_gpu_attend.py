@@ -250,3 +250,40 @@ def test_host_tier_rejects_pageable_memory(msa, cuda_device):
     with pytest.raises(msa.MSAError) as e:
         msa.gather_kv(dims, K, V, co, tk, capacity_chunks=10)
     assert e.value.code == 1 and "pinned" in str(e.value)
+
+
+def test_kv_append_matches_rotation_and_copy(msa, cuda_device):
+    # the fused append = rotate a copy of the new key at pos_offset + slot, copy both rows in
+    import torch
+    from helpers import torch_bits
+
+    rng = np.random.default_rng(61)
+    B, T, n_kv, D, o = 3, 40, 8, 128, 16
+    dims = W.Dims(hidden=256, n_q=32, n_kv=n_kv, head_dim=D, n_r=4, d_r=64, rope_base=1e6)
+    K = _dev(W.normal_bf16(rng, (B, T, n_kv, D)), cuda_device)
+    V = _dev(W.normal_bf16(rng, (B, T, n_kv, D)), cuda_device)
+    kn_np = W.normal_bf16(rng, (B, n_kv, D))
+    kn, vn = _dev(kn_np, cuda_device), _dev(W.normal_bf16(rng, (B, n_kv, D)), cuda_device)
+    slots = torch.tensor([0, 17, T - 1], dtype=torch.int32, device=cuda_device)
+    K0, V0 = K.clone(), V.clone()
+    msa.kv_append(dims, kn, vn, K, V, slots, o)
+    ref = kn.clone()
+    msa.rope_rows(dims, ref, (o + slots).to(torch.int32))
+    torch.cuda.synchronize()
+    assert msa.check_device_errors() == 0
+    for b, s in enumerate(slots.tolist()):
+        assert torch.equal(K[b, s], ref[b]) and torch.equal(V[b, s], vn[b])
+        want = O.rope(O.bf16_to_f64(kn_np[b]), o + s, 1e6)
+        got = O.bf16_to_f64(torch_bits(K[b, s]))
+        assert np.all(np.abs(got - want) <= 2.0 ** -8 * np.abs(want) + 1e-6)
+        keep = [t for t in range(T) if t != s]
+        assert torch.equal(K[b, keep], K0[b, keep]) and torch.equal(V[b, keep], V0[b, keep])
+    # a slot outside the cache is skipped and reported
+    bad = torch.tensor([T, 0, -1], dtype=torch.int32, device=cuda_device)
+    K1 = K.clone()
+    msa.kv_append(dims, kn, vn, K, V, bad, o)
+    torch.cuda.synchronize()
+    with pytest.raises(msa.MSAError, match="out-of-range index"):
+        msa.check_device_errors()
+    assert msa.check_device_errors() == 0   # reading the word clears it
+    assert torch.equal(K[0], K1[0]) and torch.equal(K[2], K1[2])

@@ -94,6 +94,20 @@ def test_route_head_major_keys(msa, cuda_device, B, n_r, d_r):
     assert np.array_equal(ds, ds0) and np.array_equal(idx, idx0) and np.array_equal(sc, sc0)
 
 
+@pytest.mark.parametrize("agg", [0, 1])
+def test_route_fused_topk_matches_separate_kernels(msa, cuda_device, agg):
+    # up to 4 queries over one slice of documents take the top-k inside the scan's last CTA;
+    # 5 queries take the separate top-k kernel: the first 4 queries' results must agree exactly
+    dims, doc_off, KR, QR, Hq, Wqr, _ = _route_case(41 + agg, 500, 5, 8, 128)
+    i4, s4, d4 = _run(msa, dims, QR[:4], None, KR, doc_off, 16, agg, cuda_device)
+    i5, s5, d5 = _run(msa, dims, QR, None, KR, doc_off, 16, agg, cuda_device)
+    assert np.array_equal(i4, i5[:4]) and np.array_equal(s4, s5[:4]) and np.array_equal(d4, d5[:4])
+    co, *_ = O.chunk_layout(doc_off)
+    s, _, _ = O.route_topk(O.bf16_to_f64(QR).reshape(5, 8, 128), KR, co, 16, "max" if agg == 0 else "mean")
+    for b in range(4):
+        check_topk(i4[b], s4[b], s[b], 16, where=f"b={b}")
+
+
 def test_route_edge_shapes(msa, cuda_device):
     # one-chunk docs, k = n_docs, chunk count not a multiple of the tile, single doc
     for seed, n_docs, lo, hi, k in [(1, 17, 1, 64, 17), (2, 1, 5, 5, 1), (3, 40, 1, 1, 40), (4, 33, 60, 70, 1)]:
