@@ -65,9 +65,7 @@ constexpr float kEps = 1e-12f;
 // only the head step runs (grid (1, n_r)).
 // --------------------------------------------------------------------------
 constexpr int kRqThreads = 256;
-constexpr int kRqRows = 12;      // rows of W held in registers per thread (resident case)
-constexpr int kRqQB = 8;         // queries per register group
-constexpr int kRqMaxSplitRows = 1024;
+constexpr int kRqMaxSplitRows = 256;
 constexpr int kRqTargetCtas = 144;
 
 struct RqGeom {
@@ -82,84 +80,11 @@ RqGeom rq_geom(int hidden, int n_r) {
   return RqGeom{(hidden + rows - 1) / rows, rows};
 }
 
-size_t rq_smem_bytes(int d_r, int rows) {
-  return (size_t)(kRqThreads / 32) * kRqQB * d_r * sizeof(float) + (size_t)kRqQB * rows * sizeof(uint16_t);
-}
-
-// one group of QB queries: stage their slice of H_q, multiply by the W slab, reduce over the
-// row threads and write the split's partial sums
-template <int QB>
-__device__ __forceinline__ void rq_group(const uint16_t* hq, const __nv_bfloat16* wcol, uint4 (&wv)[kRqRows],
-                                         bool resident, int B, int b0, int hidden, int NR, int h, int d_r, int k0,
-                                         int nrows, int split, int split_rows, int cg, int rt, int RT, int CG, int lane,
-                                         int warp, int tid, uint16_t* hs, float* red, float* qpart) {
-  __syncthreads();
-  const int vec = nrows / 8;  // 16-byte vectors per query row
-  for (int i = tid; i < QB * vec; i += kRqThreads) {
-    const int j = i / vec, v = i % vec;
-    uint4 x = make_uint4(0, 0, 0, 0);
-    if (b0 + j < B) x = __ldg(reinterpret_cast<const uint4*>(hq + (size_t)(b0 + j) * hidden + k0) + v);
-    reinterpret_cast<uint4*>(hs + (size_t)j * split_rows)[v] = x;
-  }
-  __syncthreads();
-  float acc[QB][8];
-#pragma unroll
-  for (int j = 0; j < QB; ++j)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[j][c] = 0.f;
-  auto fma_row = [&](const uint4 w4, int r) {
-    float wf[8];
-    float2 t;
-    t = unpack_bf16x2(w4.x); wf[0] = t.x; wf[1] = t.y;
-    t = unpack_bf16x2(w4.y); wf[2] = t.x; wf[3] = t.y;
-    t = unpack_bf16x2(w4.z); wf[4] = t.x; wf[5] = t.y;
-    t = unpack_bf16x2(w4.w); wf[6] = t.x; wf[7] = t.y;
-#pragma unroll
-    for (int j = 0; j < QB; ++j) {
-      const float hv = bf16_bits_to_float(hs[(size_t)j * split_rows + r]);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) acc[j][c] = fmaf(hv, wf[c], acc[j][c]);
-    }
-  };
-  if (resident) {
-#pragma unroll
-    for (int u = 0; u < kRqRows; ++u) {
-      const int r = rt + RT * u;
-      if (r < nrows) fma_row(wv[u], r);
-    }
-  } else {
-    for (int r0 = rt; r0 < nrows; r0 += RT * kRqRows) {
-      uint4 w2[kRqRows];
-#pragma unroll
-      for (int u = 0; u < kRqRows; ++u) {
-        const int r = r0 + RT * u;
-        w2[u] = r < nrows ? __ldg(reinterpret_cast<const uint4*>(wcol + (size_t)r * NR)) : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int u = 0; u < kRqRows; ++u) {
-        const int r = r0 + RT * u;
-        if (r < nrows) fma_row(w2[u], r);
-      }
-    }
-  }
-  // reduce over the row threads: lanes cg, cg + CG, ... of a warp, then the 8 warps
-#pragma unroll
-  for (int j = 0; j < QB; ++j)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      float v = acc[j][c];
-      for (int o = CG; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane < CG) red[((size_t)warp * kRqQB + j) * d_r + cg * 8 + c] = v;
-    }
-  __syncthreads();
-  for (int i = tid; i < QB * d_r; i += kRqThreads) {
-    const int j = i / d_r, col = i % d_r;
-    float v = 0.f;
-#pragma unroll
-    for (int w = 0; w < kRqThreads / 32; ++w) v += red[((size_t)w * kRqQB + j) * d_r + col];
-    if (b0 + j < B) qpart[((size_t)split * B + b0 + j) * NR + h * d_r + col] = v;
-  }
-}
+// shared memory: the W slab [rows][d_r] and 16 query rows [16][rows], both bf16 with rows
+// padded by 16 bytes so that ldmatrix's 8 row addresses fall in distinct bank groups
+__host__ __device__ inline int rq_w_stride(int d_r) { return d_r * 2 + 16; }
+__host__ __device__ inline int rq_h_stride(int rows) { return rows * 2 + 16; }
+size_t rq_smem_bytes(int d_r, int rows) { return (size_t)rows * rq_w_stride(d_r) + 16 * (size_t)rq_h_stride(rows); }
 
 __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
     const __nv_bfloat16* __restrict__ Hq, const __nv_bfloat16* __restrict__ W, int B, int b_pad, int hidden,
@@ -167,8 +92,6 @@ __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
     __nv_bfloat16* __restrict__ q_hl, uint32_t* __restrict__ clear, size_t n_clear,
     uint32_t* __restrict__ scan_ticket) {
   extern __shared__ __align__(16) uint8_t rq_smem[];
-  float* red = reinterpret_cast<float*>(rq_smem);                                 // [8 warps][kRqQB][d_r]
-  uint16_t* hs = reinterpret_cast<uint16_t*>(red + (kRqThreads / 32) * kRqQB * d_r);  // [kRqQB][split_rows]
   __shared__ float invn[kRqThreads / 32];
   __shared__ bool last;
   pdl_launch_dependents();
@@ -187,31 +110,68 @@ __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
   }
 
   if (W) {
-    const int CG = d_r / 8;               // 8-column groups of the head (16 or 8)
-    const int RT = kRqThreads / CG;       // row threads (16 or 32)
-    const int cg = tid % CG, rt = tid / CG;
+    // Q^R partial of this split on the tensor cores (mma.sync m16n8k16, bf16 in, fp32 out):
+    // D[16 query rows][d_r] = H_q slice [16][rows] x W slab [rows][d_r]; warp w owns the
+    // n-tiles 2w, 2w + 1 (d_r = 128) or w (d_r = 64)
     const int k0 = split * split_rows;
-    const int nrows = min(split_rows, hidden - k0);
-    const bool resident = (nrows + RT - 1) / RT <= kRqRows;  // block-uniform
-    const __nv_bfloat16* wcol = W + (size_t)k0 * NR + h * d_r + cg * 8;
-    uint4 wv[kRqRows];
-    if (resident) {
-#pragma unroll
-      for (int u = 0; u < kRqRows; ++u) {
-        const int r = rt + RT * u;
-        wv[u] = r < nrows ? __ldg(reinterpret_cast<const uint4*>(wcol + (size_t)r * NR)) : make_uint4(0, 0, 0, 0);
+    const int nrows = min(split_rows, hidden - k0);  // multiple of 16
+    const int ws = rq_w_stride(d_r), hstr = rq_h_stride(split_rows);
+    uint8_t* wsm = rq_smem;
+    uint8_t* hsm = rq_smem + (size_t)split_rows * ws;
+    {  // W slab: 16-byte pieces, a row's pieces on consecutive threads (coalesced)
+      const int per_row = d_r / 8;
+      const __nv_bfloat16* wsrc = W + (size_t)k0 * NR + h * d_r;
+      for (int i = tid; i < nrows * per_row; i += kRqThreads) {
+        const int r = i / per_row, c = i % per_row;
+        *reinterpret_cast<uint4*>(wsm + (size_t)r * ws + c * 16) =
+            __ldg(reinterpret_cast<const uint4*>(wsrc + (size_t)r * NR) + c);
       }
     }
-    for (int b0 = 0; b0 < B; b0 += kRqQB) {
-      const int nb = min(kRqQB, B - b0);  // queries in this group (block-uniform)
-      if (nb == 1) rq_group<1>(hq, wcol, wv, resident, B, b0, hidden, NR, h, d_r, k0, nrows, split, split_rows, cg, rt,
-                               RT, CG, lane, warp, tid, hs, red, qpart);
-      else if (nb == 2) rq_group<2>(hq, wcol, wv, resident, B, b0, hidden, NR, h, d_r, k0, nrows, split, split_rows, cg,
-                                    rt, RT, CG, lane, warp, tid, hs, red, qpart);
-      else if (nb <= 4) rq_group<4>(hq, wcol, wv, resident, B, b0, hidden, NR, h, d_r, k0, nrows, split, split_rows, cg,
-                                    rt, RT, CG, lane, warp, tid, hs, red, qpart);
-      else rq_group<8>(hq, wcol, wv, resident, B, b0, hidden, NR, h, d_r, k0, nrows, split, split_rows, cg, rt, RT, CG,
-                       lane, warp, tid, hs, red, qpart);
+    const int n_nt = d_r / 8;                 // n-tiles of 8 columns
+    const int nt_per_warp = n_nt / 8;         // 2 or 1
+    const int ksteps = nrows / 16;
+    for (int b0 = 0; b0 < B; b0 += 16) {
+      __syncthreads();  // W slab landed / previous query rows consumed
+      {
+        const int vec = nrows / 8;
+        for (int i = tid; i < 16 * vec; i += kRqThreads) {
+          const int j = i / vec, v = i % vec;
+          uint4 x = make_uint4(0, 0, 0, 0);
+          if (b0 + j < B) x = __ldg(reinterpret_cast<const uint4*>(hq + (size_t)(b0 + j) * hidden + k0) + v);
+          *reinterpret_cast<uint4*>(hsm + (size_t)j * hstr + v * 16) = x;
+        }
+      }
+      __syncthreads();
+      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      const int n0 = warp * nt_per_warp;     // first n-tile of this warp
+      for (int ks = 0; ks < ksteps; ++ks) {
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4(a0, a1, a2, a3, smem_u32(hsm + (size_t)(lane & 15) * hstr + (ks * 16 + 8 * (lane >> 4)) * 2));
+        const int krow = ks * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+        if (nt_per_warp == 2) {
+          uint32_t b0r, b1r, b2r, b3r;
+          ldmatrix_x4_trans(b0r, b1r, b2r, b3r, smem_u32(wsm + (size_t)krow * ws + (8 * n0 + 8 * (lane >> 4)) * 2));
+          mma_bf16_16816(acc[0], a0, a1, a2, a3, b0r, b1r);
+          mma_bf16_16816(acc[1], a0, a1, a2, a3, b2r, b3r);
+        } else {
+          uint32_t b0r, b1r, b2r, b3r;  // two k-halves of one n-tile (the upper lanes' rows repeat)
+          ldmatrix_x4_trans(b0r, b1r, b2r, b3r, smem_u32(wsm + (size_t)krow * ws + (8 * n0) * 2));
+          mma_bf16_16816(acc[0], a0, a1, a2, a3, b0r, b1r);
+        }
+      }
+      // D fragment: rows lane/4 and lane/4 + 8, columns 2 (lane % 4) + {0, 1} of each n-tile
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (t >= nt_per_warp) break;
+        const int col = 8 * (n0 + t) + 2 * (lane & 3);
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          const int b = b0 + (lane >> 2) + 8 * rr;
+          if (b < B)
+            *reinterpret_cast<float2*>(qpart + ((size_t)split * B + b) * NR + h * d_r + col) =
+                make_float2(acc[t][2 * rr], acc[t][2 * rr + 1]);
+        }
+      }
     }
     // this CTA's partials are written: take a ticket; the head's last CTA goes on
     __threadfence();
@@ -599,9 +559,22 @@ __device__ void block_topk(const uint64_t* keys, int n, int k, uint64_t* out, ui
     const int shift = 56 - 8 * pass;
     for (int i = tid; i < 256; i += nt) hist[i] = 0;
     __syncthreads();
-    for (int i = tid; i < n; i += nt) {
-      const uint64_t key = keys[i];
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1u);
+    // one shared-memory atomic per distinct digit per warp: scores cluster in a few digits
+    // (the high bytes of nearby floats agree), and per-lane atomics on one address serialise
+    for (int i0 = 0; i0 < n; i0 += nt) {
+      const int i = i0 + tid;
+      uint64_t key = 0;
+      bool in = false;
+      if (i < n) {
+        key = keys[i];
+        in = (key & mask) == prefix;
+      }
+      const unsigned act = __ballot_sync(0xffffffffu, in);
+      if (in) {
+        const uint32_t digit = (uint32_t)(key >> shift) & 255u;
+        const unsigned grp = __match_any_sync(act, digit);
+        if ((threadIdx.x & 31) == __ffs(grp) - 1) atomicAdd(&hist[digit], (uint32_t)__popc(grp));
+      }
     }
     __syncthreads();
     if (tid < 32) {
