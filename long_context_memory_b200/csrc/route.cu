@@ -288,7 +288,12 @@ struct ScanGeom {
   static constexpr int kKBox = kScanM * 128;            // one 64-dim x 128-row box
   static constexpr int kQBox = NQ * 128;                // one 64-dim x NQ-row box
   static constexpr int kKBytes = kHalves * kKBox;
-  static constexpr int kQBytes = 2 * kHalves * kQBox;   // hi and lo
+  static constexpr int kQBytes = 2 * kHalves * kQBox;   // hi and lo: [half j][hi | lo][NQ rows]
+  // NQ = 16: one MMA per k-step with N = 2 NQ (the hi and lo rows side by side, summed in the
+  // epilogue) - half the MMA chain of accumulating hi and lo into one accumulator, so each
+  // stage is released sooner; NQ = 32 keeps one accumulator per head (TMEM holds 512 columns)
+  static constexpr bool kWide = NQ == 16;
+  static constexpr int kCols = kWide ? 2 * NQ : NQ;     // TMEM columns per head
   static constexpr int kStageBytes = kKBytes + kQBytes;
   static constexpr int kStages = (NQ == 16 || DR == 64) ? 5 : 4;
   static constexpr int kNormBytes = 2 * 8 * kScanM * 4;  // [2 tiles][8 heads][128 rows] fp32
@@ -343,7 +348,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t buf_cols = (uint32_t)n_r * NQ;
+  const uint32_t buf_cols = (uint32_t)n_r * Gm::kCols;
   pdl_launch_dependents();
   pdl_wait();
 
@@ -365,7 +370,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
             tma_load_2d(k_s + j * Gm::kKBox, &kr_map, &full[st], h * DR + j * 64, tile * kScanM);
 #pragma unroll
           for (int hl = 0; hl < 2; ++hl)
-            tma_load_2d(q_s + (hl * Gm::kHalves + j) * Gm::kQBox, &q_map, &full[st], j * 64,
+            tma_load_2d(q_s + (j * 2 + hl) * Gm::kQBox, &q_map, &full[st], j * 64,
                         ((p.pass * n_r + h) * 2 + hl) * NQ);
         }
       }
@@ -373,7 +378,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   } else if (warp == 1) {
     // ------------------------- MMA issuer -------------------------
     if (lane == 0) {
-      constexpr uint32_t idesc = umma_idesc_bf16(kScanM, NQ);
+      constexpr uint32_t idesc = umma_idesc_bf16(kScanM, Gm::kCols);
       for (int it = 0; it < n_it; ++it) {
         const int lt = it / n_r, h = it % n_r;
         const int buf = lt & 1;
@@ -381,15 +386,19 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         if (h == 0 && lt >= 2) mbar_wait(&tempty[buf], ((lt >> 1) - 1) & 1);
         mbar_wait(&full[st], (it / S) & 1);
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + buf * buf_cols + h * NQ;
+        const uint32_t d_tmem = tmem_base + buf * buf_cols + h * Gm::kCols;
         const uint32_t k_addr = smem_u32(stages + st * Gm::kStageBytes);
         const uint32_t q_addr = k_addr + Gm::kKBytes;
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
           const int j = ks >> 2, off = (ks & 3) * 32;
           const uint64_t a_desc = umma_desc_k_sw128(k_addr + j * Gm::kKBox + off);
-          umma_bf16(d_tmem, a_desc, umma_desc_k_sw128(q_addr + j * Gm::kQBox + off), idesc, ks > 0);
-          umma_bf16(d_tmem, a_desc, umma_desc_k_sw128(q_addr + (Gm::kHalves + j) * Gm::kQBox + off), idesc, 1);
+          if constexpr (Gm::kWide) {  // B = the 2 NQ rows [hi; lo] of this k-half
+            umma_bf16(d_tmem, a_desc, umma_desc_k_sw128(q_addr + j * 2 * Gm::kQBox + off), idesc, ks > 0);
+          } else {
+            umma_bf16(d_tmem, a_desc, umma_desc_k_sw128(q_addr + j * 2 * Gm::kQBox + off), idesc, ks > 0);
+            umma_bf16(d_tmem, a_desc, umma_desc_k_sw128(q_addr + (j * 2 + 1) * Gm::kQBox + off), idesc, 1);
+          }
         }
         umma_commit(&empty[st]);
         if (h == n_r - 1) umma_commit(&tfull[buf]);
@@ -446,12 +455,16 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       for (int hh = 0; hh < 8; ++hh) {
         if (hh < n_r) {
           const float inv = 1.0f / fmaxf(sqrtf(nb2[hh * kScanM + row]), kEps);
-          float v[NQ];
-          if constexpr (NQ == 16) tmem_ld16(t_row + hh * NQ, v);
-          else tmem_ld32(t_row + hh * NQ, v);
+          float v[32];
+          tmem_ld32(t_row + hh * Gm::kCols, v);
           tmem_ld_wait();
+          if constexpr (Gm::kWide) {
 #pragma unroll
-          for (int b = 0; b < NQ; ++b) acc[b] = fmaf(v[b], inv, acc[b]);
+            for (int b = 0; b < NQ; ++b) acc[b] = fmaf(v[b] + v[NQ + b], inv, acc[b]);
+          } else {
+#pragma unroll
+            for (int b = 0; b < NQ; ++b) acc[b] = fmaf(v[b], inv, acc[b]);
+          }
         }
       }
       tc_fence_before();
@@ -857,7 +870,7 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
     const int n_tiles = (n_chunks + kScanM - 1) / kScanM;
     const int grid = std::max(1, std::min(sm_count(), n_tiles));
     uint32_t cols = 32;
-    while (cols < 2u * d.n_r * w.nq) cols <<= 1;
+    while (cols < 2u * d.n_r * w.nq * (w.nq == 16 ? 2u : 1u)) cols <<= 1;  // double buffer x columns per head
     for (int pass = 0; pass < w.passes; ++pass) {
       ScanParams p;
       p.chunk_off = chunk_off;
