@@ -289,15 +289,17 @@ struct ScanGeom {
   static constexpr int kQBox = NQ * 128;                // one 64-dim x NQ-row box
   static constexpr int kKBytes = kHalves * kKBox;
   static constexpr int kQBytes = 2 * kHalves * kQBox;   // hi and lo: [half j][hi | lo][NQ rows]
-  // NQ = 16: one MMA per k-step with N = 2 NQ (the hi and lo rows side by side, summed in the
-  // epilogue) - half the MMA chain of accumulating hi and lo into one accumulator, so each
-  // stage is released sooner; NQ = 32 keeps one accumulator per head (TMEM holds 512 columns)
-  static constexpr bool kWide = NQ == 16;
-  static constexpr int kCols = kWide ? 2 * NQ : NQ;     // TMEM columns per head
+  // one MMA per k-step with N = 2 NQ (the hi and lo rows side by side, summed in the
+  // epilogue): half the MMA chain of accumulating hi and lo into one accumulator, so each
+  // stage is released sooner.  TMEM (512 columns) holds two tiles' accumulators for NQ = 16,
+  // one for NQ = 32; either way a head's columns are released as soon as the epilogue has
+  // read them, so the next tile's MMA of that head need not wait for the whole epilogue.
+  static constexpr int kCols = 2 * NQ;                  // TMEM columns per head
+  static constexpr int kBufs = NQ == 16 ? 2 : 1;        // tiles in flight in TMEM
   static constexpr int kStageBytes = kKBytes + kQBytes;
   static constexpr int kStages = (NQ == 16 || DR == 64) ? 5 : 4;
   static constexpr int kNormBytes = 2 * 8 * kScanM * 4;  // [2 tiles][8 heads][128 rows] fp32
-  static constexpr int kBars = 2 * kStages + 6;
+  static constexpr int kBars = 2 * kStages + kBufs * 9 + 4;
   static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + kNormBytes + kBars * 8 + 16;
 };
 
@@ -314,10 +316,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   float* n2s = reinterpret_cast<float*>(smem + S * Gm::kStageBytes);  // [2 tiles][8 heads][128]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * Gm::kStageBytes + Gm::kNormBytes);
   uint64_t* empty = full + S;
-  uint64_t* tfull = empty + S;   // [2] MMA of a tile committed
-  uint64_t* tempty = tfull + 2;  // [2] epilogue done with a tile's TMEM buffer and norms
-  uint64_t* nfull = tempty + 2;  // [2] norms of a tile written
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(nfull + 2);
+  uint64_t* tfull = empty + S;                 // [kBufs] MMA of a tile committed
+  uint64_t* tempty = tfull + Gm::kBufs;        // [kBufs][8] epilogue has read a head's accumulator
+  uint64_t* nfull = tempty + Gm::kBufs * 8;    // [2] norms of a tile written
+  uint64_t* nempty = nfull + 2;                // [2] epilogue has read a tile's norms
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(nempty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_r = p.n_r;
@@ -331,10 +334,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1 + kScanNormWarps);  // MMA commit + the norm warps
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < Gm::kBufs; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], kScanEpiWarps);
+      for (int hh = 0; hh < 8; ++hh) mbar_init(&tempty[b * 8 + hh], kScanEpiWarps);
+    }
+    for (int b = 0; b < 2; ++b) {
       mbar_init(&nfull[b], kScanNormWarps);
+      mbar_init(&nempty[b], kScanEpiWarps);
     }
     fence_mbar_init();
     prefetch_tensormap(&kr_map);
@@ -381,9 +387,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       constexpr uint32_t idesc = umma_idesc_bf16(kScanM, Gm::kCols);
       for (int it = 0; it < n_it; ++it) {
         const int lt = it / n_r, h = it % n_r;
-        const int buf = lt & 1;
+        const int buf = lt % Gm::kBufs, use = lt / Gm::kBufs;
         const int st = it % S;
-        if (h == 0 && lt >= 2) mbar_wait(&tempty[buf], ((lt >> 1) - 1) & 1);
+        if (use >= 1) mbar_wait(&tempty[buf * 8 + h], (use - 1) & 1);  // this head's columns read
         mbar_wait(&full[st], (it / S) & 1);
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * buf_cols + h * Gm::kCols;
@@ -393,12 +399,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         for (int ks = 0; ks < KS; ++ks) {
           const int j = ks >> 2, off = (ks & 3) * 32;
           const uint64_t a_desc = umma_desc_k_sw128(k_addr + j * Gm::kKBox + off);
-          if constexpr (Gm::kWide) {  // B = the 2 NQ rows [hi; lo] of this k-half
-            umma_bf16(d_tmem, a_desc, umma_desc_k_sw128(q_addr + j * 2 * Gm::kQBox + off), idesc, ks > 0);
-          } else {
-            umma_bf16(d_tmem, a_desc, umma_desc_k_sw128(q_addr + j * 2 * Gm::kQBox + off), idesc, ks > 0);
-            umma_bf16(d_tmem, a_desc, umma_desc_k_sw128(q_addr + (j * 2 + 1) * Gm::kQBox + off), idesc, 1);
-          }
+          // B = the 2 NQ rows [hi; lo] of this k-half
+          umma_bf16(d_tmem, a_desc, umma_desc_k_sw128(q_addr + j * 2 * Gm::kQBox + off), idesc, ks > 0);
         }
         umma_commit(&empty[st]);
         if (h == n_r - 1) umma_commit(&tfull[buf]);
@@ -409,9 +411,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     const int row = 32 * (warp & 3) + lane;  // chunk within the tile
     for (int it = 0; it < n_it; ++it) {
       const int lt = it / n_r, h = it % n_r;
-      const int buf = lt & 1;
+      const int buf = lt & 1;  // norm buffer
       const int st = it % S;
-      if (h == 0 && lt >= 2) mbar_wait(&tempty[buf], ((lt >> 1) - 1) & 1);  // n2s[buf] is free again
+      if (h == 0 && lt >= 2) mbar_wait(&nempty[buf], ((lt >> 1) - 1) & 1);  // n2s[buf] is free again
       mbar_wait(&full[st], (it / S) & 1);
       const uint8_t* k_s = stages + st * Gm::kStageBytes;
       float n2p[4] = {0.f, 0.f, 0.f, 0.f};
@@ -442,11 +444,12 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     int cur = 0;                     // lower bound for this warp's document search
     for (int lt = 0; lt < n_lt; ++lt) {
       const int tile = t_begin + lt;
-      const int buf = lt & 1;
-      mbar_wait(&nfull[buf], (lt >> 1) & 1);
-      mbar_wait(&tfull[buf], (lt >> 1) & 1);
+      const int nbuf = lt & 1;                                    // norm buffer
+      const int buf = lt % Gm::kBufs, use = lt / Gm::kBufs;      // TMEM buffer
+      mbar_wait(&nfull[nbuf], (lt >> 1) & 1);
+      mbar_wait(&tfull[buf], use & 1);
       tc_fence_after();
-      const float* nb2 = n2s + (size_t)buf * 8 * kScanM;
+      const float* nb2 = n2s + (size_t)nbuf * 8 * kScanM;
       float acc[NQ];
 #pragma unroll
       for (int b = 0; b < NQ; ++b) acc[b] = 0.f;
@@ -457,19 +460,24 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
           const float inv = 1.0f / fmaxf(sqrtf(nb2[hh * kScanM + row]), kEps);
           float v[32];
           tmem_ld32(t_row + hh * Gm::kCols, v);
-          tmem_ld_wait();
-          if constexpr (Gm::kWide) {
+          if constexpr (NQ == 32) {
+            float w[32];
+            tmem_ld32(t_row + hh * Gm::kCols + 32, w);
+            tmem_ld_wait();
+#pragma unroll
+            for (int b = 0; b < NQ; ++b) acc[b] = fmaf(v[b] + w[b], inv, acc[b]);
+          } else {
+            tmem_ld_wait();
 #pragma unroll
             for (int b = 0; b < NQ; ++b) acc[b] = fmaf(v[b] + v[NQ + b], inv, acc[b]);
-          } else {
-#pragma unroll
-            for (int b = 0; b < NQ; ++b) acc[b] = fmaf(v[b], inv, acc[b]);
           }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[buf * 8 + hh]);  // the next tile may reuse these columns
         }
       }
-      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[buf]);
+      if (lane == 0) mbar_arrive(&nempty[nbuf]);
 
       // documents of this warp's 32 rows: a warp-wide 32-ary search for the first row's
       // document, then one lookahead of 32 document boundaries (32 consecutive rows cross at
@@ -870,7 +878,8 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
     const int n_tiles = (n_chunks + kScanM - 1) / kScanM;
     const int grid = std::max(1, std::min(sm_count(), n_tiles));
     uint32_t cols = 32;
-    while (cols < 2u * d.n_r * w.nq * (w.nq == 16 ? 2u : 1u)) cols <<= 1;  // double buffer x columns per head
+    // columns: 2 NQ per head (hi and lo side by side), two tiles in flight for NQ = 16, one for 32
+    while (cols < (w.nq == 16 ? 2u : 1u) * d.n_r * 2u * w.nq) cols <<= 1;
     for (int pass = 0; pass < w.passes; ++pass) {
       ScanParams p;
       p.chunk_off = chunk_off;
