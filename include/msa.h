@@ -161,6 +161,9 @@ msa_status msa_append_memory(const msa_dims* dims, const void* H_new, int64_t T_
  *            head-major [n_r, n_chunks, d_r] for kr_layout 1 (each head's keys contiguous:
  *            the scan then streams whole 32 KB slices instead of 256-byte pieces).
  *   chunk_off[n_docs + 1] device int32 chunk offsets of the documents.
+ *   kr_inv_norm  optional [n_chunks, n_r] fp32 from msa_router_key_norms: the keys'
+ *            inverse norms, computed once offline; NULL = computed during the scan
+ *            (the same values: both square-sum the stored bf16 keys in fp32).
  *   doc_scores [B, n_docs] fp32 out, optional (NULL = not written).
  *   topk_idx [B, k] int32 out: document ids, descending score, ties to the
  *            lower id.  topk_score [B, k] fp32 out: their scores.
@@ -175,8 +178,22 @@ size_t msa_route_workspace_size(const msa_dims* dims, int32_t B, int32_t q_token
                                 int32_t n_chunks, int32_t k, msa_doc_agg agg);
 msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR, int32_t B, int32_t q_tokens,
                           const void* KR_bar, const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks,
-                          int32_t k, msa_doc_agg agg, int32_t kr_layout, float* doc_scores, int32_t* topk_idx,
+                          int32_t k, msa_doc_agg agg, int32_t kr_layout, const float* kr_inv_norm,
+                          float* doc_scores, int32_t* topk_idx,
                           float* topk_score, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Inverse norms of the pooled router keys (offline, once per memory).
+ * Pages: IRMaD "M. Materials & Methods", routing item (the cosine divides by the
+ * norm of every pooled router key; the keys are fixed once the memory is
+ * encoded).  kr_inv_norm[j, h] = 1 / max(||K̄^R_{j,h}||, 1e-12), the norm square-
+ * summed in fp32 from the stored bf16 values.  Passing the result to
+ * msa_route_topk spares the scan its per-chunk norm work.
+ *   KR_bar   [n_chunks, n_r, d_r] (kr_layout 0) or [n_r, n_chunks, d_r] (kr_layout 1) bf16.
+ *   kr_inv_norm [n_chunks, n_r] fp32 device out.
+ * ------------------------------------------------------------------------- */
+msa_status msa_router_key_norms(const msa_dims* dims, const void* KR_bar, int32_t n_chunks, int32_t kr_layout,
+                                float* kr_inv_norm, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Merge of top-k candidates (memory-parallel routing).

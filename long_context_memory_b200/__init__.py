@@ -18,7 +18,7 @@ from typing import Optional
 
 __all__ = [
     "Dims", "MSAError", "lib", "chunk_offsets", "encode_memory", "append_memory", "route_topk", "sparse_attend",
-    "aux_loss", "kv_append",
+    "aux_loss", "kv_append", "router_key_norms",
     "route_workspace_size", "attend_workspace_size", "rope_cache_build", "topk_merge", "rope_rows", "gather_kv", "encode_workspace_size", "check_device_errors",
     "trace_enable", "trace_reset", "trace_read", "trace_kernel_names", "AGG_MAX", "AGG_MEAN",
 ]
@@ -69,7 +69,8 @@ def _load():
         "msa_aux_loss_workspace_size": (SZ, [DP, I32, I32]),
         "msa_aux_loss": (I32, [DP, P, P, P, I32, I32, F, P, P, P, P, P, SZ, P]),
         "msa_route_workspace_size": (SZ, [DP, I32, I32, I32, I32, I32, I32]),
-        "msa_route_topk": (I32, [DP, P, P, I32, I32, P, P, I32, I32, I32, I32, I32, P, P, P, P, SZ, P]),
+        "msa_route_topk": (I32, [DP, P, P, I32, I32, P, P, I32, I32, I32, I32, I32, P, P, P, P, P, SZ, P]),
+        "msa_router_key_norms": (I32, [DP, P, I32, I32, P, P]),
         "msa_attend_workspace_size": (SZ, [DP, I32, I32, I32, I32, I32]),
         "msa_sparse_attend": (I32, [DP, P, I32, I32, P, P, P, I32, I32, P, I32, P, P, P, I32, I32, P, I32, F, P, P, SZ,
                                     P]),
@@ -219,13 +220,14 @@ def route_workspace_size(dims, B: int, n_docs: int, n_chunks: int, k: int, agg: 
 
 
 def route_topk(dims, Hq, W_QR, KR_bar, chunk_off, k: int, agg: int = AGG_MAX, want_doc_scores: bool = False,
-               out=None, ws=None, stream=None, kr_head_major: bool = False, q_tokens: int = 1):
+               out=None, ws=None, stream=None, kr_head_major: bool = False, q_tokens: int = 1, kr_inv_norm=None):
     """Top-k documents per query.  Returns (topk_idx [B,k] int32, topk_score [B,k] fp32, doc_scores|None).
 
     ``Hq`` holds B * q_tokens rows (token t of query b at row b * q_tokens + t); a chunk's
     score for a query is the largest over its tokens.
     ``W_QR=None`` means ``Hq`` already holds the router queries Q^R [B * q_tokens, n_r*d_r].
     ``kr_head_major``: KR_bar is [n_r, C, d_r] instead of [C, n_r, d_r].
+    ``kr_inv_norm``: the keys' inverse norms from ``router_key_norms`` (computed once per memory).
     """
     import torch
 
@@ -242,8 +244,20 @@ def route_topk(dims, Hq, W_QR, KR_bar, chunk_off, k: int, agg: int = AGG_MAX, wa
     nbytes = route_workspace_size(dims, B, n_docs, n_chunks, k, agg, q_tokens)
     ws = _workspace(nbytes, dev, ws)
     _check(lib.msa_route_topk(ctypes.byref(dd), _ptr(Hq), _ptr(W_QR), B, q_tokens, _ptr(KR_bar), _ptr(chunk_off), n_docs,
-                              n_chunks, k, agg, int(bool(kr_head_major)), _ptr(out[2]), _ptr(out[0]), _ptr(out[1]), _aligned_ptr(ws), nbytes,
+                              n_chunks, k, agg, int(bool(kr_head_major)), _ptr(kr_inv_norm), _ptr(out[2]), _ptr(out[0]), _ptr(out[1]), _aligned_ptr(ws), nbytes,
                               _stream(stream)))
+    return out
+
+
+def router_key_norms(dims, KR_bar, kr_head_major: bool = False, out=None, stream=None):
+    """[n_chunks, n_r] fp32 inverse norms of the pooled router keys (offline, once per memory)."""
+    import torch
+
+    n_chunks = KR_bar.shape[1] if kr_head_major else KR_bar.shape[0]
+    if out is None:
+        out = torch.empty((n_chunks, dims.n_r), dtype=torch.float32, device=KR_bar.device)
+    _check(lib.msa_router_key_norms(ctypes.byref(Dims.of(dims)), _ptr(KR_bar), n_chunks, int(bool(kr_head_major)),
+                                    _ptr(out), _stream(stream)))
     return out
 
 

@@ -52,6 +52,7 @@ enum KernelId : int {
   kKChunkOffExtend,
   kKAuxLoss,
   kKKvAppend,
+  kKKrNorms,
   kKernelCount
 };
 
@@ -120,9 +121,11 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // ---------------------------------------------------------------------------
 size_t route_workspace(const msa_dims& d, int B, int M, int n_docs, int n_chunks, int k, msa_doc_agg agg,
                        void* ws, struct RouteWs* out);
+msa_status kr_norms_launch(const msa_dims& d, const void* KR_bar, int n_chunks, int kr_layout, float* inv_norm,
+                           cudaStream_t s);
 msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int B, int M, const void* KR_bar,
                         const int32_t* chunk_off, int n_docs, int n_chunks, int k, msa_doc_agg agg, int kr_layout,
-                        float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws,
+                        const float* kr_inv_norm, float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws,
                         cudaStream_t s);
 
 msa_status topk_merge_launch(const float* cand_score, const int32_t* cand_idx, int B, int n_cand, int k,

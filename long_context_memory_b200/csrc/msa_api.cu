@@ -110,7 +110,7 @@ namespace {
 const char* kKernelNames[kKernelCount] = {
     "router_query", "scan", "topk_slice", "topk_merge", "rope_table", "attn_split", "attn_combine",
     "enc_chunk_map", "enc_transpose_w", "enc_gemm_k", "enc_pool_h", "enc_gemm_pooled", "rope_rows", "gather_plan", "gather_copy",
-    "chunk_off_extend", "aux_loss", "kv_append"};
+    "chunk_off_extend", "aux_loss", "kv_append", "kr_norms"};
 
 struct TraceState {
   std::mutex mu;
@@ -265,7 +265,8 @@ size_t msa_route_workspace_size(const msa_dims* dims, int32_t B, int32_t q_token
 msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR, int32_t B, int32_t q_tokens,
                           const void* KR_bar,
                           const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks, int32_t k, msa_doc_agg agg,
-                          int32_t kr_layout, float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws, size_t ws_bytes,
+                          int32_t kr_layout, const float* kr_inv_norm, float* doc_scores, int32_t* topk_idx,
+                          float* topk_score, void* ws, size_t ws_bytes,
                           void* stream) {
   msa_status st = check_dims(dims, false, true);
   if (st != MSA_OK) return st;
@@ -293,9 +294,23 @@ msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR
   if (ws_bytes < need) return fail(MSA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
   if (need && (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)))
     return fail(MSA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
+  CHECK_OPT_PTR(kr_inv_norm);
   if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
-  return route_launch(*dims, Hq, W_QR, B, q_tokens, KR_bar, chunk_off, n_docs, n_chunks, k, agg, kr_layout, doc_scores, topk_idx,
+  return route_launch(*dims, Hq, W_QR, B, q_tokens, KR_bar, chunk_off, n_docs, n_chunks, k, agg, kr_layout, kr_inv_norm,
+                      doc_scores, topk_idx,
                       topk_score, ws, static_cast<cudaStream_t>(stream));
+}
+
+msa_status msa_router_key_norms(const msa_dims* dims, const void* KR_bar, int32_t n_chunks, int32_t kr_layout,
+                                float* kr_inv_norm, void* stream) {
+  msa_status st = check_dims(dims, false, true);
+  if (st != MSA_OK) return st;
+  if (n_chunks < 1) return fail(MSA_ERR_INVALID_ARG, "n_chunks must be >= 1 (got %d)", n_chunks);
+  if (kr_layout != 0 && kr_layout != 1) return fail(MSA_ERR_INVALID_ARG, "kr_layout must be 0 or 1 (got %d)", kr_layout);
+  CHECK_PTR(KR_bar);
+  CHECK_PTR(kr_inv_norm);
+  if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
+  return kr_norms_launch(*dims, KR_bar, n_chunks, kr_layout, kr_inv_norm, static_cast<cudaStream_t>(stream));
 }
 
 msa_status msa_topk_merge(const float* cand_score, const int32_t* cand_idx, int32_t B, int32_t n_cand, int32_t k,

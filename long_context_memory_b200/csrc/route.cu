@@ -278,6 +278,7 @@ struct ScanParams {
   int q_tokens;    // query tokens per query: scan row r belongs to query r / q_tokens
   int q_base, q_count, pass;
   int head_major;  // K̄^R stored [n_r][C][d_r] instead of [C][n_r][d_r]
+  const float* inv_norm;  // [C][n_r] 1 / max(||K̄^R_jh||, eps) precomputed, or null (norm warps compute it)
   uint32_t tmem_cols;
   float inv_nr;
 };
@@ -332,7 +333,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + kScanNormWarps);  // MMA commit + the norm warps
+      mbar_init(&empty[s], 1 + (p.inv_norm ? 0 : kScanNormWarps));  // MMA commit (+ the norm warps)
     }
     for (int b = 0; b < Gm::kBufs; ++b) {
       mbar_init(&tfull[b], 1);
@@ -409,7 +410,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   } else if (warp < 2 + kScanNormWarps) {
     // ------- norm warps: squared norm of every row's head-h slice, stage released at once -------
     const int row = 32 * (warp & 3) + lane;  // chunk within the tile
-    for (int it = 0; it < n_it; ++it) {
+    for (int it = 0; it < (p.inv_norm ? 0 : n_it); ++it) {
       const int lt = it / n_r, h = it % n_r;
       const int buf = lt & 1;  // norm buffer
       const int st = it % S;
@@ -446,7 +447,15 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       const int tile = t_begin + lt;
       const int nbuf = lt & 1;                                    // norm buffer
       const int buf = lt % Gm::kBufs, use = lt / Gm::kBufs;      // TMEM buffer
-      mbar_wait(&nfull[nbuf], (lt >> 1) & 1);
+      const int jrow = tile * kScanM + row;
+      float invg[8];  // precomputed inverse norms of this row (loads in flight during the waits)
+      if (p.inv_norm) {
+#pragma unroll
+        for (int hh = 0; hh < 8; ++hh)
+          invg[hh] = (hh < n_r && jrow < p.n_chunks) ? __ldg(&p.inv_norm[(size_t)jrow * n_r + hh]) : 0.f;
+      } else {
+        mbar_wait(&nfull[nbuf], (lt >> 1) & 1);
+      }
       mbar_wait(&tfull[buf], use & 1);
       tc_fence_after();
       const float* nb2 = n2s + (size_t)nbuf * 8 * kScanM;
@@ -457,7 +466,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
 #pragma unroll
       for (int hh = 0; hh < 8; ++hh) {
         if (hh < n_r) {
-          const float inv = 1.0f / fmaxf(sqrtf(nb2[hh * kScanM + row]), kEps);
+          const float inv = p.inv_norm ? invg[hh] : 1.0f / fmaxf(sqrtf(nb2[hh * kScanM + row]), kEps);
           float v[32];
           tmem_ld32(t_row + hh * Gm::kCols, v);
           if constexpr (NQ == 32) {
@@ -509,13 +518,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       }
       const int prev = __shfl_up_sync(0xffffffffu, doc, 1);
       const bool head = (lane == 0) || (prev != doc);
-      // the document pattern is the same for every query: which shuffle partners share my document
-      uint32_t same = 0;
-#pragma unroll
-      for (int e = 0; e < 5; ++e) {
-        const int od = __shfl_down_sync(0xffffffffu, doc, 1 << e);
-        if (lane + (1 << e) < 32 && od == doc) same |= 1u << e;
-      }
+      // rows are in chunk order, so a document's rows are a contiguous lane range starting at
+      // a head lane; rows past the memory (doc -1) trail the last range and carry key 0, below
+      // every ordered score
+      const unsigned heads = __ballot_sync(0xffffffffu, head && doc >= 0);
 #pragma unroll
       for (int b = 0; b < NQ; ++b) {
         if (b >= p.q_count) break;  // warp-uniform
@@ -528,13 +534,15 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
             else atomicMax(dst, float_to_ordered(sc));
           }
         } else {
-          float x = doc >= 0 ? sc : -__int_as_float(0x7f800000);
-#pragma unroll
-          for (int e = 0; e < 5; ++e) {
-            const float ox = __shfl_down_sync(0xffffffffu, x, 1 << e);
-            if (same & (1u << e)) x = fmaxf(x, ox);
+          const uint32_t key = doc >= 0 ? float_to_ordered(sc) : 0u;
+          unsigned rem = heads;
+          while (rem) {  // one warp reduction and one atomic per document range
+            const int L = __ffs(rem) - 1;
+            rem &= rem - 1;
+            const int E = rem ? __ffs(rem) - 1 : 32;
+            const uint32_t mx = __reduce_max_sync(0xffffffffu, (lane >= L && lane < E) ? key : 0u);
+            if (lane == L) atomicMax(&p.doc_key[qi * p.n_docs + doc], mx);
           }
-          if (head && doc >= 0) atomicMax(&p.doc_key[qi * p.n_docs + doc], float_to_ordered(x));
         }
       }
     }
@@ -788,6 +796,36 @@ cudaError_t launch_scan(int d_r, int nq, bool mean, const CUtensorMap& kmap, con
               : launch_scan_t<64, 32, false>(kmap, qmap, p, grid, s);
 }
 
+// 1 / max(||K̄^R_jh||, eps) of every pooled router key (one pass over K̄^R): lanes of a row
+// each take 16 bytes (coalesced), the row's lanes reduce with shuffles
+__global__ void __launch_bounds__(256) kr_norms_kernel(const __nv_bfloat16* __restrict__ KR, int n_chunks, int n_r,
+                                                       int d_r, int head_major, float* __restrict__ inv_norm) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int L = d_r / 8;  // lanes per row (16 or 8)
+  const int lane = threadIdx.x & 31;
+  const int rpw = 32 / L;  // rows per warp step
+  const size_t n_rows = (size_t)n_chunks * n_r;
+  const size_t warp_id = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
+  const size_t n_warps = (size_t)gridDim.x * blockDim.x / 32;
+  for (size_t r0 = warp_id * rpw; r0 < n_rows; r0 += n_warps * rpw) {  // warp-uniform
+    const size_t r = r0 + lane / L;
+    const bool ok = r < n_rows;
+    const uint4 w = ok ? __ldg(reinterpret_cast<const uint4*>(KR + r * d_r) + (lane % L)) : make_uint4(0, 0, 0, 0);
+    float ss = 0.f;
+    float2 f;
+    f = unpack_bf16x2(w.x); ss = fmaf(f.x, f.x, ss); ss = fmaf(f.y, f.y, ss);
+    f = unpack_bf16x2(w.y); ss = fmaf(f.x, f.x, ss); ss = fmaf(f.y, f.y, ss);
+    f = unpack_bf16x2(w.z); ss = fmaf(f.x, f.x, ss); ss = fmaf(f.y, f.y, ss);
+    f = unpack_bf16x2(w.w); ss = fmaf(f.x, f.x, ss); ss = fmaf(f.y, f.y, ss);
+    for (int o = 1; o < L; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (ok && lane % L == 0) {
+      const size_t out = head_major ? (r % n_chunks) * n_r + r / n_chunks : r;
+      inv_norm[out] = 1.0f / fmaxf(sqrtf(ss), kEps);
+    }
+  }
+}
+
 size_t topk_slice_smem() { return (kSliceDocs + 512 + 4) * sizeof(uint64_t) + 256 * sizeof(uint32_t); }
 size_t topk_merge_smem(int n) { return ((size_t)n + 512 + 4) * sizeof(uint64_t) + 256 * sizeof(uint32_t); }
 
@@ -800,6 +838,18 @@ msa_status topk_merge_launch(const float* cand_score, const int32_t* cand_idx, i
   MSA_CUDA_CHECK(cudaFuncSetAttribute(topk_merge_pairs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
   MSA_CUDA_CHECK(launch_pdl(topk_merge_pairs_kernel, dim3(B), dim3(kTopkThreads), sm, s, cand_score, cand_idx, n_cand,
                             k, topk_idx, topk_score));
+  return MSA_OK;
+}
+
+msa_status kr_norms_launch(const msa_dims& d, const void* KR_bar, int n_chunks, int kr_layout, float* inv_norm,
+                           cudaStream_t s) {
+  TraceScope ts(kKKrNorms, s);
+  const size_t n_rows = (size_t)n_chunks * d.n_r;
+  const int rows_per_cta = 256 / (d.d_r / 8);
+  const int blocks = (int)std::max<size_t>(1, std::min<size_t>((n_rows + rows_per_cta - 1) / rows_per_cta,
+                                                               (size_t)sm_count() * 8));
+  MSA_CUDA_CHECK(launch_pdl(kr_norms_kernel, dim3(blocks), dim3(256), 0, s, static_cast<const __nv_bfloat16*>(KR_bar),
+                            n_chunks, d.n_r, d.d_r, kr_layout, inv_norm));
   return MSA_OK;
 }
 
@@ -826,7 +876,7 @@ size_t route_workspace(const msa_dims& d, int B, int M, int n_docs, int n_chunks
 
 msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int B, int M, const void* KR_bar,
                         const int32_t* chunk_off, int n_docs, int n_chunks, int k, msa_doc_agg agg, int kr_layout,
-                        float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws, cudaStream_t s) {
+                        const float* kr_inv_norm, float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws, cudaStream_t s) {
   RouteWs w;
   route_workspace(d, B, M, n_docs, n_chunks, k, agg, ws, &w);
   const int NR = d.n_r * d.d_r;
@@ -900,6 +950,7 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
       p.q_count = std::min(R - p.q_base, w.nq);
       p.pass = pass;
       p.head_major = kr_layout == 1;
+      p.inv_norm = kr_inv_norm;
       p.tmem_cols = cols;
       p.inv_nr = 1.0f / (float)d.n_r;
       TraceScope ts(kKScan, s);

@@ -66,7 +66,8 @@ extern "C" msa_status msa_route_topk_static(const msa_dims* dims, const void* Hq
                                             int32_t n_chunks, int32_t k, msa_doc_agg agg, float* doc_scores,
                                             int32_t* topk_idx, float* topk_score, void* stream) {
   if (!dims || B < 1 || q_tokens < 1 || (int64_t)B * q_tokens > 65535 || n_docs < 1 || n_chunks < 1 || k < 1)
-    return msa_route_topk(dims, Hq, W_QR, B, q_tokens, KR_bar, chunk_off, n_docs, n_chunks, k, agg, 0, doc_scores, topk_idx,
+    return msa_route_topk(dims, Hq, W_QR, B, q_tokens, KR_bar, chunk_off, n_docs, n_chunks, k, agg, 0, nullptr,
+                          doc_scores, topk_idx,
                           topk_score, nullptr, 0, stream);  // reports the argument error, launches nothing
   const size_t need = msa_route_workspace_size(dims, B, q_tokens, n_docs, n_chunks, k, agg);
   if (need > kStaticScratchBytes)
@@ -77,6 +78,7 @@ extern "C" msa_status msa_route_topk_static(const msa_dims* dims, const void* Hq
   void* scratch = nullptr;
   msa_status st = static_scratch(&scratch);
   if (st != MSA_OK) return st;
-  return msa_route_topk(dims, Hq, W_QR, B, q_tokens, KR_bar, chunk_off, n_docs, n_chunks, k, agg, 0, doc_scores, topk_idx,
+  return msa_route_topk(dims, Hq, W_QR, B, q_tokens, KR_bar, chunk_off, n_docs, n_chunks, k, agg, 0, nullptr,
+                        doc_scores, topk_idx,
                         topk_score, scratch, kStaticScratchBytes, stream);
 }

@@ -51,7 +51,8 @@ def randn_bf16(shape, g, device):
 
 
 class RouteCase:
-    def __init__(self, T, B, median, seed, device, k=16, dims=W.QWEN3_4B_DIMS, layers=1, head_major=False):
+    def __init__(self, T, B, median, seed, device, k=16, dims=W.QWEN3_4B_DIMS, layers=1, head_major=False,
+                 norms=False):
         import torch
 
         import long_context_memory_b200 as msa
@@ -65,6 +66,8 @@ class RouteCase:
         self.head_major = head_major
         kr_shape = (dims.n_r, C, dims.d_r) if head_major else (C, dims.n_r, dims.d_r)
         self.KR = [randn_bf16(kr_shape, g, device) for _ in range(layers)]
+        # inverse key norms computed once per memory (offline), as a deployment would keep them
+        self.inv = [msa.router_key_norms(dims, kr, kr_head_major=head_major) for kr in self.KR] if norms else None
         self.Hq = randn_bf16((B, dims.hidden), g, device)
         self.W_QR = (torch.randn((dims.hidden, dims.n_r * dims.d_r), generator=g, device=device) /
                      math.sqrt(dims.hidden)).to(torch.bfloat16)
@@ -89,7 +92,8 @@ class RouteCase:
 
     def run(self, layer=0):
         self.msa.route_topk(self.d, self.Hq, self.W_QR, self.KR[layer], self.chunk_off, self.k,
-                            out=(self.idx, self.sc, None), ws=self.ws, kr_head_major=self.head_major)
+                            out=(self.idx, self.sc, None), ws=self.ws, kr_head_major=self.head_major,
+                            kr_inv_norm=self.inv[layer] if self.inv else None)
 
     @property
     def scan_bytes(self):
@@ -201,16 +205,17 @@ def main():
     ap.add_argument("--tokens", type=int, default=None, help="memory tokens (encode default 1M; route cases: "
                     "their own size unless given)")
     ap.add_argument("--kr-layout", choices=["chunk", "head"], default="chunk")
+    ap.add_argument("--norms", action="store_true", help="route cases: pass precomputed key norms")
     a = ap.parse_args()
     dev = torch.device("cuda:0")
     seed = W.BASE_SEED + 7
-    hm = a.kr_layout == "head"
+    hm, nm = a.kr_layout == "head", a.norms
     if a.case == "route1m":
-        case = RouteCase(a.tokens or 1_000_000, a.batch or 1, 2048, seed, dev, head_major=hm)
+        case = RouteCase(a.tokens or 1_000_000, a.batch or 1, 2048, seed, dev, head_major=hm, norms=nm)
     elif a.case == "route16m":
-        case = RouteCase(a.tokens or 16_000_000, a.batch or 32, 2048, seed, dev, head_major=hm)
+        case = RouteCase(a.tokens or 16_000_000, a.batch or 32, 2048, seed, dev, head_major=hm, norms=nm)
     elif a.case == "route100m":
-        case = RouteCase(a.tokens or 100_000_000, a.batch or 1, 4096, seed, dev, head_major=hm)
+        case = RouteCase(a.tokens or 100_000_000, a.batch or 1, 4096, seed, dev, head_major=hm, norms=nm)
     elif a.case == "attend1m":
         case = AttendCase(1_000_000, a.batch or 1, 2048, 4096, seed, dev)
     elif a.case == "attend16m":
@@ -230,7 +235,7 @@ def main():
             case.run()
             e1.record(s)
             torch.cuda.synchronize()
-            tag = f"{a.case}[{a.kr_layout}]" if a.case.startswith("route") else a.case
+            tag = f"{a.case}[{a.kr_layout}{',norms' if a.norms else ''}]" if a.case.startswith("route") else a.case
             print(f"{tag} launch {i}: {e0.elapsed_time(e1) * 1e3:.1f} us", flush=True)
 
 

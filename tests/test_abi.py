@@ -78,7 +78,7 @@ def _route(msa, dims, B=1, n_docs=10, n_chunks=20, k=4, agg=0, ws_bytes=None, Hq
     if ws_bytes is None:
         ws_bytes = need
     return msa.lib.msa_route_topk(ctypes.byref(dd), Hq, None, B, M, kr, FAKE, n_docs, n_chunks, k, agg, layout, None,
-                                  idx,
+                                  None, idx,
                                   FAKE,
                                   0x100000 if ws_bytes else None, ws_bytes, None)
 
@@ -182,6 +182,15 @@ def test_kv_append_validation(msa):
     assert lib.msa_kv_append(ctypes.byref(dd), FAKE, FAKE, FAKE, FAKE, 1, 16, FAKE, -1, None) == 1
     assert lib.msa_kv_append(ctypes.byref(msa.Dims.of(_dims(head_dim=96))), FAKE, FAKE, FAKE, FAKE, 1, 16, FAKE, 2,
                              None) == 2
+
+
+def test_router_key_norms_validation(msa):
+    lib = msa.lib
+    dd = msa.Dims.of(_dims())
+    assert lib.msa_router_key_norms(ctypes.byref(dd), FAKE, 0, 0, FAKE, None) == 1       # no chunks
+    assert lib.msa_router_key_norms(ctypes.byref(dd), FAKE, 10, 2, FAKE, None) == 1      # layout
+    assert lib.msa_router_key_norms(ctypes.byref(dd), FAKE, 10, 0, None, None) == 1      # NULL output
+    assert lib.msa_router_key_norms(ctypes.byref(msa.Dims.of(_dims(d_r=96))), FAKE, 10, 0, FAKE, None) == 2
 
 
 def test_topk_merge_validation(msa):

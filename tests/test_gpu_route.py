@@ -108,6 +108,35 @@ def test_route_fused_topk_matches_separate_kernels(msa, cuda_device, agg):
         check_topk(i4[b], s4[b], s[b], 16, where=f"b={b}")
 
 
+@pytest.mark.parametrize("head_major", [False, True])
+@pytest.mark.parametrize("B,n_r,d_r", [(1, 8, 128), (13, 4, 64), (32, 3, 128)])
+def test_route_with_precomputed_key_norms(msa, cuda_device, head_major, B, n_r, d_r):
+    # inverse norms computed once (msa_router_key_norms) and passed to the scan
+    import torch
+
+    dims, doc_off, KR, QR, *_ = _route_case(700 + B + n_r, 400, B, n_r, d_r)
+    co, C = msa.chunk_offsets(doc_off)
+    kr = np.ascontiguousarray(KR.transpose(1, 0, 2)) if head_major else KR
+    krd = _dev(kr, cuda_device)
+    inv = msa.router_key_norms(dims, krd, kr_head_major=head_major)
+    co_d = torch.from_numpy(co).to(cuda_device)
+    idx, sc, ds = msa.route_topk(dims, _dev(QR, cuda_device), None, krd, co_d, 12, want_doc_scores=True,
+                                 kr_head_major=head_major, kr_inv_norm=inv)
+    _, _, ds0 = msa.route_topk(dims, _dev(QR, cuda_device), None, krd, co_d, 12, want_doc_scores=True,
+                               kr_head_major=head_major)
+    torch.cuda.synchronize()
+    assert msa.check_device_errors() == 0
+    want = 1.0 / np.maximum(np.sqrt((O.bf16_to_f64(KR) ** 2).sum(-1)), O.EPS)   # [C, n_r]
+    assert np.allclose(inv.cpu().numpy(), want, rtol=2e-6, atol=0)
+    ds, ds0 = ds.cpu().numpy(), ds0.cpu().numpy()
+    assert np.max(np.abs(ds - ds0)) < 1e-5          # the same norms up to fp32 summation order
+    s, _, _ = O.route_topk(O.bf16_to_f64(QR).reshape(B, n_r, d_r), KR, co, 12)
+    assert np.max(np.abs(ds - s)) < SCORE_ATOL
+    idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+    for b in range(B):
+        check_topk(idx[b], sc[b], s[b], 12, where=f"b={b}")
+
+
 def test_route_edge_shapes(msa, cuda_device):
     # one-chunk docs, k = n_docs, chunk count not a multiple of the tile, single doc
     for seed, n_docs, lo, hi, k in [(1, 17, 1, 64, 17), (2, 1, 5, 5, 1), (3, 40, 1, 1, 40), (4, 33, 60, 70, 1)]:
