@@ -260,7 +260,7 @@ def run_extras(msa, dev, hbm_peak):
                      "kernels_us": {k: v[0] / v[1] * 1e3 for k, v in kt.items() if v[1]}}
 
     try:
-        c16 = PC.RouteCase(16_000_000, 32, 2048, W.BASE_SEED + 2, dev)
+        c16 = PC.RouteCase(16_000_000, 32, 2048, W.BASE_SEED + 2, dev, norms=True)
         route_entry("mem16m_b32_route", c16, 1)
         del c16
         a16 = PC.AttendCase(16_000_000, 32, 2048, 8192, W.BASE_SEED + 2, dev, rotated=True)
@@ -278,7 +278,7 @@ def run_extras(msa, dev, hbm_peak):
         torch.cuda.empty_cache()
         free = torch.cuda.mem_get_info(dev)[0]
         layers = int(max(1, min(36, (free - (8 << 30)) // 3_300_000_000)))
-        c100 = PC.RouteCase(100_000_000, 1, 4096, W.BASE_SEED + 4, dev, layers=layers)
+        c100 = PC.RouteCase(100_000_000, 1, 4096, W.BASE_SEED + 4, dev, layers=layers, norms=True)
         route_entry("mem100m_b1_route", c100, layers)
         c100.set_batch(16, seed=W.BASE_SEED + 40)
         route_entry("mem100m_b16_route", c100, layers)
@@ -337,6 +337,8 @@ def run_gpu(args):
     loc_len = torch.from_numpy(c["loc_len"]).to(dev)
     # distinct copies at distinct addresses so that consecutive steps miss L2
     rot = [base] + [{kk: v.clone() for kk, v in base.items()} for _ in range(N_ROT - 1)]
+    # the pooled router keys' inverse norms, computed once per memory (offline, like the encoding)
+    inv_rot = [msa.router_key_norms(d, x["KR"]) for x in rot]
     out_idx = [torch.empty((B, k), dtype=torch.int32, device=dev) for _ in range(N_ROT)]
     out_sc = [torch.empty((B, k), dtype=torch.float32, device=dev) for _ in range(N_ROT)]
     out_o = [torch.empty((B, d.n_q, d.head_dim), dtype=torch.bfloat16, device=dev) for _ in range(N_ROT)]
@@ -360,7 +362,8 @@ def run_gpu(args):
     def step(i):
         x = rot[i % N_ROT]
         j = i % N_ROT
-        msa.route_topk(d, x["Hq"], W_QR, x["KR"], chunk_off, k, out=(out_idx[j], out_sc[j], None), ws=r_ws)
+        msa.route_topk(d, x["Hq"], W_QR, x["KR"], chunk_off, k, out=(out_idx[j], out_sc[j], None), ws=r_ws,
+                       kr_inv_norm=inv_rot[j])
         msa.kv_append(d, k_new, v_new, x["K_loc"], x["V_loc"], slots, c["pos_offset"])
         msa.sparse_attend(d, x["q"], x["K_bar"], x["V_bar"], chunk_off, out_idx[j], x["K_loc"], x["V_loc"], loc_len,
                           c["pos_offset"], out=out_o[j], ws=a_ws, k_loc_rotated=True)
@@ -426,7 +429,7 @@ def run_gpu(args):
     sel = out_idx[0].cpu().numpy()
     n_sel = int(sum(co_np[i + 1] - co_np[i] for i in sel[0]))
     per_kernel = {n: (ms, cnt) for n, (ms, cnt) in kt.items() if cnt > 0}
-    scan_bytes = C * d.n_r * d.d_r * 2
+    scan_bytes = C * d.n_r * (d.d_r * 2 + 4)  # the pooled router keys and their inverse norms
     attn_bytes = B * (n_sel + int(c["loc_len"][0])) * d.n_kv * d.head_dim * 2 * 2
     cand = {"scan": scan_bytes, "attn_split": attn_bytes}
     dom = max(cand, key=lambda n: per_kernel.get(n, (0, 1))[0])
@@ -468,7 +471,8 @@ def run_gpu(args):
         dev_kn.copy_(host["k_new"], non_blocking=True)
         dev_vn.copy_(host["v_new"], non_blocking=True)
         msa.kv_append(d, dev_kn, dev_vn, x["K_loc"], x["V_loc"], slots, c["pos_offset"])
-        msa.route_topk(d, dev_hq, W_QR, x["KR"], chunk_off, k, out=(out_idx[0], out_sc[0], None), ws=r_ws)
+        msa.route_topk(d, dev_hq, W_QR, x["KR"], chunk_off, k, out=(out_idx[0], out_sc[0], None), ws=r_ws,
+                       kr_inv_norm=inv_rot[i % N_ROT])
         msa.sparse_attend(d, dev_q, x["K_bar"], x["V_bar"], chunk_off, out_idx[0], x["K_loc"], x["V_loc"], loc_len,
                           c["pos_offset"], out=out_o[0], ws=a_ws, k_loc_rotated=True)
         h_idx.copy_(out_idx[0], non_blocking=True)

@@ -518,10 +518,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       }
       const int prev = __shfl_up_sync(0xffffffffu, doc, 1);
       const bool head = (lane == 0) || (prev != doc);
-      // rows are in chunk order, so a document's rows are a contiguous lane range starting at
-      // a head lane; rows past the memory (doc -1) trail the last range and carry key 0, below
-      // every ordered score
-      const unsigned heads = __ballot_sync(0xffffffffu, head && doc >= 0);
+      // the document pattern is the same for every query: which shuffle partners share my document
+      uint32_t same = 0;
+#pragma unroll
+      for (int e = 0; e < 5; ++e) {
+        const int od = __shfl_down_sync(0xffffffffu, doc, 1 << e);
+        if (lane + (1 << e) < 32 && od == doc) same |= 1u << e;
+      }
 #pragma unroll
       for (int b = 0; b < NQ; ++b) {
         if (b >= p.q_count) break;  // warp-uniform
@@ -534,15 +537,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
             else atomicMax(dst, float_to_ordered(sc));
           }
         } else {
-          const uint32_t key = doc >= 0 ? float_to_ordered(sc) : 0u;
-          unsigned rem = heads;
-          while (rem) {  // one warp reduction and one atomic per document range
-            const int L = __ffs(rem) - 1;
-            rem &= rem - 1;
-            const int E = rem ? __ffs(rem) - 1 : 32;
-            const uint32_t mx = __reduce_max_sync(0xffffffffu, (lane >= L && lane < E) ? key : 0u);
-            if (lane == L) atomicMax(&p.doc_key[qi * p.n_docs + doc], mx);
+          float x = doc >= 0 ? sc : -__int_as_float(0x7f800000);
+#pragma unroll
+          for (int e = 0; e < 5; ++e) {
+            const float ox = __shfl_down_sync(0xffffffffu, x, 1 << e);
+            if (same & (1u << e)) x = fmaxf(x, ox);
           }
+          if (head && doc >= 0) atomicMax(&p.doc_key[qi * p.n_docs + doc], float_to_ordered(x));
         }
       }
     }

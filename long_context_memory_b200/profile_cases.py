@@ -97,7 +97,8 @@ class RouteCase:
 
     @property
     def scan_bytes(self):
-        return self.C * self.d.n_r * self.d.d_r * 2
+        """Algorithmic bytes of one scan: the pooled router keys (and their inverse norms when given)."""
+        return self.C * self.d.n_r * (self.d.d_r * 2 + (4 if self.inv else 0))
 
 
 class AttendCase:
