@@ -304,6 +304,133 @@ struct ScanGeom {
   static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + kNormBytes + kBars * 8 + 16;
 };
 
+// The scan's epilogue for one warp: TMEM lane quarter q4 (32 rows of every tile) and the QW
+// queries q_off .. q_off + QW - 1.  Per tile: wait for the tile's MMA (and its norms), read each
+// head's accumulator columns (the hi and lo halves of this warp's queries) and release them, find
+// each row's document, and fold each document segment's maximum into doc_key (or store the chunk
+// scores for the mean).  A warp whose queries are all past q_count still takes part in the
+// barrier protocol but does no work.
+template <int DR, int NQ, bool MEAN, int QW>
+__device__ __forceinline__ void scan_epilogue(const ScanParams& p, int q4, int q_off, int lane, int t_begin, int n_lt,
+                                              uint32_t tmem_base, uint32_t buf_cols, const float* n2s, uint64_t* tfull,
+                                              uint64_t* tempty, uint64_t* nfull, uint64_t* nempty) {
+  using Gm = ScanGeom<DR, NQ>;
+  const int n_r = p.n_r;
+  const int row = 32 * q4 + lane;  // chunk within the tile
+  const bool active = q_off < p.q_count;
+  int cur = 0;                     // lower bound for this warp's document search
+  for (int lt = 0; lt < n_lt; ++lt) {
+    const int tile = t_begin + lt;
+    const int nbuf = lt & 1;                                    // norm buffer
+    const int buf = lt % Gm::kBufs, use = lt / Gm::kBufs;      // TMEM buffer
+    const int jrow = tile * kScanM + row;
+    float invg[8];  // precomputed inverse norms of this row (loads in flight during the waits)
+    if (p.inv_norm) {
+#pragma unroll
+      for (int hh = 0; hh < 8; ++hh)
+        invg[hh] = (active && hh < n_r && jrow < p.n_chunks) ? __ldg(&p.inv_norm[(size_t)jrow * n_r + hh]) : 0.f;
+    } else {
+      mbar_wait(&nfull[nbuf], (lt >> 1) & 1);
+    }
+    mbar_wait(&tfull[buf], use & 1);
+    tc_fence_after();
+    const float* nb2 = n2s + (size_t)nbuf * 8 * kScanM;
+    float acc[QW];
+#pragma unroll
+    for (int b = 0; b < QW; ++b) acc[b] = 0.f;
+    const uint32_t t_row = tmem_base + ((uint32_t)(32 * q4) << 16) + buf * buf_cols;
+#pragma unroll
+    for (int hh = 0; hh < 8; ++hh) {
+      if (hh < n_r) {
+        if (active) {
+          const float inv = p.inv_norm ? invg[hh] : 1.0f / fmaxf(sqrtf(nb2[hh * kScanM + row]), kEps);
+          const uint32_t c_hi = t_row + hh * Gm::kCols + q_off, c_lo = c_hi + NQ;
+          float v[QW], w[QW];
+          if constexpr (QW == 32) {
+            tmem_ld32(c_hi, v);
+            tmem_ld32(c_lo, w);
+          } else if constexpr (QW == 16) {
+            tmem_ld16(c_hi, v);
+            tmem_ld16(c_lo, w);
+          } else {
+            tmem_ld8(c_hi, v);
+            tmem_ld8(c_lo, w);
+          }
+          tmem_ld_wait();
+#pragma unroll
+          for (int b = 0; b < QW; ++b) acc[b] = fmaf(v[b] + w[b], inv, acc[b]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[buf * 8 + hh]);  // the next tile may reuse these columns
+      }
+    }
+    __syncwarp();
+    if (lane == 0 && !p.inv_norm) mbar_arrive(&nempty[nbuf]);
+    if (!active) continue;
+
+    // documents of this warp's 32 rows: a warp-wide 32-ary search for the first row's
+    // document, then one lookahead of 32 document boundaries (32 consecutive rows cross at
+    // most 31 of them)
+    const int j = tile * kScanM + row;
+    const int j0 = tile * kScanM + 32 * q4;
+    int doc = -1;
+    if (j0 < p.n_chunks) {
+      int lo = cur, hi = p.n_docs;  // answer in [lo, hi): largest d with chunk_off[d] <= j0
+      while (hi - lo > 1) {
+        const int step = (hi - lo + 31) >> 5;
+        const int probe = lo + lane * step;
+        const bool ok = probe < hi && __ldg(&p.chunk_off[probe]) <= j0;
+        const unsigned m = __ballot_sync(0xffffffffu, ok);
+        const int L = 31 - __clz(m);  // lane 0 always qualifies (chunk_off[lo] <= j0)
+        lo = lo + L * step;
+        hi = min(hi, lo + step);
+      }
+      const int d0 = lo;
+      const int bi = d0 + 1 + lane;
+      const int bnd = bi <= p.n_docs ? __ldg(&p.chunk_off[bi]) : 0x7fffffff;
+#pragma unroll 4
+      for (int r = 0; r < 32; ++r) {
+        const unsigned m = __ballot_sync(0xffffffffu, bnd <= j0 + r);
+        if (lane == r) doc = d0 + __popc(m);
+      }
+      if (j >= p.n_chunks) doc = -1;
+      cur = d0;
+    }
+    const int prev = __shfl_up_sync(0xffffffffu, doc, 1);
+    const bool head = (lane == 0) || (prev != doc);
+    // the document pattern is the same for every query: which shuffle partners share my document
+    uint32_t same = 0;
+#pragma unroll
+    for (int e = 0; e < 5; ++e) {
+      const int od = __shfl_down_sync(0xffffffffu, doc, 1 << e);
+      if (lane + (1 << e) < 32 && od == doc) same |= 1u << e;
+    }
+#pragma unroll
+    for (int bb = 0; bb < QW; ++bb) {
+      const int b = q_off + bb;
+      if (b >= p.q_count) break;  // warp-uniform
+      const float sc = acc[bb] * p.inv_nr;
+      const size_t qi = (size_t)((p.q_base + b) / p.q_tokens);  // max over a query's tokens: atomicMax
+      if (MEAN) {
+        if (doc >= 0) {
+          uint32_t* dst = &p.chunk_k[qi * p.n_chunks + j];
+          if (p.q_tokens == 1) *dst = float_to_ordered(sc);
+          else atomicMax(dst, float_to_ordered(sc));
+        }
+      } else {
+        float x = doc >= 0 ? sc : -__int_as_float(0x7f800000);
+#pragma unroll
+        for (int e = 0; e < 5; ++e) {
+          const float ox = __shfl_down_sync(0xffffffffu, x, 1 << e);
+          if (same & (1u << e)) x = fmaxf(x, ox);
+        }
+        if (head && doc >= 0) atomicMax(&p.doc_key[qi * p.n_docs + doc], float_to_ordered(x));
+      }
+    }
+  }
+}
+
 template <int DR, int NQ, bool MEAN>
 __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_constant__ CUtensorMap kr_map,
                                                                const __grid_constant__ CUtensorMap q_map,
@@ -337,7 +464,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     }
     for (int b = 0; b < Gm::kBufs; ++b) {
       mbar_init(&tfull[b], 1);
-      for (int hh = 0; hh < 8; ++hh) mbar_init(&tempty[b * 8 + hh], kScanEpiWarps);
+      for (int hh = 0; hh < 8; ++hh) mbar_init(&tempty[b * 8 + hh], p.inv_norm ? 8 : kScanEpiWarps);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&nfull[b], kScanNormWarps);
@@ -407,6 +534,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         if (h == n_r - 1) umma_commit(&tfull[buf]);
       }
     }
+  } else if (warp < 2 + kScanNormWarps && p.inv_norm) {
+    // norms given: these four warps take the second half of the queries of each row
+    scan_epilogue<DR, NQ, MEAN, NQ / 2>(p, warp & 3, NQ / 2, lane, t_begin, n_lt, tmem_base, buf_cols, n2s, tfull,
+                                        tempty, nfull, nempty);
   } else if (warp < 2 + kScanNormWarps) {
     // ------- norm warps: squared norm of every row's head-h slice, stage released at once -------
     const int row = 32 * (warp & 3) + lane;  // chunk within the tile
@@ -439,114 +570,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       }
     }
   } else {
-    // ------- epilogue warps: head mean of cosines, per-document max (TMEM lane quarter = warp % 4) -------
-    const int q4 = warp & 3;
-    const int row = 32 * q4 + lane;  // chunk within the tile
-    int cur = 0;                     // lower bound for this warp's document search
-    for (int lt = 0; lt < n_lt; ++lt) {
-      const int tile = t_begin + lt;
-      const int nbuf = lt & 1;                                    // norm buffer
-      const int buf = lt % Gm::kBufs, use = lt / Gm::kBufs;      // TMEM buffer
-      const int jrow = tile * kScanM + row;
-      float invg[8];  // precomputed inverse norms of this row (loads in flight during the waits)
-      if (p.inv_norm) {
-#pragma unroll
-        for (int hh = 0; hh < 8; ++hh)
-          invg[hh] = (hh < n_r && jrow < p.n_chunks) ? __ldg(&p.inv_norm[(size_t)jrow * n_r + hh]) : 0.f;
-      } else {
-        mbar_wait(&nfull[nbuf], (lt >> 1) & 1);
-      }
-      mbar_wait(&tfull[buf], use & 1);
-      tc_fence_after();
-      const float* nb2 = n2s + (size_t)nbuf * 8 * kScanM;
-      float acc[NQ];
-#pragma unroll
-      for (int b = 0; b < NQ; ++b) acc[b] = 0.f;
-      const uint32_t t_row = tmem_base + ((uint32_t)(32 * q4) << 16) + buf * buf_cols;
-#pragma unroll
-      for (int hh = 0; hh < 8; ++hh) {
-        if (hh < n_r) {
-          const float inv = p.inv_norm ? invg[hh] : 1.0f / fmaxf(sqrtf(nb2[hh * kScanM + row]), kEps);
-          float v[32];
-          tmem_ld32(t_row + hh * Gm::kCols, v);
-          if constexpr (NQ == 32) {
-            float w[32];
-            tmem_ld32(t_row + hh * Gm::kCols + 32, w);
-            tmem_ld_wait();
-#pragma unroll
-            for (int b = 0; b < NQ; ++b) acc[b] = fmaf(v[b] + w[b], inv, acc[b]);
-          } else {
-            tmem_ld_wait();
-#pragma unroll
-            for (int b = 0; b < NQ; ++b) acc[b] = fmaf(v[b] + v[NQ + b], inv, acc[b]);
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[buf * 8 + hh]);  // the next tile may reuse these columns
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&nempty[nbuf]);
-
-      // documents of this warp's 32 rows: a warp-wide 32-ary search for the first row's
-      // document, then one lookahead of 32 document boundaries (32 consecutive rows cross at
-      // most 31 of them)
-      const int j = tile * kScanM + row;
-      const int j0 = tile * kScanM + 32 * q4;
-      int doc = -1;
-      if (j0 < p.n_chunks) {
-        int lo = cur, hi = p.n_docs;  // answer in [lo, hi): largest d with chunk_off[d] <= j0
-        while (hi - lo > 1) {
-          const int step = (hi - lo + 31) >> 5;
-          const int probe = lo + lane * step;
-          const bool ok = probe < hi && __ldg(&p.chunk_off[probe]) <= j0;
-          const unsigned m = __ballot_sync(0xffffffffu, ok);
-          const int L = 31 - __clz(m);  // lane 0 always qualifies (chunk_off[lo] <= j0)
-          lo = lo + L * step;
-          hi = min(hi, lo + step);
-        }
-        const int d0 = lo;
-        const int bi = d0 + 1 + lane;
-        const int bnd = bi <= p.n_docs ? __ldg(&p.chunk_off[bi]) : 0x7fffffff;
-#pragma unroll 4
-        for (int r = 0; r < 32; ++r) {
-          const unsigned m = __ballot_sync(0xffffffffu, bnd <= j0 + r);
-          if (lane == r) doc = d0 + __popc(m);
-        }
-        if (j >= p.n_chunks) doc = -1;
-        cur = d0;
-      }
-      const int prev = __shfl_up_sync(0xffffffffu, doc, 1);
-      const bool head = (lane == 0) || (prev != doc);
-      // the document pattern is the same for every query: which shuffle partners share my document
-      uint32_t same = 0;
-#pragma unroll
-      for (int e = 0; e < 5; ++e) {
-        const int od = __shfl_down_sync(0xffffffffu, doc, 1 << e);
-        if (lane + (1 << e) < 32 && od == doc) same |= 1u << e;
-      }
-#pragma unroll
-      for (int b = 0; b < NQ; ++b) {
-        if (b >= p.q_count) break;  // warp-uniform
-        const float sc = acc[b] * p.inv_nr;
-        const size_t qi = (size_t)((p.q_base + b) / p.q_tokens);  // max over a query's tokens: atomicMax
-        if (MEAN) {
-          if (doc >= 0) {
-            uint32_t* dst = &p.chunk_k[qi * p.n_chunks + j];
-            if (p.q_tokens == 1) *dst = float_to_ordered(sc);
-            else atomicMax(dst, float_to_ordered(sc));
-          }
-        } else {
-          float x = doc >= 0 ? sc : -__int_as_float(0x7f800000);
-#pragma unroll
-          for (int e = 0; e < 5; ++e) {
-            const float ox = __shfl_down_sync(0xffffffffu, x, 1 << e);
-            if (same & (1u << e)) x = fmaxf(x, ox);
-          }
-          if (head && doc >= 0) atomicMax(&p.doc_key[qi * p.n_docs + doc], float_to_ordered(x));
-        }
-      }
-    }
+    // epilogue warps: every query of each row, or the first half when the norms are given
+    if (p.inv_norm)
+      scan_epilogue<DR, NQ, MEAN, NQ / 2>(p, warp & 3, 0, lane, t_begin, n_lt, tmem_base, buf_cols, n2s, tfull, tempty,
+                                          nfull, nempty);
+    else
+      scan_epilogue<DR, NQ, MEAN, NQ>(p, warp & 3, 0, lane, t_begin, n_lt, tmem_base, buf_cols, n2s, tfull, tempty,
+                                      nfull, nempty);
   }
   tc_fence_before();
   __syncthreads();
