@@ -32,14 +32,12 @@
 namespace msa {
 
 struct RouteWs {
-  float* qr;          // [rq_splits][B][NR] fp32 partial router queries (W_QR given)
-  uint32_t* head_done;  // [n_r] CTAs finished per router head (back to 0 after each call)
   uint32_t* scan_ticket;  // scan CTAs finished (fused top-k); zeroed by the router query kernel
   __nv_bfloat16* q_hl; // [passes][n_r][2][NQ][d_r] normalised query, bf16 hi and lo terms
   uint32_t* doc_key;  // [B][n_docs] ordered-uint32 doc max (MAX)
   uint32_t* chunk_k;  // [B][n_chunks] ordered chunk scores (MEAN)
   uint64_t* cand;     // [B][n_slices][k] slice winners
-  int nq, passes, n_slices, rq_splits;
+  int nq, passes, n_slices;
 };
 
 namespace {
@@ -50,170 +48,172 @@ constexpr int kTopkThreads = 1024;
 constexpr float kEps = 1e-12f;
 
 // --------------------------------------------------------------------------
-// Router query, one kernel: Q^R = H_q W^QR, per-head normalisation, bf16 hi + lo
-// terms in the layout the scan's TMA reads (q_hl[pass][head][hi|lo][NQ rows][d_r];
-// rows of padding queries are zero), and the clearing of the scan's max keys.
-// A row is one query token (B queries x M tokens).
+// Router query: Q^R = H_q W^QR, per-head normalisation, bf16 hi + lo terms in the
+// layout the scan's TMA reads (q_hl[pass][head][hi|lo][NQ rows][d_r]; rows of
+// padding queries are zero), and the clearing of the scan's max keys.  A row is
+// one query token (B queries x M tokens).
 //
-// Grid (n_splits, n_r): CTA (s, h) multiplies rows [s*RS, (s+1)*RS) of W^QR's
-// head-h column block (a contiguous RS x d_r slab, read once, coalesced: each
-// warp reads whole 256-byte row pieces) by the matching slice of every query,
-// staged in shared memory, and writes fp32 partial sums qpart[s][b][h*d_r + c].
-// The last CTA of a head (per-head ticket) sums the n_splits partials in split
-// order (so the result does not depend on scheduling), normalises the head and
-// writes the hi/lo rows.  With W_QR == NULL the rows of Hq already hold Q^R and
-// only the head step runs (grid (1, n_r)).
+// Grid (8, n_r), one thread-block cluster of 8 CTAs per router head: CTA r of
+// head h multiplies rows [r*RS, (r+1)*RS) of W^QR's head-h column block (staged in
+// shared memory 256 rows at a time, coalesced) by the matching slice of 16 query
+// rows on the tensor cores (mma.sync m16n8k16, bf16 in, fp32 out).  The 8 partial
+// products meet in distributed shared memory: after a cluster barrier CTA r sums,
+// in rank order, rows r and r + 8 of the 16-row block over the cluster's CTAs,
+// normalises them and writes their hi/lo terms.  No global partials, no counters.
+// With W_QR == NULL the rows of Hq already hold Q^R and router_query_direct_kernel
+// only normalises them.
 // --------------------------------------------------------------------------
 constexpr int kRqThreads = 256;
-constexpr int kRqMaxSplitRows = 256;
-constexpr int kRqTargetCtas = 144;
+constexpr int kRqCluster = 8;   // CTAs per router head
+constexpr int kRqPiece = 384;   // rows of W staged at a time (hidden <= 3072: one piece)
 
-struct RqGeom {
-  int n_splits, rows;  // CTAs per head, rows of W per CTA (multiple of 16)
-};
+// rows of W per CTA (a multiple of 16)
+int rq_split_rows(int hidden) { return ((hidden + kRqCluster - 1) / kRqCluster + 15) / 16 * 16; }
 
-RqGeom rq_geom(int hidden, int n_r) {
-  int splits = std::max(1, kRqTargetCtas / n_r);
-  splits = std::max(splits, (hidden + kRqMaxSplitRows - 1) / kRqMaxSplitRows);
-  int rows = (hidden + splits - 1) / splits;
-  rows = (rows + 15) / 16 * 16;
-  return RqGeom{(hidden + rows - 1) / rows, rows};
+// shared memory: a W piece [kRqPiece][d_r] and 16 query rows [16][kRqPiece], both bf16 with rows
+// padded by 16 bytes (ldmatrix's 8 row addresses in distinct bank groups), then the CTA's
+// partial product [16][d_r] fp32
+__host__ __device__ inline int rq_w_stride(int d_r) { return d_r * 2 + 16; }
+__host__ __device__ inline int rq_h_stride() { return kRqPiece * 2 + 16; }
+size_t rq_smem_bytes(int d_r) {
+  return (size_t)kRqPiece * rq_w_stride(d_r) + 16 * (size_t)rq_h_stride() + 16 * (size_t)d_r * sizeof(float);
 }
 
-// shared memory: the W slab [rows][d_r] and 16 query rows [16][rows], both bf16 with rows
-// padded by 16 bytes so that ldmatrix's 8 row addresses fall in distinct bank groups
-__host__ __device__ inline int rq_w_stride(int d_r) { return d_r * 2 + 16; }
-__host__ __device__ inline int rq_h_stride(int rows) { return rows * 2 + 16; }
-size_t rq_smem_bytes(int d_r, int rows) { return (size_t)rows * rq_w_stride(d_r) + 16 * (size_t)rq_h_stride(rows); }
+__device__ __forceinline__ void rq_clear(uint32_t* clear, size_t n_clear, uint32_t* scan_ticket) {
+  if (scan_ticket && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *scan_ticket = 0u;
+  if (clear) {
+    const size_t cta = (size_t)blockIdx.y * gridDim.x + blockIdx.x, n_cta = (size_t)gridDim.x * gridDim.y;
+    for (size_t i = cta * blockDim.x + threadIdx.x; i < n_clear; i += n_cta * blockDim.x) clear[i] = 0u;
+  }
+}
+
+// one normalised row of head h: hi/lo bf16 terms into the scan's query layout
+__device__ __forceinline__ void rq_store_row(__nv_bfloat16* q_hl, int b, int h, int i, float x, int n_r, int d_r,
+                                             int nq) {
+  const int pass = b / nq, row = b % nq;
+  const size_t base = (((size_t)pass * n_r + h) * 2) * nq;
+  const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+  q_hl[(base + row) * d_r + i] = hi;
+  q_hl[(base + nq + row) * d_r + i] = lo;
+}
 
 __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
     const __nv_bfloat16* __restrict__ Hq, const __nv_bfloat16* __restrict__ W, int B, int b_pad, int hidden,
-    int n_r, int d_r, int nq, int split_rows, float* __restrict__ qpart, uint32_t* __restrict__ head_done,
-    __nv_bfloat16* __restrict__ q_hl, uint32_t* __restrict__ clear, size_t n_clear,
-    uint32_t* __restrict__ scan_ticket) {
+    int n_r, int d_r, int nq, int split_rows, __nv_bfloat16* __restrict__ q_hl, uint32_t* __restrict__ clear,
+    size_t n_clear, uint32_t* __restrict__ scan_ticket) {
   extern __shared__ __align__(16) uint8_t rq_smem[];
-  __shared__ float invn[kRqThreads / 32];
-  __shared__ bool last;
+  __shared__ float wsum[kRqThreads / 32];
   pdl_launch_dependents();
   pdl_wait();
   const int NR = n_r * d_r;
-  const int h = blockIdx.y, split = blockIdx.x, n_splits = gridDim.x;
+  const int rank = blockIdx.x, h = blockIdx.y;  // the cluster spans blockIdx.x
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint16_t* hq = reinterpret_cast<const uint16_t*>(Hq);
+  rq_clear(clear, n_clear, scan_ticket);
 
-  // clear the scan's max keys (grid-stride) and its ticket; the scan only runs after this
-  // kernel completes
-  if (scan_ticket && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *scan_ticket = 0u;
-  if (clear) {
-    const size_t cta = (size_t)blockIdx.y * gridDim.x + blockIdx.x, n_cta = (size_t)gridDim.x * gridDim.y;
-    for (size_t i = cta * kRqThreads + tid; i < n_clear; i += n_cta * kRqThreads) clear[i] = 0u;
-  }
+  const int ws = rq_w_stride(d_r), hstr = rq_h_stride();
+  uint8_t* wsm = rq_smem;
+  uint8_t* hsm = rq_smem + (size_t)kRqPiece * ws;
+  float* part = reinterpret_cast<float*>(hsm + 16 * (size_t)hstr);  // [16][d_r]
+  const int k0 = rank * split_rows;
+  const int nrows = max(0, min(split_rows, hidden - k0));  // a multiple of 16
+  const int n_nt = d_r / 8;                 // n-tiles of 8 columns
+  const int nt_per_warp = n_nt / 8;         // 2 or 1
+  const int n0 = warp * nt_per_warp;        // first n-tile of this warp
+  const int per_row = d_r / 8;              // 16-byte pieces of a W row
 
-  if (W) {
-    // Q^R partial of this split on the tensor cores (mma.sync m16n8k16, bf16 in, fp32 out):
-    // D[16 query rows][d_r] = H_q slice [16][rows] x W slab [rows][d_r]; warp w owns the
-    // n-tiles 2w, 2w + 1 (d_r = 128) or w (d_r = 64)
-    const int k0 = split * split_rows;
-    const int nrows = min(split_rows, hidden - k0);  // multiple of 16
-    const int ws = rq_w_stride(d_r), hstr = rq_h_stride(split_rows);
-    uint8_t* wsm = rq_smem;
-    uint8_t* hsm = rq_smem + (size_t)split_rows * ws;
-    {  // W slab: 16-byte pieces, a row's pieces on consecutive threads (coalesced)
-      const int per_row = d_r / 8;
-      const __nv_bfloat16* wsrc = W + (size_t)k0 * NR + h * d_r;
-      for (int i = tid; i < nrows * per_row; i += kRqThreads) {
+  for (int b0 = 0; b0 < b_pad; b0 += 16) {
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    for (int p0 = 0; p0 < nrows; p0 += kRqPiece) {
+      const int pr = min(kRqPiece, nrows - p0);
+      __syncthreads();  // the previous piece is consumed
+      const __nv_bfloat16* wsrc = W + (size_t)(k0 + p0) * NR + h * d_r;
+      for (int i = tid; i < pr * per_row; i += kRqThreads) {
         const int r = i / per_row, c = i % per_row;
         *reinterpret_cast<uint4*>(wsm + (size_t)r * ws + c * 16) =
             __ldg(reinterpret_cast<const uint4*>(wsrc + (size_t)r * NR) + c);
       }
-    }
-    const int n_nt = d_r / 8;                 // n-tiles of 8 columns
-    const int nt_per_warp = n_nt / 8;         // 2 or 1
-    const int ksteps = nrows / 16;
-    for (int b0 = 0; b0 < B; b0 += 16) {
-      __syncthreads();  // W slab landed / previous query rows consumed
-      {
-        const int vec = nrows / 8;
-        for (int i = tid; i < 16 * vec; i += kRqThreads) {
-          const int j = i / vec, v = i % vec;
-          uint4 x = make_uint4(0, 0, 0, 0);
-          if (b0 + j < B) x = __ldg(reinterpret_cast<const uint4*>(hq + (size_t)(b0 + j) * hidden + k0) + v);
-          *reinterpret_cast<uint4*>(hsm + (size_t)j * hstr + v * 16) = x;
-        }
+      const int vec = pr / 8;
+      for (int i = tid; i < 16 * vec; i += kRqThreads) {
+        const int j = i / vec, v = i % vec;
+        uint4 x = make_uint4(0, 0, 0, 0);
+        if (b0 + j < B) x = __ldg(reinterpret_cast<const uint4*>(hq + (size_t)(b0 + j) * hidden + k0 + p0) + v);
+        *reinterpret_cast<uint4*>(hsm + (size_t)j * hstr + v * 16) = x;
       }
       __syncthreads();
-      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      const int n0 = warp * nt_per_warp;     // first n-tile of this warp
-      for (int ks = 0; ks < ksteps; ++ks) {
+      for (int ks = 0; ks < pr / 16; ++ks) {
         uint32_t a0, a1, a2, a3;
         ldmatrix_x4(a0, a1, a2, a3, smem_u32(hsm + (size_t)(lane & 15) * hstr + (ks * 16 + 8 * (lane >> 4)) * 2));
         const int krow = ks * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+        uint32_t b0r, b1r, b2r, b3r;
         if (nt_per_warp == 2) {
-          uint32_t b0r, b1r, b2r, b3r;
           ldmatrix_x4_trans(b0r, b1r, b2r, b3r, smem_u32(wsm + (size_t)krow * ws + (8 * n0 + 8 * (lane >> 4)) * 2));
           mma_bf16_16816(acc[0], a0, a1, a2, a3, b0r, b1r);
           mma_bf16_16816(acc[1], a0, a1, a2, a3, b2r, b3r);
-        } else {
-          uint32_t b0r, b1r, b2r, b3r;  // two k-halves of one n-tile (the upper lanes' rows repeat)
+        } else {  // two k-halves of one n-tile (the upper lanes' rows repeat)
           ldmatrix_x4_trans(b0r, b1r, b2r, b3r, smem_u32(wsm + (size_t)krow * ws + (8 * n0) * 2));
           mma_bf16_16816(acc[0], a0, a1, a2, a3, b0r, b1r);
         }
       }
-      // D fragment: rows lane/4 and lane/4 + 8, columns 2 (lane % 4) + {0, 1} of each n-tile
+    }
+    // this CTA's partial product of the 16-row block: D fragment rows lane/4 (+8), columns
+    // 2 (lane % 4) + {0, 1} of each n-tile
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        if (t >= nt_per_warp) break;
-        const int col = 8 * (n0 + t) + 2 * (lane & 3);
+    for (int t = 0; t < 2; ++t) {
+      if (t >= nt_per_warp) break;
+      const int col = 8 * (n0 + t) + 2 * (lane & 3);
 #pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-          const int b = b0 + (lane >> 2) + 8 * rr;
-          if (b < B)
-            *reinterpret_cast<float2*>(qpart + ((size_t)split * B + b) * NR + h * d_r + col) =
-                make_float2(acc[t][2 * rr], acc[t][2 * rr + 1]);
-        }
+      for (int rr = 0; rr < 2; ++rr)
+        *reinterpret_cast<float2*>(part + ((lane >> 2) + 8 * rr) * d_r + col) =
+            make_float2(acc[t][2 * rr], acc[t][2 * rr + 1]);
+    }
+    cluster_sync();  // every CTA's partial is written
+
+    // rows rank and rank + 8 of the block: the sum over the cluster's CTAs in rank order
+    {
+      const int q = tid / d_r, i = tid % d_r;  // q: which of the two rows (threads with q > 1 idle)
+      const int row = rank + 8 * q;
+      float v = 0.f;
+      if (q < 2) {
+#pragma unroll
+        for (int r = 0; r < kRqCluster; ++r) v += ld_dsmem_f32(part + row * d_r + i, r);
+      }
+      float ss = v * v;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (lane == 0) wsum[warp] = ss;
+      __syncthreads();
+      if (q < 2) {
+        const int w0 = q * d_r / 32, nw = d_r / 32;  // the warps holding this row
+        float tot = 0.f;
+        for (int w = 0; w < nw; ++w) tot += wsum[w0 + w];
+        const float sc = 1.0f / fmaxf(sqrtf(tot), kEps);
+        rq_store_row(q_hl, b0 + row, h, i, v * sc, n_r, d_r, nq);
       }
     }
-    // this CTA's partials are written: take a ticket; the head's last CTA goes on
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-      const uint32_t prev = atomicAdd(&head_done[h], 1u);
-      last = prev == (uint32_t)(n_splits - 1);
-      if (last) head_done[h] = 0u;  // ready for the next call
-    }
-    __syncthreads();
-    if (!last) return;
-    __threadfence();
+    cluster_sync();  // the partials may be overwritten / the CTAs may exit
   }
+}
 
-  // ---- head step: Q^R of head h for every query (partials summed in split order),
-  //      normalised, written as bf16 hi/lo rows ----
-  const int n_parts = W ? n_splits : 0;
+// Q^R given directly (W_QR == NULL): normalise each row of head h, write the hi/lo terms
+__global__ void __launch_bounds__(kRqThreads) router_query_direct_kernel(
+    const __nv_bfloat16* __restrict__ Hq, int B, int b_pad, int n_r, int d_r, int nq, __nv_bfloat16* __restrict__ q_hl,
+    uint32_t* __restrict__ clear, size_t n_clear, uint32_t* __restrict__ scan_ticket) {
+  __shared__ float invn[kRqThreads / 32];
+  pdl_launch_dependents();
+  pdl_wait();
+  rq_clear(clear, n_clear, scan_ticket);
+  const int NR = n_r * d_r, h = blockIdx.y;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint16_t* hq = reinterpret_cast<const uint16_t*>(Hq);
   for (int b = warp; b < b_pad; b += kRqThreads / 32) {
     float v[4] = {0.f, 0.f, 0.f, 0.f};  // dims lane, lane + 32, ... (d_r <= 128)
     float ss = 0.f;
     if (b < B) {
-      if (W) {
-        // eight splits' loads in flight at a time; the sum still runs in split order
-        const float* src = qpart + (size_t)b * NR + h * d_r + lane;
-        const size_t sstride = (size_t)B * NR;
-        for (int sp0 = 0; sp0 < n_parts; sp0 += 8) {
-          float x[8][4];
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              x[u][e] = (sp0 + u < n_parts && lane + 32 * e < d_r) ? __ldcg(src + (sp0 + u) * sstride + 32 * e) : 0.f;
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) v[e] += x[u][e];
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (lane + 32 * e < d_r) v[e] = bf16_bits_to_float(hq[(size_t)b * NR + h * d_r + lane + 32 * e]);
-      }
+      for (int e = 0; e < 4; ++e)
+        if (lane + 32 * e < d_r) v[e] = bf16_bits_to_float(hq[(size_t)b * NR + h * d_r + lane + 32 * e]);
 #pragma unroll
       for (int e = 0; e < 4; ++e) ss = fmaf(v[e], v[e], ss);
     }
@@ -223,19 +223,9 @@ __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
     __syncwarp();
     const float sc = invn[warp];
     __syncwarp();
-    const int pass = b / nq, row = b % nq;
-    const size_t base = (((size_t)pass * n_r + h) * 2) * nq;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int i = lane + 32 * e;
-      if (i < d_r) {
-        const float x = v[e] * sc;
-        const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-        const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
-        q_hl[(base + row) * d_r + i] = hi;
-        q_hl[(base + nq + row) * d_r + i] = lo;
-      }
-    }
+    for (int e = 0; e < 4; ++e)
+      if (lane + 32 * e < d_r) rq_store_row(q_hl, b, h, lane + 32 * e, v[e] * sc, n_r, d_r, nq);
   }
 }
 
@@ -888,14 +878,10 @@ size_t route_workspace(const msa_dims& d, int B, int M, int n_docs, int n_chunks
                        RouteWs* out) {
   Carver cv(ws);
   RouteWs w{};
-  const int NR = d.n_r * d.d_r;
   const int R = B * M;  // query-token rows
   w.nq = R <= 16 ? 16 : 32;
   w.passes = (R + w.nq - 1) / w.nq;
   w.n_slices = (n_docs + kSliceDocs - 1) / kSliceDocs;
-  w.rq_splits = rq_geom(d.hidden, d.n_r).n_splits;
-  w.qr = cv.take<float>((size_t)w.rq_splits * R * NR);
-  w.head_done = cv.take<uint32_t>(8);
   w.scan_ticket = cv.take<uint32_t>(1);
   w.q_hl = cv.take<__nv_bfloat16>((size_t)w.passes * d.n_r * 2 * w.nq * d.d_r);
   w.doc_key = agg == MSA_AGG_MAX ? cv.take<uint32_t>((size_t)B * n_docs) : nullptr;
@@ -922,15 +908,20 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
 
   // K1: router query (projection, normalisation, hi/lo layout) and document keys cleared
   {
-    MSA_CUDA_CHECK(cudaMemsetAsync(w.head_done, 0, 8 * sizeof(uint32_t), s));
     TraceScope ts(kKRouterQuery, s);
-    const RqGeom g = rq_geom(d.hidden, d.n_r);
-    const size_t sm = W_QR ? rq_smem_bytes(d.d_r, g.rows) : 0;
-    MSA_CUDA_CHECK(cudaFuncSetAttribute(router_query_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-    MSA_CUDA_CHECK(launch_pdl(router_query_kernel, dim3(W_QR ? g.n_splits : 1, d.n_r), dim3(kRqThreads), sm, s,
-                              static_cast<const __nv_bfloat16*>(Hq), static_cast<const __nv_bfloat16*>(W_QR), R,
-                              w.passes * w.nq, d.hidden, d.n_r, d.d_r, w.nq, g.rows, w.qr, w.head_done, w.q_hl,
-                              clear, n_clear, w.scan_ticket));
+    if (W_QR) {
+      const size_t sm = rq_smem_bytes(d.d_r);
+      MSA_CUDA_CHECK(cudaFuncSetAttribute(router_query_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+      MSA_CUDA_CHECK(launch_pdl_cluster(router_query_kernel, dim3(kRqCluster, d.n_r), dim3(kRqThreads), sm, s,
+                                        kRqCluster, static_cast<const __nv_bfloat16*>(Hq),
+                                        static_cast<const __nv_bfloat16*>(W_QR), R, w.passes * w.nq, d.hidden, d.n_r,
+                                        d.d_r, w.nq, rq_split_rows(d.hidden), w.q_hl, clear, n_clear,
+                                        w.scan_ticket));
+    } else {
+      MSA_CUDA_CHECK(launch_pdl(router_query_direct_kernel, dim3(1, d.n_r), dim3(kRqThreads), 0, s,
+                                static_cast<const __nv_bfloat16*>(Hq), R, w.passes * w.nq, d.n_r, d.d_r, w.nq,
+                                w.q_hl, clear, n_clear, w.scan_ticket));
+    }
   }
   // K3: scan, NQ (16 or 32) queries per pass
   {
