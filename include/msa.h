@@ -279,6 +279,13 @@ msa_status msa_aux_loss(const msa_dims* dims, const void* QR, const void* K_pos,
  *              1: K_loc already holds every local key rotated at pos_offset + j
  *              (see msa_rope_rows); rope_cache is then unused.
  *   softmax_scale  0 -> 1/sqrt(head_dim).
+ *   phase    0: the whole call.  1 and 2 split it in two so that the local part can run
+ *            while the query is still being routed: phase 1 attends over the local keys
+ *            only and leaves its partial results in ws (topk_idx, K_bar, V_bar, chunk_off
+ *            and out are not read and may be NULL); phase 2, with the same ws and sizes,
+ *            attends over the selected chunks and merges both parts into out (K_loc and
+ *            V_loc are not read).  Phase 2 must be ordered after phase 1 (same stream, or
+ *            an event).  The result equals phase 0's up to fp32 summation order.
  *   out      [B, M, n_q, head_dim] bf16.
  * Limits: 1 <= M, B * M <= 65535.
  * Query head g attends with KV head g / (n_q / n_kv).  Every query token sees
@@ -294,8 +301,8 @@ msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, int
                              const void* V_bar, const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks,
                              const int32_t* topk_idx, int32_t k, const void* K_loc, const void* V_loc,
                              const int32_t* loc_len, int32_t t_loc_max, int32_t pos_offset,
-                             const void* rope_cache, int32_t k_loc_rotated, float softmax_scale, void* out,
-                             void* ws, size_t ws_bytes, void* stream);
+                             const void* rope_cache, int32_t k_loc_rotated, float softmax_scale, int32_t phase,
+                             void* out, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Host tier: gather the selected documents' pooled K̄/V̄ from pinned host memory.

@@ -72,8 +72,8 @@ def _load():
         "msa_route_topk": (I32, [DP, P, P, I32, I32, P, P, I32, I32, I32, I32, I32, P, P, P, P, P, SZ, P]),
         "msa_router_key_norms": (I32, [DP, P, I32, I32, P, P]),
         "msa_attend_workspace_size": (SZ, [DP, I32, I32, I32, I32, I32]),
-        "msa_sparse_attend": (I32, [DP, P, I32, I32, P, P, P, I32, I32, P, I32, P, P, P, I32, I32, P, I32, F, P, P, SZ,
-                                    P]),
+        "msa_sparse_attend": (I32, [DP, P, I32, I32, P, P, P, I32, I32, P, I32, P, P, P, I32, I32, P, I32, F, I32, P, P,
+                                    SZ, P]),
         "msa_rope_rows": (I32, [DP, P, I32, I32, P, P]),
         "msa_kv_append": (I32, [DP, P, P, P, P, I32, I32, P, I32, P]),
         "msa_gather_kv": (I32, [DP, P, P, I32, P, I32, P, I32, I32, P, P, I32, P, P, P, SZ, P]),
@@ -334,13 +334,14 @@ def kv_append(dims, k_new, v_new, K_loc, V_loc, slots, pos_offset: int, stream=N
 
 def sparse_attend(dims, q, K_bar, V_bar, chunk_off, topk_idx, K_loc, V_loc, loc_len, pos_offset: int,
                   softmax_scale: float = 0.0, out=None, ws=None, stream=None, rope_cache=None,
-                  k_loc_rotated: bool = False):
+                  k_loc_rotated: bool = False, phase: int = 0):
     """GQA attention of the query tokens over [selected docs' K̄; local K].
 
     ``q`` is [B, n_q, head_dim] (one decode token) or [B, M, n_q, head_dim] (the last M local
     tokens, causal among the local keys); ``out`` has the shape of ``q``.
     ``rope_cache`` (from ``rope_cache_build`` with the same pos_offset and t_loc_max) skips
-    rebuilding the local-position rotation table."""
+    rebuilding the local-position rotation table.  ``phase`` 1 / 2 splits the call into the
+    local-keys part and the selected-chunks part (which merges both); pass the same ``ws``."""
     import torch
 
     dd = Dims.of(dims)
@@ -356,7 +357,7 @@ def sparse_attend(dims, q, K_bar, V_bar, chunk_off, topk_idx, K_loc, V_loc, loc_
     _check(lib.msa_sparse_attend(ctypes.byref(dd), _ptr(q), B, M, _ptr(K_bar), _ptr(V_bar), _ptr(chunk_off), n_docs,
                                  K_bar.shape[0], _ptr(topk_idx), k, _ptr(K_loc), _ptr(V_loc), _ptr(loc_len),
                                  t_loc_max, pos_offset, _ptr(rope_cache), int(bool(k_loc_rotated)),
-                                 float(softmax_scale), _ptr(out),
+                                 float(softmax_scale), int(phase), _ptr(out),
                                  _aligned_ptr(ws), nbytes, _stream(stream)))
     return out
 

@@ -33,7 +33,10 @@ struct AttendWs {
   float2* rope_tab;  // [t_loc_max][D/2] (cos, sin)
   float* part_ml;    // [B][n_q][S][2]  running max (log2 domain) and sum
   float* part_o;     // [B][n_q][S][D]  unnormalised output
-  int n_splits;
+  int n_splits;        // splits of the one-launch call (every key)
+  int n_split_local;   // splits of the local-keys phase (ids 0 .. n_split_local - 1)
+  int n_split_chunk;   // splits of the selected-chunks phase (ids after the local ones)
+  int n_parts;         // partial slots per (query token, q head)
 };
 
 namespace {
@@ -70,6 +73,9 @@ struct AttnParams {
   float* part_o;
   int n_q, n_kv, k, n_docs, t_loc_max, pos_offset, n_splits, n_stages;
   int q_tokens;      // M: query tokens per query (the last M local tokens)
+  int phase;         // 0: every key; 1: the local keys only; 2: the selected chunks only
+  int split_base;    // this launch's first split id in the partial arrays
+  int n_splits_total;  // splits per (query token, q head) in the partial arrays
   int tok_per_cta;   // MT: tokens per CTA, MT * G <= 16 mma rows
   int n_tgroups;     // ceil(M / MT)
   float scale_log2;  // softmax scale * log2(e)
@@ -124,7 +130,7 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = warp;               // the KV head this warp serves (warps 0 .. n_kv-1)
   const bool producer = warp == n_kv;  // the last warp only streams tiles in
-  const int k = p.k;
+  const int k = p.phase == 1 ? 0 : p.k;  // the local-keys phase has no selected documents
 
   // ---- no global memory yet: overlaps the previous kernel's tail ----
   for (int i = tid; i < L_.n_stages * L_.stage_bytes / 16; i += blockDim.x)
@@ -187,7 +193,7 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
   __syncthreads();
 
   const int n_sel = seg_v[k];
-  const int n_keys = n_sel + L;
+  const int n_keys = n_sel + (p.phase == 2 ? 0 : L);
   int per_split = (n_keys + p.n_splits - 1) / p.n_splits;
   per_split = (per_split + kTK - 1) / kTK * kTK;
   const int v0 = min(n_keys, split * per_split);
@@ -415,13 +421,14 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
     const int tt = row / G;
     if (tt < nt) {
       const size_t qh = ((size_t)b * p.q_tokens + t0 + tt) * p.n_q + (size_t)h * G + (row - tt * G);
-      float* po = p.part_o + (qh * p.n_splits + split) * D;
+      const size_t ps = qh * p.n_splits_total + p.split_base + split;
+      float* po = p.part_o + ps * D;
 #pragma unroll
       for (int n = 0; n < NBLK; ++n)
         *reinterpret_cast<float2*>(po + 8 * n + 2 * c) = make_float2(acc[n][2 * rr], acc[n][2 * rr + 1]);
       if (c == 0) {
-        p.part_ml[(qh * p.n_splits + split) * 2 + 0] = m_run[rr];
-        p.part_ml[(qh * p.n_splits + split) * 2 + 1] = l_run[rr];
+        p.part_ml[ps * 2 + 0] = m_run[rr];
+        p.part_ml[ps * 2 + 1] = l_run[rr];
       }
     }
   }
@@ -681,9 +688,15 @@ size_t attend_workspace(const msa_dims& d, int B, int M, int k, int t_loc_max, i
   const int mt = tokens_per_cta(d, M);
   const int n_tg = (M + mt - 1) / mt;
   w.n_splits = choose_splits(B * n_tg, t_loc_max, k);
+  // the two-phase call: at least 64 local keys and about 32 selected-chunk keys per split
+  // (the selection's size is known only on the device), about two waves each
+  const int waves2 = std::max(1, (2 * sm_count() + B * n_tg - 1) / (B * n_tg));
+  w.n_split_local = std::max(1, std::min({waves2, (t_loc_max + 63) / 64, kMaxSplits / 2}));
+  w.n_split_chunk = std::max(1, std::min({waves2, 2 * k, kMaxSplits / 2}));
+  w.n_parts = std::max(w.n_splits, w.n_split_local + w.n_split_chunk);
   w.rope_tab = cv.take<float2>((size_t)std::max(1, t_loc_max) * (d.head_dim / 2));
-  w.part_ml = cv.take<float>((size_t)B * M * d.n_q * w.n_splits * 2);
-  w.part_o = cv.take<float>((size_t)B * M * d.n_q * w.n_splits * d.head_dim);
+  w.part_ml = cv.take<float>((size_t)B * M * d.n_q * w.n_parts * 2);
+  w.part_o = cv.take<float>((size_t)B * M * d.n_q * w.n_parts * d.head_dim);
   if (out) *out = w;
   return cv.size();
 }
@@ -756,13 +769,14 @@ msa_status kv_append_launch(const msa_dims& d, const void* k_new, const void* v_
 msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const void* K_bar, const void* V_bar,
                          const int32_t* chunk_off, int n_docs, const int32_t* topk_idx, int k, const void* K_loc,
                          const void* V_loc, const int32_t* loc_len, int t_loc_max, int pos_offset,
-                         const void* rope_cache, int k_loc_rotated, float scale, void* out, void* ws,
+                         const void* rope_cache, int k_loc_rotated, float scale, int phase, void* out, void* ws,
                          cudaStream_t s) {
   AttendWs w;
   attend_workspace(d, B, M, k, t_loc_max, pos_offset, ws, &w);
   const int D = d.head_dim;
-  const float2* tab = k_loc_rotated ? nullptr : static_cast<const float2*>(rope_cache);
-  if (!tab && !k_loc_rotated && t_loc_max > 0) {
+  const bool local_keys = phase != 2;
+  const float2* tab = (k_loc_rotated || !local_keys) ? nullptr : static_cast<const float2*>(rope_cache);
+  if (!tab && !k_loc_rotated && local_keys && t_loc_max > 0) {
     msa_status st = rope_cache_build(d, t_loc_max, pos_offset, w.rope_tab, s);
     if (st != MSA_OK) return st;
     tab = w.rope_tab;
@@ -785,7 +799,10 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
   p.n_docs = n_docs;
   p.t_loc_max = t_loc_max;
   p.pos_offset = pos_offset;
-  p.n_splits = w.n_splits;
+  p.phase = phase;
+  p.n_splits = phase == 0 ? w.n_splits : phase == 1 ? w.n_split_local : w.n_split_chunk;
+  p.split_base = phase == 2 ? w.n_split_local : 0;
+  p.n_splits_total = phase == 0 ? w.n_splits : w.n_split_local + w.n_split_chunk;
   p.q_tokens = M;
   p.tok_per_cta = tokens_per_cta(d, M);
   p.n_tgroups = (M + p.tok_per_cta - 1) / p.tok_per_cta;
@@ -794,7 +811,7 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
   p.n_stages = stages_that_fit(d.n_kv, d.n_q, D, tab != nullptr, p.tok_per_cta);
   {
     TraceScope ts(kKAttnSplit, s);
-    dim3 grid(w.n_splits, B * p.n_tgroups);
+    dim3 grid(p.n_splits, B * p.n_tgroups);
     const size_t sm = AttnSmem(d.n_kv, D, p.n_stages, tab != nullptr).total(d.n_q, D, p.tok_per_cta);
     if (D == 128) {
       MSA_CUDA_CHECK(cudaFuncSetAttribute(attn_split_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
@@ -804,16 +821,16 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
       MSA_CUDA_CHECK(launch_pdl(attn_split_kernel<64>, grid, dim3(32 * (d.n_kv + 1)), sm, s, p));
     }
   }
-  {
+  if (phase != 1) {  // the local-keys phase leaves its partials for the selected-chunks phase's combine
     TraceScope ts(kKAttnCombine, s);
     dim3 grid(d.n_q, B * M);
     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
     if (D == 128)
       MSA_CUDA_CHECK(launch_pdl(attn_combine_kernel<128>, grid, dim3(256), 0, s, (const float*)w.part_ml,
-                                (const float*)w.part_o, w.n_splits, o));
+                                (const float*)w.part_o, p.n_splits_total, o));
     else
       MSA_CUDA_CHECK(launch_pdl(attn_combine_kernel<64>, grid, dim3(256), 0, s, (const float*)w.part_ml,
-                                (const float*)w.part_o, w.n_splits, o));
+                                (const float*)w.part_o, p.n_splits_total, o));
   }
   return MSA_OK;
 }

@@ -54,14 +54,17 @@ struct AuxParams {
 };
 
 // shared memory: ring [kAuxStages][kAuxRows][n_r * DR] bf16 | cos, |k| [NK][8] fp32 | g [NK] |
-// dq partials [kAuxCompute][n_r * DR] fp32 | barriers
+// per compute warp a slice of kSlice floats (its dK row staged for coalesced stores, then its
+// dQ partial) | barriers
 template <int DR>
 struct AuxSmem {
   static constexpr int kRowBytes = 8 * DR * 2;  // room for 8 router heads
   static constexpr int kStageBytes = kAuxRows * kRowBytes;
+  static constexpr int kLanePad = DR / 4 + 4;   // a lane's DR/4 values + 4 floats of padding
+  static constexpr int kSlice = 32 * kLanePad;  // >= 8 * DR
   static __host__ __device__ size_t bytes(int nk) {
     return (size_t)kAuxStages * kStageBytes + (size_t)nk * 8 * 4 * 2 + (size_t)nk * 4 +
-           (size_t)kAuxCompute * 8 * DR * 4 + 2 * kAuxStages * 8 + 16;
+           (size_t)kAuxCompute * kSlice * 4 + 2 * kAuxStages * 8 + 16;
   }
 };
 
@@ -76,20 +79,6 @@ __device__ __forceinline__ int unit_of_slot(int e, int lane) {
   return (e + lane / (8 / U)) % U;
 }
 
-template <int DR>
-__device__ __forceinline__ void load_row_quarter(const uint8_t* row, int lane, float* v) {
-  constexpr int U = DR / 32;  // 16-byte units per lane (4 or 2)
-  const uint8_t* base = row + lane * U * 16;
-#pragma unroll
-  for (int e = 0; e < U; ++e) {
-    const uint4 w = *reinterpret_cast<const uint4*>(base + unit_of_slot<DR>(e, lane) * 16);
-    float2 f;
-    f = unpack_bf16x2(w.x); v[8 * e + 0] = f.x; v[8 * e + 1] = f.y;
-    f = unpack_bf16x2(w.y); v[8 * e + 2] = f.x; v[8 * e + 3] = f.y;
-    f = unpack_bf16x2(w.z); v[8 * e + 4] = f.x; v[8 * e + 5] = f.y;
-    f = unpack_bf16x2(w.w); v[8 * e + 6] = f.x; v[8 * e + 7] = f.y;
-  }
-}
 
 __device__ __forceinline__ void aux_bar_sync() { named_bar_sync(1, 32 * kAuxCompute); }
 
@@ -103,9 +92,10 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
   float* cosv = reinterpret_cast<float*>(aux_sm + kAuxStages * Sm::kStageBytes);  // [NK][8]
   float* nkv = cosv + (size_t)NK * 8;                                            // [NK][8]
   float* gs = nkv + (size_t)NK * 8;                                              // [NK]
-  float* red = gs + NK;                                                          // [kAuxCompute][8 * DR]
+  float* red = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(gs + NK) + 15) & ~uintptr_t(15));
+  // red: [kAuxCompute][Sm::kSlice]
   uint64_t* full = reinterpret_cast<uint64_t*>(
-      (reinterpret_cast<uintptr_t>(red + (size_t)kAuxCompute * 8 * DR) + 7) & ~uintptr_t(7));
+      (reinterpret_cast<uintptr_t>(red + (size_t)kAuxCompute * Sm::kSlice) + 7) & ~uintptr_t(7));
   uint64_t* empty = full + kAuxStages;
   __shared__ float qn[8];      // clamped query norms (negative: below eps)
   __shared__ float chead[8];   // sum_j g_j cos_jh
@@ -162,7 +152,7 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
   const float inv_p = 1.0f / (float)p.P;
   int it = 0;
   for (int i = blockIdx.x; i < p.P; i += gridDim.x) {
-    // this lane's query values (rotated unit order as in load_row_quarter) and the head norms
+    // this lane's query values (in slot order, see unit_of_slot) and the head norms
     float q[V];
     {
       const uint16_t* qrow = reinterpret_cast<const uint16_t*>(p.Q + (size_t)i * NR);
@@ -187,15 +177,28 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
       const int st = it % kAuxStages;
       mbar_wait(&full[st], (it / kAuxStages) & 1);
       const int j = c * kAuxRows + warp;
+      uint4 kw[DR / 32];
+      if (j < NK && hl) {
+        const uint8_t* base = ring + (size_t)st * Sm::kStageBytes + (size_t)warp * row_bytes + lane * (DR / 32) * 16;
+#pragma unroll
+        for (int e = 0; e < DR / 32; ++e) kw[e] = *reinterpret_cast<const uint4*>(base + unit_of_slot<DR>(e, lane) * 16);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);  // the row is in registers: the stage may refill
       if (j < NK) {
-        float kv[V];
         float dot = 0.f, kk = 0.f;
         if (hl) {
-          load_row_quarter<DR>(ring + (size_t)st * Sm::kStageBytes + (size_t)warp * row_bytes, lane, kv);
 #pragma unroll
-          for (int e = 0; e < V; ++e) {
-            dot = fmaf(kv[e], q[e], dot);
-            kk = fmaf(kv[e], kv[e], kk);
+          for (int e = 0; e < DR / 32; ++e) {
+            const uint32_t wv[4] = {kw[e].x, kw[e].y, kw[e].z, kw[e].w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              const float2 f = unpack_bf16x2(wv[t]);
+              dot = fmaf(f.x, q[8 * e + 2 * t], dot);
+              dot = fmaf(f.y, q[8 * e + 2 * t + 1], dot);
+              kk = fmaf(f.x, f.x, kk);
+              kk = fmaf(f.y, f.y, kk);
+            }
           }
         }
         dot += __shfl_xor_sync(0xffffffffu, dot, 1);
@@ -208,8 +211,6 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
           nkv[(size_t)j * 8 + h] = nk > kAuxEps ? nk : -kAuxEps;
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);
     }
     aux_bar_sync();
 
@@ -258,50 +259,75 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
       if (lane == 0) chead[warp] = cc;
     }
 
-    // ---- pass 2: gradients (the rows again, from L2) ----
+    // ---- pass 2: gradients (the rows again, from L2), one 16-byte unit of the row at a time ----
     float acc[V];
 #pragma unroll
     for (int e = 0; e < V; ++e) acc[e] = 0.f;
     const float nq = hl ? fabsf(qn[h]) : 1.f;
+    float* slice = red + (size_t)warp * Sm::kSlice;
     for (int c = 0; c < n_ch; ++c, ++it) {
       const int st = it % kAuxStages;
       mbar_wait(&full[st], (it / kAuxStages) & 1);
       const int j = c * kAuxRows + warp;
+      uint4 kw[DR / 32];
       if (j < NK && hl) {
-        float kv[V];
-        load_row_quarter<DR>(ring + (size_t)st * Sm::kStageBytes + (size_t)warp * row_bytes, lane, kv);
+        const uint8_t* base = ring + (size_t)st * Sm::kStageBytes + (size_t)warp * row_bytes + lane * (DR / 32) * 16;
+#pragma unroll
+        for (int e = 0; e < DR / 32; ++e) kw[e] = *reinterpret_cast<const uint4*>(base + unit_of_slot<DR>(e, lane) * 16);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);  // the row is in registers: the stage may refill
+      float* dk = nullptr;
+      if (j < NK) dk = j == 0 ? (p.dK_pos ? p.dK_pos + (size_t)i * NR : nullptr)
+                              : (p.dK_neg ? p.dK_neg + ((size_t)i * p.N + (j - 1)) * NR : nullptr);
+      if (j < NK && hl) {
         const float nks = nkv[(size_t)j * 8 + h], nk = fabsf(nks);
         const float g = gs[j] * inv_nr;
         const float a = g / (nq * nk);  // coefficient of k in dL/dq and of q in dL/dk
+        const float b = nks > 0.f ? g * cosv[(size_t)j * 8 + h] / (nk * nk) : 0.f;
 #pragma unroll
-        for (int e = 0; e < V; ++e) acc[e] = fmaf(a, kv[e], acc[e]);
-        float* dk = j == 0 ? (p.dK_pos ? p.dK_pos + (size_t)i * NR : nullptr)
-                           : (p.dK_neg ? p.dK_neg + ((size_t)i * p.N + (j - 1)) * NR : nullptr);
-        if (dk) {
-          const float b = nks > 0.f ? g * cosv[(size_t)j * 8 + h] / (nk * nk) : 0.f;
+        for (int e = 0; e < DR / 32; ++e) {
+          float kv[8];
+          float2 f;
+          f = unpack_bf16x2(kw[e].x); kv[0] = f.x; kv[1] = f.y;
+          f = unpack_bf16x2(kw[e].y); kv[2] = f.x; kv[3] = f.y;
+          f = unpack_bf16x2(kw[e].z); kv[4] = f.x; kv[5] = f.y;
+          f = unpack_bf16x2(kw[e].w); kv[6] = f.x; kv[7] = f.y;
 #pragma unroll
-          for (int e = 0; e < V / 4; ++e) {
-            float4* d4 = reinterpret_cast<float4*>(dk + lane * V + unit_of_slot<DR>(e / 2, lane) * 8 + (e % 2) * 4);
-            *d4 = make_float4(a * q[4 * e + 0] - b * kv[4 * e + 0], a * q[4 * e + 1] - b * kv[4 * e + 1],
-                              a * q[4 * e + 2] - b * kv[4 * e + 2], a * q[4 * e + 3] - b * kv[4 * e + 3]);
+          for (int t = 0; t < 8; ++t) acc[8 * e + t] = fmaf(a, kv[t], acc[8 * e + t]);
+          if (dk) {
+            // staged in this warp's slice (lane rows padded: no bank conflicts)
+            float* s8 = slice + lane * Sm::kLanePad + unit_of_slot<DR>(e, lane) * 8;
+            *reinterpret_cast<float4*>(s8) =
+                make_float4(a * q[8 * e + 0] - b * kv[0], a * q[8 * e + 1] - b * kv[1], a * q[8 * e + 2] - b * kv[2],
+                            a * q[8 * e + 3] - b * kv[3]);
+            *reinterpret_cast<float4*>(s8 + 4) =
+                make_float4(a * q[8 * e + 4] - b * kv[4], a * q[8 * e + 5] - b * kv[5], a * q[8 * e + 6] - b * kv[6],
+                            a * q[8 * e + 7] - b * kv[7]);
           }
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);
+      if (dk) {  // consecutive lanes store consecutive 16-byte pieces: whole 512-byte segments
+        for (int i4 = lane; i4 < NR / 4; i4 += 32) {
+          const int e0 = i4 * 4;
+          *reinterpret_cast<float4*>(dk + e0) = *reinterpret_cast<const float4*>(slice + (e0 / V) * Sm::kLanePad + e0 % V);
+        }
+      }
+      __syncwarp();  // the slice is read before the next row is staged
     }
     if (p.dQ != nullptr) {
       if (hl) {
 #pragma unroll
         for (int e = 0; e < V; ++e)
-          red[(size_t)warp * 8 * DR + lane * V + unit_of_slot<DR>(e / 8, lane) * 8 + e % 8] = acc[e];
+          red[(size_t)warp * Sm::kSlice + lane * V + unit_of_slot<DR>(e / 8, lane) * 8 + e % 8] = acc[e];
       }
       aux_bar_sync();
       for (int e = ct; e < NR; e += 32 * kAuxCompute) {
         const int hh = e / DR;
         float v = 0.f;
 #pragma unroll
-        for (int w = 0; w < kAuxCompute; ++w) v += red[(size_t)w * 8 * DR + e];
+        for (int w = 0; w < kAuxCompute; ++w) v += red[(size_t)w * Sm::kSlice + e];
         const float nqs = qn[hh], nqa = fabsf(nqs);
         if (nqs > 0.f) {
           const float qe = bf16_bits_to_float(__ldg(reinterpret_cast<const uint16_t*>(p.Q) + (size_t)i * NR + e));

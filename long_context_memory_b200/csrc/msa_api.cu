@@ -340,7 +340,7 @@ msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, int
                              const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks, const int32_t* topk_idx,
                              int32_t k, const void* K_loc, const void* V_loc, const int32_t* loc_len,
                              int32_t t_loc_max, int32_t pos_offset, const void* rope_cache,
-                             int32_t k_loc_rotated, float softmax_scale, void* out, void* ws,
+                             int32_t k_loc_rotated, float softmax_scale, int32_t phase, void* out, void* ws,
                              size_t ws_bytes, void* stream) {
   msa_status st = check_dims(dims, true, false);
   if (st != MSA_OK) return st;
@@ -356,25 +356,28 @@ msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, int
     return fail(MSA_ERR_INVALID_ARG, "positions must lie in [0, 2^24)");
   if (!(softmax_scale >= 0.f) || !std::isfinite(softmax_scale))
     return fail(MSA_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+  if (phase < 0 || phase > 2) return fail(MSA_ERR_INVALID_ARG, "phase must be 0, 1 or 2 (got %d)", phase);
   CHECK_PTR(q);
-  CHECK_PTR(K_bar);
-  CHECK_PTR(V_bar);
-  CHECK_PTR(chunk_off);
-  CHECK_PTR(topk_idx);
-  if (t_loc_max > 0) {
+  if (phase != 1) {  // the selected chunks
+    CHECK_PTR(K_bar);
+    CHECK_PTR(V_bar);
+    CHECK_PTR(chunk_off);
+    CHECK_PTR(topk_idx);
+    CHECK_PTR(out);
+  }
+  if (phase != 2 && t_loc_max > 0) {  // the local keys
     CHECK_PTR(K_loc);
     CHECK_PTR(V_loc);
   }
   CHECK_PTR(loc_len);
   CHECK_OPT_PTR(rope_cache);
-  CHECK_PTR(out);
   const size_t need = attend_workspace(*dims, B, q_tokens, k, t_loc_max, pos_offset, nullptr, nullptr);
   if (ws_bytes < need) return fail(MSA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
   if (need && (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)))
     return fail(MSA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
   if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
   return attend_launch(*dims, q, B, q_tokens, K_bar, V_bar, chunk_off, n_docs, topk_idx, k, K_loc, V_loc, loc_len, t_loc_max,
-                       pos_offset, rope_cache, k_loc_rotated, softmax_scale, out, ws,
+                       pos_offset, rope_cache, k_loc_rotated, softmax_scale, phase, out, ws,
                        static_cast<cudaStream_t>(stream));
 }
 

@@ -108,13 +108,14 @@ def test_route_fault_injection_before_launch(msa, monkeypatch):
     assert "injected" in msa.lib.msa_last_error().decode()
 
 
-def _attend(msa, dims, B=1, k=2, n_docs=4, n_chunks=8, t_loc=16, pos=2, scale=0.0, ws_bytes=None, q=FAKE, M=1):
+def _attend(msa, dims, B=1, k=2, n_docs=4, n_chunks=8, t_loc=16, pos=2, scale=0.0, ws_bytes=None, q=FAKE, M=1,
+            phase=0):
     dd = msa.Dims.of(dims)
     need = msa.lib.msa_attend_workspace_size(ctypes.byref(dd), B, max(M, 1), k, t_loc, pos)
     if ws_bytes is None:
         ws_bytes = need
     return msa.lib.msa_sparse_attend(ctypes.byref(dd), q, B, M, FAKE, FAKE, FAKE, n_docs, n_chunks, FAKE, k, FAKE, FAKE,
-                                     FAKE, t_loc, pos, None, 0, scale, FAKE, 0x100000, ws_bytes, None)
+                                     FAKE, t_loc, pos, None, 0, scale, phase, FAKE, 0x100000, ws_bytes, None)
 
 
 def test_attend_validation(msa):
@@ -129,6 +130,7 @@ def test_attend_validation(msa):
     assert _attend(msa, ok, q=FAKE + 2) == 1
     assert _attend(msa, ok, ws_bytes=8) == 3
     assert _attend(msa, ok, M=0) == 1
+    assert _attend(msa, ok, phase=3) == 1
 
 
 def test_encode_validation(msa):

@@ -287,3 +287,39 @@ def test_kv_append_matches_rotation_and_copy(msa, cuda_device):
         msa.check_device_errors()
     assert msa.check_device_errors() == 0   # reading the word clears it
     assert torch.equal(K[0], K1[0]) and torch.equal(K[2], K1[2])
+
+
+@pytest.mark.parametrize("rotated,M,B", [(True, 1, 1), (False, 1, 3), (True, 4, 2), (False, 3, 5)])
+def test_attend_two_phase_equals_one_call(msa, cuda_device, rotated, M, B):
+    # phase 1 (local keys) then phase 2 (selected chunks + merge) on one workspace
+    import torch
+
+    rng = np.random.default_rng(90 + M + B)
+    n_q, n_kv, D = 32, 8, 128
+    c = _case(91 + M + B, B, n_q, n_kv, D, n_docs=30, k=6, t_loc=200, loc_len=rng.integers(M, 201, size=B))
+    c["q"] = W.normal_bf16(rng, (B, M, n_q, D)) if M > 1 else c["q"]
+    dims = W.Dims(hidden=256, n_q=n_q, n_kv=n_kv, head_dim=D, n_r=4, d_r=64, rope_base=1e6)
+    dev = cuda_device
+    co, C = msa.chunk_offsets(c["doc_off"])
+    K_loc = _dev(c["K_loc"], dev)
+    if rotated:
+        pos = (5 + torch.arange(200, dtype=torch.int32, device=dev)).repeat(B)
+        msa.rope_rows(dims, K_loc.view(B * 200, n_kv, D), pos)
+    args = (dims, _dev(c["q"], dev), _dev(c["K_bar"], dev), _dev(c["V_bar"], dev), torch.from_numpy(co).to(dev),
+            torch.from_numpy(c["topk"].astype(np.int32)).to(dev), K_loc, _dev(c["V_loc"], dev),
+            torch.from_numpy(c["loc_len"].astype(np.int32)).to(dev), 5)
+    one = msa.sparse_attend(*args, k_loc_rotated=rotated)
+    ws = torch.empty(msa.attend_workspace_size(dims, B, 6, 200, 5, M) + 256, dtype=torch.uint8, device=dev)
+    out = torch.zeros_like(one)
+    msa.sparse_attend(*args, k_loc_rotated=rotated, phase=1, ws=ws, out=out)
+    msa.sparse_attend(*args, k_loc_rotated=rotated, phase=2, ws=ws, out=out)
+    torch.cuda.synchronize()
+    assert msa.check_device_errors() == 0
+    a, b = one.float().cpu().numpy(), out.float().cpu().numpy()
+    assert np.max(np.abs(a - b)) < 2e-2
+    if M == 1:
+        check_attention(b, _oracle(c, 5, 1e6), where=f"two-phase B={B}")
+    else:
+        ref = O.sparse_attend_tokens(c["q"], c["K_bar"], c["V_bar"], c["chunk_off"], c["topk"], c["K_loc"], c["V_loc"],
+                                     c["loc_len"], 5, 1e6)
+        check_attention(b, ref, where=f"two-phase M={M}")
