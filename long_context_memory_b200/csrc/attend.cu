@@ -158,9 +158,10 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
     seg_c[r] = c0;
     seg_v[r + 1] = n;
   }
-  {
+  {  // all of the query's 16-byte pieces in flight at once (waited for before the barrier below)
     const uint4* qg = reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.q_tokens + t0) * p.n_q * D);
-    for (int i = tid; i < nt * p.n_q * D / 8; i += blockDim.x) reinterpret_cast<uint4*>(qsm)[i] = __ldg(qg + i);
+    for (int i = tid; i < nt * p.n_q * D / 8; i += blockDim.x) cp_async16(reinterpret_cast<uint4*>(qsm) + i, qg + i);
+    cp_async_wait_all();
   }
   int L = p.loc_len[b];
   L = max(0, min(L, p.t_loc_max));

@@ -62,9 +62,10 @@ struct AuxSmem {
   static constexpr int kStageBytes = kAuxRows * kRowBytes;
   static constexpr int kLanePad = DR / 4 + 4;   // a lane's DR/4 values + 4 floats of padding
   static constexpr int kSlice = 32 * kLanePad;  // >= 8 * DR
+  static constexpr int kQBytes = 8 * DR * 2;    // one query row (room for 8 router heads)
   static __host__ __device__ size_t bytes(int nk) {
-    return (size_t)kAuxStages * kStageBytes + (size_t)nk * 8 * 4 * 2 + (size_t)nk * 4 +
-           (size_t)kAuxCompute * kSlice * 4 + 2 * kAuxStages * 8 + 16;
+    return (size_t)kAuxStages * kStageBytes + 2 * kQBytes + (size_t)nk * 8 * 4 * 2 + (size_t)nk * 4 + 16 +
+           (size_t)kAuxCompute * kSlice * 4 + (2 * kAuxStages + 4) * 8 + 16;
   }
 };
 
@@ -89,7 +90,8 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
   extern __shared__ __align__(128) uint8_t aux_sm[];
   const int n_r = p.n_r, NK = p.N + 1, NR = n_r * DR;
   uint8_t* ring = aux_sm;
-  float* cosv = reinterpret_cast<float*>(aux_sm + kAuxStages * Sm::kStageBytes);  // [NK][8]
+  uint8_t* qbuf = aux_sm + kAuxStages * Sm::kStageBytes;                          // [2][n_r * DR] bf16
+  float* cosv = reinterpret_cast<float*>(qbuf + 2 * Sm::kQBytes);                 // [NK][8]
   float* nkv = cosv + (size_t)NK * 8;                                            // [NK][8]
   float* gs = nkv + (size_t)NK * 8;                                              // [NK]
   float* red = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(gs + NK) + 15) & ~uintptr_t(15));
@@ -97,6 +99,8 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
   uint64_t* full = reinterpret_cast<uint64_t*>(
       (reinterpret_cast<uintptr_t>(red + (size_t)kAuxCompute * Sm::kSlice) + 7) & ~uintptr_t(7));
   uint64_t* empty = full + kAuxStages;
+  uint64_t* qfull = empty + kAuxStages;  // [2] a positive's query row landed
+  uint64_t* qempty = qfull + 2;          // [2] every compute warp is done with it
   __shared__ float qn[8];      // clamped query norms (negative: below eps)
   __shared__ float chead[8];   // sum_j g_j cos_jh
   __shared__ float wred[kAuxCompute];
@@ -112,6 +116,10 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kAuxCompute);
     }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&qfull[s], 1);
+      mbar_init(&qempty[s], kAuxCompute);
+    }
     fence_mbar_init();
   }
   __syncthreads();
@@ -121,8 +129,14 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
   if (warp == kAuxCompute) {
     // ------------------------- producer -------------------------
     if (lane == 0) {
-      int it = 0;
-      for (int i = blockIdx.x; i < p.P; i += gridDim.x) {
+      int it = 0, pi = 0;
+      for (int i = blockIdx.x; i < p.P; i += gridDim.x, ++pi) {
+        {  // the positive's query row (double-buffered)
+          const int qb = pi & 1;
+          if (pi >= 2) mbar_wait(&qempty[qb], ((pi >> 1) - 1) & 1);
+          mbar_arrive_expect_tx(&qfull[qb], (uint32_t)row_bytes);
+          bulk_load(qbuf + qb * Sm::kQBytes, p.Q + (size_t)i * NR, (uint32_t)row_bytes, &qfull[qb]);
+        }
         for (int pass = 0; pass < passes; ++pass) {
           for (int c = 0; c < n_ch; ++c, ++it) {
             const int st = it % kAuxStages;
@@ -150,15 +164,26 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
   const bool hl = h < n_r;
   const float inv_nr = 1.0f / (float)n_r;
   const float inv_p = 1.0f / (float)p.P;
-  int it = 0;
-  for (int i = blockIdx.x; i < p.P; i += gridDim.x) {
+  int it = 0, pi = 0;
+  for (int i = blockIdx.x; i < p.P; i += gridDim.x, ++pi) {
     // this lane's query values (in slot order, see unit_of_slot) and the head norms
+    const int qb = pi & 1;
+    const uint16_t* qrow = reinterpret_cast<const uint16_t*>(qbuf + qb * Sm::kQBytes);
     float q[V];
     {
-      const uint16_t* qrow = reinterpret_cast<const uint16_t*>(p.Q + (size_t)i * NR);
+      mbar_wait(&qfull[qb], (pi >> 1) & 1);
 #pragma unroll
-      for (int e = 0; e < V; ++e)
-        q[e] = hl ? bf16_bits_to_float(__ldg(qrow + lane * V + unit_of_slot<DR>(e / 8, lane) * 8 + e % 8)) : 0.f;
+      for (int e = 0; e < DR / 32; ++e) {
+        uint4 w = make_uint4(0, 0, 0, 0);
+        if (hl) w = *reinterpret_cast<const uint4*>(qrow + lane * V + unit_of_slot<DR>(e, lane) * 8);
+        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float2 f = unpack_bf16x2(wv[t]);
+          q[8 * e + 2 * t] = f.x;
+          q[8 * e + 2 * t + 1] = f.y;
+        }
+      }
       float ss = 0.f;
 #pragma unroll
       for (int e = 0; e < V; ++e) ss = fmaf(q[e], q[e], ss);
@@ -188,18 +213,21 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
       if (j < NK) {
         float dot = 0.f, kk = 0.f;
         if (hl) {
+          float d4[4] = {0.f, 0.f, 0.f, 0.f}, k4[4] = {0.f, 0.f, 0.f, 0.f};  // independent chains
 #pragma unroll
           for (int e = 0; e < DR / 32; ++e) {
             const uint32_t wv[4] = {kw[e].x, kw[e].y, kw[e].z, kw[e].w};
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
               const float2 f = unpack_bf16x2(wv[t]);
-              dot = fmaf(f.x, q[8 * e + 2 * t], dot);
-              dot = fmaf(f.y, q[8 * e + 2 * t + 1], dot);
-              kk = fmaf(f.x, f.x, kk);
-              kk = fmaf(f.y, f.y, kk);
+              d4[t] = fmaf(f.x, q[8 * e + 2 * t], d4[t]);
+              d4[t] = fmaf(f.y, q[8 * e + 2 * t + 1], d4[t]);
+              k4[t] = fmaf(f.x, f.x, k4[t]);
+              k4[t] = fmaf(f.y, f.y, k4[t]);
             }
           }
+          dot = (d4[0] + d4[1]) + (d4[2] + d4[3]);
+          kk = (k4[0] + k4[1]) + (k4[2] + k4[3]);
         }
         dot += __shfl_xor_sync(0xffffffffu, dot, 1);
         kk += __shfl_xor_sync(0xffffffffu, kk, 1);
@@ -250,7 +278,11 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
       gs[j] = j == 0 ? -se_neg * scale : expf(gs[j] - zmax) * scale;  // dL/ds_j
     if (ct == 0) p.term[i] = (zmax - z0) + log1pf((e0 - 1.0f) + se_neg);  // -log p_0
     aux_bar_sync();
-    if (!grads) continue;
+    if (!grads) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&qempty[qb]);  // the query buffer may take the positive after next
+      continue;
+    }
     if (warp < n_r) {  // c_h = sum_j g_j cos_jh
       float cc = 0.f;
       for (int j = lane; j < NK; j += 32) cc = fmaf(gs[j], cosv[(size_t)j * 8 + warp], cc);
@@ -329,13 +361,12 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
 #pragma unroll
         for (int w = 0; w < kAuxCompute; ++w) v += red[(size_t)w * Sm::kSlice + e];
         const float nqs = qn[hh], nqa = fabsf(nqs);
-        if (nqs > 0.f) {
-          const float qe = bf16_bits_to_float(__ldg(reinterpret_cast<const uint16_t*>(p.Q) + (size_t)i * NR + e));
-          v -= chead[hh] * inv_nr * qe / (nqa * nqa);
-        }
+        if (nqs > 0.f) v -= chead[hh] * inv_nr * bf16_bits_to_float(qrow[e]) / (nqa * nqa);
         p.dQ[(size_t)i * NR + e] = v;
       }
     }
+    aux_bar_sync();  // every warp is done with the query row
+    if (lane == 0) mbar_arrive(&qempty[qb]);  // the query buffer may take the positive after next
   }
 
   // ---- loss: the last CTA sums the terms in positive order ----

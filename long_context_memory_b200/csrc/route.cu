@@ -128,19 +128,22 @@ __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
     for (int p0 = 0; p0 < nrows; p0 += kRqPiece) {
       const int pr = min(kRqPiece, nrows - p0);
       __syncthreads();  // the previous piece is consumed
+      // every 16-byte piece of the W piece and of the query rows in flight at once
       const __nv_bfloat16* wsrc = W + (size_t)(k0 + p0) * NR + h * d_r;
       for (int i = tid; i < pr * per_row; i += kRqThreads) {
         const int r = i / per_row, c = i % per_row;
-        *reinterpret_cast<uint4*>(wsm + (size_t)r * ws + c * 16) =
-            __ldg(reinterpret_cast<const uint4*>(wsrc + (size_t)r * NR) + c);
+        cp_async16(wsm + (size_t)r * ws + c * 16, reinterpret_cast<const uint4*>(wsrc + (size_t)r * NR) + c);
       }
       const int vec = pr / 8;
       for (int i = tid; i < 16 * vec; i += kRqThreads) {
         const int j = i / vec, v = i % vec;
-        uint4 x = make_uint4(0, 0, 0, 0);
-        if (b0 + j < B) x = __ldg(reinterpret_cast<const uint4*>(hq + (size_t)(b0 + j) * hidden + k0 + p0) + v);
-        *reinterpret_cast<uint4*>(hsm + (size_t)j * hstr + v * 16) = x;
+        if (b0 + j < B)
+          cp_async16(hsm + (size_t)j * hstr + v * 16,
+                     reinterpret_cast<const uint4*>(hq + (size_t)(b0 + j) * hidden + k0 + p0) + v);
+        else
+          *reinterpret_cast<uint4*>(hsm + (size_t)j * hstr + v * 16) = make_uint4(0, 0, 0, 0);
       }
+      cp_async_wait_all();
       __syncthreads();
       for (int ks = 0; ks < pr / 16; ++ks) {
         uint32_t a0, a1, a2, a3;
