@@ -72,6 +72,7 @@ struct AttnParams {
   float* part_ml;
   float* part_o;
   int n_q, n_kv, k, n_docs, t_loc_max, pos_offset, n_splits, n_stages;
+  int n_queries;     // B
   int q_tokens;      // M: query tokens per query (the last M local tokens)
   int phase;         // 0: every key; 1: the local keys only; 2: the selected chunks only
   int split_base;    // this launch's first split id in the partial arrays
@@ -96,8 +97,11 @@ struct AttnSmem {
     stage_bytes = 2 * kbytes + tbytes;
     n_stages = stages;
   }
+  // two query buffers, barriers (ring, item header), two item headers and segment tables, the
+  // tokens' cos/sin
   __host__ __device__ size_t fixed_bytes(int n_q, int D, int mt) const {
-    return 2 * kMaxStages * 8 + (2 * kMaxK + 2) * 4 + (size_t)mt * (D / 2) * 8 + (size_t)mt * n_q * D * 2;
+    return 2 * (size_t)mt * n_q * D * 2 + (2 * kMaxStages + 4) * 8 + 2 * 8 * 4 + 2 * (2 * kMaxK + 2) * 4 +
+           (size_t)mt * (D / 2) * 8;
   }
   __host__ __device__ size_t total(int n_q, int D, int mt) const {
     return (size_t)n_stages * stage_bytes + fixed_bytes(n_q, D, mt);
@@ -116,21 +120,22 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
   // the RoPE rows are bulk-copy or 16-byte vector destinations)
   uint8_t* stage_mem = sm;
   const int MT = p.tok_per_cta;
-  uint16_t* qsm = reinterpret_cast<uint16_t*>(sm + (size_t)L_.n_stages * L_.stage_bytes);  // [MT][n_q][D] raw query
-  uint64_t* bars = reinterpret_cast<uint64_t*>(qsm + (size_t)MT * p.n_q * D);  // [stage] tile landed
-  uint64_t* ebars = bars + kMaxStages;                                      // [stage] every warp done with it
-  int* seg_v = reinterpret_cast<int*>(ebars + kMaxStages);  // [k + 1] virtual starts
-  int* seg_c = seg_v + kMaxK + 2;                          // [k] chunk starts
-  float2* qcs = reinterpret_cast<float2*>(seg_c + kMaxK);  // [MT][D/2] cos/sin at the tokens' positions
+  const size_t q_elems = (size_t)MT * p.n_q * D;
+  uint16_t* qsm = reinterpret_cast<uint16_t*>(sm + (size_t)L_.n_stages * L_.stage_bytes);  // [2][MT][n_q][D]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(qsm + 2 * q_elems);  // [stage] tile landed
+  uint64_t* ebars = bars + kMaxStages;                               // [stage] every warp done with it
+  uint64_t* hfull = ebars + kMaxStages;                              // [2] an item's header and query landed
+  uint64_t* hempty = hfull + 2;                                      // [2] every warp done with them
+  int* hdr = reinterpret_cast<int*>(hempty + 2);                     // [2][8] item headers
+  int* segs = hdr + 16;                                              // [2][2 kMaxK + 2] segment tables
+  float2* qcs = reinterpret_cast<float2*>(segs + 2 * (2 * kMaxK + 2));  // [MT][D/2] cos/sin at the tokens' positions
 
-  const int split = blockIdx.x;
-  const int b = blockIdx.y / p.n_tgroups;                       // query
-  const int t0 = (blockIdx.y % p.n_tgroups) * MT;               // first token of this CTA
-  const int nt = min(MT, p.q_tokens - t0);                      // tokens of this CTA
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = warp;               // the KV head this warp serves (warps 0 .. n_kv-1)
-  const bool producer = warp == n_kv;  // the last warp only streams tiles in
+  const bool producer = warp == n_kv;  // the last warp builds each item and streams its tiles
   const int k = p.phase == 1 ? 0 : p.k;  // the local-keys phase has no selected documents
+  // items: (split, query, token group); this CTA takes items blockIdx.x, + gridDim.x, ...
+  const int n_items = p.n_splits * p.n_queries * p.n_tgroups;
 
   // ---- no global memory yet: overlaps the previous kernel's tail ----
   for (int i = tid; i < L_.n_stages * L_.stage_bytes / 16; i += blockDim.x)
@@ -140,296 +145,329 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
       mbar_init(&bars[s], 1);
       mbar_init(&ebars[s], n_kv);
     }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&hfull[s], 1);
+      mbar_init(&hempty[s], n_kv);
+    }
     fence_mbar_init();
   }
+  __syncthreads();
   pdl_launch_dependents();
   pdl_wait();
-
-  // ---- segment table (selected docs in top-k order, then local) and the raw query ----
-  for (int r = tid; r < k; r += blockDim.x) {
-    int doc = p.topk_idx[(size_t)b * k + r];
-    int c0 = 0, n = 0;
-    if (doc >= 0 && doc < p.n_docs) {
-      c0 = __ldg(&p.chunk_off[doc]);
-      n = __ldg(&p.chunk_off[doc + 1]) - c0;
-    } else {
-      raise_dev_error(kDevErrBadIndex);
-    }
-    seg_c[r] = c0;
-    seg_v[r + 1] = n;
-  }
-  {  // all of the query's 16-byte pieces in flight at once (waited for before the barrier below)
-    const uint4* qg = reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.q_tokens + t0) * p.n_q * D);
-    for (int i = tid; i < nt * p.n_q * D / 8; i += blockDim.x) cp_async16(reinterpret_cast<uint4*>(qsm) + i, qg + i);
-    cp_async_wait_all();
-  }
-  int L = p.loc_len[b];
-  L = max(0, min(L, p.t_loc_max));
-  __syncthreads();
-  if (warp == 0) {
-    // inclusive scan of chunk counts -> virtual starts (lane owns a run of entries)
-    const int per = (k + 31) / 32;
-    int local = 0;
-    for (int j = 0; j < per; ++j) {
-      const int r = lane * per + j;
-      if (r < k) local += seg_v[r + 1];
-    }
-    int incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    int run = incl - local;
-    for (int j = 0; j < per; ++j) {
-      const int r = lane * per + j;
-      if (r < k) {
-        run += seg_v[r + 1];
-        seg_v[r + 1] = run;
-      }
-    }
-    if (lane == 0) seg_v[0] = 0;
-  }
-  fence_proxy_async_smem();
-  __syncthreads();
-
-  const int n_sel = seg_v[k];
-  const int n_keys = n_sel + (p.phase == 2 ? 0 : L);
-  int per_split = (n_keys + p.n_splits - 1) / p.n_splits;
-  per_split = (per_split + kTK - 1) / kTK * kTK;
-  const int v0 = min(n_keys, split * per_split);
-  const int v1 = min(n_keys, v0 + per_split);
-  const int n_tiles = (v1 - v0 + kTK - 1) / kTK;
   const int row_bytes = n_kv * D * 2;  // one key, every KV head
 
-  // ---- one tile = kTK keys: a 2-row bulk copy pair per key plus one copy of the RoPE rows ----
-  auto issue = [&](int t, int st) {
-    if (t >= L_.n_stages) mbar_wait(&ebars[st], ((t / L_.n_stages) - 1) & 1);
-    const int tv0 = v0 + t * kTK;
-    const int rows = min(kTK, v1 - tv0);
-    const int n_chunk_rows = max(0, min(rows, n_sel - tv0));
-    const int n_loc_rows = rows - n_chunk_rows;
-    const uint32_t tb = (table && n_loc_rows > 0) ? (uint32_t)(n_loc_rows * (D / 2) * 8) : 0u;
-    if (lane == 0) mbar_arrive_expect_tx(&bars[st], (uint32_t)(2 * rows * row_bytes) + tb);
-    __syncwarp();
-    uint8_t* kdst = stage_mem + (size_t)st * L_.stage_bytes;
-    uint8_t* vdst = kdst + L_.kbytes;
-    if (lane < rows) {
-      const int v = tv0 + lane;
-      const __nv_bfloat16 *ks, *vs;
-      if (v < n_sel) {
-        int lo = 0, hi = k - 1;  // segment with seg_v[lo] <= v < seg_v[lo + 1]
-        while (lo < hi) {
-          const int mid = (lo + hi + 1) >> 1;
-          if (seg_v[mid] <= v) lo = mid; else hi = mid - 1;
-        }
-        const size_t ch = (size_t)(seg_c[lo] + (v - seg_v[lo]));
-        ks = p.K_bar + ch * n_kv * D;
-        vs = p.V_bar + ch * n_kv * D;
-      } else {
-        const size_t off = ((size_t)b * p.t_loc_max + (size_t)(v - n_sel)) * n_kv * D;
-        ks = p.K_loc + off;
-        vs = p.V_loc + off;
-      }
-      bulk_load(kdst + lane * L_.krow, ks, row_bytes, &bars[st]);
-      bulk_load(vdst + lane * L_.krow, vs, row_bytes, &bars[st]);
-    }
-    if (tb && lane == 31) {
-      const int j0 = tv0 + n_chunk_rows - n_sel;
-      bulk_load(vdst + L_.kbytes + n_chunk_rows * (D / 2) * 8, p.rope_tab + (size_t)j0 * (D / 2), tb, &bars[st]);
-    }
-  };
   if (producer) {
-    for (int t = 0; t < n_tiles; ++t) issue(t, t % L_.n_stages);
+    // ---- per item: the segment table (selected docs in top-k order, then local), the header
+    //      and the query rows for the compute warps, then the item's tiles into the ring ----
+    int gt = 0;
+    for (int it = blockIdx.x, j = 0; it < n_items; it += gridDim.x, ++j) {
+      const int hb = j & 1;
+      const int split = it % p.n_splits, bq = it / p.n_splits;
+      const int b = bq / p.n_tgroups, t0 = (bq % p.n_tgroups) * MT;
+      const int nt = min(MT, p.q_tokens - t0);
+      if (j >= 2) mbar_wait(&hempty[hb], ((j >> 1) - 1) & 1);  // item j-2's header and query read
+      int* seg_v = segs + hb * (2 * kMaxK + 2);  // [k + 1] virtual starts
+      int* seg_c = seg_v + kMaxK + 2;            // [k] chunk starts
+      for (int r = lane; r < k; r += 32) {
+        const int doc = p.topk_idx[(size_t)b * k + r];
+        int c0 = 0, n = 0;
+        if (doc >= 0 && doc < p.n_docs) {
+          c0 = __ldg(&p.chunk_off[doc]);
+          n = __ldg(&p.chunk_off[doc + 1]) - c0;
+        } else {
+          raise_dev_error(kDevErrBadIndex);
+        }
+        seg_c[r] = c0;
+        seg_v[r + 1] = n;
+      }
+      int L = p.loc_len[b];
+      L = max(0, min(L, p.t_loc_max));
+      __syncwarp();
+      {  // inclusive scan of chunk counts -> virtual starts (lane owns a run of entries)
+        const int per = (k + 31) / 32;
+        int local = 0;
+        for (int q = 0; q < per; ++q) {
+          const int r = lane * per + q;
+          if (r < k) local += seg_v[r + 1];
+        }
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        int run = incl - local;
+        for (int q = 0; q < per; ++q) {
+          const int r = lane * per + q;
+          if (r < k) {
+            run += seg_v[r + 1];
+            seg_v[r + 1] = run;
+          }
+        }
+        if (lane == 0) seg_v[0] = 0;
+      }
+      __syncwarp();
+      const int n_sel = seg_v[k];
+      const int n_keys = n_sel + (p.phase == 2 ? 0 : L);
+      int per_split = (n_keys + p.n_splits - 1) / p.n_splits;
+      per_split = (per_split + kTK - 1) / kTK * kTK;
+      const int v0 = min(n_keys, split * per_split);
+      const int v1 = min(n_keys, v0 + per_split);
+      const int n_tiles = (v1 - v0 + kTK - 1) / kTK;
+      if (lane == 0) {
+        int* hd = hdr + hb * 8;
+        hd[0] = b; hd[1] = t0; hd[2] = nt; hd[3] = L; hd[4] = n_sel; hd[5] = v0; hd[6] = v1; hd[7] = split;
+        const uint32_t qbytes = (uint32_t)(nt * p.n_q * D * 2);
+        mbar_arrive_expect_tx(&hfull[hb], qbytes);  // releases the header writes above
+        bulk_load(qsm + hb * q_elems, p.q + ((size_t)b * p.q_tokens + t0) * p.n_q * D, qbytes, &hfull[hb]);
+      }
+      // ---- the item's tiles: kTK keys each, a bulk copy per key and tensor plus the RoPE rows ----
+      for (int t = 0; t < n_tiles; ++t, ++gt) {
+        const int st = gt % L_.n_stages;
+        if (gt >= L_.n_stages) mbar_wait(&ebars[st], ((gt / L_.n_stages) - 1) & 1);
+        const int tv0 = v0 + t * kTK;
+        const int rows = min(kTK, v1 - tv0);
+        const int n_chunk_rows = max(0, min(rows, n_sel - tv0));
+        const int n_loc_rows = rows - n_chunk_rows;
+        const uint32_t tb = (table && n_loc_rows > 0) ? (uint32_t)(n_loc_rows * (D / 2) * 8) : 0u;
+        if (lane == 0) mbar_arrive_expect_tx(&bars[st], (uint32_t)(2 * rows * row_bytes) + tb);
+        __syncwarp();
+        uint8_t* kdst = stage_mem + (size_t)st * L_.stage_bytes;
+        uint8_t* vdst = kdst + L_.kbytes;
+        if (lane < rows) {
+          const int v = tv0 + lane;
+          const __nv_bfloat16 *ks, *vs;
+          if (v < n_sel) {
+            int lo = 0, hi = k - 1;  // segment with seg_v[lo] <= v < seg_v[lo + 1]
+            while (lo < hi) {
+              const int mid = (lo + hi + 1) >> 1;
+              if (seg_v[mid] <= v) lo = mid; else hi = mid - 1;
+            }
+            const size_t ch = (size_t)(seg_c[lo] + (v - seg_v[lo]));
+            ks = p.K_bar + ch * n_kv * D;
+            vs = p.V_bar + ch * n_kv * D;
+          } else {
+            const size_t off = ((size_t)b * p.t_loc_max + (size_t)(v - n_sel)) * n_kv * D;
+            ks = p.K_loc + off;
+            vs = p.V_loc + off;
+          }
+          bulk_load(kdst + lane * L_.krow, ks, row_bytes, &bars[st]);
+          bulk_load(vdst + lane * L_.krow, vs, row_bytes, &bars[st]);
+        }
+        if (tb && lane == 31) {
+          const int j0 = tv0 + n_chunk_rows - n_sel;
+          bulk_load(vdst + L_.kbytes + n_chunk_rows * (D / 2) * 8, p.rope_tab + (size_t)j0 * (D / 2), tb, &bars[st]);
+        }
+      }
+    }
     return;  // the compute warps no longer synchronise with the whole block
   }
 
-  // ---- query fragments of this warp's GQA group: mma row = tt * G + gg (token t0 + tt,
-  //      q head h * G + gg); token t sits at pos_offset + L - M + t; scale, bf16 ----
+  // ---- compute warps, item by item ----
   const int n_compute = 32 * n_kv;
-  const int64_t pos_q0 = (int64_t)p.pos_offset + L - p.q_tokens + t0;
-  for (int i = tid; i < nt * (D / 2); i += n_compute)
-    qcs[i] = rope_cos_sin(p.turns, i % (D / 2), pos_q0 + i / (D / 2));
-  named_bar_sync(1, n_compute);
-  const int g = lane >> 2, c = lane & 3;
-  uint32_t qa[KS][4];
-  {
-#pragma unroll
-    for (int s = 0; s < KS; ++s) {
-#pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {        // rows g and g + 8
-        const int row = g + 8 * rr;
-        const int tt = row / G, gg = row - tt * G;
-        const uint16_t* qb = qsm + ((size_t)tt * p.n_q + h * G + gg) * D;
-#pragma unroll
-        for (int hk = 0; hk < 2; ++hk) {      // k cols 2c.. and 2c+8..
-          const int dim = 16 * s + 8 * hk + 2 * c;
-          float v[2] = {0.f, 0.f};
-          if (tt < nt) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int dd = dim + e;
-              const bool first = dd < D / 2;
-              const int i = first ? dd : dd - D / 2;
-              const int partner = first ? dd + D / 2 : dd - D / 2;
-              const float x = bf16_bits_to_float(qb[dd]);
-              const float y = bf16_bits_to_float(qb[partner]);
-              const float2 cs = qcs[tt * (D / 2) + i];
-              // first half: x cos - y sin; second half: x cos + y sin (y = first-half partner)
-              const float rot = first ? (x * cs.x - y * cs.y) : (x * cs.x + y * cs.y);
-              v[e] = rot * p.scale_log2;
-            }
-          }
-          qa[s][rr + 2 * hk] = pack_bf16x2(v[0], v[1]);
-        }
-      }
-    }
-  }
-
-  float acc[NBLK][4];
-#pragma unroll
-  for (int n = 0; n < NBLK; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-  float m_run[2] = {-INFINITY, -INFINITY};
-  float l_run[2] = {0.f, 0.f};
-  const int hoff = h * D * 2;  // this head's bytes within a key row
-  // causal limit of rows g and g + 8: token t sees the chunks and local tokens j <= L - M + t
-  int lim[2];
-#pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    const int tt = (g + 8 * rr) / G;
-    lim[rr] = tt < nt ? n_sel + max(0, min(L, L - p.q_tokens + t0 + tt + 1)) : v1;
-  }
-
-  for (int t = 0; t < n_tiles; ++t) {
-    const int st = t % L_.n_stages;
-    mbar_wait(&bars[st], (t / L_.n_stages) & 1);
-
-    const int tv0 = v0 + t * kTK;
-    const uint8_t* kst = stage_mem + (size_t)st * L_.stage_bytes;
-    const uint32_t kbase = smem_u32(kst) + hoff;
-    const uint32_t vbase = kbase + L_.kbytes;
-    const float2* tab = reinterpret_cast<const float2*>(kst + 2 * L_.kbytes);
-
-    // ---- K fragments (B operand, keys = n) ----
-    uint32_t kb[KS][2][2];
+  int gt = 0;
+  for (int it = blockIdx.x, j = 0; it < n_items; it += gridDim.x, ++j) {
+    const int hb = j & 1;
+    mbar_wait(&hfull[hb], (j >> 1) & 1);
+    const int* hd = hdr + hb * 8;
+    const int b = hd[0], t0 = hd[1], nt = hd[2], L = hd[3], n_sel = hd[4], v0 = hd[5], v1 = hd[6], split = hd[7];
+    const int n_tiles = (v1 - v0 + kTK - 1) / kTK;
+    const uint16_t* qsm_b = qsm + hb * q_elems;
+    // ---- query fragments of this warp's GQA group: mma row = tt * G + gg (token t0 + tt,
+    //      q head h * G + gg); token t sits at pos_offset + L - M + t; scale, bf16 ----
+    named_bar_sync(1, n_compute);  // every warp has built its previous fragments (qcs is reused)
+    const int64_t pos_q0 = (int64_t)p.pos_offset + L - p.q_tokens + t0;
+    for (int i = tid; i < nt * (D / 2); i += n_compute)
+      qcs[i] = rope_cos_sin(p.turns, i % (D / 2), pos_q0 + i / (D / 2));
+    named_bar_sync(1, n_compute);
+    const int g = lane >> 2, c = lane & 3;
+    uint32_t qa[KS][4];
     {
-      const int key = (lane & 7) + 8 * (lane >> 4);
-      const int dsel = 8 * ((lane >> 3) & 1);
-#pragma unroll
-      for (int s = 0; s < KS; ++s)
-        ldmatrix_x4(kb[s][0][0], kb[s][0][1], kb[s][1][0], kb[s][1][1], kbase + key * L_.krow + (16 * s + dsel) * 2);
-    }
-    // ---- rotate local keys in registers (pairs i, i + D/2 sit in ksteps s, s + KS/2) ----
-    if (table) {
-#pragma unroll
-      for (int nb = 0; nb < 2; ++nb) {
-        const int r = 8 * nb + g;
-        const int v = tv0 + r;
-        if (v >= n_sel && v < v1) {
-          const float2* trow = tab + r * (D / 2);
-#pragma unroll
-          for (int s = 0; s < KS / 2; ++s) {
-#pragma unroll
-            for (int hk = 0; hk < 2; ++hk) {
-              const int i = 16 * s + 8 * hk + 2 * c;
-              const float4 cs = *reinterpret_cast<const float4*>(trow + i);  // (cos_i, sin_i, cos_i+1, sin_i+1)
-              const float2 x = unpack_bf16x2(kb[s][nb][hk]);
-              const float2 y = unpack_bf16x2(kb[s + KS / 2][nb][hk]);
-              const float x0 = x.x * cs.x - y.x * cs.y, y0 = y.x * cs.x + x.x * cs.y;
-              const float x1 = x.y * cs.z - y.y * cs.w, y1 = y.y * cs.z + x.y * cs.w;
-              kb[s][nb][hk] = pack_bf16x2(x0, x1);
-              kb[s + KS / 2][nb][hk] = pack_bf16x2(y0, y1);
+  #pragma unroll
+      for (int s = 0; s < KS; ++s) {
+  #pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {        // rows g and g + 8
+          const int row = g + 8 * rr;
+          const int tt = row / G, gg = row - tt * G;
+          const uint16_t* qb = qsm_b + ((size_t)tt * p.n_q + h * G + gg) * D;
+  #pragma unroll
+          for (int hk = 0; hk < 2; ++hk) {      // k cols 2c.. and 2c+8..
+            const int dim = 16 * s + 8 * hk + 2 * c;
+            float v[2] = {0.f, 0.f};
+            if (tt < nt) {
+  #pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int dd = dim + e;
+                const bool first = dd < D / 2;
+                const int i = first ? dd : dd - D / 2;
+                const int partner = first ? dd + D / 2 : dd - D / 2;
+                const float x = bf16_bits_to_float(qb[dd]);
+                const float y = bf16_bits_to_float(qb[partner]);
+                const float2 cs = qcs[tt * (D / 2) + i];
+                // first half: x cos - y sin; second half: x cos + y sin (y = first-half partner)
+                const float rot = first ? (x * cs.x - y * cs.y) : (x * cs.x + y * cs.y);
+                v[e] = rot * p.scale_log2;
+              }
             }
+            qa[s][rr + 2 * hk] = pack_bf16x2(v[0], v[1]);
           }
         }
       }
     }
-    // ---- S = q K^T (rows = heads, cols = 16 keys) ----
-    float sc[2][4];
-#pragma unroll
-    for (int nb = 0; nb < 2; ++nb) {
-      sc[nb][0] = sc[nb][1] = sc[nb][2] = sc[nb][3] = 0.f;
-#pragma unroll
-      for (int s = 0; s < KS; ++s)
-        mma_bf16_16816(sc[nb], qa[s][0], qa[s][1], qa[s][2], qa[s][3], kb[s][nb][0], kb[s][nb][1]);
-    }
-#pragma unroll
-    for (int nb = 0; nb < 2; ++nb)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int v = tv0 + 8 * nb + 2 * c + e;
-        if (v >= v1 || v >= lim[0]) sc[nb][e] = -INFINITY;
-        if (v >= v1 || v >= lim[1]) sc[nb][2 + e] = -INFINITY;
-      }
-    // ---- online softmax (rows g and g + 8) ----
-    float alpha[2];
-#pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-      float mx = fmaxf(fmaxf(sc[0][2 * rr], sc[0][2 * rr + 1]), fmaxf(sc[1][2 * rr], sc[1][2 * rr + 1]));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      const float m_new = fmaxf(m_run[rr], mx);
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      alpha[rr] = exp2f(m_run[rr] - m_use);
-      m_run[rr] = m_new;
-      float ls = 0.f;
-#pragma unroll
-      for (int nb = 0; nb < 2; ++nb)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float pv = exp2f(sc[nb][2 * rr + e] - m_use);
-          sc[nb][2 * rr + e] = pv;
-          ls += pv;
-        }
-      l_run[rr] = l_run[rr] * alpha[rr] + ls;
-    }
-#pragma unroll
-    for (int n = 0; n < NBLK; ++n) {
-      acc[n][0] *= alpha[0];
-      acc[n][1] *= alpha[0];
-      acc[n][2] *= alpha[1];
-      acc[n][3] *= alpha[1];
-    }
-    // ---- O += P V ----
-    const uint32_t pa0 = pack_bf16x2(sc[0][0], sc[0][1]);
-    const uint32_t pa1 = pack_bf16x2(sc[0][2], sc[0][3]);
-    const uint32_t pa2 = pack_bf16x2(sc[1][0], sc[1][1]);
-    const uint32_t pa3 = pack_bf16x2(sc[1][2], sc[1][3]);
-    {
-      const int key = (lane & 7) + 8 * ((lane >> 3) & 1);
-      const int dsel = 8 * (lane >> 4);
-#pragma unroll
-      for (int n = 0; n < NBLK; n += 2) {
-        uint32_t b0, b1, b2, b3;
-        ldmatrix_x4_trans(b0, b1, b2, b3, vbase + key * L_.krow + (8 * n + dsel) * 2);
-        mma_bf16_16816(acc[n], pa0, pa1, pa2, pa3, b0, b1);
-        mma_bf16_16816(acc[n + 1], pa0, pa1, pa2, pa3, b2, b3);
-      }
-    }
+
+
     __syncwarp();
-    if (lane == 0) mbar_arrive(&ebars[st]);  // this warp is done with stage st
-  }
+    if (lane == 0) mbar_arrive(&hempty[hb]);  // header and query rows read: the buffer may refill
 
-  // ---- this warp's split partial: unnormalised output, running max and sum per q head ----
-#pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 1);
-    l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 2);
-  }
-#pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    const int row = g + 8 * rr;
-    const int tt = row / G;
-    if (tt < nt) {
-      const size_t qh = ((size_t)b * p.q_tokens + t0 + tt) * p.n_q + (size_t)h * G + (row - tt * G);
-      const size_t ps = qh * p.n_splits_total + p.split_base + split;
-      float* po = p.part_o + ps * D;
-#pragma unroll
-      for (int n = 0; n < NBLK; ++n)
-        *reinterpret_cast<float2*>(po + 8 * n + 2 * c) = make_float2(acc[n][2 * rr], acc[n][2 * rr + 1]);
-      if (c == 0) {
-        p.part_ml[ps * 2 + 0] = m_run[rr];
-        p.part_ml[ps * 2 + 1] = l_run[rr];
+    float acc[NBLK][4];
+  #pragma unroll
+    for (int n = 0; n < NBLK; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY};
+    float l_run[2] = {0.f, 0.f};
+    const int hoff = h * D * 2;  // this head's bytes within a key row
+    // causal limit of rows g and g + 8: token t sees the chunks and local tokens j <= L - M + t
+    int lim[2];
+  #pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const int tt = (g + 8 * rr) / G;
+      lim[rr] = tt < nt ? n_sel + max(0, min(L, L - p.q_tokens + t0 + tt + 1)) : v1;
+    }
+
+    for (int t = 0; t < n_tiles; ++t) {
+      const int gtt = gt + t;  // tile counter over this CTA's items: the ring position
+      const int st = gtt % L_.n_stages;
+      mbar_wait(&bars[st], (gtt / L_.n_stages) & 1);
+
+      const int tv0 = v0 + t * kTK;
+      const uint8_t* kst = stage_mem + (size_t)st * L_.stage_bytes;
+      const uint32_t kbase = smem_u32(kst) + hoff;
+      const uint32_t vbase = kbase + L_.kbytes;
+      const float2* tab = reinterpret_cast<const float2*>(kst + 2 * L_.kbytes);
+
+      // ---- K fragments (B operand, keys = n) ----
+      uint32_t kb[KS][2][2];
+      {
+        const int key = (lane & 7) + 8 * (lane >> 4);
+        const int dsel = 8 * ((lane >> 3) & 1);
+  #pragma unroll
+        for (int s = 0; s < KS; ++s)
+          ldmatrix_x4(kb[s][0][0], kb[s][0][1], kb[s][1][0], kb[s][1][1], kbase + key * L_.krow + (16 * s + dsel) * 2);
+      }
+      // ---- rotate local keys in registers (pairs i, i + D/2 sit in ksteps s, s + KS/2) ----
+      if (table) {
+  #pragma unroll
+        for (int nb = 0; nb < 2; ++nb) {
+          const int r = 8 * nb + g;
+          const int v = tv0 + r;
+          if (v >= n_sel && v < v1) {
+            const float2* trow = tab + r * (D / 2);
+  #pragma unroll
+            for (int s = 0; s < KS / 2; ++s) {
+  #pragma unroll
+              for (int hk = 0; hk < 2; ++hk) {
+                const int i = 16 * s + 8 * hk + 2 * c;
+                const float4 cs = *reinterpret_cast<const float4*>(trow + i);  // (cos_i, sin_i, cos_i+1, sin_i+1)
+                const float2 x = unpack_bf16x2(kb[s][nb][hk]);
+                const float2 y = unpack_bf16x2(kb[s + KS / 2][nb][hk]);
+                const float x0 = x.x * cs.x - y.x * cs.y, y0 = y.x * cs.x + x.x * cs.y;
+                const float x1 = x.y * cs.z - y.y * cs.w, y1 = y.y * cs.z + x.y * cs.w;
+                kb[s][nb][hk] = pack_bf16x2(x0, x1);
+                kb[s + KS / 2][nb][hk] = pack_bf16x2(y0, y1);
+              }
+            }
+          }
+        }
+      }
+      // ---- S = q K^T (rows = heads, cols = 16 keys) ----
+      float sc[2][4];
+  #pragma unroll
+      for (int nb = 0; nb < 2; ++nb) {
+        sc[nb][0] = sc[nb][1] = sc[nb][2] = sc[nb][3] = 0.f;
+  #pragma unroll
+        for (int s = 0; s < KS; ++s)
+          mma_bf16_16816(sc[nb], qa[s][0], qa[s][1], qa[s][2], qa[s][3], kb[s][nb][0], kb[s][nb][1]);
+      }
+  #pragma unroll
+      for (int nb = 0; nb < 2; ++nb)
+  #pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int v = tv0 + 8 * nb + 2 * c + e;
+          if (v >= v1 || v >= lim[0]) sc[nb][e] = -INFINITY;
+          if (v >= v1 || v >= lim[1]) sc[nb][2 + e] = -INFINITY;
+        }
+      // ---- online softmax (rows g and g + 8) ----
+      float alpha[2];
+  #pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        float mx = fmaxf(fmaxf(sc[0][2 * rr], sc[0][2 * rr + 1]), fmaxf(sc[1][2 * rr], sc[1][2 * rr + 1]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float m_new = fmaxf(m_run[rr], mx);
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+        alpha[rr] = exp2f(m_run[rr] - m_use);
+        m_run[rr] = m_new;
+        float ls = 0.f;
+  #pragma unroll
+        for (int nb = 0; nb < 2; ++nb)
+  #pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float pv = exp2f(sc[nb][2 * rr + e] - m_use);
+            sc[nb][2 * rr + e] = pv;
+            ls += pv;
+          }
+        l_run[rr] = l_run[rr] * alpha[rr] + ls;
+      }
+  #pragma unroll
+      for (int n = 0; n < NBLK; ++n) {
+        acc[n][0] *= alpha[0];
+        acc[n][1] *= alpha[0];
+        acc[n][2] *= alpha[1];
+        acc[n][3] *= alpha[1];
+      }
+      // ---- O += P V ----
+      const uint32_t pa0 = pack_bf16x2(sc[0][0], sc[0][1]);
+      const uint32_t pa1 = pack_bf16x2(sc[0][2], sc[0][3]);
+      const uint32_t pa2 = pack_bf16x2(sc[1][0], sc[1][1]);
+      const uint32_t pa3 = pack_bf16x2(sc[1][2], sc[1][3]);
+      {
+        const int key = (lane & 7) + 8 * ((lane >> 3) & 1);
+        const int dsel = 8 * (lane >> 4);
+  #pragma unroll
+        for (int n = 0; n < NBLK; n += 2) {
+          uint32_t b0, b1, b2, b3;
+          ldmatrix_x4_trans(b0, b1, b2, b3, vbase + key * L_.krow + (8 * n + dsel) * 2);
+          mma_bf16_16816(acc[n], pa0, pa1, pa2, pa3, b0, b1);
+          mma_bf16_16816(acc[n + 1], pa0, pa1, pa2, pa3, b2, b3);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ebars[st]);  // this warp is done with stage st
+    }
+
+
+    gt += n_tiles;
+
+    // ---- this warp's split partial: unnormalised output, running max and sum per q head ----
+  #pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 1);
+      l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 2);
+    }
+  #pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const int row = g + 8 * rr;
+      const int tt = row / G;
+      if (tt < nt) {
+        const size_t qh = ((size_t)b * p.q_tokens + t0 + tt) * p.n_q + (size_t)h * G + (row - tt * G);
+        const size_t ps = qh * p.n_splits_total + p.split_base + split;
+        float* po = p.part_o + ps * D;
+  #pragma unroll
+        for (int n = 0; n < NBLK; ++n)
+          *reinterpret_cast<float2*>(po + 8 * n + 2 * c) = make_float2(acc[n][2 * rr], acc[n][2 * rr + 1]);
+        if (c == 0) {
+          p.part_ml[ps * 2 + 0] = m_run[rr];
+          p.part_ml[ps * 2 + 1] = l_run[rr];
+        }
       }
     }
   }
@@ -500,7 +538,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
 }
 
 int stages_that_fit(int n_kv, int n_q, int D, bool table, int mt) {
-  const int budget = 210 * 1024;
+  const int budget = 224 * 1024;
   for (int st = kMaxStages; st >= 2; --st) {
     AttnSmem L(n_kv, D, st, table);
     if (L.total(n_q, D, mt) <= (size_t)budget) return st;
@@ -804,6 +842,7 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
   p.n_splits = phase == 0 ? w.n_splits : phase == 1 ? w.n_split_local : w.n_split_chunk;
   p.split_base = phase == 2 ? w.n_split_local : 0;
   p.n_splits_total = phase == 0 ? w.n_splits : w.n_split_local + w.n_split_chunk;
+  p.n_queries = B;
   p.q_tokens = M;
   p.tok_per_cta = tokens_per_cta(d, M);
   p.n_tgroups = (M + p.tok_per_cta - 1) / p.tok_per_cta;
@@ -812,7 +851,9 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
   p.n_stages = stages_that_fit(d.n_kv, d.n_q, D, tab != nullptr, p.tok_per_cta);
   {
     TraceScope ts(kKAttnSplit, s);
-    dim3 grid(p.n_splits, B * p.n_tgroups);
+    // persistent: each CTA takes items (split, query, token group) in turn
+    const int n_items = p.n_splits * B * p.n_tgroups;
+    dim3 grid(std::max(1, std::min(n_items, sm_count())));
     const size_t sm = AttnSmem(d.n_kv, D, p.n_stages, tab != nullptr).total(d.n_q, D, p.tok_per_cta);
     if (D == 128) {
       MSA_CUDA_CHECK(cudaFuncSetAttribute(attn_split_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
