@@ -360,16 +360,16 @@ def run_gpu(args):
     torch.cuda.synchronize()
 
     def step(i):
-        # one stream: routing, the new token into the rotated local cache, sparse attention.  (Running
-        # the local half of the attention on a second stream beside the routing, with the two-phase
-        # call, measured slower here: at 1M tokens the scan wants most SMs at once.)
+        # one stream: the new token into the rotated local cache, routing, sparse attention.  The
+        # attention's local-key work starts while the routing's kernels finish (early_local: q and
+        # the local cache were final before the routing call was enqueued).
         x = rot[i % N_ROT]
         j = i % N_ROT
+        msa.kv_append(d, k_new, v_new, x["K_loc"], x["V_loc"], slots, c["pos_offset"])
         msa.route_topk(d, x["Hq"], W_QR, x["KR"], chunk_off, k, out=(out_idx[j], out_sc[j], None), ws=r_ws,
                        kr_inv_norm=inv_rot[j])
-        msa.kv_append(d, k_new, v_new, x["K_loc"], x["V_loc"], slots, c["pos_offset"])
         msa.sparse_attend(d, x["q"], x["K_bar"], x["V_bar"], chunk_off, out_idx[j], x["K_loc"], x["V_loc"], loc_len,
-                          c["pos_offset"], out=out_o[j], ws=a_ws, k_loc_rotated=True)
+                          c["pos_offset"], out=out_o[j], ws=a_ws, k_loc_rotated=True, early_local=True)
 
     # ---- capture one graph per rotation copy (untraced) ----
     graphs = []
@@ -479,7 +479,7 @@ def run_gpu(args):
         msa.route_topk(d, dev_hq, W_QR, x["KR"], chunk_off, k, out=(out_idx[0], out_sc[0], None), ws=r_ws,
                        kr_inv_norm=inv_rot[i % N_ROT])
         msa.sparse_attend(d, dev_q, x["K_bar"], x["V_bar"], chunk_off, out_idx[0], x["K_loc"], x["V_loc"], loc_len,
-                          c["pos_offset"], out=out_o[0], ws=a_ws, k_loc_rotated=True)
+                          c["pos_offset"], out=out_o[0], ws=a_ws, k_loc_rotated=True, early_local=True)
         h_idx.copy_(out_idx[0], non_blocking=True)
         h_sc.copy_(out_sc[0], non_blocking=True)
         h_out.copy_(out_o[0], non_blocking=True)

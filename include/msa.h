@@ -286,6 +286,14 @@ msa_status msa_aux_loss(const msa_dims* dims, const void* QR, const void* K_pos,
  *            attends over the selected chunks and merges both parts into out (K_loc and
  *            V_loc are not read).  Phase 2 must be ordered after phase 1 (same stream, or
  *            an event).  The result equals phase 0's up to fp32 summation order.
+ *            phase | MSA_ATTEND_EARLY_LOCAL (phases 0 and 1): the work on the local keys may
+ *            start before the kernels of the preceding library call on the stream have
+ *            finished (typically msa_route_topk producing topk_idx), hiding it behind the
+ *            routing.  The caller guarantees that q, K_loc, V_loc, loc_len (and rope_cache)
+ *            were final before that preceding call was enqueued, and that the preceding call
+ *            is not an msa_sparse_attend on this workspace.  The flag has no effect when
+ *            the call builds its own rotation table (k_loc_rotated 0 and rope_cache NULL).
+ *            The result is the same as without the flag.
  *   out      [B, M, n_q, head_dim] bf16.
  * Limits: 1 <= M, B * M <= 65535.
  * Query head g attends with KV head g / (n_q / n_kv).  Every query token sees
@@ -295,6 +303,7 @@ msa_status msa_aux_loss(const msa_dims* dims, const void* QR, const void* K_pos,
  * fp32 then rounded to bf16; local keys are rotated in fp32 and rounded to
  * bf16; products and softmax in fp32.
  * ------------------------------------------------------------------------- */
+#define MSA_ATTEND_EARLY_LOCAL 16
 size_t msa_attend_workspace_size(const msa_dims* dims, int32_t B, int32_t q_tokens, int32_t k,
                                  int32_t t_loc_max, int32_t pos_offset);
 msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, int32_t q_tokens, const void* K_bar,

@@ -20,7 +20,7 @@ __all__ = [
     "Dims", "MSAError", "lib", "chunk_offsets", "encode_memory", "append_memory", "route_topk", "sparse_attend",
     "aux_loss", "kv_append", "router_key_norms",
     "route_workspace_size", "attend_workspace_size", "rope_cache_build", "topk_merge", "rope_rows", "gather_kv", "encode_workspace_size", "check_device_errors",
-    "trace_enable", "trace_reset", "trace_read", "trace_kernel_names", "AGG_MAX", "AGG_MEAN",
+    "trace_enable", "trace_reset", "trace_read", "trace_kernel_names", "AGG_MAX", "AGG_MEAN", "ATTEND_EARLY_LOCAL",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -28,6 +28,7 @@ LIB_PATH = os.path.join(_HERE, "libmsa.so")
 
 AGG_MAX = 0
 AGG_MEAN = 1
+ATTEND_EARLY_LOCAL = 16  # msa.h MSA_ATTEND_EARLY_LOCAL, OR-ed into the phase argument
 
 STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED", 3: "MSA_ERR_WORKSPACE",
           4: "MSA_ERR_CUDA", 5: "MSA_ERR_TIMEOUT"}
@@ -334,14 +335,17 @@ def kv_append(dims, k_new, v_new, K_loc, V_loc, slots, pos_offset: int, stream=N
 
 def sparse_attend(dims, q, K_bar, V_bar, chunk_off, topk_idx, K_loc, V_loc, loc_len, pos_offset: int,
                   softmax_scale: float = 0.0, out=None, ws=None, stream=None, rope_cache=None,
-                  k_loc_rotated: bool = False, phase: int = 0):
+                  k_loc_rotated: bool = False, phase: int = 0, early_local: bool = False):
     """GQA attention of the query tokens over [selected docs' K̄; local K].
 
     ``q`` is [B, n_q, head_dim] (one decode token) or [B, M, n_q, head_dim] (the last M local
     tokens, causal among the local keys); ``out`` has the shape of ``q``.
     ``rope_cache`` (from ``rope_cache_build`` with the same pos_offset and t_loc_max) skips
     rebuilding the local-position rotation table.  ``phase`` 1 / 2 splits the call into the
-    local-keys part and the selected-chunks part (which merges both); pass the same ``ws``."""
+    local-keys part and the selected-chunks part (which merges both); pass the same ``ws``.
+    ``early_local`` (MSA_ATTEND_EARLY_LOCAL) lets the local-key work start before the
+    preceding library call's kernels finish; q, K_loc, V_loc and loc_len must have been final
+    before that call was enqueued, and it must not be a sparse_attend on the same ``ws``."""
     import torch
 
     dd = Dims.of(dims)
@@ -357,7 +361,8 @@ def sparse_attend(dims, q, K_bar, V_bar, chunk_off, topk_idx, K_loc, V_loc, loc_
     _check(lib.msa_sparse_attend(ctypes.byref(dd), _ptr(q), B, M, _ptr(K_bar), _ptr(V_bar), _ptr(chunk_off), n_docs,
                                  K_bar.shape[0], _ptr(topk_idx), k, _ptr(K_loc), _ptr(V_loc), _ptr(loc_len),
                                  t_loc_max, pos_offset, _ptr(rope_cache), int(bool(k_loc_rotated)),
-                                 float(softmax_scale), int(phase), _ptr(out),
+                                 float(softmax_scale), int(phase) | (ATTEND_EARLY_LOCAL if early_local else 0),
+                                 _ptr(out),
                                  _aligned_ptr(ws), nbytes, _stream(stream)))
     return out
 

@@ -33,9 +33,8 @@ struct AttendWs {
   float2* rope_tab;  // [t_loc_max][D/2] (cos, sin)
   float* part_ml;    // [B][n_q][S][2]  running max (log2 domain) and sum
   float* part_o;     // [B][n_q][S][D]  unnormalised output
-  int n_splits;        // splits of the one-launch call (every key)
-  int n_split_local;   // splits of the local-keys phase (ids 0 .. n_split_local - 1)
-  int n_split_chunk;   // splits of the selected-chunks phase (ids after the local ones)
+  int n_split_local;   // splits of the local keys (partial slots 0 .. n_split_local - 1)
+  int n_split_chunk;   // splits of the selected chunks (the slots after the local ones)
   int n_parts;         // partial slots per (query token, q head)
 };
 
@@ -45,13 +44,14 @@ constexpr int kTK = 16;          // keys per tile (one mma K-step of P V)
 constexpr int kMaxStages = 4;
 constexpr int kMaxK = 256;
 constexpr int kMaxSplits = 1024;
+constexpr int kChunksPerDocEst = 40;  // expected pooled chunks per selected document (split planning only)
+constexpr int kCoSmemMax = 4096;      // chunk_off entries the split kernel may keep in shared memory
 constexpr float kLog2e = 1.4426950408889634f;
 
 // cos/sin of (pos_offset + j) * theta_i, theta_i = base^(-2i/D), for local positions j
 __global__ void __launch_bounds__(256) rope_table_kernel(float2* __restrict__ tab, int t_loc_max, int half,
                                                          int pos_offset, const RopeTurns turns) {
-  pdl_launch_dependents();
-  pdl_wait();
+  pdl_enter();
   const int64_t n = (int64_t)t_loc_max * half;
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
     const int j = (int)(e / half), i = (int)(e % half);
@@ -71,12 +71,15 @@ struct AttnParams {
   const float2* rope_tab;
   float* part_ml;
   float* part_o;
-  int n_q, n_kv, k, n_docs, t_loc_max, pos_offset, n_splits, n_stages;
+  int n_q, n_kv, k, n_docs, t_loc_max, pos_offset, n_stages;
   int n_queries;     // B
   int q_tokens;      // M: query tokens per query (the last M local tokens)
-  int phase;         // 0: every key; 1: the local keys only; 2: the selected chunks only
-  int split_base;    // this launch's first split id in the partial arrays
-  int n_splits_total;  // splits per (query token, q head) in the partial arrays
+  int n_loc_splits;    // this launch's splits of the local keys (0: none)
+  int n_chunk_splits;  // this launch's splits of the selected chunks (0: none)
+  int chunk_part_base;  // partial slot of chunk split 0 (the local splits take slots 0 ..)
+  int n_parts;       // partial slots per (query token, q head)
+  int early;         // local-key items run before the predecessor kernel has finished
+  int co_cap;        // chunk_off entries copied to shared memory (n_docs + 1), or 0 (read from L2)
   int tok_per_cta;   // MT: tokens per CTA, MT * G <= 16 mma rows
   int n_tgroups;     // ceil(M / MT)
   float scale_log2;  // softmax scale * log2(e)
@@ -97,14 +100,14 @@ struct AttnSmem {
     stage_bytes = 2 * kbytes + tbytes;
     n_stages = stages;
   }
-  // two query buffers, barriers (ring, item header), two item headers and segment tables, the
-  // tokens' cos/sin
-  __host__ __device__ size_t fixed_bytes(int n_q, int D, int mt) const {
-    return 2 * (size_t)mt * n_q * D * 2 + (2 * kMaxStages + 4) * 8 + 2 * 8 * 4 + 2 * (2 * kMaxK + 2) * 4 +
-           (size_t)mt * (D / 2) * 8;
+  // two query buffers, barriers (ring, item header and selection), two item headers and
+  // segment tables, the tokens' cos/sin, the document table (co_cap entries, 16-byte multiple)
+  __host__ __device__ size_t fixed_bytes(int n_q, int D, int mt, int co_cap) const {
+    return 2 * (size_t)mt * n_q * D * 2 + (2 * kMaxStages + 6) * 8 + 2 * 8 * 4 + 2 * (2 * kMaxK + 2) * 4 +
+           (size_t)mt * (D / 2) * 8 + (size_t)(co_cap + 3) / 4 * 16;
   }
-  __host__ __device__ size_t total(int n_q, int D, int mt) const {
-    return (size_t)n_stages * stage_bytes + fixed_bytes(n_q, D, mt);
+  __host__ __device__ size_t total(int n_q, int D, int mt, int co_cap) const {
+    return (size_t)n_stages * stage_bytes + fixed_bytes(n_q, D, mt, co_cap);
   }
 };
 
@@ -126,16 +129,22 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
   uint64_t* ebars = bars + kMaxStages;                               // [stage] every warp done with it
   uint64_t* hfull = ebars + kMaxStages;                              // [2] an item's header and query landed
   uint64_t* hempty = hfull + 2;                                      // [2] every warp done with them
-  int* hdr = reinterpret_cast<int*>(hempty + 2);                     // [2][8] item headers
+  uint64_t* hsel = hempty + 2;                                       // [2] the item's key range is known
+  int* hdr = reinterpret_cast<int*>(hsel + 2);                       // [2][8] item headers
   int* segs = hdr + 16;                                              // [2][2 kMaxK + 2] segment tables
   float2* qcs = reinterpret_cast<float2*>(segs + 2 * (2 * kMaxK + 2));  // [MT][D/2] cos/sin at the tokens' positions
+  int* co_sm = reinterpret_cast<int*>(qcs + (size_t)MT * (D / 2));   // [co_cap] chunk_off
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = warp;               // the KV head this warp serves (warps 0 .. n_kv-1)
   const bool producer = warp == n_kv;  // the last warp builds each item and streams its tiles
-  const int k = p.phase == 1 ? 0 : p.k;  // the local-keys phase has no selected documents
-  // items: (split, query, token group); this CTA takes items blockIdx.x, + gridDim.x, ...
-  const int n_items = p.n_splits * p.n_queries * p.n_tgroups;
+  const int k = p.k;
+  // items: every (query, token group)'s local-key splits first, then its selected-chunk
+  // splits; this CTA takes items blockIdx.x, + gridDim.x, ... in increasing order, so its
+  // local-key items come first
+  const int n_groups = p.n_queries * p.n_tgroups;
+  const int n_loc_items = p.n_loc_splits * n_groups;
+  const int n_items = n_loc_items + p.n_chunk_splits * n_groups;
 
   // ---- no global memory yet: overlaps the previous kernel's tail ----
   for (int i = tid; i < L_.n_stages * L_.stage_bytes / 16; i += blockDim.x)
@@ -148,42 +157,72 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
     for (int s = 0; s < 2; ++s) {
       mbar_init(&hfull[s], 1);
       mbar_init(&hempty[s], n_kv);
+      mbar_init(&hsel[s], 1);
     }
     fence_mbar_init();
   }
   __syncthreads();
-  pdl_launch_dependents();
-  pdl_wait();
+  // Without `early` every thread waits for the predecessor here.  With it, the caller has
+  // guaranteed that q, the local KV, loc_len and chunk_off were final before the
+  // predecessor's call was enqueued (and that the predecessor does not touch this workspace):
+  // only topk_idx comes from the predecessor, so the producer waits just before it reads
+  // topk_idx for its first selected-chunk item, the compute warps once they have built that
+  // item's query fragments, and every thread at its end at the latest.
+  bool waited = !p.early;
+  if (waited) pdl_enter();
   const int row_bytes = n_kv * D * 2;  // one key, every KV head
 
   if (producer) {
-    // ---- per item: the segment table (selected docs in top-k order, then local), the header
-    //      and the query rows for the compute warps, then the item's tiles into the ring ----
+    // ---- the document table in shared memory (one round trip, 16-byte asynchronous copies;
+    //      the tail past the last whole 16 bytes with plain loads) ----
+    if (p.co_cap && p.n_chunk_splits) {
+      const int n = p.n_docs + 1, n16 = n / 4;
+      for (int i = lane; i < n16; i += 32) cp_async16(co_sm + 4 * i, reinterpret_cast<const uint4*>(p.chunk_off) + i);
+      for (int i = 4 * n16 + lane; i < n; i += 32) co_sm[i] = __ldg(&p.chunk_off[i]);
+      cp_async_wait_all();
+      __syncwarp();
+    }
+    // ---- per item: the header and the query rows for the compute warps, then the segment table
+    //      (selected docs in top-k order) and the key range, then the item's tiles ----
     int gt = 0;
     for (int it = blockIdx.x, j = 0; it < n_items; it += gridDim.x, ++j) {
       const int hb = j & 1;
-      const int split = it % p.n_splits, bq = it / p.n_splits;
+      const bool is_chunk = it >= n_loc_items;
+      const int i2 = is_chunk ? it - n_loc_items : it;
+      const int ns = is_chunk ? p.n_chunk_splits : p.n_loc_splits;
+      const int split = i2 % ns, bq = i2 / ns;
       const int b = bq / p.n_tgroups, t0 = (bq % p.n_tgroups) * MT;
       const int nt = min(MT, p.q_tokens - t0);
       if (j >= 2) mbar_wait(&hempty[hb], ((j >> 1) - 1) & 1);  // item j-2's header and query read
+      int L = p.loc_len[b];
+      L = max(0, min(L, p.t_loc_max));
+      int* hd = hdr + hb * 8;
+      if (lane == 0) {
+        hd[0] = b; hd[1] = t0; hd[2] = nt; hd[3] = L;
+        const uint32_t qbytes = (uint32_t)(nt * p.n_q * D * 2);
+        mbar_arrive_expect_tx(&hfull[hb], qbytes);  // releases the header writes above
+        bulk_load(qsm + hb * q_elems, p.q + ((size_t)b * p.q_tokens + t0) * p.n_q * D, qbytes, &hfull[hb]);
+      }
+      if (is_chunk && !waited) {
+        pdl_enter();
+        waited = true;
+      }
       int* seg_v = segs + hb * (2 * kMaxK + 2);  // [k + 1] virtual starts
       int* seg_c = seg_v + kMaxK + 2;            // [k] chunk starts
-      for (int r = lane; r < k; r += 32) {
+      for (int r = lane; r < (is_chunk ? k : 0); r += 32) {
         const int doc = p.topk_idx[(size_t)b * k + r];
         int c0 = 0, n = 0;
         if (doc >= 0 && doc < p.n_docs) {
-          c0 = __ldg(&p.chunk_off[doc]);
-          n = __ldg(&p.chunk_off[doc + 1]) - c0;
+          c0 = p.co_cap ? co_sm[doc] : __ldg(&p.chunk_off[doc]);
+          n = (p.co_cap ? co_sm[doc + 1] : __ldg(&p.chunk_off[doc + 1])) - c0;
         } else {
           raise_dev_error(kDevErrBadIndex);
         }
         seg_c[r] = c0;
         seg_v[r + 1] = n;
       }
-      int L = p.loc_len[b];
-      L = max(0, min(L, p.t_loc_max));
       __syncwarp();
-      {  // inclusive scan of chunk counts -> virtual starts (lane owns a run of entries)
+      if (is_chunk) {  // inclusive scan of chunk counts -> virtual starts (lane owns a run of entries)
         const int per = (k + 31) / 32;
         int local = 0;
         for (int q = 0; q < per; ++q) {
@@ -207,19 +246,17 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
         if (lane == 0) seg_v[0] = 0;
       }
       __syncwarp();
-      const int n_sel = seg_v[k];
-      const int n_keys = n_sel + (p.phase == 2 ? 0 : L);
-      int per_split = (n_keys + p.n_splits - 1) / p.n_splits;
-      per_split = (per_split + kTK - 1) / kTK * kTK;
-      const int v0 = min(n_keys, split * per_split);
-      const int v1 = min(n_keys, v0 + per_split);
+      // a chunk item covers a run of the selected chunks (virtual keys 0 .. n_sel), a local
+      // item a run of the local keys (virtual keys 0 .. L with n_sel = 0)
+      const int n_sel = is_chunk ? seg_v[k] : 0;
+      const int n_keys = is_chunk ? n_sel : L;
+      const int v0 = (int)(((long long)split * n_keys) / ns);  // an even share of the keys
+      const int v1 = (int)(((long long)(split + 1) * n_keys) / ns);
       const int n_tiles = (v1 - v0 + kTK - 1) / kTK;
       if (lane == 0) {
-        int* hd = hdr + hb * 8;
-        hd[0] = b; hd[1] = t0; hd[2] = nt; hd[3] = L; hd[4] = n_sel; hd[5] = v0; hd[6] = v1; hd[7] = split;
-        const uint32_t qbytes = (uint32_t)(nt * p.n_q * D * 2);
-        mbar_arrive_expect_tx(&hfull[hb], qbytes);  // releases the header writes above
-        bulk_load(qsm + hb * q_elems, p.q + ((size_t)b * p.q_tokens + t0) * p.n_q * D, qbytes, &hfull[hb]);
+        hd[4] = n_sel; hd[5] = v0; hd[6] = v1;
+        hd[7] = is_chunk ? p.chunk_part_base + split : split;  // the item's partial slot
+        mbar_arrive(&hsel[hb]);  // releases the key-range writes
       }
       // ---- the item's tiles: kTK keys each, a bulk copy per key and tensor plus the RoPE rows ----
       for (int t = 0; t < n_tiles; ++t, ++gt) {
@@ -260,6 +297,7 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
         }
       }
     }
+    if (!waited) pdl_enter();  // the grid completes only after its predecessor
     return;  // the compute warps no longer synchronise with the whole block
   }
 
@@ -270,8 +308,7 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
     const int hb = j & 1;
     mbar_wait(&hfull[hb], (j >> 1) & 1);
     const int* hd = hdr + hb * 8;
-    const int b = hd[0], t0 = hd[1], nt = hd[2], L = hd[3], n_sel = hd[4], v0 = hd[5], v1 = hd[6], split = hd[7];
-    const int n_tiles = (v1 - v0 + kTK - 1) / kTK;
+    const int b = hd[0], t0 = hd[1], nt = hd[2], L = hd[3];
     const uint16_t* qsm_b = qsm + hb * q_elems;
     // ---- query fragments of this warp's GQA group: mma row = tt * G + gg (token t0 + tt,
     //      q head h * G + gg); token t sits at pos_offset + L - M + t; scale, bf16 ----
@@ -316,6 +353,13 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
     }
 
 
+    if (it >= n_loc_items && !waited) {  // the first selected-chunk item: its fragments are ready
+      pdl_enter();
+      waited = true;
+    }
+    mbar_wait(&hsel[hb], (j >> 1) & 1);
+    const int n_sel = hd[4], v0 = hd[5], v1 = hd[6], part = hd[7];
+    const int n_tiles = (v1 - v0 + kTK - 1) / kTK;
     __syncwarp();
     if (lane == 0) mbar_arrive(&hempty[hb]);  // header and query rows read: the buffer may refill
 
@@ -459,7 +503,7 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
       const int tt = row / G;
       if (tt < nt) {
         const size_t qh = ((size_t)b * p.q_tokens + t0 + tt) * p.n_q + (size_t)h * G + (row - tt * G);
-        const size_t ps = qh * p.n_splits_total + p.split_base + split;
+        const size_t ps = qh * p.n_parts + part;
         float* po = p.part_o + ps * D;
   #pragma unroll
         for (int n = 0; n < NBLK; ++n)
@@ -471,6 +515,7 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
       }
     }
   }
+  if (!waited) pdl_enter();  // the grid completes only after its predecessor
 }
 
 // log-sum-exp merge of the split partials of one (query, q head).  Warp w sums the splits
@@ -480,16 +525,33 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
                                                            const float* __restrict__ part_o, int n_splits,
                                                            __nv_bfloat16* __restrict__ out) {
   constexpr int PER = D / 32;
+  constexpr int kHold = 24;  // partial rows per warp loaded before the weights are known
   __shared__ float w_s[kMaxSplits];
   __shared__ float red[2][8];
   __shared__ float osum[8][D];
-  pdl_launch_dependents();
-  pdl_wait();
+  pdl_enter();
   const size_t qh = (size_t)blockIdx.y * gridDim.x + blockIdx.x;  // b * n_q + head
   const float* ml = part_ml + qh * n_splits * 2;
+  const float* po = part_o + qh * n_splits * D + (threadIdx.x & 31) * PER;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // every load in flight at once: the (m, l) pairs and this warp's first kHold partial rows
+  // (warp w takes splits w, w + 8, ...)
+  float hold[kHold][PER];
+#pragma unroll
+  for (int i = 0; i < kHold; ++i) {
+    const int sp = warp + 8 * i;
+    if (sp < n_splits) {
+      if constexpr (PER == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(po + (size_t)sp * D);
+        hold[i][0] = v.x; hold[i][1] = v.y; hold[i][2] = v.z; hold[i][3] = v.w;
+      } else {
+        const float2 v = *reinterpret_cast<const float2*>(po + (size_t)sp * D);
+        hold[i][0] = v.x; hold[i][1] = v.y;
+      }
+    }
+  }
   float m = -INFINITY;
-  for (int s = tid; s < n_splits; s += blockDim.x) m = fmaxf(m, ml[2 * s]);
+  for (int sp = tid; sp < n_splits; sp += blockDim.x) m = fmaxf(m, ml[2 * sp]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if (lane == 0) red[0][warp] = m;
@@ -499,10 +561,10 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
   for (int w = 1; w < 8; ++w) M = fmaxf(M, red[0][w]);
   const float Mu = (M == -INFINITY) ? 0.f : M;
   float l = 0.f;
-  for (int s = tid; s < n_splits; s += blockDim.x) {
-    const float w = exp2f(ml[2 * s] - Mu);
-    w_s[s] = w;
-    l += w * ml[2 * s + 1];
+  for (int sp = tid; sp < n_splits; sp += blockDim.x) {  // (m, l) are L1 hits by now
+    const float w = exp2f(ml[2 * sp] - Mu);
+    w_s[sp] = w;
+    l += w * ml[2 * sp + 1];
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
@@ -511,18 +573,26 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
   float Ls = 0.f;
 #pragma unroll
   for (int w = 0; w < 8; ++w) Ls += red[1][w];
-  const float* po = part_o + qh * n_splits * D + lane * PER;
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+#pragma unroll
+  for (int i = 0; i < kHold; ++i) {
+    const int sp = warp + 8 * i;
+    if (sp < n_splits) {
+      const float w = w_s[sp];
+#pragma unroll
+      for (int e = 0; e < PER; ++e) acc[e] += w * hold[i][e];
+    }
+  }
 #pragma unroll 4
-  for (int s = warp; s < n_splits; s += 8) {
-    const float w = w_s[s];
+  for (int sp = warp + 8 * kHold; sp < n_splits; sp += 8) {  // splits past the held rows
+    const float w = w_s[sp];
     if constexpr (PER == 4) {
-      const float4 v = *reinterpret_cast<const float4*>(po + (size_t)s * D);
+      const float4 v = *reinterpret_cast<const float4*>(po + (size_t)sp * D);
       acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
     } else {
-      const float2 v = *reinterpret_cast<const float2*>(po + (size_t)s * D);
+      const float2 v = *reinterpret_cast<const float2*>(po + (size_t)sp * D);
       acc[0] += w * v.x; acc[1] += w * v.y;
     }
   }
@@ -537,11 +607,11 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
   }
 }
 
-int stages_that_fit(int n_kv, int n_q, int D, bool table, int mt) {
+int stages_that_fit(int n_kv, int n_q, int D, bool table, int mt, int co_cap) {
   const int budget = 224 * 1024;
   for (int st = kMaxStages; st >= 2; --st) {
     AttnSmem L(n_kv, D, st, table);
-    if (L.total(n_q, D, mt) <= (size_t)budget) return st;
+    if (L.total(n_q, D, mt, co_cap) <= (size_t)budget) return st;
   }
   return 2;
 }
@@ -553,8 +623,7 @@ int tokens_per_cta(const msa_dims& d, int M) { return std::max(1, std::min(M, 16
 template <int D>
 __global__ void __launch_bounds__(256) rope_rows_kernel(__nv_bfloat16* __restrict__ x, int rows, int heads,
                                                         const int32_t* __restrict__ pos, const RopeTurns turns) {
-  pdl_launch_dependents();
-  pdl_wait();
+  pdl_enter();
   const int64_t n = (int64_t)rows * heads * (D / 2);
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
     const int i = (int)(e % (D / 2));
@@ -577,8 +646,7 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const __nv_bfloat16* __r
                                                         __nv_bfloat16* __restrict__ V_loc, int n_kv, int t_loc_max,
                                                         const int32_t* __restrict__ slots, int pos_offset,
                                                         const RopeTurns turns) {
-  pdl_launch_dependents();
-  pdl_wait();
+  pdl_enter();
   const int b = blockIdx.x;
   const int slot = slots[b];
   if (slot < 0 || slot >= t_loc_max) {
@@ -630,8 +698,7 @@ __global__ void __launch_bounds__(1024) gather_plan_kernel(const int32_t* __rest
                                                            int32_t* __restrict__ stage_idx) {
   __shared__ int cnt[1024];
   __shared__ int carry;
-  pdl_launch_dependents();
-  pdl_wait();
+  pdl_enter();
   if (threadIdx.x == 0) carry = 0;
   __syncthreads();
   for (int base = 0; base < n_sel; base += blockDim.x) {
@@ -679,8 +746,7 @@ __global__ void __launch_bounds__(256) gather_copy_kernel(const uint4* __restric
                                                           const int32_t* __restrict__ stage_src, int n_sel,
                                                           int row_vec, uint4* __restrict__ K_stage,
                                                           uint4* __restrict__ V_stage) {
-  pdl_launch_dependents();
-  pdl_wait();
+  pdl_enter();
   const int total_rows = stage_off[n_sel];
   const int64_t n = (int64_t)total_rows * row_vec;  // 16-byte vectors
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -726,13 +792,20 @@ size_t attend_workspace(const msa_dims& d, int B, int M, int k, int t_loc_max, i
   AttendWs w{};
   const int mt = tokens_per_cta(d, M);
   const int n_tg = (M + mt - 1) / mt;
-  w.n_splits = choose_splits(B * n_tg, t_loc_max, k);
-  // the two-phase call: at least 64 local keys and about 32 selected-chunk keys per split
-  // (the selection's size is known only on the device), about two waves each
-  const int waves2 = std::max(1, (2 * sm_count() + B * n_tg - 1) / (B * n_tg));
-  w.n_split_local = std::max(1, std::min({waves2, (t_loc_max + 63) / 64, kMaxSplits / 2}));
-  w.n_split_chunk = std::max(1, std::min({waves2, 2 * k, kMaxSplits / 2}));
-  w.n_parts = std::max(w.n_splits, w.n_split_local + w.n_split_chunk);
+  // splits per (query, token group): a total that makes the item count a whole number of
+  // waves, shared between the local keys and the selected chunks in proportion to their
+  // expected key counts (the selection's size is known only on the device: about
+  // kChunksPerDocEst chunks per selected document), each side at least one split
+  const int n_total = std::max(2, choose_splits(B * n_tg, t_loc_max, k));
+  const double sel_est = (double)kChunksPerDocEst * k;
+  int n_chunk = (int)std::lround(n_total * sel_est / (sel_est + std::max(0, t_loc_max)));
+  // one wave or less (few queries: latency): the selected chunks, which wait for the routing,
+  // in splits of at most two 16-key tiles
+  if ((long long)n_total * B * n_tg <= sm_count()) n_chunk = std::max(n_chunk, (int)std::ceil(sel_est / 32.0));
+  n_chunk = std::max(1, std::min({n_chunk, 2 * k, n_total - 1}));
+  w.n_split_chunk = n_chunk;
+  w.n_split_local = std::max(1, std::min(n_total - n_chunk, std::max(1, (t_loc_max + kTK - 1) / kTK)));
+  w.n_parts = w.n_split_local + w.n_split_chunk;
   w.rope_tab = cv.take<float2>((size_t)std::max(1, t_loc_max) * (d.head_dim / 2));
   w.part_ml = cv.take<float>((size_t)B * M * d.n_q * w.n_parts * 2);
   w.part_o = cv.take<float>((size_t)B * M * d.n_q * w.n_parts * d.head_dim);
@@ -808,8 +881,8 @@ msa_status kv_append_launch(const msa_dims& d, const void* k_new, const void* v_
 msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const void* K_bar, const void* V_bar,
                          const int32_t* chunk_off, int n_docs, const int32_t* topk_idx, int k, const void* K_loc,
                          const void* V_loc, const int32_t* loc_len, int t_loc_max, int pos_offset,
-                         const void* rope_cache, int k_loc_rotated, float scale, int phase, void* out, void* ws,
-                         cudaStream_t s) {
+                         const void* rope_cache, int k_loc_rotated, float scale, int phase, int early, void* out,
+                         void* ws, cudaStream_t s) {
   AttendWs w;
   attend_workspace(d, B, M, k, t_loc_max, pos_offset, ws, &w);
   const int D = d.head_dim;
@@ -838,23 +911,32 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
   p.n_docs = n_docs;
   p.t_loc_max = t_loc_max;
   p.pos_offset = pos_offset;
-  p.phase = phase;
-  p.n_splits = phase == 0 ? w.n_splits : phase == 1 ? w.n_split_local : w.n_split_chunk;
-  p.split_base = phase == 2 ? w.n_split_local : 0;
-  p.n_splits_total = phase == 0 ? w.n_splits : w.n_split_local + w.n_split_chunk;
+  p.n_loc_splits = phase == 2 ? 0 : w.n_split_local;
+  p.n_chunk_splits = phase == 1 ? 0 : w.n_split_chunk;
+  p.chunk_part_base = w.n_split_local;
+  p.n_parts = w.n_parts;
+  // the local-key items may start before the predecessor finishes only if this call launches
+  // nothing before them (no rotation table built here)
+  p.early = early && phase != 2 && (k_loc_rotated || rope_cache || t_loc_max == 0);
   p.n_queries = B;
   p.q_tokens = M;
   p.tok_per_cta = tokens_per_cta(d, M);
   p.n_tgroups = (M + p.tok_per_cta - 1) / p.tok_per_cta;
   p.scale_log2 = (scale > 0.f ? scale : 1.0f / std::sqrt((float)D)) * kLog2e;
   rope_turns(d, p.turns.f);
-  p.n_stages = stages_that_fit(d.n_kv, d.n_q, D, tab != nullptr, p.tok_per_cta);
+  // the document table goes to shared memory when it is small and costs no pipeline stage
+  p.co_cap = 0;
+  if (phase != 1 && n_docs + 1 <= kCoSmemMax) {
+    const int st0 = stages_that_fit(d.n_kv, d.n_q, D, tab != nullptr, p.tok_per_cta, 0);
+    if (stages_that_fit(d.n_kv, d.n_q, D, tab != nullptr, p.tok_per_cta, n_docs + 1) == st0) p.co_cap = n_docs + 1;
+  }
+  p.n_stages = stages_that_fit(d.n_kv, d.n_q, D, tab != nullptr, p.tok_per_cta, p.co_cap);
   {
     TraceScope ts(kKAttnSplit, s);
     // persistent: each CTA takes items (split, query, token group) in turn
-    const int n_items = p.n_splits * B * p.n_tgroups;
+    const int n_items = (p.n_loc_splits + p.n_chunk_splits) * B * p.n_tgroups;
     dim3 grid(std::max(1, std::min(n_items, sm_count())));
-    const size_t sm = AttnSmem(d.n_kv, D, p.n_stages, tab != nullptr).total(d.n_q, D, p.tok_per_cta);
+    const size_t sm = AttnSmem(d.n_kv, D, p.n_stages, tab != nullptr).total(d.n_q, D, p.tok_per_cta, p.co_cap);
     if (D == 128) {
       MSA_CUDA_CHECK(cudaFuncSetAttribute(attn_split_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
       MSA_CUDA_CHECK(launch_pdl(attn_split_kernel<128>, grid, dim3(32 * (d.n_kv + 1)), sm, s, p));
@@ -869,10 +951,10 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
     if (D == 128)
       MSA_CUDA_CHECK(launch_pdl(attn_combine_kernel<128>, grid, dim3(256), 0, s, (const float*)w.part_ml,
-                                (const float*)w.part_o, p.n_splits_total, o));
+                                (const float*)w.part_o, p.n_parts, o));
     else
       MSA_CUDA_CHECK(launch_pdl(attn_combine_kernel<64>, grid, dim3(256), 0, s, (const float*)w.part_ml,
-                                (const float*)w.part_o, p.n_splits_total, o));
+                                (const float*)w.part_o, p.n_parts, o));
   }
   return MSA_OK;
 }

@@ -123,8 +123,7 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
     fence_mbar_init();
   }
   __syncthreads();
-  pdl_launch_dependents();
-  pdl_wait();
+  pdl_enter();
 
   if (warp == kAuxCompute) {
     // ------------------------- producer -------------------------

@@ -330,9 +330,18 @@ namespace msa {
 // programmatic dependent launch: a kernel launched with programmatic stream
 // serialization may start while its predecessor drains; it must call
 // pdl_wait() before touching global memory the predecessor reads or writes.
+// Every kernel of the library waits for its predecessor BEFORE it lets its own
+// dependent start (pdl_enter).  So when a library kernel starts, the kernel
+// before it has passed its wait and everything earlier on the stream has
+// completed: a kernel may read before its own wait whatever its immediate
+// predecessor does not write (the scan's first key tiles).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_enter() {
+  pdl_wait();
+  pdl_launch_dependents();
+}
 }  // namespace msa
 
 namespace msa {

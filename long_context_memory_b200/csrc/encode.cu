@@ -401,8 +401,7 @@ __global__ void __launch_bounds__(256) chunk_off_extend_kernel(int32_t* __restri
                                                                int n_chunks_old,
                                                                const int32_t* __restrict__ chunk_off_new,
                                                                int n_docs_new) {
-  pdl_launch_dependents();
-  pdl_wait();
+  pdl_enter();
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i <= n_docs_new; i += gridDim.x * blockDim.x)
     chunk_off[n_docs_old + i] = n_chunks_old + chunk_off_new[i];
 }

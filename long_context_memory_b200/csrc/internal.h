@@ -158,7 +158,7 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
                          const int32_t* chunk_off, int n_docs, const int32_t* topk_idx, int k,
                          const void* K_loc, const void* V_loc, const int32_t* loc_len, int t_loc_max,
                          int pos_offset, const void* rope_cache, int k_loc_rotated, float scale, int phase,
-                         void* out, void* ws, cudaStream_t s);
+                         int early, void* out, void* ws, cudaStream_t s);
 msa_status gather_kv_launch(const msa_dims& d, const void* K_host, const void* V_host, const int32_t* chunk_off,
                             int n_docs, const int32_t* topk_idx, int B, int k, void* K_stage, void* V_stage,
                             int capacity_chunks, int32_t* stage_off, int32_t* stage_idx, int32_t* stage_src,

@@ -356,7 +356,10 @@ msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, int
     return fail(MSA_ERR_INVALID_ARG, "positions must lie in [0, 2^24)");
   if (!(softmax_scale >= 0.f) || !std::isfinite(softmax_scale))
     return fail(MSA_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
-  if (phase < 0 || phase > 2) return fail(MSA_ERR_INVALID_ARG, "phase must be 0, 1 or 2 (got %d)", phase);
+  const int early = (phase & MSA_ATTEND_EARLY_LOCAL) != 0;
+  phase &= ~MSA_ATTEND_EARLY_LOCAL;
+  if (phase < 0 || phase > 2)
+    return fail(MSA_ERR_INVALID_ARG, "phase must be 0, 1 or 2, optionally | MSA_ATTEND_EARLY_LOCAL (got %d)", phase);
   CHECK_PTR(q);
   if (phase != 1) {  // the selected chunks
     CHECK_PTR(K_bar);
@@ -377,7 +380,7 @@ msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, int
     return fail(MSA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
   if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
   return attend_launch(*dims, q, B, q_tokens, K_bar, V_bar, chunk_off, n_docs, topk_idx, k, K_loc, V_loc, loc_len, t_loc_max,
-                       pos_offset, rope_cache, k_loc_rotated, softmax_scale, phase, out, ws,
+                       pos_offset, rope_cache, k_loc_rotated, softmax_scale, phase, early, out, ws,
                        static_cast<cudaStream_t>(stream));
 }
 

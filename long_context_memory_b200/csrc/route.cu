@@ -104,8 +104,7 @@ __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
     size_t n_clear, uint32_t* __restrict__ scan_ticket) {
   extern __shared__ __align__(16) uint8_t rq_smem[];
   __shared__ float wsum[kRqThreads / 32];
-  pdl_launch_dependents();
-  pdl_wait();
+  pdl_enter();
   const int NR = n_r * d_r;
   const int rank = blockIdx.x, h = blockIdx.y;  // the cluster spans blockIdx.x
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -204,8 +203,7 @@ __global__ void __launch_bounds__(kRqThreads) router_query_direct_kernel(
     const __nv_bfloat16* __restrict__ Hq, int B, int b_pad, int n_r, int d_r, int nq, __nv_bfloat16* __restrict__ q_hl,
     uint32_t* __restrict__ clear, size_t n_clear, uint32_t* __restrict__ scan_ticket) {
   __shared__ float invn[kRqThreads / 32];
-  pdl_launch_dependents();
-  pdl_wait();
+  pdl_enter();
   rq_clear(clear, n_clear, scan_ticket);
   const int NR = n_r * d_r, h = blockIdx.y;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -298,10 +296,10 @@ struct ScanGeom {
 };
 
 // The scan's epilogue for one warp: TMEM lane quarter q4 (32 rows of every tile) and the QW
-// queries q_off .. q_off + QW - 1.  Per tile: wait for the tile's MMA (and its norms), read each
-// head's accumulator columns (the hi and lo halves of this warp's queries) and release them, find
-// each row's document, and fold each document segment's maximum into doc_key (or store the chunk
-// scores for the mean).  A warp whose queries are all past q_count still takes part in the
+// queries q_off .. q_off + QW - 1.  Per tile: find each row's document (while the tile streams),
+// wait for the tile's MMA (and its norms), read each head's accumulator columns (the hi and lo
+// halves of this warp's queries) and release them, and fold each document segment's maximum into
+// doc_key (or store the chunk scores for the mean).  A warp whose queries are all past q_count still takes part in the
 // barrier protocol but does no work.
 template <int DR, int NQ, bool MEAN, int QW>
 __device__ __forceinline__ void scan_epilogue(const ScanParams& p, int q4, int q_off, int lane, int t_begin, int n_lt,
@@ -317,6 +315,43 @@ __device__ __forceinline__ void scan_epilogue(const ScanParams& p, int q4, int q
     const int nbuf = lt & 1;                                    // norm buffer
     const int buf = lt % Gm::kBufs, use = lt / Gm::kBufs;      // TMEM buffer
     const int jrow = tile * kScanM + row;
+    // documents of this warp's 32 rows, found before the accumulators are ready (they depend
+    // on the tile alone): a warp-wide 32-ary search for the first row's document, then one
+    // lookahead of 32 document boundaries (32 consecutive rows cross at most 31 of them)
+    const int j = tile * kScanM + row;
+    const int j0 = tile * kScanM + 32 * q4;
+    int doc = -1;
+    if (active && j0 < p.n_chunks) {
+      int lo = cur, hi = p.n_docs;  // answer in [lo, hi): largest d with chunk_off[d] <= j0
+      while (hi - lo > 1) {
+        const int step = (hi - lo + 31) >> 5;
+        const int probe = lo + lane * step;
+        const bool ok = probe < hi && __ldg(&p.chunk_off[probe]) <= j0;
+        const unsigned m = __ballot_sync(0xffffffffu, ok);
+        const int L = 31 - __clz(m);  // lane 0 always qualifies (chunk_off[lo] <= j0)
+        lo = lo + L * step;
+        hi = min(hi, lo + step);
+      }
+      const int d0 = lo;
+      const int bi = d0 + 1 + lane;
+      const int bnd = bi <= p.n_docs ? __ldg(&p.chunk_off[bi]) : 0x7fffffff;
+#pragma unroll 4
+      for (int r = 0; r < 32; ++r) {
+        const unsigned m = __ballot_sync(0xffffffffu, bnd <= j0 + r);
+        if (lane == r) doc = d0 + __popc(m);
+      }
+      if (j >= p.n_chunks) doc = -1;
+      cur = d0;
+    }
+    const int prev = __shfl_up_sync(0xffffffffu, doc, 1);
+    const bool head = (lane == 0) || (prev != doc);
+    // the document pattern is the same for every query: which shuffle partners share my document
+    uint32_t same = 0;
+#pragma unroll
+    for (int e = 0; e < 5; ++e) {
+      const int od = __shfl_down_sync(0xffffffffu, doc, 1 << e);
+      if (lane + (1 << e) < 32 && od == doc) same |= 1u << e;
+    }
     float invg[8];  // precomputed inverse norms of this row (loads in flight during the waits)
     if (p.inv_norm) {
 #pragma unroll
@@ -362,43 +397,6 @@ __device__ __forceinline__ void scan_epilogue(const ScanParams& p, int q4, int q
     if (lane == 0 && !p.inv_norm) mbar_arrive(&nempty[nbuf]);
     if (!active) continue;
 
-    // documents of this warp's 32 rows: a warp-wide 32-ary search for the first row's
-    // document, then one lookahead of 32 document boundaries (32 consecutive rows cross at
-    // most 31 of them)
-    const int j = tile * kScanM + row;
-    const int j0 = tile * kScanM + 32 * q4;
-    int doc = -1;
-    if (j0 < p.n_chunks) {
-      int lo = cur, hi = p.n_docs;  // answer in [lo, hi): largest d with chunk_off[d] <= j0
-      while (hi - lo > 1) {
-        const int step = (hi - lo + 31) >> 5;
-        const int probe = lo + lane * step;
-        const bool ok = probe < hi && __ldg(&p.chunk_off[probe]) <= j0;
-        const unsigned m = __ballot_sync(0xffffffffu, ok);
-        const int L = 31 - __clz(m);  // lane 0 always qualifies (chunk_off[lo] <= j0)
-        lo = lo + L * step;
-        hi = min(hi, lo + step);
-      }
-      const int d0 = lo;
-      const int bi = d0 + 1 + lane;
-      const int bnd = bi <= p.n_docs ? __ldg(&p.chunk_off[bi]) : 0x7fffffff;
-#pragma unroll 4
-      for (int r = 0; r < 32; ++r) {
-        const unsigned m = __ballot_sync(0xffffffffu, bnd <= j0 + r);
-        if (lane == r) doc = d0 + __popc(m);
-      }
-      if (j >= p.n_chunks) doc = -1;
-      cur = d0;
-    }
-    const int prev = __shfl_up_sync(0xffffffffu, doc, 1);
-    const bool head = (lane == 0) || (prev != doc);
-    // the document pattern is the same for every query: which shuffle partners share my document
-    uint32_t same = 0;
-#pragma unroll
-    for (int e = 0; e < 5; ++e) {
-      const int od = __shfl_down_sync(0xffffffffu, doc, 1 << e);
-      if (lane + (1 << e) < 32 && od == doc) same |= 1u << e;
-    }
 #pragma unroll
     for (int bb = 0; bb < QW; ++bb) {
       const int b = q_off + bb;
@@ -476,30 +474,45 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t buf_cols = (uint32_t)n_r * Gm::kCols;
-  pdl_launch_dependents();
-  pdl_wait();
+  // stage it = (tile, head): the head's 128 x DR key rows, then the head's query rows (hi, lo)
+  auto load_keys = [&](int it) {
+    const int tile = t_begin + it / n_r, h = it % n_r, st = it % S;
+    uint8_t* k_s = stages + st * Gm::kStageBytes;
+    mbar_arrive_expect_tx(&full[st], Gm::kStageBytes);  // the query rows' bytes included
+#pragma unroll
+    for (int j = 0; j < Gm::kHalves; ++j) {
+      if (p.head_major)
+        tma_load_3d(k_s + j * Gm::kKBox, &kr_map, &full[st], j * 64, tile * kScanM, h);
+      else
+        tma_load_2d(k_s + j * Gm::kKBox, &kr_map, &full[st], h * DR + j * 64, tile * kScanM);
+    }
+  };
+  auto load_query = [&](int it) {
+    const int h = it % n_r, st = it % S;
+    uint8_t* q_s = stages + st * Gm::kStageBytes + Gm::kKBytes;
+#pragma unroll
+    for (int j = 0; j < Gm::kHalves; ++j)
+#pragma unroll
+      for (int hl = 0; hl < 2; ++hl)
+        tma_load_2d(q_s + (j * 2 + hl) * Gm::kQBox, &q_map, &full[st], j * 64, ((p.pass * n_r + h) * 2 + hl) * NQ);
+  };
+  // The previous kernel of this call (the router query, or the previous pass) does not write
+  // K̄^R, and it started this grid only after its own wait, so whatever wrote K̄^R has
+  // completed: the first ring's key tiles stream in while the router query finishes.
+  const int n_pre = min(S, n_it);
+  if (warp == 0 && lane == 0)
+    for (int it = 0; it < n_pre; ++it) load_keys(it);
+  pdl_enter();
 
   if (warp == 0) {
     // ------------------------- TMA producer -------------------------
     if (lane == 0) {
       for (int it = 0; it < n_it; ++it) {
-        const int tile = t_begin + it / n_r, h = it % n_r;
-        const int st = it % S;
-        if (it >= S) mbar_wait(&empty[st], ((it / S) - 1) & 1);
-        uint8_t* k_s = stages + st * Gm::kStageBytes;
-        uint8_t* q_s = k_s + Gm::kKBytes;
-        mbar_arrive_expect_tx(&full[st], Gm::kStageBytes);
-#pragma unroll
-        for (int j = 0; j < Gm::kHalves; ++j) {
-          if (p.head_major)
-            tma_load_3d(k_s + j * Gm::kKBox, &kr_map, &full[st], j * 64, tile * kScanM, h);
-          else
-            tma_load_2d(k_s + j * Gm::kKBox, &kr_map, &full[st], h * DR + j * 64, tile * kScanM);
-#pragma unroll
-          for (int hl = 0; hl < 2; ++hl)
-            tma_load_2d(q_s + (j * 2 + hl) * Gm::kQBox, &q_map, &full[st], j * 64,
-                        ((p.pass * n_r + h) * 2 + hl) * NQ);
+        if (it >= n_pre) {
+          if (it >= S) mbar_wait(&empty[it % S], ((it / S) - 1) & 1);
+          load_keys(it);
         }
+        load_query(it);
       }
     }
   } else if (warp == 1) {
@@ -599,12 +612,190 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
 // --------------------------------------------------------------------------
 // exact block-wide top-k of distinct 64-bit keys in shared memory
 // key = (ordered score << 32) | (0xFFFFFFFF - doc id): larger key = better,
-// equal scores prefer the lower id.  Radix select from the most significant
-// byte; it stops as soon as the k-th key's bucket is taken whole.  Writes the
-// k best keys, descending, to out[0..k); tmp holds k unsorted winners.
+// equal scores prefer the lower id; no key is 0 (the low word is at least 1),
+// so 0 serves as an empty slot.  Writes the k best keys, descending, to out[0..k).
 // --------------------------------------------------------------------------
-__device__ void block_topk(const uint64_t* keys, int n, int k, uint64_t* out, uint64_t* tmp, uint32_t* hist,
-                           uint64_t* sh_state) {
+__device__ __forceinline__ uint64_t shfl_u64(uint64_t v, int src) {
+  const uint32_t lo = __shfl_sync(0xffffffffu, (uint32_t)v, src);
+  const uint32_t hi = __shfl_sync(0xffffffffu, (uint32_t)(v >> 32), src);
+  return ((uint64_t)hi << 32) | lo;
+}
+__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int m) {
+  const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, m);
+  const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), m);
+  return ((uint64_t)hi << 32) | lo;
+}
+
+// 64 keys, element e = lane + 32 r held in x_r, sorted descending over e (bitonic sorting
+// network: in a block of `size` elements the lower element of each pair keeps the larger key
+// when the block is to end up descending, the smaller when ascending; the last block, all 64,
+// is descending).  Pairs 32 apart sit in one lane; the others are one shuffle apart.
+__device__ __forceinline__ void warp_sort64_desc(uint64_t& x0, uint64_t& x1, int lane) {
+#pragma unroll
+  for (int size = 2; size <= 64; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride == 32) {
+        const uint64_t hi = x0 > x1 ? x0 : x1, lo = x0 > x1 ? x1 : x0;
+        x0 = hi;
+        x1 = lo;
+      } else {
+        const uint64_t y0 = shfl_xor_u64(x0, stride), y1 = shfl_xor_u64(x1, stride);
+        const bool lower = (lane & stride) == 0;
+        const bool desc0 = (lane & size) == 0, desc1 = ((lane + 32) & size) == 0;
+        x0 = (lower == desc0) ? (x0 > y0 ? x0 : y0) : (x0 < y0 ? x0 : y0);
+        x1 = (lower == desc1) ? (x1 > y1 ? x1 : y1) : (x1 < y1 ? x1 : y1);
+      }
+    }
+  }
+}
+
+// the 32 largest keys of two descending lists (one key per lane each), descending: lane i
+// takes max(a_i, b_31-i), which holds the 32 largest as a bitonic sequence, and a half-cleaner
+// cascade sorts it
+__device__ __forceinline__ uint64_t warp_merge_desc(uint64_t a, uint64_t b, int lane) {
+  const uint64_t br = shfl_u64(b, 31 - lane);
+  uint64_t x = a > br ? a : br;
+#pragma unroll
+  for (int stride = 16; stride > 0; stride >>= 1) {
+    const uint64_t y = shfl_xor_u64(x, stride);
+    x = ((lane & stride) == 0) ? (x > y ? x : y) : (x < y ? x : y);
+  }
+  return x;
+}
+
+// k <= 32.  (1) Every warp keeps its k best keys sorted across its lanes and folds in 64 keys
+// at a time (a round whose keys all fall below the warp's current k-th best is skipped after
+// one vote).  (2) The warps' lists, zero-padded to 32, meet in shared memory, and each entry
+// counts the larger entries of every list (a 5-step search per sorted list).  An entry with
+// fewer than k larger entries is one of the k best overall, and that count is its rank: every
+// key above a global winner is itself among its warp's k best, and an entry outside the
+// winners sees k larger entries in some list or in total.  lists: [blockDim.x] words, and
+// blockDim.x is a multiple of 32.
+__device__ void block_topk_small(const uint64_t* keys, int n, int k, uint64_t* out, uint64_t* lists) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  uint64_t best = 0;
+  bool first = true;
+  for (int base = warp * 64; base < n; base += nw * 64) {
+    uint64_t x0 = base + lane < n ? keys[base + lane] : 0ull;
+    uint64_t x1 = base + 32 + lane < n ? keys[base + 32 + lane] : 0ull;
+    const uint64_t kth = shfl_u64(best, k - 1);
+    if (!__any_sync(0xffffffffu, x0 > kth || x1 > kth)) continue;
+    warp_sort64_desc(x0, x1, lane);
+    best = first ? x0 : warp_merge_desc(best, x0, lane);
+    first = false;
+  }
+  lists[tid] = lane < k ? best : 0ull;
+  __syncthreads();
+  const uint64_t c = lists[tid];
+  if (c != 0ull) {
+    int rank = 0;
+#pragma unroll 4
+    for (int v = 0; v < nw; ++v) {
+      const uint64_t* a = lists + v * 32;
+      int pos = 0;  // entries of list v above c: a[0 .. pos)
+#pragma unroll
+      for (int step = 16; step > 0; step >>= 1)
+        if (a[pos + step - 1] > c) pos += step;
+      if (pos == 31 && a[31] > c) pos = 32;  // all 32 entries (k = 32)
+      rank += pos;
+    }
+    if (rank < k) out[rank] = c;
+  }
+  __syncthreads();
+}
+
+// k <= 32, few candidates: (1) warp w takes keys [w n / nw, (w + 1) n / nw), at most 4 per
+// lane, and finds its m-th largest key T_w (m = ceil(k / nw); m rounds of a warp-wide max, the
+// owner lane dropping its maximum each time).  (2) T = min over warps of T_w: every warp holds m
+// keys >= T_w >= T, so at least k keys are >= T and the k best all are.  (3) The keys >= T are
+// compacted (one shared-memory atomic per warp) and each counts the larger ones, which is its
+// rank.  Returns false, having written nothing, when the split does not apply (n above 128 keys
+// per warp, a warp with fewer than m keys, m above 4) or more than kTopkMaxCand keys pass.
+constexpr int kTopkMaxCand = 256;
+__device__ bool block_topk_threshold(const uint64_t* keys, int n, int k, uint64_t* out, uint64_t* cand,
+                                     uint64_t* warp_t, uint32_t* count) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  const int m = (k + nw - 1) / nw;
+  if (m > 4 || n < m * nw || n > 128 * nw) return false;  // block-uniform
+  const int lo = warp * n / nw, hi = (warp + 1) * n / nw;  // n <= 4096: no overflow
+  if (tid == 0) *count = 0u;
+  uint64_t v[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) v[j] = lo + lane + 32 * j < hi ? keys[lo + lane + 32 * j] : 0ull;
+  const uint64_t v0 = v[0], v1 = v[1], v2 = v[2], v3 = v[3];  // kept for the compaction
+  // the lane's keys in descending order
+#define MSA_CX(a, b) { const uint64_t x_ = v[a] > v[b] ? v[a] : v[b]; v[b] = v[a] > v[b] ? v[b] : v[a]; v[a] = x_; }
+  MSA_CX(0, 1) MSA_CX(2, 3) MSA_CX(0, 2) MSA_CX(1, 3) MSA_CX(1, 2)
+#undef MSA_CX
+  uint64_t t_w = 0;
+  for (int r = 0; r < m; ++r) {
+    uint64_t x = v[0];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const uint64_t y = shfl_xor_u64(x, o);
+      x = x > y ? x : y;
+    }
+    t_w = x;
+    if (v[0] == x) {  // the owner (keys are distinct) drops its maximum
+      v[0] = v[1];
+      v[1] = v[2];
+      v[2] = v[3];
+      v[3] = 0ull;
+    }
+  }
+  if (lane == 0) warp_t[warp] = t_w;
+  __syncthreads();
+  // T: the smallest warp threshold (lane w reads warp w's, a butterfly takes the minimum)
+  uint64_t T = lane < nw ? warp_t[lane] : ~0ull;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint64_t y = shfl_xor_u64(T, o);
+    T = y < T ? y : T;
+  }
+  const bool p0 = v0 != 0ull && v0 >= T, p1 = v1 != 0ull && v1 >= T;
+  const bool p2 = v2 != 0ull && v2 >= T, p3 = v3 != 0ull && v3 >= T;
+  const unsigned b0 = __ballot_sync(0xffffffffu, p0), b1 = __ballot_sync(0xffffffffu, p1);
+  const unsigned b2 = __ballot_sync(0xffffffffu, p2), b3 = __ballot_sync(0xffffffffu, p3);
+  const int n0 = __popc(b0), n1 = __popc(b1), n2 = __popc(b2), n3 = __popc(b3);
+  uint32_t base = 0;
+  if (lane == 0 && n0 + n1 + n2 + n3 > 0) base = atomicAdd(count, (uint32_t)(n0 + n1 + n2 + n3));
+  base = __shfl_sync(0xffffffffu, base, 0);
+  const unsigned below = (1u << lane) - 1u;
+  if (p0 && base + __popc(b0 & below) < (uint32_t)kTopkMaxCand) cand[base + __popc(b0 & below)] = v0;
+  base += n0;
+  if (p1 && base + __popc(b1 & below) < (uint32_t)kTopkMaxCand) cand[base + __popc(b1 & below)] = v1;
+  base += n1;
+  if (p2 && base + __popc(b2 & below) < (uint32_t)kTopkMaxCand) cand[base + __popc(b2 & below)] = v2;
+  base += n2;
+  if (p3 && base + __popc(b3 & below) < (uint32_t)kTopkMaxCand) cand[base + __popc(b3 & below)] = v3;
+  __syncthreads();
+  const int c = (int)*count;
+  if (c > kTopkMaxCand) {
+    __syncthreads();  // every thread has read the count before the fallback reuses the scratch
+    return false;
+  }
+  // rank of each candidate among the candidates: 8 independent partial counts per step
+  for (int i = tid; i < c; i += blockDim.x) {
+    const uint64_t x = cand[i];
+    int r8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    int j = 0;
+    for (; j + 8 <= c; j += 8) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) r8[u] += cand[j + u] > x;
+    }
+    for (; j < c; ++j) r8[0] += cand[j] > x;
+    const int rank = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
+    if (rank < k) out[rank] = x;
+  }
+  __syncthreads();
+  return true;
+}
+
+// any k (up to 256): radix select from the most significant byte; it stops as soon as the
+// k-th key's bucket is taken whole; tmp holds k unsorted winners, then a rank sort
+__device__ void block_topk_radix(const uint64_t* keys, int n, int k, uint64_t* out, uint64_t* tmp, uint32_t* hist,
+                                 uint64_t* sh_state) {
   const int tid = threadIdx.x, nt = blockDim.x;
   uint64_t prefix = 0, mask = 0;
   int kk = k;
@@ -689,6 +880,26 @@ __device__ void block_topk(const uint64_t* keys, int n, int k, uint64_t* out, ui
   __syncthreads();
 }
 
+// shared memory after the keys: out[256], tmp[256], state[4] (64-bit), hist[256] (32-bit),
+// lists[kTopkThreads] (64-bit)
+struct TopkScratch {
+  uint64_t *out, *tmp, *state, *lists;
+  uint32_t* hist;
+  __device__ explicit TopkScratch(uint64_t* base) {
+    out = base;
+    tmp = out + 256;
+    state = tmp + 256;
+    hist = reinterpret_cast<uint32_t*>(state + 4);
+    lists = reinterpret_cast<uint64_t*>(hist + 256);
+  }
+};
+constexpr size_t kTopkScratchBytes = (512 + 4) * sizeof(uint64_t) + 256 * sizeof(uint32_t) + kTopkThreads * 8;
+
+__device__ void block_topk(const uint64_t* keys, int n, int k, const TopkScratch& t) {
+  if (k > 32) block_topk_radix(keys, n, k, t.out, t.tmp, t.hist, t.state);
+  else if (!block_topk_threshold(keys, n, k, t.out, t.lists, t.tmp, t.hist)) block_topk_small(keys, n, k, t.out, t.lists);
+}
+
 __device__ __forceinline__ uint64_t make_key(uint32_t ordered, int id) {
   return ((uint64_t)ordered << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)id);
 }
@@ -696,15 +907,13 @@ __device__ __forceinline__ uint64_t make_key(uint32_t ordered, int id) {
 // top-k of one slice of documents for query b (whole block): document scores from the
 // scan's max keys (or the mean of its chunk keys), written out when asked, then the block
 // top-k; with one slice the result is final, otherwise the slice's winners become
-// candidates for the merge.  sm64 holds (kSliceDocs + 516) 64-bit words + 256 words of 32 bits.
+// candidates for the merge.  sm64 holds kSliceDocs 64-bit keys, then the TopkScratch.
 __device__ void slice_topk(const uint32_t* doc_key, const uint32_t* chunk_k, const int32_t* chunk_off, int n_docs,
                            int n_chunks, int k, int n_slices, float* doc_scores, uint64_t* cand, int32_t* topk_idx,
                            float* topk_score, int slice, int b, uint64_t* sm64) {
-  uint64_t* keys = sm64;              // [kSliceDocs]
-  uint64_t* out = keys + kSliceDocs;  // [256]
-  uint64_t* tmp = out + 256;          // [256]
-  uint64_t* state = tmp + 256;        // [4]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(state + 4);
+  uint64_t* keys = sm64;  // [kSliceDocs]
+  const TopkScratch ts(keys + kSliceDocs);
+  uint64_t* out = ts.out;
   const int d0 = slice * kSliceDocs;
   const int n = min(kSliceDocs, n_docs - d0);
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
@@ -724,7 +933,7 @@ __device__ void slice_topk(const uint32_t* doc_key, const uint32_t* chunk_k, con
   }
   __syncthreads();
   const int kk = min(k, n);
-  block_topk(keys, n, kk, out, tmp, hist, state);
+  block_topk(keys, n, kk, ts);
   if (n_slices == 1) {
     for (int i = threadIdx.x; i < kk; i += blockDim.x) {
       topk_idx[(size_t)b * k + i] = (int32_t)(0xFFFFFFFFu - (uint32_t)(out[i] & 0xFFFFFFFFu));
@@ -742,8 +951,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_slice_kernel(
     int n_docs, int n_chunks, int k, int n_slices, float* __restrict__ doc_scores, uint64_t* __restrict__ cand,
     int32_t* __restrict__ topk_idx, float* __restrict__ topk_score) {
   extern __shared__ uint64_t sm64[];
-  pdl_launch_dependents();
-  pdl_wait();
+  pdl_enter();
   slice_topk(doc_key, chunk_k, chunk_off, n_docs, n_chunks, k, n_slices, doc_scores, cand, topk_idx, topk_score,
              blockIdx.x, blockIdx.y, sm64);
 }
@@ -755,16 +963,13 @@ __global__ void __launch_bounds__(kTopkThreads) topk_merge_kernel(const uint64_t
   extern __shared__ uint64_t sm64[];
   const int n = n_slices * k;
   uint64_t* keys = sm64;
-  uint64_t* out = keys + n;
-  uint64_t* tmp = out + 256;
-  uint64_t* state = tmp + 256;
-  uint32_t* hist = reinterpret_cast<uint32_t*>(state + 4);
-  pdl_launch_dependents();
-  pdl_wait();
+  const TopkScratch ts(keys + n);
+  uint64_t* out = ts.out;
+  pdl_enter();
   const int b = blockIdx.x;
   for (int i = threadIdx.x; i < n; i += blockDim.x) keys[i] = cand[(size_t)b * n + i];
   __syncthreads();
-  block_topk(keys, n, k, out, tmp, hist, state);
+  block_topk(keys, n, k, ts);
   for (int i = threadIdx.x; i < k; i += blockDim.x) {
     topk_idx[(size_t)b * k + i] = (int32_t)(0xFFFFFFFFu - (uint32_t)(out[i] & 0xFFFFFFFFu));
     topk_score[(size_t)b * k + i] = ordered_to_float((uint32_t)(out[i] >> 32));
@@ -779,17 +984,14 @@ __global__ void __launch_bounds__(kTopkThreads) topk_merge_pairs_kernel(const fl
                                                                         float* __restrict__ topk_score) {
   extern __shared__ uint64_t sm64[];
   uint64_t* keys = sm64;
-  uint64_t* out = keys + n_cand;
-  uint64_t* tmp = out + 256;
-  uint64_t* state = tmp + 256;
-  uint32_t* hist = reinterpret_cast<uint32_t*>(state + 4);
-  pdl_launch_dependents();
-  pdl_wait();
+  const TopkScratch ts(keys + n_cand);
+  uint64_t* out = ts.out;
+  pdl_enter();
   const int b = blockIdx.x;
   for (int i = threadIdx.x; i < n_cand; i += blockDim.x)
     keys[i] = make_key(float_to_ordered(cand_score[(size_t)b * n_cand + i]), cand_idx[(size_t)b * n_cand + i]);
   __syncthreads();
-  block_topk(keys, n_cand, k, out, tmp, hist, state);
+  block_topk(keys, n_cand, k, ts);
   for (int i = threadIdx.x; i < k; i += blockDim.x) {
     topk_idx[(size_t)b * k + i] = (int32_t)(0xFFFFFFFFu - (uint32_t)(out[i] & 0xFFFFFFFFu));
     topk_score[(size_t)b * k + i] = ordered_to_float((uint32_t)(out[i] >> 32));
@@ -800,6 +1002,9 @@ template <int DR, int NQ, bool MEAN>
 cudaError_t launch_scan_t(const CUtensorMap& kmap, const CUtensorMap& qmap, const ScanParams& p, int grid,
                           cudaStream_t s) {
   auto kern = scan_kernel<DR, NQ, MEAN>;
+  static_assert(kSliceDocs * sizeof(uint64_t) + kTopkScratchBytes <=
+                    (size_t)ScanGeom<DR, NQ>::kStages * ScanGeom<DR, NQ>::kStageBytes,
+                "the fused top-k reuses the pipeline stages");
   const size_t smem = ScanGeom<DR, NQ>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -824,8 +1029,7 @@ cudaError_t launch_scan(int d_r, int nq, bool mean, const CUtensorMap& kmap, con
 // each take 16 bytes (coalesced), the row's lanes reduce with shuffles
 __global__ void __launch_bounds__(256) kr_norms_kernel(const __nv_bfloat16* __restrict__ KR, int n_chunks, int n_r,
                                                        int d_r, int head_major, float* __restrict__ inv_norm) {
-  pdl_launch_dependents();
-  pdl_wait();
+  pdl_enter();
   const int L = d_r / 8;  // lanes per row (16 or 8)
   const int lane = threadIdx.x & 31;
   const int rpw = 32 / L;  // rows per warp step
@@ -850,8 +1054,8 @@ __global__ void __launch_bounds__(256) kr_norms_kernel(const __nv_bfloat16* __re
   }
 }
 
-size_t topk_slice_smem() { return (kSliceDocs + 512 + 4) * sizeof(uint64_t) + 256 * sizeof(uint32_t); }
-size_t topk_merge_smem(int n) { return ((size_t)n + 512 + 4) * sizeof(uint64_t) + 256 * sizeof(uint32_t); }
+size_t topk_slice_smem() { return kSliceDocs * sizeof(uint64_t) + kTopkScratchBytes; }
+size_t topk_merge_smem(int n) { return (size_t)n * sizeof(uint64_t) + kTopkScratchBytes; }
 
 }  // namespace
 

@@ -316,10 +316,64 @@ def test_attend_two_phase_equals_one_call(msa, cuda_device, rotated, M, B):
     torch.cuda.synchronize()
     assert msa.check_device_errors() == 0
     a, b = one.float().cpu().numpy(), out.float().cpu().numpy()
-    assert np.max(np.abs(a - b)) < 2e-2
+    assert np.array_equal(a, b)  # the same splits and partial slots as the one-launch call
     if M == 1:
         check_attention(b, _oracle(c, 5, 1e6), where=f"two-phase B={B}")
     else:
         ref = O.sparse_attend_tokens(c["q"], c["K_bar"], c["V_bar"], c["chunk_off"], c["topk"], c["K_loc"], c["V_loc"],
                                      c["loc_len"], 5, 1e6)
         check_attention(b, ref, where=f"two-phase M={M}")
+
+
+@pytest.mark.parametrize("B,M", [(1, 1), (3, 1), (2, 4)])
+def test_attend_early_local_behind_routing(msa, cuda_device, B, M):
+    # append -> route -> attend on one stream, the attention's local-key work allowed to start
+    # while the routing kernels finish: the same result, bit for bit, as the ordinary call,
+    # and the oracle's attention over the routed documents
+    import torch
+
+    rng = np.random.default_rng(700 + B + M)
+    n_q, n_kv, D, n_r, d_r, k, T_loc = 32, 8, 128, 8, 128, 16, 1024
+    lens = np.clip(rng.lognormal(np.log(2048), 0.5, size=300).astype(np.int64), 64, 32768)
+    doc_off = W.offsets_from_lengths(lens)
+    co, C = msa.chunk_offsets(doc_off)
+    dims = W.Dims(hidden=256, n_q=n_q, n_kv=n_kv, head_dim=D, n_r=n_r, d_r=d_r, rope_base=1e6)
+    dev = cuda_device
+    KR = _dev(W.normal_bf16(rng, (C, n_r, d_r)), dev)
+    K_bar_np, V_bar_np = W.normal_bf16(rng, (C, n_kv, D)), W.normal_bf16(rng, (C, n_kv, D))
+    K_loc_np, V_loc_np = W.normal_bf16(rng, (B, T_loc, n_kv, D)), W.normal_bf16(rng, (B, T_loc, n_kv, D))
+    q_np = W.normal_bf16(rng, (B, M, n_q, D)) if M > 1 else W.normal_bf16(rng, (B, n_q, D))
+    QR = _dev(W.normal_bf16(rng, (B * M, n_r * d_r)), dev)
+    loc_len_np = rng.integers(max(M, T_loc // 2), T_loc + 1, size=B).astype(np.int32)
+    K_bar, V_bar, q = _dev(K_bar_np, dev), _dev(V_bar_np, dev), _dev(q_np, dev)
+    K_loc, V_loc = _dev(K_loc_np, dev), _dev(V_loc_np, dev)
+    co_d, loc_len = torch.from_numpy(co).to(dev), torch.from_numpy(loc_len_np).to(dev)
+    o = k
+    pos = (o + torch.arange(T_loc, dtype=torch.int32, device=dev)).repeat(B)
+    msa.rope_rows(dims, K_loc.view(B * T_loc, n_kv, D), pos)
+    # the append writes the last slot of each query with its own (rotated) row: a no-op on values
+    slots = torch.from_numpy(loc_len_np - 1).to(dev)
+    kn_np = W.normal_bf16(rng, (B, n_kv, D))
+    k_new = _dev(kn_np, dev)
+    v_new = V_loc[torch.arange(B, device=dev), slots.long()].clone()
+    ws = torch.empty(msa.attend_workspace_size(dims, B, k, T_loc, o, M) + 256, dtype=torch.uint8, device=dev)
+    outs = []
+    for early in (True, False, True):
+        msa.kv_append(dims, k_new, v_new, K_loc, V_loc, slots, o)
+        idx, _, _ = msa.route_topk(dims, QR, None, KR, co_d, k, q_tokens=M)
+        out = msa.sparse_attend(dims, q, K_bar, V_bar, co_d, idx, K_loc, V_loc, loc_len, o, ws=ws,
+                                k_loc_rotated=True, early_local=early)
+        torch.cuda.synchronize()
+        assert msa.check_device_errors() == 0
+        outs.append(out.float().cpu().numpy())
+    assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[2], outs[1])
+    # the oracle, on the routed documents and the cache as appended (keys before RoPE)
+    K_loc_ref = K_loc_np.copy()
+    for b in range(B):
+        K_loc_ref[b, loc_len_np[b] - 1] = kn_np[b]
+    topk = idx.cpu().numpy()
+    if M == 1:
+        ref = O.sparse_attend(q_np, K_bar_np, V_bar_np, co, topk, K_loc_ref, V_loc_np, loc_len_np, o, 1e6)
+    else:
+        ref = O.sparse_attend_tokens(q_np, K_bar_np, V_bar_np, co, topk, K_loc_ref, V_loc_np, loc_len_np, o, 1e6)
+    check_attention(outs[0], ref, where=f"early B={B} M={M}")
