@@ -524,31 +524,23 @@ template <int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restrict__ part_ml,
                                                            const float* __restrict__ part_o, int n_splits,
                                                            __nv_bfloat16* __restrict__ out) {
-  constexpr int PER = D / 32;
-  constexpr int kHold = 24;  // partial rows per warp loaded before the weights are known
+  // CTA = (q head, query token, 32-dim slice): lane l holds dim 32 z + l of the slice; warp w
+  // sums the splits w, w + 8, ...; every CTA of a head reduces the (m, l) pairs itself
+  constexpr int kHold = 24;  // partial values per lane loaded before the weights are known
   __shared__ float w_s[kMaxSplits];
   __shared__ float red[2][8];
-  __shared__ float osum[8][D];
+  __shared__ float osum[8][32];
   pdl_enter();
-  const size_t qh = (size_t)blockIdx.y * gridDim.x + blockIdx.x;  // b * n_q + head
-  const float* ml = part_ml + qh * n_splits * 2;
-  const float* po = part_o + qh * n_splits * D + (threadIdx.x & 31) * PER;
+  const size_t qh = (size_t)blockIdx.y * gridDim.x + blockIdx.x;  // (b * M + t) * n_q + head
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // every load in flight at once: the (m, l) pairs and this warp's first kHold partial rows
-  // (warp w takes splits w, w + 8, ...)
-  float hold[kHold][PER];
+  const float* ml = part_ml + qh * n_splits * 2;
+  const float* po = part_o + qh * n_splits * D + blockIdx.z * 32 + lane;
+  // every load in flight at once: this lane's first kHold partial values and the (m, l) pairs
+  float hold[kHold];
 #pragma unroll
   for (int i = 0; i < kHold; ++i) {
     const int sp = warp + 8 * i;
-    if (sp < n_splits) {
-      if constexpr (PER == 4) {
-        const float4 v = *reinterpret_cast<const float4*>(po + (size_t)sp * D);
-        hold[i][0] = v.x; hold[i][1] = v.y; hold[i][2] = v.z; hold[i][3] = v.w;
-      } else {
-        const float2 v = *reinterpret_cast<const float2*>(po + (size_t)sp * D);
-        hold[i][0] = v.x; hold[i][1] = v.y;
-      }
-    }
+    hold[i] = sp < n_splits ? po[(size_t)sp * D] : 0.f;
   }
   float m = -INFINITY;
   for (int sp = tid; sp < n_splits; sp += blockDim.x) m = fmaxf(m, ml[2 * sp]);
@@ -573,37 +565,21 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
   float Ls = 0.f;
 #pragma unroll
   for (int w = 0; w < 8; ++w) Ls += red[1][w];
-  float acc[PER];
-#pragma unroll
-  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+  float acc = 0.f;
 #pragma unroll
   for (int i = 0; i < kHold; ++i) {
     const int sp = warp + 8 * i;
-    if (sp < n_splits) {
-      const float w = w_s[sp];
-#pragma unroll
-      for (int e = 0; e < PER; ++e) acc[e] += w * hold[i][e];
-    }
+    if (sp < n_splits) acc += w_s[sp] * hold[i];
   }
 #pragma unroll 4
-  for (int sp = warp + 8 * kHold; sp < n_splits; sp += 8) {  // splits past the held rows
-    const float w = w_s[sp];
-    if constexpr (PER == 4) {
-      const float4 v = *reinterpret_cast<const float4*>(po + (size_t)sp * D);
-      acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
-    } else {
-      const float2 v = *reinterpret_cast<const float2*>(po + (size_t)sp * D);
-      acc[0] += w * v.x; acc[1] += w * v.y;
-    }
-  }
-#pragma unroll
-  for (int e = 0; e < PER; ++e) osum[warp][lane * PER + e] = acc[e];
+  for (int sp = warp + 8 * kHold; sp < n_splits; sp += 8) acc += w_s[sp] * po[(size_t)sp * D];
+  osum[warp][lane] = acc;
   __syncthreads();
-  for (int dim = tid; dim < D; dim += blockDim.x) {
+  if (tid < 32) {
     float o = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) o += osum[w][dim];
-    out[qh * D + dim] = __float2bfloat16_rn(Ls > 0.f ? o / Ls : 0.f);
+    for (int w = 0; w < 8; ++w) o += osum[w][tid];
+    out[qh * D + blockIdx.z * 32 + tid] = __float2bfloat16_rn(Ls > 0.f ? o / Ls : 0.f);
   }
 }
 
@@ -947,7 +923,7 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
   }
   if (phase != 1) {  // the local-keys phase leaves its partials for the selected-chunks phase's combine
     TraceScope ts(kKAttnCombine, s);
-    dim3 grid(d.n_q, B * M);
+    dim3 grid(d.n_q, B * M, D / 32);
     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
     if (D == 128)
       MSA_CUDA_CHECK(launch_pdl(attn_combine_kernel<128>, grid, dim3(256), 0, s, (const float*)w.part_ml,

@@ -123,7 +123,9 @@ __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
   const int per_row = d_r / 8;              // 16-byte pieces of a W row
 
   for (int b0 = 0; b0 < b_pad; b0 += 16) {
+    // two accumulator sets (even and odd k-steps): half the dependent MMA chain
     float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     for (int p0 = 0; p0 < nrows; p0 += kRqPiece) {
       const int pr = min(kRqPiece, nrows - p0);
       __syncthreads();  // the previous piece is consumed
@@ -149,16 +151,21 @@ __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
         ldmatrix_x4(a0, a1, a2, a3, smem_u32(hsm + (size_t)(lane & 15) * hstr + (ks * 16 + 8 * (lane >> 4)) * 2));
         const int krow = ks * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
         uint32_t b0r, b1r, b2r, b3r;
+        float (*dst)[4] = (ks & 1) ? acc2 : acc;
         if (nt_per_warp == 2) {
           ldmatrix_x4_trans(b0r, b1r, b2r, b3r, smem_u32(wsm + (size_t)krow * ws + (8 * n0 + 8 * (lane >> 4)) * 2));
-          mma_bf16_16816(acc[0], a0, a1, a2, a3, b0r, b1r);
-          mma_bf16_16816(acc[1], a0, a1, a2, a3, b2r, b3r);
+          mma_bf16_16816(dst[0], a0, a1, a2, a3, b0r, b1r);
+          mma_bf16_16816(dst[1], a0, a1, a2, a3, b2r, b3r);
         } else {  // two k-halves of one n-tile (the upper lanes' rows repeat)
           ldmatrix_x4_trans(b0r, b1r, b2r, b3r, smem_u32(wsm + (size_t)krow * ws + (8 * n0) * 2));
-          mma_bf16_16816(acc[0], a0, a1, a2, a3, b0r, b1r);
+          mma_bf16_16816(dst[0], a0, a1, a2, a3, b0r, b1r);
         }
       }
     }
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[t][e] += acc2[t][e];
     // this CTA's partial product of the 16-row block: D fragment rows lane/4 (+8), columns
     // 2 (lane % 4) + {0, 1} of each n-tile
 #pragma unroll
