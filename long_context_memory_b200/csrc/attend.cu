@@ -518,29 +518,42 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
   if (!waited) pdl_enter();  // the grid completes only after its predecessor
 }
 
-// log-sum-exp merge of the split partials of one (query, q head).  Warp w sums the splits
-// s = w (mod 8); lane l holds D/32 consecutive dims; the warps' sums meet in shared memory.
-template <int D>
+// log-sum-exp merge of the split partials of one (query token, q head), or of a 32-dim slice of
+// it (SL = D / 32 slices: more CTAs when there are few queries).  Lane l holds W = D / (32 SL)
+// consecutive dims of the CTA's part; warp w sums the splits w, w + 8, ...; every CTA reduces
+// the (m, l) pairs itself and the warps' sums meet in shared memory.
+template <int D, int SL>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restrict__ part_ml,
                                                            const float* __restrict__ part_o, int n_splits,
                                                            __nv_bfloat16* __restrict__ out) {
-  // CTA = (q head, query token, 32-dim slice): lane l holds dim 32 z + l of the slice; warp w
-  // sums the splits w, w + 8, ...; every CTA of a head reduces the (m, l) pairs itself
-  constexpr int kHold = 24;  // partial values per lane loaded before the weights are known
+  constexpr int W = D / (32 * SL);          // dims per lane
+  constexpr int kHold = W == 1 ? 24 : 12;   // partial rows per lane loaded before the weights are known
   __shared__ float w_s[kMaxSplits];
   __shared__ float red[2][8];
-  __shared__ float osum[8][32];
+  __shared__ float osum[8][32 * W];
   pdl_enter();
   const size_t qh = (size_t)blockIdx.y * gridDim.x + blockIdx.x;  // (b * M + t) * n_q + head
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int d0 = blockIdx.z * 32 * W;       // this CTA's first dim
   const float* ml = part_ml + qh * n_splits * 2;
-  const float* po = part_o + qh * n_splits * D + blockIdx.z * 32 + lane;
-  // every load in flight at once: this lane's first kHold partial values and the (m, l) pairs
-  float hold[kHold];
+  const float* po = part_o + qh * n_splits * D + d0 + lane * W;
+  auto load = [&](int sp, float* v) {
+    if constexpr (W == 4) {
+      const float4 x = *reinterpret_cast<const float4*>(po + (size_t)sp * D);
+      v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+    } else if constexpr (W == 2) {
+      const float2 x = *reinterpret_cast<const float2*>(po + (size_t)sp * D);
+      v[0] = x.x; v[1] = x.y;
+    } else {
+      v[0] = po[(size_t)sp * D];
+    }
+  };
+  // every load in flight at once: this lane's first kHold partial rows and the (m, l) pairs
+  float hold[kHold][W];
 #pragma unroll
   for (int i = 0; i < kHold; ++i) {
     const int sp = warp + 8 * i;
-    hold[i] = sp < n_splits ? po[(size_t)sp * D] : 0.f;
+    if (sp < n_splits) load(sp, hold[i]);
   }
   float m = -INFINITY;
   for (int sp = tid; sp < n_splits; sp += blockDim.x) m = fmaxf(m, ml[2 * sp]);
@@ -565,21 +578,34 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
   float Ls = 0.f;
 #pragma unroll
   for (int w = 0; w < 8; ++w) Ls += red[1][w];
-  float acc = 0.f;
+  float acc[W];
+#pragma unroll
+  for (int e = 0; e < W; ++e) acc[e] = 0.f;
 #pragma unroll
   for (int i = 0; i < kHold; ++i) {
     const int sp = warp + 8 * i;
-    if (sp < n_splits) acc += w_s[sp] * hold[i];
+    if (sp < n_splits) {
+      const float w = w_s[sp];
+#pragma unroll
+      for (int e = 0; e < W; ++e) acc[e] += w * hold[i][e];
+    }
   }
 #pragma unroll 4
-  for (int sp = warp + 8 * kHold; sp < n_splits; sp += 8) acc += w_s[sp] * po[(size_t)sp * D];
-  osum[warp][lane] = acc;
+  for (int sp = warp + 8 * kHold; sp < n_splits; sp += 8) {  // splits past the held rows
+    float v[W];
+    load(sp, v);
+    const float w = w_s[sp];
+#pragma unroll
+    for (int e = 0; e < W; ++e) acc[e] += w * v[e];
+  }
+#pragma unroll
+  for (int e = 0; e < W; ++e) osum[warp][lane * W + e] = acc[e];
   __syncthreads();
-  if (tid < 32) {
+  for (int dim = tid; dim < 32 * W; dim += blockDim.x) {
     float o = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) o += osum[w][tid];
-    out[qh * D + blockIdx.z * 32 + tid] = __float2bfloat16_rn(Ls > 0.f ? o / Ls : 0.f);
+    for (int w = 0; w < 8; ++w) o += osum[w][dim];
+    out[qh * D + d0 + dim] = __float2bfloat16_rn(Ls > 0.f ? o / Ls : 0.f);
   }
 }
 
@@ -923,14 +949,15 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
   }
   if (phase != 1) {  // the local-keys phase leaves its partials for the selected-chunks phase's combine
     TraceScope ts(kKAttnCombine, s);
-    dim3 grid(d.n_q, B * M, D / 32);
+    // few query tokens: a CTA per 32-dim slice of each head (enough CTAs to fill the GPU);
+    // many: a CTA per head
+    const bool sliced = (long long)B * M * d.n_q < 2LL * sm_count();
+    dim3 grid(d.n_q, B * M, sliced ? D / 32 : 1);
     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
-    if (D == 128)
-      MSA_CUDA_CHECK(launch_pdl(attn_combine_kernel<128>, grid, dim3(256), 0, s, (const float*)w.part_ml,
-                                (const float*)w.part_o, p.n_parts, o));
-    else
-      MSA_CUDA_CHECK(launch_pdl(attn_combine_kernel<64>, grid, dim3(256), 0, s, (const float*)w.part_ml,
-                                (const float*)w.part_o, p.n_parts, o));
+    auto kern = D == 128 ? (sliced ? attn_combine_kernel<128, 4> : attn_combine_kernel<128, 1>)
+                         : (sliced ? attn_combine_kernel<64, 2> : attn_combine_kernel<64, 1>);
+    MSA_CUDA_CHECK(launch_pdl(kern, grid, dim3(256), 0, s, (const float*)w.part_ml, (const float*)w.part_o, p.n_parts,
+                              o));
   }
   return MSA_OK;
 }
