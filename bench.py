@@ -224,7 +224,8 @@ def kernel_times(msa, stream, step, n):
 
 
 def run_extras(msa, dev, hbm_peak):
-    """Routing at 16M (B=32) and 100M tokens (36 layer instances, B=1 and 16), and encoding 1M tokens."""
+    """Routing at 16M (B=32) and 100M tokens (36 layer instances, B=1 and 16), the 100M-token host tier
+    (gather + attention, B=1 and 16), and encoding 1M tokens."""
     import torch
 
     from long_context_memory_b200 import profile_cases as PC
@@ -284,6 +285,22 @@ def run_extras(msa, dev, hbm_peak):
         route_entry("mem100m_b16_route", c100, layers)
         del c100
         torch.cuda.empty_cache()
+        # host tier: one layer's K̄/V̄ (100M tokens, 6.4 GB) in pinned host memory; per step only the
+        # selected documents cross the host link, then attention over them + 8K local tokens
+        for Bh in (1, 16):
+            try:
+                ht = PC.HostTierCase(100_000_000, Bh, 4096, 8192, W.BASE_SEED + 4, dev)
+                g_ms = timed(lambda i: ht.gather(), 10)
+                a_ms = timed(lambda i: ht.attend(), 10)
+                out[f"mem100m_b{Bh}_host_tier"] = {
+                    "workload": f"100M-token memory, K̄/V̄ in pinned host memory, B={Bh}, top-{ht.k}, 8K local KV",
+                    "gather_ms": g_ms, "gathered_MB": ht.gather_bytes / 1e6,
+                    "host_link_GB/s": ht.gather_bytes / (g_ms * 1e-3) / 1e9, "attend_ms": a_ms,
+                    "attend_GB/s": ht.kv_bytes / (a_ms * 1e-3) / 1e9}
+                del ht
+            except Exception as e:  # e.g. pinned host memory unavailable: report it, keep the rest
+                out[f"mem100m_b{Bh}_host_tier"] = {"error": f"{type(e).__name__}: {e}"}
+            torch.cuda.empty_cache()
         enc = PC.EncodeCase(1_000_000, W.BASE_SEED + 5, dev)
         ms = timed(lambda i: enc.run(), 3, warm=1)
         kt = kernel_times(msa, stream, lambda i: enc.run(), 3)

@@ -142,6 +142,62 @@ class AttendCase:
                                k_loc_rotated=self.rotated)
 
 
+class HostTierCase:
+    """The host tier of a large memory: pooled K̄/V̄ in pinned host memory; per step the selected
+    documents of every query cross the host link (msa_gather_kv) into a device staging area, then
+    the attention runs over them and the local KV (rotated cache)."""
+
+    def __init__(self, T, B, median, t_loc, seed, device, k=16, dims=W.QWEN3_4B_DIMS):
+        import torch
+
+        import long_context_memory_b200 as msa
+
+        self.msa, self.d, self.B, self.k = msa, dims, B, k
+        doc_off, co, C = chunk_layout_host(T, median, seed)
+        n_docs = len(co) - 1
+        g = torch.Generator(device=device)
+        g.manual_seed(seed + 1)
+        shape = (C, dims.n_kv, dims.head_dim)
+        self.K_host = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
+        self.V_host = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
+        step = 1 << 16  # rows per device-generated slab
+        for dst in (self.K_host, self.V_host):
+            for a in range(0, C, step):
+                e = min(C, a + step)
+                dst[a:e].copy_(randn_bf16((e - a,) + shape[1:], g, device))
+        torch.cuda.synchronize()
+        self.chunk_off = torch.from_numpy(co).to(device)
+        rng = np.random.default_rng(seed)
+        sel = np.stack([rng.permutation(n_docs)[:k] for _ in range(B)]).astype(np.int32)
+        self.topk = torch.from_numpy(sel).to(device)
+        self.n_sel = sum(int(co[i + 1] - co[i]) for row in sel for i in row)
+        self.capacity = self.n_sel
+        self.stage = (torch.empty((self.capacity,) + shape[1:], dtype=torch.bfloat16, device=device),
+                      torch.empty((self.capacity,) + shape[1:], dtype=torch.bfloat16, device=device),
+                      torch.empty(B * k + 1, dtype=torch.int32, device=device),
+                      torch.empty((B, k), dtype=torch.int32, device=device))
+        self.gather_bytes = self.n_sel * dims.n_kv * dims.head_dim * 2 * 2
+        self.q = randn_bf16((B, dims.n_q, dims.head_dim), g, device)
+        self.K_loc = randn_bf16((B, t_loc, dims.n_kv, dims.head_dim), g, device)
+        self.V_loc = randn_bf16((B, t_loc, dims.n_kv, dims.head_dim), g, device)
+        self.loc_len = torch.full((B,), t_loc, dtype=torch.int32, device=device)
+        self.pos = k
+        msa.rope_rows(dims, self.K_loc.view(B * t_loc, dims.n_kv, dims.head_dim),
+                      (self.pos + torch.arange(t_loc, dtype=torch.int32, device=device)).repeat(B))
+        self.out = torch.empty((B, dims.n_q, dims.head_dim), dtype=torch.bfloat16, device=device)
+        self.ws = torch.empty(msa.attend_workspace_size(dims, B, k, t_loc, self.pos) + 256, dtype=torch.uint8,
+                              device=device)
+        self.kv_bytes = (self.n_sel + B * t_loc) * dims.n_kv * dims.head_dim * 2 * 2
+
+    def gather(self):
+        self.msa.gather_kv(self.d, self.K_host, self.V_host, self.chunk_off, self.topk, self.capacity, out=self.stage)
+
+    def attend(self):
+        K_s, V_s, off_s, idx_s = self.stage
+        self.msa.sparse_attend(self.d, self.q, K_s, V_s, off_s, idx_s, self.K_loc, self.V_loc, self.loc_len, self.pos,
+                               out=self.out, ws=self.ws, k_loc_rotated=True)
+
+
 class AuxCase:
     def __init__(self, P, N, seed, device, dims=W.QWEN3_4B_DIMS, tau=0.05):
         import torch

@@ -172,6 +172,33 @@ def test_route_ties_prefer_lower_id(msa, cuda_device):
     assert np.all(sc[0] == sc[0][0])
 
 
+@pytest.mark.parametrize("n_docs,k", [(600, 32), (3000, 20), (4000, 1)])
+def test_route_all_ties_every_selection_path(msa, cuda_device, n_docs, k):
+    # every document identical: every score ties, the ids must come out ascending.  With
+    # thousands of tied keys the warp-threshold selection sees too many candidates and hands
+    # over to the sorting fallback; k = 32 fills a whole warp list
+    rng = np.random.default_rng(6 + n_docs)
+    dims = W.Dims(hidden=256, n_q=8, n_kv=2, head_dim=64, n_r=4, d_r=64)
+    KR = np.concatenate([W.normal_bf16(rng, (1, 4, 64))] * n_docs)
+    doc_off = W.offsets_from_lengths(np.full(n_docs, 64))        # one chunk each
+    QR = W.normal_bf16(rng, (2, 256))
+    idx, sc, ds = _run(msa, dims, QR, None, KR, doc_off, k, 0, cuda_device)
+    for b in range(2):
+        assert list(idx[b]) == list(range(k)), idx[b]
+        assert np.all(sc[b] == sc[b][0])
+
+
+@pytest.mark.parametrize("k", [31, 32, 33])
+def test_route_k_at_the_selection_boundaries(msa, cuda_device, k):
+    # k = 32 is the largest warp-list selection, 33 the smallest radix one
+    dims, doc_off, KR, QR, *_ = _route_case(40 + k, 700, 3, 8, 128, lo=1, hi=300)
+    idx, sc, ds = _run(msa, dims, QR, None, KR, doc_off, k, 0, cuda_device)
+    co, *_ = O.chunk_layout(doc_off)
+    s, _, _ = O.route_topk(O.bf16_to_f64(QR).reshape(3, 8, 128), KR, co, k)
+    for b in range(3):
+        check_topk(idx[b], sc[b], s[b], k, where=f"k={k} b={b}")
+
+
 def test_route_planted_equal_key_scores_one(msa, cuda_device):
     dims, doc_off, KR, QR, *_ = _route_case(21, 100, 2, 8, 128)
     co, *_ = O.chunk_layout(doc_off)
