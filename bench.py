@@ -475,49 +475,85 @@ def run_gpu(args):
     # the new token's K/V row, which is rotated and appended to the device-resident
     # local KV cache at position loc_len - 1; the step returns top-k ids/scores and
     # the attention output.
-    host = {"Hq": base["Hq"].cpu().pin_memory(), "q": base["q"].cpu().pin_memory(),
-            "k_new": k_new.cpu().contiguous().pin_memory(),
-            "v_new": base["V_loc"][:, Lm1].cpu().contiguous().pin_memory()}
-    dev_hq, dev_q = torch.empty_like(base["Hq"]), torch.empty_like(base["q"])
-    dev_kn, dev_vn = torch.empty_like(k_new), torch.empty_like(v_new)
-    h_idx = torch.empty((B, k), dtype=torch.int32).pin_memory()
-    h_sc = torch.empty((B, k), dtype=torch.float32).pin_memory()
-    h_out = torch.empty((B, d.n_q, d.head_dim), dtype=torch.bfloat16).pin_memory()
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = h_idx.numel() * 4 + h_sc.numel() * 4 + h_out.numel() * 2
+    # The step's inputs travel in one pinned host buffer and one copy (H_q | q | new K | new V, each
+    # at a 16-byte offset), its results come back the same way (top-k ids | scores | output):
+    # one host-to-device and one device-to-host transfer per step.
+    def packed(tensors):
+        offs, n = [], 0
+        for t in tensors:
+            offs.append(n)
+            n += (t.numel() * t.element_size() + 15) // 16 * 16
+        return offs, n
+
+    def views(buf, tensors, offs):
+        return [buf[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape) for t, o in zip(tensors, offs)]
+
+    v_row = base["V_loc"][:, Lm1].contiguous()
+    ins = [base["Hq"], base["q"], k_new, v_row]
+    in_offs, in_bytes = packed(ins)
+    host_in = torch.empty(in_bytes, dtype=torch.uint8).pin_memory()
+    for hv, t in zip(views(host_in, ins, in_offs), ins):
+        hv.copy_(t.cpu())
+    dev_in = torch.empty(in_bytes, dtype=torch.uint8, device=dev)
+    dev_hq, dev_q, dev_kn, dev_vn = views(dev_in, ins, in_offs)
+    outs = [torch.empty((B, k), dtype=torch.int32), torch.empty((B, k), dtype=torch.float32),
+            torch.empty((B, d.n_q, d.head_dim), dtype=torch.bfloat16)]
+    out_offs, out_bytes = packed(outs)
+    dev_out = torch.empty(out_bytes, dtype=torch.uint8, device=dev)
+    e_idx, e_sc, e_out = views(dev_out, outs, out_offs)
+    host_out = torch.empty(out_bytes, dtype=torch.uint8).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in ins)
+    d2h = sum(t.numel() * t.element_size() for t in outs)
 
     def e2e_step(i):
         x = rot[i % N_ROT]
-        dev_hq.copy_(host["Hq"], non_blocking=True)
-        dev_q.copy_(host["q"], non_blocking=True)
-        dev_kn.copy_(host["k_new"], non_blocking=True)
-        dev_vn.copy_(host["v_new"], non_blocking=True)
+        dev_in.copy_(host_in, non_blocking=True)
         msa.kv_append(d, dev_kn, dev_vn, x["K_loc"], x["V_loc"], slots, c["pos_offset"])
-        msa.route_topk(d, dev_hq, W_QR, x["KR"], chunk_off, k, out=(out_idx[0], out_sc[0], None), ws=r_ws,
+        msa.route_topk(d, dev_hq, W_QR, x["KR"], chunk_off, k, out=(e_idx, e_sc, None), ws=r_ws,
                        kr_inv_norm=inv_rot[i % N_ROT])
-        msa.sparse_attend(d, dev_q, x["K_bar"], x["V_bar"], chunk_off, out_idx[0], x["K_loc"], x["V_loc"], loc_len,
-                          c["pos_offset"], out=out_o[0], ws=a_ws, k_loc_rotated=True, early_local=True)
-        h_idx.copy_(out_idx[0], non_blocking=True)
-        h_sc.copy_(out_sc[0], non_blocking=True)
-        h_out.copy_(out_o[0], non_blocking=True)
+        msa.sparse_attend(d, dev_q, x["K_bar"], x["V_bar"], chunk_off, e_idx, x["K_loc"], x["V_loc"], loc_len,
+                          c["pos_offset"], out=e_out, ws=a_ws, k_loc_rotated=True, early_local=True)
+        host_out.copy_(dev_out, non_blocking=True)
 
-    with torch.cuda.stream(stream):
-        for i in range(args.warmup):
-            e2e_step(i)
-        torch.cuda.synchronize()
+    def e2e_time(run):
+        with torch.cuda.stream(stream):
+            for i in range(args.warmup):
+                run(i)
+            torch.cuda.synchronize()
+            if ws > 1:
+                dist.barrier()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for i in range(args.steps):
+                run(i)
+            e1.record(stream)
+            torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
         if ws > 1:
-            dist.barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for i in range(args.steps):
-            e2e_step(i)
-        e1.record(stream)
+            tt = torch.tensor([ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ms = float(tt.item())
+        return ms
+
+    # eager: every step issues its copies and library calls from Python
+    e2e_eager_ms = e2e_time(e2e_step)
+    # the same calls captured once per rotation copy in a CUDA graph (copies from and to the
+    # pinned host buffers included), replayed every step: the way a decode loop issues a step
+    e2e_graphs = []
+    try:
+        with torch.cuda.stream(stream):
+            for i in range(N_ROT):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    e2e_step(i)
+                e2e_graphs.append(g)
         torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.steps
-    if ws > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+        e2e_graph_ms = e2e_time(lambda i: e2e_graphs[i % N_ROT].replay())
+    except Exception as e:  # pragma: no cover
+        print(f"e2e graph capture failed ({e})", file=sys.stderr)
+        e2e_graph_ms = None
+    del e2e_graphs
+    e2e_ms = e2e_eager_ms
     e2e_val = T * B * ws / (e2e_ms * 1e-3)
 
     extras = None
@@ -541,7 +577,9 @@ def run_gpu(args):
                        "graphs": use_graphs, "parallelism": f"replicas x{ws}"},
             "roofline": roofline, "kernels": kernels, "gpu_launches": gpu_launches,
             "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e2e_ms},
+                    "ms_per_step": e2e_ms, "issue": "eager: every step's copies and calls issued from Python",
+                    "graph_ms_per_step": e2e_graph_ms,
+                    "graph_value": T * B * ws / (e2e_graph_ms * 1e-3) if e2e_graph_ms else None},
             "cpu_baseline": cpu, "clocks": clocks, "extras": extras,
             "notes": "value: device time of CUDA-graph replays of the full decode step (route, append the new "
                      "token's rotated key and value to the local cache, sparse attention over the rotated cache); "

@@ -48,7 +48,16 @@ class Dims(ctypes.Structure):
 
     @classmethod
     def of(cls, d) -> "Dims":
-        return cls(d.hidden, d.n_q, d.n_kv, d.head_dim, d.n_r, d.d_r, d.chunk, float(d.rope_base))
+        if isinstance(d, cls):
+            return d
+        key = (d.hidden, d.n_q, d.n_kv, d.head_dim, d.n_r, d.d_r, d.chunk, float(d.rope_base))
+        hit = _DIMS_CACHE.get(key)
+        if hit is None:
+            hit = _DIMS_CACHE[key] = cls(*key)
+        return hit
+
+
+_DIMS_CACHE: dict = {}  # the ctypes struct of each dims tuple (read-only after construction)
 
 
 def _load():
@@ -125,6 +134,9 @@ def _stream(stream) -> Optional[int]:
         return stream if isinstance(stream, int) else stream.cuda_stream
     import torch
 
+    raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)  # the current stream's handle, cheaply
+    if raw is not None:
+        return raw(torch.cuda.current_device())
     return torch.cuda.current_stream().cuda_stream
 
 
@@ -242,8 +254,11 @@ def route_topk(dims, Hq, W_QR, KR_bar, chunk_off, k: int, agg: int = AGG_MAX, wa
     if out is None:
         out = (torch.empty((B, k), dtype=torch.int32, device=dev), torch.empty((B, k), dtype=torch.float32, device=dev),
                torch.empty((B, n_docs), dtype=torch.float32, device=dev) if want_doc_scores else None)
-    nbytes = route_workspace_size(dims, B, n_docs, n_chunks, k, agg, q_tokens)
-    ws = _workspace(nbytes, dev, ws)
+    if ws is not None:  # the library checks the caller's buffer against what it needs
+        nbytes = max(0, ws.numel() * ws.element_size() - 256)
+    else:
+        nbytes = route_workspace_size(dims, B, n_docs, n_chunks, k, agg, q_tokens)
+        ws = _workspace(nbytes, dev, ws)
     _check(lib.msa_route_topk(ctypes.byref(dd), _ptr(Hq), _ptr(W_QR), B, q_tokens, _ptr(KR_bar), _ptr(chunk_off), n_docs,
                               n_chunks, k, agg, int(bool(kr_head_major)), _ptr(kr_inv_norm), _ptr(out[2]), _ptr(out[0]), _ptr(out[1]), _aligned_ptr(ws), nbytes,
                               _stream(stream)))
@@ -356,8 +371,11 @@ def sparse_attend(dims, q, K_bar, V_bar, chunk_off, topk_idx, K_loc, V_loc, loc_
     dev = q.device
     if out is None:
         out = torch.empty(tuple(q.shape), dtype=torch.bfloat16, device=dev)
-    nbytes = attend_workspace_size(dims, B, k, t_loc_max, pos_offset, M)
-    ws = _workspace(nbytes, dev, ws)
+    if ws is not None:  # the library checks the caller's buffer against what it needs
+        nbytes = max(0, ws.numel() * ws.element_size() - 256)
+    else:
+        nbytes = attend_workspace_size(dims, B, k, t_loc_max, pos_offset, M)
+        ws = _workspace(nbytes, dev, ws)
     _check(lib.msa_sparse_attend(ctypes.byref(dd), _ptr(q), B, M, _ptr(K_bar), _ptr(V_bar), _ptr(chunk_off), n_docs,
                                  K_bar.shape[0], _ptr(topk_idx), k, _ptr(K_loc), _ptr(V_loc), _ptr(loc_len),
                                  t_loc_max, pos_offset, _ptr(rope_cache), int(bool(k_loc_rotated)),

@@ -940,10 +940,10 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
     dim3 grid(std::max(1, std::min(n_items, sm_count())));
     const size_t sm = AttnSmem(d.n_kv, D, p.n_stages, tab != nullptr).total(d.n_q, D, p.tok_per_cta, p.co_cap);
     if (D == 128) {
-      MSA_CUDA_CHECK(cudaFuncSetAttribute(attn_split_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+      MSA_CUDA_CHECK(set_max_dynamic_smem(reinterpret_cast<const void*>(attn_split_kernel<128>), (int)sm));
       MSA_CUDA_CHECK(launch_pdl(attn_split_kernel<128>, grid, dim3(32 * (d.n_kv + 1)), sm, s, p));
     } else {
-      MSA_CUDA_CHECK(cudaFuncSetAttribute(attn_split_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+      MSA_CUDA_CHECK(set_max_dynamic_smem(reinterpret_cast<const void*>(attn_split_kernel<64>), (int)sm));
       MSA_CUDA_CHECK(launch_pdl(attn_split_kernel<64>, grid, dim3(32 * (d.n_kv + 1)), sm, s, p));
     }
   }

@@ -426,11 +426,11 @@ msa_status aux_loss_launch(const msa_dims& d, const void* QR, const void* K_pos,
   TraceScope ts(kKAuxLoss, s);
   if (d.d_r == 128) {
     const size_t sm = AuxSmem<128>::bytes(N + 1);
-    MSA_CUDA_CHECK(cudaFuncSetAttribute(aux_loss_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+    MSA_CUDA_CHECK(set_max_dynamic_smem(reinterpret_cast<const void*>(aux_loss_kernel<128>), (int)sm));
     MSA_CUDA_CHECK(launch_pdl(aux_loss_kernel<128>, dim3(grid), dim3(kAuxThreads), sm, s, p));
   } else {
     const size_t sm = AuxSmem<64>::bytes(N + 1);
-    MSA_CUDA_CHECK(cudaFuncSetAttribute(aux_loss_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+    MSA_CUDA_CHECK(set_max_dynamic_smem(reinterpret_cast<const void*>(aux_loss_kernel<64>), (int)sm));
     MSA_CUDA_CHECK(launch_pdl(aux_loss_kernel<64>, dim3(grid), dim3(kAuxThreads), sm, s, p));
   }
   return MSA_OK;

@@ -382,11 +382,11 @@ template <int MODE>
 cudaError_t launch_gemm(int bn, int grid, size_t smem, cudaStream_t s, const CUtensorMap& ma, const CUtensorMap& mb,
                         const GemmParams& p) {
   if (bn == 256) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<MODE, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(gemm_kernel<MODE, 256>), (int)smem);
     if (e != cudaSuccess) return e;
     gemm_kernel<MODE, 256><<<grid, kEncThreads, smem, s>>>(ma, mb, p);
   } else {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<MODE, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(gemm_kernel<MODE, 128>), (int)smem);
     if (e != cudaSuccess) return e;
     gemm_kernel<MODE, 128><<<grid, kEncThreads, smem, s>>>(ma, mb, p);
   }

@@ -88,6 +88,8 @@ struct Carver {
 // ---------------------------------------------------------------------------
 int sm_count();
 int max_smem_optin();
+// cudaFuncSetAttribute(kernel, MaxDynamicSharedMemorySize, bytes), skipped when already set
+cudaError_t set_max_dynamic_smem(const void* kernel, int bytes);
 msa_status encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, void* gaddr,
                              const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
                              CUtensorMapSwizzle swizzle);
@@ -95,6 +97,7 @@ msa_status encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int ra
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // theta_i / (2 pi) as 64-bit binary fractions, theta_i = base^(-2i/head_dim) (computed in long double)
+constexpr int kRopeMaxHalf = 128;  // head_dim / 2 of the largest supported head
 void rope_turns(const msa_dims& d, uint64_t* f /* [head_dim / 2] */);
 
 // Launch with programmatic stream serialization: the kernel may be scheduled

@@ -10,6 +10,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -51,22 +52,70 @@ bool fault_injected() {
 }
 
 void rope_turns(const msa_dims& d, uint64_t* f) {
-  const long double two_pi = 6.283185307179586476925286766559005768L;
-  const long double lb = logl((long double)d.rope_base);
-  for (int i = 0; i < d.head_dim / 2; ++i) {
-    const long double theta = expl(-2.0L * (long double)i / (long double)d.head_dim * lb);
-    const long double turns = theta / two_pi;  // in (0, 1)
-    f[i] = (uint64_t)ldexpl(turns, 64);
+  // the last (head_dim, base) of this host thread is kept: decode loops ask every step
+  thread_local int c_dim = -1;
+  thread_local float c_base = 0.f;
+  thread_local uint64_t c_f[kRopeMaxHalf];
+  const int half = d.head_dim / 2;
+  if (c_dim != d.head_dim || c_base != d.rope_base || half > kRopeMaxHalf) {
+    const long double two_pi = 6.283185307179586476925286766559005768L;
+    const long double lb = logl((long double)d.rope_base);
+    for (int i = 0; i < half && i < kRopeMaxHalf; ++i) {
+      const long double theta = expl(-2.0L * (long double)i / (long double)d.head_dim * lb);
+      const long double turns = theta / two_pi;  // in (0, 1)
+      c_f[i] = (uint64_t)ldexpl(turns, 64);
+    }
+    c_dim = d.head_dim;
+    c_base = d.rope_base;
   }
+  for (int i = 0; i < half; ++i) f[i] = c_f[i];
 }
 
 // ---------------------------------------------------------------------------
 // device properties
 // ---------------------------------------------------------------------------
+namespace {
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];  // 0: not queried yet
+}  // namespace
+
 int sm_count() {
-  int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+  if (dev < kMaxDevices) {
+    const int c = g_sm_count[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int n = 148;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  n = n > 0 ? n : 148;
+  if (dev < kMaxDevices) g_sm_count[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (device, kernel, size): a decode loop
+// calls the same kernels every step
+cudaError_t set_max_dynamic_smem(const void* kernel, int bytes) {
+  struct Entry {
+    int dev;
+    const void* fn;
+    int bytes;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    for (const Entry& e : done)
+      if (e.dev == dev && e.fn == kernel && e.bytes >= bytes) return cudaSuccess;
+  }
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) {
+    std::lock_guard<std::mutex> lk(mu);
+    done.push_back({dev, kernel, bytes});
+  }
+  return e;
 }
 
 int max_smem_optin() {
@@ -94,12 +143,50 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
 msa_status encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, void* gaddr,
                              const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
                              CUtensorMapSwizzle swizzle) {
+  // the maps of the last calls of this host thread are kept (a decode loop encodes the same
+  // few maps every step); the key is every argument
+  struct Key {
+    int dtype, rank, swizzle;
+    void* gaddr;
+    uint64_t dims[5], strides[4];
+    uint32_t box[5];
+    bool operator==(const Key& o) const { return std::memcmp(this, &o, sizeof(Key)) == 0; }
+  };
+  struct Slot {
+    Key key;
+    CUtensorMap map;
+    bool used;
+  };
+  constexpr int kSlots = 32;
+  thread_local Slot cache[kSlots] = {};
+  thread_local int next = 0;
+  Key key;
+  std::memset(&key, 0, sizeof(key));
+  key.dtype = (int)dtype;
+  key.rank = rank;
+  key.swizzle = (int)swizzle;
+  key.gaddr = gaddr;
+  for (int i = 0; i < rank && i < 5; ++i) {
+    key.dims[i] = dims[i];
+    key.box[i] = box[i];
+    if (i + 1 < rank) key.strides[i] = strides_bytes[i];
+  }
+  for (int i = 0; i < kSlots; ++i)
+    if (cache[i].used && cache[i].key == key) {
+      *map = cache[i].map;
+      return MSA_OK;
+    }
   auto fn = get_encoder();
   if (!fn) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
   uint32_t elem_strides[5] = {1, 1, 1, 1, 1};
   CUresult r = fn(map, dtype, rank, gaddr, dims, strides_bytes, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+  Slot& sl = cache[next];
+  next = (next + 1) % kSlots;
+  sl.key = key;
+  sl.map = *map;
+  sl.used = true;
   return MSA_OK;
 }
 

@@ -1013,7 +1013,7 @@ cudaError_t launch_scan_t(const CUtensorMap& kmap, const CUtensorMap& qmap, cons
                     (size_t)ScanGeom<DR, NQ>::kStages * ScanGeom<DR, NQ>::kStageBytes,
                 "the fused top-k reuses the pipeline stages");
   const size_t smem = ScanGeom<DR, NQ>::kSmemBytes;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), (int)smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(grid), dim3(kScanThreads), smem, s, kmap, qmap, p);
 }
@@ -1070,7 +1070,7 @@ msa_status topk_merge_launch(const float* cand_score, const int32_t* cand_idx, i
                              int32_t* topk_idx, float* topk_score, cudaStream_t s) {
   TraceScope ts(kKTopkMerge, s);
   const size_t sm = topk_merge_smem(n_cand);
-  MSA_CUDA_CHECK(cudaFuncSetAttribute(topk_merge_pairs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+  MSA_CUDA_CHECK(set_max_dynamic_smem(reinterpret_cast<const void*>(topk_merge_pairs_kernel), (int)sm));
   MSA_CUDA_CHECK(launch_pdl(topk_merge_pairs_kernel, dim3(B), dim3(kTopkThreads), sm, s, cand_score, cand_idx, n_cand,
                             k, topk_idx, topk_score));
   return MSA_OK;
@@ -1125,7 +1125,7 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
     TraceScope ts(kKRouterQuery, s);
     if (W_QR) {
       const size_t sm = rq_smem_bytes(d.d_r);
-      MSA_CUDA_CHECK(cudaFuncSetAttribute(router_query_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+      MSA_CUDA_CHECK(set_max_dynamic_smem(reinterpret_cast<const void*>(router_query_kernel), (int)sm));
       MSA_CUDA_CHECK(launch_pdl_cluster(router_query_kernel, dim3(kRqCluster, d.n_r), dim3(kRqThreads), sm, s,
                                         kRqCluster, static_cast<const __nv_bfloat16*>(Hq),
                                         static_cast<const __nv_bfloat16*>(W_QR), R, w.passes * w.nq, d.hidden, d.n_r,
@@ -1198,7 +1198,7 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
   if (!fuse_topk) {
     TraceScope ts(kKTopkSlice, s);
     const size_t sm = topk_slice_smem();
-    MSA_CUDA_CHECK(cudaFuncSetAttribute(topk_slice_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+    MSA_CUDA_CHECK(set_max_dynamic_smem(reinterpret_cast<const void*>(topk_slice_kernel), (int)sm));
     MSA_CUDA_CHECK(launch_pdl(topk_slice_kernel, dim3(w.n_slices, B), dim3(kTopkThreads), sm, s,
                               (const uint32_t*)w.doc_key, (const uint32_t*)w.chunk_k, chunk_off, n_docs, n_chunks, k,
                               w.n_slices, doc_scores, w.cand, topk_idx, topk_score));
@@ -1206,7 +1206,7 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
   if (w.n_slices > 1) {
     TraceScope ts(kKTopkMerge, s);
     const size_t sm = topk_merge_smem(w.n_slices * k);
-    MSA_CUDA_CHECK(cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+    MSA_CUDA_CHECK(set_max_dynamic_smem(reinterpret_cast<const void*>(topk_merge_kernel), (int)sm));
     MSA_CUDA_CHECK(launch_pdl(topk_merge_kernel, dim3(B), dim3(kTopkThreads), sm, s, (const uint64_t*)w.cand,
                               w.n_slices, k, topk_idx, topk_score));
   }
