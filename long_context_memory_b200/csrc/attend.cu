@@ -802,9 +802,10 @@ size_t attend_workspace(const msa_dims& d, int B, int M, int k, int t_loc_max, i
   const double sel_est = (double)kChunksPerDocEst * k;
   int n_chunk = (int)std::lround(n_total * sel_est / (sel_est + std::max(0, t_loc_max)));
   // one wave or less (few queries: latency): the selected chunks, which wait for the routing,
-  // in splits of at most two 16-key tiles
-  if ((long long)n_total * B * n_tg <= sm_count()) n_chunk = std::max(n_chunk, (int)std::ceil(sel_est / 32.0));
-  n_chunk = std::max(1, std::min({n_chunk, 2 * k, n_total - 1}));
+  // in splits of about one 16-key tile
+  const bool latency = (long long)n_total * B * n_tg <= sm_count();
+  if (latency) n_chunk = std::max(n_chunk, (int)std::ceil(sel_est / 16.0));
+  n_chunk = std::max(1, std::min({n_chunk, (latency ? 4 : 2) * k, n_total - 1}));
   w.n_split_chunk = n_chunk;
   w.n_split_local = std::max(1, std::min(n_total - n_chunk, std::max(1, (t_loc_max + kTK - 1) / kTK)));
   w.n_parts = w.n_split_local + w.n_split_chunk;
