@@ -131,6 +131,9 @@ def test_attend_validation(msa):
     assert _attend(msa, ok, ws_bytes=8) == 3
     assert _attend(msa, ok, M=0) == 1
     assert _attend(msa, ok, phase=3) == 1
+    assert _attend(msa, ok, phase=3 | msa.ATTEND_EARLY_LOCAL) == 1  # the flag does not make a bad phase valid
+    assert _attend(msa, ok, phase=-1) == 1
+    assert _attend(msa, ok, phase=msa.ATTEND_EARLY_LOCAL | 32) == 1  # an unknown flag bit
 
 
 def test_encode_validation(msa):
