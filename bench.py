@@ -378,13 +378,15 @@ def run_gpu(args):
 
     def step(i):
         # one stream: the new token into the rotated local cache, routing, sparse attention.  The
-        # attention's local-key work starts while the routing's kernels finish (early_local: q and
-        # the local cache were final before the routing call was enqueued).
+        # routing's query and memory are not written by the append (early_inputs: the router query
+        # multiplies and the scan streams while the append runs); the attention's local-key work
+        # starts while the routing's kernels finish (early_local: q and the local cache are not
+        # written by the routing).
         x = rot[i % N_ROT]
         j = i % N_ROT
         msa.kv_append(d, k_new, v_new, x["K_loc"], x["V_loc"], slots, c["pos_offset"])
         msa.route_topk(d, x["Hq"], W_QR, x["KR"], chunk_off, k, out=(out_idx[j], out_sc[j], None), ws=r_ws,
-                       kr_inv_norm=inv_rot[j])
+                       kr_inv_norm=inv_rot[j], early_inputs=True)
         msa.sparse_attend(d, x["q"], x["K_bar"], x["V_bar"], chunk_off, out_idx[j], x["K_loc"], x["V_loc"], loc_len,
                           c["pos_offset"], out=out_o[j], ws=a_ws, k_loc_rotated=True, early_local=True)
 
@@ -510,7 +512,7 @@ def run_gpu(args):
         dev_in.copy_(host_in, non_blocking=True)
         msa.kv_append(d, dev_kn, dev_vn, x["K_loc"], x["V_loc"], slots, c["pos_offset"])
         msa.route_topk(d, dev_hq, W_QR, x["KR"], chunk_off, k, out=(e_idx, e_sc, None), ws=r_ws,
-                       kr_inv_norm=inv_rot[i % N_ROT])
+                       kr_inv_norm=inv_rot[i % N_ROT], early_inputs=True)
         msa.sparse_attend(d, dev_q, x["K_bar"], x["V_bar"], chunk_off, e_idx, x["K_loc"], x["V_loc"], loc_len,
                           c["pos_offset"], out=e_out, ws=a_ws, k_loc_rotated=True, early_local=True)
         host_out.copy_(dev_out, non_blocking=True)

@@ -160,6 +160,13 @@ msa_status msa_append_memory(const msa_dims* dims, const void* H_new, int64_t T_
  *   KR_bar   pooled router keys, bf16: [n_chunks, n_r, d_r] for kr_layout 0, or
  *            head-major [n_r, n_chunks, d_r] for kr_layout 1 (each head's keys contiguous:
  *            the scan then streams whole 32 KB slices instead of 256-byte pieces).
+ *            kr_layout | MSA_ROUTE_EARLY_INPUTS: the router query reads H_q and W_QR and
+ *            multiplies them, and the scan starts streaming KR_bar, before the preceding work
+ *            on the stream has finished (the writes still wait for it).  The caller
+ *            guarantees that H_q, W_QR, KR_bar, kr_inv_norm and chunk_off are not written by
+ *            the work immediately preceding this call on the stream, and that this work is a
+ *            call of this library, a copy, or a kernel that does not start its dependents
+ *            early (programmatic dependent launch).  The result is the same as without it.
  *   chunk_off[n_docs + 1] device int32 chunk offsets of the documents.
  *   kr_inv_norm  optional [n_chunks, n_r] fp32 from msa_router_key_norms: the keys'
  *            inverse norms, computed once offline; NULL = computed during the scan
@@ -174,6 +181,7 @@ msa_status msa_append_memory(const msa_dims* dims, const void* H_new, int64_t T_
  * the normalised query split into two bf16 terms (hi + lo) and fp32
  * accumulation, so scores carry ~1e-6 relative error.
  * ------------------------------------------------------------------------- */
+#define MSA_ROUTE_EARLY_INPUTS 16
 size_t msa_route_workspace_size(const msa_dims* dims, int32_t B, int32_t q_tokens, int32_t n_docs,
                                 int32_t n_chunks, int32_t k, msa_doc_agg agg);
 msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR, int32_t B, int32_t q_tokens,
@@ -287,13 +295,15 @@ msa_status msa_aux_loss(const msa_dims* dims, const void* QR, const void* K_pos,
  *            V_loc are not read).  Phase 2 must be ordered after phase 1 (same stream, or
  *            an event).  The result equals phase 0's up to fp32 summation order.
  *            phase | MSA_ATTEND_EARLY_LOCAL (phases 0 and 1): the work on the local keys may
- *            start before the kernels of the preceding library call on the stream have
- *            finished (typically msa_route_topk producing topk_idx), hiding it behind the
- *            routing.  The caller guarantees that q, K_loc, V_loc, loc_len (and rope_cache)
- *            were final before that preceding call was enqueued, and that the preceding call
- *            is not an msa_sparse_attend on this workspace.  The flag has no effect when
- *            the call builds its own rotation table (k_loc_rotated 0 and rope_cache NULL).
- *            The result is the same as without the flag.
+ *            start before the preceding work on the stream has finished (typically
+ *            msa_route_topk producing topk_idx), hiding it behind the routing.  The caller
+ *            guarantees that q, K_loc, V_loc, loc_len, chunk_off (and rope_cache) are not
+ *            written by the work immediately preceding this call on the stream, that this
+ *            work does not use this workspace, and that it is a call of this library, a
+ *            copy, or a kernel that does not start its dependents early (programmatic
+ *            dependent launch).  The flag has no effect when the call builds its own
+ *            rotation table (k_loc_rotated 0 and rope_cache NULL).  The result is the same
+ *            as without the flag.
  *   out      [B, M, n_q, head_dim] bf16.
  * Limits: 1 <= M, B * M <= 65535.
  * Query head g attends with KV head g / (n_q / n_kv).  Every query token sees

@@ -20,7 +20,7 @@ __all__ = [
     "Dims", "MSAError", "lib", "chunk_offsets", "encode_memory", "append_memory", "route_topk", "sparse_attend",
     "aux_loss", "kv_append", "router_key_norms",
     "route_workspace_size", "attend_workspace_size", "rope_cache_build", "topk_merge", "rope_rows", "gather_kv", "encode_workspace_size", "check_device_errors",
-    "trace_enable", "trace_reset", "trace_read", "trace_kernel_names", "AGG_MAX", "AGG_MEAN", "ATTEND_EARLY_LOCAL",
+    "trace_enable", "trace_reset", "trace_read", "trace_kernel_names", "AGG_MAX", "AGG_MEAN", "ATTEND_EARLY_LOCAL", "ROUTE_EARLY_INPUTS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -29,6 +29,7 @@ LIB_PATH = os.path.join(_HERE, "libmsa.so")
 AGG_MAX = 0
 AGG_MEAN = 1
 ATTEND_EARLY_LOCAL = 16  # msa.h MSA_ATTEND_EARLY_LOCAL, OR-ed into the phase argument
+ROUTE_EARLY_INPUTS = 16  # msa.h MSA_ROUTE_EARLY_INPUTS, OR-ed into the kr_layout argument
 
 STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED", 3: "MSA_ERR_WORKSPACE",
           4: "MSA_ERR_CUDA", 5: "MSA_ERR_TIMEOUT"}
@@ -233,7 +234,8 @@ def route_workspace_size(dims, B: int, n_docs: int, n_chunks: int, k: int, agg: 
 
 
 def route_topk(dims, Hq, W_QR, KR_bar, chunk_off, k: int, agg: int = AGG_MAX, want_doc_scores: bool = False,
-               out=None, ws=None, stream=None, kr_head_major: bool = False, q_tokens: int = 1, kr_inv_norm=None):
+               out=None, ws=None, stream=None, kr_head_major: bool = False, q_tokens: int = 1, kr_inv_norm=None,
+               early_inputs: bool = False):
     """Top-k documents per query.  Returns (topk_idx [B,k] int32, topk_score [B,k] fp32, doc_scores|None).
 
     ``Hq`` holds B * q_tokens rows (token t of query b at row b * q_tokens + t); a chunk's
@@ -241,6 +243,9 @@ def route_topk(dims, Hq, W_QR, KR_bar, chunk_off, k: int, agg: int = AGG_MAX, wa
     ``W_QR=None`` means ``Hq`` already holds the router queries Q^R [B * q_tokens, n_r*d_r].
     ``kr_head_major``: KR_bar is [n_r, C, d_r] instead of [C, n_r, d_r].
     ``kr_inv_norm``: the keys' inverse norms from ``router_key_norms`` (computed once per memory).
+    ``early_inputs`` (MSA_ROUTE_EARLY_INPUTS): ``Hq``, ``W_QR``, ``KR_bar``, ``kr_inv_norm`` and
+    ``chunk_off`` were final before the preceding work on the stream was enqueued, so the routing
+    may read them before that work finishes.
     """
     import torch
 
@@ -260,7 +265,8 @@ def route_topk(dims, Hq, W_QR, KR_bar, chunk_off, k: int, agg: int = AGG_MAX, wa
         nbytes = route_workspace_size(dims, B, n_docs, n_chunks, k, agg, q_tokens)
         ws = _workspace(nbytes, dev, ws)
     _check(lib.msa_route_topk(ctypes.byref(dd), _ptr(Hq), _ptr(W_QR), B, q_tokens, _ptr(KR_bar), _ptr(chunk_off), n_docs,
-                              n_chunks, k, agg, int(bool(kr_head_major)), _ptr(kr_inv_norm), _ptr(out[2]), _ptr(out[0]), _ptr(out[1]), _aligned_ptr(ws), nbytes,
+                              n_chunks, k, agg, int(bool(kr_head_major)) | (ROUTE_EARLY_INPUTS if early_inputs else 0),
+                              _ptr(kr_inv_norm), _ptr(out[2]), _ptr(out[0]), _ptr(out[1]), _aligned_ptr(ws), nbytes,
                               _stream(stream)))
     return out
 

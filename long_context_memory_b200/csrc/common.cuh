@@ -334,7 +334,9 @@ namespace msa {
 // dependent start (pdl_enter).  So when a library kernel starts, the kernel
 // before it has passed its wait and everything earlier on the stream has
 // completed: a kernel may read before its own wait whatever its immediate
-// predecessor does not write (the scan's first key tiles).
+// predecessor does not write (the scan's first key tiles).  The one exception,
+// the router query under the caller's early-inputs guarantee, starts the scan
+// at once: that guarantee covers everything the scan reads before its wait.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }

@@ -150,7 +150,7 @@ msa_status kr_norms_launch(const msa_dims& d, const void* KR_bar, int n_chunks, 
 msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int B, int M, const void* KR_bar,
                         const int32_t* chunk_off, int n_docs, int n_chunks, int k, msa_doc_agg agg, int kr_layout,
                         const float* kr_inv_norm, float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws,
-                        cudaStream_t s);
+                        cudaStream_t s, bool early_inputs = false);
 
 msa_status topk_merge_launch(const float* cand_score, const int32_t* cand_idx, int B, int n_cand, int k,
                              int32_t* topk_idx, float* topk_score, cudaStream_t s);

@@ -367,7 +367,10 @@ msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR
   if (k < 1 || k > n_docs || k > 256)
     return fail(MSA_ERR_INVALID_ARG, "k must be in [1, min(n_docs, 256)] (got %d, n_docs %d)", k, n_docs);
   if (agg != MSA_AGG_MAX && agg != MSA_AGG_MEAN) return fail(MSA_ERR_INVALID_ARG, "unknown aggregation %d", (int)agg);
-  if (kr_layout != 0 && kr_layout != 1) return fail(MSA_ERR_INVALID_ARG, "kr_layout must be 0 or 1 (got %d)", kr_layout);
+  const bool early_inputs = (kr_layout & MSA_ROUTE_EARLY_INPUTS) != 0;
+  kr_layout &= ~MSA_ROUTE_EARLY_INPUTS;
+  if (kr_layout != 0 && kr_layout != 1)
+    return fail(MSA_ERR_INVALID_ARG, "kr_layout must be 0 or 1, optionally | MSA_ROUTE_EARLY_INPUTS (got %d)", kr_layout);
   const int n_slices = (n_docs + 4095) / 4096;
   if ((size_t)n_slices * k > 24576) return fail(MSA_ERR_UNSUPPORTED, "n_docs * k too large for the top-k merge");
   CHECK_PTR(Hq);
@@ -384,8 +387,7 @@ msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR
   CHECK_OPT_PTR(kr_inv_norm);
   if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
   return route_launch(*dims, Hq, W_QR, B, q_tokens, KR_bar, chunk_off, n_docs, n_chunks, k, agg, kr_layout, kr_inv_norm,
-                      doc_scores, topk_idx,
-                      topk_score, ws, static_cast<cudaStream_t>(stream));
+                      doc_scores, topk_idx, topk_score, ws, static_cast<cudaStream_t>(stream), early_inputs);
 }
 
 msa_status msa_router_key_norms(const msa_dims* dims, const void* KR_bar, int32_t n_chunks, int32_t kr_layout,

@@ -101,15 +101,23 @@ __device__ __forceinline__ void rq_store_row(__nv_bfloat16* q_hl, int b, int h, 
 __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
     const __nv_bfloat16* __restrict__ Hq, const __nv_bfloat16* __restrict__ W, int B, int b_pad, int hidden,
     int n_r, int d_r, int nq, int split_rows, __nv_bfloat16* __restrict__ q_hl, uint32_t* __restrict__ clear,
-    size_t n_clear, uint32_t* __restrict__ scan_ticket) {
+    size_t n_clear, uint32_t* __restrict__ scan_ticket, int early) {
   extern __shared__ __align__(16) uint8_t rq_smem[];
   __shared__ float wsum[kRqThreads / 32];
-  pdl_enter();
+  // early: H_q, W^QR and the memory the scan reads (K̄^R, its norms, chunk_off) were final
+  // before the preceding work was enqueued, so the scan may start at once and every thread
+  // reads and multiplies before it waits; the writes (workspace) come after the wait
+  bool waited = !early;
+  if (waited) {
+    pdl_enter();
+    rq_clear(clear, n_clear, scan_ticket);
+  } else {
+    pdl_launch_dependents();
+  }
   const int NR = n_r * d_r;
   const int rank = blockIdx.x, h = blockIdx.y;  // the cluster spans blockIdx.x
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint16_t* hq = reinterpret_cast<const uint16_t*>(Hq);
-  rq_clear(clear, n_clear, scan_ticket);
 
   const int ws = rq_w_stride(d_r), hstr = rq_h_stride();
   uint8_t* wsm = rq_smem;
@@ -193,6 +201,11 @@ __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
       for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
       if (lane == 0) wsum[warp] = ss;
       __syncthreads();
+      if (!waited) {  // every thread, before its first write
+        pdl_wait();
+        rq_clear(clear, n_clear, scan_ticket);
+        waited = true;
+      }
       if (q < 2) {
         const int w0 = q * d_r / 32, nw = d_r / 32;  // the warps holding this row
         float tot = 0.f;
@@ -203,15 +216,16 @@ __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
     }
     cluster_sync();  // the partials may be overwritten / the CTAs may exit
   }
+  if (!waited) pdl_wait();  // the grid completes only after its predecessor
 }
 
 // Q^R given directly (W_QR == NULL): normalise each row of head h, write the hi/lo terms
 __global__ void __launch_bounds__(kRqThreads) router_query_direct_kernel(
     const __nv_bfloat16* __restrict__ Hq, int B, int b_pad, int n_r, int d_r, int nq, __nv_bfloat16* __restrict__ q_hl,
-    uint32_t* __restrict__ clear, size_t n_clear, uint32_t* __restrict__ scan_ticket) {
+    uint32_t* __restrict__ clear, size_t n_clear, uint32_t* __restrict__ scan_ticket, int early) {
   __shared__ float invn[kRqThreads / 32];
-  pdl_enter();
-  rq_clear(clear, n_clear, scan_ticket);
+  if (!early) pdl_enter();  // early: H_q is read before the wait, the writes come after it
+  else pdl_launch_dependents();
   const int NR = n_r * d_r, h = blockIdx.y;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint16_t* hq = reinterpret_cast<const uint16_t*>(Hq);
@@ -231,10 +245,13 @@ __global__ void __launch_bounds__(kRqThreads) router_query_direct_kernel(
     __syncwarp();
     const float sc = invn[warp];
     __syncwarp();
+    if (early && b == warp) pdl_wait();  // this warp's first write
 #pragma unroll
     for (int e = 0; e < 4; ++e)
       if (lane + 32 * e < d_r) rq_store_row(q_hl, b, h, lane + 32 * e, v[e] * sc, n_r, d_r, nq);
   }
+  if (early && warp >= b_pad) pdl_wait();  // warps with no rows
+  rq_clear(clear, n_clear, scan_ticket);
 }
 
 // --------------------------------------------------------------------------
@@ -1107,7 +1124,8 @@ size_t route_workspace(const msa_dims& d, int B, int M, int n_docs, int n_chunks
 
 msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int B, int M, const void* KR_bar,
                         const int32_t* chunk_off, int n_docs, int n_chunks, int k, msa_doc_agg agg, int kr_layout,
-                        const float* kr_inv_norm, float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws, cudaStream_t s) {
+                        const float* kr_inv_norm, float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws, cudaStream_t s,
+                        bool early_inputs) {
   RouteWs w;
   route_workspace(d, B, M, n_docs, n_chunks, k, agg, ws, &w);
   const int NR = d.n_r * d.d_r;
@@ -1130,11 +1148,11 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
                                         kRqCluster, static_cast<const __nv_bfloat16*>(Hq),
                                         static_cast<const __nv_bfloat16*>(W_QR), R, w.passes * w.nq, d.hidden, d.n_r,
                                         d.d_r, w.nq, rq_split_rows(d.hidden), w.q_hl, clear, n_clear,
-                                        w.scan_ticket));
+                                        w.scan_ticket, early_inputs ? 1 : 0));
     } else {
       MSA_CUDA_CHECK(launch_pdl(router_query_direct_kernel, dim3(1, d.n_r), dim3(kRqThreads), 0, s,
                                 static_cast<const __nv_bfloat16*>(Hq), R, w.passes * w.nq, d.n_r, d.d_r, w.nq,
-                                w.q_hl, clear, n_clear, w.scan_ticket));
+                                w.q_hl, clear, n_clear, w.scan_ticket, early_inputs ? 1 : 0));
     }
   }
   // K3: scan, NQ (16 or 32) queries per pass

@@ -260,3 +260,31 @@ def test_route_mem16m_batch32_sampled(msa, cuda_device):
         assert list(idx[b]) == list(want), (b, idx[b], want)
         others = np.setdiff1d(np.arange(len(co) - 1), c["planted_docs"][b])
         assert ds[b, others].max() < sc[b, -1] - 2e-3
+
+
+@pytest.mark.parametrize("projection", [True, False])
+@pytest.mark.parametrize("B", [1, 5])
+def test_route_early_inputs_behind_another_call(msa, cuda_device, projection, B):
+    # routing launched right behind another library call with MSA_ROUTE_EARLY_INPUTS (the router
+    # query multiplies and the scan streams before that call's kernel finishes): the same top-k,
+    # scores and document scores, bit for bit, as the ordinary call
+    import torch
+
+    dims, doc_off, KR, QR, Hq, Wqr, rng = _route_case(300 + B, 900, B, 8, 128, lo=64, hi=4000, hidden=512)
+    dev = cuda_device
+    co, C = msa.chunk_offsets(doc_off)
+    KR_d, co_d = _dev(KR, dev), torch.from_numpy(co).to(dev)
+    inv = msa.router_key_norms(dims, KR_d)
+    q_in = _dev(Hq, dev) if projection else _dev(QR, dev)
+    w_in = _dev(Wqr, dev) if projection else None
+    other = _dev(W.normal_bf16(rng, (20000, 8, 128)), dev)  # a busy preceding call on unrelated data
+    res = []
+    for early in (False, True, True):
+        msa.router_key_norms(dims, other)
+        res.append(msa.route_topk(dims, q_in, w_in, KR_d, co_d, 12, want_doc_scores=True, kr_inv_norm=inv,
+                                  early_inputs=early))
+    torch.cuda.synchronize()
+    assert msa.check_device_errors() == 0
+    for r in res[1:]:
+        for a, b in zip(res[0], r):
+            assert torch.equal(a, b)
