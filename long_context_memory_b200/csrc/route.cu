@@ -622,11 +622,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     if (threadIdx.x == 0) {
       const uint32_t prev = atomicAdd(p.ticket, 1u);
       last_cta = prev == gridDim.x - 1;
-      if (last_cta) *p.ticket = 0u;
     }
     __syncthreads();
     if (!last_cta) return;
     __threadfence();
+    if (threadIdx.x == 0) *p.ticket = 0u;  // ready for the next launch
     for (int b = 0; b < p.n_queries; ++b)
       slice_topk(p.doc_key, p.chunk_k, p.chunk_off, p.n_docs, p.n_chunks, p.k, 1, p.doc_scores, nullptr,
                  p.topk_idx, p.topk_score, 0, b, reinterpret_cast<uint64_t*>(smem));
@@ -730,11 +730,11 @@ __device__ void block_topk_small(const uint64_t* keys, int n, int k, uint64_t* o
 }
 
 // k <= 32, few candidates: (1) warp w takes keys [w n / nw, (w + 1) n / nw), at most 4 per
-// lane, and finds its m-th largest key T_w (m = ceil(k / nw); m rounds of a warp-wide max, the
-// owner lane dropping its maximum each time).  (2) T = min over warps of T_w: every warp holds m
-// keys >= T_w >= T, so at least k keys are >= T and the k best all are.  (3) The keys >= T are
-// compacted (one shared-memory atomic per warp) and each counts the larger ones, which is its
-// rank.  Returns false, having written nothing, when the split does not apply (n above 128 keys
+// lane, and finds the m-th largest score (the key's upper word) T_w among them (m = ceil(k / nw);
+// m rounds of a warp-wide 32-bit max, one owner lane dropping its maximum each time).  (2) T =
+// min over warps of T_w: every warp holds m keys scoring >= T_w >= T, so at least k keys score
+// >= T and the k best all do.  (3) The keys scoring >= T are compacted (one shared-memory atomic
+// per warp) and each counts the larger keys, which is its rank.  Returns false, having written nothing, when the split does not apply (n above 128 keys
 // per warp, a warp with fewer than m keys, m above 4) or more than kTopkMaxCand keys pass.
 constexpr int kTopkMaxCand = 256;
 __device__ bool block_topk_threshold(const uint64_t* keys, int n, int k, uint64_t* out, uint64_t* cand,
@@ -752,33 +752,26 @@ __device__ bool block_topk_threshold(const uint64_t* keys, int n, int k, uint64_
 #define MSA_CX(a, b) { const uint64_t x_ = v[a] > v[b] ? v[a] : v[b]; v[b] = v[a] > v[b] ? v[b] : v[a]; v[a] = x_; }
   MSA_CX(0, 1) MSA_CX(2, 3) MSA_CX(0, 2) MSA_CX(1, 3) MSA_CX(1, 2)
 #undef MSA_CX
-  uint64_t t_w = 0;
+  uint32_t t_w = 0;
   for (int r = 0; r < m; ++r) {
-    uint64_t x = v[0];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const uint64_t y = shfl_xor_u64(x, o);
-      x = x > y ? x : y;
-    }
+    const uint32_t x = __reduce_max_sync(0xffffffffu, (uint32_t)(v[0] >> 32));
     t_w = x;
-    if (v[0] == x) {  // the owner (keys are distinct) drops its maximum
+    // one owner of the maximum score drops it (scores may tie: the lowest such lane)
+    const unsigned own = __ballot_sync(0xffffffffu, (uint32_t)(v[0] >> 32) == x);
+    if (lane == __ffs(own) - 1) {
       v[0] = v[1];
       v[1] = v[2];
       v[2] = v[3];
       v[3] = 0ull;
     }
   }
-  if (lane == 0) warp_t[warp] = t_w;
+  uint32_t* warp_t32 = reinterpret_cast<uint32_t*>(warp_t);
+  if (lane == 0) warp_t32[warp] = t_w;
   __syncthreads();
-  // T: the smallest warp threshold (lane w reads warp w's, a butterfly takes the minimum)
-  uint64_t T = lane < nw ? warp_t[lane] : ~0ull;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const uint64_t y = shfl_xor_u64(T, o);
-    T = y < T ? y : T;
-  }
-  const bool p0 = v0 != 0ull && v0 >= T, p1 = v1 != 0ull && v1 >= T;
-  const bool p2 = v2 != 0ull && v2 >= T, p3 = v3 != 0ull && v3 >= T;
+  // T: the smallest warp threshold
+  const uint32_t T = __reduce_min_sync(0xffffffffu, lane < nw ? warp_t32[lane] : 0xffffffffu);
+  const bool p0 = v0 != 0ull && (uint32_t)(v0 >> 32) >= T, p1 = v1 != 0ull && (uint32_t)(v1 >> 32) >= T;
+  const bool p2 = v2 != 0ull && (uint32_t)(v2 >> 32) >= T, p3 = v3 != 0ull && (uint32_t)(v3 >> 32) >= T;
   const unsigned b0 = __ballot_sync(0xffffffffu, p0), b1 = __ballot_sync(0xffffffffu, p1);
   const unsigned b2 = __ballot_sync(0xffffffffu, p2), b3 = __ballot_sync(0xffffffffu, p3);
   const int n0 = __popc(b0), n1 = __popc(b1), n2 = __popc(b2), n3 = __popc(b3);
