@@ -179,11 +179,23 @@ class ClockSampler:
 # ----------------------------------------------------------------------------
 # the GPU arm
 # ----------------------------------------------------------------------------
+def source_digest(names) -> str:
+    """sha256 over the named csrc files with // comments and blank lines removed: a change
+    to the code (not to its comments) changes the digest."""
+    h = hashlib.sha256()
+    for name in names:
+        for line in open(os.path.join(ROOT, "long_context_memory_b200", "csrc", name), encoding="utf-8"):
+            code = line.split("//", 1)[0].rstrip()
+            if code:
+                h.update(code.encode() + b"\n")
+    return h.hexdigest()
+
+
 def scan_traffic_record(kernel: str):
     """Per-launch DRAM bytes of `kernel` from a committed ncu summary, or None.
 
-    A summary records the sha256 of the kernel's source file; if the source has
-    changed since the counters were taken the figure is stale and not used."""
+    A summary records the digest of the kernel's source files (`source_digest`); if the code
+    has changed since the counters were taken the figure is stale and not used."""
     path = os.path.join(ROOT, "profiles", f"{kernel}_traffic.txt")
     if not os.path.exists(path):
         return None
@@ -192,12 +204,12 @@ def scan_traffic_record(kernel: str):
         if ":" in line and not line.startswith("#"):
             a, b = line.split(":", 1)
             kv[a.strip()] = b.strip()
-    src = os.path.join(ROOT, "long_context_memory_b200", "csrc", kv.get("source", ""))
-    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != kv.get("source_sha256"):
-        return None
+    names = kv.get("sources", "").split()
     try:
+        if not names or source_digest(names) != kv.get("code_sha256"):
+            return None
         return float(kv["dram_bytes_per_launch_full_size"])
-    except (KeyError, ValueError):
+    except (OSError, KeyError, ValueError):
         return None
 
 

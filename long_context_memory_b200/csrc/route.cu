@@ -8,16 +8,20 @@
 // with the memory size (complexity item of the same section: O(ML/P)).
 //
 // Kernels, in launch order:
-//   router_query_kernel  Q^R = H_q W^QR (CTA = a row slab of one head's columns,
-//                    split-K partials summed in a fixed order by the head's
-//                    last CTA), per-head normalisation, bf16 hi + lo rows for
-//                    the scan's TMA; clears the doc keys
-//   scan_kernel      TMA-staged streaming scan of K̄^R: tensor-core dots and
-//                    Gram diagonal (norm), cosine, head mean, per-document
-//                    segmented max folded in with atomicMax on ordered keys
+//   router_query_kernel  Q^R = H_q W^QR (a thread-block cluster per router head,
+//                    each CTA a row slab of the head's columns; the split-K
+//                    partials meet in distributed shared memory in rank order),
+//                    per-head normalisation, bf16 hi + lo rows for the scan's
+//                    TMA; clears the doc keys
+//   scan_kernel      TMA-staged streaming scan of K̄^R: tensor-core dots,
+//                    cosine (precomputed or in-kernel key norms), head mean,
+//                    per-document segmented max folded in with atomicMax on
+//                    ordered keys; for few queries over one slice of documents
+//                    its last CTA also selects the top-k
 //   topk_slice_kernel / topk_merge_kernel
-//                    exact radix select of the top-k (score, id) keys per
-//                    slice of documents, then a merge of the slice winners
+//                    exact top-k of the (score, id) keys per slice of
+//                    documents (warp thresholds, a bitonic fallback, or a radix
+//                    select for k > 32), then a merge of the slice winners
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -55,8 +59,9 @@ constexpr float kEps = 1e-12f;
 //
 // Grid (8, n_r), one thread-block cluster of 8 CTAs per router head: CTA r of
 // head h multiplies rows [r*RS, (r+1)*RS) of W^QR's head-h column block (staged in
-// shared memory 256 rows at a time, coalesced) by the matching slice of 16 query
-// rows on the tensor cores (mma.sync m16n8k16, bf16 in, fp32 out).  The 8 partial
+// shared memory with asynchronous 16-byte copies, kRqPiece rows at a time) by the
+// matching slice of 16 query rows on the tensor cores (mma.sync m16n8k16, bf16 in,
+// fp32 out).  The 8 partial
 // products meet in distributed shared memory: after a cluster barrier CTA r sums,
 // in rank order, rows r and r + 8 of the 16-row block over the cluster's CTAs,
 // normalises them and writes their hi/lo terms.  No global partials, no counters.
