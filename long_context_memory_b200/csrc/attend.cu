@@ -639,6 +639,58 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(__nv_bfloat16* __restric
   }
 }
 
+// log-sum-exp merge with one warp per (query token, q head), 8 per CTA: for many query tokens
+// (short CTAs are launched at a limited rate, so a CTA per head or per slice costs more than the
+// merge).  Lane l holds dims l*W .. l*W + W - 1; each split's weight is computed by the lane that
+// loaded its (m, l) and broadcast with a shuffle; no shared memory, no block barrier.
+template <int D>
+__global__ void __launch_bounds__(256) attn_combine_warp_kernel(const float* __restrict__ part_ml,
+                                                                const float* __restrict__ part_o, int n_splits,
+                                                                int n_rows, __nv_bfloat16* __restrict__ out) {
+  constexpr int W = D / 32;
+  pdl_enter();
+  const int lane = threadIdx.x & 31;
+  const size_t qh = (size_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (qh >= (size_t)n_rows) return;
+  const float* ml = part_ml + qh * n_splits * 2;
+  const float* po = part_o + qh * n_splits * D + lane * W;
+  float m = -INFINITY;
+  for (int sp = lane; sp < n_splits; sp += 32) m = fmaxf(m, ml[2 * sp]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const float Mu = (m == -INFINITY) ? 0.f : m;
+  float l = 0.f, acc[W];
+#pragma unroll
+  for (int e = 0; e < W; ++e) acc[e] = 0.f;
+  for (int base = 0; base < n_splits; base += 32) {
+    const int sp = base + lane;
+    float w = 0.f;
+    if (sp < n_splits) {
+      w = exp2f(ml[2 * sp] - Mu);
+      l = fmaf(w, ml[2 * sp + 1], l);
+    }
+    const int cnt = min(32, n_splits - base);
+#pragma unroll 8
+    for (int j = 0; j < cnt; ++j) {
+      const float wj = __shfl_sync(0xffffffffu, w, j);
+      const float* src = po + (size_t)(base + j) * D;
+      if constexpr (W == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(src);
+        acc[0] = fmaf(wj, v.x, acc[0]); acc[1] = fmaf(wj, v.y, acc[1]);
+        acc[2] = fmaf(wj, v.z, acc[2]); acc[3] = fmaf(wj, v.w, acc[3]);
+      } else {
+        const float2 v = *reinterpret_cast<const float2*>(src);
+        acc[0] = fmaf(wj, v.x, acc[0]); acc[1] = fmaf(wj, v.y, acc[1]);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+  const float inv = l > 0.f ? 1.0f / l : 0.f;
+#pragma unroll
+  for (int e = 0; e < W; ++e) out[qh * D + lane * W + e] = __float2bfloat16_rn(acc[e] * inv);
+}
+
 // the decode step's new token into the rotated cache: CTA = one query; key rotated at
 // pos_offset + slot, value copied (D/2 pairs x n_kv heads per thread block)
 template <int D>
@@ -951,14 +1003,20 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
   if (phase != 1) {  // the local-keys phase leaves its partials for the selected-chunks phase's combine
     TraceScope ts(kKAttnCombine, s);
     // few query tokens: a CTA per 32-dim slice of each head (enough CTAs to fill the GPU);
-    // many: a CTA per head
-    const bool sliced = (long long)B * M * d.n_q < 2LL * sm_count();
-    dim3 grid(d.n_q, B * M, sliced ? D / 32 : 1);
+    // many: a warp per head, 8 per CTA
+    const long long rows = (long long)B * M * d.n_q;
     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
-    auto kern = D == 128 ? (sliced ? attn_combine_kernel<128, 4> : attn_combine_kernel<128, 1>)
-                         : (sliced ? attn_combine_kernel<64, 2> : attn_combine_kernel<64, 1>);
-    MSA_CUDA_CHECK(launch_pdl(kern, grid, dim3(256), 0, s, (const float*)w.part_ml, (const float*)w.part_o, p.n_parts,
-                              o));
+    if (rows < 2LL * sm_count()) {
+      dim3 grid(d.n_q, B * M, D / 32);
+      auto kern = D == 128 ? attn_combine_kernel<128, 4> : attn_combine_kernel<64, 2>;
+      MSA_CUDA_CHECK(launch_pdl(kern, grid, dim3(256), 0, s, (const float*)w.part_ml, (const float*)w.part_o,
+                                p.n_parts, o));
+    } else {
+      dim3 grid((unsigned)((rows + 7) / 8));
+      auto kern = D == 128 ? attn_combine_warp_kernel<128> : attn_combine_warp_kernel<64>;
+      MSA_CUDA_CHECK(launch_pdl(kern, grid, dim3(256), 0, s, (const float*)w.part_ml, (const float*)w.part_o,
+                                p.n_parts, (int)rows, o));
+    }
   }
   return MSA_OK;
 }
