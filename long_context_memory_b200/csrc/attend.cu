@@ -9,13 +9,18 @@
 //
 // Kernels:
 //   rope_table_kernel    cos/sin of (pos_offset + j) * theta_i for every local
-//                        position j, angle reduced in fp64
-//   attn_split_kernel    split-KV flash-decode: CTA = (split, KV head, query);
-//                        gathers its key/value rows with per-row bulk async
-//                        copies into padded shared memory, QK^T and PV on the
-//                        tensor cores (mma.sync, the GQA group as the M rows),
-//                        local keys rotated in registers, online softmax
-//   attn_combine_kernel  log-sum-exp merge of the split partials -> bf16
+//                        position j (angles from 64-bit fixed-point turns)
+//   attn_split_kernel    split-KV flash-decode, persistent: each CTA takes work
+//                        items (a run of local keys, or a run of the selected
+//                        chunks, of one query token group); a producer warp
+//                        gathers the rows with per-row bulk async copies into
+//                        padded shared memory; one compute warp per KV head runs
+//                        QK^T and PV on the tensor cores (mma.sync, the GQA group
+//                        x the CTA's query tokens as the M rows), rotates local
+//                        keys in registers when needed, online softmax; the local
+//                        items can run before the routing result is known
+//   attn_combine_kernel, attn_combine_warp_kernel
+//                        log-sum-exp merge of the split partials -> bf16
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
