@@ -595,10 +595,11 @@ def run_gpu(args):
                     "graph_ms_per_step": e2e_graph_ms,
                     "graph_value": T * B * ws / (e2e_graph_ms * 1e-3) if e2e_graph_ms else None},
             "cpu_baseline": cpu, "clocks": clocks, "extras": extras,
-            "notes": "value: device time of CUDA-graph replays of the full decode step (route, append the new "
-                     "token's rotated key and value to the local cache, sparse attention over the rotated cache); "
-                     "kernels: trace-event "
-                     "brackets of eager launches queued behind a bounded sleep kernel",
+            "notes": "value: device time of CUDA-graph replays of the full decode step (append the new token's "
+                     "rotated key and value to the local cache, route with early inputs, sparse attention over the "
+                     "rotated cache with early local work); kernels: trace-event brackets of eager launches queued "
+                     "behind a bounded sleep kernel; e2e: the same calls issued eagerly with one packed copy each "
+                     "way per step",
         }
         print(json.dumps(line), flush=True)
     if ws > 1:
