@@ -389,18 +389,17 @@ def run_gpu(args):
     torch.cuda.synchronize()
 
     def step(i):
-        # one stream: the new token into the rotated local cache, routing, sparse attention.  The
-        # routing's query and memory are not written by the append (early_inputs: the router query
-        # multiplies and the scan streams while the append runs); the attention's local-key work
-        # starts while the routing's kernels finish (early_local: q and the local cache are not
-        # written by the routing).
+        # one stream: routing, then sparse attention, which first writes the new token's rotated key
+        # and value into the local cache (k_new / v_new: the append fused into the call).  The
+        # attention's local-key work starts while the routing's kernels finish (early_local: q and
+        # the local cache are not written by the routing).
         x = rot[i % N_ROT]
         j = i % N_ROT
-        msa.kv_append(d, k_new, v_new, x["K_loc"], x["V_loc"], slots, c["pos_offset"])
         msa.route_topk(d, x["Hq"], W_QR, x["KR"], chunk_off, k, out=(out_idx[j], out_sc[j], None), ws=r_ws,
-                       kr_inv_norm=inv_rot[j], early_inputs=True)
+                       kr_inv_norm=inv_rot[j])
         msa.sparse_attend(d, x["q"], x["K_bar"], x["V_bar"], chunk_off, out_idx[j], x["K_loc"], x["V_loc"], loc_len,
-                          c["pos_offset"], out=out_o[j], ws=a_ws, k_loc_rotated=True, early_local=True)
+                          c["pos_offset"], out=out_o[j], ws=a_ws, k_loc_rotated=True, early_local=True,
+                          k_new=k_new, v_new=v_new)
 
     # ---- capture one graph per rotation copy (untraced) ----
     graphs = []
@@ -522,11 +521,11 @@ def run_gpu(args):
     def e2e_step(i):
         x = rot[i % N_ROT]
         dev_in.copy_(host_in, non_blocking=True)
-        msa.kv_append(d, dev_kn, dev_vn, x["K_loc"], x["V_loc"], slots, c["pos_offset"])
         msa.route_topk(d, dev_hq, W_QR, x["KR"], chunk_off, k, out=(e_idx, e_sc, None), ws=r_ws,
-                       kr_inv_norm=inv_rot[i % N_ROT], early_inputs=True)
+                       kr_inv_norm=inv_rot[i % N_ROT])
         msa.sparse_attend(d, dev_q, x["K_bar"], x["V_bar"], chunk_off, e_idx, x["K_loc"], x["V_loc"], loc_len,
-                          c["pos_offset"], out=e_out, ws=a_ws, k_loc_rotated=True, early_local=True)
+                          c["pos_offset"], out=e_out, ws=a_ws, k_loc_rotated=True, early_local=True,
+                          k_new=dev_kn, v_new=dev_vn)
         host_out.copy_(dev_out, non_blocking=True)
 
     def e2e_time(run):
@@ -596,8 +595,9 @@ def run_gpu(args):
                     "graph_value": T * B * ws / (e2e_graph_ms * 1e-3) if e2e_graph_ms else None},
             "cpu_baseline": cpu, "clocks": clocks, "extras": extras,
             "notes": "value: device time of CUDA-graph replays of the full decode step (append the new token's "
-                     "rotated key and value to the local cache, route with early inputs, sparse attention over the "
-                     "rotated cache with early local work); kernels: trace-event brackets of eager launches queued "
+                     "rotated key and value to the local cache (fused into the attention call), route, sparse "
+                     "attention over the rotated cache with early local work); kernels: trace-event brackets of eager "
+                     "launches queued "
                      "behind a bounded sleep kernel; e2e: the same calls issued eagerly with one packed copy each "
                      "way per step",
         }

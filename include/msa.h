@@ -304,6 +304,13 @@ msa_status msa_aux_loss(const msa_dims* dims, const void* QR, const void* K_pos,
  *            dependent launch).  The flag has no effect when the call builds its own
  *            rotation table (k_loc_rotated 0 and rope_cache NULL).  The result is the same
  *            as without the flag.
+ *   k_new, v_new  optional [B, n_kv, head_dim] bf16 (both or neither; M = 1; not phase 2):
+ *            the decode step's new token, the query's own key (before RoPE) and value.
+ *            The call first writes them at slot loc_len[b] - 1 of K_loc / V_loc (the key
+ *            rotated at pos_offset + slot when k_loc_rotated is 1, as msa_kv_append does;
+ *            unrotated otherwise) and attends over the cache as written: the same result
+ *            as msa_kv_append followed by this call, one launch fewer.  K_loc and V_loc are
+ *            then written (a loc_len of 0 raises the device error bit 1 and writes nothing).
  *   out      [B, M, n_q, head_dim] bf16.
  * Limits: 1 <= M, B * M <= 65535.
  * Query head g attends with KV head g / (n_q / n_kv).  Every query token sees
@@ -318,7 +325,8 @@ size_t msa_attend_workspace_size(const msa_dims* dims, int32_t B, int32_t q_toke
                                  int32_t t_loc_max, int32_t pos_offset);
 msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, int32_t q_tokens, const void* K_bar,
                              const void* V_bar, const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks,
-                             const int32_t* topk_idx, int32_t k, const void* K_loc, const void* V_loc,
+                             const int32_t* topk_idx, int32_t k, void* K_loc, void* V_loc,
+                             const void* k_new, const void* v_new,
                              const int32_t* loc_len, int32_t t_loc_max, int32_t pos_offset,
                              const void* rope_cache, int32_t k_loc_rotated, float softmax_scale, int32_t phase,
                              void* out, void* ws, size_t ws_bytes, void* stream);

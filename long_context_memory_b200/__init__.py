@@ -83,7 +83,7 @@ def _load():
         "msa_route_topk": (I32, [DP, P, P, I32, I32, P, P, I32, I32, I32, I32, I32, P, P, P, P, P, SZ, P]),
         "msa_router_key_norms": (I32, [DP, P, I32, I32, P, P]),
         "msa_attend_workspace_size": (SZ, [DP, I32, I32, I32, I32, I32]),
-        "msa_sparse_attend": (I32, [DP, P, I32, I32, P, P, P, I32, I32, P, I32, P, P, P, I32, I32, P, I32, F, I32, P, P,
+        "msa_sparse_attend": (I32, [DP, P, I32, I32, P, P, P, I32, I32, P, I32, P, P, P, P, P, I32, I32, P, I32, F, I32, P, P,
                                     SZ, P]),
         "msa_rope_rows": (I32, [DP, P, I32, I32, P, P]),
         "msa_kv_append": (I32, [DP, P, P, P, P, I32, I32, P, I32, P]),
@@ -356,7 +356,7 @@ def kv_append(dims, k_new, v_new, K_loc, V_loc, slots, pos_offset: int, stream=N
 
 def sparse_attend(dims, q, K_bar, V_bar, chunk_off, topk_idx, K_loc, V_loc, loc_len, pos_offset: int,
                   softmax_scale: float = 0.0, out=None, ws=None, stream=None, rope_cache=None,
-                  k_loc_rotated: bool = False, phase: int = 0, early_local: bool = False):
+                  k_loc_rotated: bool = False, phase: int = 0, early_local: bool = False, k_new=None, v_new=None):
     """GQA attention of the query tokens over [selected docs' K̄; local K].
 
     ``q`` is [B, n_q, head_dim] (one decode token) or [B, M, n_q, head_dim] (the last M local
@@ -366,7 +366,10 @@ def sparse_attend(dims, q, K_bar, V_bar, chunk_off, topk_idx, K_loc, V_loc, loc_
     local-keys part and the selected-chunks part (which merges both); pass the same ``ws``.
     ``early_local`` (MSA_ATTEND_EARLY_LOCAL) lets the local-key work start before the
     preceding library call's kernels finish; q, K_loc, V_loc and loc_len must have been final
-    before that call was enqueued, and it must not be a sparse_attend on the same ``ws``."""
+    before that call was enqueued, and it must not be a sparse_attend on the same ``ws``.
+    ``k_new``/``v_new`` [B, n_kv, head_dim] (decode, M = 1): the new token's key (before RoPE) and
+    value are first written at slot loc_len - 1 of K_loc/V_loc (the key rotated when
+    ``k_loc_rotated``), as ``kv_append`` would, and the call attends over the cache as written."""
     import torch
 
     dd = Dims.of(dims)
@@ -383,7 +386,8 @@ def sparse_attend(dims, q, K_bar, V_bar, chunk_off, topk_idx, K_loc, V_loc, loc_
         nbytes = attend_workspace_size(dims, B, k, t_loc_max, pos_offset, M)
         ws = _workspace(nbytes, dev, ws)
     _check(lib.msa_sparse_attend(ctypes.byref(dd), _ptr(q), B, M, _ptr(K_bar), _ptr(V_bar), _ptr(chunk_off), n_docs,
-                                 K_bar.shape[0], _ptr(topk_idx), k, _ptr(K_loc), _ptr(V_loc), _ptr(loc_len),
+                                 K_bar.shape[0], _ptr(topk_idx), k, _ptr(K_loc), _ptr(V_loc), _ptr(k_new), _ptr(v_new),
+                                 _ptr(loc_len),
                                  t_loc_max, pos_offset, _ptr(rope_cache), int(bool(k_loc_rotated)),
                                  float(softmax_scale), int(phase) | (ATTEND_EARLY_LOCAL if early_local else 0),
                                  _ptr(out),

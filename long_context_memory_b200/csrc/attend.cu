@@ -73,6 +73,9 @@ struct AttnParams {
   const __nv_bfloat16* K_loc;
   const __nv_bfloat16* V_loc;
   const int32_t* loc_len;
+  const __nv_bfloat16* k_new;  // [B][n_kv][D] the new token's key (before RoPE), or null: no append
+  const __nv_bfloat16* v_new;  // [B][n_kv][D] its value
+  int append_rotate;           // the appended key is rotated at its position (rotated cache)
   const float2* rope_tab;
   float* part_ml;
   float* part_o;
@@ -195,7 +198,9 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
       const bool is_chunk = it >= n_loc_items;
       const int i2 = is_chunk ? it - n_loc_items : it;
       const int ns = is_chunk ? p.n_chunk_splits : p.n_loc_splits;
-      const int split = i2 % ns, bq = i2 / ns;
+      // a query's local splits run last-first: the last one (it holds the newest local row, which
+      // a fused append writes first) goes to the lowest CTA, which starts earliest
+      const int split = is_chunk ? i2 % ns : ns - 1 - i2 % ns, bq = i2 / ns;
       const int b = bq / p.n_tgroups, t0 = (bq % p.n_tgroups) * MT;
       const int nt = min(MT, p.q_tokens - t0);
       if (j >= 2) mbar_wait(&hempty[hb], ((j >> 1) - 1) & 1);  // item j-2's header and query read
@@ -262,6 +267,37 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
         hd[4] = n_sel; hd[5] = v0; hd[6] = v1;
         hd[7] = is_chunk ? p.chunk_part_base + split : split;  // the item's partial slot
         mbar_arrive(&hsel[hb]);  // releases the key-range writes
+      }
+      if (p.k_new && !is_chunk) {
+        if (v1 == L && v1 > v0) {
+          // the item holding the query's last local row writes the new token there first (no
+          // other item reads that row): key rotated at its position (or as given), value copied;
+          // then orders the writes before its bulk copies read the row back
+          const int slot = L - 1;
+          const size_t src = (size_t)b * n_kv * D;
+          const size_t dst = ((size_t)b * p.t_loc_max + slot) * n_kv * D;
+          __nv_bfloat16* kd = const_cast<__nv_bfloat16*>(p.K_loc) + dst;
+          __nv_bfloat16* vd = const_cast<__nv_bfloat16*>(p.V_loc) + dst;
+          for (int e = lane; e < n_kv * (D / 2); e += 32) {
+            const int hh = e / (D / 2), i = e % (D / 2);
+            const __nv_bfloat16* kr = p.k_new + src + (size_t)hh * D;
+            if (p.append_rotate) {
+              const float2 cs = rope_cos_sin(p.turns, i, (int64_t)p.pos_offset + slot);
+              const float x1 = __bfloat162float(kr[i]), x2 = __bfloat162float(kr[i + D / 2]);
+              kd[(size_t)hh * D + i] = __float2bfloat16_rn(x1 * cs.x - x2 * cs.y);
+              kd[(size_t)hh * D + i + D / 2] = __float2bfloat16_rn(x2 * cs.x + x1 * cs.y);
+            } else {
+              kd[(size_t)hh * D + i] = kr[i];
+              kd[(size_t)hh * D + i + D / 2] = kr[i + D / 2];
+            }
+          }
+          for (int e = lane; e < n_kv * D / 8; e += 32)
+            reinterpret_cast<uint4*>(vd)[e] = __ldg(reinterpret_cast<const uint4*>(p.v_new + src) + e);
+          fence_proxy_async_global();
+          __syncwarp();
+        } else if (L == 0 && split == 0 && lane == 0) {
+          raise_dev_error(kDevErrBadIndex);  // no local position to take the new token
+        }
       }
       // ---- the item's tiles: kTK keys each, a bulk copy per key and tensor plus the RoPE rows ----
       for (int t = 0; t < n_tiles; ++t, ++gt) {
@@ -940,7 +976,8 @@ msa_status kv_append_launch(const msa_dims& d, const void* k_new, const void* v_
 
 msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const void* K_bar, const void* V_bar,
                          const int32_t* chunk_off, int n_docs, const int32_t* topk_idx, int k, const void* K_loc,
-                         const void* V_loc, const int32_t* loc_len, int t_loc_max, int pos_offset,
+                         const void* V_loc, const void* k_new, const void* v_new, const int32_t* loc_len,
+                         int t_loc_max, int pos_offset,
                          const void* rope_cache, int k_loc_rotated, float scale, int phase, int early, void* out,
                          void* ws, cudaStream_t s) {
   AttendWs w;
@@ -962,6 +999,9 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
   p.K_loc = static_cast<const __nv_bfloat16*>(K_loc);
   p.V_loc = static_cast<const __nv_bfloat16*>(V_loc);
   p.loc_len = loc_len;
+  p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  p.append_rotate = k_loc_rotated ? 1 : 0;
   p.rope_tab = tab;
   p.part_ml = w.part_ml;
   p.part_o = w.part_o;

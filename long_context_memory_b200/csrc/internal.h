@@ -159,7 +159,8 @@ size_t attend_workspace(const msa_dims& d, int B, int M, int k, int t_loc_max, i
                         struct AttendWs* out);
 msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const void* K_bar, const void* V_bar,
                          const int32_t* chunk_off, int n_docs, const int32_t* topk_idx, int k,
-                         const void* K_loc, const void* V_loc, const int32_t* loc_len, int t_loc_max,
+                         const void* K_loc, const void* V_loc, const void* k_new, const void* v_new,
+                         const int32_t* loc_len, int t_loc_max,
                          int pos_offset, const void* rope_cache, int k_loc_rotated, float scale, int phase,
                          int early, void* out, void* ws, cudaStream_t s);
 msa_status gather_kv_launch(const msa_dims& d, const void* K_host, const void* V_host, const int32_t* chunk_off,

@@ -427,8 +427,8 @@ size_t msa_attend_workspace_size(const msa_dims* dims, int32_t B, int32_t q_toke
 msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, int32_t q_tokens, const void* K_bar,
                              const void* V_bar,
                              const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks, const int32_t* topk_idx,
-                             int32_t k, const void* K_loc, const void* V_loc, const int32_t* loc_len,
-                             int32_t t_loc_max, int32_t pos_offset, const void* rope_cache,
+                             int32_t k, void* K_loc, void* V_loc, const void* k_new, const void* v_new,
+                             const int32_t* loc_len, int32_t t_loc_max, int32_t pos_offset, const void* rope_cache,
                              int32_t k_loc_rotated, float softmax_scale, int32_t phase, void* out, void* ws,
                              size_t ws_bytes, void* stream) {
   msa_status st = check_dims(dims, true, false);
@@ -463,12 +463,18 @@ msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, int
   }
   CHECK_PTR(loc_len);
   CHECK_OPT_PTR(rope_cache);
+  CHECK_OPT_PTR(k_new);
+  CHECK_OPT_PTR(v_new);
+  if ((k_new == nullptr) != (v_new == nullptr)) return fail(MSA_ERR_INVALID_ARG, "k_new and v_new go together");
+  if (k_new && (q_tokens != 1 || phase == 2 || t_loc_max < 1))
+    return fail(MSA_ERR_INVALID_ARG, "the fused append needs q_tokens 1, a local cache and phase 0 or 1");
   const size_t need = attend_workspace(*dims, B, q_tokens, k, t_loc_max, pos_offset, nullptr, nullptr);
   if (ws_bytes < need) return fail(MSA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
   if (need && (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)))
     return fail(MSA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
   if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
-  return attend_launch(*dims, q, B, q_tokens, K_bar, V_bar, chunk_off, n_docs, topk_idx, k, K_loc, V_loc, loc_len, t_loc_max,
+  return attend_launch(*dims, q, B, q_tokens, K_bar, V_bar, chunk_off, n_docs, topk_idx, k, K_loc, V_loc, k_new,
+                       v_new, loc_len, t_loc_max,
                        pos_offset, rope_cache, k_loc_rotated, softmax_scale, phase, early, out, ws,
                        static_cast<cudaStream_t>(stream));
 }

@@ -109,13 +109,14 @@ def test_route_fault_injection_before_launch(msa, monkeypatch):
 
 
 def _attend(msa, dims, B=1, k=2, n_docs=4, n_chunks=8, t_loc=16, pos=2, scale=0.0, ws_bytes=None, q=FAKE, M=1,
-            phase=0):
+            phase=0, k_new=None, v_new=None):
     dd = msa.Dims.of(dims)
     need = msa.lib.msa_attend_workspace_size(ctypes.byref(dd), B, max(M, 1), k, t_loc, pos)
     if ws_bytes is None:
         ws_bytes = need
     return msa.lib.msa_sparse_attend(ctypes.byref(dd), q, B, M, FAKE, FAKE, FAKE, n_docs, n_chunks, FAKE, k, FAKE, FAKE,
-                                     FAKE, t_loc, pos, None, 0, scale, phase, FAKE, 0x100000, ws_bytes, None)
+                                     k_new, v_new, FAKE, t_loc, pos, None, 0, scale, phase, FAKE, 0x100000, ws_bytes,
+                                     None)
 
 
 def test_attend_validation(msa):
@@ -134,6 +135,11 @@ def test_attend_validation(msa):
     assert _attend(msa, ok, phase=3 | msa.ATTEND_EARLY_LOCAL) == 1  # the flag does not make a bad phase valid
     assert _attend(msa, ok, phase=-1) == 1
     assert _attend(msa, ok, phase=msa.ATTEND_EARLY_LOCAL | 32) == 1  # an unknown flag bit
+    assert _attend(msa, ok, k_new=FAKE) == 1                        # k_new without v_new
+    assert _attend(msa, ok, k_new=FAKE, v_new=FAKE, M=2) == 1       # the fused append is for M = 1
+    assert _attend(msa, ok, k_new=FAKE, v_new=FAKE, phase=2) == 1   # phase 2 reads no local keys
+    assert _attend(msa, ok, k_new=FAKE, v_new=FAKE, t_loc=0) == 1   # no local cache to write
+    assert _attend(msa, ok, k_new=FAKE + 2, v_new=FAKE) == 1        # misaligned
 
 
 def test_encode_validation(msa):

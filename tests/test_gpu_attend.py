@@ -377,3 +377,51 @@ def test_attend_early_local_behind_routing(msa, cuda_device, B, M):
     else:
         ref = O.sparse_attend_tokens(q_np, K_bar_np, V_bar_np, co, topk, K_loc_ref, V_loc_np, loc_len_np, o, 1e6)
     check_attention(outs[0], ref, where=f"early B={B} M={M}")
+
+
+@pytest.mark.parametrize("rotated", [True, False])
+@pytest.mark.parametrize("early", [False, True])
+def test_attend_fused_append_equals_append_then_attend(msa, cuda_device, rotated, early):
+    # sparse_attend with k_new / v_new = the new token written at slot loc_len - 1 (rotated at its
+    # position for a rotated cache, as kv_append does; as given for a pre-RoPE cache), then the
+    # attention: the same output and the same cache, bit for bit
+    import torch
+
+    B, n_q, n_kv, D, T, o = 3, 32, 8, 128, 300, 6
+    c = _case(820 + rotated + 2 * early, B, n_q, n_kv, D, n_docs=30, k=5, t_loc=T, loc_len=[T, 57, 1])
+    dims = W.Dims(hidden=256, n_q=n_q, n_kv=n_kv, head_dim=D, n_r=4, d_r=64, rope_base=1e6)
+    dev = cuda_device
+    rng = np.random.default_rng(821)
+    kn = _dev(W.normal_bf16(rng, (B, n_kv, D)), dev)
+    vn = _dev(W.normal_bf16(rng, (B, n_kv, D)), dev)
+    co, C = msa.chunk_offsets(c["doc_off"])
+    K0 = _dev(c["K_loc"], dev)
+    if rotated:
+        msa.rope_rows(dims, K0.view(B * T, n_kv, D), (o + torch.arange(T, dtype=torch.int32, device=dev)).repeat(B))
+    V0 = _dev(c["V_loc"], dev)
+    loc_len = torch.from_numpy(c["loc_len"].astype(np.int32)).to(dev)
+    slots = loc_len - 1
+    args = (_dev(c["q"], dev), _dev(c["K_bar"], dev), _dev(c["V_bar"], dev), torch.from_numpy(co).to(dev),
+            torch.from_numpy(c["topk"].astype(np.int32)).to(dev))
+    K1, V1, K2, V2 = K0.clone(), V0.clone(), K0.clone(), V0.clone()
+    if rotated:
+        msa.kv_append(dims, kn, vn, K1, V1, slots, o)
+    else:
+        for b in range(B):
+            K1[b, int(slots[b])] = kn[b]
+            V1[b, int(slots[b])] = vn[b]
+    ref = msa.sparse_attend(dims, *args, K1, V1, loc_len, o, k_loc_rotated=rotated)
+    out = msa.sparse_attend(dims, *args, K2, V2, loc_len, o, k_loc_rotated=rotated, early_local=early,
+                            k_new=kn, v_new=vn)
+    torch.cuda.synchronize()
+    assert msa.check_device_errors() == 0
+    assert torch.equal(K1, K2) and torch.equal(V1, V2)
+    assert torch.equal(ref, out)
+    # no local position for the new token: reported, nothing written
+    K3, V3 = K0.clone(), V0.clone()
+    zero = torch.zeros_like(loc_len)
+    msa.sparse_attend(dims, *args, K3, V3, zero, o, k_loc_rotated=rotated, k_new=kn, v_new=vn)
+    torch.cuda.synchronize()
+    with pytest.raises(msa.MSAError, match="out-of-range index"):
+        msa.check_device_errors()
+    assert torch.equal(K3, K0) and torch.equal(V3, V0)
