@@ -293,7 +293,8 @@ msa_status msa_aux_loss(const msa_dims* dims, const void* QR, const void* K_pos,
  *            and out are not read and may be NULL); phase 2, with the same ws and sizes,
  *            attends over the selected chunks and merges both parts into out (K_loc and
  *            V_loc are not read).  Phase 2 must be ordered after phase 1 (same stream, or
- *            an event).  The result equals phase 0's up to fp32 summation order.
+ *            an event).  The result equals phase 0's bit for bit (the same work items and
+ *            partial slots).
  *            phase | MSA_ATTEND_EARLY_LOCAL (phases 0 and 1): the work on the local keys may
  *            start before the preceding work on the stream has finished (typically
  *            msa_route_topk producing topk_idx), hiding it behind the routing.  The caller
