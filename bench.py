@@ -5,7 +5,8 @@ One step = one pass of the whole online path for one batch of queries:
 msa_route_topk (projection from H_q, scan + per-document max, top-k) followed by
 msa_sparse_attend (gather of the selected docs' pooled K̄/V̄ + local KV with
 global RoPE, split-KV flash-decode, combine).  Inputs are synthetic (seeded) with
-the shapes of the 1M-token, Qwen3-4B-like workload; see the design doc.
+the shapes of the 1M-token, Qwen3-4B-like workload (documents of varied length,
+32 query heads over 8 KV heads of 128, 8 router heads of 128, top-16, 64-token chunks, 4K local KV, B=1).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl msa|reference]
 
