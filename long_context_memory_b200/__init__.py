@@ -3,8 +3,8 @@
 A thin ctypes layer over ``libmsa.so`` (C ABI declared in ``include/msa.h``).
 It only marshals arguments: every step of the path runs in the library's CUDA
 kernels.  PyTorch supplies device memory (outputs and workspaces) and the
-current stream.  Importing this package fails loudly when the library is
-missing; there is no CPU fallback.
+current stream.  The library is loaded on the first call into it, and that
+call raises ImportError when the library is missing; there is no CPU fallback.
 
 Entry points (same names as the C ABI, minus the ``msa_`` prefix):
   chunk_offsets, encode_memory, append_memory, route_topk, sparse_attend, kv_append, aux_loss,
