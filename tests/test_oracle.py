@@ -205,6 +205,18 @@ def test_route_hand_derived_golden():
     assert list(O.topk(smean, 3)[0]) == g["top3_mean"]
 
 
+def test_router_query_one_hot_rows_and_head_columns():
+    # Q^R = H_q W^QR: a one-hot hidden state picks one row of W^QR; a sum of rows gives the
+    # sum; router head h holds the columns [h d_r, (h + 1) d_r).  W^QR is not symmetric, so
+    # a transposed operand or a head-major reshape gives other numbers.
+    W_QR = np.arange(16, dtype=np.float64).reshape(4, 4)
+    Hq = np.array([[0.0, 1.0, 0.0, 0.0], [1.0, 2.0, 0.0, 0.0]])
+    QR = O.router_query(Hq, W_QR, 2, 2)
+    assert QR.shape == (2, 2, 2)
+    assert np.array_equal(QR[0], [[4.0, 5.0], [6.0, 7.0]])
+    assert np.array_equal(QR[1], [[8.0, 11.0], [14.0, 17.0]])
+
+
 def test_cosine_closed_forms_and_range():
     rng = np.random.default_rng(5)
     x = rng.standard_normal((10, 64))
@@ -257,6 +269,24 @@ def test_max_vs_mean_aggregation_discriminates():
     off = [0, 3, 5]
     assert list(O.topk(O.doc_scores(O.chunk_scores(QR, KR), off, "max")[0], 1)[0]) == [0]
     assert list(O.topk(O.doc_scores(O.chunk_scores(QR, KR), off, "mean")[0], 1)[0]) == [1]
+
+
+def test_route_topk_per_query_and_aggregation_by_hand():
+    # the chunks of the aggregation case, two queries: (1, 0) and (0, 1).  Hand values:
+    # query 0 scores the chunks 1, -1/sqrt(1.01) twice, 0.6 twice; query 1 scores them
+    # 0, 0.1/sqrt(1.01) twice, 0.8 twice.
+    QR = np.array([[[1.0, 0.0]], [[0.0, 1.0]]])
+    KR = np.array([[[1.0, 0.0]], [[-1.0, 0.1]], [[-1.0, 0.1]], [[0.6, 0.8]], [[0.6, 0.8]]])
+    off = [0, 3, 5]
+    r = 1.0 / math.sqrt(1.01)
+    s, idx, val = O.route_topk(QR, KR, off, 1, "max")
+    assert np.allclose(s, [[1.0, 0.6], [0.1 * r, 0.8]], atol=1e-15)
+    assert idx.tolist() == [[0], [1]] and np.allclose(val, [[1.0], [0.8]], atol=1e-15)
+    s, idx, val = O.route_topk(QR, KR, off, 1, "mean")
+    assert np.allclose(s, [[(1.0 - 2 * r) / 3, 0.6], [0.2 * r / 3, 0.8]], atol=1e-15)
+    assert idx.tolist() == [[1], [1]]
+    s, idx, _ = O.route_topk(QR, KR, off, 2, "max")
+    assert idx.tolist() == [[0, 1], [1, 0]]
 
 
 @pytest.mark.parametrize("seed", [0, 1, 2])
