@@ -71,6 +71,13 @@ def workload_config():
     return c
 
 
+def workload_label(c) -> str:
+    """The workload's name and sizes, the same on both arms."""
+    return ("mem1m: 1M-token memory (C=%d chunks, %d docs), Qwen3-4B-like dims (hidden 2560, 32q/8kv x 128, "
+            "8 router heads x 128), B=%d, top-%d, %d-token local KV"
+            % (c["KR"].shape[0], len(c["doc_off"]) - 1, c["B"], c["k"], c["t_loc_max"]))
+
+
 # ----------------------------------------------------------------------------
 # oracle timing (cpu_baseline and --impl reference)
 # ----------------------------------------------------------------------------
@@ -115,7 +122,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": args.gpus,
         "steps": steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "mem1m: 1M-token memory, Qwen3-4B-like dims, B=1, top-16, 4K local KV"},
+        "config": {"workload": workload_label(c), "parallelism": "one host thread"},
         "cpu_baseline": {"value": r["value"], "unit": UNIT, "cores": r["cores"], "kind": "oracle",
                          "sample": r["sample"]},
         "e2e": {"value": r["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -584,9 +591,7 @@ def run_gpu(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16 pooled memory, lognormal docs)",
-            "config": {"workload": "mem1m: 1M-token memory (C=%d chunks, %d docs), Qwen3-4B-like dims "
-                                   "(hidden 2560, 32q/8kv x 128, 8 router heads x 128), B=%d, top-%d, %d-token local KV"
-                                   % (C, n_docs, B, k, c["t_loc_max"]),
+            "config": {"workload": workload_label(c),
                        "l2": "8 rotating input copies (%.2f GB) > L2" % (N_ROT * sum(v.numel() * 2 for v in base.values()) / 1e9),
                        "graphs": use_graphs, "parallelism": f"replicas x{ws}"},
             "roofline": roofline, "kernels": kernels, "gpu_launches": gpu_launches,

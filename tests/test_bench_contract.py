@@ -23,4 +23,8 @@ def test_reference_arm_prints_one_contract_line():
     assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
-    assert "workload" in d["config"]
+    # the same workload name and sizes as the GPU arm's line
+    sys.path.insert(0, ROOT)
+    import bench
+
+    assert d["config"]["workload"] == bench.workload_label(bench.workload_config())
