@@ -222,3 +222,46 @@ def test_workspace_sizes_grow_with_problem(msa):
     x = msa.lib.msa_attend_workspace_size(ctypes.byref(d), 1, 1, 16, 4096, 16)
     assert x >= 4096 * 64 * 8   # the local RoPE table alone
     assert msa.lib.msa_attend_workspace_size(ctypes.byref(d), 1, 8, 16, 4096, 16) > x
+
+
+def _header_functions():
+    """name -> (return type, parameter count) of every function declared in msa.h."""
+    src = open(os.path.join(ROOT, "include", "msa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for ret, name, params in re.findall(
+            r"\b(msa_status|size_t|int32_t|const char\s*\*)\s+(msa_[a-z_0-9]+)\s*\(([^)]*)\)\s*;", src):
+        p = params.strip()
+        out[name] = (re.sub(r"\s+", "", ret), 0 if p in ("", "void") else p.count(",") + 1)
+    return out
+
+
+def test_binding_signatures_match_header(msa):
+    # ctypes marshals by the binding's argtypes: a parameter added to the header but not to the
+    # binding would shift every later argument silently
+    hdr = _header_functions()
+    assert set(hdr) == set(declared_symbols())
+    cdll = msa._load()
+    restype = {"msa_status": ctypes.c_int32, "size_t": ctypes.c_size_t, "int32_t": ctypes.c_int32,
+               "constchar*": ctypes.c_char_p}
+    unbound = set()
+    for name, (ret, n) in hdr.items():
+        fn = getattr(cdll, name)
+        if fn.argtypes is None:
+            unbound.add(name)
+            continue
+        assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
+        assert fn.restype is restype[ret], (name, fn.restype, ret)
+    # the one entry point the binding leaves to direct ctypes callers (its test declares it itself)
+    assert unbound == {"msa_route_topk_static"}, unbound
+
+
+def test_binding_constants_match_header(msa):
+    src = open(os.path.join(ROOT, "include", "msa.h")).read()
+    defines = dict((k, int(v)) for k, v in re.findall(r"#define (MSA_[A-Z_]+) (\d+)", src))
+    assert defines["MSA_ROUTE_EARLY_INPUTS"] == msa.ROUTE_EARLY_INPUTS
+    assert defines["MSA_ATTEND_EARLY_LOCAL"] == msa.ATTEND_EARLY_LOCAL
+    enums = dict((k, int(v)) for k, v in re.findall(r"\b(MSA_[A-Z_]+) = (\d+)", src))
+    for code, name in msa.STATUS.items():
+        assert enums[name] == code, name
+    assert enums["MSA_AGG_MAX"] == msa.AGG_MAX and enums["MSA_AGG_MEAN"] == msa.AGG_MEAN
