@@ -28,3 +28,34 @@ def test_reference_arm_prints_one_contract_line():
     import bench
 
     assert d["config"]["workload"] == bench.workload_label(bench.workload_config())
+
+
+def test_traffic_record_follows_the_code_not_the_comments(tmp_path, monkeypatch):
+    # the DRAM-traffic figure is used only while the scan's code hashes to the recorded digest;
+    # comments and blank lines do not count
+    sys.path.insert(0, ROOT)
+    import bench
+
+    csrc = tmp_path / "long_context_memory_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    (csrc / "k.cu").write_text("int f() {  // a comment\n  return 1;\n}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    digest = bench.source_digest(["k.cu"])
+    (tmp_path / "profiles" / "scan_traffic.txt").write_text(
+        f"# capture notes\nsources: k.cu\ncode_sha256: {digest}\ndram_bytes_per_launch_full_size: 1234\n")
+    assert bench.scan_traffic_record("scan") == 1234.0
+    (csrc / "k.cu").write_text("int f() {  // another comment\n\n  return 1;\n}\n")
+    assert bench.scan_traffic_record("scan") == 1234.0
+    (csrc / "k.cu").write_text("int f() {\n  return 2;\n}\n")
+    assert bench.scan_traffic_record("scan") is None
+    assert bench.scan_traffic_record("no_such_kernel") is None
+
+
+def test_profiles_are_short_text_summaries_with_their_commands():
+    d = os.path.join(ROOT, "profiles")
+    for f in sorted(os.listdir(d)):
+        assert f.endswith((".md", ".txt")), f
+        text = open(os.path.join(d, f), encoding="utf-8").read()
+        assert len(text) < 16_000, f
+        assert any(cmd in text for cmd in ("ncu ", "nvcc ")), f"{f} does not give the command that made it"
