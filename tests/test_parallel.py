@@ -55,7 +55,7 @@ def oracle_merge(cand_s, cand_i, k):
     return torch.tensor(np.array(out_i), dtype=torch.int32), torch.tensor(np.array(out_s), dtype=torch.float32)
 
 
-def _rank_main(rank, world, port, seed, k, dup, ret):
+def _rank_main(rank, world, port, seed, k, dup, ret, n_docs=60):
     import torch
     import torch.distributed as dist
 
@@ -63,7 +63,7 @@ def _rank_main(rank, world, port, seed, k, dup, ret):
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        co, KR, QR = _memory(seed, dup=dup)
+        co, KR, QR = _memory(seed, n_docs=n_docs, dup=dup)
         B = QR.shape[0]
         sh = P.shard_memory(co, world, rank)
         qr = O.bf16_to_f64(QR).reshape(B, 4, 64)
@@ -78,14 +78,14 @@ def _rank_main(rank, world, port, seed, k, dup, ret):
         dist.destroy_process_group()
 
 
-def _run(world, seed, k, dup=False):
+def _run(world, seed, k, dup=False, n_docs=60):
     import torch.multiprocessing as mp
 
     ctx = mp.get_context("spawn")
     mgr = ctx.Manager()
     ret = mgr.dict()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, world, port, seed, k, dup, ret)) for r in range(world)]
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, seed, k, dup, ret, n_docs)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
@@ -135,3 +135,19 @@ def test_two_rank_ties_go_to_lower_global_id():
             if 0 in gi[b] and n - 1 in gi[b]:
                 assert list(gi[b]).index(0) < list(gi[b]).index(n - 1)
         assert np.array_equal(gi, idx[:, :4])
+
+
+@pytest.mark.parametrize("k", [5, 8])
+def test_three_ranks_with_shards_smaller_than_k(k):
+    # 8 documents over 3 ranks: every shard holds fewer than k documents, so each rank pads its
+    # candidates (score -inf) before the exchange; k = 8 selects every document
+    ret = _run(3, seed=23, k=k, n_docs=8)
+    co, KR, QR = _memory(23, n_docs=8)
+    B = QR.shape[0]
+    _, idx, val = O.route_topk(O.bf16_to_f64(QR).reshape(B, 4, 64), KR, co, k)
+    spans = sorted(r[2] for r in ret.values())
+    assert all(hi - lo < k for lo, hi, _, _ in spans)
+    for rank in range(3):
+        gi, gs, _ = ret[rank]
+        assert np.array_equal(gi, idx), (rank, gi, idx)
+        assert np.allclose(gs, val, atol=1e-6)
