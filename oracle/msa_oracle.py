@@ -41,7 +41,12 @@ with its reason in the design notes):
     gathered chunk and the local tokens j <= loc_len - M + t (causal).
 
 Every function here is pinned by tests in ``tests/test_oracle.py`` against
-closed forms, invariants, brute force and hand-derived values.
+closed forms, invariants, brute force and hand-derived values, and
+``tests/test_oracle_mutants.py`` checks that a planted mistake in any of them
+fails a pin.  Parity unpinned: three readings above are choices the pages do
+not fix - the rotate-half RoPE convention, the offset k of the global
+positions, and the routing score inside L_aux.  The tests pin the
+implementation of each choice, not the choice itself.
 """
 from __future__ import annotations
 
