@@ -153,6 +153,14 @@ def _workspace(nbytes: int, device, ws=None):
     return torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
 
 
+def _expect(t, name: str, shape, dtype, device) -> None:
+    """Raise ValueError unless t is a contiguous tensor of this shape, dtype and device (the
+    library reads it by its sizes alone)."""
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or t.device != device or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous {dtype} tensor of shape {tuple(shape)} on {device}, got "
+                         f"{t.dtype} {tuple(t.shape)} on {t.device}{'' if t.is_contiguous() else ', not contiguous'}")
+
+
 def _aligned_ptr(ws) -> Optional[int]:
     if ws is None:
         return None
@@ -375,6 +383,9 @@ def sparse_attend(dims, q, K_bar, V_bar, chunk_off, topk_idx, K_loc, V_loc, loc_
     dd = Dims.of(dims)
     B, k = topk_idx.shape
     M = q.shape[1] if q.dim() == 4 else 1
+    for name, t in (("k_new", k_new), ("v_new", v_new)):  # one row per query, written into the cache
+        if t is not None:
+            _expect(t, name, (B, dd.n_kv, dd.head_dim), torch.bfloat16, q.device)
     t_loc_max = K_loc.shape[1] if K_loc is not None else 0
     n_docs = chunk_off.numel() - 1
     dev = q.device

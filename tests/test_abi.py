@@ -265,3 +265,22 @@ def test_binding_constants_match_header(msa):
     for code, name in msa.STATUS.items():
         assert enums[name] == code, name
     assert enums["MSA_AGG_MAX"] == msa.AGG_MAX and enums["MSA_AGG_MEAN"] == msa.AGG_MEAN
+
+
+def test_fused_append_rows_checked_by_the_binding(msa):
+    # k_new / v_new are read by their sizes alone: a wrong shape, dtype or layout is refused
+    # before anything is launched
+    import torch
+
+    d = _dims()
+    B = 2
+    q = torch.zeros(B, d.n_q, d.head_dim, dtype=torch.bfloat16)
+    idx = torch.zeros(B, 3, dtype=torch.int32)
+    good = torch.zeros(B, d.n_kv, d.head_dim, dtype=torch.bfloat16)
+    bad = [torch.zeros(B, d.n_kv, d.head_dim // 2, dtype=torch.bfloat16),
+           torch.zeros(B, d.n_kv, d.head_dim, dtype=torch.float32),
+           torch.zeros(d.n_kv, B, d.head_dim, dtype=torch.bfloat16).transpose(0, 1)]
+    for kn in bad:
+        for kw in (dict(k_new=kn, v_new=good), dict(k_new=good, v_new=kn)):
+            with pytest.raises(ValueError):
+                msa.sparse_attend(d, q, None, None, torch.zeros(4, dtype=torch.int32), idx, None, None, None, 4, **kw)
