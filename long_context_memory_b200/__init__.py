@@ -357,7 +357,13 @@ def kv_append(dims, k_new, v_new, K_loc, V_loc, slots, pos_offset: int, stream=N
     k_new, v_new [B, n_kv, head_dim]; K_loc, V_loc [B, t_loc_max, n_kv, head_dim]; slots [B] int32
     (device): K_loc[b, slots[b]] = RoPE(k_new[b], pos_offset + slots[b]), V_loc[b, slots[b]] = v_new[b].
     """
+    import torch
+
     B, t_loc_max = K_loc.shape[0], K_loc.shape[1]
+    dd = Dims.of(dims)
+    for name, t in (("k_new", k_new), ("v_new", v_new)):
+        _expect(t, name, (B, dd.n_kv, dd.head_dim), torch.bfloat16, K_loc.device)
+    _expect(slots, "slots", (B,), torch.int32, K_loc.device)
     _check(lib.msa_kv_append(ctypes.byref(Dims.of(dims)), _ptr(k_new), _ptr(v_new), _ptr(K_loc), _ptr(V_loc), B,
                              t_loc_max, _ptr(slots), pos_offset, _stream(stream)))
 

@@ -284,3 +284,17 @@ def test_fused_append_rows_checked_by_the_binding(msa):
         for kw in (dict(k_new=kn, v_new=good), dict(k_new=good, v_new=kn)):
             with pytest.raises(ValueError):
                 msa.sparse_attend(d, q, None, None, torch.zeros(4, dtype=torch.int32), idx, None, None, None, 4, **kw)
+
+
+def test_kv_append_rows_and_slots_checked_by_the_binding(msa):
+    import torch
+
+    d = _dims()
+    B, T = 3, 10
+    K = torch.zeros(B, T, d.n_kv, d.head_dim, dtype=torch.bfloat16)
+    rows = torch.zeros(B, d.n_kv, d.head_dim, dtype=torch.bfloat16)
+    slots = torch.zeros(B, dtype=torch.int32)
+    for args in ((rows[:2], rows, slots), (rows, rows.float(), slots), (rows, rows, slots.long()),
+                 (rows, rows, slots[:2])):
+        with pytest.raises(ValueError):
+            msa.kv_append(d, args[0], args[1], K, K, args[2], 4)
