@@ -298,3 +298,34 @@ def test_kv_append_rows_and_slots_checked_by_the_binding(msa):
                  (rows, rows, slots[:2])):
         with pytest.raises(ValueError):
             msa.kv_append(d, args[0], args[1], K, K, args[2], 4)
+
+
+def test_fault_injection_reaches_every_launching_entry_point(msa, monkeypatch):
+    # MSA_FAULT=launch: each entry point validates its arguments, then fails with MSA_ERR_CUDA
+    # before its first launch.  (msa_gather_kv first asks the driver whether its sources are
+    # pinned, which needs a GPU, so it is not in this CPU list.)
+    monkeypatch.setenv("MSA_FAULT", "launch")
+    lib = msa.lib
+    dd = msa.Dims.of(_dims())
+    r = ctypes.byref(dd)
+    enc = lib.msa_encode_workspace_size(r, 1000, 3, 17)
+    aux = lib.msa_aux_loss_workspace_size(r, 4, 8)
+    calls = {
+        "route": lambda: _route(msa, _dims()),
+        "attend": lambda: _attend(msa, _dims()),
+        "encode": lambda: lib.msa_encode_memory(r, FAKE, 1000, FAKE, 3, FAKE, 17, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                                0, 0x100000, enc, None),
+        "append": lambda: lib.msa_append_memory(r, FAKE, 1000, FAKE, 3, FAKE, 17, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                                200, FAKE, 30, 90, 0x100000, enc, None),
+        "aux_loss": lambda: lib.msa_aux_loss(r, FAKE, FAKE, FAKE, 4, 8, 0.1, FAKE, FAKE, None, None, 0x100000, aux,
+                                             None),
+        "kv_append": lambda: lib.msa_kv_append(r, FAKE, FAKE, FAKE, FAKE, 1, 16, FAKE, 2, None),
+        "router_key_norms": lambda: lib.msa_router_key_norms(r, FAKE, 10, 0, FAKE, None),
+        "topk_merge": lambda: lib.msa_topk_merge(FAKE, FAKE, 1, 8, 4, FAKE, FAKE, None),
+        "rope_rows": lambda: lib.msa_rope_rows(r, FAKE, 4, 2, FAKE, None),
+        "rope_cache_build": lambda: lib.msa_rope_cache_build(r, 16, 2, 0x100000, lib.msa_rope_cache_size(r, 16),
+                                                             None),
+    }
+    for name, call in calls.items():
+        assert call() == 4, name
+        assert "injected" in lib.msa_last_error().decode(), name
