@@ -198,6 +198,108 @@ class HostTierCase:
                                out=self.out, ws=self.ws, k_loc_rotated=True)
 
 
+class TieredCase:
+    """A memory of T tokens served from two tiers, over ``layers`` independent layer instances.
+
+    Per layer: pooled router keys K̄^R [C, n_r, d_r] (and their inverse norms) resident in HBM,
+    W^QR, the query's hidden state, q, an 8K-token rotated local KV cache and the new token's key
+    and value per query; content K̄/V̄ [C, n_kv, head_dim] in pinned host memory (``host_layers``
+    distinct host instances, layer l reading instance l % host_layers).  ``run`` makes one
+    msa_tiered_decode call: route every layer, gather its routed documents over the host link on
+    the copy stream, attend over them and the local cache."""
+
+    def __init__(self, T, median, t_loc, seed, device, layers, host_layers, B=1, k=16, dims=W.QWEN3_4B_DIMS):
+        import torch
+
+        import long_context_memory_b200 as msa
+
+        self.msa, self.d, self.k, self.T, self.t_loc = msa, dims, k, T, t_loc
+        self.dev = device
+        doc_off, co, C = chunk_layout_host(T, median, seed)
+        self.C, self.n_docs = C, len(co) - 1
+        self.co_np = co
+        self.max_doc_chunks = int(np.max(co[1:] - co[:-1]))
+        self.chunk_off = torch.from_numpy(co).to(device)
+        g = torch.Generator(device=device)
+        g.manual_seed(seed)
+        self.n_layers = layers
+        self.KR = [randn_bf16((C, dims.n_r, dims.d_r), g, device) for _ in range(layers)]
+        # inverse key norms computed once per memory (offline), as a deployment keeps them
+        self.inv = [msa.router_key_norms(dims, kr) for kr in self.KR]
+        self.W_QR = [(torch.randn((dims.hidden, dims.n_r * dims.d_r), generator=g, device=device) /
+                      math.sqrt(dims.hidden)).to(torch.bfloat16) for _ in range(layers)]
+        shape = (C, dims.n_kv, dims.head_dim)
+        self.K_host, self.V_host = [], []
+        step = 1 << 16  # rows per device-generated slab
+        for _ in range(host_layers):
+            pair = []
+            for _t in range(2):
+                dst = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
+                for a in range(0, C, step):
+                    e = min(C, a + step)
+                    dst[a:e].copy_(randn_bf16((e - a,) + shape[1:], g, device))
+                pair.append(dst)
+            self.K_host.append(pair[0])
+            self.V_host.append(pair[1])
+        torch.cuda.synchronize()
+        self.host_layers = host_layers
+        self.B = 0
+        self.set_batch(B, seed + 100)
+
+    def set_batch(self, B, seed):
+        """A new batch of B queries per layer (query states, local caches, outputs, workspace)."""
+        import torch
+
+        msa, d, dev, L = self.msa, self.d, self.dev, self.n_layers
+        self.B = B
+        self.q_state = None
+        torch.cuda.empty_cache()
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed)
+        self.pos = self.k
+        self.loc_len = torch.full((B,), self.t_loc, dtype=torch.int32, device=dev)
+        self.per_layer = []
+        pos = (self.pos + torch.arange(self.t_loc, dtype=torch.int32, device=dev)).repeat(B)
+        for l in range(L):
+            x = dict(Hq=randn_bf16((B, d.hidden), g, dev), q=randn_bf16((B, d.n_q, d.head_dim), g, dev),
+                     K_loc=randn_bf16((B, self.t_loc, d.n_kv, d.head_dim), g, dev),
+                     V_loc=randn_bf16((B, self.t_loc, d.n_kv, d.head_dim), g, dev),
+                     k_new=randn_bf16((B, d.n_kv, d.head_dim), g, dev),
+                     v_new=randn_bf16((B, d.n_kv, d.head_dim), g, dev),
+                     topk_idx=torch.empty((B, self.k), dtype=torch.int32, device=dev),
+                     topk_score=torch.empty((B, self.k), dtype=torch.float32, device=dev),
+                     out=torch.empty((B, d.n_q, d.head_dim), dtype=torch.bfloat16, device=dev),
+                     W_QR=self.W_QR[l], KR_bar=self.KR[l], kr_inv_norm=self.inv[l],
+                     K_bar_host=self.K_host[l % self.host_layers], V_bar_host=self.V_host[l % self.host_layers])
+            # the local cache holds keys rotated at their global positions (rotated once, when appended)
+            msa.rope_rows(d, x["K_loc"].view(B * self.t_loc, d.n_kv, d.head_dim), pos)
+            self.per_layer.append(x)
+        self.capacity = B * self.k * self.max_doc_chunks  # the largest possible selection
+        self.arr = msa.tiered_layers(self.per_layer)
+        self.ws = torch.empty(msa.tiered_workspace_size(d, B, self.n_docs, self.C, self.k, self.t_loc, self.pos,
+                                                        self.capacity) + 256, dtype=torch.uint8, device=dev)
+        torch.cuda.synchronize()
+
+    def run(self, stream=None, copy_stream=None, arr=None):
+        self.msa.tiered_decode(self.d, self.arr if arr is None else arr, self.B, self.chunk_off, self.C, self.k,
+                               self.loc_len, self.t_loc, self.pos, self.capacity, ws=self.ws, stream=stream,
+                               copy_stream=copy_stream)
+
+    @property
+    def scan_bytes(self):
+        """Algorithmic bytes of one scan: the pooled router keys and their inverse norms."""
+        return self.C * self.d.n_r * (self.d.d_r * 2 + 4)
+
+    def gathered_chunks(self):
+        """Chunks of the documents the last call routed, per layer (host sync)."""
+        co = self.co_np
+        out = []
+        for x in self.per_layer:
+            sel = x["topk_idx"].cpu().numpy()
+            out.append(int(sum(int(co[i + 1] - co[i]) for i in sel.reshape(-1))))
+        return out
+
+
 class AuxCase:
     def __init__(self, P, N, seed, device, dims=W.QWEN3_4B_DIMS, tau=0.05):
         import torch

@@ -1,7 +1,7 @@
 """The bench's reference arm (the oracle on the host cores) prints one JSON line of the contract.
 
-Runs on CPU: `bench.py --impl reference` times the oracle on a bounded sample of the 1M-token
-workload and never touches a GPU."""
+Runs on CPU: `bench.py --impl reference` times the oracle on a bounded sample of the 100M-token
+workload (a process pool over the host cores) and never touches a GPU."""
 import json
 import os
 import subprocess
@@ -27,7 +27,7 @@ def test_reference_arm_prints_one_contract_line():
     sys.path.insert(0, ROOT)
     import bench
 
-    assert d["config"]["workload"] == bench.workload_label(bench.workload_config())
+    assert d["config"]["workload"] == bench.workload_label()
 
 
 def test_traffic_record_follows_the_code_not_the_comments(tmp_path, monkeypatch):

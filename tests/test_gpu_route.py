@@ -63,6 +63,44 @@ def test_route_direct_query_parity(msa, cuda_device, B, n_r, d_r):
         check_topk(idx[b], sc[b], s[b], k, where=f"b={b}")
 
 
+@pytest.mark.parametrize("norms", [False, True])
+def test_route_zero_norm_heads(msa, cuda_device, norms):
+    # zero router-key head rows, a zero query head and an all-zero query: the clamped norms make
+    # every cosine with a zero vector 0 (scan norms, precomputed norms, query normalisation)
+    import torch
+
+    B, k = 3, 16
+    dims, doc_off, KR, QR, Hq, Wqr, rng = _route_case(31 + norms, 200, B, 8, 128)
+    co, C = msa.chunk_offsets(doc_off)
+    KR, QR = KR.copy(), QR.copy().reshape(B, 8, 128)
+    for j in rng.choice(C, 300, replace=False):
+        KR[j, rng.integers(0, 8)] = 0
+    KR[5] = 0          # a chunk with every head zero
+    QR[1, 2] = 0       # one zero head of query 1
+    QR[2] = 0          # query 2 entirely zero: every document scores 0, ties to the lower ids
+    kr = _dev(KR, cuda_device)
+    inv = msa.router_key_norms(dims, kr) if norms else None
+    idx, sc, ds = msa.route_topk(dims, _dev(QR.reshape(B, -1), cuda_device), None, kr,
+                                 torch.from_numpy(co).to(cuda_device), k, want_doc_scores=True, kr_inv_norm=inv)
+    torch.cuda.synchronize()
+    assert msa.check_device_errors() == 0
+    idx, sc, ds = idx.cpu().numpy(), sc.cpu().numpy(), ds.cpu().numpy()
+    co_o, *_ = O.chunk_layout(doc_off)
+    s, _, _ = O.route_topk(O.bf16_to_f64(QR), KR, co_o, k)
+    assert np.all(np.isfinite(ds))
+    assert np.max(np.abs(ds - s)) < SCORE_ATOL, np.max(np.abs(ds - s))
+    for b in range(B):
+        check_topk(idx[b], sc[b], s[b], k, where=f"b={b}")
+    assert np.all(ds[2] == 0.0) and idx[2].tolist() == list(range(k))
+    # the projection path: a zero hidden state gives a zero router query in every head
+    Hz = Hq.copy()
+    Hz[1] = 0
+    idx2, _, ds2 = msa.route_topk(dims, _dev(Hz, cuda_device), _dev(Wqr, cuda_device), kr,
+                                  torch.from_numpy(co).to(cuda_device), k, want_doc_scores=True, kr_inv_norm=inv)
+    torch.cuda.synchronize()
+    assert np.all(ds2.cpu().numpy()[1] == 0.0) and idx2.cpu().numpy()[1].tolist() == list(range(k))
+
+
 @pytest.mark.parametrize("agg", [0, 1])
 def test_route_projection_and_aggregation(msa, cuda_device, agg):
     B = 5
