@@ -82,6 +82,17 @@ int32_t msa_version(void);
  * Synchronises the device.  *bits_out may be NULL. */
 msa_status msa_check_device_errors(uint32_t* bits_out);
 
+/* Self-test of the library's bounded device waits (failure handling; the paper has
+ * no counterpart).  Launches one CTA whose four warps each wait n_waits times, with
+ * a limit of limit_us microseconds per wait, on an mbarrier that nothing ever
+ * arrives on; no copy or tensor-core operation is outstanding.  The first wait
+ * that gives up sets bit 0 of the device error word (msa_check_device_errors then
+ * returns MSA_ERR_TIMEOUT) and the CTA's abort flag; every other wait of the CTA
+ * then returns at once, as in the library's pipelined kernels, so the kernel ends
+ * after about one limit, not n_waits of them.  elapsed_ns: [1] device uint64 out,
+ * the kernel's wall time in ns.  Limits: 1 <= limit_us <= 100000, 1 <= n_waits <= 1000. */
+msa_status msa_selftest_wait_timeout(int32_t limit_us, int32_t n_waits, uint64_t* elapsed_ns, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Stage 1 - chunk layout (host helper).
  * Pages: digest "Method step details", Stage 1 (chunk mean pooling, P = 64);
@@ -225,13 +236,17 @@ msa_status msa_topk_merge(const float* cand_score, const int32_t* cand_idx, int3
  * program that embeds the library as a plugin without a CUDA allocator, code
  * running while a stream is captured into a CUDA graph (cudaMalloc is not
  * allowed there), or a loop that must not pay cudaMalloc's implicit device
- * synchronisation.  Same arguments and results as msa_route_topk, minus
- * ws/ws_bytes.  The scratch is a library-owned device array of 8 MiB
- * (8388608 bytes) that every GPU loading the library holds until the process
- * exits; a problem whose msa_route_workspace_size exceeds it is rejected with
- * MSA_ERR_WORKSPACE before any launch.  The first call on a device (with that
- * device current) looks up the array's address once; make it before any stream
- * capture.  All calls on a device share the array, so calls whose work
+ * synchronisation.  Same arguments and results as msa_route_topk with
+ * kr_layout 0 (chunk-major K̄^R [n_chunks, n_r, d_r]) and kr_inv_norm NULL
+ * (the scan computes the key norms), minus ws/ws_bytes; the arguments are
+ * checked as msa_route_topk checks them and give the same status.  The scratch
+ * is a library-owned device array of 8 MiB (8388608 bytes) that every GPU
+ * loading the library holds until the process exits; a problem whose
+ * msa_route_workspace_size exceeds it is rejected with MSA_ERR_WORKSPACE
+ * before any launch.  The first call on a device (with that device current)
+ * looks up the array's address once, and again after the device's context has
+ * been destroyed and re-created (cudaDeviceReset); make those calls before any
+ * stream capture.  All calls on a device share the array, so calls whose work
  * overlaps on the GPU race: order them on one stream.  No cudaMalloc, cudaFree
  * or allocating library routine is called.
  * ------------------------------------------------------------------------- */
@@ -356,6 +371,70 @@ msa_status msa_gather_kv(const msa_dims* dims, const void* K_bar_host, const voi
                          const int32_t* chunk_off, int32_t n_docs, const int32_t* topk_idx, int32_t B, int32_t k,
                          void* K_stage, void* V_stage, int32_t capacity_chunks, int32_t* stage_chunk_off,
                          int32_t* stage_topk_idx, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Tiered decode: routing, host-tier gather and sparse attention of several
+ * layers in one call, the gather of each layer overlapped with the routing of
+ * the next.
+ * Pages: IRMaD "M. Materials & Methods", Memory Parallel and tiered storage
+ * item (router keys K̄^R resident on the GPU, content K̄/V̄ in host DRAM, loaded
+ * asynchronously once the top-k documents are known) and three-stage inference
+ * item (stages 2 and 3 per layer); EverMind article 2.3.
+ * One msa_layer per layer instance (all pointers as in the single calls):
+ *   Hq, W_QR, KR_bar, kr_inv_norm   as msa_route_topk (chunk-major K̄^R);
+ *   K_bar_host, V_bar_host          [n_chunks, n_kv, head_dim] bf16, pinned host
+ *                                   (as msa_gather_kv);
+ *   q, K_loc, V_loc, k_new, v_new   as msa_sparse_attend with k_loc_rotated = 1
+ *                                   (the local cache holds rotated keys; k_new /
+ *                                   v_new both NULL or both set: the fused append);
+ *   topk_idx, topk_score, out       outputs: [B, k] int32, [B, k] fp32 and
+ *                                   [B, n_q, head_dim] bf16.
+ * `layers` is a host array of n_layers entries.  The layers are independent
+ * instances: no layer reads what another layer of the call writes (its inputs
+ * must not alias another layer's outputs or local cache).  They share the
+ * document layout (chunk_off, n_docs, n_chunks), B, k, loc_len, t_loc_max and
+ * pos_offset.  Per layer l the call enqueues, on
+ * `stream`, msa_route_topk (agg MAX); on `copy_stream`, after an event on the
+ * routing, msa_gather_kv of the routed documents into one of two staging areas
+ * in ws; on `stream`, after the routing of layer l + 1 and an event on that
+ * gather, msa_sparse_attend over the staged documents and the local keys.  The
+ * results equal those calls made one after the other, bit for bit.  The
+ * copy-stream work is joined back into `stream` before the call's last
+ * attention, so work enqueued later on `stream` sees every output.
+ * copy_stream may be NULL or equal to stream (no overlap; same results).
+ *   capacity_chunks  staging rows per layer (>= the chunks of the B * k routed
+ *                    documents; a selection needing more stages what fits and
+ *                    raises device error bit 1, as msa_gather_kv).
+ *   ws        >= msa_tiered_workspace_size(...) bytes, 256-byte aligned; holds the
+ *             routing and attention workspaces and the two staging areas.
+ * The call keeps three CUDA events per host thread and device (created by its
+ * first call on that device from that thread: make that call before any stream
+ * capture).  Limits: those of msa_route_topk, msa_gather_kv and
+ * msa_sparse_attend with q_tokens = 1; 1 <= n_layers <= 4096.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  const void* Hq;
+  const void* W_QR;
+  const void* KR_bar;
+  const float* kr_inv_norm;
+  const void* K_bar_host;
+  const void* V_bar_host;
+  const void* q;
+  void* K_loc;
+  void* V_loc;
+  const void* k_new;
+  const void* v_new;
+  int32_t* topk_idx;
+  float* topk_score;
+  void* out;
+} msa_layer;
+
+size_t msa_tiered_workspace_size(const msa_dims* dims, int32_t B, int32_t n_docs, int32_t n_chunks, int32_t k,
+                                 int32_t t_loc_max, int32_t pos_offset, int32_t capacity_chunks);
+msa_status msa_tiered_decode(const msa_dims* dims, const msa_layer* layers, int32_t n_layers, int32_t B,
+                             const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks, int32_t k,
+                             const int32_t* loc_len, int32_t t_loc_max, int32_t pos_offset, int32_t capacity_chunks,
+                             void* ws, size_t ws_bytes, void* stream, void* copy_stream);
 
 /* ---------------------------------------------------------------------------
  * In-place RoPE of key rows (global positions of the active context).

@@ -8,7 +8,7 @@ call raises ImportError when the library is missing; there is no CPU fallback.
 
 Entry points (same names as the C ABI, minus the ``msa_`` prefix):
   chunk_offsets, encode_memory, append_memory, route_topk, sparse_attend, kv_append, aux_loss,
-  *_workspace_size, check_device_errors, trace_*.
+  gather_kv, tiered_decode, *_workspace_size, check_device_errors, trace_*.
 """
 from __future__ import annotations
 
@@ -18,8 +18,8 @@ from typing import Optional
 
 __all__ = [
     "Dims", "MSAError", "lib", "chunk_offsets", "encode_memory", "append_memory", "route_topk", "sparse_attend",
-    "aux_loss", "kv_append", "router_key_norms",
-    "route_workspace_size", "attend_workspace_size", "rope_cache_build", "topk_merge", "rope_rows", "gather_kv", "encode_workspace_size", "check_device_errors",
+    "aux_loss", "kv_append", "router_key_norms", "Layer", "tiered_layers", "tiered_workspace_size", "tiered_decode",
+    "route_workspace_size", "attend_workspace_size", "rope_cache_build", "topk_merge", "rope_rows", "gather_kv", "encode_workspace_size", "check_device_errors", "selftest_wait_timeout",
     "trace_enable", "trace_reset", "trace_read", "trace_kernel_names", "AGG_MAX", "AGG_MEAN", "ATTEND_EARLY_LOCAL", "ROUTE_EARLY_INPUTS",
 ]
 
@@ -60,6 +60,14 @@ class Dims(ctypes.Structure):
 
 _DIMS_CACHE: dict = {}  # the ctypes struct of each dims tuple (read-only after construction)
 
+_LAYER_FIELDS = ("Hq", "W_QR", "KR_bar", "kr_inv_norm", "K_bar_host", "V_bar_host", "q", "K_loc", "V_loc", "k_new",
+                 "v_new", "topk_idx", "topk_score", "out")
+
+
+class Layer(ctypes.Structure):
+    """msa_layer: the pointers of one layer instance of msa_tiered_decode (NULL for an absent optional)."""
+    _fields_ = [(n, ctypes.c_void_p) for n in _LAYER_FIELDS]
+
 
 def _load():
     if not os.path.exists(LIB_PATH):
@@ -73,6 +81,7 @@ def _load():
         "msa_last_error": (ctypes.c_char_p, []),
         "msa_version": (I32, []),
         "msa_check_device_errors": (I32, [ctypes.POINTER(ctypes.c_uint32)]),
+        "msa_selftest_wait_timeout": (I32, [I32, I32, P, P]),
         "msa_chunk_offsets": (I32, [P, I32, I32, P, ctypes.POINTER(I32)]),
         "msa_encode_workspace_size": (SZ, [DP, I64, I32, I32]),
         "msa_encode_memory": (I32, [DP, P, I64, P, I32, P, I32, P, P, P, P, P, P, I32, P, SZ, P]),
@@ -88,6 +97,9 @@ def _load():
         "msa_rope_rows": (I32, [DP, P, I32, I32, P, P]),
         "msa_kv_append": (I32, [DP, P, P, P, P, I32, I32, P, I32, P]),
         "msa_gather_kv": (I32, [DP, P, P, I32, P, I32, P, I32, I32, P, P, I32, P, P, P, SZ, P]),
+        "msa_tiered_workspace_size": (SZ, [DP, I32, I32, I32, I32, I32, I32, I32]),
+        "msa_tiered_decode": (I32, [DP, ctypes.POINTER(Layer), I32, I32, P, I32, I32, I32, P, I32, I32, I32, P, SZ, P,
+                                    P]),
         "msa_rope_cache_size": (SZ, [DP, I32]),
         "msa_rope_cache_build": (I32, [DP, I32, I32, P, SZ, P]),
         "msa_topk_merge": (I32, [P, P, I32, I32, I32, P, P, P]),
@@ -344,6 +356,47 @@ def gather_kv(dims, K_bar_host, V_bar_host, chunk_off, topk_idx, capacity_chunks
     return out
 
 
+def tiered_layers(layers):
+    """A ctypes array of msa_layer from a list of dicts {field: tensor or None} (fields of ``Layer``).
+
+    Build it once per set of buffers and pass it to every ``tiered_decode`` call: the call then
+    marshals nothing per layer."""
+    arr = (Layer * len(layers))()
+    for i, L in enumerate(layers):
+        for f in _LAYER_FIELDS:
+            t = L.get(f)
+            setattr(arr[i], f, None if t is None else t.data_ptr())
+    return arr
+
+
+def tiered_workspace_size(dims, B: int, n_docs: int, n_chunks: int, k: int, t_loc_max: int, pos_offset: int,
+                          capacity_chunks: int) -> int:
+    return int(lib.msa_tiered_workspace_size(ctypes.byref(Dims.of(dims)), B, n_docs, n_chunks, k, t_loc_max,
+                                             pos_offset, capacity_chunks))
+
+
+def tiered_decode(dims, layers, B: int, chunk_off, n_chunks: int, k: int, loc_len, t_loc_max: int, pos_offset: int,
+                  capacity_chunks: int, ws=None, stream=None, copy_stream=None):
+    """Route, gather (host tier) and attend for several independent layer instances in one call.
+
+    ``layers``: the array from ``tiered_layers`` (or a list of dicts, converted here).  Per layer the
+    routing runs on ``stream`` (default: the current stream), the gather of the routed documents
+    from pinned host memory on ``copy_stream`` (None: on ``stream``, no overlap), and the attention
+    over the staged documents and the rotated local cache on ``stream``; outputs land in each
+    layer's topk_idx, topk_score and out tensors."""
+    arr = layers if isinstance(layers, ctypes.Array) else tiered_layers(layers)
+    n_docs = chunk_off.numel() - 1
+    dd = Dims.of(dims)
+    if ws is not None:  # the library checks the caller's buffer against what it needs
+        nbytes = max(0, ws.numel() * ws.element_size() - 256)
+    else:
+        nbytes = tiered_workspace_size(dims, B, n_docs, n_chunks, k, t_loc_max, pos_offset, capacity_chunks)
+        ws = _workspace(nbytes, chunk_off.device, ws)
+    _check(lib.msa_tiered_decode(ctypes.byref(dd), arr, len(arr), B, _ptr(chunk_off), n_docs, n_chunks, k, _ptr(loc_len),
+                                 t_loc_max, pos_offset, capacity_chunks, _aligned_ptr(ws), nbytes, _stream(stream),
+                                 None if copy_stream is None else _stream(copy_stream)))
+
+
 def rope_rows(dims, x, positions, stream=None):
     """Rotate x [rows, heads, head_dim] (bf16, in place) at positions [rows] (int32, device)."""
     rows, heads = x.shape[0], x.shape[1]
@@ -446,6 +499,16 @@ def check_device_errors() -> int:
     bits = ctypes.c_uint32(0)
     _check(lib.msa_check_device_errors(ctypes.byref(bits)))
     return int(bits.value)
+
+
+def selftest_wait_timeout(limit_us: int, n_waits: int, stream=None):
+    """Run the bounded-wait self-test kernel (see msa.h); returns the device uint64 [1] that receives
+    its wall time in ns.  Afterwards check_device_errors() raises MSAError with MSA_ERR_TIMEOUT."""
+    import torch
+
+    out = torch.zeros(2, dtype=torch.int64, device=torch.cuda.current_device())
+    _check(lib.msa_selftest_wait_timeout(int(limit_us), int(n_waits), _ptr(out), _stream(stream)))
+    return out[:1]
 
 
 def trace_enable(on: bool = True):

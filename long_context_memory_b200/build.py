@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["msa_api.cu", "route.cu", "route_static.cu", "attend.cu", "encode.cu", "aux_loss.cu"]
+SOURCES = ["msa_api.cu", "route.cu", "route_static.cu", "attend.cu", "encode.cu", "aux_loss.cu", "tiered.cu"]
 LIB = os.path.join(HERE, "libmsa.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 

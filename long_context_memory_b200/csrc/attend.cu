@@ -142,6 +142,7 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
   int* segs = hdr + 16;                                              // [2][2 kMaxK + 2] segment tables
   float2* qcs = reinterpret_cast<float2*>(segs + 2 * (2 * kMaxK + 2));  // [MT][D/2] cos/sin at the tokens' positions
   int* co_sm = reinterpret_cast<int*>(qcs + (size_t)MT * (D / 2));   // [co_cap] chunk_off
+  __shared__ int abort_flag;                                         // a bounded wait of this CTA gave up
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = warp;               // the KV head this warp serves (warps 0 .. n_kv-1)
@@ -167,6 +168,7 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
       mbar_init(&hempty[s], n_kv);
       mbar_init(&hsel[s], 1);
     }
+    abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -193,7 +195,9 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
     // ---- per item: the header and the query rows for the compute warps, then the segment table
     //      (selected docs in top-k order) and the key range, then the item's tiles ----
     int gt = 0;
-    for (int it = blockIdx.x, j = 0; it < n_items; it += gridDim.x, ++j) {
+    int n_hdr = 0;      // items whose query rows were requested
+    bool stop = false;  // a wait gave up
+    for (int it = blockIdx.x, j = 0; it < n_items && !stop; it += gridDim.x, ++j) {
       const int hb = j & 1;
       const bool is_chunk = it >= n_loc_items;
       const int i2 = is_chunk ? it - n_loc_items : it;
@@ -203,7 +207,7 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
       const int split = is_chunk ? i2 % ns : ns - 1 - i2 % ns, bq = i2 / ns;
       const int b = bq / p.n_tgroups, t0 = (bq % p.n_tgroups) * MT;
       const int nt = min(MT, p.q_tokens - t0);
-      if (j >= 2) mbar_wait(&hempty[hb], ((j >> 1) - 1) & 1);  // item j-2's header and query read
+      if (j >= 2 && !warp_wait(&hempty[hb], ((j >> 1) - 1) & 1, &abort_flag)) break;  // item j-2's header, query read
       int L = p.loc_len[b];
       L = max(0, min(L, p.t_loc_max));
       int* hd = hdr + hb * 8;
@@ -213,6 +217,7 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
         mbar_arrive_expect_tx(&hfull[hb], qbytes);  // releases the header writes above
         bulk_load(qsm + hb * q_elems, p.q + ((size_t)b * p.q_tokens + t0) * p.n_q * D, qbytes, &hfull[hb]);
       }
+      n_hdr = j + 1;
       if (is_chunk && !waited) {
         pdl_enter();
         waited = true;
@@ -302,7 +307,10 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
       // ---- the item's tiles: kTK keys each, a bulk copy per key and tensor plus the RoPE rows ----
       for (int t = 0; t < n_tiles; ++t, ++gt) {
         const int st = gt % L_.n_stages;
-        if (gt >= L_.n_stages) mbar_wait(&ebars[st], ((gt / L_.n_stages) - 1) & 1);
+        if (gt >= L_.n_stages && !warp_wait(&ebars[st], ((gt / L_.n_stages) - 1) & 1, &abort_flag)) {
+          stop = true;
+          break;
+        }
         const int tv0 = v0 + t * kTK;
         const int rows = min(kTK, v1 - tv0);
         const int n_chunk_rows = max(0, min(rows, n_sel - tv0));
@@ -338,6 +346,11 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
         }
       }
     }
+    if (abort_flag && lane == 0) {  // the copies still in flight land before the CTA exits
+      mbar_drain_ring(bars, L_.n_stages, gt - L_.n_stages, gt);
+      mbar_drain_ring(hfull, 2, n_hdr - 2, n_hdr);
+    }
+    __syncwarp();
     if (!waited) pdl_enter();  // the grid completes only after its predecessor
     return;  // the compute warps no longer synchronise with the whole block
   }
@@ -345,15 +358,17 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
   // ---- compute warps, item by item ----
   const int n_compute = 32 * n_kv;
   int gt = 0;
+  bool failed = false;  // a wait of this warp gave up: the compute warps leave together at the next item
   for (int it = blockIdx.x, j = 0; it < n_items; it += gridDim.x, ++j) {
     const int hb = j & 1;
-    mbar_wait(&hfull[hb], (j >> 1) & 1);
+    failed |= !warp_wait(&hfull[hb], (j >> 1) & 1, &abort_flag);
+    // every warp has built its previous fragments (qcs is reused), and none has given up a wait
+    if (named_bar_any(1, n_compute, failed)) break;
     const int* hd = hdr + hb * 8;
     const int b = hd[0], t0 = hd[1], nt = hd[2], L = hd[3];
     const uint16_t* qsm_b = qsm + hb * q_elems;
     // ---- query fragments of this warp's GQA group: mma row = tt * G + gg (token t0 + tt,
     //      q head h * G + gg); token t sits at pos_offset + L - M + t; scale, bf16 ----
-    named_bar_sync(1, n_compute);  // every warp has built its previous fragments (qcs is reused)
     const int64_t pos_q0 = (int64_t)p.pos_offset + L - p.q_tokens + t0;
     for (int i = tid; i < nt * (D / 2); i += n_compute)
       qcs[i] = rope_cos_sin(p.turns, i % (D / 2), pos_q0 + i / (D / 2));
@@ -398,7 +413,10 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
       pdl_enter();
       waited = true;
     }
-    mbar_wait(&hsel[hb], (j >> 1) & 1);
+    if (!warp_wait(&hsel[hb], (j >> 1) & 1, &abort_flag)) {
+      failed = true;
+      continue;
+    }
     const int n_sel = hd[4], v0 = hd[5], v1 = hd[6], part = hd[7];
     const int n_tiles = (v1 - v0 + kTK - 1) / kTK;
     __syncwarp();
@@ -421,7 +439,10 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
     for (int t = 0; t < n_tiles; ++t) {
       const int gtt = gt + t;  // tile counter over this CTA's items: the ring position
       const int st = gtt % L_.n_stages;
-      mbar_wait(&bars[st], (gtt / L_.n_stages) & 1);
+      if (!warp_wait(&bars[st], (gtt / L_.n_stages) & 1, &abort_flag)) {
+        failed = true;
+        break;
+      }
 
       const int tv0 = v0 + t * kTK;
       const uint8_t* kst = stage_mem + (size_t)st * L_.stage_bytes;
@@ -530,6 +551,7 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
     }
 
 
+    if (failed) continue;  // the item is abandoned; the warps leave at the next item
     gt += n_tiles;
 
     // ---- this warp's split partial: unnormalised output, running max and sum per q head ----
@@ -834,47 +856,58 @@ __global__ void __launch_bounds__(1024) gather_plan_kernel(const int32_t* __rest
   if (threadIdx.x == 0) stage_off[0] = 0;
 }
 
-// copy the planned chunk rows (row = n_kv*D bf16 of K and of V) from host to the staging
-__global__ void __launch_bounds__(256) gather_copy_kernel(const uint4* __restrict__ K_host,
-                                                          const uint4* __restrict__ V_host,
-                                                          const int32_t* __restrict__ stage_off,
-                                                          const int32_t* __restrict__ stage_src, int n_sel,
-                                                          int row_vec, uint4* __restrict__ K_stage,
-                                                          uint4* __restrict__ V_stage) {
+// copy the planned chunk rows (row = n_kv*D bf16 of K and of V) from host to the staging.
+// One warp per row at a time: its lanes hold up to 4 sixteen-byte pieces of the K row and 4 of
+// the V row in flight (a 4 KB row pair per warp, 512 KB over the whole grid: about three times
+// what a ~55 GB/s host link needs in flight at a few microseconds of latency).  The grid is small
+// (kGatherCtas CTAs of 256 threads, at most 64 registers a thread): it runs beside the routing
+// scan or the attention of another layer without taking an SM from them.
+constexpr int kGatherThreads = 256;
+#ifndef MSA_GATHER_CTAS
+#define MSA_GATHER_CTAS 16
+#endif
+constexpr int kGatherCtas = MSA_GATHER_CTAS;
+__global__ void __launch_bounds__(kGatherThreads, 4) gather_copy_kernel(const uint4* __restrict__ K_host,
+                                                                        const uint4* __restrict__ V_host,
+                                                                        const int32_t* __restrict__ stage_off,
+                                                                        const int32_t* __restrict__ stage_src,
+                                                                        int n_sel, int row_vec,
+                                                                        uint4* __restrict__ K_stage,
+                                                                        uint4* __restrict__ V_stage) {
   pdl_enter();
   const int total_rows = stage_off[n_sel];
-  const int64_t n = (int64_t)total_rows * row_vec;  // 16-byte vectors
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += 4 * stride) {
-    uint4 kv[4], vv[4];
-    int64_t dst[4], src[4];
+  const int lane = threadIdx.x & 31;
+  const int warp = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int n_warps = (int)((gridDim.x * blockDim.x) >> 5);
+  int doc = 0;  // a warp's rows only grow, so its document search starts where the last one ended
+  for (int row = warp; row < total_rows; row += n_warps) {
+    int lo = doc, hi = n_sel - 1;  // the last staged document starting at or before this row
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (stage_off[mid] <= row) lo = mid; else hi = mid - 1;
+    }
+    doc = lo;
+    const int64_t src = (int64_t)(stage_src[doc] + (row - stage_off[doc])) * row_vec;
+    const int64_t dst = (int64_t)row * row_vec;
+    for (int v0 = 0; v0 < row_vec; v0 += 128) {
+      uint4 kv[4], vv[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int64_t ee = e + u * stride;
-      dst[u] = -1;
-      if (ee < n) {
-        const int row = (int)(ee / row_vec), col = (int)(ee % row_vec);
-        int lo = 0, hi = n_sel - 1;  // staged document holding this row
-        while (lo < hi) {
-          const int mid = (lo + hi + 1) >> 1;
-          if (stage_off[mid] <= row) lo = mid; else hi = mid - 1;
+      for (int u = 0; u < 4; ++u) {
+        const int v = v0 + lane + 32 * u;
+        if (v < row_vec) {
+          kv[u] = K_host[src + v];
+          vv[u] = V_host[src + v];
         }
-        dst[u] = ee;
-        src[u] = (int64_t)(stage_src[lo] + (row - stage_off[lo])) * row_vec + col;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int v = v0 + lane + 32 * u;
+        if (v < row_vec) {
+          K_stage[dst + v] = kv[u];
+          V_stage[dst + v] = vv[u];
+        }
       }
     }
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (dst[u] >= 0) {
-        kv[u] = K_host[src[u]];
-        vv[u] = V_host[src[u]];
-      }
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (dst[u] >= 0) {
-        K_stage[dst[u]] = kv[u];
-        V_stage[dst[u]] = vv[u];
-      }
   }
 }
 
@@ -922,7 +955,7 @@ msa_status gather_kv_launch(const msa_dims& d, const void* K_host, const void* V
   {
     TraceScope ts(kKGatherCopy, s);
     const int row_vec = d.n_kv * d.head_dim * 2 / 16;
-    MSA_CUDA_CHECK(launch_pdl(gather_copy_kernel, dim3(4 * sm_count()), dim3(256), 0, s,
+    MSA_CUDA_CHECK(launch_pdl(gather_copy_kernel, dim3(kGatherCtas), dim3(kGatherThreads), 0, s,
                               static_cast<const uint4*>(K_host), static_cast<const uint4*>(V_host),
                               (const int32_t*)stage_off, (const int32_t*)stage_src, n_sel, row_vec,
                               static_cast<uint4*>(K_stage), static_cast<uint4*>(V_stage)));

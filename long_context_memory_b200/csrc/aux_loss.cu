@@ -82,6 +82,8 @@ __device__ __forceinline__ int unit_of_slot(int e, int lane) {
 
 
 __device__ __forceinline__ void aux_bar_sync() { named_bar_sync(1, 32 * kAuxCompute); }
+// the same barrier, returning whether any compute thread passed `failed` (then all leave together)
+__device__ __forceinline__ bool aux_bar_any(bool failed) { return named_bar_any(1, 32 * kAuxCompute, failed); }
 
 template <int DR>
 __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParams p) {
@@ -105,6 +107,7 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
   __shared__ float chead[8];   // sum_j g_j cos_jh
   __shared__ float wred[kAuxCompute];
   __shared__ bool last;
+  __shared__ int abort_flag;   // a bounded wait of this CTA gave up
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool grads = p.dQ != nullptr || p.dK_pos != nullptr || p.dK_neg != nullptr;
@@ -120,6 +123,7 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
       mbar_init(&qfull[s], 1);
       mbar_init(&qempty[s], kAuxCompute);
     }
+    abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -129,17 +133,21 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
     // ------------------------- producer -------------------------
     if (lane == 0) {
       int it = 0, pi = 0;
-      for (int i = blockIdx.x; i < p.P; i += gridDim.x, ++pi) {
+      bool stop = false;
+      for (int i = blockIdx.x; i < p.P && !stop; i += gridDim.x, ++pi) {
         {  // the positive's query row (double-buffered)
           const int qb = pi & 1;
-          if (pi >= 2) mbar_wait(&qempty[qb], ((pi >> 1) - 1) & 1);
+          if (pi >= 2 && !mbar_wait(&qempty[qb], ((pi >> 1) - 1) & 1, &abort_flag)) break;
           mbar_arrive_expect_tx(&qfull[qb], (uint32_t)row_bytes);
           bulk_load(qbuf + qb * Sm::kQBytes, p.Q + (size_t)i * NR, (uint32_t)row_bytes, &qfull[qb]);
         }
-        for (int pass = 0; pass < passes; ++pass) {
+        for (int pass = 0; pass < passes && !stop; ++pass) {
           for (int c = 0; c < n_ch; ++c, ++it) {
             const int st = it % kAuxStages;
-            if (it >= kAuxStages) mbar_wait(&empty[st], ((it / kAuxStages) - 1) & 1);
+            if (it >= kAuxStages && !mbar_wait(&empty[st], ((it / kAuxStages) - 1) & 1, &abort_flag)) {
+              stop = true;
+              break;
+            }
             const int j0 = c * kAuxRows, j1 = min(NK, j0 + kAuxRows);
             uint8_t* dst = ring + (size_t)st * Sm::kStageBytes;
             mbar_arrive_expect_tx(&full[st], (uint32_t)((j1 - j0) * row_bytes));
@@ -154,6 +162,11 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
           }
         }
       }
+      if (abort_flag) {  // the copies still in flight land before the CTA exits
+        const int q_issued = stop ? pi + 1 : pi;
+        mbar_drain_ring(full, kAuxStages, it - kAuxStages, it);
+        mbar_drain_ring(qfull, 2, q_issued - 2, q_issued);
+      }
     }
     return;
   }
@@ -164,13 +177,14 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
   const float inv_nr = 1.0f / (float)n_r;
   const float inv_p = 1.0f / (float)p.P;
   int it = 0, pi = 0;
+  bool failed = false;   // a wait of this warp gave up: the compute warps leave together at their next barrier
   for (int i = blockIdx.x; i < p.P; i += gridDim.x, ++pi) {
     // this lane's query values (in slot order, see unit_of_slot) and the head norms
     const int qb = pi & 1;
     const uint16_t* qrow = reinterpret_cast<const uint16_t*>(qbuf + qb * Sm::kQBytes);
     float q[V];
     {
-      mbar_wait(&qfull[qb], (pi >> 1) & 1);
+      failed |= !warp_wait(&qfull[qb], (pi >> 1) & 1, &abort_flag);
 #pragma unroll
       for (int e = 0; e < DR / 32; ++e) {
         uint4 w = make_uint4(0, 0, 0, 0);
@@ -188,7 +202,10 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
       for (int e = 0; e < V; ++e) ss = fmaf(q[e], q[e], ss);
       ss += __shfl_xor_sync(0xffffffffu, ss, 1);
       ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-      aux_bar_sync();  // the previous positive's readers of qn, cos, g and the dq partials are done
+      // the previous positive's readers of qn, cos, g and the dq partials are done; the compute
+      // warps leave together here once any of their waits has given up (until then every wait
+      // of an aborted CTA returns at once and the warps keep to the same barriers)
+      if (aux_bar_any(failed)) break;
       if (warp == 0 && hl && (lane & 3) == 0) {
         const float n = sqrtf(ss);
         qn[h] = n > kAuxEps ? n : -kAuxEps;  // sign marks a clamped norm
@@ -199,7 +216,7 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
     // ---- pass 1: cosines ----
     for (int c = 0; c < n_ch; ++c, ++it) {
       const int st = it % kAuxStages;
-      mbar_wait(&full[st], (it / kAuxStages) & 1);
+      failed |= !warp_wait(&full[st], (it / kAuxStages) & 1, &abort_flag);  // on failure: left at the next barrier
       const int j = c * kAuxRows + warp;
       uint4 kw[DR / 32];
       if (j < NK && hl) {
@@ -298,7 +315,7 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
     float* slice = red + (size_t)warp * Sm::kSlice;
     for (int c = 0; c < n_ch; ++c, ++it) {
       const int st = it % kAuxStages;
-      mbar_wait(&full[st], (it / kAuxStages) & 1);
+      failed |= !warp_wait(&full[st], (it / kAuxStages) & 1, &abort_flag);  // on failure: left at the next barrier
       const int j = c * kAuxRows + warp;
       uint4 kw[DR / 32];
       if (j < NK && hl) {
@@ -370,7 +387,7 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
 
   // ---- loss: the last CTA sums the terms in positive order ----
   __threadfence();
-  aux_bar_sync();
+  if (aux_bar_any(abort_flag != 0)) return;  // a CTA that gave up leaves the loss unsummed (error word set)
   if (tid == 0) {
     const uint32_t prev = atomicAdd(p.ticket, 1u);
     last = prev == gridDim.x - 1;

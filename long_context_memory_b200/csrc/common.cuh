@@ -109,18 +109,62 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait on phase `parity`.  Returns false (and raises the device error
-// word) if the phase did not complete within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Bounded wait on phase `parity`, with a CTA-wide abort flag in shared memory.
+// Returns false if the phase did not complete within limit_ns: the first wait of
+// the CTA that gives up raises the device error word and sets *abort; every later
+// wait of the CTA that does not find its phase complete at once returns false as
+// soon as it sees the flag, so a stalled pipeline ends after one limit, not one per
+// remaining wait.  A caller that gets false leaves its loop; the thread that issued
+// copies then drains them (mbar_drain_ring) before the CTA frees its TMEM and exits.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *abort = 1;
+      __threadfence_block();
       raise_dev_error(kDevErrWaitTimeout);
       return false;
     }
   }
+}
+
+// mbar_wait made by every lane of a warp, with one answer for the whole warp (a lane whose wait
+// completes just after another lane gave up still leaves with it).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+}
+
+// Named barrier among `nthreads` threads that also returns whether any of them passed `pred`
+// (bar.red.or): a group of warps that must stay in step (their named barriers have no time
+// limit) decides together whether to leave its loop.
+__device__ __forceinline__ bool named_bar_any(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
+// After an abort, the thread that filled a ring of S stages waits, within limit_ns in all, for
+// the copies it issued for iterations first .. last-1 (stage j % S, phase parity (j / S) & 1) to
+// land, so that no copy writes shared memory after the CTA has exited.  Only the last phase of
+// each stage can be outstanding (a stage is refilled only after its previous phase completed).
+// Returns false if some did not land in time.
+__device__ __forceinline__ bool mbar_drain_ring(uint64_t* full, int S, int first, int last,
+                                                uint64_t limit_ns = kWaitLimitNs) {
+  const uint64_t t0 = globaltimer_ns();
+  for (int j = first < 0 ? 0 : first; j < last; ++j) {
+    while (!mbar_try_wait(&full[j % S], (uint32_t)(j / S) & 1u)) {
+      if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+  }
+  return true;
 }
 
 // ---------------------------------------------------------------------------

@@ -9,12 +9,14 @@
 // Kernels:
 //   chunk_map_kernel   first token, length and document-relative position of every chunk
 //   transpose_kernel   W [hidden, N] -> W^T [N, hidden] (K-major B operand)
-//   pool_h_kernel      H̄ = chunk mean of H, stored as bf16 hi + lo terms [C, 2*hidden]
 //   gemm_kernel<K>     per-token K projection on tcgen05 tensor cores: M = two
 //                      chunks (2 x 64 token rows, each chunk loaded by its own TMA
 //                      box), N = 256 (or 128), accumulators in TMEM; the epilogue rotates
 //                      each row at its document-relative position and pools the
-//                      64 rows of each chunk -> K̄
+//                      64 rows of each chunk -> K̄.  A pool warp sums the same H
+//                      tiles in shared memory (for one N tile of each chunk pair):
+//                      H̄ = chunk mean of H, stored as bf16 hi + lo terms [C, 2*hidden],
+//                      so H is read from HBM once
 //   gemm_kernel<POOL>  (H̄_hi | H̄_lo) [W_V | W^KR] over K = 2*hidden -> V̄, K̄^R.
 //                      Pooling before the projection is exact by linearity;
 //                      splitting H̄ into two bf16 terms keeps ~16 mantissa bits.
@@ -46,6 +48,7 @@ constexpr int kBM = 128, kBK = 64;
 constexpr int kEncStagesMax = 4;
 constexpr int kABytes = kBM * kBK * 2;  // 16 KB
 constexpr int kEncThreads = 192;        // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kEncThreadsK = 224;       // mode K: + warp 6, the pool warp (chunk means of H)
 
 __global__ void chunk_map_kernel(const int64_t* __restrict__ doc_off, const int32_t* __restrict__ chunk_off,
                                  int n_docs, int n_chunks, int64_t T, int64_t* __restrict__ tok0,
@@ -87,41 +90,6 @@ __global__ void transpose_kernel(const uint16_t* __restrict__ in, int K, int N, 
   }
 }
 
-// H̄[c] = mean of the chunk's token rows; one block per chunk, 8 columns per thread per pass
-__global__ void __launch_bounds__(256) pool_h_kernel(const __nv_bfloat16* __restrict__ H, int hidden,
-                                                     const int64_t* __restrict__ tok0,
-                                                     const int32_t* __restrict__ clen,
-                                                     __nv_bfloat16* __restrict__ hbar) {
-  const int c = blockIdx.x;
-  const int64_t t0 = tok0[c];
-  const int n = clen[c];
-  const float inv = 1.0f / (float)n;
-  for (int col = threadIdx.x * 8; col < hidden; col += blockDim.x * 8) {
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    const __nv_bfloat16* src = H + (size_t)t0 * hidden + col;
-    for (int r = 0; r < n; ++r) {
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(src + (size_t)r * hidden));
-      float2 f;
-      f = unpack_bf16x2(w.x); acc[0] += f.x; acc[1] += f.y;
-      f = unpack_bf16x2(w.y); acc[2] += f.x; acc[3] += f.y;
-      f = unpack_bf16x2(w.z); acc[4] += f.x; acc[5] += f.y;
-      f = unpack_bf16x2(w.w); acc[6] += f.x; acc[7] += f.y;
-    }
-    uint32_t hi[4], lo[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float m0 = acc[2 * j] * inv, m1 = acc[2 * j + 1] * inv;
-      const float h0 = __bfloat162float(__float2bfloat16_rn(m0));
-      const float h1 = __bfloat162float(__float2bfloat16_rn(m1));
-      hi[j] = pack_bf16x2(h0, h1);
-      lo[j] = pack_bf16x2(m0 - h0, m1 - h1);
-    }
-    __nv_bfloat16* dst = hbar + (size_t)c * 2 * hidden + col;
-    *reinterpret_cast<uint4*>(dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-    *reinterpret_cast<uint4*>(dst + hidden) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-  }
-}
-
 // Sum of v[0..31] over the 32 lanes of a warp, transposed: on return v[0] of
 // lane l holds the warp-wide sum of column l (31 shuffles for 32 columns).
 __device__ __forceinline__ void warp_transpose_reduce32(float (&v)[32], int lane) {
@@ -150,6 +118,7 @@ struct GemmParams {
   const int64_t* tok0;
   const int32_t* clen;
   const int32_t* pos0;
+  __nv_bfloat16* hbar;   // mode K: chunk means of H, [C][2*hidden] bf16 hi | lo (written by the pool warp)
   __nv_bfloat16* out0;   // K̄ (mode K) or V̄ (pooled)
   __nv_bfloat16* out1;   // K̄^R (pooled)
   int n_out0;            // columns of out0 (n_kv*D); pooled: columns >= n_out0 go to out1
@@ -159,7 +128,7 @@ struct GemmParams {
 };
 
 template <int MODE, int kBN>
-__global__ void __launch_bounds__(kEncThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap map_a,
+__global__ void __launch_bounds__(MODE == 0 ? kEncThreadsK : kEncThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                                                               const __grid_constant__ CUtensorMap map_b,
                                                               const GemmParams p) {
   constexpr int kBBytes = kBN * kBK * 2;
@@ -179,7 +148,9 @@ __global__ void __launch_bounds__(kEncThreads, 1) gemm_kernel(const __grid_const
   uint64_t* empty = full + kEncStages;
   uint64_t* tfull = empty + kEncStages;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* drained = tempty + 2;  // after an abort: every MMA issued has completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
+  __shared__ int abort_flag;       // a bounded wait of this CTA gave up
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total_tiles = p.m_tiles * p.n_tiles;
@@ -187,12 +158,14 @@ __global__ void __launch_bounds__(kEncThreads, 1) gemm_kernel(const __grid_const
   if (threadIdx.x == 0) {
     for (int s = 0; s < kEncStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], MODE == kModeK ? 2 : 1);  // MMA commit (+ the pool warp in mode K)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], 4);
     }
+    mbar_init(drained, 1);
+    abort_flag = 0;
     fence_mbar_init();
   }
   if (MODE == kModeK) {
@@ -214,7 +187,7 @@ __global__ void __launch_bounds__(kEncThreads, 1) gemm_kernel(const __grid_const
       prefetch_tensormap(&map_a);
       prefetch_tensormap(&map_b);
       int it = 0;
-      for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      for (int tile = blockIdx.x; tile < total_tiles && !abort_flag; tile += gridDim.x) {
         const int m = tile / p.n_tiles, n = tile % p.n_tiles;
         int ya0, ya1;
         if (MODE == kModeK) {
@@ -228,7 +201,7 @@ __global__ void __launch_bounds__(kEncThreads, 1) gemm_kernel(const __grid_const
         }
         for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
           const int st = it % kEncStages;
-          if (it >= kEncStages) mbar_wait(&empty[st], ((it / kEncStages) - 1) & 1);
+          if (it >= kEncStages && !mbar_wait(&empty[st], ((it / kEncStages) - 1) & 1, &abort_flag)) break;
           uint8_t* a_s = stages + st * kStageBytes;
           uint8_t* b_s = a_s + kABytes;
           mbar_arrive_expect_tx(&full[st], kStageBytes);
@@ -238,20 +211,22 @@ __global__ void __launch_bounds__(kEncThreads, 1) gemm_kernel(const __grid_const
           tma_load_2d(b_s, &map_b, &full[st], kx, n * kBN);
         }
       }
+      // after an abort: the stages issued and possibly still in flight land before the CTA exits
+      if (abort_flag) mbar_drain_ring(full, kEncStages, it - kEncStages, it);
     }
   } else if (warp == 1) {
     // ------------------------- MMA issuer -------------------------
     if (lane == 0) {
       constexpr uint32_t idesc = umma_idesc_bf16(kBM, kBN);
       int it = 0, lt = 0;
-      for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++lt) {
+      for (int tile = blockIdx.x; tile < total_tiles && !abort_flag; tile += gridDim.x, ++lt) {
         const int buf = lt & 1;
-        if (lt >= 2) mbar_wait(&tempty[buf], ((lt >> 1) - 1) & 1);
+        if (lt >= 2 && !mbar_wait(&tempty[buf], ((lt >> 1) - 1) & 1, &abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * kBN;
         for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
           const int st = it % kEncStages;
-          mbar_wait(&full[st], (it / kEncStages) & 1);
+          if (!mbar_wait(&full[st], (it / kEncStages) & 1, &abort_flag)) break;
           tc_fence_after();
           const uint32_t a_addr = smem_u32(stages + st * kStageBytes);
           const uint32_t b_addr = a_addr + kABytes;
@@ -264,6 +239,52 @@ __global__ void __launch_bounds__(kEncThreads, 1) gemm_kernel(const __grid_const
         }
         umma_commit(&tfull[buf]);
       }
+      if (abort_flag) {  // every MMA issued completes before the TMEM is freed
+        umma_commit(drained);
+        mbar_drain_ring(drained, 1, 0, 1);
+      }
+    }
+  } else if (MODE == kModeK && warp == 6) {
+    // ------------- pool warp: chunk means of the H tiles the MMA reads -------------
+    // For the first N tile of each chunk pair, sum every 64-column block of the pair's two
+    // 64-row boxes over each chunk's own rows (in row order, fp32) and store the mean as bf16
+    // hi + lo terms; for the other N tiles only release the stage.  Lane l owns columns 2l, 2l+1.
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total_tiles && !abort_flag; tile += gridDim.x) {
+      const int m = tile / p.n_tiles, n = tile % p.n_tiles;
+      const int c0 = 2 * m, c1 = 2 * m + 1;
+      const int len0 = p.clen[c0];
+      const int len1 = c1 < p.n_chunks ? p.clen[c1] : 0;
+      for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
+        const int st = it % kEncStages;
+        if (!warp_wait(&full[st], (it / kEncStages) & 1, &abort_flag)) break;
+        if (n == 0) {
+          const uint8_t* a_s = stages + st * kStageBytes;
+#pragma unroll
+          for (int box = 0; box < 2; ++box) {
+            const int len = box ? len1 : len0;
+            if (len == 0) continue;
+            const uint8_t* bx = a_s + box * (kABytes / 2);
+            float s0 = 0.f, s1 = 0.f;
+            for (int r = 0; r < len; ++r) {  // 128-byte rows, 16-byte units swizzled by the row
+              const uint32_t w =
+                  *reinterpret_cast<const uint32_t*>(bx + r * 128 + ((((lane >> 2) ^ (r & 7))) << 4) + (lane & 3) * 4);
+              const float2 f = unpack_bf16x2(w);
+              s0 += f.x;
+              s1 += f.y;
+            }
+            const float inv = 1.0f / (float)len;
+            const float m0 = s0 * inv, m1 = s1 * inv;
+            const float h0 = __bfloat162float(__float2bfloat16_rn(m0));
+            const float h1 = __bfloat162float(__float2bfloat16_rn(m1));
+            __nv_bfloat16* dst = p.hbar + (size_t)(c0 + box) * 2 * p.hidden + kb * kBK + 2 * lane;
+            *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(h0, h1);
+            *reinterpret_cast<uint32_t*>(dst + p.hidden) = pack_bf16x2(m0 - h0, m1 - h1);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+      }
     }
   } else {
     // ------------------------- epilogue (warps 2..5) -------------------------
@@ -274,7 +295,10 @@ __global__ void __launch_bounds__(kEncThreads, 1) gemm_kernel(const __grid_const
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++lt) {
       const int m = tile / p.n_tiles, n = tile % p.n_tiles;
       const int buf = lt & 1;
-      mbar_wait(&tfull[buf], (lt >> 1) & 1);
+      // the four epilogue warps meet at named barriers (mode K): they decide together, at the top of
+      // a tile, whether to leave
+      const bool ok = warp_wait(&tfull[buf], (lt >> 1) & 1, &abort_flag);
+      if (MODE == kModeK ? named_bar_any(3, 128, !ok) : !ok) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + ((uint32_t)(32 * q) << 16) + buf * kBN;
       if (MODE == kModeK) {
@@ -375,7 +399,7 @@ size_t gemm_smem_bytes(int mode, int bn) {
   const int stages = mode == kModeK ? 3 : 4;
   const size_t tables = mode == kModeK ? (64 * 64 + 2 * 64) * sizeof(float2) : 0;
   return 1024 + (size_t)stages * (kABytes + bn * kBK * 2) + 2 * 4 * bn * sizeof(float) + tables +
-         (2 * kEncStagesMax + 4) * sizeof(uint64_t) + 16;
+         (2 * kEncStagesMax + 5) * sizeof(uint64_t) + 16;
 }
 
 template <int MODE>
@@ -384,11 +408,11 @@ cudaError_t launch_gemm(int bn, int grid, size_t smem, cudaStream_t s, const CUt
   if (bn == 256) {
     cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(gemm_kernel<MODE, 256>), (int)smem);
     if (e != cudaSuccess) return e;
-    gemm_kernel<MODE, 256><<<grid, kEncThreads, smem, s>>>(ma, mb, p);
+    gemm_kernel<MODE, 256><<<grid, MODE == kModeK ? kEncThreadsK : kEncThreads, smem, s>>>(ma, mb, p);
   } else {
     cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(gemm_kernel<MODE, 128>), (int)smem);
     if (e != cudaSuccess) return e;
-    gemm_kernel<MODE, 128><<<grid, kEncThreads, smem, s>>>(ma, mb, p);
+    gemm_kernel<MODE, 128><<<grid, MODE == kModeK ? kEncThreadsK : kEncThreads, smem, s>>>(ma, mb, p);
   }
   return cudaGetLastError();
 }
@@ -459,7 +483,7 @@ msa_status encode_launch(const msa_dims& d, const void* H, int64_t T, const int6
         static_cast<const uint16_t*>(W_KR), hidden, NR, reinterpret_cast<uint16_t*>(w.wvrT), NV);
     MSA_CUDA_CHECK(cudaGetLastError());
   }
-  // ---- K̄: per-token projection + RoPE + pooling on tcgen05 ----
+  // ---- K̄: per-token projection + RoPE + pooling on tcgen05; H̄ (hi | lo) from the same tiles ----
   {
     CUtensorMap ma, mb;
     const uint64_t adims[2] = {(uint64_t)hidden, (uint64_t)T};
@@ -485,17 +509,12 @@ msa_status encode_launch(const msa_dims& d, const void* H, int64_t T, const int6
     p.tok0 = w.tok0;
     p.clen = w.clen;
     p.pos0 = w.pos0;
+    p.hbar = w.hbar;
     p.out0 = static_cast<__nv_bfloat16*>(K_bar);
     p.n_out0 = NK;
     const int grid = std::max(1, std::min(sm_count(), p.m_tiles * p.n_tiles));
     TraceScope ts(kKEncGemmK, s);
     MSA_CUDA_CHECK(launch_gemm<kModeK>(bn, grid, gemm_smem_bytes(kModeK, bn), s, ma, mb, p));
-  }
-  // ---- H̄ (hi | lo) ----
-  {
-    TraceScope ts(kKEncPoolH, s);
-    pool_h_kernel<<<n_chunks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(H), hidden, w.tok0, w.clen, w.hbar);
-    MSA_CUDA_CHECK(cudaGetLastError());
   }
   // ---- V̄ | K̄^R = H̄ [W_V | W^KR] ----
   {

@@ -44,7 +44,6 @@ enum KernelId : int {
   kKEncChunkMap,
   kKEncTransposeW,
   kKEncGemmK,
-  kKEncPoolH,
   kKEncGemmPooled,
   kKRopeRows,
   kKGatherPlan,
@@ -90,6 +89,13 @@ int sm_count();
 int max_smem_optin();
 // cudaFuncSetAttribute(kernel, MaxDynamicSharedMemorySize, bytes), skipped when already set
 cudaError_t set_max_dynamic_smem(const void* kernel, int bytes);
+// cudaFuncSetAttribute(kernel, PreferredSharedMemoryCarveout, max shared), once per device and kernel.
+// The large kernels (scan, attention, GEMM) need the largest shared-memory carveout; a small kernel
+// that prefers another carveout keeps an SM in that configuration while its CTAs run there, and a
+// large kernel's CTA cannot start on that SM until they leave.  With every kernel of the library
+// preferring the same carveout, small kernels on a second stream (the host-tier gather) share SMs
+// with a running scan or attention instead of holding them.
+void prefer_shared_carveout(const void* kernel);
 msa_status encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, void* gaddr,
                              const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
                              CUtensorMapSwizzle swizzle);
@@ -106,6 +112,7 @@ void rope_turns(const msa_dims& d, uint64_t* f /* [head_dim / 2] */);
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                        Args&&... args) {
+  prefer_shared_carveout(reinterpret_cast<const void*>(kernel));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -123,6 +130,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                                int cluster_x, Args&&... args) {
+  prefer_shared_carveout(reinterpret_cast<const void*>(kernel));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -152,6 +160,11 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
                         const float* kr_inv_norm, float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws,
                         cudaStream_t s, bool early_inputs = false);
 
+msa_status validate_route(const msa_dims* dims, const void* Hq, const void* W_QR, int32_t B, int32_t q_tokens,
+                          const void* KR_bar, const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks, int32_t k,
+                          msa_doc_agg agg, int32_t kr_layout, const float* kr_inv_norm, const float* doc_scores,
+                          const int32_t* topk_idx, const float* topk_score);
+
 msa_status topk_merge_launch(const float* cand_score, const int32_t* cand_idx, int B, int n_cand, int k,
                              int32_t* topk_idx, float* topk_score, cudaStream_t s);
 
@@ -167,6 +180,12 @@ msa_status gather_kv_launch(const msa_dims& d, const void* K_host, const void* V
                             int n_docs, const int32_t* topk_idx, int B, int k, void* K_stage, void* V_stage,
                             int capacity_chunks, int32_t* stage_off, int32_t* stage_idx, int32_t* stage_src,
                             cudaStream_t s);
+size_t tiered_workspace_size(const msa_dims& d, int B, int n_docs, int n_chunks, int k, int t_loc_max, int pos_offset,
+                             int capacity);
+msa_status tiered_launch(const msa_dims& d, const msa_layer* layers, const void* const* K_dev, const void* const* V_dev,
+                         int n_layers, int B, const int32_t* chunk_off, int n_docs, int n_chunks, int k,
+                         const int32_t* loc_len, int t_loc_max, int pos_offset, int capacity, void* ws,
+                         cudaStream_t s, cudaStream_t cs);
 msa_status rope_rows_launch(const msa_dims& d, void* x, int rows, int heads, const int32_t* pos, cudaStream_t s);
 msa_status rope_cache_build(const msa_dims& d, int t_loc_max, int pos_offset, float2* tab, cudaStream_t s);
 

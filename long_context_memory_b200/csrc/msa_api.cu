@@ -118,6 +118,28 @@ cudaError_t set_max_dynamic_smem(const void* kernel, int bytes) {
   return e;
 }
 
+void prefer_shared_carveout(const void* kernel) {
+  struct Entry {
+    int dev;
+    const void* fn;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    for (const Entry& e : done)
+      if (e.dev == dev && e.fn == kernel) return;
+  }
+  // a hint: a device that cannot honour it keeps its default (the launch still succeeds)
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared) !=
+      cudaSuccess)
+    cudaGetLastError();
+  std::lock_guard<std::mutex> lk(mu);
+  done.push_back({dev, kernel});
+}
+
 int max_smem_optin() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
@@ -157,7 +179,7 @@ msa_status encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int ra
     CUtensorMap map;
     bool used;
   };
-  constexpr int kSlots = 32;
+  constexpr int kSlots = 128;  // a multi-layer call encodes one key map per layer
   thread_local Slot cache[kSlots] = {};
   thread_local int next = 0;
   Key key;
@@ -196,7 +218,7 @@ msa_status encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int ra
 namespace {
 const char* kKernelNames[kKernelCount] = {
     "router_query", "scan", "topk_slice", "topk_merge", "rope_table", "attn_split", "attn_combine",
-    "enc_chunk_map", "enc_transpose_w", "enc_gemm_k", "enc_pool_h", "enc_gemm_pooled", "rope_rows", "gather_plan", "gather_copy",
+    "enc_chunk_map", "enc_transpose_w", "enc_gemm_k", "enc_gemm_pooled", "rope_rows", "gather_plan", "gather_copy",
     "chunk_off_extend", "aux_loss", "kv_append", "kr_norms"};
 
 struct TraceState {
@@ -262,6 +284,29 @@ TraceScope::~TraceScope() {
   if (slot < (int)t.recs.size()) cudaEventRecordWithFlags(t.recs[slot].b, stream, flags);
 }
 
+// ---------------------------------------------------------------------------
+// self-test of the bounded waits: four warps wait on mbarriers that nothing arrives on
+// ---------------------------------------------------------------------------
+namespace {
+__global__ void __launch_bounds__(128) wait_selftest_kernel(uint64_t limit_ns, int n_waits,
+                                                            unsigned long long* elapsed_ns) {
+  __shared__ uint64_t bars[4];
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);  // no thread ever arrives
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const uint64_t t0 = globaltimer_ns();
+  if (lane == 0)
+    for (int i = 0; i < n_waits; ++i) mbar_wait(&bars[warp], 0, &abort_flag, limit_ns);
+  __syncthreads();
+  if (threadIdx.x == 0) *elapsed_ns = globaltimer_ns() - t0;
+}
+}  // namespace
+
 }  // namespace msa
 
 using namespace msa;
@@ -323,6 +368,17 @@ msa_status msa_check_device_errors(uint32_t* bits_out) {
   return MSA_OK;
 }
 
+msa_status msa_selftest_wait_timeout(int32_t limit_us, int32_t n_waits, uint64_t* elapsed_ns, void* stream) {
+  if (limit_us < 1 || limit_us > 100000) return fail(MSA_ERR_INVALID_ARG, "limit_us must be in [1, 100000]");
+  if (n_waits < 1 || n_waits > 1000) return fail(MSA_ERR_INVALID_ARG, "n_waits must be in [1, 1000]");
+  CHECK_PTR(elapsed_ns);
+  if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
+  wait_selftest_kernel<<<1, 128, 0, static_cast<cudaStream_t>(stream)>>>((uint64_t)limit_us * 1000ull, n_waits,
+                                                                         reinterpret_cast<unsigned long long*>(elapsed_ns));
+  MSA_CUDA_CHECK(cudaGetLastError());
+  return MSA_OK;
+}
+
 msa_status msa_chunk_offsets(const int64_t* doc_off_host, int32_t n_docs, int32_t chunk, int32_t* chunk_off_host,
                              int32_t* n_chunks_out) {
   if (!doc_off_host || !chunk_off_host) return fail(MSA_ERR_INVALID_ARG, "NULL offset array");
@@ -349,12 +405,15 @@ size_t msa_route_workspace_size(const msa_dims* dims, int32_t B, int32_t q_token
   return route_workspace(*dims, B, q_tokens, n_docs, n_chunks, k, agg, nullptr, nullptr);
 }
 
-msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR, int32_t B, int32_t q_tokens,
-                          const void* KR_bar,
-                          const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks, int32_t k, msa_doc_agg agg,
-                          int32_t kr_layout, const float* kr_inv_norm, float* doc_scores, int32_t* topk_idx,
-                          float* topk_score, void* ws, size_t ws_bytes,
-                          void* stream) {
+}  // extern "C"
+
+namespace msa {
+// Every argument check of msa_route_topk except the workspace's (shared with the static-scratch
+// entry point, which must report the same errors for the same arguments).
+msa_status validate_route(const msa_dims* dims, const void* Hq, const void* W_QR, int32_t B, int32_t q_tokens,
+                          const void* KR_bar, const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks, int32_t k,
+                          msa_doc_agg agg, int32_t kr_layout, const float* kr_inv_norm, const float* doc_scores,
+                          const int32_t* topk_idx, const float* topk_score) {
   msa_status st = check_dims(dims, false, true);
   if (st != MSA_OK) return st;
   if (W_QR && (dims->hidden < 64 || dims->hidden % 64 != 0 || dims->hidden > 8192))
@@ -367,7 +426,6 @@ msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR
   if (k < 1 || k > n_docs || k > 256)
     return fail(MSA_ERR_INVALID_ARG, "k must be in [1, min(n_docs, 256)] (got %d, n_docs %d)", k, n_docs);
   if (agg != MSA_AGG_MAX && agg != MSA_AGG_MEAN) return fail(MSA_ERR_INVALID_ARG, "unknown aggregation %d", (int)agg);
-  const bool early_inputs = (kr_layout & MSA_ROUTE_EARLY_INPUTS) != 0;
   kr_layout &= ~MSA_ROUTE_EARLY_INPUTS;
   if (kr_layout != 0 && kr_layout != 1)
     return fail(MSA_ERR_INVALID_ARG, "kr_layout must be 0 or 1, optionally | MSA_ROUTE_EARLY_INPUTS (got %d)", kr_layout);
@@ -380,11 +438,28 @@ msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR
   CHECK_OPT_PTR(doc_scores);
   CHECK_PTR(topk_idx);
   CHECK_PTR(topk_score);
+  CHECK_OPT_PTR(kr_inv_norm);
+  return MSA_OK;
+}
+}  // namespace msa
+
+extern "C" {
+
+msa_status msa_route_topk(const msa_dims* dims, const void* Hq, const void* W_QR, int32_t B, int32_t q_tokens,
+                          const void* KR_bar,
+                          const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks, int32_t k, msa_doc_agg agg,
+                          int32_t kr_layout, const float* kr_inv_norm, float* doc_scores, int32_t* topk_idx,
+                          float* topk_score, void* ws, size_t ws_bytes,
+                          void* stream) {
+  msa_status st = validate_route(dims, Hq, W_QR, B, q_tokens, KR_bar, chunk_off, n_docs, n_chunks, k, agg, kr_layout,
+                                 kr_inv_norm, doc_scores, topk_idx, topk_score);
+  if (st != MSA_OK) return st;
+  const bool early_inputs = (kr_layout & MSA_ROUTE_EARLY_INPUTS) != 0;
+  kr_layout &= ~MSA_ROUTE_EARLY_INPUTS;
   const size_t need = route_workspace(*dims, B, q_tokens, n_docs, n_chunks, k, agg, nullptr, nullptr);
   if (ws_bytes < need) return fail(MSA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
   if (need && (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)))
     return fail(MSA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
-  CHECK_OPT_PTR(kr_inv_norm);
   if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
   return route_launch(*dims, Hq, W_QR, B, q_tokens, KR_bar, chunk_off, n_docs, n_chunks, k, agg, kr_layout, kr_inv_norm,
                       doc_scores, topk_idx, topk_score, ws, static_cast<cudaStream_t>(stream), early_inputs);
@@ -516,6 +591,81 @@ msa_status msa_gather_kv(const msa_dims* dims, const void* K_bar_host, const voi
   return gather_kv_launch(*dims, dev_ptr[0], dev_ptr[1], chunk_off, n_docs, topk_idx, B, k, K_stage, V_stage,
                           capacity_chunks, stage_chunk_off, stage_topk_idx, static_cast<int32_t*>(ws),
                           static_cast<cudaStream_t>(stream));
+}
+
+// the device address of pinned host memory, or an error when it is not pinned and device-mapped
+static msa_status mapped_host(const void* p, const char* name, const void** dev) {
+  cudaPointerAttributes a;
+  cudaError_t e = cudaPointerGetAttributes(&a, p);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaPointerGetAttributes");
+  if (a.type != cudaMemoryTypeHost || !a.devicePointer)
+    return fail(MSA_ERR_INVALID_ARG, "%s must be pinned (page-locked, device-mapped) host memory", name);
+  *dev = a.devicePointer;
+  return MSA_OK;
+}
+
+static bool tiered_sizes_ok(const msa_dims* dims, int32_t B, int32_t n_docs, int32_t n_chunks, int32_t k,
+                            int32_t t_loc_max, int32_t pos_offset, int32_t capacity_chunks) {
+  return dims && B >= 1 && B <= 65535 && n_docs >= 1 && n_chunks >= n_docs && k >= 1 && k <= n_docs && k <= 256 &&
+         t_loc_max >= 1 && pos_offset >= 0 && (int64_t)pos_offset + t_loc_max <= (1 << 24) && capacity_chunks >= 1 &&
+         dims->n_kv >= 1 && dims->n_q >= dims->n_kv && dims->n_r >= 1 && dims->d_r >= 1;
+}
+
+size_t msa_tiered_workspace_size(const msa_dims* dims, int32_t B, int32_t n_docs, int32_t n_chunks, int32_t k,
+                                 int32_t t_loc_max, int32_t pos_offset, int32_t capacity_chunks) {
+  if (!tiered_sizes_ok(dims, B, n_docs, n_chunks, k, t_loc_max, pos_offset, capacity_chunks)) return 0;
+  return tiered_workspace_size(*dims, B, n_docs, n_chunks, k, t_loc_max, pos_offset, capacity_chunks);
+}
+
+msa_status msa_tiered_decode(const msa_dims* dims, const msa_layer* layers, int32_t n_layers, int32_t B,
+                             const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks, int32_t k,
+                             const int32_t* loc_len, int32_t t_loc_max, int32_t pos_offset, int32_t capacity_chunks,
+                             void* ws, size_t ws_bytes, void* stream, void* copy_stream) {
+  msa_status st = check_dims(dims, true, true);
+  if (st != MSA_OK) return st;
+  if (!layers) return fail(MSA_ERR_INVALID_ARG, "layers is NULL");
+  if (n_layers < 1 || n_layers > 4096) return fail(MSA_ERR_INVALID_ARG, "n_layers must be in [1, 4096] (got %d)", n_layers);
+  if (B < 1 || B > 65535) return fail(MSA_ERR_INVALID_ARG, "B must be in [1, 65535] (got %d)", B);
+  if (n_docs < 1 || n_chunks < n_docs)
+    return fail(MSA_ERR_INVALID_ARG, "need 1 <= n_docs <= n_chunks (got %d, %d)", n_docs, n_chunks);
+  if (k < 1 || k > n_docs || k > 256)
+    return fail(MSA_ERR_INVALID_ARG, "k must be in [1, min(n_docs, 256)] (got %d, n_docs %d)", k, n_docs);
+  if ((size_t)((n_docs + 4095) / 4096) * k > 24576)
+    return fail(MSA_ERR_UNSUPPORTED, "n_docs * k too large for the top-k merge");
+  if (t_loc_max < 1) return fail(MSA_ERR_INVALID_ARG, "t_loc_max must be >= 1 (got %d)", t_loc_max);
+  if (pos_offset < 0 || (int64_t)pos_offset + t_loc_max > (1 << 24))
+    return fail(MSA_ERR_INVALID_ARG, "positions must lie in [0, 2^24)");
+  if (capacity_chunks < 1) return fail(MSA_ERR_INVALID_ARG, "capacity_chunks must be >= 1");
+  CHECK_PTR(chunk_off);
+  CHECK_PTR(loc_len);
+  std::vector<const void*> K_dev((size_t)n_layers), V_dev((size_t)n_layers);
+  for (int32_t l = 0; l < n_layers; ++l) {
+    const msa_layer& L = layers[l];
+    if (L.W_QR && (dims->hidden < 64 || dims->hidden % 64 != 0 || dims->hidden > 8192))
+      return fail(MSA_ERR_UNSUPPORTED, "hidden must be a multiple of 64 in [64, 8192] (got %d)", dims->hidden);
+    if (!L.Hq || !aligned16(L.Hq) || !L.KR_bar || !aligned16(L.KR_bar) || !L.q || !aligned16(L.q) || !L.K_loc ||
+        !aligned16(L.K_loc) || !L.V_loc || !aligned16(L.V_loc) || !L.topk_idx || !aligned16(L.topk_idx) ||
+        !L.topk_score || !aligned16(L.topk_score) || !L.out || !aligned16(L.out) || !L.K_bar_host ||
+        !aligned16(L.K_bar_host) || !L.V_bar_host || !aligned16(L.V_bar_host))
+      return fail(MSA_ERR_INVALID_ARG, "layer %d: a required pointer is NULL or not 16-byte aligned", l);
+    if ((L.W_QR && !aligned16(L.W_QR)) || (L.kr_inv_norm && !aligned16(L.kr_inv_norm)) ||
+        (L.k_new && !aligned16(L.k_new)) || (L.v_new && !aligned16(L.v_new)))
+      return fail(MSA_ERR_INVALID_ARG, "layer %d: an optional pointer is not 16-byte aligned", l);
+    if ((L.k_new == nullptr) != (L.v_new == nullptr))
+      return fail(MSA_ERR_INVALID_ARG, "layer %d: k_new and v_new go together", l);
+    st = mapped_host(L.K_bar_host, "K_bar_host", &K_dev[l]);
+    if (st != MSA_OK) return st;
+    st = mapped_host(L.V_bar_host, "V_bar_host", &V_dev[l]);
+    if (st != MSA_OK) return st;
+  }
+  const size_t need = tiered_workspace_size(*dims, B, n_docs, n_chunks, k, t_loc_max, pos_offset, capacity_chunks);
+  if (ws_bytes < need) return fail(MSA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(MSA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
+  if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
+  return tiered_launch(*dims, layers, K_dev.data(), V_dev.data(), n_layers, B, chunk_off, n_docs, n_chunks, k, loc_len,
+                       t_loc_max, pos_offset, capacity_chunks, ws, static_cast<cudaStream_t>(stream),
+                       static_cast<cudaStream_t>(copy_stream));
 }
 
 msa_status msa_rope_rows(const msa_dims* dims, void* x, int32_t rows, int32_t heads, const int32_t* positions,

@@ -320,7 +320,7 @@ struct ScanGeom {
   static constexpr int kStageBytes = kKBytes + kQBytes;
   static constexpr int kStages = (NQ == 16 || DR == 64) ? 5 : 4;
   static constexpr int kNormBytes = 2 * 8 * kScanM * 4;  // [2 tiles][8 heads][128 rows] fp32
-  static constexpr int kBars = 2 * kStages + kBufs * 9 + 4;
+  static constexpr int kBars = 2 * kStages + kBufs * 9 + 5;
   static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + kNormBytes + kBars * 8 + 16;
 };
 
@@ -333,7 +333,8 @@ struct ScanGeom {
 template <int DR, int NQ, bool MEAN, int QW>
 __device__ __forceinline__ void scan_epilogue(const ScanParams& p, int q4, int q_off, int lane, int t_begin, int n_lt,
                                               uint32_t tmem_base, uint32_t buf_cols, const float* n2s, uint64_t* tfull,
-                                              uint64_t* tempty, uint64_t* nfull, uint64_t* nempty) {
+                                              uint64_t* tempty, uint64_t* nfull, uint64_t* nempty,
+                                              volatile int* abort) {
   using Gm = ScanGeom<DR, NQ>;
   const int n_r = p.n_r;
   const int row = 32 * q4 + lane;  // chunk within the tile
@@ -386,10 +387,10 @@ __device__ __forceinline__ void scan_epilogue(const ScanParams& p, int q4, int q
 #pragma unroll
       for (int hh = 0; hh < 8; ++hh)
         invg[hh] = (active && hh < n_r && jrow < p.n_chunks) ? __ldg(&p.inv_norm[(size_t)jrow * n_r + hh]) : 0.f;
-    } else {
-      mbar_wait(&nfull[nbuf], (lt >> 1) & 1);
+    } else if (!warp_wait(&nfull[nbuf], (lt >> 1) & 1, abort)) {
+      return;
     }
-    mbar_wait(&tfull[buf], use & 1);
+    if (!warp_wait(&tfull[buf], use & 1, abort)) return;
     tc_fence_after();
     const float* nb2 = n2s + (size_t)nbuf * 8 * kScanM;
     float acc[QW];
@@ -468,7 +469,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   uint64_t* tempty = tfull + Gm::kBufs;        // [kBufs][8] epilogue has read a head's accumulator
   uint64_t* nfull = tempty + Gm::kBufs * 8;    // [2] norms of a tile written
   uint64_t* nempty = nfull + 2;                // [2] epilogue has read a tile's norms
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(nempty + 2);
+  uint64_t* drained = nempty + 2;              // [1] after an abort: every MMA issued has completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
+  __shared__ int abort_flag;                   // a bounded wait of this CTA gave up
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_r = p.n_r;
@@ -490,6 +493,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       mbar_init(&nfull[b], kScanNormWarps);
       mbar_init(&nempty[b], kScanEpiWarps);
     }
+    mbar_init(drained, 1);
+    abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&kr_map);
     prefetch_tensormap(&q_map);
@@ -536,13 +541,16 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   if (warp == 0) {
     // ------------------------- TMA producer -------------------------
     if (lane == 0) {
-      for (int it = 0; it < n_it; ++it) {
+      int it = 0;
+      for (; it < n_it; ++it) {
         if (it >= n_pre) {
-          if (it >= S) mbar_wait(&empty[it % S], ((it / S) - 1) & 1);
+          if (it >= S && !mbar_wait(&empty[it % S], ((it / S) - 1) & 1, &abort_flag)) break;
           load_keys(it);
         }
         load_query(it);
       }
+      // after an abort: the stages issued and possibly still in flight land before the CTA exits
+      if (abort_flag) mbar_drain_ring(full, S, it - S, it);
     }
   } else if (warp == 1) {
     // ------------------------- MMA issuer -------------------------
@@ -552,8 +560,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         const int lt = it / n_r, h = it % n_r;
         const int buf = lt % Gm::kBufs, use = lt / Gm::kBufs;
         const int st = it % S;
-        if (use >= 1) mbar_wait(&tempty[buf * 8 + h], (use - 1) & 1);  // this head's columns read
-        mbar_wait(&full[st], (it / S) & 1);
+        if (use >= 1 && !mbar_wait(&tempty[buf * 8 + h], (use - 1) & 1, &abort_flag)) break;  // head's columns read
+        if (!mbar_wait(&full[st], (it / S) & 1, &abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * buf_cols + h * Gm::kCols;
         const uint32_t k_addr = smem_u32(stages + st * Gm::kStageBytes);
@@ -568,11 +576,15 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         umma_commit(&empty[st]);
         if (h == n_r - 1) umma_commit(&tfull[buf]);
       }
+      if (abort_flag) {  // every MMA issued completes before the TMEM is freed
+        umma_commit(drained);
+        mbar_drain_ring(drained, 1, 0, 1);
+      }
     }
   } else if (warp < 2 + kScanNormWarps && p.inv_norm) {
     // norms given: these four warps take the second half of the queries of each row
     scan_epilogue<DR, NQ, MEAN, NQ / 2>(p, warp & 3, NQ / 2, lane, t_begin, n_lt, tmem_base, buf_cols, n2s, tfull,
-                                        tempty, nfull, nempty);
+                                        tempty, nfull, nempty, &abort_flag);
   } else if (warp < 2 + kScanNormWarps) {
     // ------- norm warps: squared norm of every row's head-h slice, stage released at once -------
     const int row = 32 * (warp & 3) + lane;  // chunk within the tile
@@ -580,8 +592,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       const int lt = it / n_r, h = it % n_r;
       const int buf = lt & 1;  // norm buffer
       const int st = it % S;
-      if (h == 0 && lt >= 2) mbar_wait(&nempty[buf], ((lt >> 1) - 1) & 1);  // n2s[buf] is free again
-      mbar_wait(&full[st], (it / S) & 1);
+      if (h == 0 && lt >= 2 && !warp_wait(&nempty[buf], ((lt >> 1) - 1) & 1, &abort_flag)) break;  // n2s[buf] free
+      if (!warp_wait(&full[st], (it / S) & 1, &abort_flag)) break;
       const uint8_t* k_s = stages + st * Gm::kStageBytes;
       float n2p[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -608,17 +620,17 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     // epilogue warps: every query of each row, or the first half when the norms are given
     if (p.inv_norm)
       scan_epilogue<DR, NQ, MEAN, NQ / 2>(p, warp & 3, 0, lane, t_begin, n_lt, tmem_base, buf_cols, n2s, tfull, tempty,
-                                          nfull, nempty);
+                                          nfull, nempty, &abort_flag);
     else
       scan_epilogue<DR, NQ, MEAN, NQ>(p, warp & 3, 0, lane, t_begin, n_lt, tmem_base, buf_cols, n2s, tfull, tempty,
-                                      nfull, nempty);
+                                      nfull, nempty, &abort_flag);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, p.tmem_cols);
 
-  if (p.ticket) {
+  if (p.ticket && !abort_flag) {  // a CTA that gave up leaves the top-k unselected (error word set)
     // every CTA's document maxima are in L2: the last one selects the top-k (the pipeline's
     // shared memory is free again and holds the keys)
     __shared__ bool last_cta;

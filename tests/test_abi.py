@@ -212,6 +212,47 @@ def test_topk_merge_validation(msa):
     assert lib.msa_topk_merge(FAKE, FAKE, 1, 30000, 4, FAKE, FAKE, None) == 1  # too many candidates
 
 
+def _tiered(msa, dims, layers=None, n_layers=1, B=1, n_docs=10, n_chunks=20, k=4, t_loc=16, pos=4, cap=64,
+            ws_bytes=None, **ptrs):
+    dd = msa.Dims.of(dims)
+    if layers is None:
+        layers = (msa.Layer * max(1, n_layers))()
+        for L in layers:
+            for f in ("Hq", "KR_bar", "K_bar_host", "V_bar_host", "q", "K_loc", "V_loc", "topk_idx", "topk_score",
+                      "out"):
+                setattr(L, f, FAKE)
+            for f, v in ptrs.items():
+                setattr(L, f, v)
+    need = msa.lib.msa_tiered_workspace_size(ctypes.byref(dd), B, n_docs, n_chunks, k, t_loc, pos, cap)
+    if ws_bytes is None:
+        ws_bytes = need
+    return msa.lib.msa_tiered_decode(ctypes.byref(dd), layers, n_layers, B, FAKE, n_docs, n_chunks, k, FAKE, t_loc, pos,
+                                     cap, 0x100000, ws_bytes, None, None)
+
+
+def test_tiered_validation(msa):
+    # every argument error is reported before the pinned-memory lookup and before any launch
+    ok = _dims(hidden=512, n_q=32, n_kv=8, head_dim=128, n_r=8, d_r=128)
+    assert _tiered(msa, ok, n_layers=0) == 1
+    assert msa.lib.msa_tiered_decode(ctypes.byref(msa.Dims.of(ok)), None, 1, 1, FAKE, 10, 20, 4, FAKE, 16, 4, 64,
+                                     0x100000, 1 << 20, None, None) == 1
+    assert _tiered(msa, ok, k=11) == 1                       # k > n_docs
+    assert _tiered(msa, ok, B=0) == 1
+    assert _tiered(msa, ok, t_loc=0) == 1                    # the attention needs a local cache
+    assert _tiered(msa, ok, cap=0) == 1
+    assert _tiered(msa, _dims(head_dim=96)) == 2
+    assert _tiered(msa, ok, q=FAKE + 4) == 1                 # misaligned
+    assert "layer 0" in msa.lib.msa_last_error().decode()
+    assert _tiered(msa, ok, K_bar_host=None) == 1
+    assert _tiered(msa, ok, k_new=FAKE) == 1                 # k_new without v_new
+    dd = ctypes.byref(msa.Dims.of(ok))
+    small = msa.lib.msa_tiered_workspace_size(dd, 1, 10, 20, 4, 16, 4, 64)
+    big = msa.lib.msa_tiered_workspace_size(dd, 1, 10, 20, 4, 16, 4, 128)
+    # two staging areas of K and V rows (n_kv * head_dim bf16 each) per extra chunk of capacity
+    assert small > 0 and big - small >= 4 * 64 * 8 * 128 * 2 - 4 * 256
+    assert msa.lib.msa_tiered_workspace_size(dd, 1, 10, 20, 4, 16, 4, 0) == 0
+
+
 def test_workspace_sizes_grow_with_problem(msa):
     d = msa.Dims.of(W.QWEN3_4B_DIMS)
     a = msa.lib.msa_route_workspace_size(ctypes.byref(d), 1, 1, 500, 16000, 16, 0)
@@ -322,6 +363,7 @@ def test_fault_injection_reaches_every_launching_entry_point(msa, monkeypatch):
         "kv_append": lambda: lib.msa_kv_append(r, FAKE, FAKE, FAKE, FAKE, 1, 16, FAKE, 2, None),
         "router_key_norms": lambda: lib.msa_router_key_norms(r, FAKE, 10, 0, FAKE, None),
         "topk_merge": lambda: lib.msa_topk_merge(FAKE, FAKE, 1, 8, 4, FAKE, FAKE, None),
+        "selftest_wait_timeout": lambda: lib.msa_selftest_wait_timeout(1000, 4, FAKE, None),
         "rope_rows": lambda: lib.msa_rope_rows(r, FAKE, 4, 2, FAKE, None),
         "rope_cache_build": lambda: lib.msa_rope_cache_build(r, 16, 2, 0x100000, lib.msa_rope_cache_size(r, 16),
                                                              None),
