@@ -348,6 +348,43 @@ msa_status msa_sparse_attend(const msa_dims* dims, const void* q, int32_t B, int
                              void* out, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Memory-parallel attention: one rank's share, and the merge of the ranks' shares.
+ * Pages: IRMaD "M. Materials & Methods", Memory Parallel and tiered storage item;
+ * EverMind article 2.3: the memory is sharded over GPUs by documents; after the
+ * global top-k (msa_topk_merge) every rank attends over the selected documents it
+ * holds and the partial results are reduced into the one softmax over
+ * [selected documents' K̄; local K].
+ * msa_sparse_attend_share: msa_sparse_attend (phase 0, no fused append) over this
+ * rank's shard, with
+ *   chunk_off [n_docs + 1], K_bar, V_bar  the shard's documents doc_base ..
+ *            doc_base + n_docs - 1 (chunk offsets rebased to the shard's first chunk);
+ *   topk_idx [B, k] GLOBAL document ids (the same array on every rank); ids outside
+ *            the shard are skipped (no error);
+ *   local_keys  1 on the one rank that attends over the local keys (K_loc, V_loc),
+ *            0 elsewhere (K_loc, V_loc may be NULL); loc_len and t_loc_max are given on
+ *            every rank: they place the query tokens (pos_offset + loc_len - M + t);
+ *   o_share  [B, M, n_q, head_dim] fp32 out: the share's softmax-weighted values
+ *            (normalised over the share's own keys; 0 for a share with no key);
+ *   lse2_share [B, M, n_q] fp32 out: log2 of the share's softmax denominator of the
+ *            scaled logits, sum_j 2^(scale log2(e) q.k_j) (-inf for no key).
+ * msa_attend_merge: out [rows, head_dim] bf16 = sum_r 2^(lse2_r - L) o_r with
+ *   L = log2 sum_r 2^lse2_r, for R shares laid out o_shares [R, rows, head_dim],
+ *   lse2_shares [R, rows] fp32 (rows = B * M * n_q); shares are added in rank order,
+ *   so every rank computes the same bits.  A row with no key anywhere gives 0.
+ * The merged result equals msa_sparse_attend over the unsharded memory up to fp32
+ * rounding of the reduction (the split-KV combine already merges partial softmaxes).
+ * ------------------------------------------------------------------------- */
+msa_status msa_sparse_attend_share(const msa_dims* dims, const void* q, int32_t B, int32_t q_tokens, const void* K_bar,
+                                   const void* V_bar, const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks,
+                                   int32_t doc_base, const int32_t* topk_idx, int32_t k, int32_t local_keys,
+                                   const void* K_loc, const void* V_loc, const int32_t* loc_len, int32_t t_loc_max,
+                                   int32_t pos_offset, const void* rope_cache, int32_t k_loc_rotated,
+                                   float softmax_scale, float* o_share, float* lse2_share, void* ws, size_t ws_bytes,
+                                   void* stream);
+msa_status msa_attend_merge(const float* o_shares, const float* lse2_shares, int32_t R, int32_t rows,
+                            int32_t head_dim, void* out, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Host tier: gather the selected documents' pooled K̄/V̄ from pinned host memory.
  * Pages: IRMaD "M. Materials & Methods", Memory Parallel and tiered storage
  * item; EverMind article 2.3: the content K̄/V̄ live in host DRAM and only the
@@ -394,10 +431,14 @@ msa_status msa_gather_kv(const msa_dims* dims, const void* K_bar_host, const voi
  * must not alias another layer's outputs or local cache).  They share the
  * document layout (chunk_off, n_docs, n_chunks), B, k, loc_len, t_loc_max and
  * pos_offset.  Per layer l the call enqueues, on
- * `stream`, msa_route_topk (agg MAX); on `copy_stream`, after an event on the
- * routing, msa_gather_kv of the routed documents into one of two staging areas
- * in ws; on `stream`, after the routing of layer l + 1 and an event on that
- * gather, msa_sparse_attend over the staged documents and the local keys.  The
+ * `stream`, msa_route_topk (agg MAX); on `copy_stream`, after an event,
+ * msa_gather_kv of the routed documents into one of two staging areas in ws;
+ * on `stream`, after the routing of layer l + 1 and an event on that gather,
+ * msa_sparse_attend over the staged documents and the local keys.  The gather
+ * of layer l waits for its routing, and also for the attention of layer l - 1
+ * when the routed documents' rows (B * k average documents over a ~50 GB/s host
+ * link) are expected to cross the bus faster than the next layer's router keys
+ * stream from HBM: it then runs beside the next routing alone.  The
  * results equal those calls made one after the other, bit for bit.  The
  * copy-stream work is joined back into `stream` before the call's last
  * attention, so work enqueued later on `stream` sees every output.

@@ -19,6 +19,7 @@ from typing import Optional
 __all__ = [
     "Dims", "MSAError", "lib", "chunk_offsets", "encode_memory", "append_memory", "route_topk", "sparse_attend",
     "aux_loss", "kv_append", "router_key_norms", "Layer", "tiered_layers", "tiered_workspace_size", "tiered_decode",
+    "sparse_attend_share", "attend_merge",
     "route_workspace_size", "attend_workspace_size", "rope_cache_build", "topk_merge", "rope_rows", "gather_kv", "encode_workspace_size", "check_device_errors", "selftest_wait_timeout",
     "trace_enable", "trace_reset", "trace_read", "trace_kernel_names", "AGG_MAX", "AGG_MEAN", "ATTEND_EARLY_LOCAL", "ROUTE_EARLY_INPUTS",
 ]
@@ -98,6 +99,9 @@ def _load():
         "msa_kv_append": (I32, [DP, P, P, P, P, I32, I32, P, I32, P]),
         "msa_gather_kv": (I32, [DP, P, P, I32, P, I32, P, I32, I32, P, P, I32, P, P, P, SZ, P]),
         "msa_tiered_workspace_size": (SZ, [DP, I32, I32, I32, I32, I32, I32, I32]),
+        "msa_sparse_attend_share": (I32, [DP, P, I32, I32, P, P, P, I32, I32, I32, P, I32, I32, P, P, P, I32, I32, P, I32, F,
+                                          P, P, P, SZ, P]),
+        "msa_attend_merge": (I32, [P, P, I32, I32, I32, P, P]),
         "msa_tiered_decode": (I32, [DP, ctypes.POINTER(Layer), I32, I32, P, I32, I32, I32, P, I32, I32, I32, P, SZ, P,
                                     P]),
         "msa_rope_cache_size": (SZ, [DP, I32]),
@@ -462,6 +466,50 @@ def sparse_attend(dims, q, K_bar, V_bar, chunk_off, topk_idx, K_loc, V_loc, loc_
                                  float(softmax_scale), int(phase) | (ATTEND_EARLY_LOCAL if early_local else 0),
                                  _ptr(out),
                                  _aligned_ptr(ws), nbytes, _stream(stream)))
+    return out
+
+
+def sparse_attend_share(dims, q, K_bar, V_bar, chunk_off, doc_base: int, topk_idx, local_keys: bool, K_loc, V_loc,
+                        loc_len, t_loc_max: int, pos_offset: int, softmax_scale: float = 0.0, rope_cache=None,
+                        k_loc_rotated: bool = False, out=None, ws=None, stream=None):
+    """One rank's share of a memory-parallel attention (see msa_sparse_attend_share).
+
+    ``K_bar``/``V_bar``/``chunk_off`` hold the shard's documents doc_base .. (chunk offsets rebased);
+    ``topk_idx`` [B, k] holds GLOBAL ids (others are skipped); the local keys count only where
+    ``local_keys``.  Returns (o [q.shape] fp32, lse2 [q.shape[:-1]] fp32)."""
+    import torch
+
+    dd = Dims.of(dims)
+    B, k = topk_idx.shape
+    M = q.shape[1] if q.dim() == 4 else 1
+    dev = q.device
+    n_docs = chunk_off.numel() - 1
+    if out is None:
+        out = (torch.empty(tuple(q.shape), dtype=torch.float32, device=dev),
+               torch.empty(tuple(q.shape[:-1]), dtype=torch.float32, device=dev))
+    if ws is not None:
+        nbytes = max(0, ws.numel() * ws.element_size() - 256)
+    else:
+        nbytes = attend_workspace_size(dims, B, k, t_loc_max, pos_offset, M)
+        ws = _workspace(nbytes, dev, ws)
+    _check(lib.msa_sparse_attend_share(ctypes.byref(dd), _ptr(q), B, M, _ptr(K_bar), _ptr(V_bar), _ptr(chunk_off), n_docs,
+                                       K_bar.shape[0], int(doc_base), _ptr(topk_idx), k, int(bool(local_keys)),
+                                       _ptr(K_loc) if local_keys else None, _ptr(V_loc) if local_keys else None,
+                                       _ptr(loc_len), t_loc_max, pos_offset, _ptr(rope_cache), int(bool(k_loc_rotated)),
+                                       float(softmax_scale), _ptr(out[0]), _ptr(out[1]), _aligned_ptr(ws), nbytes,
+                                       _stream(stream)))
+    return out
+
+
+def attend_merge(o_shares, lse2_shares, out=None, stream=None):
+    """Merge R shares: o_shares [R, ..., head_dim] fp32, lse2_shares [R, ...] fp32 -> bf16 [..., head_dim]."""
+    import torch
+
+    R, D = o_shares.shape[0], o_shares.shape[-1]
+    rows = lse2_shares[0].numel()
+    if out is None:
+        out = torch.empty(tuple(o_shares.shape[1:]), dtype=torch.bfloat16, device=o_shares.device)
+    _check(lib.msa_attend_merge(_ptr(o_shares), _ptr(lse2_shares), R, rows, D, _ptr(out), _stream(stream)))
     return out
 
 

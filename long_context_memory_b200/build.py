@@ -22,20 +22,36 @@ def needs_build() -> bool:
 
 
 def build(verbose: bool = False, ptxas_verbose: bool = False) -> str:
-    cmd = [NVCC, "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
-           "-rdc=true", "-shared", "-Xcompiler", "-fPIC", "-cudart", "static",
-           "-I", os.path.join(ROOT, "include"), "-o", LIB]
+    """Compile every source to an object in parallel (relocatable device code), then link libmsa.so."""
+    import concurrent.futures as cf
+    import tempfile
+
+    flags = [NVCC, "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-rdc=true",
+             "-Xcompiler", "-fPIC", "-I", os.path.join(ROOT, "include")]
     if ptxas_verbose:
-        cmd += ["-Xptxas", "-v"]
-    cmd += [os.path.join(CSRC, s) for s in SOURCES]
-    if verbose:
-        print(" ".join(cmd), flush=True)
-    r = subprocess.run(cmd, capture_output=True, text=True)
-    if r.returncode != 0:
-        sys.stderr.write(r.stdout + r.stderr)
-        raise RuntimeError("nvcc failed building libmsa.so")
-    if verbose or ptxas_verbose:
-        sys.stderr.write(r.stderr)
+        flags += ["-Xptxas", "-v"]
+    with tempfile.TemporaryDirectory(prefix="msa_build_") as tmp:
+        objs = [os.path.join(tmp, os.path.splitext(src)[0] + ".o") for src in SOURCES]
+        cmds = [flags + ["-c", os.path.join(CSRC, src), "-o", obj] for src, obj in zip(SOURCES, objs)]
+        if verbose:
+            for c in cmds:
+                print(" ".join(c), flush=True)
+        with cf.ThreadPoolExecutor(max_workers=len(cmds)) as ex:
+            results = list(ex.map(lambda c: subprocess.run(c, capture_output=True, text=True), cmds))
+        for r in results:
+            if r.returncode != 0:
+                sys.stderr.write(r.stdout + r.stderr)
+                raise RuntimeError("nvcc failed building libmsa.so")
+            if verbose or ptxas_verbose:
+                sys.stderr.write(r.stderr)
+        link = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-rdc=true", "-shared", "-Xcompiler", "-fPIC",
+                "-cudart", "static", "-o", LIB] + objs
+        if verbose:
+            print(" ".join(link), flush=True)
+        r = subprocess.run(link, capture_output=True, text=True)
+        if r.returncode != 0:
+            sys.stderr.write(r.stdout + r.stderr)
+            raise RuntimeError("nvcc failed linking libmsa.so")
     return LIB
 
 

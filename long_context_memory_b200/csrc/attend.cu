@@ -87,6 +87,8 @@ struct AttnParams {
   int chunk_part_base;  // partial slot of chunk split 0 (the local splits take slots 0 ..)
   int n_parts;       // partial slots per (query token, q head)
   int early;         // local-key items run before the predecessor kernel has finished
+  int doc_base;      // global id of chunk_off's first document (topk_idx holds global ids)
+  int foreign_ok;    // a selected document outside [doc_base, doc_base + n_docs) is another rank's: skipped
   int co_cap;        // chunk_off entries copied to shared memory (n_docs + 1), or 0 (read from L2)
   int tok_per_cta;   // MT: tokens per CTA, MT * G <= 16 mma rows
   int n_tgroups;     // ceil(M / MT)
@@ -225,12 +227,12 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
       int* seg_v = segs + hb * (2 * kMaxK + 2);  // [k + 1] virtual starts
       int* seg_c = seg_v + kMaxK + 2;            // [k] chunk starts
       for (int r = lane; r < (is_chunk ? k : 0); r += 32) {
-        const int doc = p.topk_idx[(size_t)b * k + r];
+        const int doc = p.topk_idx[(size_t)b * k + r] - p.doc_base;
         int c0 = 0, n = 0;
         if (doc >= 0 && doc < p.n_docs) {
           c0 = p.co_cap ? co_sm[doc] : __ldg(&p.chunk_off[doc]);
           n = (p.co_cap ? co_sm[doc + 1] : __ldg(&p.chunk_off[doc + 1])) - c0;
-        } else {
+        } else if (!p.foreign_ok) {
           raise_dev_error(kDevErrBadIndex);
         }
         seg_c[r] = c0;
@@ -588,7 +590,8 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
 template <int D, int SL>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restrict__ part_ml,
                                                            const float* __restrict__ part_o, int n_splits,
-                                                           __nv_bfloat16* __restrict__ out) {
+                                                           __nv_bfloat16* __restrict__ out, float* __restrict__ out_f32,
+                                                           float* __restrict__ out_lse2) {
   constexpr int W = D / (32 * SL);          // dims per lane
   constexpr int kHold = W == 1 ? 24 : 12;   // partial rows per lane loaded before the weights are known
   __shared__ float w_s[kMaxSplits];
@@ -668,8 +671,11 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
     float o = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) o += osum[w][dim];
-    out[qh * D + d0 + dim] = __float2bfloat16_rn(Ls > 0.f ? o / Ls : 0.f);
+    const float v = Ls > 0.f ? o / Ls : 0.f;
+    if (out_f32) out_f32[qh * D + d0 + dim] = v;  // a rank's share: fp32, merged across ranks later
+    else out[qh * D + d0 + dim] = __float2bfloat16_rn(v);
   }
+  if (out_lse2 && blockIdx.z == 0 && tid == 0) out_lse2[qh] = Ls > 0.f ? Mu + log2f(Ls) : -INFINITY;
 }
 
 int stages_that_fit(int n_kv, int n_q, int D, bool table, int mt, int co_cap) {
@@ -709,7 +715,9 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(__nv_bfloat16* __restric
 template <int D>
 __global__ void __launch_bounds__(256) attn_combine_warp_kernel(const float* __restrict__ part_ml,
                                                                 const float* __restrict__ part_o, int n_splits,
-                                                                int n_rows, __nv_bfloat16* __restrict__ out) {
+                                                                int n_rows, __nv_bfloat16* __restrict__ out,
+                                                                float* __restrict__ out_f32,
+                                                                float* __restrict__ out_lse2) {
   constexpr int W = D / 32;
   pdl_enter();
   const int lane = threadIdx.x & 31;
@@ -750,8 +758,46 @@ __global__ void __launch_bounds__(256) attn_combine_warp_kernel(const float* __r
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
   const float inv = l > 0.f ? 1.0f / l : 0.f;
+  if (out_f32) {  // a rank's share: fp32, merged across ranks later
 #pragma unroll
-  for (int e = 0; e < W; ++e) out[qh * D + lane * W + e] = __float2bfloat16_rn(acc[e] * inv);
+    for (int e = 0; e < W; ++e) out_f32[qh * D + lane * W + e] = acc[e] * inv;
+    if (lane == 0) out_lse2[qh] = l > 0.f ? Mu + log2f(l) : -INFINITY;
+  } else {
+#pragma unroll
+    for (int e = 0; e < W; ++e) out[qh * D + lane * W + e] = __float2bfloat16_rn(acc[e] * inv);
+  }
+}
+
+// merge of R shares of one attention (memory-parallel ranks): out = sum_r w_r o_r / sum_r w_r with
+// w_r = 2^(lse2_r - max_r lse2_r); one warp per (query token, q head), lane l holds dims l*W ..
+template <int D>
+__global__ void __launch_bounds__(256) attend_merge_kernel(const float* __restrict__ o_parts,
+                                                           const float* __restrict__ lse2_parts, int R, int n_rows,
+                                                           __nv_bfloat16* __restrict__ out) {
+  constexpr int W = D / 32;
+  pdl_enter();
+  const int lane = threadIdx.x & 31;
+  const size_t row = (size_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (row >= (size_t)n_rows) return;
+  float m = -INFINITY;
+  for (int r = lane; r < R; r += 32) m = fmaxf(m, lse2_parts[(size_t)r * n_rows + row]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float acc[W], wsum = 0.f;
+#pragma unroll
+  for (int e = 0; e < W; ++e) acc[e] = 0.f;
+  if (m != -INFINITY) {
+    for (int r = 0; r < R; ++r) {  // in rank order: the same result on every rank
+      const float w = exp2f(lse2_parts[(size_t)r * n_rows + row] - m);
+      wsum += w;
+      const float* src = o_parts + ((size_t)r * n_rows + row) * D + lane * W;
+#pragma unroll
+      for (int e = 0; e < W; ++e) acc[e] = fmaf(w, src[e], acc[e]);
+    }
+  }
+  const float inv = wsum > 0.f ? 1.0f / wsum : 0.f;
+#pragma unroll
+  for (int e = 0; e < W; ++e) out[row * D + lane * W + e] = __float2bfloat16_rn(acc[e] * inv);
 }
 
 // the decode step's new token into the rotated cache: CTA = one query; key rotated at
@@ -963,6 +1009,16 @@ msa_status gather_kv_launch(const msa_dims& d, const void* K_host, const void* V
   return MSA_OK;
 }
 
+msa_status attend_merge_launch(const float* o_parts, const float* lse2_parts, int R, int n_rows, int D, void* out,
+                               cudaStream_t s) {
+  TraceScope ts(kKAttnMerge, s);
+  const dim3 grid((unsigned)((n_rows + 7) / 8));
+  auto kern = D == 128 ? attend_merge_kernel<128> : attend_merge_kernel<64>;
+  MSA_CUDA_CHECK(launch_pdl(kern, grid, dim3(256), 0, s, o_parts, lse2_parts, R, n_rows,
+                            static_cast<__nv_bfloat16*>(out)));
+  return MSA_OK;
+}
+
 msa_status rope_cache_build(const msa_dims& d, int t_loc_max, int pos_offset, float2* tab, cudaStream_t s) {
   if (t_loc_max <= 0) return MSA_OK;
   const int D = d.head_dim;
@@ -1012,11 +1068,11 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
                          const void* V_loc, const void* k_new, const void* v_new, const int32_t* loc_len,
                          int t_loc_max, int pos_offset,
                          const void* rope_cache, int k_loc_rotated, float scale, int phase, int early, void* out,
-                         void* ws, cudaStream_t s) {
+                         void* ws, cudaStream_t s, const AttendShare* share) {
   AttendWs w;
   attend_workspace(d, B, M, k, t_loc_max, pos_offset, ws, &w);
   const int D = d.head_dim;
-  const bool local_keys = phase != 2;
+  const bool local_keys = phase != 2 && (!share || share->local_keys);
   const float2* tab = (k_loc_rotated || !local_keys) ? nullptr : static_cast<const float2*>(rope_cache);
   if (!tab && !k_loc_rotated && local_keys && t_loc_max > 0) {
     msa_status st = rope_cache_build(d, t_loc_max, pos_offset, w.rope_tab, s);
@@ -1044,10 +1100,14 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
   p.n_docs = n_docs;
   p.t_loc_max = t_loc_max;
   p.pos_offset = pos_offset;
-  p.n_loc_splits = phase == 2 ? 0 : w.n_split_local;
+  p.n_loc_splits = local_keys ? w.n_split_local : 0;
   p.n_chunk_splits = phase == 1 ? 0 : w.n_split_chunk;
-  p.chunk_part_base = w.n_split_local;
-  p.n_parts = w.n_parts;
+  // a share without the local keys uses the chunk splits' slots alone
+  const bool chunks_only = share && !share->local_keys;
+  p.chunk_part_base = chunks_only ? 0 : w.n_split_local;
+  p.n_parts = chunks_only ? w.n_split_chunk : w.n_parts;
+  p.doc_base = share ? share->doc_base : 0;
+  p.foreign_ok = share ? 1 : 0;
   // the local-key items may start before the predecessor finishes only if this call launches
   // nothing before them (no rotation table built here)
   p.early = early && phase != 2 && (k_loc_rotated || rope_cache || t_loc_max == 0);
@@ -1088,12 +1148,12 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
       dim3 grid(d.n_q, B * M, D / 32);
       auto kern = D == 128 ? attn_combine_kernel<128, 4> : attn_combine_kernel<64, 2>;
       MSA_CUDA_CHECK(launch_pdl(kern, grid, dim3(256), 0, s, (const float*)w.part_ml, (const float*)w.part_o,
-                                p.n_parts, o));
+                                p.n_parts, o, share ? share->o : nullptr, share ? share->lse2 : nullptr));
     } else {
       dim3 grid((unsigned)((rows + 7) / 8));
       auto kern = D == 128 ? attn_combine_warp_kernel<128> : attn_combine_warp_kernel<64>;
       MSA_CUDA_CHECK(launch_pdl(kern, grid, dim3(256), 0, s, (const float*)w.part_ml, (const float*)w.part_o,
-                                p.n_parts, (int)rows, o));
+                                p.n_parts, (int)rows, o, share ? share->o : nullptr, share ? share->lse2 : nullptr));
     }
   }
   return MSA_OK;

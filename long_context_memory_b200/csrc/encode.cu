@@ -13,7 +13,7 @@
 //                      chunks (2 x 64 token rows, each chunk loaded by its own TMA
 //                      box), N = 256 (or 128), accumulators in TMEM; the epilogue rotates
 //                      each row at its document-relative position and pools the
-//                      64 rows of each chunk -> K̄.  A pool warp sums the same H
+//                      64 rows of each chunk -> K̄.  Two pool warps sum the same H
 //                      tiles in shared memory (for one N tile of each chunk pair):
 //                      H̄ = chunk mean of H, stored as bf16 hi + lo terms [C, 2*hidden],
 //                      so H is read from HBM once
@@ -48,7 +48,7 @@ constexpr int kBM = 128, kBK = 64;
 constexpr int kEncStagesMax = 4;
 constexpr int kABytes = kBM * kBK * 2;  // 16 KB
 constexpr int kEncThreads = 192;        // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
-constexpr int kEncThreadsK = 224;       // mode K: + warp 6, the pool warp (chunk means of H)
+constexpr int kEncThreadsK = 256;       // mode K: + warps 6, 7, the pool warps (chunk means of H)
 
 __global__ void chunk_map_kernel(const int64_t* __restrict__ doc_off, const int32_t* __restrict__ chunk_off,
                                  int n_docs, int n_chunks, int64_t T, int64_t* __restrict__ tok0,
@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(MODE == 0 ? kEncThreadsK : kEncThreads, 1) gem
   if (threadIdx.x == 0) {
     for (int s = 0; s < kEncStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], MODE == kModeK ? 2 : 1);  // MMA commit (+ the pool warp in mode K)
+      mbar_init(&empty[s], MODE == kModeK ? 3 : 1);  // MMA commit (+ the two pool warps in mode K)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
@@ -244,42 +244,57 @@ __global__ void __launch_bounds__(MODE == 0 ? kEncThreadsK : kEncThreads, 1) gem
         mbar_drain_ring(drained, 1, 0, 1);
       }
     }
-  } else if (MODE == kModeK && warp == 6) {
-    // ------------- pool warp: chunk means of the H tiles the MMA reads -------------
-    // For the first N tile of each chunk pair, sum every 64-column block of the pair's two
-    // 64-row boxes over each chunk's own rows (in row order, fp32) and store the mean as bf16
-    // hi + lo terms; for the other N tiles only release the stage.  Lane l owns columns 2l, 2l+1.
+  } else if (MODE == kModeK && warp >= 6) {
+    // ------------- pool warps: chunk means of the H tiles the MMA reads -------------
+    // For the first N tile of each chunk pair, warp 6 (chunk 2m) and warp 7 (chunk 2m + 1) sum
+    // their chunk's 64-row box of every 64-column block over the chunk's own rows (fp32) and store
+    // the mean as bf16 hi + lo terms; for the other N tiles they only release the stage.  Lane l
+    // reads 16-byte unit u = l % 8 (columns 8u .. 8u + 7) of rows 4i + l / 8; the four row groups
+    // are then added across lanes, and lanes 0..7 store their unit.
+    const int box = warp - 6;
+    const int u = lane & 7, rg = lane >> 3;
     int it = 0;
     for (int tile = blockIdx.x; tile < total_tiles && !abort_flag; tile += gridDim.x) {
       const int m = tile / p.n_tiles, n = tile % p.n_tiles;
-      const int c0 = 2 * m, c1 = 2 * m + 1;
-      const int len0 = p.clen[c0];
-      const int len1 = c1 < p.n_chunks ? p.clen[c1] : 0;
+      const int c = 2 * m + box;
+      const int len = c < p.n_chunks ? p.clen[c] : 0;
       for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
         const int st = it % kEncStages;
         if (!warp_wait(&full[st], (it / kEncStages) & 1, &abort_flag)) break;
-        if (n == 0) {
-          const uint8_t* a_s = stages + st * kStageBytes;
+        if (n == 0 && len > 0) {
+          const uint8_t* bx = stages + st * kStageBytes + box * (kABytes / 2);
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int box = 0; box < 2; ++box) {
-            const int len = box ? len1 : len0;
-            if (len == 0) continue;
-            const uint8_t* bx = a_s + box * (kABytes / 2);
-            float s0 = 0.f, s1 = 0.f;
-            for (int r = 0; r < len; ++r) {  // 128-byte rows, 16-byte units swizzled by the row
-              const uint32_t w =
-                  *reinterpret_cast<const uint32_t*>(bx + r * 128 + ((((lane >> 2) ^ (r & 7))) << 4) + (lane & 3) * 4);
-              const float2 f = unpack_bf16x2(w);
-              s0 += f.x;
-              s1 += f.y;
+          for (int i = 0; i < 16; ++i) {
+            const int r = 4 * i + rg;  // 128-byte rows, 16-byte units swizzled by the row
+            if (r < len) {
+              const uint4 w = *reinterpret_cast<const uint4*>(bx + r * 128 + ((u ^ (r & 7)) << 4));
+              float2 f;
+              f = unpack_bf16x2(w.x); acc[0] += f.x; acc[1] += f.y;
+              f = unpack_bf16x2(w.y); acc[2] += f.x; acc[3] += f.y;
+              f = unpack_bf16x2(w.z); acc[4] += f.x; acc[5] += f.y;
+              f = unpack_bf16x2(w.w); acc[6] += f.x; acc[7] += f.y;
             }
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 8);
+            acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+          }
+          if (rg == 0) {
             const float inv = 1.0f / (float)len;
-            const float m0 = s0 * inv, m1 = s1 * inv;
-            const float h0 = __bfloat162float(__float2bfloat16_rn(m0));
-            const float h1 = __bfloat162float(__float2bfloat16_rn(m1));
-            __nv_bfloat16* dst = p.hbar + (size_t)(c0 + box) * 2 * p.hidden + kb * kBK + 2 * lane;
-            *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(h0, h1);
-            *reinterpret_cast<uint32_t*>(dst + p.hidden) = pack_bf16x2(m0 - h0, m1 - h1);
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float m0 = acc[2 * j] * inv, m1 = acc[2 * j + 1] * inv;
+              const float h0 = __bfloat162float(__float2bfloat16_rn(m0));
+              const float h1 = __bfloat162float(__float2bfloat16_rn(m1));
+              hi[j] = pack_bf16x2(h0, h1);
+              lo[j] = pack_bf16x2(m0 - h0, m1 - h1);
+            }
+            __nv_bfloat16* dst = p.hbar + (size_t)c * 2 * p.hidden + kb * kBK + 8 * u;
+            *reinterpret_cast<uint4*>(dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4*>(dst + p.hidden) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
           }
         }
         __syncwarp();

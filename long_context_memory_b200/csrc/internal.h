@@ -52,6 +52,7 @@ enum KernelId : int {
   kKAuxLoss,
   kKKvAppend,
   kKKrNorms,
+  kKAttnMerge,
   kKernelCount
 };
 
@@ -170,12 +171,23 @@ msa_status topk_merge_launch(const float* cand_score, const int32_t* cand_idx, i
 
 size_t attend_workspace(const msa_dims& d, int B, int M, int k, int t_loc_max, int pos_offset, void* ws,
                         struct AttendWs* out);
+// One rank's share of a memory-parallel attention: the selected documents it holds (global ids,
+// the others skipped), the local keys only where local_keys is set, and the share's normalised
+// fp32 output with its base-2 log-sum-exp instead of the bf16 result.
+struct AttendShare {
+  int doc_base;    // global id of the shard's first document
+  int local_keys;  // 1: this share also attends over the local keys
+  float* o;        // [B * M * n_q, head_dim] fp32 out
+  float* lse2;     // [B * M * n_q] fp32 out
+};
 msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const void* K_bar, const void* V_bar,
                          const int32_t* chunk_off, int n_docs, const int32_t* topk_idx, int k,
                          const void* K_loc, const void* V_loc, const void* k_new, const void* v_new,
                          const int32_t* loc_len, int t_loc_max,
                          int pos_offset, const void* rope_cache, int k_loc_rotated, float scale, int phase,
-                         int early, void* out, void* ws, cudaStream_t s);
+                         int early, void* out, void* ws, cudaStream_t s, const AttendShare* share = nullptr);
+msa_status attend_merge_launch(const float* o_parts, const float* lse2_parts, int R, int n_rows, int D, void* out,
+                               cudaStream_t s);
 msa_status gather_kv_launch(const msa_dims& d, const void* K_host, const void* V_host, const int32_t* chunk_off,
                             int n_docs, const int32_t* topk_idx, int B, int k, void* K_stage, void* V_stage,
                             int capacity_chunks, int32_t* stage_off, int32_t* stage_idx, int32_t* stage_src,

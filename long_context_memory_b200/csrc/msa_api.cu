@@ -219,7 +219,7 @@ namespace {
 const char* kKernelNames[kKernelCount] = {
     "router_query", "scan", "topk_slice", "topk_merge", "rope_table", "attn_split", "attn_combine",
     "enc_chunk_map", "enc_transpose_w", "enc_gemm_k", "enc_gemm_pooled", "rope_rows", "gather_plan", "gather_copy",
-    "chunk_off_extend", "aux_loss", "kv_append", "kr_norms"};
+    "chunk_off_extend", "aux_loss", "kv_append", "kr_norms", "attn_merge"};
 
 struct TraceState {
   std::mutex mu;
@@ -591,6 +591,65 @@ msa_status msa_gather_kv(const msa_dims* dims, const void* K_bar_host, const voi
   return gather_kv_launch(*dims, dev_ptr[0], dev_ptr[1], chunk_off, n_docs, topk_idx, B, k, K_stage, V_stage,
                           capacity_chunks, stage_chunk_off, stage_topk_idx, static_cast<int32_t*>(ws),
                           static_cast<cudaStream_t>(stream));
+}
+
+msa_status msa_sparse_attend_share(const msa_dims* dims, const void* q, int32_t B, int32_t q_tokens, const void* K_bar,
+                                   const void* V_bar, const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks,
+                                   int32_t doc_base, const int32_t* topk_idx, int32_t k, int32_t local_keys,
+                                   const void* K_loc, const void* V_loc, const int32_t* loc_len, int32_t t_loc_max,
+                                   int32_t pos_offset, const void* rope_cache, int32_t k_loc_rotated,
+                                   float softmax_scale, float* o_share, float* lse2_share, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  msa_status st = check_dims(dims, true, false);
+  if (st != MSA_OK) return st;
+  if (B < 1) return fail(MSA_ERR_INVALID_ARG, "B must be >= 1 (got %d)", B);
+  if (q_tokens < 1 || (int64_t)B * q_tokens > 65535)
+    return fail(MSA_ERR_INVALID_ARG, "q_tokens must be >= 1 with B * q_tokens <= 65535 (got %d, B %d)", q_tokens, B);
+  if (n_docs < 1 || n_chunks < n_docs)
+    return fail(MSA_ERR_INVALID_ARG, "need 1 <= n_docs <= n_chunks (got %d, %d)", n_docs, n_chunks);
+  if (doc_base < 0) return fail(MSA_ERR_INVALID_ARG, "doc_base must be >= 0 (got %d)", doc_base);
+  if (k < 1 || k > 256) return fail(MSA_ERR_INVALID_ARG, "k must be in [1, 256] (got %d)", k);
+  if (local_keys != 0 && local_keys != 1) return fail(MSA_ERR_INVALID_ARG, "local_keys must be 0 or 1");
+  if (t_loc_max < 0) return fail(MSA_ERR_INVALID_ARG, "t_loc_max must be >= 0");
+  if (pos_offset < 0 || (int64_t)pos_offset + t_loc_max > (1 << 24))
+    return fail(MSA_ERR_INVALID_ARG, "positions must lie in [0, 2^24)");
+  if (!(softmax_scale >= 0.f) || !std::isfinite(softmax_scale))
+    return fail(MSA_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+  CHECK_PTR(q);
+  CHECK_PTR(K_bar);
+  CHECK_PTR(V_bar);
+  CHECK_PTR(chunk_off);
+  CHECK_PTR(topk_idx);
+  CHECK_PTR(loc_len);
+  CHECK_PTR(o_share);
+  CHECK_PTR(lse2_share);
+  if (local_keys && t_loc_max > 0) {
+    CHECK_PTR(K_loc);
+    CHECK_PTR(V_loc);
+  }
+  CHECK_OPT_PTR(rope_cache);
+  const size_t need = attend_workspace(*dims, B, q_tokens, k, t_loc_max, pos_offset, nullptr, nullptr);
+  if (ws_bytes < need) return fail(MSA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
+  if (need && (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)))
+    return fail(MSA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
+  if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
+  AttendShare share{doc_base, local_keys, o_share, lse2_share};
+  return attend_launch(*dims, q, B, q_tokens, K_bar, V_bar, chunk_off, n_docs, topk_idx, k, K_loc, V_loc, nullptr,
+                       nullptr, loc_len, t_loc_max, pos_offset, rope_cache, k_loc_rotated, softmax_scale, 0, 0, nullptr,
+                       ws, static_cast<cudaStream_t>(stream), &share);
+}
+
+msa_status msa_attend_merge(const float* o_shares, const float* lse2_shares, int32_t R, int32_t rows,
+                            int32_t head_dim, void* out, void* stream) {
+  if (R < 1 || R > 4096) return fail(MSA_ERR_INVALID_ARG, "R must be in [1, 4096] (got %d)", R);
+  if (rows < 1) return fail(MSA_ERR_INVALID_ARG, "rows must be >= 1 (got %d)", rows);
+  if (head_dim != 64 && head_dim != 128)
+    return fail(MSA_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", head_dim);
+  CHECK_PTR(o_shares);
+  CHECK_PTR(lse2_shares);
+  CHECK_PTR(out);
+  if (fault_injected()) return fail(MSA_ERR_CUDA, "injected fault (MSA_FAULT=launch)");
+  return attend_merge_launch(o_shares, lse2_shares, R, rows, head_dim, out, static_cast<cudaStream_t>(stream));
 }
 
 // the device address of pinned host memory, or an error when it is not pinned and device-mapped

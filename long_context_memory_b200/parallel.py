@@ -10,6 +10,14 @@ all-gather of the B x k (score, global document id) candidates, a few KB,
 followed by the exact merge of ``msa_topk_merge`` on the device; every rank
 ends with the same top-k, in the same order as routing the unsharded memory.
 
+The attention follows the same split: every rank attends over the selected
+documents it holds (msa_sparse_attend_share; the local keys on one rank), the
+ranks all-gather their shares, each the normalised fp32 output and its base-2
+log-sum-exp per (query token, head), and msa_attend_merge weighs them into the
+softmax over the whole context, in rank order, so every rank ends with the same
+output.  Per step that exchange is B x n_q x (head_dim + 1) fp32 per rank (16.5 KB
+for one query of 32 heads of 128).
+
 One process per GPU; the collective runs on the default process group (NCCL on
 GPUs, gloo in the CPU tests).
 """
@@ -90,13 +98,60 @@ def exchange_topk(local_idx, local_score, doc_base: int, k: int, group=None,
     return merge(cand_s, cand_i, k)
 
 
-def route_topk_sharded(dims, Hq, W_QR, KR_local, shard: Shard, k: int, group=None):
-    """This rank's routing over its shard, then the exchange; returns (topk_idx, topk_score)."""
+def route_topk_sharded(dims, Hq, W_QR, KR_local, shard: Shard, k: int, group=None, route: Optional[Callable] = None,
+                       merge: Optional[Callable] = None):
+    """This rank's routing over its shard, then the exchange; returns (topk_idx, topk_score).
+
+    ``route(dims, Hq, W_QR, KR_local, chunk_off, k)`` -> (idx, score, ...) defaults to msa_route_topk
+    and ``merge`` to msa_topk_merge (both replaceable so that the protocol runs on CPU ranks)."""
     import torch
 
-    from . import route_topk
+    if route is None:
+        from . import route_topk as route
 
     chunk_off = torch.from_numpy(shard.chunk_off).to(KR_local.device)
     kl = min(k, shard.n_docs)
-    idx, sc, _ = route_topk(dims, Hq, W_QR, KR_local, chunk_off, kl)
-    return exchange_topk(idx, sc, shard.doc_lo, k, group=group)
+    idx, sc = route(dims, Hq, W_QR, KR_local, chunk_off, kl)[:2]
+    return exchange_topk(idx, sc, shard.doc_lo, k, group=group, merge=merge)
+
+
+def exchange_attention(o_share, lse2_share, group=None, merge: Optional[Callable] = None):
+    """All-gather every rank's attention share and merge them (rank order).
+
+    o_share [..., head_dim] fp32, lse2_share [...] fp32 (msa_sparse_attend_share's outputs);
+    ``merge(o_shares [R, ...], lse2_shares [R, ...])`` defaults to the device merge."""
+    import torch
+    import torch.distributed as dist
+
+    world = dist.get_world_size(group)
+    all_o = [torch.empty_like(o_share) for _ in range(world)]
+    all_l = [torch.empty_like(lse2_share) for _ in range(world)]
+    dist.all_gather(all_o, o_share.contiguous(), group=group)
+    dist.all_gather(all_l, lse2_share.contiguous(), group=group)
+    o = torch.stack(all_o).contiguous()
+    l = torch.stack(all_l).contiguous()
+    if merge is None:
+        from . import attend_merge
+
+        return attend_merge(o, l)
+    return merge(o, l)
+
+
+def attend_sharded(dims, q, K_bar_local, V_bar_local, shard: Shard, topk_idx, K_loc, V_loc, loc_len, pos_offset: int,
+                   local_rank: int = 0, k_loc_rotated: bool = False, group=None, share: Optional[Callable] = None,
+                   merge: Optional[Callable] = None):
+    """This rank's share of the attention over the global top-k (global ids), then the exchange.
+
+    The local keys belong to rank ``local_rank``; every rank passes loc_len (it places the query).
+    ``share`` (same arguments as msa_sparse_attend_share's binding) and ``merge`` default to the
+    device calls."""
+    import torch
+
+    if share is None:
+        from . import sparse_attend_share as share
+
+    chunk_off = torch.from_numpy(shard.chunk_off).to(q.device)
+    t_loc_max = K_loc.shape[1] if K_loc is not None else 0
+    o, l = share(dims, q, K_bar_local, V_bar_local, chunk_off, shard.doc_lo, topk_idx, shard.rank == local_rank, K_loc,
+                 V_loc, loc_len, t_loc_max, pos_offset, k_loc_rotated=k_loc_rotated)
+    return exchange_attention(o, l, group=group, merge=merge)

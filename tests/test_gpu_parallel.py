@@ -61,3 +61,71 @@ def test_merge_ties_prefer_lower_global_id(cuda_device):
     idx, val = msa.topk_merge(sc, ids, 4)
     assert idx.cpu().tolist() == [[12, 40, 3, 7]]
     assert val.cpu().tolist()[0] == pytest.approx([0.9, 0.9, 0.5, 0.5])
+
+
+@pytest.mark.parametrize("world,B,M,k", [(2, 1, 1, 16), (3, 3, 1, 8), (8, 2, 1, 4), (2, 2, 3, 8)])
+def test_sharded_attention_shares_merge_to_whole_memory(cuda_device, world, B, M, k):
+    # every shard attends over the selected documents it holds (global ids; the local keys on
+    # shard 0 only), msa_attend_merge weighs the shares: the result equals msa_sparse_attend over
+    # the unsharded memory and the oracle.  With world 8 and k 4 some shards hold no selected
+    # document and no local key (an empty share, log-sum-exp -inf).
+    import torch
+
+    import long_context_memory_b200 as msa
+
+    rng = np.random.default_rng(300 + world + B + M)
+    dims = W.Dims(hidden=256, n_q=32, n_kv=8, head_dim=128, n_r=4, d_r=64, rope_base=1e6)
+    lens = rng.integers(1, 2000, size=60)
+    co, C = msa.chunk_offsets(W.offsets_from_lengths(lens))
+    t_loc, dev = 40, cuda_device
+    Kb = W.normal_bf16(rng, (C, 8, 128))
+    Vb = W.normal_bf16(rng, (C, 8, 128))
+    q = W.normal_bf16(rng, (B, M, 32, 128) if M > 1 else (B, 32, 128))
+    Kl = W.normal_bf16(rng, (B, t_loc, 8, 128))
+    Vl = W.normal_bf16(rng, (B, t_loc, 8, 128))
+    loc_len = rng.integers(M, t_loc + 1, size=B).astype(np.int32)
+    sel = np.stack([rng.permutation(len(lens))[:k] for _ in range(B)]).astype(np.int32)
+    t = lambda a: W.to_torch(np.ascontiguousarray(a)).to(dev)
+    topk, ll = torch.from_numpy(sel).to(dev), torch.from_numpy(loc_len).to(dev)
+    whole = msa.sparse_attend(dims, t(q), t(Kb), t(Vb), torch.from_numpy(co).to(dev), topk, t(Kl), t(Vl), ll, k)
+    os_, ls_ = [], []
+    for r in range(world):
+        sh = P.shard_memory(co, world, r)
+        rows = slice(sh.chunk_lo, sh.chunk_hi)
+        o, l = msa.sparse_attend_share(dims, t(q), t(Kb[rows]), t(Vb[rows]), torch.from_numpy(sh.chunk_off).to(dev),
+                                       sh.doc_lo, topk, r == 0, t(Kl) if r == 0 else None,
+                                       t(Vl) if r == 0 else None, ll, t_loc, k)
+        os_.append(o)
+        ls_.append(l)
+    out = msa.attend_merge(torch.stack(os_).contiguous(), torch.stack(ls_).contiguous())
+    torch.cuda.synchronize()
+    assert msa.check_device_errors() == 0
+    assert out.shape == whole.shape
+    g, w = out.float().cpu().numpy(), whole.float().cpu().numpy()
+    assert np.max(np.abs(g - w)) <= 2 ** -7 * np.max(np.abs(w)) + 1e-3, np.max(np.abs(g - w))
+    if world == 8:  # some share saw no key at all
+        assert any(bool(torch.isinf(l).any()) for l in ls_)
+    from helpers import check_attention
+
+    co_o, *_ = O.chunk_layout(W.offsets_from_lengths(lens))
+    if M == 1:
+        ref = O.sparse_attend(q, Kb, Vb, co_o, sel, Kl, Vl, loc_len, k, 1e6)
+    else:
+        ref = O.sparse_attend_tokens(q, Kb, Vb, co_o, sel, Kl, Vl, loc_len, k, 1e6)
+    check_attention(g, ref, where=f"world={world}")
+
+
+def test_attend_merge_weights_by_log_sum_exp(cuda_device):
+    # two shares of one row: lse2 0 and 1 -> weights 1/3 and 2/3; an empty share (-inf) counts 0
+    import torch
+
+    import long_context_memory_b200 as msa
+
+    o = torch.zeros((3, 1, 64), dtype=torch.float32, device=cuda_device)
+    o[0] += 1.0
+    o[1] += 4.0
+    o[2] += 100.0
+    l = torch.tensor([[0.0], [1.0], [float("-inf")]], device=cuda_device)
+    out = msa.attend_merge(o, l)
+    torch.cuda.synchronize()
+    assert torch.allclose(out.float(), torch.full((1, 64), 3.0, device=cuda_device), atol=1e-2)

@@ -6,6 +6,7 @@ an all-gather, and the merged top-k must equal the oracle's top-k over the
 whole memory, on every rank.  The device merge (msa_topk_merge) and the
 per-shard GPU routing are covered by test_gpu_parallel.py.
 """
+import math
 import os
 import socket
 
@@ -151,3 +152,134 @@ def test_three_ranks_with_shards_smaller_than_k(k):
         gi, gs, _ = ret[rank]
         assert np.array_equal(gi, idx), (rank, gi, idx)
         assert np.allclose(gs, val, atol=1e-6)
+
+
+# ----------------------------------------------------------------------------
+# the composed functions on CPU ranks: route_topk_sharded, then attend_sharded
+# ----------------------------------------------------------------------------
+DIMS_CPU = W.Dims(hidden=128, n_q=4, n_kv=2, head_dim=64, n_r=4, d_r=64, rope_base=1e4)
+
+
+def _bits(t):
+    """bf16 torch tensor -> uint16 bit patterns (numpy)."""
+    import torch
+
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def _oracle_route(dims, Hq, W_QR, KR_local, chunk_off, k):
+    """Stands in for msa_route_topk on a CPU rank (the oracle's scores of the shard's documents)."""
+    import torch
+
+    qr = O.bf16_to_f64(_bits(Hq)).reshape(-1, dims.n_r, dims.d_r)
+    s = O.doc_scores(O.chunk_scores(qr, _bits(KR_local)), chunk_off.numpy())
+    idx = np.stack([O.topk(s[b], k)[0] for b in range(s.shape[0])]).astype(np.int32)
+    sc = np.stack([s[b][idx[b]] for b in range(s.shape[0])]).astype(np.float32)
+    return torch.from_numpy(idx), torch.from_numpy(sc)
+
+
+def _oracle_share(dims, q, K_bar, V_bar, chunk_off, doc_base, topk_idx, local_keys, K_loc, V_loc, loc_len, t_loc_max,
+                  pos_offset, k_loc_rotated=False):
+    """Stands in for msa_sparse_attend_share on a CPU rank: the softmax over the selected documents this
+    shard holds (and the local keys where local_keys), its normalised output and base-2 log-sum-exp."""
+    import torch
+
+    qf = O.bf16_to_f64(_bits(q))
+    B, n_q, D = qf.shape
+    Kb, Vb = O.bf16_to_f64(_bits(K_bar)), O.bf16_to_f64(_bits(V_bar))
+    co = chunk_off.numpy()
+    G = n_q // dims.n_kv
+    o = np.zeros((B, n_q, D))
+    l2 = np.full((B, n_q), -np.inf)
+    for b in range(B):
+        L = int(loc_len[b])
+        ks, vs = [], []
+        for doc in topk_idx[b].tolist():
+            i = doc - doc_base
+            if 0 <= i < len(co) - 1:
+                ks.append(Kb[co[i]:co[i + 1]])
+                vs.append(Vb[co[i]:co[i + 1]])
+        if local_keys and L > 0:
+            ks.append(O.rope(O.bf16_to_f64(_bits(K_loc[b, :L].contiguous())), (pos_offset + np.arange(L))[:, None], dims.rope_base))
+            vs.append(O.bf16_to_f64(_bits(V_loc[b, :L].contiguous())))
+        if not ks:
+            continue
+        K, V = np.concatenate(ks), np.concatenate(vs)
+        qr = O.rope(qf[b], pos_offset + L - 1, dims.rope_base)
+        for g in range(n_q):
+            logits = (K[:, g // G] @ qr[g]) / math.sqrt(D)
+            m = logits.max()
+            p = np.exp(logits - m)
+            o[b, g] = (p[:, None] * V[:, g // G]).sum(0) / p.sum()
+            l2[b, g] = (m + math.log(p.sum())) / math.log(2.0)
+    return torch.from_numpy(o), torch.from_numpy(l2)
+
+
+def _numpy_attend_merge(o_sh, l_sh):
+    o, l = o_sh.numpy(), l_sh.numpy()
+    m = l.max(axis=0)
+    w = np.where(np.isfinite(l), np.exp2(l - np.where(np.isfinite(m), m, 0.0)), 0.0)
+    import torch
+
+    return torch.from_numpy((w[..., None] * o).sum(0) / np.maximum(w.sum(0), 1e-300)[..., None])
+
+
+def _composed_rank(rank, world, port, ret):
+    import torch
+    import torch.distributed as dist
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        c = _composed_case()
+        d, co, k = DIMS_CPU, c["co"], c["k"]
+        sh = P.shard_memory(co, world, rank)
+        rows = slice(sh.chunk_lo, sh.chunk_hi)
+        t = W.to_torch
+        idx, sc = P.route_topk_sharded(d, t(c["QR"]), None, t(c["KR"][rows]), sh, k, route=_oracle_route,
+                                       merge=oracle_merge)
+        out = P.attend_sharded(d, t(c["q"]), t(c["K_bar"][rows]), t(c["V_bar"][rows]), sh, idx, t(c["K_loc"]),
+                               t(c["V_loc"]), c["loc_len"], k, share=_oracle_share, merge=_numpy_attend_merge)
+        ret[rank] = (idx.numpy(), sc.numpy(), out.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def _composed_case():
+    d = DIMS_CPU
+    rng = np.random.default_rng(404)
+    lens = rng.integers(1, 400, size=40)
+    co, *_ = O.chunk_layout(W.offsets_from_lengths(lens))
+    C, B, t_loc = int(co[-1]), 3, 20
+    return dict(co=co, k=5, KR=W.normal_bf16(rng, (C, d.n_r, d.d_r)), QR=W.normal_bf16(rng, (B, d.n_r * d.d_r)),
+                K_bar=W.normal_bf16(rng, (C, d.n_kv, d.head_dim)), V_bar=W.normal_bf16(rng, (C, d.n_kv, d.head_dim)),
+                q=W.normal_bf16(rng, (B, d.n_q, d.head_dim)), K_loc=W.normal_bf16(rng, (B, t_loc, d.n_kv, d.head_dim)),
+                V_loc=W.normal_bf16(rng, (B, t_loc, d.n_kv, d.head_dim)), loc_len=np.array([20, 7, 1]))
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_composed_route_and_attend_on_gloo_ranks(world):
+    # route_topk_sharded then attend_sharded on every rank: the global top-k and the merged attention
+    # (the local keys on rank 0 only) equal the oracle over the unsharded memory, on every rank
+    import torch.multiprocessing as mp
+
+    ctx = mp.get_context("spawn")
+    ret = ctx.Manager().dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_composed_rank, args=(r, world, port, ret)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+        assert p.exitcode == 0, f"rank exited with {p.exitcode}"
+    c, d = _composed_case(), DIMS_CPU
+    B = c["q"].shape[0]
+    _, idx, val = O.route_topk(O.bf16_to_f64(c["QR"]).reshape(B, d.n_r, d.d_r), c["KR"], c["co"], c["k"])
+    ref = O.sparse_attend(c["q"], c["K_bar"], c["V_bar"], c["co"], idx, c["K_loc"], c["V_loc"], c["loc_len"], c["k"],
+                          d.rope_base)
+    for rank in range(world):
+        gi, gs, out = ret[rank]
+        assert np.array_equal(gi, idx), rank
+        assert np.allclose(gs, val, atol=1e-6)
+        assert np.max(np.abs(out - ref)) < 1e-10, np.max(np.abs(out - ref))
