@@ -908,11 +908,14 @@ __global__ void __launch_bounds__(1024) gather_plan_kernel(const int32_t* __rest
 // what a ~55 GB/s host link needs in flight at a few microseconds of latency).  The grid is small
 // (kGatherCtas CTAs of 256 threads, at most 64 registers a thread): it runs beside the routing
 // scan or the attention of another layer without taking an SM from them.
-constexpr int kGatherThreads = 256;
+#ifndef MSA_GATHER_THREADS
+#define MSA_GATHER_THREADS 256
+#endif
 #ifndef MSA_GATHER_CTAS
 #define MSA_GATHER_CTAS 16
 #endif
-constexpr int kGatherCtas = MSA_GATHER_CTAS;
+constexpr int kGatherThreads = MSA_GATHER_THREADS;
+constexpr int kGatherCtas = MSA_GATHER_CTAS;  // 0: one CTA per SM
 __global__ void __launch_bounds__(kGatherThreads, 4) gather_copy_kernel(const uint4* __restrict__ K_host,
                                                                         const uint4* __restrict__ V_host,
                                                                         const int32_t* __restrict__ stage_off,
@@ -1001,7 +1004,8 @@ msa_status gather_kv_launch(const msa_dims& d, const void* K_host, const void* V
   {
     TraceScope ts(kKGatherCopy, s);
     const int row_vec = d.n_kv * d.head_dim * 2 / 16;
-    MSA_CUDA_CHECK(launch_pdl(gather_copy_kernel, dim3(kGatherCtas), dim3(kGatherThreads), 0, s,
+    MSA_CUDA_CHECK(launch_pdl(gather_copy_kernel, dim3(kGatherCtas > 0 ? kGatherCtas : sm_count()),
+                              dim3(kGatherThreads), 0, s,
                               static_cast<const uint4*>(K_host), static_cast<const uint4*>(V_host),
                               (const int32_t*)stage_off, (const int32_t*)stage_src, n_sel, row_vec,
                               static_cast<uint4*>(K_stage), static_cast<uint4*>(V_stage)));

@@ -14,7 +14,7 @@
 //                      box), N = 256 (or 128), accumulators in TMEM; the epilogue rotates
 //                      each row at its document-relative position and pools the
 //                      64 rows of each chunk -> K̄.  Two pool warps sum the same H
-//                      tiles in shared memory (for one N tile of each chunk pair):
+//                      tiles in shared memory (each block once over the chunk pair's N tiles):
 //                      H̄ = chunk mean of H, stored as bf16 hi + lo terms [C, 2*hidden],
 //                      so H is read from HBM once
 //   gemm_kernel<POOL>  (H̄_hi | H̄_lo) [W_V | W^KR] over K = 2*hidden -> V̄, K̄^R.
@@ -246,11 +246,13 @@ __global__ void __launch_bounds__(MODE == 0 ? kEncThreadsK : kEncThreads, 1) gem
     }
   } else if (MODE == kModeK && warp >= 6) {
     // ------------- pool warps: chunk means of the H tiles the MMA reads -------------
-    // For the first N tile of each chunk pair, warp 6 (chunk 2m) and warp 7 (chunk 2m + 1) sum
-    // their chunk's 64-row box of every 64-column block over the chunk's own rows (fp32) and store
-    // the mean as bf16 hi + lo terms; for the other N tiles they only release the stage.  Lane l
-    // reads 16-byte unit u = l % 8 (columns 8u .. 8u + 7) of rows 4i + l / 8; the four row groups
-    // are then added across lanes, and lanes 0..7 store their unit.
+    // Every N tile of a chunk pair loads the same H blocks; the CTA of N tile n pools the blocks
+    // kb with kb % n_tiles == n (so each block is pooled once, and every CTA gets an equal share):
+    // warp 6 (chunk 2m) and warp 7 (chunk 2m + 1) sum their chunk's 64-row box of the block over
+    // the chunk's own rows (fp32) and store the mean as bf16 hi + lo terms; for the other blocks
+    // they only release the stage.  Lane l reads 16-byte unit u = l % 8 (columns 8u .. 8u + 7) of
+    // rows 4i + l / 8; the four row groups are then added across lanes, and lanes 0..7 store their
+    // unit.
     const int box = warp - 6;
     const int u = lane & 7, rg = lane >> 3;
     int it = 0;
@@ -261,7 +263,7 @@ __global__ void __launch_bounds__(MODE == 0 ? kEncThreadsK : kEncThreads, 1) gem
       for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
         const int st = it % kEncStages;
         if (!warp_wait(&full[st], (it / kEncStages) & 1, &abort_flag)) break;
-        if (n == 0 && len > 0) {
+        if (kb % p.n_tiles == n && len > 0) {
           const uint8_t* bx = stages + st * kStageBytes + box * (kABytes / 2);
           float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll

@@ -14,6 +14,8 @@ Cases
              (route cases: --kr-layout head stores K̄^R head-major [n_r, C, d_r])
   attend1m   sparse attention, 1M-token memory, B = 1, 4K local tokens (rotated key cache)
   attend16m  sparse attention, 16M-token memory, B = 32, 8K local tokens (rotated key cache)
+  tiered     one msa_tiered_decode call over --layers layer instances (default 2) of a
+             --tokens-token memory (default 100M): routing, host-tier gather, attention; B = --batch
   encode     offline encoding of --tokens tokens (default 1M), hidden 2560
   aux        router training loss L_aux + gradients: P = 4096 positives x (1 + 63 negatives),
              8 router heads x 128 (--batch to change P)
@@ -357,7 +359,7 @@ def main():
 
     ap = argparse.ArgumentParser()
     ap.add_argument("--case", required=True,
-                    choices=["route1m", "route16m", "route100m", "attend1m", "attend16m", "encode", "aux"])
+                    choices=["route1m", "route16m", "route100m", "attend1m", "attend16m", "tiered", "encode", "aux"])
     ap.add_argument("--launches", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=2)
     ap.add_argument("--batch", type=int, default=None)
@@ -365,6 +367,7 @@ def main():
                     "their own size unless given)")
     ap.add_argument("--kr-layout", choices=["chunk", "head"], default="chunk")
     ap.add_argument("--norms", action="store_true", help="route cases: pass precomputed key norms")
+    ap.add_argument("--layers", type=int, default=2, help="tiered case: layer instances per call")
     a = ap.parse_args()
     dev = torch.device("cuda:0")
     seed = W.BASE_SEED + 7
@@ -381,9 +384,15 @@ def main():
         case = AttendCase(16_000_000, a.batch or 32, 2048, 8192, seed, dev)
     elif a.case == "aux":
         case = AuxCase(a.batch or 4096, 63, seed, dev)
+    elif a.case == "tiered":
+        case = TieredCase(a.tokens or 100_000_000, 4096, 8192, W.BASE_SEED + 4, dev, a.layers, 1, B=a.batch or 1)
     else:
         case = EncodeCase(a.tokens or 1_000_000, seed, dev)
     s = torch.cuda.Stream()
+    if a.case == "tiered":  # the gather on its own stream, as a decode loop runs it
+        cs = torch.cuda.Stream()
+        tcase = case
+        case = type("Run", (), {"run": staticmethod(lambda: tcase.run(s, cs))})
     with torch.cuda.stream(s):
         for _ in range(a.warmup):
             case.run()

@@ -107,11 +107,6 @@ def offsets_from_lengths(lens: np.ndarray) -> np.ndarray:
     return off
 
 
-def n_chunks_of(lens: np.ndarray, chunk: int = 64) -> np.ndarray:
-    """Chunk counts per document (ceil(L/P)); layout bookkeeping for generators."""
-    return (lens + chunk - 1) // chunk
-
-
 # ----------------------------------------------------------------------------
 # planting helpers (input construction geometry)
 # ----------------------------------------------------------------------------
@@ -190,11 +185,15 @@ def tiny_config(seed: int = BASE_SEED, n_docs: int = 64, lo: int = 256, hi: int 
 # ----------------------------------------------------------------------------
 # pooled memory (route + attend), configs from 1M to 100M tokens
 # ----------------------------------------------------------------------------
-def memory_config(T: int, B: int, seed: int, median: int = 2048, dims: Dims = QWEN3_4B_DIMS,
+def memory_config(T: int, B: int, seed: int, layout, median: int = 2048, dims: Dims = QWEN3_4B_DIMS,
                   k: int = 16, t_loc: int = 4096, n_planted: int = 16,
                   planted_cos: Optional[np.ndarray] = None, with_kv: bool = True,
                   name: str = "memory") -> dict:
     """Pooled memory given directly: K̄, V̄, K̄^R ~ N(0,1) bf16 [C, heads, dim].
+
+    ``layout(doc_off) -> chunk_off`` is the caller's chunk layout of the drawn documents (the
+    generator itself computes none of it): it says how many pooled rows to draw and which rows
+    belong to a planted document.
 
     Per query b, ``n_planted`` distinct documents get one random chunk whose
     router key has per-head cosine ``planted_cos[p]`` with the query's planted
@@ -206,9 +205,8 @@ def memory_config(T: int, B: int, seed: int, median: int = 2048, dims: Dims = QW
     rng = np.random.default_rng(seed)
     lens = doc_lengths_lognormal(rng, T, median)
     doc_off = offsets_from_lengths(lens)
-    nch = n_chunks_of(lens, dims.chunk)
-    chunk_off = np.zeros(len(lens) + 1, dtype=np.int64)
-    chunk_off[1:] = np.cumsum(nch)
+    chunk_off = np.asarray(layout(doc_off), dtype=np.int64)
+    nch = chunk_off[1:] - chunk_off[:-1]
     C = int(chunk_off[-1])
     N = len(lens)
     KR = normal_bf16(rng, (C, dims.n_r, dims.d_r))
@@ -248,13 +246,13 @@ def memory_config(T: int, B: int, seed: int, median: int = 2048, dims: Dims = QW
     return out
 
 
-def mem1m_config(seed: int = BASE_SEED + 1, T: int = 1_000_000, **kw) -> dict:
+def mem1m_config(layout, seed: int = BASE_SEED + 1, T: int = 1_000_000, **kw) -> dict:
     """1M-token memory, batch 1, 4K local KV, 16 planted docs at cosine 0.9."""
     kw.setdefault("t_loc", 4096)
-    return memory_config(T=T, B=1, seed=seed, median=2048, name="mem1m", **kw)
+    return memory_config(T=T, B=1, seed=seed, layout=layout, median=2048, name="mem1m", **kw)
 
 
-def mem16m_config(seed: int = BASE_SEED + 2, T: int = 16_000_000, B: int = 32, **kw) -> dict:
+def mem16m_config(layout, seed: int = BASE_SEED + 2, T: int = 16_000_000, B: int = 32, **kw) -> dict:
     """16M-token memory, 32 queries routed together, 8K local KV per query.
 
     Planted per-head cosines are 0.21 + 0.01 p (p = 0..15): the expected
@@ -263,7 +261,7 @@ def mem16m_config(seed: int = BASE_SEED + 2, T: int = 16_000_000, B: int = 32, *
     0.05 above the background and consecutive planted docs differ by 0.01.
     """
     kw.setdefault("t_loc", 8192)
-    return memory_config(T=T, B=B, seed=seed, median=2048,
+    return memory_config(T=T, B=B, seed=seed, layout=layout, median=2048,
                          planted_cos=0.21 + 0.01 * np.arange(16), name="mem16m", **kw)
 
 

@@ -8,6 +8,12 @@ import oracle as O
 from long_context_memory_b200 import workloads as W
 from helpers import bf16_of, check_attention
 
+
+def LAYOUT(doc_off):
+    """The oracle's chunk layout (the generator takes the layout from its caller)."""
+    return O.chunk_layout(doc_off)[0]
+
+
 pytestmark = pytest.mark.gpu
 
 
@@ -116,7 +122,7 @@ def test_attend_tiny_config_full_pipeline(msa, cuda_device):
 
 
 def test_attend_mem1m_full_size(msa, cuda_device):
-    m = W.mem1m_config()
+    m = W.mem1m_config(LAYOUT)
     d = m["dims"]
     co, *_ = O.chunk_layout(m["doc_off"])
     case = dict(doc_off=m["doc_off"], chunk_off=co, q=m["q"], K_bar=m["K_bar"], V_bar=m["V_bar"], K_loc=m["K_loc"],
@@ -126,7 +132,7 @@ def test_attend_mem1m_full_size(msa, cuda_device):
 
 
 def test_attend_mem16m_batch32_sampled(msa, cuda_device):
-    m = W.mem16m_config()
+    m = W.mem16m_config(LAYOUT)
     d = m["dims"]
     co, *_ = O.chunk_layout(m["doc_off"])
     case = dict(doc_off=m["doc_off"], chunk_off=co, q=m["q"], K_bar=m["K_bar"], V_bar=m["V_bar"], K_loc=m["K_loc"],
@@ -188,7 +194,7 @@ def test_attend_rotated_cache_mode(msa, cuda_device, D, n_q, n_kv):
 def test_attend_rotated_cache_mem16m_sampled(msa, cuda_device):
     import torch
 
-    m = W.mem16m_config()
+    m = W.mem16m_config(LAYOUT)
     d = m["dims"]
     co, *_ = O.chunk_layout(m["doc_off"])
     case = dict(doc_off=m["doc_off"], chunk_off=co, q=m["q"], K_bar=m["K_bar"], V_bar=m["V_bar"], K_loc=m["K_loc"],

@@ -6,6 +6,12 @@ import oracle as O
 from long_context_memory_b200 import workloads as W
 from helpers import SCORE_ATOL, bf16_of, check_topk
 
+
+def LAYOUT(doc_off):
+    """The oracle's chunk layout (the generator takes the layout from its caller)."""
+    return O.chunk_layout(doc_off)[0]
+
+
 pytestmark = pytest.mark.gpu
 
 
@@ -261,7 +267,7 @@ def test_route_tiny_config_full_pipeline(msa, cuda_device):
 
 
 def test_route_mem1m_full_size(msa, cuda_device):
-    c = W.mem1m_config(with_kv=False)
+    c = W.mem1m_config(LAYOUT, with_kv=False)
     d = c["dims"]
     idx, sc, ds = _run(msa, d, c["QR"], None, c["KR"], c["doc_off"], 16, 0, cuda_device)
     co, *_ = O.chunk_layout(c["doc_off"])
@@ -277,7 +283,7 @@ def test_route_mem1m_full_size(msa, cuda_device):
 
 
 def test_route_mem16m_batch32_sampled(msa, cuda_device):
-    c = W.mem16m_config(with_kv=False)
+    c = W.mem16m_config(LAYOUT, with_kv=False)
     d = c["dims"]
     B = c["B"]
     idx, sc, ds = _run(msa, d, c["QR"], None, c["KR"], c["doc_off"], 16, 0, cuda_device)

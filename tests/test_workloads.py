@@ -9,7 +9,13 @@ import math
 
 import numpy as np
 
+import oracle as O
 from long_context_memory_b200 import workloads as W
+
+
+def LAYOUT(doc_off):
+    """The oracle's chunk layout (the generator takes the layout from its caller)."""
+    return O.chunk_layout(doc_off)[0]
 
 
 def _f64(bits):
@@ -27,7 +33,7 @@ def test_lognormal_lengths_sum_to_T_within_bounds():
 
 
 def test_mem1m_layout_and_planted_cosines():
-    c = W.mem1m_config()
+    c = W.mem1m_config(LAYOUT)
     d = c["dims"]
     lens = c["lens"]
     assert int(np.sum(lens)) == c["T"] == 1_000_000
@@ -51,10 +57,10 @@ def test_mem1m_layout_and_planted_cosines():
 
 
 def test_same_seed_same_bytes():
-    a, b = W.mem1m_config(), W.mem1m_config()
+    a, b = W.mem1m_config(LAYOUT), W.mem1m_config(LAYOUT)
     for key in ("KR", "K_bar", "V_bar", "K_loc", "V_loc", "q", "Hq", "W_QR", "QR"):
         assert hashlib.sha256(a[key].tobytes()).digest() == hashlib.sha256(b[key].tobytes()).digest(), key
-    c = W.mem1m_config(seed=W.BASE_SEED + 99)
+    c = W.mem1m_config(LAYOUT, seed=W.BASE_SEED + 99)
     assert not np.array_equal(a["KR"], c["KR"])
 
 
