@@ -904,19 +904,21 @@ __global__ void __launch_bounds__(1024) gather_plan_kernel(const int32_t* __rest
 
 // copy the planned chunk rows (row = n_kv*D bf16 of K and of V) from host to the staging.
 // One warp per row at a time: its lanes hold up to 4 sixteen-byte pieces of the K row and 4 of
-// the V row in flight (a 4 KB row pair per warp, 512 KB over the whole grid: about three times
-// what a ~55 GB/s host link needs in flight at a few microseconds of latency).  The grid is small
-// (kGatherCtas CTAs of 256 threads, at most 64 registers a thread): it runs beside the routing
-// scan or the attention of another layer without taking an SM from them.
+// the V row in flight (a 4 KB row pair per warp).  One warp per SM (148 CTAs of 32 threads,
+// ~600 KB in flight over the grid: a few times what a ~55 GB/s host link needs at a few
+// microseconds of latency).  Spread this thin, the bus reads cost each SM little: measured on
+// the 100M-token tiered step, the scan beside the gather took 482 us per launch with one warp per
+// SM against 525 us with 16 CTAs of 256 threads (the scan's tiles are split evenly over its CTAs,
+// so its slowest SM sets its end), and the gather itself was no slower.
 #ifndef MSA_GATHER_THREADS
-#define MSA_GATHER_THREADS 256
+#define MSA_GATHER_THREADS 32
 #endif
 #ifndef MSA_GATHER_CTAS
-#define MSA_GATHER_CTAS 16
+#define MSA_GATHER_CTAS 0
 #endif
 constexpr int kGatherThreads = MSA_GATHER_THREADS;
 constexpr int kGatherCtas = MSA_GATHER_CTAS;  // 0: one CTA per SM
-__global__ void __launch_bounds__(kGatherThreads, 4) gather_copy_kernel(const uint4* __restrict__ K_host,
+__global__ void __launch_bounds__(kGatherThreads, 1024 / kGatherThreads) gather_copy_kernel(const uint4* __restrict__ K_host,
                                                                         const uint4* __restrict__ V_host,
                                                                         const int32_t* __restrict__ stage_off,
                                                                         const int32_t* __restrict__ stage_src,

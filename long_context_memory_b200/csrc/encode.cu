@@ -263,20 +263,28 @@ __global__ void __launch_bounds__(MODE == 0 ? kEncThreadsK : kEncThreads, 1) gem
       for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
         const int st = it % kEncStages;
         if (!warp_wait(&full[st], (it / kEncStages) & 1, &abort_flag)) break;
-        if (kb % p.n_tiles == n && len > 0) {
+        const bool mine = kb % p.n_tiles == n && len > 0;
+        uint4 wv[16];  // the box's rows of this lane, copied out so the stage is released at once
+        if (mine) {
           const uint8_t* bx = stages + st * kStageBytes + box * (kABytes / 2);
-          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int r = 4 * i + rg;  // 128-byte rows, 16-byte units swizzled by the row
-            if (r < len) {
-              const uint4 w = *reinterpret_cast<const uint4*>(bx + r * 128 + ((u ^ (r & 7)) << 4));
-              float2 f;
-              f = unpack_bf16x2(w.x); acc[0] += f.x; acc[1] += f.y;
-              f = unpack_bf16x2(w.y); acc[2] += f.x; acc[3] += f.y;
-              f = unpack_bf16x2(w.z); acc[4] += f.x; acc[5] += f.y;
-              f = unpack_bf16x2(w.w); acc[6] += f.x; acc[7] += f.y;
-            }
+            wv[i] = r < len ? *reinterpret_cast<const uint4*>(bx + r * 128 + ((u ^ (r & 7)) << 4))
+                            : make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+        if (mine) {
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float2 f;
+            f = unpack_bf16x2(wv[i].x); acc[0] += f.x; acc[1] += f.y;
+            f = unpack_bf16x2(wv[i].y); acc[2] += f.x; acc[3] += f.y;
+            f = unpack_bf16x2(wv[i].z); acc[4] += f.x; acc[5] += f.y;
+            f = unpack_bf16x2(wv[i].w); acc[6] += f.x; acc[7] += f.y;
           }
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
@@ -299,8 +307,6 @@ __global__ void __launch_bounds__(MODE == 0 ? kEncThreadsK : kEncThreads, 1) gem
             *reinterpret_cast<uint4*>(dst + p.hidden) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[st]);
       }
     }
   } else {
