@@ -13,10 +13,8 @@
 //                      chunks (2 x 64 token rows, each chunk loaded by its own TMA
 //                      box), N = 256 (or 128), accumulators in TMEM; the epilogue rotates
 //                      each row at its document-relative position and pools the
-//                      64 rows of each chunk -> K̄.  Two pool warps sum the same H
-//                      tiles in shared memory (each block once over the chunk pair's N tiles):
-//                      H̄ = chunk mean of H, stored as bf16 hi + lo terms [C, 2*hidden],
-//                      so H is read from HBM once
+//                      64 rows of each chunk -> K̄
+//   pool_h_kernel      H̄ = chunk mean of H, stored as bf16 hi + lo terms [C, 2*hidden]
 //   gemm_kernel<POOL>  (H̄_hi | H̄_lo) [W_V | W^KR] over K = 2*hidden -> V̄, K̄^R.
 //                      Pooling before the projection is exact by linearity;
 //                      splitting H̄ into two bf16 terms keeps ~16 mantissa bits.
@@ -48,7 +46,6 @@ constexpr int kBM = 128, kBK = 64;
 constexpr int kEncStagesMax = 4;
 constexpr int kABytes = kBM * kBK * 2;  // 16 KB
 constexpr int kEncThreads = 192;        // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
-constexpr int kEncThreadsK = 256;       // mode K: + warps 6, 7, the pool warps (chunk means of H)
 
 __global__ void chunk_map_kernel(const int64_t* __restrict__ doc_off, const int32_t* __restrict__ chunk_off,
                                  int n_docs, int n_chunks, int64_t T, int64_t* __restrict__ tok0,
@@ -90,6 +87,41 @@ __global__ void transpose_kernel(const uint16_t* __restrict__ in, int K, int N, 
   }
 }
 
+// H̄[c] = mean of the chunk's token rows; one block per chunk, 8 columns per thread per pass
+__global__ void __launch_bounds__(256) pool_h_kernel(const __nv_bfloat16* __restrict__ H, int hidden,
+                                                     const int64_t* __restrict__ tok0,
+                                                     const int32_t* __restrict__ clen,
+                                                     __nv_bfloat16* __restrict__ hbar) {
+  const int c = blockIdx.x;
+  const int64_t t0 = tok0[c];
+  const int n = clen[c];
+  const float inv = 1.0f / (float)n;
+  for (int col = threadIdx.x * 8; col < hidden; col += blockDim.x * 8) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const __nv_bfloat16* src = H + (size_t)t0 * hidden + col;
+    for (int r = 0; r < n; ++r) {
+      const uint4 w = __ldg(reinterpret_cast<const uint4*>(src + (size_t)r * hidden));
+      float2 f;
+      f = unpack_bf16x2(w.x); acc[0] += f.x; acc[1] += f.y;
+      f = unpack_bf16x2(w.y); acc[2] += f.x; acc[3] += f.y;
+      f = unpack_bf16x2(w.z); acc[4] += f.x; acc[5] += f.y;
+      f = unpack_bf16x2(w.w); acc[6] += f.x; acc[7] += f.y;
+    }
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float m0 = acc[2 * j] * inv, m1 = acc[2 * j + 1] * inv;
+      const float h0 = __bfloat162float(__float2bfloat16_rn(m0));
+      const float h1 = __bfloat162float(__float2bfloat16_rn(m1));
+      hi[j] = pack_bf16x2(h0, h1);
+      lo[j] = pack_bf16x2(m0 - h0, m1 - h1);
+    }
+    __nv_bfloat16* dst = hbar + (size_t)c * 2 * hidden + col;
+    *reinterpret_cast<uint4*>(dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(dst + hidden) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  }
+}
+
 // Sum of v[0..31] over the 32 lanes of a warp, transposed: on return v[0] of
 // lane l holds the warp-wide sum of column l (31 shuffles for 32 columns).
 __device__ __forceinline__ void warp_transpose_reduce32(float (&v)[32], int lane) {
@@ -118,7 +150,6 @@ struct GemmParams {
   const int64_t* tok0;
   const int32_t* clen;
   const int32_t* pos0;
-  __nv_bfloat16* hbar;   // mode K: chunk means of H, [C][2*hidden] bf16 hi | lo (written by the pool warp)
   __nv_bfloat16* out0;   // K̄ (mode K) or V̄ (pooled)
   __nv_bfloat16* out1;   // K̄^R (pooled)
   int n_out0;            // columns of out0 (n_kv*D); pooled: columns >= n_out0 go to out1
@@ -128,7 +159,7 @@ struct GemmParams {
 };
 
 template <int MODE, int kBN>
-__global__ void __launch_bounds__(MODE == 0 ? kEncThreadsK : kEncThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap map_a,
+__global__ void __launch_bounds__(kEncThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                                                               const __grid_constant__ CUtensorMap map_b,
                                                               const GemmParams p) {
   constexpr int kBBytes = kBN * kBK * 2;
@@ -158,7 +189,7 @@ __global__ void __launch_bounds__(MODE == 0 ? kEncThreadsK : kEncThreads, 1) gem
   if (threadIdx.x == 0) {
     for (int s = 0; s < kEncStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], MODE == kModeK ? 3 : 1);  // MMA commit (+ the two pool warps in mode K)
+      mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
@@ -242,71 +273,6 @@ __global__ void __launch_bounds__(MODE == 0 ? kEncThreadsK : kEncThreads, 1) gem
       if (abort_flag) {  // every MMA issued completes before the TMEM is freed
         umma_commit(drained);
         mbar_drain_ring(drained, 1, 0, 1);
-      }
-    }
-  } else if (MODE == kModeK && warp >= 6) {
-    // ------------- pool warps: chunk means of the H tiles the MMA reads -------------
-    // Every N tile of a chunk pair loads the same H blocks; the CTA of N tile n pools the blocks
-    // kb with kb % n_tiles == n (so each block is pooled once, and every CTA gets an equal share):
-    // warp 6 (chunk 2m) and warp 7 (chunk 2m + 1) sum their chunk's 64-row box of the block over
-    // the chunk's own rows (fp32) and store the mean as bf16 hi + lo terms; for the other blocks
-    // they only release the stage.  Lane l reads 16-byte unit u = l % 8 (columns 8u .. 8u + 7) of
-    // rows 4i + l / 8; the four row groups are then added across lanes, and lanes 0..7 store their
-    // unit.
-    const int box = warp - 6;
-    const int u = lane & 7, rg = lane >> 3;
-    int it = 0;
-    for (int tile = blockIdx.x; tile < total_tiles && !abort_flag; tile += gridDim.x) {
-      const int m = tile / p.n_tiles, n = tile % p.n_tiles;
-      const int c = 2 * m + box;
-      const int len = c < p.n_chunks ? p.clen[c] : 0;
-      for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
-        const int st = it % kEncStages;
-        if (!warp_wait(&full[st], (it / kEncStages) & 1, &abort_flag)) break;
-        const bool mine = kb % p.n_tiles == n && len > 0;
-        uint4 wv[16];  // the box's rows of this lane, copied out so the stage is released at once
-        if (mine) {
-          const uint8_t* bx = stages + st * kStageBytes + box * (kABytes / 2);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int r = 4 * i + rg;  // 128-byte rows, 16-byte units swizzled by the row
-            wv[i] = r < len ? *reinterpret_cast<const uint4*>(bx + r * 128 + ((u ^ (r & 7)) << 4))
-                            : make_uint4(0u, 0u, 0u, 0u);
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[st]);
-        if (mine) {
-          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float2 f;
-            f = unpack_bf16x2(wv[i].x); acc[0] += f.x; acc[1] += f.y;
-            f = unpack_bf16x2(wv[i].y); acc[2] += f.x; acc[3] += f.y;
-            f = unpack_bf16x2(wv[i].z); acc[4] += f.x; acc[5] += f.y;
-            f = unpack_bf16x2(wv[i].w); acc[6] += f.x; acc[7] += f.y;
-          }
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 8);
-            acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
-          }
-          if (rg == 0) {
-            const float inv = 1.0f / (float)len;
-            uint32_t hi[4], lo[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float m0 = acc[2 * j] * inv, m1 = acc[2 * j + 1] * inv;
-              const float h0 = __bfloat162float(__float2bfloat16_rn(m0));
-              const float h1 = __bfloat162float(__float2bfloat16_rn(m1));
-              hi[j] = pack_bf16x2(h0, h1);
-              lo[j] = pack_bf16x2(m0 - h0, m1 - h1);
-            }
-            __nv_bfloat16* dst = p.hbar + (size_t)c * 2 * p.hidden + kb * kBK + 8 * u;
-            *reinterpret_cast<uint4*>(dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-            *reinterpret_cast<uint4*>(dst + p.hidden) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-          }
-        }
       }
     }
   } else {
@@ -431,11 +397,11 @@ cudaError_t launch_gemm(int bn, int grid, size_t smem, cudaStream_t s, const CUt
   if (bn == 256) {
     cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(gemm_kernel<MODE, 256>), (int)smem);
     if (e != cudaSuccess) return e;
-    gemm_kernel<MODE, 256><<<grid, MODE == kModeK ? kEncThreadsK : kEncThreads, smem, s>>>(ma, mb, p);
+    gemm_kernel<MODE, 256><<<grid, kEncThreads, smem, s>>>(ma, mb, p);
   } else {
     cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(gemm_kernel<MODE, 128>), (int)smem);
     if (e != cudaSuccess) return e;
-    gemm_kernel<MODE, 128><<<grid, MODE == kModeK ? kEncThreadsK : kEncThreads, smem, s>>>(ma, mb, p);
+    gemm_kernel<MODE, 128><<<grid, kEncThreads, smem, s>>>(ma, mb, p);
   }
   return cudaGetLastError();
 }
@@ -506,7 +472,7 @@ msa_status encode_launch(const msa_dims& d, const void* H, int64_t T, const int6
         static_cast<const uint16_t*>(W_KR), hidden, NR, reinterpret_cast<uint16_t*>(w.wvrT), NV);
     MSA_CUDA_CHECK(cudaGetLastError());
   }
-  // ---- K̄: per-token projection + RoPE + pooling on tcgen05; H̄ (hi | lo) from the same tiles ----
+  // ---- K̄: per-token projection + RoPE + pooling on tcgen05 ----
   {
     CUtensorMap ma, mb;
     const uint64_t adims[2] = {(uint64_t)hidden, (uint64_t)T};
@@ -532,12 +498,17 @@ msa_status encode_launch(const msa_dims& d, const void* H, int64_t T, const int6
     p.tok0 = w.tok0;
     p.clen = w.clen;
     p.pos0 = w.pos0;
-    p.hbar = w.hbar;
     p.out0 = static_cast<__nv_bfloat16*>(K_bar);
     p.n_out0 = NK;
     const int grid = std::max(1, std::min(sm_count(), p.m_tiles * p.n_tiles));
     TraceScope ts(kKEncGemmK, s);
     MSA_CUDA_CHECK(launch_gemm<kModeK>(bn, grid, gemm_smem_bytes(kModeK, bn), s, ma, mb, p));
+  }
+  // ---- H̄ (hi | lo) ----
+  {
+    TraceScope ts(kKEncPoolH, s);
+    pool_h_kernel<<<n_chunks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(H), hidden, w.tok0, w.clen, w.hbar);
+    MSA_CUDA_CHECK(cudaGetLastError());
   }
   // ---- V̄ | K̄^R = H̄ [W_V | W^KR] ----
   {

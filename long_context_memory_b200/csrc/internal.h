@@ -44,6 +44,7 @@ enum KernelId : int {
   kKEncChunkMap,
   kKEncTransposeW,
   kKEncGemmK,
+  kKEncPoolH,
   kKEncGemmPooled,
   kKRopeRows,
   kKGatherPlan,

@@ -218,7 +218,7 @@ msa_status encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int ra
 namespace {
 const char* kKernelNames[kKernelCount] = {
     "router_query", "scan", "topk_slice", "topk_merge", "rope_table", "attn_split", "attn_combine",
-    "enc_chunk_map", "enc_transpose_w", "enc_gemm_k", "enc_gemm_pooled", "rope_rows", "gather_plan", "gather_copy",
+    "enc_chunk_map", "enc_transpose_w", "enc_gemm_k", "enc_pool_h", "enc_gemm_pooled", "rope_rows", "gather_plan", "gather_copy",
     "chunk_off_extend", "aux_loss", "kv_append", "kr_norms", "attn_merge"};
 
 struct TraceState {
