@@ -58,6 +58,9 @@ def parse():
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the B=16 tiered step, the 1M/16M-token cases and the encode measurement")
     ap.add_argument("--layers", type=int, default=LAYERS)
+    ap.add_argument("--memory-parallel", action="store_true",
+                    help="shard the 100M-token memory's documents over the ranks (routing, top-k exchange, "
+                         "attention shares and their merge) instead of running replicas")
     return ap.parse_args()
 
 
@@ -652,7 +655,7 @@ def mem1m_step(msa, S, dev, hbm_peak, n_rot=8):
 
     from long_context_memory_b200 import workloads as W
 
-    c = W.mem1m_config()
+    c = W.mem1m_config(lambda off: msa.chunk_offsets(off)[0])
     d = c["dims"]
     B, k, T = c["B"], c["k"], c["T"]
     co_np, C = msa.chunk_offsets(c["doc_off"])
@@ -703,10 +706,77 @@ def mem1m_step(msa, S, dev, hbm_peak, n_rot=8):
             "kernels_us": {k: v[0] / v[1] * 1e3 for k, v in kt.items()}}
 
 
+def run_memory_parallel(args):
+    """The pages' memory-parallel deployment: every rank holds a contiguous range of the 100M-token
+    memory's documents (its K̄^R, inverse norms and K̄/V̄, device-resident); per layer every rank
+    routes its shard, the ranks exchange their (score, id) candidates and merge them, every rank
+    attends over the selected documents it holds (the local cache on rank 0), and the shares are
+    exchanged and merged.  value = layers x T x B / step time (the memory's tokens are split over
+    the ranks: the total work is fixed, scaling "strong")."""
+    import torch
+    import torch.distributed as dist
+
+    import long_context_memory_b200 as msa
+    from long_context_memory_b200 import parallel as P
+    from long_context_memory_b200 import profile_cases as PC
+    from long_context_memory_b200 import workloads as W
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ.setdefault("MASTER_PORT", "29533")
+    os.environ.setdefault("RANK", str(rank))
+    os.environ.setdefault("WORLD_SIZE", str(ws))
+    dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
+    d = W.QWEN3_4B_DIMS
+    layers = min(args.layers, 8)
+    doc_off, co, C = PC.chunk_layout_host(T_MEM, MEDIAN, W.BASE_SEED + SEED_OFF)
+    sh = P.shard_memory(co, ws, rank)
+    g = torch.Generator(device=dev)
+    g.manual_seed(W.BASE_SEED + SEED_OFF + 1000 * rank)
+    KR = [PC.randn_bf16((sh.n_chunks, d.n_r, d.d_r), g, dev) for _ in range(layers)]
+    inv = [msa.router_key_norms(d, kr) for kr in KR]
+    Kb = PC.randn_bf16((sh.n_chunks, d.n_kv, d.head_dim), g, dev)  # content rows, shared by the layers
+    Vb = PC.randn_bf16((sh.n_chunks, d.n_kv, d.head_dim), g, dev)
+    gq = torch.Generator(device=dev)
+    gq.manual_seed(W.BASE_SEED + SEED_OFF + 7)  # the same queries and weights on every rank
+    W_QR = [(torch.randn((d.hidden, d.n_r * d.d_r), generator=gq, device=dev) / math.sqrt(d.hidden)).to(torch.bfloat16)
+            for _ in range(layers)]
+    Hq = [PC.randn_bf16((1, d.hidden), gq, dev) for _ in range(layers)]
+    q = [PC.randn_bf16((1, d.n_q, d.head_dim), gq, dev) for _ in range(layers)]
+    K_loc = PC.randn_bf16((1, T_LOC, d.n_kv, d.head_dim), gq, dev)
+    V_loc = PC.randn_bf16((1, T_LOC, d.n_kv, d.head_dim), gq, dev)
+    loc_len = torch.full((1,), T_LOC, dtype=torch.int32, device=dev)
+    S = torch.cuda.Stream(device=dev)
+
+    def step(i):
+        for l in range(layers):
+            idx, _ = P.route_topk_sharded(d, Hq[l], W_QR[l], KR[l], sh, TOPK, route=lambda *a: msa.route_topk(
+                *a, kr_inv_norm=inv[l]))
+            P.attend_sharded(d, q[l], Kb, Vb, sh, idx, K_loc, V_loc, loc_len, TOPK)
+
+    ms = device_time(S, step, args.steps, args.warmup, dist, dev)
+    if rank == 0:
+        value = layers * T_MEM * 1 / (ms * 1e-3)
+        print(json.dumps({
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 pooled memory and queries, lognormal document lengths)",
+            "config": {"workload": f"mem100m memory-parallel: 100M-token memory sharded by documents over {ws} "
+                                   f"rank(s), B=1, top-{TOPK}, {T_LOC}-token local KV on rank 0, {layers} layer "
+                                   f"instances (K̄/V̄ device-resident, one content copy shared by the layers)",
+                       "parallelism": f"memory-parallel x{ws}"}}), flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.memory_parallel:
+        run_memory_parallel(args)
     else:
         run_gpu(args)
 

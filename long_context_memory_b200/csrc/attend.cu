@@ -1074,9 +1074,19 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
                          const void* V_loc, const void* k_new, const void* v_new, const int32_t* loc_len,
                          int t_loc_max, int pos_offset,
                          const void* rope_cache, int k_loc_rotated, float scale, int phase, int early, void* out,
-                         void* ws, cudaStream_t s, const AttendShare* share) {
+                         void* ws, cudaStream_t s, const AttendShare* share, const AttendPlan* plan) {
   AttendWs w;
   attend_workspace(d, B, M, k, t_loc_max, pos_offset, ws, &w);
+  int n_loc = w.n_split_local, n_chk = w.n_split_chunk;
+  if (plan) {  // the same slots of the workspace (at most w.n_parts per row), shared by expected keys
+    int n_total = w.n_parts;
+    if (plan->max_total > 0) n_total = std::min(n_total, plan->max_total);
+    n_total = std::max(2, n_total);
+    const double sel = std::max(1.0, plan->chunks_per_doc) * k;
+    n_chk = (int)std::lround(n_total * sel / (sel + std::max(0, t_loc_max)));
+    n_chk = std::max(1, std::min(n_chk, n_total - 1));
+    n_loc = std::max(1, std::min(n_total - n_chk, std::max(1, (t_loc_max + kTK - 1) / kTK)));
+  }
   const int D = d.head_dim;
   const bool local_keys = phase != 2 && (!share || share->local_keys);
   const float2* tab = (k_loc_rotated || !local_keys) ? nullptr : static_cast<const float2*>(rope_cache);
@@ -1106,12 +1116,12 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
   p.n_docs = n_docs;
   p.t_loc_max = t_loc_max;
   p.pos_offset = pos_offset;
-  p.n_loc_splits = local_keys ? w.n_split_local : 0;
-  p.n_chunk_splits = phase == 1 ? 0 : w.n_split_chunk;
+  p.n_loc_splits = local_keys ? n_loc : 0;
+  p.n_chunk_splits = phase == 1 ? 0 : n_chk;
   // a share without the local keys uses the chunk splits' slots alone
   const bool chunks_only = share && !share->local_keys;
-  p.chunk_part_base = chunks_only ? 0 : w.n_split_local;
-  p.n_parts = chunks_only ? w.n_split_chunk : w.n_parts;
+  p.chunk_part_base = chunks_only ? 0 : n_loc;
+  p.n_parts = chunks_only ? n_chk : n_loc + n_chk;
   p.doc_base = share ? share->doc_base : 0;
   p.foreign_ok = share ? 1 : 0;
   // the local-key items may start before the predecessor finishes only if this call launches

@@ -224,8 +224,12 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
 #pragma unroll
         for (int e = 0; e < DR / 32; ++e) kw[e] = *reinterpret_cast<const uint4*>(base + unit_of_slot<DR>(e, lane) * 16);
       }
+      // the row is in registers: the stage may refill.  The proxy fence orders these generic-proxy
+      // reads before the bulk copy (async proxy) that will overwrite the stage once every warp has
+      // arrived, so the last warp to arrive cannot have its loads overtaken by the refill.
+      fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);  // the row is in registers: the stage may refill
+      if (lane == 0) mbar_arrive(&empty[st]);
       if (j < NK) {
         float dot = 0.f, kk = 0.f;
         if (hl) {
@@ -323,8 +327,12 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
 #pragma unroll
         for (int e = 0; e < DR / 32; ++e) kw[e] = *reinterpret_cast<const uint4*>(base + unit_of_slot<DR>(e, lane) * 16);
       }
+      // the row is in registers: the stage may refill.  The proxy fence orders these generic-proxy
+      // reads before the bulk copy (async proxy) that will overwrite the stage once every warp has
+      // arrived, so the last warp to arrive cannot have its loads overtaken by the refill.
+      fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);  // the row is in registers: the stage may refill
+      if (lane == 0) mbar_arrive(&empty[st]);
       float* dk = nullptr;
       if (j < NK) dk = j == 0 ? (p.dK_pos ? p.dK_pos + (size_t)i * NR : nullptr)
                               : (p.dK_neg ? p.dK_neg + ((size_t)i * p.N + (j - 1)) * NR : nullptr);
