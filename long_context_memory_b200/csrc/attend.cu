@@ -1074,19 +1074,10 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
                          const void* V_loc, const void* k_new, const void* v_new, const int32_t* loc_len,
                          int t_loc_max, int pos_offset,
                          const void* rope_cache, int k_loc_rotated, float scale, int phase, int early, void* out,
-                         void* ws, cudaStream_t s, const AttendShare* share, const AttendPlan* plan) {
+                         void* ws, cudaStream_t s, const AttendShare* share) {
   AttendWs w;
   attend_workspace(d, B, M, k, t_loc_max, pos_offset, ws, &w);
-  int n_loc = w.n_split_local, n_chk = w.n_split_chunk;
-  if (plan) {  // the same slots of the workspace (at most w.n_parts per row), shared by expected keys
-    int n_total = w.n_parts;
-    if (plan->max_total > 0) n_total = std::min(n_total, plan->max_total);
-    n_total = std::max(2, n_total);
-    const double sel = std::max(1.0, plan->chunks_per_doc) * k;
-    n_chk = (int)std::lround(n_total * sel / (sel + std::max(0, t_loc_max)));
-    n_chk = std::max(1, std::min(n_chk, n_total - 1));
-    n_loc = std::max(1, std::min(n_total - n_chk, std::max(1, (t_loc_max + kTK - 1) / kTK)));
-  }
+  const int n_loc = w.n_split_local, n_chk = w.n_split_chunk;
   const int D = d.head_dim;
   const bool local_keys = phase != 2 && (!share || share->local_keys);
   const float2* tab = (k_loc_rotated || !local_keys) ? nullptr : static_cast<const float2*>(rope_cache);

@@ -36,7 +36,16 @@ namespace {
 constexpr int kAuxCompute = 8;                      // compute warps
 constexpr int kAuxThreads = 32 * (kAuxCompute + 1);  // + the producer warp
 constexpr int kAuxRows = 8;                         // key rows per stage (one per compute warp)
-constexpr int kAuxStages = 6;
+constexpr int kAuxStagesMax = 8;  // ring stages when a positive's rows stay resident (<= 64 rows)
+constexpr int kAuxStagesRing = 6; // ring stages when they stream twice (more than 63 negatives)
+
+// a positive's rows stay in the ring for both passes when the gradients are wanted and they fit
+__host__ __device__ inline bool aux_resident(bool grads, int nk) {
+  return grads && (nk + kAuxRows - 1) / kAuxRows <= kAuxStagesMax;
+}
+__host__ __device__ inline int aux_stages(bool grads, int nk) {
+  return aux_resident(grads, nk) ? kAuxStagesMax : kAuxStagesRing;
+}
 constexpr float kAuxEps = 1e-12f;
 
 struct AuxParams {
@@ -53,7 +62,7 @@ struct AuxParams {
   float inv_tau;
 };
 
-// shared memory: ring [kAuxStages][kAuxRows][n_r * DR] bf16 | cos, |k| [NK][8] fp32 | g [NK] |
+// shared memory: ring [stages][kAuxRows][n_r * DR] bf16 | cos, |k| [NK][8] fp32 | g [NK] |
 // per compute warp a slice of kSlice floats (its dK row staged for coalesced stores, then its
 // dQ partial) | barriers
 template <int DR>
@@ -63,9 +72,9 @@ struct AuxSmem {
   static constexpr int kLanePad = DR / 4 + 4;   // a lane's DR/4 values + 4 floats of padding
   static constexpr int kSlice = 32 * kLanePad;  // >= 8 * DR
   static constexpr int kQBytes = 8 * DR * 2;    // one query row (room for 8 router heads)
-  static __host__ __device__ size_t bytes(int nk) {
-    return (size_t)kAuxStages * kStageBytes + 2 * kQBytes + (size_t)nk * 8 * 4 * 2 + (size_t)nk * 4 + 16 +
-           (size_t)kAuxCompute * kSlice * 4 + (2 * kAuxStages + 4) * 8 + 16;
+  static __host__ __device__ size_t bytes(int nk, int stages) {
+    return (size_t)stages * kStageBytes + 2 * kQBytes + (size_t)nk * 8 * 4 * 2 + (size_t)nk * 4 + 16 +
+           (size_t)kAuxCompute * kSlice * 4 + (2 * kAuxStagesMax + 4) * 8 + 16;
   }
 };
 
@@ -92,7 +101,9 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
   extern __shared__ __align__(128) uint8_t aux_sm[];
   const int n_r = p.n_r, NK = p.N + 1, NR = n_r * DR;
   uint8_t* ring = aux_sm;
-  uint8_t* qbuf = aux_sm + kAuxStages * Sm::kStageBytes;                          // [2][n_r * DR] bf16
+  const bool grads = p.dQ != nullptr || p.dK_pos != nullptr || p.dK_neg != nullptr;
+  const int S = aux_stages(grads, NK);  // ring stages
+  uint8_t* qbuf = aux_sm + S * Sm::kStageBytes;                                   // [2][n_r * DR] bf16
   float* cosv = reinterpret_cast<float*>(qbuf + 2 * Sm::kQBytes);                 // [NK][8]
   float* nkv = cosv + (size_t)NK * 8;                                            // [NK][8]
   float* gs = nkv + (size_t)NK * 8;                                              // [NK]
@@ -100,8 +111,8 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
   // red: [kAuxCompute][Sm::kSlice]
   uint64_t* full = reinterpret_cast<uint64_t*>(
       (reinterpret_cast<uintptr_t>(red + (size_t)kAuxCompute * Sm::kSlice) + 7) & ~uintptr_t(7));
-  uint64_t* empty = full + kAuxStages;
-  uint64_t* qfull = empty + kAuxStages;  // [2] a positive's query row landed
+  uint64_t* empty = full + kAuxStagesMax;
+  uint64_t* qfull = empty + kAuxStagesMax;  // [2] a positive's query row landed
   uint64_t* qempty = qfull + 2;          // [2] every compute warp is done with it
   __shared__ float qn[8];      // clamped query norms (negative: below eps)
   __shared__ float chead[8];   // sum_j g_j cos_jh
@@ -110,12 +121,15 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
   __shared__ int abort_flag;   // a bounded wait of this CTA gave up
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const bool grads = p.dQ != nullptr || p.dK_pos != nullptr || p.dK_neg != nullptr;
   const int n_ch = (NK + kAuxRows - 1) / kAuxRows;  // stages per pass
   const int passes = grads ? 2 : 1;
+  // With gradients and at most kAuxStagesMax chunks of rows, a positive's rows stay in the ring for
+  // both passes: the producer loads them once and pass 2 reads them again from shared memory.
+  const bool resident = aux_resident(grads, NK);
+  const int loads = resident ? 1 : passes;  // producer passes over a positive's rows
   const size_t row_bytes = (size_t)NR * 2;
   if (tid == 0) {
-    for (int s = 0; s < kAuxStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kAuxCompute);
     }
@@ -141,10 +155,10 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
           mbar_arrive_expect_tx(&qfull[qb], (uint32_t)row_bytes);
           bulk_load(qbuf + qb * Sm::kQBytes, p.Q + (size_t)i * NR, (uint32_t)row_bytes, &qfull[qb]);
         }
-        for (int pass = 0; pass < passes && !stop; ++pass) {
+        for (int pass = 0; pass < loads && !stop; ++pass) {
           for (int c = 0; c < n_ch; ++c, ++it) {
-            const int st = it % kAuxStages;
-            if (it >= kAuxStages && !mbar_wait(&empty[st], ((it / kAuxStages) - 1) & 1, &abort_flag)) {
+            const int st = it % S;
+            if (it >= S && !mbar_wait(&empty[st], ((it / S) - 1) & 1, &abort_flag)) {
               stop = true;
               break;
             }
@@ -164,7 +178,7 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
       }
       if (abort_flag) {  // the copies still in flight land before the CTA exits
         const int q_issued = stop ? pi + 1 : pi;
-        mbar_drain_ring(full, kAuxStages, it - kAuxStages, it);
+        mbar_drain_ring(full, S, it - S, it);
         mbar_drain_ring(qfull, 2, q_issued - 2, q_issued);
       }
     }
@@ -214,9 +228,10 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
     aux_bar_sync();  // qn written
 
     // ---- pass 1: cosines ----
+    const int it_first = it;  // ring position of this positive's first chunk
     for (int c = 0; c < n_ch; ++c, ++it) {
-      const int st = it % kAuxStages;
-      failed |= !warp_wait(&full[st], (it / kAuxStages) & 1, &abort_flag);  // on failure: left at the next barrier
+      const int st = it % S;
+      failed |= !warp_wait(&full[st], (it / S) & 1, &abort_flag);  // on failure: left at the next barrier
       const int j = c * kAuxRows + warp;
       uint4 kw[DR / 32];
       if (j < NK && hl) {
@@ -224,12 +239,14 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
 #pragma unroll
         for (int e = 0; e < DR / 32; ++e) kw[e] = *reinterpret_cast<const uint4*>(base + unit_of_slot<DR>(e, lane) * 16);
       }
-      // the row is in registers: the stage may refill.  The proxy fence orders these generic-proxy
-      // reads before the bulk copy (async proxy) that will overwrite the stage once every warp has
-      // arrived, so the last warp to arrive cannot have its loads overtaken by the refill.
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);
+      if (!resident) {
+        // the row is in registers: the stage may refill.  The proxy fence orders these generic-proxy
+        // reads before the bulk copy (async proxy) that will overwrite the stage once every warp
+        // has arrived, so the last warp to arrive cannot have its loads overtaken by the refill.
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+      }
       if (j < NK) {
         float dot = 0.f, kk = 0.f;
         if (hl) {
@@ -311,15 +328,18 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
       if (lane == 0) chead[warp] = cc;
     }
 
-    // ---- pass 2: gradients (the rows again, from L2), one 16-byte unit of the row at a time ----
+    // ---- pass 2: gradients (the rows again: still in the ring when resident, otherwise reloaded
+    //      from L2), one 16-byte unit of the row at a time ----
     float acc[V];
 #pragma unroll
     for (int e = 0; e < V; ++e) acc[e] = 0.f;
     const float nq = hl ? fabsf(qn[h]) : 1.f;
     float* slice = red + (size_t)warp * Sm::kSlice;
-    for (int c = 0; c < n_ch; ++c, ++it) {
-      const int st = it % kAuxStages;
-      failed |= !warp_wait(&full[st], (it / kAuxStages) & 1, &abort_flag);  // on failure: left at the next barrier
+    for (int c = 0; c < n_ch; ++c) {
+      const int ring_it = resident ? it_first + c : it++;
+      const int st = ring_it % S;
+      if (!resident)  // on failure: left at the next barrier
+        failed |= !warp_wait(&full[st], (ring_it / S) & 1, &abort_flag);
       const int j = c * kAuxRows + warp;
       uint4 kw[DR / 32];
       if (j < NK && hl) {
@@ -450,11 +470,11 @@ msa_status aux_loss_launch(const msa_dims& d, const void* QR, const void* K_pos,
   const int grid = std::max(1, std::min(P, sm_count()));
   TraceScope ts(kKAuxLoss, s);
   if (d.d_r == 128) {
-    const size_t sm = AuxSmem<128>::bytes(N + 1);
+    const size_t sm = AuxSmem<128>::bytes(N + 1, aux_stages(dQ || dK_pos || dK_neg, N + 1));
     MSA_CUDA_CHECK(set_max_dynamic_smem(reinterpret_cast<const void*>(aux_loss_kernel<128>), (int)sm));
     MSA_CUDA_CHECK(launch_pdl(aux_loss_kernel<128>, dim3(grid), dim3(kAuxThreads), sm, s, p));
   } else {
-    const size_t sm = AuxSmem<64>::bytes(N + 1);
+    const size_t sm = AuxSmem<64>::bytes(N + 1, aux_stages(dQ || dK_pos || dK_neg, N + 1));
     MSA_CUDA_CHECK(set_max_dynamic_smem(reinterpret_cast<const void*>(aux_loss_kernel<64>), (int)sm));
     MSA_CUDA_CHECK(launch_pdl(aux_loss_kernel<64>, dim3(grid), dim3(kAuxThreads), sm, s, p));
   }

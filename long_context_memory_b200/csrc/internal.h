@@ -175,15 +175,6 @@ size_t attend_workspace(const msa_dims& d, int B, int M, int k, int t_loc_max, i
 // One rank's share of a memory-parallel attention: the selected documents it holds (global ids,
 // the others skipped), the local keys only where local_keys is set, and the share's normalised
 // fp32 output with its base-2 log-sum-exp instead of the bf16 result.
-// The split plan of an attention whose selected chunks are in place when it starts (the tiered
-// decode stages them before it): the splits are shared between the local keys and the selected
-// chunks in proportion to the expected key counts, with the memory's own chunks per document,
-// and no split is kept small for latency (nothing is waited for); at most max_total splits per
-// (query, token group) when max_total > 0.
-struct AttendPlan {
-  double chunks_per_doc;
-  int max_total;
-};
 struct AttendShare {
   int doc_base;    // global id of the shard's first document
   int local_keys;  // 1: this share also attends over the local keys
@@ -195,8 +186,7 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
                          const void* K_loc, const void* V_loc, const void* k_new, const void* v_new,
                          const int32_t* loc_len, int t_loc_max,
                          int pos_offset, const void* rope_cache, int k_loc_rotated, float scale, int phase,
-                         int early, void* out, void* ws, cudaStream_t s, const AttendShare* share = nullptr,
-                         const struct AttendPlan* plan = nullptr);
+                         int early, void* out, void* ws, cudaStream_t s, const AttendShare* share = nullptr);
 msa_status attend_merge_launch(const float* o_parts, const float* lse2_parts, int R, int n_rows, int D, void* out,
                                cudaStream_t s);
 msa_status gather_kv_launch(const msa_dims& d, const void* K_host, const void* V_host, const int32_t* chunk_off,

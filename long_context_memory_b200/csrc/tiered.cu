@@ -25,13 +25,6 @@
 
 #include "internal.h"
 
-#ifndef TIERED_USE_PLAN
-#define TIERED_USE_PLAN 1
-#endif
-#ifndef TIERED_PLAN_MAX_TOTAL
-#define TIERED_PLAN_MAX_TOTAL 0
-#endif
-
 namespace msa {
 
 namespace {
@@ -123,9 +116,6 @@ msa_status tiered_launch(const msa_dims& d, const msa_layer* layers, const void*
   const double gather_bytes = (double)B * k * ((double)n_chunks / n_docs) * 2.0 * d.n_kv * d.head_dim * 2.0;
   const double scan_bytes = (double)n_chunks * d.n_r * d.d_r * 2.0;
   const bool late = gather_bytes / 50e9 < scan_bytes / 6.5e12;
-  // the staged documents are in place when an attention starts: its splits follow the memory's
-  // own document size, with none kept small for latency
-  const AttendPlan plan{(double)n_chunks / n_docs, TIERED_PLAN_MAX_TOTAL};
   auto attend = [&](int l) -> msa_status {
     const msa_layer& L = layers[l];
     const int slot = l & 1;
@@ -134,8 +124,7 @@ msa_status tiered_launch(const msa_dims& d, const msa_layer* layers, const void*
     // neither this layer's query, cache nor attention workspace
     return attend_launch(d, L.q, B, 1, w.K_stage[slot], w.V_stage[slot], w.stage_off[slot], n_stage_docs,
                          w.stage_idx[slot], k, L.K_loc, L.V_loc, L.k_new, L.v_new, loc_len, t_loc_max, pos_offset,
-                         nullptr, 1, 0.0f, 0, l + 1 < n_layers ? 1 : 0, L.out, w.attend_ws, s, nullptr,
-                         TIERED_USE_PLAN ? &plan : nullptr);
+                         nullptr, 1, 0.0f, 0, l + 1 < n_layers ? 1 : 0, L.out, w.attend_ws, s);
   };
   for (int l = 0; l < n_layers; ++l) {
     const msa_layer& L = layers[l];
