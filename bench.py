@@ -426,7 +426,9 @@ def run_gpu(args):
     C_est = 1_580_000
     per_layer = C_est * d.n_r * (d.d_r * 2 + 4) + d.hidden * d.n_r * d.d_r * 2 + 2 * T_LOC * d.n_kv * d.head_dim * 2
     n_layers = layers_that_fit(dev, args.layers, per_layer, 24 << 30)
-    host_layers = host_layers_that_fit(2 * C_est * d.n_kv * d.head_dim * 2)
+    # distinct pinned host copies of a layer's K̄/V̄ (6.4 GB each): one per rank when several ranks
+    # share the host's memory
+    host_layers = host_layers_that_fit(2 * C_est * d.n_kv * d.head_dim * 2, want=2 if ws == 1 else 1)
     case = PC.TieredCase(T_MEM, MEDIAN, T_LOC, W.BASE_SEED + SEED_OFF, dev, n_layers, host_layers, B=1, k=TOPK)
     n_chunks, n_docs = case.C, case.n_docs
     S = torch.cuda.Stream(device=dev)

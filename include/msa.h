@@ -430,25 +430,32 @@ msa_status msa_gather_kv(const msa_dims* dims, const void* K_bar_host, const voi
  * instances: no layer reads what another layer of the call writes (its inputs
  * must not alias another layer's outputs or local cache).  They share the
  * document layout (chunk_off, n_docs, n_chunks), B, k, loc_len, t_loc_max and
- * pos_offset.  Per layer l the call enqueues, on
- * `stream`, msa_route_topk (agg MAX); on `copy_stream`, after an event,
- * msa_gather_kv of the routed documents into one of two staging areas in ws;
- * on `stream`, after the routing of layer l + 1 and an event on that gather,
- * msa_sparse_attend over the staged documents and the local keys.  The gather
- * of layer l waits for its routing, and also for the attention of layer l - 1
- * when the routed documents' rows (B * k average documents over a ~50 GB/s host
- * link) are expected to cross the bus faster than the next layer's router keys
- * stream from HBM: it then runs beside the next routing alone.  The
- * results equal those calls made one after the other, bit for bit.  The
- * copy-stream work is joined back into `stream` before the call's last
- * attention, so work enqueued later on `stream` sees every output.
+ * pos_offset.  Per layer l the call enqueues msa_route_topk (agg MAX),
+ * msa_gather_kv of the routed documents into one of two staging areas in ws,
+ * and msa_sparse_attend over the staged documents and the local keys, on two
+ * streams joined by events, in one of two orders:
+ *   - when the routed documents' rows (B * k average documents over a ~50 GB/s
+ *     host link) are expected to cross the bus faster than the next layer's
+ *     router keys stream from HBM: `stream` carries the router queries of
+ *     all layers, then the scans one after the other, each on all SMs but 8;
+ *     `copy_stream`, after an event on a layer's scan, its top-k kernels, the
+ *     gather and the attention, which run beside the next layer's scan.  Two
+ *     routing workspaces in ws alternate between layers;
+ *   - otherwise: `stream` carries each layer's routing and, after the routing
+ *     of layer l + 1 and an event on the gather, the attention of layer l;
+ *     `copy_stream` the gather of each layer, after an event on its routing.
+ * The results equal those calls made one after the other, bit for bit.  The
+ * copy-stream work is joined back into `stream` before the call returns, so
+ * work enqueued later on `stream` sees every output.
  * copy_stream may be NULL or equal to stream (no overlap; same results).
  *   capacity_chunks  staging rows per layer (>= the chunks of the B * k routed
  *                    documents; a selection needing more stages what fits and
  *                    raises device error bit 1, as msa_gather_kv).
- *   ws        >= msa_tiered_workspace_size(...) bytes, 256-byte aligned; holds the
- *             routing and attention workspaces and the two staging areas.
- * The call keeps three CUDA events per host thread and device (created by its
+ *   ws        >= msa_tiered_workspace_size(dims, n_layers, ...) bytes, 256-byte
+ *             aligned; holds each layer's router-query rows, two routing workspaces,
+ *             the attention workspace and the two staging areas.
+ * msa_tiered_workspace_size returns 0 for arguments outside the limits below.
+ * The call keeps six CUDA events per host thread and device (created by its
  * first call on that device from that thread: make that call before any stream
  * capture).  Limits: those of msa_route_topk, msa_gather_kv and
  * msa_sparse_attend with q_tokens = 1; 1 <= n_layers <= 4096.
@@ -470,8 +477,8 @@ typedef struct {
   void* out;
 } msa_layer;
 
-size_t msa_tiered_workspace_size(const msa_dims* dims, int32_t B, int32_t n_docs, int32_t n_chunks, int32_t k,
-                                 int32_t t_loc_max, int32_t pos_offset, int32_t capacity_chunks);
+size_t msa_tiered_workspace_size(const msa_dims* dims, int32_t n_layers, int32_t B, int32_t n_docs, int32_t n_chunks,
+                                 int32_t k, int32_t t_loc_max, int32_t pos_offset, int32_t capacity_chunks);
 msa_status msa_tiered_decode(const msa_dims* dims, const msa_layer* layers, int32_t n_layers, int32_t B,
                              const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks, int32_t k,
                              const int32_t* loc_len, int32_t t_loc_max, int32_t pos_offset, int32_t capacity_chunks,

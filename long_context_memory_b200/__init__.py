@@ -98,7 +98,7 @@ def _load():
         "msa_rope_rows": (I32, [DP, P, I32, I32, P, P]),
         "msa_kv_append": (I32, [DP, P, P, P, P, I32, I32, P, I32, P]),
         "msa_gather_kv": (I32, [DP, P, P, I32, P, I32, P, I32, I32, P, P, I32, P, P, P, SZ, P]),
-        "msa_tiered_workspace_size": (SZ, [DP, I32, I32, I32, I32, I32, I32, I32]),
+        "msa_tiered_workspace_size": (SZ, [DP, I32, I32, I32, I32, I32, I32, I32, I32]),
         "msa_sparse_attend_share": (I32, [DP, P, I32, I32, P, P, P, I32, I32, I32, P, I32, I32, P, P, P, I32, I32, P, I32, F,
                                           P, P, P, SZ, P]),
         "msa_attend_merge": (I32, [P, P, I32, I32, I32, P, P]),
@@ -373,9 +373,9 @@ def tiered_layers(layers):
     return arr
 
 
-def tiered_workspace_size(dims, B: int, n_docs: int, n_chunks: int, k: int, t_loc_max: int, pos_offset: int,
-                          capacity_chunks: int) -> int:
-    return int(lib.msa_tiered_workspace_size(ctypes.byref(Dims.of(dims)), B, n_docs, n_chunks, k, t_loc_max,
+def tiered_workspace_size(dims, n_layers: int, B: int, n_docs: int, n_chunks: int, k: int, t_loc_max: int,
+                          pos_offset: int, capacity_chunks: int) -> int:
+    return int(lib.msa_tiered_workspace_size(ctypes.byref(Dims.of(dims)), n_layers, B, n_docs, n_chunks, k, t_loc_max,
                                              pos_offset, capacity_chunks))
 
 
@@ -384,17 +384,18 @@ def tiered_decode(dims, layers, B: int, chunk_off, n_chunks: int, k: int, loc_le
     """Route, gather (host tier) and attend for several independent layer instances in one call.
 
     ``layers``: the array from ``tiered_layers`` (or a list of dicts, converted here).  Per layer the
-    routing runs on ``stream`` (default: the current stream), the gather of the routed documents
-    from pinned host memory on ``copy_stream`` (None: on ``stream``, no overlap), and the attention
-    over the staged documents and the rotated local cache on ``stream``; outputs land in each
-    layer's topk_idx, topk_score and out tensors."""
+    routing, the gather of the routed documents from pinned host memory and the attention over the
+    staged documents and the rotated local cache are split between ``stream`` (default: the current
+    stream) and ``copy_stream`` (None: everything on ``stream``, no overlap) as msa_tiered_decode
+    describes; outputs land in each layer's topk_idx, topk_score and out tensors, ordered before
+    later work on ``stream``."""
     arr = layers if isinstance(layers, ctypes.Array) else tiered_layers(layers)
     n_docs = chunk_off.numel() - 1
     dd = Dims.of(dims)
     if ws is not None:  # the library checks the caller's buffer against what it needs
         nbytes = max(0, ws.numel() * ws.element_size() - 256)
     else:
-        nbytes = tiered_workspace_size(dims, B, n_docs, n_chunks, k, t_loc_max, pos_offset, capacity_chunks)
+        nbytes = tiered_workspace_size(dims, len(arr), B, n_docs, n_chunks, k, t_loc_max, pos_offset, capacity_chunks)
         ws = _workspace(nbytes, chunk_off.device, ws)
     _check(lib.msa_tiered_decode(ctypes.byref(dd), arr, len(arr), B, _ptr(chunk_off), n_docs, n_chunks, k, _ptr(loc_len),
                                  t_loc_max, pos_offset, capacity_chunks, _aligned_ptr(ws), nbytes, _stream(stream),

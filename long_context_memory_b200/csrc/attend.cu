@@ -50,6 +50,7 @@ constexpr int kMaxStages = 4;
 constexpr int kMaxK = 256;
 constexpr int kMaxSplits = 1024;
 constexpr int kChunksPerDocEst = 40;  // expected pooled chunks per selected document (split planning only)
+constexpr int kLatencyGroups = 8;     // (query, token group)s up to which the split plan is one wave
 constexpr int kCoSmemMax = 4096;      // chunk_off entries the split kernel may keep in shared memory
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -121,12 +122,14 @@ struct AttnSmem {
   }
 };
 
-template <int D>
+// TABLE: the local keys are rotated in registers with the RoPE rows of p.rope_tab (a cache of
+// unrotated keys); without it they are used as stored (a cache of rotated keys)
+template <int D, bool TABLE>
 __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) {
   constexpr int KS = D / 16;
   constexpr int NBLK = D / 8;
   const int n_kv = p.n_kv, G = p.n_q / n_kv;
-  const bool table = p.rope_tab != nullptr;  // local keys still need their global rotation
+  constexpr bool table = TABLE;  // local keys still need their global rotation
   const AttnSmem L_(n_kv, D, p.n_stages, table);
   extern __shared__ __align__(128) uint8_t sm[];
   // offsets: every region below starts on a 16-byte boundary (stage rows, query rows and
@@ -361,6 +364,10 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
   const int n_compute = 32 * n_kv;
   int gt = 0;
   bool failed = false;  // a wait of this warp gave up: the compute warps leave together at the next item
+  // the query fragments stay in registers from one item to the next of the same (query, token
+  // group): a CTA that takes several items of one query rotates its query once
+  uint32_t qa[KS][4];
+  int frag_b = -1, frag_t0 = -1;
   for (int it = blockIdx.x, j = 0; it < n_items; it += gridDim.x, ++j) {
     const int hb = j & 1;
     failed |= !warp_wait(&hfull[hb], (j >> 1) & 1, &abort_flag);
@@ -369,15 +376,14 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
     const int* hd = hdr + hb * 8;
     const int b = hd[0], t0 = hd[1], nt = hd[2], L = hd[3];
     const uint16_t* qsm_b = qsm + hb * q_elems;
-    // ---- query fragments of this warp's GQA group: mma row = tt * G + gg (token t0 + tt,
-    //      q head h * G + gg); token t sits at pos_offset + L - M + t; scale, bf16 ----
-    const int64_t pos_q0 = (int64_t)p.pos_offset + L - p.q_tokens + t0;
-    for (int i = tid; i < nt * (D / 2); i += n_compute)
-      qcs[i] = rope_cos_sin(p.turns, i % (D / 2), pos_q0 + i / (D / 2));
-    named_bar_sync(1, n_compute);
     const int g = lane >> 2, c = lane & 3;
-    uint32_t qa[KS][4];
-    {
+    if (b != frag_b || t0 != frag_t0) {  // block-uniform
+      // ---- query fragments of this warp's GQA group: mma row = tt * G + gg (token t0 + tt,
+      //      q head h * G + gg); token t sits at pos_offset + L - M + t; scale, bf16 ----
+      const int64_t pos_q0 = (int64_t)p.pos_offset + L - p.q_tokens + t0;
+      for (int i = tid; i < nt * (D / 2); i += n_compute)
+        qcs[i] = rope_cos_sin(p.turns, i % (D / 2), pos_q0 + i / (D / 2));
+      named_bar_sync(1, n_compute);
   #pragma unroll
       for (int s = 0; s < KS; ++s) {
   #pragma unroll
@@ -386,30 +392,29 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
           const int tt = row / G, gg = row - tt * G;
           const uint16_t* qb = qsm_b + ((size_t)tt * p.n_q + h * G + gg) * D;
   #pragma unroll
-          for (int hk = 0; hk < 2; ++hk) {      // k cols 2c.. and 2c+8..
-            const int dim = 16 * s + 8 * hk + 2 * c;
-            float v[2] = {0.f, 0.f};
+          for (int hk = 0; hk < 2; ++hk) {      // k cols 2c.. and 2c+8..: dims d0 and d0 + 1, one half
+            const int d0 = 16 * s + 8 * hk + 2 * c;
+            float v0 = 0.f, v1 = 0.f;
             if (tt < nt) {
-  #pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const int dd = dim + e;
-                const bool first = dd < D / 2;
-                const int i = first ? dd : dd - D / 2;
-                const int partner = first ? dd + D / 2 : dd - D / 2;
-                const float x = bf16_bits_to_float(qb[dd]);
-                const float y = bf16_bits_to_float(qb[partner]);
-                const float2 cs = qcs[tt * (D / 2) + i];
-                // first half: x cos - y sin; second half: x cos + y sin (y = first-half partner)
-                const float rot = first ? (x * cs.x - y * cs.y) : (x * cs.x + y * cs.y);
-                v[e] = rot * p.scale_log2;
-              }
+              const bool first = d0 < D / 2;
+              const int i0 = first ? d0 : d0 - D / 2;
+              const int p0 = first ? d0 + D / 2 : d0 - D / 2;
+              const float2 x = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(qb + d0));
+              const float2 y = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(qb + p0));
+              const float4 cs = *reinterpret_cast<const float4*>(qcs + tt * (D / 2) + i0);  // cos, sin of i0, i0 + 1
+              // first half: x cos - y sin; second half: x cos + y sin (y = first-half partner)
+              const float r0 = first ? (x.x * cs.x - y.x * cs.y) : (x.x * cs.x + y.x * cs.y);
+              const float r1 = first ? (x.y * cs.z - y.y * cs.w) : (x.y * cs.z + y.y * cs.w);
+              v0 = r0 * p.scale_log2;
+              v1 = r1 * p.scale_log2;
             }
-            qa[s][rr + 2 * hk] = pack_bf16x2(v[0], v[1]);
+            qa[s][rr + 2 * hk] = pack_bf16x2(v0, v1);
           }
         }
       }
+      frag_b = b;
+      frag_t0 = t0;
     }
-
 
     if (it >= n_loc_items && !waited) {  // the first selected-chunk item: its fragments are ready
       pdl_enter();
@@ -452,48 +457,49 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
       const uint32_t vbase = kbase + L_.kbytes;
       const float2* tab = reinterpret_cast<const float2*>(kst + 2 * L_.kbytes);
 
-      // ---- K fragments (B operand, keys = n) ----
-      uint32_t kb[KS][2][2];
+      // ---- S = q K^T (rows = heads, cols = 16 keys), k-steps in pairs (s, s + KS/2): the pair
+      //      holds dims i and i + D/2, which the RoPE of a local key mixes; only one pair's K
+      //      fragments (B operand, keys = n) are live at a time ----
+      float sc[2][4];
+  #pragma unroll
+      for (int nb = 0; nb < 2; ++nb) sc[nb][0] = sc[nb][1] = sc[nb][2] = sc[nb][3] = 0.f;
       {
         const int key = (lane & 7) + 8 * (lane >> 4);
         const int dsel = 8 * ((lane >> 3) & 1);
   #pragma unroll
-        for (int s = 0; s < KS; ++s)
-          ldmatrix_x4(kb[s][0][0], kb[s][0][1], kb[s][1][0], kb[s][1][1], kbase + key * L_.krow + (16 * s + dsel) * 2);
-      }
-      // ---- rotate local keys in registers (pairs i, i + D/2 sit in ksteps s, s + KS/2) ----
-      if (table) {
+        for (int sp = 0; sp < KS / 2; ++sp) {
+          uint32_t kx[2][2], ky[2][2];  // [nb][hk] of k-steps sp and sp + KS/2
+          ldmatrix_x4(kx[0][0], kx[0][1], kx[1][0], kx[1][1], kbase + key * L_.krow + (16 * sp + dsel) * 2);
+          ldmatrix_x4(ky[0][0], ky[0][1], ky[1][0], ky[1][1],
+                      kbase + key * L_.krow + (16 * (sp + KS / 2) + dsel) * 2);
+          if (table) {  // rotate local keys in registers
   #pragma unroll
-        for (int nb = 0; nb < 2; ++nb) {
-          const int r = 8 * nb + g;
-          const int v = tv0 + r;
-          if (v >= n_sel && v < v1) {
-            const float2* trow = tab + r * (D / 2);
+            for (int nb = 0; nb < 2; ++nb) {
+              const int r = 8 * nb + g;
+              const int v = tv0 + r;
+              if (v >= n_sel && v < v1) {
+                const float2* trow = tab + r * (D / 2);
   #pragma unroll
-            for (int s = 0; s < KS / 2; ++s) {
-  #pragma unroll
-              for (int hk = 0; hk < 2; ++hk) {
-                const int i = 16 * s + 8 * hk + 2 * c;
-                const float4 cs = *reinterpret_cast<const float4*>(trow + i);  // (cos_i, sin_i, cos_i+1, sin_i+1)
-                const float2 x = unpack_bf16x2(kb[s][nb][hk]);
-                const float2 y = unpack_bf16x2(kb[s + KS / 2][nb][hk]);
-                const float x0 = x.x * cs.x - y.x * cs.y, y0 = y.x * cs.x + x.x * cs.y;
-                const float x1 = x.y * cs.z - y.y * cs.w, y1 = y.y * cs.z + x.y * cs.w;
-                kb[s][nb][hk] = pack_bf16x2(x0, x1);
-                kb[s + KS / 2][nb][hk] = pack_bf16x2(y0, y1);
+                for (int hk = 0; hk < 2; ++hk) {
+                  const int i = 16 * sp + 8 * hk + 2 * c;
+                  const float4 cs = *reinterpret_cast<const float4*>(trow + i);  // (cos_i, sin_i, cos_i+1, sin_i+1)
+                  const float2 x = unpack_bf16x2(kx[nb][hk]);
+                  const float2 y = unpack_bf16x2(ky[nb][hk]);
+                  const float x0 = x.x * cs.x - y.x * cs.y, y0 = y.x * cs.x + x.x * cs.y;
+                  const float x1 = x.y * cs.z - y.y * cs.w, y1 = y.y * cs.z + x.y * cs.w;
+                  kx[nb][hk] = pack_bf16x2(x0, x1);
+                  ky[nb][hk] = pack_bf16x2(y0, y1);
+                }
               }
             }
           }
+  #pragma unroll
+          for (int nb = 0; nb < 2; ++nb) {
+            mma_bf16_16816(sc[nb], qa[sp][0], qa[sp][1], qa[sp][2], qa[sp][3], kx[nb][0], kx[nb][1]);
+            mma_bf16_16816(sc[nb], qa[sp + KS / 2][0], qa[sp + KS / 2][1], qa[sp + KS / 2][2], qa[sp + KS / 2][3],
+                           ky[nb][0], ky[nb][1]);
+          }
         }
-      }
-      // ---- S = q K^T (rows = heads, cols = 16 keys) ----
-      float sc[2][4];
-  #pragma unroll
-      for (int nb = 0; nb < 2; ++nb) {
-        sc[nb][0] = sc[nb][1] = sc[nb][2] = sc[nb][3] = 0.f;
-  #pragma unroll
-        for (int s = 0; s < KS; ++s)
-          mma_bf16_16816(sc[nb], qa[s][0], qa[s][1], qa[s][2], qa[s][3], kb[s][nb][0], kb[s][nb][1]);
       }
   #pragma unroll
       for (int nb = 0; nb < 2; ++nb)
@@ -971,16 +977,21 @@ size_t attend_workspace(const msa_dims& d, int B, int M, int k, int t_loc_max, i
   AttendWs w{};
   const int mt = tokens_per_cta(d, M);
   const int n_tg = (M + mt - 1) / mt;
-  // splits per (query, token group): a total that makes the item count a whole number of
-  // waves, shared between the local keys and the selected chunks in proportion to their
-  // expected key counts (the selection's size is known only on the device: about
-  // kChunksPerDocEst chunks per selected document), each side at least one split
-  const int n_total = std::max(2, choose_splits(B * n_tg, t_loc_max, k));
+  // splits per (query, token group), shared between the local keys and the selected chunks in
+  // proportion to their expected key counts (the selection's size is known only on the device:
+  // about kChunksPerDocEst chunks per selected document), each side at least one split.  Few
+  // query groups (latency): one wave, an item per CTA, so that each CTA pays an item's setup
+  // (its header, the rotated query fragments, the first tile's round trip) once.  Otherwise a
+  // total that makes the item count a whole number of waves.
+  const int groups = B * n_tg;
+  const bool latency = groups <= kLatencyGroups;
+  const int max_useful = std::max(2, std::min((t_loc_max + 16 * k) / 32, kMaxSplits));
+  const int n_total = latency ? std::max(2, std::min(sm_count() / groups, max_useful))
+                              : std::max(2, choose_splits(groups, t_loc_max, k));
   const double sel_est = (double)kChunksPerDocEst * k;
   int n_chunk = (int)std::lround(n_total * sel_est / (sel_est + std::max(0, t_loc_max)));
-  // one wave or less (few queries: latency): the selected chunks, which wait for the routing,
-  // in splits of about one 16-key tile
-  const bool latency = (long long)n_total * B * n_tg <= sm_count();
+  // latency: the selected chunks, which wait for the routing, in splits of about one 16-key tile
+  // of the estimate (an underestimate of the selection still leaves them a few tiles each)
   if (latency) n_chunk = std::max(n_chunk, (int)std::ceil(sel_est / 16.0));
   n_chunk = std::max(1, std::min({n_chunk, (latency ? 4 : 2) * k, n_total - 1}));
   w.n_split_chunk = n_chunk;
@@ -1074,11 +1085,12 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
                          const void* V_loc, const void* k_new, const void* v_new, const int32_t* loc_len,
                          int t_loc_max, int pos_offset,
                          const void* rope_cache, int k_loc_rotated, float scale, int phase, int early, void* out,
-                         void* ws, cudaStream_t s, const AttendShare* share) {
+                         void* ws, cudaStream_t s, const AttendShare* share, int max_ctas) {
   AttendWs w;
   attend_workspace(d, B, M, k, t_loc_max, pos_offset, ws, &w);
   const int n_loc = w.n_split_local, n_chk = w.n_split_chunk;
   const int D = d.head_dim;
+  const bool side = max_ctas > 0;
   const bool local_keys = phase != 2 && (!share || share->local_keys);
   const float2* tab = (k_loc_rotated || !local_keys) ? nullptr : static_cast<const float2*>(rope_cache);
   if (!tab && !k_loc_rotated && local_keys && t_loc_max > 0) {
@@ -1133,17 +1145,19 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
   p.n_stages = stages_that_fit(d.n_kv, d.n_q, D, tab != nullptr, p.tok_per_cta, p.co_cap);
   {
     TraceScope ts(kKAttnSplit, s);
-    // persistent: each CTA takes items (split, query, token group) in turn
+    // persistent: each CTA takes items (split, query, token group) in turn.  The results do not
+    // depend on the grid (an item's partial is the same whichever CTA computes it): max_ctas caps
+    // it for a launch that runs beside other work on a few SMs, where fewer CTAs that each
+    // pipeline many items beat many that each pay an item's setup; such a launch is in plain
+    // stream order
     const int n_items = (p.n_loc_splits + p.n_chunk_splits) * B * p.n_tgroups;
-    dim3 grid(std::max(1, std::min(n_items, sm_count())));
+    const int cap = side ? std::min(max_ctas, sm_count()) : sm_count();
+    dim3 grid(std::max(1, std::min(n_items, cap)));
     const size_t sm = AttnSmem(d.n_kv, D, p.n_stages, tab != nullptr).total(d.n_q, D, p.tok_per_cta, p.co_cap);
-    if (D == 128) {
-      MSA_CUDA_CHECK(set_max_dynamic_smem(reinterpret_cast<const void*>(attn_split_kernel<128>), (int)sm));
-      MSA_CUDA_CHECK(launch_pdl(attn_split_kernel<128>, grid, dim3(32 * (d.n_kv + 1)), sm, s, p));
-    } else {
-      MSA_CUDA_CHECK(set_max_dynamic_smem(reinterpret_cast<const void*>(attn_split_kernel<64>), (int)sm));
-      MSA_CUDA_CHECK(launch_pdl(attn_split_kernel<64>, grid, dim3(32 * (d.n_kv + 1)), sm, s, p));
-    }
+    auto kern = D == 128 ? (tab ? attn_split_kernel<128, true> : attn_split_kernel<128, false>)
+                         : (tab ? attn_split_kernel<64, true> : attn_split_kernel<64, false>);
+    MSA_CUDA_CHECK(set_max_dynamic_smem(reinterpret_cast<const void*>(kern), (int)sm));
+    MSA_CUDA_CHECK(launch_ordered(!side, kern, grid, dim3(32 * (d.n_kv + 1)), sm, s, p));
   }
   if (phase != 1) {  // the local-keys phase leaves its partials for the selected-chunks phase's combine
     TraceScope ts(kKAttnCombine, s);
@@ -1151,16 +1165,20 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
     // many: a warp per head, 8 per CTA
     const long long rows = (long long)B * M * d.n_q;
     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
+    // (beside other work: a CTA per head; every output is summed in the same order either way)
     if (rows < 2LL * sm_count()) {
-      dim3 grid(d.n_q, B * M, D / 32);
-      auto kern = D == 128 ? attn_combine_kernel<128, 4> : attn_combine_kernel<64, 2>;
-      MSA_CUDA_CHECK(launch_pdl(kern, grid, dim3(256), 0, s, (const float*)w.part_ml, (const float*)w.part_o,
-                                p.n_parts, o, share ? share->o : nullptr, share ? share->lse2 : nullptr));
+      dim3 grid(d.n_q, B * M, side ? 1 : D / 32);
+      auto kern = D == 128 ? (side ? attn_combine_kernel<128, 1> : attn_combine_kernel<128, 4>)
+                           : (side ? attn_combine_kernel<64, 1> : attn_combine_kernel<64, 2>);
+      MSA_CUDA_CHECK(launch_ordered(!side, kern, grid, dim3(256), 0, s, (const float*)w.part_ml,
+                                    (const float*)w.part_o, p.n_parts, o, share ? share->o : nullptr,
+                                    share ? share->lse2 : nullptr));
     } else {
       dim3 grid((unsigned)((rows + 7) / 8));
       auto kern = D == 128 ? attn_combine_warp_kernel<128> : attn_combine_warp_kernel<64>;
-      MSA_CUDA_CHECK(launch_pdl(kern, grid, dim3(256), 0, s, (const float*)w.part_ml, (const float*)w.part_o,
-                                p.n_parts, (int)rows, o, share ? share->o : nullptr, share ? share->lse2 : nullptr));
+      MSA_CUDA_CHECK(launch_ordered(!side, kern, grid, dim3(256), 0, s, (const float*)w.part_ml,
+                                    (const float*)w.part_o, p.n_parts, (int)rows, o, share ? share->o : nullptr,
+                                    share ? share->lse2 : nullptr));
     }
   }
   return MSA_OK;

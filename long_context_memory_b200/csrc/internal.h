@@ -111,9 +111,14 @@ void rope_turns(const msa_dims& d, uint64_t* f /* [head_dim / 2] */);
 // Launch with programmatic stream serialization: the kernel may be scheduled
 // while the previous kernel on the stream finishes; every kernel launched this
 // way calls pdl_wait() before its first global-memory access.
+// Launch with programmatic dependent launch (early: the kernel may start while its predecessor
+// on the stream runs, and waits for it inside, pdl_enter) or in plain stream order (the kernel
+// starts once its predecessor has completed; its pdl_enter then returns at once).  A kernel that
+// runs beside other work on a few SMs is launched in plain order: started early, its CTAs would
+// sit on SMs, waiting, that the other work needs.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                       Args&&... args) {
+cudaError_t launch_ordered(bool early, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                           Args&&... args) {
   prefer_shared_carveout(reinterpret_cast<const void*>(kernel));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -124,8 +129,14 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = early ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  return launch_ordered(true, kernel, grid, block, smem, s, std::forward<Args>(args)...);
 }
 
 // the same with thread-block clusters of cluster_x CTAs along x
@@ -157,10 +168,32 @@ size_t route_workspace(const msa_dims& d, int B, int M, int n_docs, int n_chunks
                        void* ws, struct RouteWs* out);
 msa_status kr_norms_launch(const msa_dims& d, const void* KR_bar, int n_chunks, int kr_layout, float* inv_norm,
                            cudaStream_t s);
+// Which kernels of the routing a call enqueues: all of them; the scoring part (router query and
+// scan, and the top-k when the scan's last CTA selects it); the scan alone, on router-query rows
+// (q_ext) that route_query_launch wrote earlier; or the remaining top-k kernels.  The parts may go
+// to different streams: the selection reads only the workspace, chunk_off and the output
+// pointers, after the scoring has completed.
+enum class RoutePart { kAll, kScore, kScan, kSelect };
+
+// scan_sm_reserve: SMs the scan leaves free (its grid is the SM count minus this), for work that
+// runs beside it on another stream
 msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int B, int M, const void* KR_bar,
                         const int32_t* chunk_off, int n_docs, int n_chunks, int k, msa_doc_agg agg, int kr_layout,
                         const float* kr_inv_norm, float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws,
-                        cudaStream_t s, bool early_inputs = false);
+                        cudaStream_t s, bool early_inputs = false, RoutePart part = RoutePart::kAll,
+                        int scan_sm_reserve = 0, const void* q_ext = nullptr);
+
+// The router query alone: Q^R rows of B x M query tokens into q_hl (route_query_bytes), in the
+// layout the scan reads; clears n_clear words at `clear` and n_tickets tickets (either may be
+// null) after its wait on the predecessor.
+size_t route_query_bytes(const msa_dims& d, int B, int M);
+msa_status route_query_launch(const msa_dims& d, const void* Hq, const void* W_QR, int B, int M, void* q_hl,
+                              uint32_t* clear, size_t n_clear, uint32_t* tickets, int n_tickets, cudaStream_t s,
+                              bool early_inputs);
+// The words a routing workspace (MAX aggregation) needs zeroed before its scan: the tickets and
+// the document keys, one contiguous region.
+void route_clear_region(const msa_dims& d, int B, int M, int n_docs, int n_chunks, int k, void* ws, void** ptr,
+                        size_t* bytes);
 
 msa_status validate_route(const msa_dims* dims, const void* Hq, const void* W_QR, int32_t B, int32_t q_tokens,
                           const void* KR_bar, const int32_t* chunk_off, int32_t n_docs, int32_t n_chunks, int32_t k,
@@ -186,15 +219,16 @@ msa_status attend_launch(const msa_dims& d, const void* q, int B, int M, const v
                          const void* K_loc, const void* V_loc, const void* k_new, const void* v_new,
                          const int32_t* loc_len, int t_loc_max,
                          int pos_offset, const void* rope_cache, int k_loc_rotated, float scale, int phase,
-                         int early, void* out, void* ws, cudaStream_t s, const AttendShare* share = nullptr);
+                         int early, void* out, void* ws, cudaStream_t s, const AttendShare* share = nullptr,
+                         int max_ctas = 0);
 msa_status attend_merge_launch(const float* o_parts, const float* lse2_parts, int R, int n_rows, int D, void* out,
                                cudaStream_t s);
 msa_status gather_kv_launch(const msa_dims& d, const void* K_host, const void* V_host, const int32_t* chunk_off,
                             int n_docs, const int32_t* topk_idx, int B, int k, void* K_stage, void* V_stage,
                             int capacity_chunks, int32_t* stage_off, int32_t* stage_idx, int32_t* stage_src,
                             cudaStream_t s);
-size_t tiered_workspace_size(const msa_dims& d, int B, int n_docs, int n_chunks, int k, int t_loc_max, int pos_offset,
-                             int capacity);
+size_t tiered_workspace_size(const msa_dims& d, int n_layers, int B, int n_docs, int n_chunks, int k, int t_loc_max,
+                             int pos_offset, int capacity);
 msa_status tiered_launch(const msa_dims& d, const msa_layer* layers, const void* const* K_dev, const void* const* V_dev,
                          int n_layers, int B, const int32_t* chunk_off, int n_docs, int n_chunks, int k,
                          const int32_t* loc_len, int t_loc_max, int pos_offset, int capacity, void* ws,

@@ -670,10 +670,12 @@ static bool tiered_sizes_ok(const msa_dims* dims, int32_t B, int32_t n_docs, int
          dims->n_kv >= 1 && dims->n_q >= dims->n_kv && dims->n_r >= 1 && dims->d_r >= 1;
 }
 
-size_t msa_tiered_workspace_size(const msa_dims* dims, int32_t B, int32_t n_docs, int32_t n_chunks, int32_t k,
-                                 int32_t t_loc_max, int32_t pos_offset, int32_t capacity_chunks) {
-  if (!tiered_sizes_ok(dims, B, n_docs, n_chunks, k, t_loc_max, pos_offset, capacity_chunks)) return 0;
-  return tiered_workspace_size(*dims, B, n_docs, n_chunks, k, t_loc_max, pos_offset, capacity_chunks);
+size_t msa_tiered_workspace_size(const msa_dims* dims, int32_t n_layers, int32_t B, int32_t n_docs, int32_t n_chunks,
+                                 int32_t k, int32_t t_loc_max, int32_t pos_offset, int32_t capacity_chunks) {
+  if (n_layers < 1 || n_layers > 4096 ||
+      !tiered_sizes_ok(dims, B, n_docs, n_chunks, k, t_loc_max, pos_offset, capacity_chunks))
+    return 0;
+  return tiered_workspace_size(*dims, n_layers, B, n_docs, n_chunks, k, t_loc_max, pos_offset, capacity_chunks);
 }
 
 msa_status msa_tiered_decode(const msa_dims* dims, const msa_layer* layers, int32_t n_layers, int32_t B,
@@ -717,7 +719,8 @@ msa_status msa_tiered_decode(const msa_dims* dims, const msa_layer* layers, int3
     st = mapped_host(L.V_bar_host, "V_bar_host", &V_dev[l]);
     if (st != MSA_OK) return st;
   }
-  const size_t need = tiered_workspace_size(*dims, B, n_docs, n_chunks, k, t_loc_max, pos_offset, capacity_chunks);
+  const size_t need =
+      tiered_workspace_size(*dims, n_layers, B, n_docs, n_chunks, k, t_loc_max, pos_offset, capacity_chunks);
   if (ws_bytes < need) return fail(MSA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u))
     return fail(MSA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");

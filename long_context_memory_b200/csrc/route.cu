@@ -36,7 +36,8 @@
 namespace msa {
 
 struct RouteWs {
-  uint32_t* scan_ticket;  // scan CTAs finished (fused top-k); zeroed by the router query kernel
+  uint32_t* scan_ticket;  // [1 + B]: scan CTAs finished (fused top-k), then per query its slices
+                          // finished (fused merge); zeroed by the router query kernel
   __nv_bfloat16* q_hl; // [passes][n_r][2][NQ][d_r] normalised query, bf16 hi and lo terms
   uint32_t* doc_key;  // [B][n_docs] ordered-uint32 doc max (MAX)
   uint32_t* chunk_k;  // [B][n_chunks] ordered chunk scores (MEAN)
@@ -84,8 +85,9 @@ size_t rq_smem_bytes(int d_r) {
   return (size_t)kRqPiece * rq_w_stride(d_r) + 16 * (size_t)rq_h_stride() + 16 * (size_t)d_r * sizeof(float);
 }
 
-__device__ __forceinline__ void rq_clear(uint32_t* clear, size_t n_clear, uint32_t* scan_ticket) {
-  if (scan_ticket && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *scan_ticket = 0u;
+__device__ __forceinline__ void rq_clear(uint32_t* clear, size_t n_clear, uint32_t* scan_ticket, int n_tickets) {
+  if (scan_ticket && blockIdx.x == 0 && blockIdx.y == 0)
+    for (int i = threadIdx.x; i < n_tickets; i += blockDim.x) scan_ticket[i] = 0u;
   if (clear) {
     const size_t cta = (size_t)blockIdx.y * gridDim.x + blockIdx.x, n_cta = (size_t)gridDim.x * gridDim.y;
     for (size_t i = cta * blockDim.x + threadIdx.x; i < n_clear; i += n_cta * blockDim.x) clear[i] = 0u;
@@ -106,7 +108,7 @@ __device__ __forceinline__ void rq_store_row(__nv_bfloat16* q_hl, int b, int h, 
 __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
     const __nv_bfloat16* __restrict__ Hq, const __nv_bfloat16* __restrict__ W, int B, int b_pad, int hidden,
     int n_r, int d_r, int nq, int split_rows, __nv_bfloat16* __restrict__ q_hl, uint32_t* __restrict__ clear,
-    size_t n_clear, uint32_t* __restrict__ scan_ticket, int early) {
+    size_t n_clear, uint32_t* __restrict__ scan_ticket, int n_tickets, int early) {
   extern __shared__ __align__(16) uint8_t rq_smem[];
   __shared__ float wsum[kRqThreads / 32];
   // early: H_q, W^QR and the memory the scan reads (K̄^R, its norms, chunk_off) were final
@@ -115,7 +117,7 @@ __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
   bool waited = !early;
   if (waited) {
     pdl_enter();
-    rq_clear(clear, n_clear, scan_ticket);
+    rq_clear(clear, n_clear, scan_ticket, n_tickets);
   } else {
     pdl_launch_dependents();
   }
@@ -208,7 +210,7 @@ __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
       __syncthreads();
       if (!waited) {  // every thread, before its first write
         pdl_wait();
-        rq_clear(clear, n_clear, scan_ticket);
+        rq_clear(clear, n_clear, scan_ticket, n_tickets);
         waited = true;
       }
       if (q < 2) {
@@ -227,7 +229,7 @@ __global__ void __launch_bounds__(kRqThreads) router_query_kernel(
 // Q^R given directly (W_QR == NULL): normalise each row of head h, write the hi/lo terms
 __global__ void __launch_bounds__(kRqThreads) router_query_direct_kernel(
     const __nv_bfloat16* __restrict__ Hq, int B, int b_pad, int n_r, int d_r, int nq, __nv_bfloat16* __restrict__ q_hl,
-    uint32_t* __restrict__ clear, size_t n_clear, uint32_t* __restrict__ scan_ticket, int early) {
+    uint32_t* __restrict__ clear, size_t n_clear, uint32_t* __restrict__ scan_ticket, int n_tickets, int early) {
   __shared__ float invn[kRqThreads / 32];
   if (!early) pdl_enter();  // early: H_q is read before the wait, the writes come after it
   else pdl_launch_dependents();
@@ -256,7 +258,7 @@ __global__ void __launch_bounds__(kRqThreads) router_query_direct_kernel(
       if (lane + 32 * e < d_r) rq_store_row(q_hl, b, h, lane + 32 * e, v[e] * sc, n_r, d_r, nq);
   }
   if (early && warp >= b_pad) pdl_wait();  // warps with no rows
-  rq_clear(clear, n_clear, scan_ticket);
+  rq_clear(clear, n_clear, scan_ticket, n_tickets);
 }
 
 // --------------------------------------------------------------------------
@@ -980,14 +982,47 @@ __device__ void slice_topk(const uint32_t* doc_key, const uint32_t* chunk_k, con
   __syncthreads();  // shared memory free for the next call
 }
 
+__device__ void merge_topk(const uint64_t* cand, int n_slices, int k, int32_t* topk_idx, float* topk_score, int b,
+                           uint64_t* sm64);
+
+// top-k of one slice of documents for query blockIdx.y; with several slices and merge_ticket set
+// (their candidates fit in one slice's keys), the slice that finishes last for its query also
+// merges the query's candidates (a ticket per query), sparing the merge kernel
 __global__ void __launch_bounds__(kTopkThreads) topk_slice_kernel(
     const uint32_t* __restrict__ doc_key, const uint32_t* __restrict__ chunk_k, const int32_t* __restrict__ chunk_off,
     int n_docs, int n_chunks, int k, int n_slices, float* __restrict__ doc_scores, uint64_t* __restrict__ cand,
-    int32_t* __restrict__ topk_idx, float* __restrict__ topk_score) {
+    int32_t* __restrict__ topk_idx, float* __restrict__ topk_score, uint32_t* __restrict__ merge_ticket) {
   extern __shared__ uint64_t sm64[];
+  __shared__ bool last;
   pdl_enter();
   slice_topk(doc_key, chunk_k, chunk_off, n_docs, n_chunks, k, n_slices, doc_scores, cand, topk_idx, topk_score,
              blockIdx.x, blockIdx.y, sm64);
+  if (!merge_ticket || n_slices == 1) return;
+  const int b = blockIdx.y;
+  __threadfence();  // this slice's candidates are visible before its ticket
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(&merge_ticket[b], 1u) == (uint32_t)(n_slices - 1);
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  if (threadIdx.x == 0) merge_ticket[b] = 0u;  // ready for the next call (also cleared by the router query)
+  merge_topk(cand, n_slices, k, topk_idx, topk_score, b, sm64);
+}
+
+// the global top-k of query b from its slices' winners (n_slices * k keys in shared memory first)
+__device__ void merge_topk(const uint64_t* cand, int n_slices, int k, int32_t* topk_idx, float* topk_score, int b,
+                           uint64_t* sm64) {
+  const int n = n_slices * k;
+  uint64_t* keys = sm64;
+  const TopkScratch ts(keys + n);
+  uint64_t* out = ts.out;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) keys[i] = __ldcg(&cand[(size_t)b * n + i]);
+  __syncthreads();
+  block_topk(keys, n, k, ts);
+  for (int i = threadIdx.x; i < k; i += blockDim.x) {
+    topk_idx[(size_t)b * k + i] = (int32_t)(0xFFFFFFFFu - (uint32_t)(out[i] & 0xFFFFFFFFu));
+    topk_score[(size_t)b * k + i] = ordered_to_float((uint32_t)(out[i] >> 32));
+  }
 }
 
 __global__ void __launch_bounds__(kTopkThreads) topk_merge_kernel(const uint64_t* __restrict__ cand,
@@ -995,19 +1030,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_merge_kernel(const uint64_t
                                                                   int32_t* __restrict__ topk_idx,
                                                                   float* __restrict__ topk_score) {
   extern __shared__ uint64_t sm64[];
-  const int n = n_slices * k;
-  uint64_t* keys = sm64;
-  const TopkScratch ts(keys + n);
-  uint64_t* out = ts.out;
   pdl_enter();
-  const int b = blockIdx.x;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) keys[i] = cand[(size_t)b * n + i];
-  __syncthreads();
-  block_topk(keys, n, k, ts);
-  for (int i = threadIdx.x; i < k; i += blockDim.x) {
-    topk_idx[(size_t)b * k + i] = (int32_t)(0xFFFFFFFFu - (uint32_t)(out[i] & 0xFFFFFFFFu));
-    topk_score[(size_t)b * k + i] = ordered_to_float((uint32_t)(out[i] >> 32));
-  }
+  merge_topk(cand, n_slices, k, topk_idx, topk_score, blockIdx.x, sm64);
 }
 
 // exact top-k of (score, global document id) candidate pairs, one block per query
@@ -1123,8 +1147,8 @@ size_t route_workspace(const msa_dims& d, int B, int M, int n_docs, int n_chunks
   w.nq = R <= 16 ? 16 : 32;
   w.passes = (R + w.nq - 1) / w.nq;
   w.n_slices = (n_docs + kSliceDocs - 1) / kSliceDocs;
-  w.scan_ticket = cv.take<uint32_t>(1);
   w.q_hl = cv.take<__nv_bfloat16>((size_t)w.passes * d.n_r * 2 * w.nq * d.d_r);
+  w.scan_ticket = cv.take<uint32_t>(1 + (size_t)B);  // the tickets, then the document keys: one region
   w.doc_key = agg == MSA_AGG_MAX ? cv.take<uint32_t>((size_t)B * n_docs) : nullptr;
   w.chunk_k = agg == MSA_AGG_MEAN ? cv.take<uint32_t>((size_t)B * n_chunks) : nullptr;
   w.cand = w.n_slices > 1 ? cv.take<uint64_t>((size_t)B * w.n_slices * k) : nullptr;
@@ -1132,10 +1156,45 @@ size_t route_workspace(const msa_dims& d, int B, int M, int n_docs, int n_chunks
   return cv.size();
 }
 
+size_t route_query_bytes(const msa_dims& d, int B, int M) {
+  const int R = B * M, nq = R <= 16 ? 16 : 32;
+  return (size_t)((R + nq - 1) / nq) * d.n_r * 2 * nq * d.d_r * sizeof(__nv_bfloat16);
+}
+
+void route_clear_region(const msa_dims& d, int B, int M, int n_docs, int n_chunks, int k, void* ws, void** ptr,
+                        size_t* bytes) {
+  RouteWs w;
+  route_workspace(d, B, M, n_docs, n_chunks, k, MSA_AGG_MAX, ws, &w);
+  *ptr = w.scan_ticket;
+  *bytes = (size_t)(reinterpret_cast<char*>(w.doc_key + (size_t)B * n_docs) - reinterpret_cast<char*>(w.scan_ticket));
+}
+
+msa_status route_query_launch(const msa_dims& d, const void* Hq, const void* W_QR, int B, int M, void* q_hl,
+                              uint32_t* clear, size_t n_clear, uint32_t* tickets, int n_tickets, cudaStream_t s,
+                              bool early_inputs) {
+  const int R = B * M, nq = R <= 16 ? 16 : 32, passes = (R + nq - 1) / nq;
+  __nv_bfloat16* q = static_cast<__nv_bfloat16*>(q_hl);
+  TraceScope ts(kKRouterQuery, s);
+  if (W_QR) {
+    const size_t sm = rq_smem_bytes(d.d_r);
+    MSA_CUDA_CHECK(set_max_dynamic_smem(reinterpret_cast<const void*>(router_query_kernel), (int)sm));
+    MSA_CUDA_CHECK(launch_pdl_cluster(router_query_kernel, dim3(kRqCluster, d.n_r), dim3(kRqThreads), sm, s,
+                                      kRqCluster, static_cast<const __nv_bfloat16*>(Hq),
+                                      static_cast<const __nv_bfloat16*>(W_QR), R, passes * nq, d.hidden, d.n_r, d.d_r,
+                                      nq, rq_split_rows(d.hidden), q, clear, n_clear, tickets, n_tickets,
+                                      early_inputs ? 1 : 0));
+  } else {
+    MSA_CUDA_CHECK(launch_pdl(router_query_direct_kernel, dim3(1, d.n_r), dim3(kRqThreads), 0, s,
+                              static_cast<const __nv_bfloat16*>(Hq), R, passes * nq, d.n_r, d.d_r, nq, q, clear,
+                              n_clear, tickets, n_tickets, early_inputs ? 1 : 0));
+  }
+  return MSA_OK;
+}
+
 msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int B, int M, const void* KR_bar,
                         const int32_t* chunk_off, int n_docs, int n_chunks, int k, msa_doc_agg agg, int kr_layout,
                         const float* kr_inv_norm, float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws, cudaStream_t s,
-                        bool early_inputs) {
+                        bool early_inputs, RoutePart part, int scan_sm_reserve, const void* q_ext) {
   RouteWs w;
   route_workspace(d, B, M, n_docs, n_chunks, k, agg, ws, &w);
   const int NR = d.n_r * d.d_r;
@@ -1147,26 +1206,17 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
   // few queries over one slice of documents: the scan's last CTA runs the top-k itself
   const bool fuse_topk = w.n_slices == 1 && w.passes == 1 && B <= kFuseTopkMaxQueries;
   const size_t n_clear = clear ? (size_t)B * (mean ? n_chunks : n_docs) : 0;
+  const bool score = part != RoutePart::kSelect, select = part != RoutePart::kScore;
 
   // K1: router query (projection, normalisation, hi/lo layout) and document keys cleared
-  {
-    TraceScope ts(kKRouterQuery, s);
-    if (W_QR) {
-      const size_t sm = rq_smem_bytes(d.d_r);
-      MSA_CUDA_CHECK(set_max_dynamic_smem(reinterpret_cast<const void*>(router_query_kernel), (int)sm));
-      MSA_CUDA_CHECK(launch_pdl_cluster(router_query_kernel, dim3(kRqCluster, d.n_r), dim3(kRqThreads), sm, s,
-                                        kRqCluster, static_cast<const __nv_bfloat16*>(Hq),
-                                        static_cast<const __nv_bfloat16*>(W_QR), R, w.passes * w.nq, d.hidden, d.n_r,
-                                        d.d_r, w.nq, rq_split_rows(d.hidden), w.q_hl, clear, n_clear,
-                                        w.scan_ticket, early_inputs ? 1 : 0));
-    } else {
-      MSA_CUDA_CHECK(launch_pdl(router_query_direct_kernel, dim3(1, d.n_r), dim3(kRqThreads), 0, s,
-                                static_cast<const __nv_bfloat16*>(Hq), R, w.passes * w.nq, d.n_r, d.d_r, w.nq,
-                                w.q_hl, clear, n_clear, w.scan_ticket, early_inputs ? 1 : 0));
-    }
+  if (score && part != RoutePart::kScan) {
+    msa_status st = route_query_launch(d, Hq, W_QR, B, M, w.q_hl, clear, n_clear, w.scan_ticket, 1 + B, s,
+                                       early_inputs);
+    if (st != MSA_OK) return st;
   }
+  const void* q_src = part == RoutePart::kScan ? q_ext : w.q_hl;
   // K3: scan, NQ (16 or 32) queries per pass
-  {
+  if (score) {
     CUtensorMap kmap, qmap;
     msa_status st;
     if (kr_layout == 1) {  // head-major [n_r][C][d_r]: one head's rows are contiguous
@@ -1186,11 +1236,11 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
     const uint64_t qdims[2] = {(uint64_t)d.d_r, (uint64_t)w.passes * d.n_r * 2 * w.nq};
     const uint64_t qstrides[1] = {(uint64_t)d.d_r * 2};
     const uint32_t qbox[2] = {64, (uint32_t)w.nq};
-    st = encode_tensor_map(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w.q_hl, qdims, qstrides, qbox,
-                           CU_TENSOR_MAP_SWIZZLE_128B);
+    st = encode_tensor_map(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q_src), qdims, qstrides,
+                           qbox, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != MSA_OK) return st;
     const int n_tiles = (n_chunks + kScanM - 1) / kScanM;
-    const int grid = std::max(1, std::min(sm_count(), n_tiles));
+    const int grid = std::max(1, std::min(sm_count() - std::max(0, scan_sm_reserve), n_tiles));
     uint32_t cols = 32;
     // columns: 2 NQ per head (hi and lo side by side), two tiles in flight for NQ = 16, one for 32
     while (cols < (w.nq == 16 ? 2u : 1u) * d.n_r * 2u * w.nq) cols <<= 1;
@@ -1222,16 +1272,20 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
       if (e != cudaSuccess) return cuda_fail(e, "scan_kernel launch");
     }
   }
-  // K4: top-k
+  // K4: top-k; the slices' winners merged by the last slice of each query when they fit in one
+  // slice's keys, otherwise by the merge kernel
+  const bool fuse_merge = w.n_slices > 1 && (size_t)w.n_slices * k <= (size_t)kSliceDocs;
+  if (!select) return MSA_OK;
   if (!fuse_topk) {
     TraceScope ts(kKTopkSlice, s);
     const size_t sm = topk_slice_smem();
     MSA_CUDA_CHECK(set_max_dynamic_smem(reinterpret_cast<const void*>(topk_slice_kernel), (int)sm));
     MSA_CUDA_CHECK(launch_pdl(topk_slice_kernel, dim3(w.n_slices, B), dim3(kTopkThreads), sm, s,
                               (const uint32_t*)w.doc_key, (const uint32_t*)w.chunk_k, chunk_off, n_docs, n_chunks, k,
-                              w.n_slices, doc_scores, w.cand, topk_idx, topk_score));
+                              w.n_slices, doc_scores, w.cand, topk_idx, topk_score,
+                              fuse_merge ? w.scan_ticket + 1 : nullptr));
   }
-  if (w.n_slices > 1) {
+  if (w.n_slices > 1 && !fuse_merge) {
     TraceScope ts(kKTopkMerge, s);
     const size_t sm = topk_merge_smem(w.n_slices * k);
     MSA_CUDA_CHECK(set_max_dynamic_smem(reinterpret_cast<const void*>(topk_merge_kernel), (int)sm));

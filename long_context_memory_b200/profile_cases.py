@@ -278,8 +278,8 @@ class TieredCase:
             self.per_layer.append(x)
         self.capacity = B * self.k * self.max_doc_chunks  # the largest possible selection
         self.arr = msa.tiered_layers(self.per_layer)
-        self.ws = torch.empty(msa.tiered_workspace_size(d, B, self.n_docs, self.C, self.k, self.t_loc, self.pos,
-                                                        self.capacity) + 256, dtype=torch.uint8, device=dev)
+        self.ws = torch.empty(msa.tiered_workspace_size(d, L, B, self.n_docs, self.C, self.k, self.t_loc,
+                                                        self.pos, self.capacity) + 256, dtype=torch.uint8, device=dev)
         torch.cuda.synchronize()
 
     def run(self, stream=None, copy_stream=None, arr=None):

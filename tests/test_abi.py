@@ -223,7 +223,7 @@ def _tiered(msa, dims, layers=None, n_layers=1, B=1, n_docs=10, n_chunks=20, k=4
                 setattr(L, f, FAKE)
             for f, v in ptrs.items():
                 setattr(L, f, v)
-    need = msa.lib.msa_tiered_workspace_size(ctypes.byref(dd), B, n_docs, n_chunks, k, t_loc, pos, cap)
+    need = msa.lib.msa_tiered_workspace_size(ctypes.byref(dd), max(1, n_layers), B, n_docs, n_chunks, k, t_loc, pos, cap)
     if ws_bytes is None:
         ws_bytes = need
     return msa.lib.msa_tiered_decode(ctypes.byref(dd), layers, n_layers, B, FAKE, n_docs, n_chunks, k, FAKE, t_loc, pos,
@@ -246,11 +246,15 @@ def test_tiered_validation(msa):
     assert _tiered(msa, ok, K_bar_host=None) == 1
     assert _tiered(msa, ok, k_new=FAKE) == 1                 # k_new without v_new
     dd = ctypes.byref(msa.Dims.of(ok))
-    small = msa.lib.msa_tiered_workspace_size(dd, 1, 10, 20, 4, 16, 4, 64)
-    big = msa.lib.msa_tiered_workspace_size(dd, 1, 10, 20, 4, 16, 4, 128)
+    small = msa.lib.msa_tiered_workspace_size(dd, 1, 1, 10, 20, 4, 16, 4, 64)
+    big = msa.lib.msa_tiered_workspace_size(dd, 1, 1, 10, 20, 4, 16, 4, 128)
     # two staging areas of K and V rows (n_kv * head_dim bf16 each) per extra chunk of capacity
     assert small > 0 and big - small >= 4 * 64 * 8 * 128 * 2 - 4 * 256
-    assert msa.lib.msa_tiered_workspace_size(dd, 1, 10, 20, 4, 16, 4, 0) == 0
+    assert msa.lib.msa_tiered_workspace_size(dd, 1, 1, 10, 20, 4, 16, 4, 0) == 0
+    # each layer adds its router-query rows: n_r heads x (hi, lo) x 16 padded rows x d_r bf16
+    more = msa.lib.msa_tiered_workspace_size(dd, 3, 1, 10, 20, 4, 16, 4, 64)
+    assert more - small == 2 * 8 * 2 * 16 * 128 * 2
+    assert msa.lib.msa_tiered_workspace_size(dd, 0, 1, 10, 20, 4, 16, 4, 64) == 0
 
 
 def test_workspace_sizes_grow_with_problem(msa):

@@ -47,13 +47,19 @@ def _rotated_cache(msa, d, K_loc_bits, pos_offset, device):
     return K
 
 
-@pytest.mark.parametrize("B,n_layers,copy", [(1, 3, True), (3, 4, True), (2, 3, False)])
-def test_tiered_decode_equals_single_calls_and_oracle(msa, cuda_device, B, n_layers, copy):
+# Few documents: the transfers are the longer part and the gather of each layer starts as soon as
+# its routing is done.  5,000 short documents at B = 1: the scans are the longer part, so the router
+# queries of every layer run first, the scans follow one another, and the selections (two slices
+# of documents, merged by the last slice CTA), gathers and attentions run on the copy stream; the
+# two routing workspaces are reused and cleared between layers.
+@pytest.mark.parametrize("B,n_layers,copy,n_docs,max_len", [(1, 3, True, 120, 3000), (3, 4, True, 120, 3000),
+                                                             (2, 3, False, 120, 3000), (1, 5, True, 5000, 600)])
+def test_tiered_decode_equals_single_calls_and_oracle(msa, cuda_device, B, n_layers, copy, n_docs, max_len):
     import torch
 
     dev, d, k, t_loc = cuda_device, DIMS, 16, 300
     rng = np.random.default_rng(500 + 10 * B + n_layers)
-    lens = rng.integers(1, 3000, size=120)
+    lens = rng.integers(1, max_len, size=n_docs)
     doc_off = W.offsets_from_lengths(lens)
     co, *_ = O.chunk_layout(doc_off)
     C, n_docs = int(co[-1]), len(lens)
