@@ -278,21 +278,26 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
         hd[7] = is_chunk ? p.chunk_part_base + split : split;  // the item's partial slot
         mbar_arrive(&hsel[hb]);  // releases the key-range writes
       }
-      if (p.k_new && !is_chunk) {
-        if (v1 == L && v1 > v0) {
-          // the item holding the query's last local row writes the new token there first (no
-          // other item reads that row): key rotated at its position (or as given), value copied;
-          // then orders the writes before its bulk copies read the row back
-          const int slot = L - 1;
-          const size_t src = (size_t)b * n_kv * D;
-          const size_t dst = ((size_t)b * p.t_loc_max + slot) * n_kv * D;
-          __nv_bfloat16* kd = const_cast<__nv_bfloat16*>(p.K_loc) + dst;
-          __nv_bfloat16* vd = const_cast<__nv_bfloat16*>(p.V_loc) + dst;
-          for (int e = lane; e < n_kv * (D / 2); e += 32) {
-            const int hh = e / (D / 2), i = e % (D / 2);
+      // the item holding the query's last local row writes the new token there (no other item
+      // reads that row) just before it requests that row's tile, so that its earlier tiles stream
+      // meanwhile: key rotated at its position (or as given), value copied; then orders the writes
+      // before its bulk copies read the row back.  A lane rotates dims i and i + D/2 of every KV
+      // head with one angle.
+      const bool appends = p.k_new && !is_chunk && v1 == L && v1 > v0;
+      if (p.k_new && !is_chunk && !appends && L == 0 && split == 0 && lane == 0)
+        raise_dev_error(kDevErrBadIndex);  // no local position to take the new token
+      auto append_token = [&]() {
+        const int slot = L - 1;
+        const size_t src = (size_t)b * n_kv * D;
+        const size_t dst = ((size_t)b * p.t_loc_max + slot) * n_kv * D;
+        __nv_bfloat16* kd = const_cast<__nv_bfloat16*>(p.K_loc) + dst;
+        __nv_bfloat16* vd = const_cast<__nv_bfloat16*>(p.V_loc) + dst;
+        for (int i = lane; i < D / 2; i += 32) {
+          const float2 cs = p.append_rotate ? rope_cos_sin(p.turns, i, (int64_t)p.pos_offset + slot)
+                                            : make_float2(1.f, 0.f);
+          for (int hh = 0; hh < n_kv; ++hh) {
             const __nv_bfloat16* kr = p.k_new + src + (size_t)hh * D;
             if (p.append_rotate) {
-              const float2 cs = rope_cos_sin(p.turns, i, (int64_t)p.pos_offset + slot);
               const float x1 = __bfloat162float(kr[i]), x2 = __bfloat162float(kr[i + D / 2]);
               kd[(size_t)hh * D + i] = __float2bfloat16_rn(x1 * cs.x - x2 * cs.y);
               kd[(size_t)hh * D + i + D / 2] = __float2bfloat16_rn(x2 * cs.x + x1 * cs.y);
@@ -301,14 +306,12 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
               kd[(size_t)hh * D + i + D / 2] = kr[i + D / 2];
             }
           }
-          for (int e = lane; e < n_kv * D / 8; e += 32)
-            reinterpret_cast<uint4*>(vd)[e] = __ldg(reinterpret_cast<const uint4*>(p.v_new + src) + e);
-          fence_proxy_async_global();
-          __syncwarp();
-        } else if (L == 0 && split == 0 && lane == 0) {
-          raise_dev_error(kDevErrBadIndex);  // no local position to take the new token
         }
-      }
+        for (int e = lane; e < n_kv * D / 8; e += 32)
+          reinterpret_cast<uint4*>(vd)[e] = __ldg(reinterpret_cast<const uint4*>(p.v_new + src) + e);
+        fence_proxy_async_global();
+        __syncwarp();
+      };
       // ---- the item's tiles: kTK keys each, a bulk copy per key and tensor plus the RoPE rows ----
       for (int t = 0; t < n_tiles; ++t, ++gt) {
         const int st = gt % L_.n_stages;
@@ -316,6 +319,7 @@ __global__ void __launch_bounds__(288, 1) attn_split_kernel(const AttnParams p) 
           stop = true;
           break;
         }
+        if (appends && t == n_tiles - 1) append_token();  // the last tile holds row L - 1
         const int tv0 = v0 + t * kTK;
         const int rows = min(kTK, v1 - tv0);
         const int n_chunk_rows = max(0, min(rows, n_sel - tv0));

@@ -368,6 +368,8 @@ def main():
     ap.add_argument("--kr-layout", choices=["chunk", "head"], default="chunk")
     ap.add_argument("--norms", action="store_true", help="route cases: pass precomputed key norms")
     ap.add_argument("--layers", type=int, default=2, help="tiered case: layer instances per call")
+    ap.add_argument("--one-stream", action="store_true", help="tiered case: every kernel on one stream (no "
+                    "copy stream: each kernel has the whole GPU)")
     a = ap.parse_args()
     dev = torch.device("cuda:0")
     seed = W.BASE_SEED + 7
@@ -390,7 +392,7 @@ def main():
         case = EncodeCase(a.tokens or 1_000_000, seed, dev)
     s = torch.cuda.Stream()
     if a.case == "tiered":  # the gather on its own stream, as a decode loop runs it
-        cs = torch.cuda.Stream()
+        cs = None if a.one_stream else torch.cuda.Stream()
         tcase = case
         case = type("Run", (), {"run": staticmethod(lambda: tcase.run(s, cs))})
     with torch.cuda.stream(s):
