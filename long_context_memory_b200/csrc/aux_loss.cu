@@ -70,7 +70,7 @@ struct AuxSmem {
   static constexpr int kRowBytes = 8 * DR * 2;  // room for 8 router heads
   static constexpr int kStageBytes = kAuxRows * kRowBytes;
   static constexpr int kLanePad = DR / 4 + 4;   // a lane's DR/4 values + 4 floats of padding
-  static constexpr int kSlice = 32 * kLanePad;  // >= 8 * DR
+  static constexpr int kSlice = 32 * kLanePad;  // >= 8 * DR, >= 32 * (DR / 4 + 1)
   static constexpr int kQBytes = 8 * DR * 2;    // one query row (room for 8 router heads)
   static __host__ __device__ size_t bytes(int nk, int stages) {
     return (size_t)stages * kStageBytes + 2 * kQBytes + (size_t)nk * 8 * 4 * 2 + (size_t)nk * 4 + 16 +
@@ -393,17 +393,21 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
       __syncwarp();  // the slice is read before the next row is staged
     }
     if (p.dQ != nullptr) {
+      // this warp's dq partial in its slice: element lane * V + o of the row at lane * V +
+      // (o + lane) % V, so that the lanes' stores of one o fall in distinct banks (a lane's V
+      // values would otherwise start in the same bank for every lane)
       if (hl) {
 #pragma unroll
         for (int e = 0; e < V; ++e)
-          red[(size_t)warp * Sm::kSlice + lane * V + unit_of_slot<DR>(e / 8, lane) * 8 + e % 8] = acc[e];
+          slice[lane * V + ((unit_of_slot<DR>(e / 8, lane) * 8 + e % 8 + lane) & (V - 1))] = acc[e];
       }
       aux_bar_sync();
       for (int e = ct; e < NR; e += 32 * kAuxCompute) {
         const int hh = e / DR;
+        const int se = (e & ~(V - 1)) + ((e + e / V) & (V - 1));  // where element e of a partial sits
         float v = 0.f;
 #pragma unroll
-        for (int w = 0; w < kAuxCompute; ++w) v += red[(size_t)w * Sm::kSlice + e];
+        for (int w = 0; w < kAuxCompute; ++w) v += red[(size_t)w * Sm::kSlice + se];
         const float nqs = qn[hh], nqa = fabsf(nqs);
         if (nqs > 0.f) v -= chead[hh] * inv_nr * bf16_bits_to_float(qrow[e]) / (nqa * nqa);
         p.dQ[(size_t)i * NR + e] = v;

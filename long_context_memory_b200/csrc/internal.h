@@ -176,12 +176,20 @@ msa_status kr_norms_launch(const msa_dims& d, const void* KR_bar, int n_chunks, 
 enum class RoutePart { kAll, kScore, kScan, kSelect };
 
 // scan_sm_reserve: SMs the scan leaves free (its grid is the SM count minus this), for work that
-// runs beside it on another stream
+// runs beside it on another stream.  after_scan (with kScan): the kernel before this scan on the
+// stream is another routing's scan, which writes nothing this routing reads or writes, and every
+// input of this routing was final when that scan started: the scan then does not wait for it.
 msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int B, int M, const void* KR_bar,
                         const int32_t* chunk_off, int n_docs, int n_chunks, int k, msa_doc_agg agg, int kr_layout,
                         const float* kr_inv_norm, float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws,
                         cudaStream_t s, bool early_inputs = false, RoutePart part = RoutePart::kAll,
-                        int scan_sm_reserve = 0, const void* q_ext = nullptr);
+                        int scan_sm_reserve = 0, const void* q_ext = nullptr, const int32_t* chunk_doc = nullptr,
+                        bool after_scan = false);
+
+// Each chunk's document id (-1 outside the documents) from chunk_off: the scan's epilogue then
+// reads a row's document instead of searching chunk_off for it (chunk_doc argument of
+// route_launch).  A property of the layout, computed once for many scans over it.
+msa_status chunk_doc_launch(const int32_t* chunk_off, int n_docs, int n_chunks, int32_t* chunk_doc, cudaStream_t s);
 
 // The router query alone: Q^R rows of B x M query tokens into q_hl (route_query_bytes), in the
 // layout the scan reads; clears n_clear words at `clear` and n_tickets tickets (either may be

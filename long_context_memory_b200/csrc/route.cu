@@ -301,6 +301,8 @@ struct ScanParams {
   int q_base, q_count, pass;
   int head_major;  // K̄^R stored [n_r][C][d_r] instead of [C][n_r][d_r]
   const float* inv_norm;  // [C][n_r] 1 / max(||K̄^R_jh||, eps) precomputed, or null (norm warps compute it)
+  const int32_t* chunk_doc;  // [C] each chunk's document (-1: none), or null (searched in chunk_off)
+  int wait_prior;  // 0: the kernel before this one on the stream writes nothing this scan reads or writes
   uint32_t tmem_cols;
   float inv_nr;
 };
@@ -342,38 +344,65 @@ __device__ __forceinline__ void scan_epilogue(const ScanParams& p, int q4, int q
   const int row = 32 * q4 + lane;  // chunk within the tile
   const bool active = q_off < p.q_count;
   int cur = 0;                     // lower bound for this warp's document search
+  // With a chunk -> document map the rows' documents and inverse norms of the next tile are
+  // loaded while this one is processed (one tile ahead); without it each tile searches chunk_off.
+  const bool mapped = !MEAN && p.chunk_doc != nullptr;  // (the mean needs no document boundaries)
+  int doc_next = -1;
+  float invg_next[8];
+  auto fetch = [&](int lt_f) {
+    const int jr = (t_begin + lt_f) * kScanM + row;
+    doc_next = (active && jr < p.n_chunks) ? __ldg(&p.chunk_doc[jr]) : -1;
+#pragma unroll
+    for (int hh = 0; hh < 8; ++hh)
+      invg_next[hh] = (p.inv_norm && active && hh < n_r && jr < p.n_chunks) ? __ldg(&p.inv_norm[(size_t)jr * n_r + hh])
+                                                                            : 0.f;
+  };
+  if (mapped && n_lt > 0) fetch(0);
   for (int lt = 0; lt < n_lt; ++lt) {
     const int tile = t_begin + lt;
     const int nbuf = lt & 1;                                    // norm buffer
     const int buf = lt % Gm::kBufs, use = lt / Gm::kBufs;      // TMEM buffer
     const int jrow = tile * kScanM + row;
-    // documents of this warp's 32 rows, found before the accumulators are ready (they depend
-    // on the tile alone): a warp-wide 32-ary search for the first row's document, then one
-    // lookahead of 32 document boundaries (32 consecutive rows cross at most 31 of them)
     const int j = tile * kScanM + row;
-    const int j0 = tile * kScanM + 32 * q4;
     int doc = -1;
-    if (active && j0 < p.n_chunks) {
-      int lo = cur, hi = p.n_docs;  // answer in [lo, hi): largest d with chunk_off[d] <= j0
-      while (hi - lo > 1) {
-        const int step = (hi - lo + 31) >> 5;
-        const int probe = lo + lane * step;
-        const bool ok = probe < hi && __ldg(&p.chunk_off[probe]) <= j0;
-        const unsigned m = __ballot_sync(0xffffffffu, ok);
-        const int L = 31 - __clz(m);  // lane 0 always qualifies (chunk_off[lo] <= j0)
-        lo = lo + L * step;
-        hi = min(hi, lo + step);
-      }
-      const int d0 = lo;
-      const int bi = d0 + 1 + lane;
-      const int bnd = bi <= p.n_docs ? __ldg(&p.chunk_off[bi]) : 0x7fffffff;
+    float invg[8];  // precomputed inverse norms of this row (loads in flight during the waits)
+    if (mapped) {
+      doc = doc_next;
+#pragma unroll
+      for (int hh = 0; hh < 8; ++hh) invg[hh] = invg_next[hh];
+      if (lt + 1 < n_lt) fetch(lt + 1);
+    } else {
+      // documents of this warp's 32 rows, found before the accumulators are ready (they depend
+      // on the tile alone): a warp-wide 32-ary search for the first row's document, then one
+      // lookahead of 32 document boundaries (32 consecutive rows cross at most 31 of them)
+      const int j0 = tile * kScanM + 32 * q4;
+      if (active && j0 < p.n_chunks) {
+        int lo = cur, hi = p.n_docs;  // answer in [lo, hi): largest d with chunk_off[d] <= j0
+        while (hi - lo > 1) {
+          const int step = (hi - lo + 31) >> 5;
+          const int probe = lo + lane * step;
+          const bool ok = probe < hi && __ldg(&p.chunk_off[probe]) <= j0;
+          const unsigned m = __ballot_sync(0xffffffffu, ok);
+          const int L = 31 - __clz(m);  // lane 0 always qualifies (chunk_off[lo] <= j0)
+          lo = lo + L * step;
+          hi = min(hi, lo + step);
+        }
+        const int d0 = lo;
+        const int bi = d0 + 1 + lane;
+        const int bnd = bi <= p.n_docs ? __ldg(&p.chunk_off[bi]) : 0x7fffffff;
 #pragma unroll 4
-      for (int r = 0; r < 32; ++r) {
-        const unsigned m = __ballot_sync(0xffffffffu, bnd <= j0 + r);
-        if (lane == r) doc = d0 + __popc(m);
+        for (int r = 0; r < 32; ++r) {
+          const unsigned m = __ballot_sync(0xffffffffu, bnd <= j0 + r);
+          if (lane == r) doc = d0 + __popc(m);
+        }
+        if (j >= p.n_chunks) doc = -1;
+        cur = d0;
       }
-      if (j >= p.n_chunks) doc = -1;
-      cur = d0;
+      if (p.inv_norm) {
+#pragma unroll
+        for (int hh = 0; hh < 8; ++hh)
+          invg[hh] = (active && hh < n_r && jrow < p.n_chunks) ? __ldg(&p.inv_norm[(size_t)jrow * n_r + hh]) : 0.f;
+      }
     }
     const int prev = __shfl_up_sync(0xffffffffu, doc, 1);
     const bool head = (lane == 0) || (prev != doc);
@@ -384,12 +413,7 @@ __device__ __forceinline__ void scan_epilogue(const ScanParams& p, int q4, int q
       const int od = __shfl_down_sync(0xffffffffu, doc, 1 << e);
       if (lane + (1 << e) < 32 && od == doc) same |= 1u << e;
     }
-    float invg[8];  // precomputed inverse norms of this row (loads in flight during the waits)
-    if (p.inv_norm) {
-#pragma unroll
-      for (int hh = 0; hh < 8; ++hh)
-        invg[hh] = (active && hh < n_r && jrow < p.n_chunks) ? __ldg(&p.inv_norm[(size_t)jrow * n_r + hh]) : 0.f;
-    } else if (!warp_wait(&nfull[nbuf], (lt >> 1) & 1, abort)) {
+    if (!p.inv_norm && !warp_wait(&nfull[nbuf], (lt >> 1) & 1, abort)) {
       return;
     }
     if (!warp_wait(&tfull[buf], use & 1, abort)) return;
@@ -538,7 +562,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   const int n_pre = min(S, n_it);
   if (warp == 0 && lane == 0)
     for (int it = 0; it < n_pre; ++it) load_keys(it);
-  pdl_enter();
+  // A scan that follows another routing's scan on the stream (the caller's guarantee: that scan
+  // writes another workspace, and everything this one reads was final before it started) does
+  // not wait for it: its CTAs stream as soon as they land, beside the other scan's last tiles.
+  if (p.wait_prior) pdl_enter();
+  else pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------- TMA producer -------------------------
@@ -1156,6 +1184,32 @@ size_t route_workspace(const msa_dims& d, int B, int M, int n_docs, int n_chunks
   return cv.size();
 }
 
+namespace {
+// each chunk's document: one warp per document writes its id over its chunks; chunks outside
+// [chunk_off[0], chunk_off[n_docs]) get -1
+__global__ void __launch_bounds__(256) chunk_doc_kernel(const int32_t* __restrict__ chunk_off, int n_docs,
+                                                        int n_chunks, int32_t* __restrict__ chunk_doc) {
+  pdl_enter();
+  const int lane = threadIdx.x & 31;
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  for (int d = gw; d < n_docs; d += warps) {
+    const int c0 = max(0, __ldg(&chunk_off[d])), c1 = min(n_chunks, __ldg(&chunk_off[d + 1]));
+    for (int c = c0 + lane; c < c1; c += 32) chunk_doc[c] = d;
+  }
+  const int lo = min(n_chunks, max(0, __ldg(&chunk_off[0]))), hi = max(lo, min(n_chunks, __ldg(&chunk_off[n_docs])));
+  const int t = blockIdx.x * blockDim.x + threadIdx.x, nt = gridDim.x * blockDim.x;
+  for (int c = t; c < lo; c += nt) chunk_doc[c] = -1;
+  for (int c = hi + t; c < n_chunks; c += nt) chunk_doc[c] = -1;
+}
+}  // namespace
+
+msa_status chunk_doc_launch(const int32_t* chunk_off, int n_docs, int n_chunks, int32_t* chunk_doc, cudaStream_t s) {
+  const int blocks = std::max(1, std::min(4 * sm_count(), (n_docs + 7) / 8));
+  MSA_CUDA_CHECK(launch_pdl(chunk_doc_kernel, dim3(blocks), dim3(256), 0, s, chunk_off, n_docs, n_chunks, chunk_doc));
+  return MSA_OK;
+}
+
 size_t route_query_bytes(const msa_dims& d, int B, int M) {
   const int R = B * M, nq = R <= 16 ? 16 : 32;
   return (size_t)((R + nq - 1) / nq) * d.n_r * 2 * nq * d.d_r * sizeof(__nv_bfloat16);
@@ -1194,7 +1248,8 @@ msa_status route_query_launch(const msa_dims& d, const void* Hq, const void* W_Q
 msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int B, int M, const void* KR_bar,
                         const int32_t* chunk_off, int n_docs, int n_chunks, int k, msa_doc_agg agg, int kr_layout,
                         const float* kr_inv_norm, float* doc_scores, int32_t* topk_idx, float* topk_score, void* ws, cudaStream_t s,
-                        bool early_inputs, RoutePart part, int scan_sm_reserve, const void* q_ext) {
+                        bool early_inputs, RoutePart part, int scan_sm_reserve, const void* q_ext,
+                        const int32_t* chunk_doc, bool after_scan) {
   RouteWs w;
   route_workspace(d, B, M, n_docs, n_chunks, k, agg, ws, &w);
   const int NR = d.n_r * d.d_r;
@@ -1265,6 +1320,8 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
       p.pass = pass;
       p.head_major = kr_layout == 1;
       p.inv_norm = kr_inv_norm;
+      p.chunk_doc = chunk_doc;
+      p.wait_prior = (pass == 0 && after_scan) ? 0 : 1;
       p.tmem_cols = cols;
       p.inv_nr = 1.0f / (float)d.n_r;
       TraceScope ts(kKScan, s);

@@ -47,6 +47,7 @@ namespace msa {
 namespace {
 
 struct TieredWs {
+  int32_t* chunk_doc;  // [n_chunks] each chunk's document: the scans' epilogues read it
   uint8_t* q_hl;      // [n_layers][q_bytes] each layer's router-query rows (short transfers)
   size_t q_bytes;
   void* route_ws[2];
@@ -62,6 +63,7 @@ size_t tiered_workspace(const msa_dims& d, int n_layers, int B, int n_docs, int 
                         int pos_offset, int capacity, void* ws, TieredWs* out) {
   Carver cv(ws);
   TieredWs w{};
+  w.chunk_doc = cv.take<int32_t>((size_t)n_chunks);
   w.q_bytes = (route_query_bytes(d, B, 1) + 255) & ~size_t(255);
   w.q_hl = cv.take<uint8_t>((size_t)n_layers * w.q_bytes);
   const size_t r_bytes = route_workspace(d, B, 1, n_docs, n_chunks, k, MSA_AGG_MAX, nullptr, nullptr);
@@ -141,9 +143,13 @@ msa_status tiered_launch(const msa_dims& d, const msa_layer* layers, const void*
   // layer's kernels), so from the second layer on it reads them early
   auto route = [&](int l, RoutePart part, int slot, cudaStream_t st, int reserve) -> msa_status {
     const msa_layer& L = layers[l];
+    // in the short-transfer order the scans follow one another on `stream`: the scan of layer
+    // l > 0 writes the other routing workspace than the scan before it, every input it reads was
+    // final before that scan started (the router queries and the chunk map run first), and the
+    // reuse of its workspace is ordered by the event on the selection two layers back
     return route_launch(d, L.Hq, L.W_QR, B, 1, L.KR_bar, chunk_off, n_docs, n_chunks, k, MSA_AGG_MAX, 0,
                         L.kr_inv_norm, nullptr, L.topk_idx, L.topk_score, w.route_ws[slot], st, l > 0, part,
-                        reserve, w.q_hl + (size_t)l * w.q_bytes);
+                        reserve, w.q_hl + (size_t)l * w.q_bytes, w.chunk_doc, part == RoutePart::kScan && l > 0);
   };
   auto gather = [&](int l, cudaStream_t st) -> msa_status {
     const int slot = l & 1;
@@ -159,7 +165,9 @@ msa_status tiered_launch(const msa_dims& d, const msa_layer* layers, const void*
                          w.stage_idx[slot], k, L.K_loc, L.V_loc, L.k_new, L.v_new, loc_len, t_loc_max, pos_offset,
                          nullptr, 1, 0.0f, 0, early, L.out, w.attend_ws, st, nullptr, max_ctas);
   };
-  msa_status st = MSA_OK;
+  // the layout's chunk -> document map, once for every scan of the call
+  msa_status st = chunk_doc_launch(chunk_off, n_docs, n_chunks, w.chunk_doc, s);
+  if (st != MSA_OK) return st;
   if (!overlap) {  // one stream: each layer's chain in order
     for (int l = 0; l < n_layers && st == MSA_OK; ++l) {
       st = route(l, RoutePart::kAll, 0, s, 0);
