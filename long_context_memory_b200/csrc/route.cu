@@ -602,12 +602,16 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     if (lane == 0) {
       int it = 0;
       bool stop = false;
+      // the tile: this CTA's own first, then one taken from the counter (-1 when none is left).
+      // Each take is issued a tile ahead, so that the atomic's round trip overlaps the loads of
+      // the tile before it.
+      unsigned claim = p.n_tiles > (int)gridDim.x ? atomicAdd(p.tile_ctr, 1u) : 0u;
       for (int lt = 0; !stop; ++lt) {
-        // the tile: this CTA's own first, then one taken from the counter (-1 when none is left)
         int tile = blockIdx.x;
         if (lt > 0) {
-          const long long c = (long long)gridDim.x + atomicAdd(p.tile_ctr, 1u);
+          const long long c = (long long)gridDim.x + claim;
           tile = c < p.n_tiles ? (int)c : -1;
+          if (tile >= 0) claim = atomicAdd(p.tile_ctr, 1u);
         }
         const int sl = lt % kTileSlots;
         if (lt >= kTileSlots && !mbar_wait(&slot_empty[sl], ((lt / kTileSlots) - 1) & 1, &abort_flag)) break;
