@@ -87,39 +87,78 @@ __global__ void transpose_kernel(const uint16_t* __restrict__ in, int K, int N, 
   }
 }
 
-// H̄[c] = mean of the chunk's token rows; one block per chunk, 8 columns per thread per pass
-__global__ void __launch_bounds__(256) pool_h_kernel(const __nv_bfloat16* __restrict__ H, int hidden,
-                                                     const int64_t* __restrict__ tok0,
-                                                     const int32_t* __restrict__ clen,
-                                                     __nv_bfloat16* __restrict__ hbar) {
-  const int c = blockIdx.x;
-  const int64_t t0 = tok0[c];
-  const int n = clen[c];
-  const float inv = 1.0f / (float)n;
-  for (int col = threadIdx.x * 8; col < hidden; col += blockDim.x * 8) {
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    const __nv_bfloat16* src = H + (size_t)t0 * hidden + col;
-    for (int r = 0; r < n; ++r) {
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(src + (size_t)r * hidden));
-      float2 f;
-      f = unpack_bf16x2(w.x); acc[0] += f.x; acc[1] += f.y;
-      f = unpack_bf16x2(w.y); acc[2] += f.x; acc[3] += f.y;
-      f = unpack_bf16x2(w.z); acc[4] += f.x; acc[5] += f.y;
-      f = unpack_bf16x2(w.w); acc[6] += f.x; acc[7] += f.y;
+// H̄[c] = mean of the chunk's token rows, as bf16 hi + lo terms.  Work item = (chunk, slice of
+// kPoolCols columns); persistent: one CTA per SM takes items blockIdx.x, + gridDim.x, ...  Thread
+// 0 streams each item's tile (the chunk's first row and the 63 after it, kPoolCols columns; rows
+// past the chunk are not used, past T zero-filled) by TMA into a 2-stage ring; thread t adds
+// column t of the chunk's rows in row order.  It lets the K-projection GEMM start at once (the
+// GEMM does not read H̄): a pooling CTA (128 threads, 32 KB of shared memory) and a GEMM CTA
+// (192 threads, 214 registers, ~187 KB) fit on one SM together, and the pooling's reads of H go
+// beside the tensor-bound GEMM.
+constexpr int kPoolThreads = 128;
+constexpr int kPoolCols = kPoolThreads;  // one column per thread
+constexpr int kPoolRows = 64;            // rows per tile: a whole chunk
+constexpr int kPoolStageBytes = kPoolRows * kPoolCols * 2;
+constexpr size_t kPoolSmem = 2 * (size_t)kPoolStageBytes + 128;
+__global__ void __launch_bounds__(kPoolThreads) pool_h_kernel(const __grid_constant__ CUtensorMap h_map, int hidden,
+                                                              int n_chunks, const int64_t* __restrict__ tok0,
+                                                              const int32_t* __restrict__ clen,
+                                                              __nv_bfloat16* __restrict__ hbar) {
+  extern __shared__ __align__(128) uint8_t pool_sm_raw[];
+  // a TMA tile's shared-memory destination must start on a 128-byte boundary; the dynamic area
+  // follows this kernel's static variables, so its start is rounded up by hand (kPoolSmem holds
+  // the 128 bytes of slack)
+  uint8_t* pool_sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pool_sm_raw) + 127) & ~uintptr_t(127));
+  __shared__ __align__(8) uint64_t full[2], empty[2];
+  __shared__ int abort_flag;
+  pdl_launch_dependents();  // the GEMM that follows reads nothing this kernel writes
+  const int tid = threadIdx.x;
+  const int n_slices = (hidden + kPoolCols - 1) / kPoolCols;
+  const long long n_items = (long long)n_chunks * n_slices;
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kPoolThreads);
     }
-    uint32_t hi[4], lo[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float m0 = acc[2 * j] * inv, m1 = acc[2 * j + 1] * inv;
-      const float h0 = __bfloat162float(__float2bfloat16_rn(m0));
-      const float h1 = __bfloat162float(__float2bfloat16_rn(m1));
-      hi[j] = pack_bf16x2(h0, h1);
-      lo[j] = pack_bf16x2(m0 - h0, m1 - h1);
-    }
-    __nv_bfloat16* dst = hbar + (size_t)c * 2 * hidden + col;
-    *reinterpret_cast<uint4*>(dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-    *reinterpret_cast<uint4*>(dst + hidden) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&h_map);
   }
+  __syncthreads();
+  auto issue = [&](long long item, int k) {  // item's tile into stage k % 2
+    const int c = (int)(item / n_slices), sl = (int)(item % n_slices);
+    uint64_t* bar = &full[k & 1];
+    mbar_arrive_expect_tx(bar, (uint32_t)kPoolStageBytes);
+    tma_load_2d(pool_sm + (size_t)(k & 1) * kPoolStageBytes, &h_map, bar, sl * kPoolCols, (int)tok0[c]);
+  };
+  long long item = blockIdx.x;
+  int issued = 0;  // tiles requested (thread 0)
+  if (tid == 0 && item < n_items) issue(item, issued++);
+  for (int k = 0; item < n_items; ++k, item += gridDim.x) {
+    // the next item's tile, once every thread is done with the stage it refills
+    const long long nxt = item + gridDim.x;
+    if (tid == 0 && nxt < n_items) {
+      if (k >= 1 && !mbar_wait(&empty[(k + 1) & 1], ((k - 1) >> 1) & 1, &abort_flag)) break;
+      issue(nxt, issued++);
+    }
+    if (!mbar_wait(&full[k & 1], (k >> 1) & 1, &abort_flag)) break;
+    const int c = (int)(item / n_slices), sl = (int)(item % n_slices);
+    const int n = clen[c];
+    const int col = sl * kPoolCols + tid;
+    const uint16_t* t = reinterpret_cast<const uint16_t*>(pool_sm + (size_t)(k & 1) * kPoolStageBytes) + tid;
+    float acc = 0.f;
+    for (int r = 0; r < n; ++r) acc += bf16_bits_to_float(t[r * kPoolCols]);
+    mbar_arrive(&empty[k & 1]);  // this thread has read the stage
+    if (col < hidden) {
+      const float m = acc * (1.0f / (float)n);
+      const __nv_bfloat16 hi = __float2bfloat16_rn(m);
+      __nv_bfloat16* dst = hbar + (size_t)c * 2 * hidden + col;
+      dst[0] = hi;
+      dst[hidden] = __float2bfloat16_rn(m - __bfloat162float(hi));
+    }
+  }
+  // after an abort: the copy this CTA may still have in flight lands before it exits
+  if (abort_flag && tid == 0) mbar_drain_ring(full, 2, issued - 2, issued);
 }
 
 // Sum of v[0..31] over the 32 lanes of a warp, transposed: on return v[0] of
@@ -382,6 +421,10 @@ __global__ void __launch_bounds__(kEncThreads, 1) gemm_kernel(const __grid_const
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+  // launched early beside the chunk pooling (programmatic dependent launch), the K GEMM completes
+  // only after the pooling has: the pooled GEMM after it then reads finished chunk means
+  // (a plain launch returns at once here)
+  pdl_wait();
 }
 
 size_t gemm_smem_bytes(int mode, int bn) {
@@ -393,17 +436,11 @@ size_t gemm_smem_bytes(int mode, int bn) {
 
 template <int MODE>
 cudaError_t launch_gemm(int bn, int grid, size_t smem, cudaStream_t s, const CUtensorMap& ma, const CUtensorMap& mb,
-                        const GemmParams& p) {
-  if (bn == 256) {
-    cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(gemm_kernel<MODE, 256>), (int)smem);
-    if (e != cudaSuccess) return e;
-    gemm_kernel<MODE, 256><<<grid, kEncThreads, smem, s>>>(ma, mb, p);
-  } else {
-    cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(gemm_kernel<MODE, 128>), (int)smem);
-    if (e != cudaSuccess) return e;
-    gemm_kernel<MODE, 128><<<grid, kEncThreads, smem, s>>>(ma, mb, p);
-  }
-  return cudaGetLastError();
+                        const GemmParams& p, bool early = false) {
+  auto kern = bn == 256 ? gemm_kernel<MODE, 256> : gemm_kernel<MODE, 128>;
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch_ordered(early, kern, dim3(grid), dim3(kEncThreads), smem, s, ma, mb, p);
 }
 
 }  // namespace
@@ -472,6 +509,22 @@ msa_status encode_launch(const msa_dims& d, const void* H, int64_t T, const int6
         static_cast<const uint16_t*>(W_KR), hidden, NR, reinterpret_cast<uint16_t*>(w.wvrT), NV);
     MSA_CUDA_CHECK(cudaGetLastError());
   }
+  // ---- H̄ (hi | lo), the chunk means for the pooled projections; the K GEMM runs beside it ----
+  {
+    CUtensorMap hm;
+    const uint64_t hdims[2] = {(uint64_t)hidden, (uint64_t)T};
+    const uint64_t hstr[1] = {(uint64_t)hidden * 2};
+    const uint32_t hbox[2] = {(uint32_t)kPoolCols, (uint32_t)kPoolRows};
+    msa_status st = encode_tensor_map(&hm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(H), hdims, hstr,
+                                      hbox, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != MSA_OK) return st;
+    TraceScope ts(kKEncPoolH, s);
+    const int grid = std::max(1, std::min(sm_count(), n_chunks));
+    MSA_CUDA_CHECK(set_max_dynamic_smem(reinterpret_cast<const void*>(pool_h_kernel), (int)kPoolSmem));
+    MSA_CUDA_CHECK(launch_ordered(false, pool_h_kernel, dim3(grid), dim3(kPoolThreads), kPoolSmem, s, hm, hidden,
+                                  n_chunks, static_cast<const int64_t*>(w.tok0), static_cast<const int32_t*>(w.clen),
+                                  w.hbar));
+  }
   // ---- K̄: per-token projection + RoPE + pooling on tcgen05 ----
   {
     CUtensorMap ma, mb;
@@ -502,13 +555,7 @@ msa_status encode_launch(const msa_dims& d, const void* H, int64_t T, const int6
     p.n_out0 = NK;
     const int grid = std::max(1, std::min(sm_count(), p.m_tiles * p.n_tiles));
     TraceScope ts(kKEncGemmK, s);
-    MSA_CUDA_CHECK(launch_gemm<kModeK>(bn, grid, gemm_smem_bytes(kModeK, bn), s, ma, mb, p));
-  }
-  // ---- H̄ (hi | lo) ----
-  {
-    TraceScope ts(kKEncPoolH, s);
-    pool_h_kernel<<<n_chunks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(H), hidden, w.tok0, w.clen, w.hbar);
-    MSA_CUDA_CHECK(cudaGetLastError());
+    MSA_CUDA_CHECK(launch_gemm<kModeK>(bn, grid, gemm_smem_bytes(kModeK, bn), s, ma, mb, p, /*early=*/true));
   }
   // ---- V̄ | K̄^R = H̄ [W_V | W^KR] ----
   {
