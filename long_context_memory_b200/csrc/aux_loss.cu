@@ -43,9 +43,6 @@ constexpr int kAuxStagesRing = 6; // ring stages when they stream twice (more th
 __host__ __device__ inline bool aux_resident(bool grads, int nk) {
   return grads && (nk + kAuxRows - 1) / kAuxRows <= kAuxStagesMax;
 }
-__host__ __device__ inline int aux_stages(bool grads, int nk) {
-  return aux_resident(grads, nk) ? kAuxStagesMax : kAuxStagesRing;
-}
 constexpr float kAuxEps = 1e-12f;
 
 struct AuxParams {
@@ -59,24 +56,36 @@ struct AuxParams {
   float* term;                 // [P] per-positive loss terms (workspace)
   uint32_t* ticket;            // [1] CTAs done (workspace)
   int P, N, n_r;
+  int stages;                  // ring stages (aux_stages, computed on the host)
   float inv_tau;
 };
 
 // shared memory: ring [stages][kAuxRows][n_r * DR] bf16 | cos, |k| [NK][8] fp32 | g [NK] |
-// per compute warp a slice of kSlice floats (its dK row staged for coalesced stores, then its
-// dQ partial) | barriers
+// per compute warp two rows of kRow floats (its dK rows, in the gradient's own order, handed to
+// bulk stores; then its dQ partial) | barriers
 template <int DR>
 struct AuxSmem {
   static constexpr int kRowBytes = 8 * DR * 2;  // room for 8 router heads
   static constexpr int kStageBytes = kAuxRows * kRowBytes;
-  static constexpr int kLanePad = DR / 4 + 4;   // a lane's DR/4 values + 4 floats of padding
-  static constexpr int kSlice = 32 * kLanePad;  // >= 8 * DR, >= 32 * (DR / 4 + 1)
+  static constexpr int kRow = 8 * DR;           // one gradient row (room for 8 router heads)
+  static constexpr int kStg = 2 * kRow;         // a compute warp's two staging rows
   static constexpr int kQBytes = 8 * DR * 2;    // one query row (room for 8 router heads)
   static __host__ __device__ size_t bytes(int nk, int stages) {
     return (size_t)stages * kStageBytes + 2 * kQBytes + (size_t)nk * 8 * 4 * 2 + (size_t)nk * 4 + 16 +
-           (size_t)kAuxCompute * kSlice * 4 + (2 * kAuxStagesMax + 4) * 8 + 16;
+           (size_t)kAuxCompute * kStg * 4 + (2 * kAuxStagesMax + 4) * 8 + 16;
   }
 };
+
+// ring stages: every row of a positive when they stay resident, otherwise kAuxStagesRing, fewer
+// when the shared memory would not hold them (many negatives: the per-row cosines and norms grow)
+constexpr size_t kAuxSmemBudget = 227 * 1024 - 1024;  // dynamic shared memory, beside the static
+template <int DR>
+__host__ __device__ inline int aux_stages(bool grads, int nk) {
+  if (aux_resident(grads, nk)) return kAuxStagesMax;
+  int st = kAuxStagesRing;
+  while (st > 2 && AuxSmem<DR>::bytes(nk, st) > kAuxSmemBudget) --st;
+  return st;
+}
 
 // lane l of a compute warp owns head l / 4, quarter l % 4: U 16-byte units of the row.
 // Slot e of a lane holds unit (e + rot) % U of its quarter (rot = l / (8 / U)), so that a
@@ -102,15 +111,15 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
   const int n_r = p.n_r, NK = p.N + 1, NR = n_r * DR;
   uint8_t* ring = aux_sm;
   const bool grads = p.dQ != nullptr || p.dK_pos != nullptr || p.dK_neg != nullptr;
-  const int S = aux_stages(grads, NK);  // ring stages
+  const int S = p.stages;  // ring stages
   uint8_t* qbuf = aux_sm + S * Sm::kStageBytes;                                   // [2][n_r * DR] bf16
   float* cosv = reinterpret_cast<float*>(qbuf + 2 * Sm::kQBytes);                 // [NK][8]
   float* nkv = cosv + (size_t)NK * 8;                                            // [NK][8]
   float* gs = nkv + (size_t)NK * 8;                                              // [NK]
   float* red = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(gs + NK) + 15) & ~uintptr_t(15));
-  // red: [kAuxCompute][Sm::kSlice]
+  // red: [kAuxCompute][Sm::kStg] (16-byte aligned: bulk-store sources)
   uint64_t* full = reinterpret_cast<uint64_t*>(
-      (reinterpret_cast<uintptr_t>(red + (size_t)kAuxCompute * Sm::kSlice) + 7) & ~uintptr_t(7));
+      (reinterpret_cast<uintptr_t>(red + (size_t)kAuxCompute * Sm::kStg) + 7) & ~uintptr_t(7));
   uint64_t* empty = full + kAuxStagesMax;
   uint64_t* qfull = empty + kAuxStagesMax;  // [2] a positive's query row landed
   uint64_t* qempty = qfull + 2;          // [2] every compute warp is done with it
@@ -334,7 +343,7 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
 #pragma unroll
     for (int e = 0; e < V; ++e) acc[e] = 0.f;
     const float nq = hl ? fabsf(qn[h]) : 1.f;
-    float* slice = red + (size_t)warp * Sm::kSlice;
+    float* slice = red + (size_t)warp * Sm::kStg;
     for (int c = 0; c < n_ch; ++c) {
       const int ring_it = resident ? it_first + c : it++;
       const int st = ring_it % S;
@@ -356,6 +365,14 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
       float* dk = nullptr;
       if (j < NK) dk = j == 0 ? (p.dK_pos ? p.dK_pos + (size_t)i * NR : nullptr)
                               : (p.dK_neg ? p.dK_neg + ((size_t)i * p.N + (j - 1)) * NR : nullptr);
+      // the row's dK goes to staging row c & 1 of this warp, in the gradient's order, and from
+      // there to global memory by one bulk store; the store issued from that row two rows ago
+      // must have read it first (lane 0 issued it: its group count is the warp's)
+      float* stg = slice + (c & 1) * Sm::kRow;
+      if (dk) {
+        if (lane == 0) bulk_store_wait_read<1>();
+        __syncwarp();
+      }
       if (j < NK && hl) {
         const float nks = nkv[(size_t)j * 8 + h], nk = fabsf(nks);
         const float g = gs[j] * inv_nr;
@@ -371,9 +388,8 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
           f = unpack_bf16x2(kw[e].w); kv[6] = f.x; kv[7] = f.y;
 #pragma unroll
           for (int t = 0; t < 8; ++t) acc[8 * e + t] = fmaf(a, kv[t], acc[8 * e + t]);
-          if (dk) {
-            // staged in this warp's slice (lane rows padded: no bank conflicts)
-            float* s8 = slice + lane * Sm::kLanePad + unit_of_slot<DR>(e, lane) * 8;
+          if (dk) {  // element lane * V + o of the row: this lane's head and quarter
+            float* s8 = stg + lane * V + unit_of_slot<DR>(e, lane) * 8;
             *reinterpret_cast<float4*>(s8) =
                 make_float4(a * q[8 * e + 0] - b * kv[0], a * q[8 * e + 1] - b * kv[1], a * q[8 * e + 2] - b * kv[2],
                             a * q[8 * e + 3] - b * kv[3]);
@@ -383,15 +399,18 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
           }
         }
       }
-      __syncwarp();
-      if (dk) {  // consecutive lanes store consecutive 16-byte pieces: whole 512-byte segments
-        for (int i4 = lane; i4 < NR / 4; i4 += 32) {
-          const int e0 = i4 * 4;
-          *reinterpret_cast<float4*>(dk + e0) = *reinterpret_cast<const float4*>(slice + (e0 / V) * Sm::kLanePad + e0 % V);
+      if (dk) {
+        fence_proxy_async_smem();  // this lane's staging writes before the bulk store reads them
+        __syncwarp();
+        if (lane == 0) {
+          bulk_store(dk, stg, (uint32_t)NR * 4);
+          bulk_store_commit();
         }
       }
-      __syncwarp();  // the slice is read before the next row is staged
     }
+    // the staging rows are free again (the dq partial reuses them) once the stores have read them
+    if (lane == 0) bulk_store_wait_read<0>();
+    __syncwarp();
     if (p.dQ != nullptr) {
       // this warp's dq partial in its slice: element lane * V + o of the row at lane * V +
       // (o + lane) % V, so that the lanes' stores of one o fall in distinct banks (a lane's V
@@ -407,7 +426,7 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
         const int se = (e & ~(V - 1)) + ((e + e / V) & (V - 1));  // where element e of a partial sits
         float v = 0.f;
 #pragma unroll
-        for (int w = 0; w < kAuxCompute; ++w) v += red[(size_t)w * Sm::kSlice + se];
+        for (int w = 0; w < kAuxCompute; ++w) v += red[(size_t)w * Sm::kStg + se];
         const float nqs = qn[hh], nqa = fabsf(nqs);
         if (nqs > 0.f) v -= chead[hh] * inv_nr * bf16_bits_to_float(qrow[e]) / (nqa * nqa);
         p.dQ[(size_t)i * NR + e] = v;
@@ -416,6 +435,10 @@ __global__ void __launch_bounds__(kAuxThreads, 1) aux_loss_kernel(const AuxParam
     aux_bar_sync();  // every warp is done with the query row
     if (lane == 0) mbar_arrive(&qempty[qb]);  // the query buffer may take the positive after next
   }
+
+  // every gradient row this warp handed to a bulk store is written before the CTA finishes
+  if (lane == 0) bulk_store_wait_all();
+  __syncwarp();
 
   // ---- loss: the last CTA sums the terms in positive order ----
   __threadfence();
@@ -473,12 +496,15 @@ msa_status aux_loss_launch(const msa_dims& d, const void* QR, const void* K_pos,
   p.inv_tau = 1.0f / tau;
   const int grid = std::max(1, std::min(P, sm_count()));
   TraceScope ts(kKAuxLoss, s);
+  const bool grads = dQ || dK_pos || dK_neg;
   if (d.d_r == 128) {
-    const size_t sm = AuxSmem<128>::bytes(N + 1, aux_stages(dQ || dK_pos || dK_neg, N + 1));
+    p.stages = aux_stages<128>(grads, N + 1);
+    const size_t sm = AuxSmem<128>::bytes(N + 1, p.stages);
     MSA_CUDA_CHECK(set_max_dynamic_smem(reinterpret_cast<const void*>(aux_loss_kernel<128>), (int)sm));
     MSA_CUDA_CHECK(launch_pdl(aux_loss_kernel<128>, dim3(grid), dim3(kAuxThreads), sm, s, p));
   } else {
-    const size_t sm = AuxSmem<64>::bytes(N + 1, aux_stages(dQ || dK_pos || dK_neg, N + 1));
+    p.stages = aux_stages<64>(grads, N + 1);
+    const size_t sm = AuxSmem<64>::bytes(N + 1, p.stages);
     MSA_CUDA_CHECK(set_max_dynamic_smem(reinterpret_cast<const void*>(aux_loss_kernel<64>), (int)sm));
     MSA_CUDA_CHECK(launch_pdl(aux_loss_kernel<64>, dim3(grid), dim3(kAuxThreads), sm, s, p));
   }

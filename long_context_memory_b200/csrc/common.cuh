@@ -197,6 +197,24 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, 
       : "memory");
 }
 
+// Contiguous bulk store, shared -> global, by the TMA unit (the issuing thread moves on); both
+// addresses 16-byte aligned, bytes a multiple of 16.  The shared source must have been written
+// before a fence_proxy_async_smem() of its writers.  Stores are grouped per issuing thread:
+// bulk_store_commit closes a group, bulk_store_wait_read<N> returns once at most N of its groups
+// still read shared memory (their sources may then be rewritten), bulk_store_wait_all once every
+// group's writes are complete.
+__device__ __forceinline__ void bulk_store(void* gmem_dst, const void* smem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gmem_dst),
+               "r"(smem_u32(smem_src)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_store_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // ---------------------------------------------------------------------------
 // thread-block clusters: barrier over the cluster's CTAs, loads from a peer CTA's
 // shared memory (distributed shared memory)
