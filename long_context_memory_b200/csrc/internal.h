@@ -54,6 +54,7 @@ enum KernelId : int {
   kKKvAppend,
   kKKrNorms,
   kKAttnMerge,
+  kKChunkDoc,
   kKernelCount
 };
 

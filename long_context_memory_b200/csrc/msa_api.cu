@@ -219,7 +219,7 @@ namespace {
 const char* kKernelNames[kKernelCount] = {
     "router_query", "scan", "topk_slice", "topk_merge", "rope_table", "attn_split", "attn_combine",
     "enc_chunk_map", "enc_transpose_w", "enc_gemm_k", "enc_pool_h", "enc_gemm_pooled", "rope_rows", "gather_plan", "gather_copy",
-    "chunk_off_extend", "aux_loss", "kv_append", "kr_norms", "attn_merge"};
+    "chunk_off_extend", "aux_loss", "kv_append", "kr_norms", "attn_merge", "chunk_doc"};
 
 struct TraceState {
   std::mutex mu;

@@ -1285,6 +1285,7 @@ __global__ void __launch_bounds__(256) chunk_doc_kernel(const int32_t* __restric
 
 msa_status chunk_doc_launch(const int32_t* chunk_off, int n_docs, int n_chunks, int32_t* chunk_doc, cudaStream_t s) {
   const int blocks = std::max(1, std::min(4 * sm_count(), (n_docs + 7) / 8));
+  TraceScope ts(kKChunkDoc, s);
   MSA_CUDA_CHECK(launch_pdl(chunk_doc_kernel, dim3(blocks), dim3(256), 0, s, chunk_off, n_docs, n_chunks, chunk_doc));
   return MSA_OK;
 }
