@@ -452,8 +452,9 @@ msa_status msa_gather_kv(const msa_dims* dims, const void* K_bar_host, const voi
  *                    documents; a selection needing more stages what fits and
  *                    raises device error bit 1, as msa_gather_kv).
  *   ws        >= msa_tiered_workspace_size(dims, n_layers, ...) bytes, 256-byte
- *             aligned; holds each layer's router-query rows, two routing workspaces,
- *             the attention workspace and the two staging areas.
+ *             aligned; holds the layout's chunk -> document map (computed by the
+ *             call), each layer's router-query rows, two routing workspaces, the
+ *             attention workspace and the two staging areas.
  * msa_tiered_workspace_size returns 0 for arguments outside the limits below.
  * The call keeps six CUDA events per host thread and device (created by its
  * first call on that device from that thread: make that call before any stream
