@@ -36,9 +36,8 @@
 namespace msa {
 
 struct RouteWs {
-  uint32_t* scan_ticket;  // [1 + B + passes]: scan CTAs finished (fused top-k), per query its slices
-                          // finished (fused merge), per scan pass its tiles taken; zeroed by the
-                          // router query kernel
+  uint32_t* scan_ticket;  // [1 + B]: scan CTAs finished (fused top-k), then per query its slices
+                          // finished (fused merge); zeroed by the router query kernel
   __nv_bfloat16* q_hl; // [passes][n_r][2][NQ][d_r] normalised query, bf16 hi and lo terms
   uint32_t* doc_key;  // [B][n_docs] ordered-uint32 doc max (MAX)
   uint32_t* chunk_k;  // [B][n_chunks] ordered chunk scores (MEAN)
@@ -279,12 +278,6 @@ __global__ void __launch_bounds__(kRqThreads) router_query_direct_kernel(
 // --------------------------------------------------------------------------
 constexpr int kScanM = 128;         // chunks per tile (MMA M)
 constexpr int kScanThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2..5 norms, warps 6..9 epilogue
-// Tiles are taken dynamically: a CTA's first tile is blockIdx.x, each later one comes from an
-// atomic counter, so that CTAs that start late or run slow (beside other work) take fewer.  The
-// producer passes each taken tile's index to the MMA thread and the 8 epilogue / norm warps
-// through a ring of kTileSlots slots (-1: no more tiles).
-constexpr int kTileSlots = 4;
-constexpr int kTileReaders = 1 + 8;  // the MMA thread and one arrival per epilogue or norm warp
 constexpr int kScanNormWarps = 4;   // one per TMEM lane quarter (32 rows each)
 constexpr int kScanEpiWarps = 4;
 
@@ -310,7 +303,6 @@ struct ScanParams {
   const float* inv_norm;  // [C][n_r] 1 / max(||K̄^R_jh||, eps) precomputed, or null (norm warps compute it)
   const int32_t* chunk_doc;  // [C] each chunk's document (-1: none), or null (searched in chunk_off)
   int wait_prior;  // 0: the kernel before this one on the stream writes nothing this scan reads or writes
-  uint32_t* tile_ctr;  // tiles taken beyond each CTA's first (zero at launch)
   uint32_t tmem_cols;
   float inv_nr;
 };
@@ -342,12 +334,11 @@ struct ScanGeom {
 // halves of this warp's queries) and release them, and fold each document segment's maximum into
 // doc_key (or store the chunk scores for the mean).  A warp whose queries are all past q_count still takes part in the
 // barrier protocol but does no work.
-template <int DR, int NQ, bool MEAN, int QW>
-__device__ __forceinline__ void scan_epilogue(const ScanParams& p, int q4, int q_off, int lane,
-                                              const volatile int* slot_tile, uint64_t* slot_full,
-                                              uint64_t* slot_empty, uint32_t tmem_base, uint32_t buf_cols,
-                                              const float* n2s, uint64_t* tfull, uint64_t* tempty, uint64_t* nfull,
-                                              uint64_t* nempty, volatile int* abort) {
+template <int DR, int NQ, bool MEAN, bool MAPPED, int QW>
+__device__ __forceinline__ void scan_epilogue(const ScanParams& p, int q4, int q_off, int lane, int t_begin, int n_lt,
+                                              uint32_t tmem_base, uint32_t buf_cols, const float* n2s, uint64_t* tfull,
+                                              uint64_t* tempty, uint64_t* nfull, uint64_t* nempty,
+                                              volatile int* abort) {
   using Gm = ScanGeom<DR, NQ>;
   const int n_r = p.n_r;
   const int row = 32 * q4 + lane;  // chunk within the tile
@@ -355,31 +346,22 @@ __device__ __forceinline__ void scan_epilogue(const ScanParams& p, int q4, int q
   int cur = 0;                     // lower bound for this warp's document search
   // With a chunk -> document map the rows' documents and inverse norms of the next tile are
   // loaded while this one is processed (one tile ahead); without it each tile searches chunk_off.
-  const bool mapped = !MEAN && p.chunk_doc != nullptr;  // (the mean needs no document boundaries)
+  // (a compile-time choice, so that routing without the map keeps the search's own code; the mean
+  // needs no document boundaries)
+  constexpr bool mapped = MAPPED && !MEAN;
   int doc_next = -1;
   float invg_next[8];
-  auto fetch = [&](int tile_f) {
-    const int jr = tile_f * kScanM + row;
+  auto fetch = [&](int lt_f) {
+    const int jr = (t_begin + lt_f) * kScanM + row;
     doc_next = (active && jr < p.n_chunks) ? __ldg(&p.chunk_doc[jr]) : -1;
 #pragma unroll
     for (int hh = 0; hh < 8; ++hh)
       invg_next[hh] = (p.inv_norm && active && hh < n_r && jr < p.n_chunks) ? __ldg(&p.inv_norm[(size_t)jr * n_r + hh])
                                                                             : 0.f;
   };
-  // the tile of local index lt: slot lt % kTileSlots, read once the producer has published it
-  auto take = [&](int lt_t, int* tile_t) -> bool {
-    const int sl = lt_t % kTileSlots;
-    if (!warp_wait(&slot_full[sl], (lt_t / kTileSlots) & 1, abort)) return false;
-    *tile_t = slot_tile[sl];
-    return true;
-  };
-  int tile = -1;
-  if (!take(0, &tile)) return;
-  if (mapped && tile >= 0) fetch(tile);
-  for (int lt = 0;; ++lt) {
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&slot_empty[lt % kTileSlots]);  // this warp has read the tile index
-    if (tile < 0) break;
+  if (mapped && n_lt > 0) fetch(0);
+  for (int lt = 0; lt < n_lt; ++lt) {
+    const int tile = t_begin + lt;
     const int nbuf = lt & 1;                                    // norm buffer
     const int buf = lt % Gm::kBufs, use = lt / Gm::kBufs;      // TMEM buffer
     const int jrow = tile * kScanM + row;
@@ -390,6 +372,7 @@ __device__ __forceinline__ void scan_epilogue(const ScanParams& p, int q4, int q
       doc = doc_next;
 #pragma unroll
       for (int hh = 0; hh < 8; ++hh) invg[hh] = invg_next[hh];
+      if (lt + 1 < n_lt) fetch(lt + 1);
     } else {
       // documents of this warp's 32 rows, found before the accumulators are ready (they depend
       // on the tile alone): a warp-wide 32-ary search for the first row's document, then one
@@ -417,11 +400,6 @@ __device__ __forceinline__ void scan_epilogue(const ScanParams& p, int q4, int q
         if (j >= p.n_chunks) doc = -1;
         cur = d0;
       }
-      if (p.inv_norm) {
-#pragma unroll
-        for (int hh = 0; hh < 8; ++hh)
-          invg[hh] = (active && hh < n_r && jrow < p.n_chunks) ? __ldg(&p.inv_norm[(size_t)jrow * n_r + hh]) : 0.f;
-      }
     }
     const int prev = __shfl_up_sync(0xffffffffu, doc, 1);
     const bool head = (lane == 0) || (prev != doc);
@@ -432,7 +410,11 @@ __device__ __forceinline__ void scan_epilogue(const ScanParams& p, int q4, int q
       const int od = __shfl_down_sync(0xffffffffu, doc, 1 << e);
       if (lane + (1 << e) < 32 && od == doc) same |= 1u << e;
     }
-    if (!p.inv_norm && !warp_wait(&nfull[nbuf], (lt >> 1) & 1, abort)) {
+    if (!mapped && p.inv_norm) {  // (with the map they were loaded a tile ahead)
+#pragma unroll
+      for (int hh = 0; hh < 8; ++hh)
+        invg[hh] = (active && hh < n_r && jrow < p.n_chunks) ? __ldg(&p.inv_norm[(size_t)jrow * n_r + hh]) : 0.f;
+    } else if (!p.inv_norm && !warp_wait(&nfull[nbuf], (lt >> 1) & 1, abort)) {
       return;
     }
     if (!warp_wait(&tfull[buf], use & 1, abort)) return;
@@ -470,12 +452,6 @@ __device__ __forceinline__ void scan_epilogue(const ScanParams& p, int q4, int q
     }
     __syncwarp();
     if (lane == 0 && !p.inv_norm) mbar_arrive(&nempty[nbuf]);
-    // the next tile (taken by the producer before this one's last stage was loaded): its rows'
-    // documents and norms load while this tile's maxima are folded in
-    int tile_next = -1;
-    if (!take(lt + 1, &tile_next)) return;
-    if (mapped && tile_next >= 0) fetch(tile_next);
-    tile = tile_next;
     if (!active) continue;
 
 #pragma unroll
@@ -503,7 +479,7 @@ __device__ __forceinline__ void scan_epilogue(const ScanParams& p, int q4, int q
   }
 }
 
-template <int DR, int NQ, bool MEAN>
+template <int DR, int NQ, bool MEAN, bool MAPPED>
 __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_constant__ CUtensorMap kr_map,
                                                                const __grid_constant__ CUtensorMap q_map,
                                                                const ScanParams p) {
@@ -523,12 +499,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   uint64_t* drained = nempty + 2;              // [1] after an abort: every MMA issued has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
   __shared__ int abort_flag;                   // a bounded wait of this CTA gave up
-  __shared__ volatile int slot_tile[kTileSlots];          // tile index of local tile lt % kTileSlots (-1: end)
-  __shared__ __align__(8) uint64_t slot_full[kTileSlots];  // the producer has published the slot
-  __shared__ __align__(8) uint64_t slot_empty[kTileSlots]; // every reader has read it
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_r = p.n_r;
+  const int t_begin = (int)(((long long)blockIdx.x * p.n_tiles) / gridDim.x);
+  const int t_end = (int)(((long long)(blockIdx.x + 1) * p.n_tiles) / gridDim.x);
+  const int n_lt = t_end - t_begin;
+  const int n_it = n_lt * n_r;  // (tile, head) stages of this CTA
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -544,10 +521,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       mbar_init(&nempty[b], kScanEpiWarps);
     }
     mbar_init(drained, 1);
-    for (int t = 0; t < kTileSlots; ++t) {
-      mbar_init(&slot_full[t], 1);
-      mbar_init(&slot_empty[t], kTileReaders);
-    }
     abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&kr_map);
@@ -563,8 +536,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t buf_cols = (uint32_t)n_r * Gm::kCols;
   // stage it = (tile, head): the head's 128 x DR key rows, then the head's query rows (hi, lo)
-  auto load_keys = [&](int it, int tile) {
-    const int h = it % n_r, st = it % S;
+  auto load_keys = [&](int it) {
+    const int tile = t_begin + it / n_r, h = it % n_r, st = it % S;
     uint8_t* k_s = stages + st * Gm::kStageBytes;
     mbar_arrive_expect_tx(&full[st], Gm::kStageBytes);  // the query rows' bytes included
 #pragma unroll
@@ -587,10 +560,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   // The previous kernel of this call (the router query, or the previous pass) does not write
   // K̄^R, and it started this grid only after its own wait, so whatever wrote K̄^R has
   // completed: the first ring's key tiles stream in while the router query finishes.
-  // (the first tile of a CTA is blockIdx.x < n_tiles: the grid is at most the tile count)
-  const int n_pre = min(S, n_r);
+  const int n_pre = min(S, n_it);
   if (warp == 0 && lane == 0)
-    for (int it = 0; it < n_pre; ++it) load_keys(it, blockIdx.x);
+    for (int it = 0; it < n_pre; ++it) load_keys(it);
   // A scan that follows another routing's scan on the stream (the caller's guarantee: that scan
   // writes another workspace, and everything this one reads was final before it started) does
   // not wait for it: its CTAs stream as soon as they land, beside the other scan's last tiles.
@@ -601,33 +573,12 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     // ------------------------- TMA producer -------------------------
     if (lane == 0) {
       int it = 0;
-      bool stop = false;
-      // the tile: this CTA's own first, then one taken from the counter (-1 when none is left).
-      // Each take is issued a tile ahead, so that the atomic's round trip overlaps the loads of
-      // the tile before it.
-      unsigned claim = p.n_tiles > (int)gridDim.x ? atomicAdd(p.tile_ctr, 1u) : 0u;
-      for (int lt = 0; !stop; ++lt) {
-        int tile = blockIdx.x;
-        if (lt > 0) {
-          const long long c = (long long)gridDim.x + claim;
-          tile = c < p.n_tiles ? (int)c : -1;
-          if (tile >= 0) claim = atomicAdd(p.tile_ctr, 1u);
+      for (; it < n_it; ++it) {
+        if (it >= n_pre) {
+          if (it >= S && !mbar_wait(&empty[it % S], ((it / S) - 1) & 1, &abort_flag)) break;
+          load_keys(it);
         }
-        const int sl = lt % kTileSlots;
-        if (lt >= kTileSlots && !mbar_wait(&slot_empty[sl], ((lt / kTileSlots) - 1) & 1, &abort_flag)) break;
-        slot_tile[sl] = tile;
-        mbar_arrive(&slot_full[sl]);  // releases the index to the readers
-        if (tile < 0) break;
-        for (int h = 0; h < n_r; ++h, ++it) {
-          if (it >= n_pre) {
-            if (it >= S && !mbar_wait(&empty[it % S], ((it / S) - 1) & 1, &abort_flag)) {
-              stop = true;
-              break;
-            }
-            load_keys(it, tile);
-          }
-          load_query(it);
-        }
+        load_query(it);
       }
       // after an abort: the stages issued and possibly still in flight land before the CTA exits
       if (abort_flag) mbar_drain_ring(full, S, it - S, it);
@@ -636,25 +587,12 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     // ------------------------- MMA issuer -------------------------
     if (lane == 0) {
       constexpr uint32_t idesc = umma_idesc_bf16(kScanM, Gm::kCols);
-      int it = 0;
-      bool stop = false;
-      for (int lt = 0; !stop; ++lt) {
-        const int sl = lt % kTileSlots;
-        if (!mbar_wait(&slot_full[sl], (lt / kTileSlots) & 1, &abort_flag)) break;
-        const int tile = slot_tile[sl];
-        mbar_arrive(&slot_empty[sl]);
-        if (tile < 0) break;
+      for (int it = 0; it < n_it; ++it) {
+        const int lt = it / n_r, h = it % n_r;
         const int buf = lt % Gm::kBufs, use = lt / Gm::kBufs;
-        for (int h = 0; h < n_r; ++h, ++it) {
         const int st = it % S;
-        if (use >= 1 && !mbar_wait(&tempty[buf * 8 + h], (use - 1) & 1, &abort_flag)) {  // head's columns read
-          stop = true;
-          break;
-        }
-        if (!mbar_wait(&full[st], (it / S) & 1, &abort_flag)) {
-          stop = true;
-          break;
-        }
+        if (use >= 1 && !mbar_wait(&tempty[buf * 8 + h], (use - 1) & 1, &abort_flag)) break;  // head's columns read
+        if (!mbar_wait(&full[st], (it / S) & 1, &abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * buf_cols + h * Gm::kCols;
         const uint32_t k_addr = smem_u32(stages + st * Gm::kStageBytes);
@@ -668,7 +606,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         }
         umma_commit(&empty[st]);
         if (h == n_r - 1) umma_commit(&tfull[buf]);
-        }
       }
       if (abort_flag) {  // every MMA issued completes before the TMEM is freed
         umma_commit(drained);
@@ -677,31 +614,17 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     }
   } else if (warp < 2 + kScanNormWarps && p.inv_norm) {
     // norms given: these four warps take the second half of the queries of each row
-    scan_epilogue<DR, NQ, MEAN, NQ / 2>(p, warp & 3, NQ / 2, lane, slot_tile, slot_full, slot_empty, tmem_base,
-                                        buf_cols, n2s, tfull, tempty, nfull, nempty, &abort_flag);
+    scan_epilogue<DR, NQ, MEAN, MAPPED, NQ / 2>(p, warp & 3, NQ / 2, lane, t_begin, n_lt, tmem_base, buf_cols, n2s, tfull,
+                                        tempty, nfull, nempty, &abort_flag);
   } else if (warp < 2 + kScanNormWarps) {
     // ------- norm warps: squared norm of every row's head-h slice, stage released at once -------
     const int row = 32 * (warp & 3) + lane;  // chunk within the tile
-    int it = 0;
-    bool stop = false;
-    for (int lt = 0; !stop; ++lt) {
-      const int sl = lt % kTileSlots;
-      if (!warp_wait(&slot_full[sl], (lt / kTileSlots) & 1, &abort_flag)) break;
-      const int tile = slot_tile[sl];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&slot_empty[sl]);
-      if (tile < 0) break;
-      for (int h = 0; h < n_r; ++h, ++it) {
+    for (int it = 0; it < (p.inv_norm ? 0 : n_it); ++it) {
+      const int lt = it / n_r, h = it % n_r;
       const int buf = lt & 1;  // norm buffer
       const int st = it % S;
-      if (h == 0 && lt >= 2 && !warp_wait(&nempty[buf], ((lt >> 1) - 1) & 1, &abort_flag)) {  // n2s[buf] free
-        stop = true;
-        break;
-      }
-      if (!warp_wait(&full[st], (it / S) & 1, &abort_flag)) {
-        stop = true;
-        break;
-      }
+      if (h == 0 && lt >= 2 && !warp_wait(&nempty[buf], ((lt >> 1) - 1) & 1, &abort_flag)) break;  // n2s[buf] free
+      if (!warp_wait(&full[st], (it / S) & 1, &abort_flag)) break;
       const uint8_t* k_s = stages + st * Gm::kStageBytes;
       float n2p[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -723,16 +646,15 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         __syncwarp();
         if (lane == 0) mbar_arrive(&nfull[buf]);
       }
-      }
     }
   } else {
     // epilogue warps: every query of each row, or the first half when the norms are given
     if (p.inv_norm)
-      scan_epilogue<DR, NQ, MEAN, NQ / 2>(p, warp & 3, 0, lane, slot_tile, slot_full, slot_empty, tmem_base, buf_cols,
-                                          n2s, tfull, tempty, nfull, nempty, &abort_flag);
+      scan_epilogue<DR, NQ, MEAN, MAPPED, NQ / 2>(p, warp & 3, 0, lane, t_begin, n_lt, tmem_base, buf_cols, n2s, tfull, tempty,
+                                          nfull, nempty, &abort_flag);
     else
-      scan_epilogue<DR, NQ, MEAN, NQ>(p, warp & 3, 0, lane, slot_tile, slot_full, slot_empty, tmem_base, buf_cols,
-                                      n2s, tfull, tempty, nfull, nempty, &abort_flag);
+      scan_epilogue<DR, NQ, MEAN, MAPPED, NQ>(p, warp & 3, 0, lane, t_begin, n_lt, tmem_base, buf_cols, n2s, tfull, tempty,
+                                      nfull, nempty, &abort_flag);
   }
   tc_fence_before();
   __syncthreads();
@@ -1163,10 +1085,10 @@ __global__ void __launch_bounds__(kTopkThreads) topk_merge_pairs_kernel(const fl
   }
 }
 
-template <int DR, int NQ, bool MEAN>
+template <int DR, int NQ, bool MEAN, bool MAPPED = false>
 cudaError_t launch_scan_t(const CUtensorMap& kmap, const CUtensorMap& qmap, const ScanParams& p, int grid,
                           cudaStream_t s) {
-  auto kern = scan_kernel<DR, NQ, MEAN>;
+  auto kern = scan_kernel<DR, NQ, MEAN, MAPPED>;
   static_assert(kSliceDocs * sizeof(uint64_t) + kTopkScratchBytes <=
                     (size_t)ScanGeom<DR, NQ>::kStages * ScanGeom<DR, NQ>::kStageBytes,
                 "the fused top-k reuses the pipeline stages");
@@ -1178,6 +1100,12 @@ cudaError_t launch_scan_t(const CUtensorMap& kmap, const CUtensorMap& qmap, cons
 
 cudaError_t launch_scan(int d_r, int nq, bool mean, const CUtensorMap& kmap, const CUtensorMap& qmap,
                         const ScanParams& p, int grid, cudaStream_t s) {
+  if (!mean && p.chunk_doc) {  // the epilogue reads each row's document from the map
+    if (d_r == 128) return nq == 16 ? launch_scan_t<128, 16, false, true>(kmap, qmap, p, grid, s)
+                                    : launch_scan_t<128, 32, false, true>(kmap, qmap, p, grid, s);
+    return nq == 16 ? launch_scan_t<64, 16, false, true>(kmap, qmap, p, grid, s)
+                    : launch_scan_t<64, 32, false, true>(kmap, qmap, p, grid, s);
+  }
   if (d_r == 128) {
     if (nq == 16) return mean ? launch_scan_t<128, 16, true>(kmap, qmap, p, grid, s)
                               : launch_scan_t<128, 16, false>(kmap, qmap, p, grid, s);
@@ -1255,7 +1183,7 @@ size_t route_workspace(const msa_dims& d, int B, int M, int n_docs, int n_chunks
   w.passes = (R + w.nq - 1) / w.nq;
   w.n_slices = (n_docs + kSliceDocs - 1) / kSliceDocs;
   w.q_hl = cv.take<__nv_bfloat16>((size_t)w.passes * d.n_r * 2 * w.nq * d.d_r);
-  w.scan_ticket = cv.take<uint32_t>(1 + (size_t)B + w.passes);  // the tickets, then the document keys: one region
+  w.scan_ticket = cv.take<uint32_t>(1 + (size_t)B);  // the tickets, then the document keys: one region
   w.doc_key = agg == MSA_AGG_MAX ? cv.take<uint32_t>((size_t)B * n_docs) : nullptr;
   w.chunk_k = agg == MSA_AGG_MEAN ? cv.take<uint32_t>((size_t)B * n_chunks) : nullptr;
   w.cand = w.n_slices > 1 ? cv.take<uint64_t>((size_t)B * w.n_slices * k) : nullptr;
@@ -1345,8 +1273,8 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
 
   // K1: router query (projection, normalisation, hi/lo layout) and document keys cleared
   if (score && part != RoutePart::kScan) {
-    msa_status st = route_query_launch(d, Hq, W_QR, B, M, w.q_hl, clear, n_clear, w.scan_ticket, 1 + B + w.passes,
-                                       s, early_inputs);
+    msa_status st = route_query_launch(d, Hq, W_QR, B, M, w.q_hl, clear, n_clear, w.scan_ticket, 1 + B, s,
+                                       early_inputs);
     if (st != MSA_OK) return st;
   }
   const void* q_src = part == RoutePart::kScan ? q_ext : w.q_hl;
@@ -1402,7 +1330,6 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
       p.inv_norm = kr_inv_norm;
       p.chunk_doc = chunk_doc;
       p.wait_prior = (pass == 0 && after_scan) ? 0 : 1;
-      p.tile_ctr = w.scan_ticket + 1 + B + pass;
       p.tmem_cols = cols;
       p.inv_nr = 1.0f / (float)d.n_r;
       TraceScope ts(kKScan, s);
