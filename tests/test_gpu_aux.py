@@ -38,8 +38,11 @@ def _case(seed, P, N, n_r, d_r, pos_scale=0.6):
     return b(Q), b(Kp), b(Kn)
 
 
+# (the last two: more negatives than stay resident in shared memory, so the rows stream twice;
+# at d_r = 128 with 1023 negatives the ring is cut to what shared memory holds)
 @pytest.mark.parametrize("P,N,n_r,d_r,tau", [(1, 0, 8, 128, 0.1), (5, 7, 8, 128, 0.05), (33, 63, 4, 64, 0.2),
-                                             (300, 15, 3, 128, 1.0), (2, 1023, 8, 64, 0.07)])
+                                             (300, 15, 3, 128, 1.0), (2, 1023, 8, 64, 0.07),
+                                             (3, 1023, 8, 128, 0.07)])
 def test_aux_loss_parity(msa, cuda_device, P, N, n_r, d_r, tau):
     import torch
 
