@@ -255,6 +255,9 @@ def test_tiered_validation(msa):
     more = msa.lib.msa_tiered_workspace_size(dd, 3, 1, 10, 20, 4, 16, 4, 64)
     assert more - small == 2 * 8 * 2 * 16 * 128 * 2
     assert msa.lib.msa_tiered_workspace_size(dd, 0, 1, 10, 20, 4, 16, 4, 64) == 0
+    # the layout's chunk -> document map: one int32 per chunk (to within the 256-byte carving)
+    wide = msa.lib.msa_tiered_workspace_size(dd, 1, 1, 10, 20 + 64 * 256, 4, 16, 4, 64)
+    assert 64 * 256 * 4 <= wide - small <= 64 * 256 * 4 + 4 * 256 + 4 * 64 * 256 // 10
 
 
 def test_workspace_sizes_grow_with_problem(msa):
