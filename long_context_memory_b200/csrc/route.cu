@@ -1269,7 +1269,9 @@ msa_status route_launch(const msa_dims& d, const void* Hq, const void* W_QR, int
   // few queries over one slice of documents: the scan's last CTA runs the top-k itself
   const bool fuse_topk = w.n_slices == 1 && w.passes == 1 && B <= kFuseTopkMaxQueries;
   const size_t n_clear = clear ? (size_t)B * (mean ? n_chunks : n_docs) : 0;
-  const bool score = part != RoutePart::kSelect, select = part != RoutePart::kScore;
+  // the scoring parts (kScore, kScan) leave the separate top-k kernels to the selection part
+  const bool score = part != RoutePart::kSelect;
+  const bool select = part == RoutePart::kAll || part == RoutePart::kSelect;
 
   // K1: router query (projection, normalisation, hi/lo layout) and document keys cleared
   if (score && part != RoutePart::kScan) {
